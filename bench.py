@@ -1,0 +1,441 @@
+"""Benchmark of the Mamba-3 SSM layer on B200: prefill tokens/s (headline) and
+decode tokens/s, with roofline fractions, an end-to-end number through host
+buffers, and the fp64 CPU oracle timed on a bounded sample as a baseline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl m3|reference]
+
+One step = one m3_scan_fwd over the workload's whole batch (all chunks,
+heads and sequences) with inputs already resident in HBM.  Under torchrun each
+rank runs its own batch (weak scaling, no collective on the data path); the
+reported value is all ranks' tokens over the slowest rank's device time.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_state_space_exp_b200 import inputs as I  # noqa: E402
+from selective_state_space_exp_b200 import m3  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {
+    "siso_prefill": I.SISO_PREFILL,
+    "mimo_prefill": I.MIMO_PREFILL,
+    "long_mimo_16k": I.LONG_MIMO_16K,
+    "long_mimo_32k": I.LONG_MIMO_32K,
+}
+DECODE = {"decode_siso": I.DECODE_SISO, "decode_mimo": I.DECODE_MIMO}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ---- algorithmic work (FLOPs at chunk Q with the causal count, bytes read
+# once + written once) -----------------------------------------------------
+
+def prefill_work(s: I.Shape):
+    """Algorithmic FLOPs and bytes of one scan.
+
+    Per chunk-head with M = Q*R rows: S = C~ B~^T over the causal (t >= s)
+    token blocks, K = N; (M o S) X, K = Q*R, N = P; chunk state B~^T X (N x P,
+    K = Q*R); chunk output C~ h (Q*R x P, K = N).  Causal token-block count:
+    Q(Q+1)/2 * R^2 entries."""
+    Q, R, N, P = s.chunk, s.rank, s.dstate, s.headdim
+    nc = math.ceil(s.seqlen / Q)
+    causal = Q * (Q + 1) // 2 * R * R
+    per_ch = 2 * causal * N + 2 * causal * P + 2 * (Q * R) * N * P + 2 * (Q * R) * N * P
+    flops = per_ch * nc * s.batch * s.nheads
+    io = 2 if s.io == "bf16" else 4
+    tok = s.batch * s.seqlen
+    byt = (2 * tok * s.nheads * R * P * io                 # x in, y out
+           + 2 * tok * s.ngroups * R * N * io              # B, C
+           + 3 * tok * s.nheads * 4                        # dt, A, lam
+           + tok * s.ngroups * (N // 2) * 4                # theta
+           + s.batch * s.nheads * N * P * 4)               # final state
+    return float(flops), float(byt)
+
+
+def decode_work(s: I.Shape):
+    R, N, P = s.rank, s.dstate, s.headdim
+    bh = s.batch * s.nheads
+    io = 2 if s.io == "bf16" else 4
+    flops = bh * N * P * (6 * R + 4)
+    byt = (2 * bh * N * P * 4 + 3 * bh * R * P * io + 3 * s.batch * s.ngroups * R * N * io
+           + 3 * bh * 4 + s.batch * s.ngroups * (N // 2) * 4)
+    return float(flops), float(byt)
+
+
+def roofline(flops, byt, seconds, peaks, src, sustained=False):
+    tf = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    t_tensor = flops / (tf * 1e12)
+    t_hbm = byt / (peaks["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        ach = flops / seconds / 1e12
+        return {"bound": "tensor", "achieved": round(ach, 2), "peak": tf, "unit": "TFLOP/s",
+                "frac": round(ach / tf, 4), "roofline_time_us": round(t_tensor * 1e6, 2),
+                "peak_source": f"{src} bf16 {'sustained' if sustained else 'burst'}"}
+    ach = byt / seconds / 1e9
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(ach / peaks["hbm_gbs"], 4), "roofline_time_us": round(t_hbm * 1e6, 2),
+            "peak_source": f"{src} HBM copy"}
+
+
+# ---- clocks ---------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---- distributed plumbing --------------------------------------------------
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---- device timing ---------------------------------------------------------
+
+L2_FLUSH_BYTES = 256 << 20
+
+
+def time_prefill(inp, s, steps, warmup, flush):
+    ws = torch.empty(max(m3.workspace_size(m3.scan_shape(inp["x"], inp["B"], s.chunk)), 1),
+                     dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(inp["x"])
+    fs = torch.empty((s.batch, s.nheads, s.dstate, s.headdim), dtype=torch.float32,
+                     device="cuda")
+
+    def step():
+        m3.m3_scan_fwd(inp["x"], inp["dt"], inp["A"], inp["lam"], inp["theta"], inp["B"],
+                       inp["C"], s.chunk, y=y, final_state=fs, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    st = m3.m3_stream_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st}")
+    return [a.elapsed_time(b) * 1e-3 for a, b in ev]
+
+
+def time_decode(dec, s, steps, warmup):
+    state = dec["state0"].clone()
+    y = torch.empty_like(dec["x"][0])
+
+    def step(t):
+        Bp = dec["B_prev"] if t == 0 else dec["B"][t - 1]
+        xp = dec["x_prev"] if t == 0 else dec["x"][t - 1]
+        m3.m3_decode_step(state, dec["x"][t], dec["dt"][t], dec["A"][t], dec["lam"][t],
+                          dec["theta"][t], dec["B"][t], dec["C"][t], Bp, xp, y=y)
+
+    for t in range(warmup):
+        step(t)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for t in range(warmup, warmup + steps):
+        step(t)
+    b.record()
+    torch.cuda.synchronize()
+    if m3.m3_stream_status() != 0:
+        raise RuntimeError("device status")
+    return a.elapsed_time(b) * 1e-3
+
+
+def time_e2e_prefill(inp_host, s, steps):
+    """Through host buffers: pinned inputs -> device, scan, y and final state
+    -> pinned host, every step, all on one stream, timed with CUDA events."""
+    names = ("x", "dt", "A", "lam", "theta", "B", "C")
+    pin = {k: inp_host[k].pin_memory() for k in names}
+    dev = {k: torch.empty_like(pin[k], device="cuda") for k in names}
+    y_h = torch.empty(pin["x"].shape, dtype=pin["x"].dtype).pin_memory()
+    fs_h = torch.empty((s.batch, s.nheads, s.dstate, s.headdim), dtype=torch.float32).pin_memory()
+    ws = torch.empty(max(m3.workspace_size(m3.scan_shape(dev["x"], dev["B"], s.chunk)), 1),
+                     dtype=torch.uint8, device="cuda")
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = y_h.numel() * y_h.element_size() + fs_h.numel() * 4
+
+    def step():
+        for k in names:
+            dev[k].copy_(pin[k], non_blocking=True)
+        y, fs = m3.m3_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["lam"], dev["theta"],
+                               dev["B"], dev["C"], s.chunk, workspace=ws)
+        y_h.copy_(y, non_blocking=True)
+        fs_h.copy_(fs, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) * 1e-3 / steps, h2d, d2h
+
+
+# ---- CPU oracle baseline ----------------------------------------------------
+
+def cpu_oracle_prefill(inp_host, s, budget_s=12.0):
+    """Time the oracle (as it stands) on whole (batch, head) chains of the same
+    workload until about `budget_s` seconds of CPU work; tokens/s counts the
+    tokens those chains cover (chains / nheads * seqlen)."""
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    total = s.batch * s.nheads
+    done, elapsed = 0, 0.0
+    step = max(cores, 1)
+    while done < total and elapsed < budget_s:
+        chains = list(range(done, min(done + step, total)))
+        t0 = time.perf_counter()
+        oracle.scan(inp_host["x"], inp_host["dt"], inp_host["A"], inp_host["lam"],
+                    inp_host["theta"], inp_host["B"], inp_host["C"], chains=chains,
+                    nthreads=cores)
+        elapsed += time.perf_counter() - t0
+        done += len(chains)
+    tokens = done / s.nheads * s.seqlen
+    return {"value": round(tokens / elapsed, 1), "unit": "tokens/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{done} of {total} (batch, head) chains, all {s.seqlen} tokens each, "
+                      f"{elapsed:.1f} s on {cores} threads"}
+
+
+# ---- main -------------------------------------------------------------------
+
+def run_reference(args, s, wname):
+    """The reference arm: the fp64 CPU oracle on the host cores, same workload
+    and metric, one bounded sample per step."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = I.make_scan_inputs(I.Workload(s), seed=1001)
+    vals = []
+    budget = max(2.0, 120.0 / max(args.steps + args.warmup, 1))
+    for i in range(args.warmup + args.steps):
+        r = cpu_oracle_prefill(inp, s, budget_s=budget)
+        if i >= args.warmup:
+            vals.append(r)
+    v = statistics.mean(r["value"] for r in vals)
+    line = {"impl": "reference", "metric": "prefill tokens/s", "value": round(v, 1),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wname, **shape_cfg(s)},
+            "cpu_baseline": {"value": round(v, 1), "unit": "tokens/s", "cores": vals[0]["cores"],
+                             "kind": "oracle", "sample": vals[0]["sample"]},
+            "e2e": {"value": round(v, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def shape_cfg(s: I.Shape):
+    return {"batch": s.batch, "seqlen": s.seqlen, "nheads": s.nheads, "headdim": s.headdim,
+            "dstate": s.dstate, "rank": s.rank, "ngroups": s.ngroups, "chunk": s.chunk,
+            "io": s.io}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="siso_prefill", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="m3", choices=["m3", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    s = WORKLOADS[args.workload].shape
+
+    if args.impl == "reference":
+        run_reference(args, s, args.workload)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    m3.load()
+    world, rank, local = dist_setup(args.gpus)
+    peaks, psrc = load_peaks()
+
+    # prefill: inputs generated on the device (seeded per rank)
+    inp = I.make_scan_inputs(I.Workload(s), seed=1001 + 7919 * rank, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        times = time_prefill(inp, s, args.steps, args.warmup, flush)
+    torch.cuda.synchronize()
+    barrier(world)
+    total = max_over_ranks(sum(times), world)
+    per_step = total / args.steps
+    tokens = s.batch * s.seqlen
+    flops, byt = prefill_work(s)
+
+    # decode (b = 128, H = 64, R as the prefill workload)
+    dw = I.DECODE_MIMO if s.rank > 1 else I.DECODE_SISO
+    ds = dw.shape
+    dsteps = args.decode_steps
+    dec = I.make_decode_inputs(dw, seed=1003 + 7919 * rank, steps=dsteps + args.warmup,
+                               device="cuda")
+    barrier(world)
+    dt_total = max_over_ranks(time_decode(dec, ds, dsteps, args.warmup), world)
+    dflops, dbyt = decode_work(ds)
+    del dec
+
+    # end to end through host buffers (inputs drawn on the host)
+    inp_host = {k: v.cpu() for k, v in inp.items()}
+    del inp
+    e2e_step, h2d, d2h = time_e2e_prefill(inp_host, s, max(3, args.steps // 4))
+    e2e_step = max_over_ranks(e2e_step, world)
+
+    launches_per_call = 3
+    line = {
+        "metric": "prefill tokens/s",
+        "value": round(world * tokens / per_step, 1),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(per_step * 1e3, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": s.io,
+        "data": "synthetic",
+        "config": {"workload": args.workload, **shape_cfg(s),
+                   "parallelism": f"dp{world} (independent batches per rank)",
+                   "l2": "flushed between timed steps (256 MiB write)",
+                   "path": "simt fp32 (3 launches per call)"},
+        "roofline": {**roofline(flops, byt, per_step, peaks, psrc),
+                     "scope": "whole m3_scan_fwd call (chunk state + state pass + chunk output)",
+                     "traffic": None, "algorithmic_flops": flops, "algorithmic_bytes": byt},
+        "decode": {
+            "metric": "decode tokens/s", "value": round(world * ds.batch * dsteps / dt_total, 1),
+            "unit": "tokens/s", "steps": dsteps, "us_per_step": round(dt_total / dsteps * 1e6, 2),
+            "config": {"workload": "decode_siso" if ds.rank == 1 else "decode_mimo",
+                       **shape_cfg(ds)},
+            "roofline": roofline(dflops, dbyt, dt_total / dsteps, peaks, psrc),
+        },
+        "e2e": {"value": round(world * tokens / e2e_step, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_step * 1e3, 3)},
+        "gpu_launches": args.steps * launches_per_call,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_prefill(inp_host, s)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+/*
+ * m3.h -- C ABI of the B200 Mamba-3 SSM layer library (libm3.so).
+ *
+ * The layer is the selective state-space recurrence of "Mamba-3: Improved
+ * Sequence Modeling using State Space Principles":
+ *   - exponential-trapezoidal discretisation (PaperWeekly page section 2.2,
+ *     "generalized trapezoidal rule"; wmrh.cn blog section 2.1):
+ *       h_t = alpha_t h_{t-1} + beta_t B_{t-1} x_{t-1}^T + gamma_t B_t x_t^T,
+ *       alpha_t = exp(dt_t A_t), gamma_t = lam_t dt_t,
+ *       beta_t = (1 - lam_t) dt_t alpha_t;
+ *   - complex-valued transition applied as data-dependent RoPE (section 2.1,
+ *     section 2.2; arXiv 2603.15569 abstract): the state rows are pairs
+ *     (2k, 2k+1); alpha_t (and the beta_t term) also rotate pair k by the angle
+ *     dt_t theta_{t,k}; equivalently B and C are rotated by the cumulative
+ *     angles;
+ *   - MIMO (section 2.3): B_t x_t^T is the rank-R product B_t (N x R) X_t^T (R x P);
+ *   - output y_t = C_t^T h_t (R x P per token and head), the real part of the
+ *     complex state read by C (section 2.1).
+ *
+ * Conventions for every call:
+ *   - Every data pointer is a DEVICE pointer owned by the caller.  The library
+ *     never allocates, frees or retains memory; it writes only the outputs
+ *     named below (and the caller's workspace).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Argument errors are detected on the host before any
+ *     launch and returned synchronously; nothing is launched then.  Launch
+ *     failures return M3_ERR_CUDA.  Faults inside kernels surface through
+ *     m3_stream_status().
+ *   - All tensors are row-major and contiguous:
+ *       x, y              [batch][seqlen][nheads][rank][headdim]   io dtype
+ *       B, C              [batch][seqlen][ngroups][rank][dstate]   io dtype
+ *       dt, A, lam        [batch][seqlen][nheads]                  fp32
+ *       theta             [batch][seqlen][ngroups][dstate/2]       fp32
+ *       h0, final_state   [batch][nheads][dstate][headdim]         fp32
+ *       B_prev            [batch][ngroups][rank][dstate]           io dtype
+ *       x_prev            [batch][nheads][rank][headdim]           io dtype
+ *     Head h reads group g = h / (nheads / ngroups).  theta is an angle RATE:
+ *     the step angle of pair k is dt * theta_k.  State pairs are adjacent rows
+ *     (2k, 2k+1); the rotation is [[cos, -sin], [sin, cos]].
+ *   - io dtype tensors (x, y, B, C, B_prev, x_prev) must be 16-byte aligned;
+ *     fp32 state tensors 16-byte aligned; dt, A, lam, theta 4-byte aligned.
+ *
+ * Supported shapes (anything else returns M3_ERR_UNSUPPORTED):
+ *   dstate N in {16, 32, 64, 128, 256}; headdim P in {16, 32, 64, 128};
+ *   N * P <= 16384; rank R in {1, 2, 4, 8}; chunk in {16, 32, 64};
+ *   batch <= 65535, nheads <= 65535.
+ */
+#ifndef M3_H_
+#define M3_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(_WIN32)
+#define M3_API __declspec(dllexport)
+#else
+#define M3_API __attribute__((visibility("default")))
+#endif
+
+/* Same underlying type as cudaStream_t / CUstream. */
+struct CUstream_st;
+typedef struct CUstream_st* m3_stream_t;
+
+/* Element type of x, y, B, C, B_prev, x_prev. */
+typedef enum { M3_F32 = 0, M3_BF16 = 1 } m3_dtype;
+
+typedef enum {
+  M3_OK = 0,
+  M3_ERR_INVALID_ARGUMENT = -1, /* null required pointer, bad extent, bad dtype */
+  M3_ERR_UNSUPPORTED = -2,      /* valid but outside the supported shape set   */
+  M3_ERR_ALIGNMENT = -3,        /* a pointer violates its alignment rule       */
+  M3_ERR_WORKSPACE = -4,        /* workspace null, misaligned or too small     */
+  M3_ERR_CUDA = -5,             /* a CUDA launch or runtime call failed        */
+  M3_ERR_TIMEOUT = -6           /* a bounded device-side wait gave up          */
+} m3_status;
+
+/* Flags (m3_shape.flags). */
+#define M3_FLAG_SIMT 1u /* force the CUDA-core fp32 scan (no tensor cores) */
+
+typedef struct {
+  int64_t batch;    /* b >= 1                                   */
+  int64_t seqlen;   /* L >= 0 (ignored by m3_decode_step)       */
+  int64_t nheads;   /* H >= 1                                   */
+  int64_t ngroups;  /* G >= 1, H % G == 0 (B, C, theta groups)  */
+  int64_t headdim;  /* P                                        */
+  int64_t dstate;   /* N (even)                                 */
+  int64_t rank;     /* R (1 = SISO)                             */
+  int64_t chunk;    /* Q, scan chunk length (ignored by decode) */
+  int32_t io_dtype; /* m3_dtype                                 */
+  uint32_t flags;   /* M3_FLAG_*; 0 = automatic choice          */
+} m3_shape;
+
+/* Library version string (static storage). */
+M3_API const char* m3_version(void);
+
+/* Human-readable name of a status code (static storage). */
+M3_API const char* m3_status_string(int status);
+
+/* Checks a shape against the rules above without touching the GPU.
+ * Returns M3_OK, M3_ERR_INVALID_ARGUMENT or M3_ERR_UNSUPPORTED. */
+M3_API int m3_check_shape(const m3_shape* shape);
+
+/* Workspace bytes that m3_scan_fwd needs for `shape` (0 when L == 0).
+ * Host-only; writes *bytes.  Returns M3_OK or the m3_check_shape error. */
+M3_API int m3_scan_workspace_size(const m3_shape* shape, size_t* bytes);
+
+/* Chunked prefill scan over a whole sequence batch: the recurrence above for
+ * every (batch, head), y_t = C_t^T h_t for every token, and the state after
+ * the last token.
+ *
+ * The scan splits each sequence into chunks of `chunk` tokens (the last chunk
+ * may be shorter).  Within a chunk it evaluates the equivalent masked
+ * quadratic form (cumulative decay times the width-2 trapezoid convolution,
+ * PaperWeekly page section 2.2, Figure 2); across chunks it passes the state.
+ *
+ *   h0          initial state h_{-1}, or NULL for zero.
+ *   B_prev,
+ *   x_prev      the token before the sequence (its B and x, not their
+ *               product): the left endpoint of the first step.  Both NULL for
+ *               none (zero), or both non-NULL.  Together with h0 this continues
+ *               a previous scan exactly.
+ *   y           output [b][L][H][R][P] in the io dtype (rounded to nearest).
+ *   final_state output h_{L-1} [b][H][N][P] fp32, or NULL to skip.  With
+ *               L == 0 it receives h0 (or zeros).
+ *   workspace   device scratch of at least m3_scan_workspace_size() bytes,
+ *               256-byte aligned; its contents on entry do not matter and are
+ *               undefined on return.  It must not be shared by scans in flight
+ *               at the same time.
+ * No input may alias an output.  Returns M3_OK when the work was enqueued. */
+M3_API int m3_scan_fwd(const m3_shape* shape, const void* x, const float* dt,
+                       const float* A, const float* lam, const float* theta,
+                       const void* B, const void* C, const float* h0,
+                       const void* B_prev, const void* x_prev, void* y,
+                       float* final_state, void* workspace,
+                       size_t workspace_bytes, m3_stream_t stream);
+
+/* One decode step for every (batch, head): reads the fp32 state once, applies
+ * the decay and rotation to it and to the previous token's left-endpoint
+ * term, adds the current token's rank-R update, writes the new state and
+ * y_t = C_t^T h_t (PaperWeekly page section 3.3; the step is memory-bound).
+ * shape->seqlen and shape->chunk are ignored.
+ *
+ *   state_in   [b][H][N][P] fp32.
+ *   state_out  [b][H][N][P] fp32; may equal state_in (in-place update), but
+ *              must not partially overlap it.
+ *   x_t        [b][H][R][P] io dtype;  dt_t, A_t, lam_t [b][H] fp32;
+ *   theta_t    [b][G][N/2] fp32;      B_t, C_t [b][G][R][N] io dtype.
+ *   B_prev,
+ *   x_prev     previous token's B [b][G][R][N] and x [b][H][R][P]; both NULL
+ *              for a zero left endpoint.
+ *   y_t        [b][H][R][P] io dtype.
+ * Returns M3_OK when the work was enqueued. */
+M3_API int m3_decode_step(const m3_shape* shape, const float* state_in,
+                          float* state_out, const void* x_t, const float* dt_t,
+                          const float* A_t, const float* lam_t,
+                          const float* theta_t, const void* B_t,
+                          const void* C_t, const void* B_prev,
+                          const void* x_prev, void* y_t, m3_stream_t stream);
+
+/* Waits for `stream`, then reports the first error since the previous call:
+ * M3_ERR_CUDA for a CUDA fault, M3_ERR_TIMEOUT if a bounded device-side wait
+ * gave up, else M3_OK.  Clears the library's device-side error word. */
+M3_API int m3_stream_status(m3_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* M3_H_ */

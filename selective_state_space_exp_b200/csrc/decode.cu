@@ -1,0 +1,174 @@
+// decode.cu -- single-token decode step of the Mamba-3 SSM layer.
+//
+// Per (batch, head) the fp32 state h (N x P) is read once and written once:
+//   g      = h + (1 - lam) dt B_prev x_prev^T          (left endpoint, rank R)
+//   h'     = alpha Rot(dt theta) g + lam dt B_t x_t^T   (pairs (2k, 2k+1))
+//   y_t    = C_t^T h'                                   (R x P)
+// This is the exponential-trapezoidal step of the paper (PaperWeekly page
+// section 2.2) with the complex transition as 2x2 rotations (section 2.1) and
+// the rank-R MIMO update (section 2.3).  The step is HBM-bound (section 3.3:
+// decode is limited by state IO, not FLOPs): 2 * 4 * N * P bytes per head.
+//
+// Layout: one CTA of 128 threads per (b, h).  Thread (kslot, pv) owns float4
+// column pv of the state and the pairs k = kslot, kslot + nslots, ...  A row
+// of the state (P floats) is read by P/4 consecutive threads as float4, so
+// each warp access is a contiguous 256-512 byte segment.  The per-head
+// operands (B, C, B_prev, x, x_prev, the cos/sin table) are staged in shared
+// memory once; y is reduced over kslots through shared memory.
+#include "m3_internal.cuh"
+
+namespace m3 {
+namespace {
+
+constexpr int kDecodeThreads = 128;
+constexpr int kPairsInFlight = 4;  // pairs loaded before any is computed
+
+template <int R>
+__global__ void __launch_bounds__(kDecodeThreads)
+decode_kernel(const DecodeArgs a) {
+  const int P = (int)a.P, N = (int)a.N, K = N / 2;
+  const int64_t bh = blockIdx.x;
+  const int64_t h = bh % a.nheads, b = bh / a.nheads;
+  const int64_t g = h / (a.nheads / a.ngroups);
+  const int64_t bg = b * a.ngroups + g;
+  const int tid = threadIdx.x;
+
+  extern __shared__ float sm[];
+  float* s_ac = sm;               // alpha cos(dt theta_k)          [K]
+  float* s_as = s_ac + K;         // alpha sin(dt theta_k)          [K]
+  float* s_Bp = s_as + K;         // B_prev                         [R][N]
+  float* s_Bt = s_Bp + R * N;     // B_t                            [R][N]
+  float* s_Ct = s_Bt + R * N;     // C_t                            [R][N]
+  float* s_xe = s_Ct + R * N;     // (1-lam) dt x_prev              [R][P]
+  float* s_xg = s_xe + R * P;     // lam dt x_t                     [R][P]
+  float* s_red = s_xg + R * P;    // partial y per kslot            [nslots][R][P]
+
+  const float dt = a.dt[bh], lamv = a.lam[bh];
+  const float alpha = expf(dt * a.A[bh]);
+  const float gamma = lamv * dt, eps = (1.f - lamv) * dt;
+  const bool prev = a.B_prev != nullptr;
+
+  for (int k = tid; k < K; k += kDecodeThreads) {
+    float sn, cs;
+    sincosf(dt * a.theta[bg * K + k], &sn, &cs);
+    s_ac[k] = alpha * cs;
+    s_as[k] = alpha * sn;
+  }
+  for (int i = tid; i < R * N; i += kDecodeThreads) {
+    s_Bt[i] = io_load(a.B, bg * R * N + i, a.bf16);
+    s_Ct[i] = io_load(a.C, bg * R * N + i, a.bf16);
+    s_Bp[i] = prev ? io_load(a.B_prev, bg * R * N + i, a.bf16) : 0.f;
+  }
+  for (int i = tid; i < R * P; i += kDecodeThreads) {
+    s_xg[i] = gamma * io_load(a.x, bh * R * P + i, a.bf16);
+    s_xe[i] = prev ? eps * io_load(a.x_prev, bh * R * P + i, a.bf16) : 0.f;
+  }
+  __syncthreads();
+
+  const int PV = P / 4;              // float4 columns per state row
+  const int nslots = kDecodeThreads / PV;
+  const int pv = tid % PV, kslot = tid / PV;
+  const int p0 = pv * 4;
+
+  float xg[R][4], xe[R][4], yacc[R][4];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      xg[r][j] = s_xg[r * P + p0 + j];
+      xe[r][j] = s_xe[r * P + p0 + j];
+      yacc[r][j] = 0.f;
+    }
+
+  const float4* src = reinterpret_cast<const float4*>(a.state_in + bh * (int64_t)N * P);
+  float4* dst = reinterpret_cast<float4*>(a.state_out + bh * (int64_t)N * P);
+
+  for (int kb = kslot; kb < K; kb += kPairsInFlight * nslots) {
+    float4 r0[kPairsInFlight], r1[kPairsInFlight];
+#pragma unroll
+    for (int u = 0; u < kPairsInFlight; ++u) {
+      const int k = kb + u * nslots;
+      if (k < K) {
+        r0[u] = __ldcs(src + (2 * k) * PV + pv);
+        r1[u] = __ldcs(src + (2 * k + 1) * PV + pv);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPairsInFlight; ++u) {
+      const int k = kb + u * nslots;
+      if (k < K) {
+        const float ac = s_ac[k], as = s_as[k];
+        float bp0[R], bp1[R], bt0[R], bt1[R], c0[R], c1[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const float2 vbp = *reinterpret_cast<const float2*>(s_Bp + r * N + 2 * k);
+          const float2 vbt = *reinterpret_cast<const float2*>(s_Bt + r * N + 2 * k);
+          const float2 vc = *reinterpret_cast<const float2*>(s_Ct + r * N + 2 * k);
+          bp0[r] = vbp.x; bp1[r] = vbp.y;
+          bt0[r] = vbt.x; bt1[r] = vbt.y;
+          c0[r] = vc.x; c1[r] = vc.y;
+        }
+        float in0[4] = {r0[u].x, r0[u].y, r0[u].z, r0[u].w};
+        float in1[4] = {r1[u].x, r1[u].y, r1[u].z, r1[u].w};
+        float o0[4], o1[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float g0 = in0[j], g1 = in1[j], u0 = 0.f, u1 = 0.f;
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            g0 = fmaf(bp0[r], xe[r][j], g0);
+            g1 = fmaf(bp1[r], xe[r][j], g1);
+            u0 = fmaf(bt0[r], xg[r][j], u0);
+            u1 = fmaf(bt1[r], xg[r][j], u1);
+          }
+          o0[j] = fmaf(ac, g0, fmaf(-as, g1, u0));
+          o1[j] = fmaf(as, g0, fmaf(ac, g1, u1));
+#pragma unroll
+          for (int r = 0; r < R; ++r)
+            yacc[r][j] = fmaf(c0[r], o0[j], fmaf(c1[r], o1[j], yacc[r][j]));
+        }
+        __stcs(dst + (2 * k) * PV + pv, make_float4(o0[0], o0[1], o0[2], o0[3]));
+        __stcs(dst + (2 * k + 1) * PV + pv, make_float4(o1[0], o1[1], o1[2], o1[3]));
+      }
+    }
+  }
+
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) s_red[(kslot * R + r) * P + p0 + j] = yacc[r][j];
+  __syncthreads();
+  for (int i = tid; i < R * P; i += kDecodeThreads) {
+    float s = 0.f;
+    for (int q = 0; q < nslots; ++q) s += s_red[q * R * P + i];
+    io_store(a.y, bh * R * P + i, s, a.bf16);
+  }
+}
+
+template <int R>
+cudaError_t launch_r(const DecodeArgs& a, cudaStream_t s) {
+  const int P = (int)a.P, N = (int)a.N;
+  const int nslots = kDecodeThreads / (P / 4);
+  const size_t smem = sizeof(float) * (N + 3 * R * N + 2 * R * P + (size_t)nslots * R * P);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<R>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  decode_kernel<R><<<(unsigned)(a.batch * a.nheads), kDecodeThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t s) {
+  switch (a.R) {
+    case 1: return launch_r<1>(a, s);
+    case 2: return launch_r<2>(a, s);
+    case 4: return launch_r<4>(a, s);
+    case 8: return launch_r<8>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace m3

@@ -1,0 +1,197 @@
+// m3_api.cu -- the C ABI declared in include/m3.h: argument checks, workspace
+// sizing, dispatch to the kernels, and the device-side error word.
+#include <cstdio>
+#include <cstring>
+
+#include "m3_internal.cuh"
+
+namespace m3 {
+
+// First device-side error raised by a kernel (M3_ERR_*), 0 if none.
+__device__ int g_device_status = 0;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+int check_common(const m3_shape* s) {
+  if (!s) return M3_ERR_INVALID_ARGUMENT;
+  if (s->batch < 1 || s->nheads < 1 || s->ngroups < 1 || s->headdim < 1 ||
+      s->dstate < 2 || s->rank < 1 || s->seqlen < 0 || s->chunk < 1)
+    return M3_ERR_INVALID_ARGUMENT;
+  if (s->dstate % 2 != 0 || s->nheads % s->ngroups != 0) return M3_ERR_INVALID_ARGUMENT;
+  if (s->io_dtype != M3_F32 && s->io_dtype != M3_BF16) return M3_ERR_INVALID_ARGUMENT;
+  if ((s->flags & ~M3_FLAG_SIMT) != 0) return M3_ERR_INVALID_ARGUMENT;
+  // supported set
+  if (!is_pow2(s->dstate) || s->dstate < 16 || s->dstate > 256) return M3_ERR_UNSUPPORTED;
+  if (!is_pow2(s->headdim) || s->headdim < 16 || s->headdim > 128) return M3_ERR_UNSUPPORTED;
+  if (s->dstate * s->headdim > 16384) return M3_ERR_UNSUPPORTED;
+  if (!(s->rank == 1 || s->rank == 2 || s->rank == 4 || s->rank == 8)) return M3_ERR_UNSUPPORTED;
+  if (!(s->chunk == 16 || s->chunk == 32 || s->chunk == 64)) return M3_ERR_UNSUPPORTED;
+  if (s->batch > 65535 || s->nheads > 65535) return M3_ERR_UNSUPPORTED;
+  if (s->batch * s->nheads > (int64_t)1 << 30) return M3_ERR_UNSUPPORTED;
+  return M3_OK;
+}
+
+ScanArgs make_scan_args(const m3_shape* s) {
+  ScanArgs a;
+  memset(&a, 0, sizeof(a));
+  a.batch = s->batch;
+  a.seqlen = s->seqlen;
+  a.nheads = s->nheads;
+  a.ngroups = s->ngroups;
+  a.P = s->headdim;
+  a.N = s->dstate;
+  a.R = s->rank;
+  a.Q = s->chunk;
+  a.nchunks = (s->seqlen + s->chunk - 1) / s->chunk;
+  a.bf16 = s->io_dtype == M3_BF16;
+  return a;
+}
+
+int status_word(int** out) {
+  // Device address of g_device_status, looked up once per device.
+  constexpr int kMaxDevices = 64;
+  static int* cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return M3_ERR_CUDA;
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return M3_ERR_CUDA;
+    cache[dev] = static_cast<int*>(p);
+  }
+  *out = cache[dev];
+  return M3_OK;
+}
+
+}  // namespace
+}  // namespace m3
+
+using namespace m3;
+
+extern "C" {
+
+M3_API const char* m3_version(void) { return "m3 0.1.0 (sm_100a)"; }
+
+M3_API const char* m3_status_string(int st) {
+  switch (st) {
+    case M3_OK: return "M3_OK";
+    case M3_ERR_INVALID_ARGUMENT: return "M3_ERR_INVALID_ARGUMENT";
+    case M3_ERR_UNSUPPORTED: return "M3_ERR_UNSUPPORTED";
+    case M3_ERR_ALIGNMENT: return "M3_ERR_ALIGNMENT";
+    case M3_ERR_WORKSPACE: return "M3_ERR_WORKSPACE";
+    case M3_ERR_CUDA: return "M3_ERR_CUDA";
+    case M3_ERR_TIMEOUT: return "M3_ERR_TIMEOUT";
+    default: return "M3_ERR_UNKNOWN";
+  }
+}
+
+M3_API int m3_check_shape(const m3_shape* s) { return check_common(s); }
+
+M3_API int m3_scan_workspace_size(const m3_shape* s, size_t* bytes) {
+  int st = check_common(s);
+  if (st != M3_OK) return st;
+  if (!bytes) return M3_ERR_INVALID_ARGUMENT;
+  if (s->seqlen == 0) {
+    *bytes = 0;
+    return M3_OK;
+  }
+  ScanArgs a = make_scan_args(s);
+  *bytes = simt_scan_workspace(a);
+  return M3_OK;
+}
+
+M3_API int m3_scan_fwd(const m3_shape* s, const void* x, const float* dt, const float* A,
+                       const float* lam, const float* theta, const void* B, const void* C,
+                       const float* h0, const void* B_prev, const void* x_prev, void* y,
+                       float* final_state, void* workspace, size_t workspace_bytes,
+                       m3_stream_t stream) {
+  int st = check_common(s);
+  if (st != M3_OK) return st;
+  if ((B_prev == nullptr) != (x_prev == nullptr)) return M3_ERR_INVALID_ARGUMENT;
+  const bool bf16 = s->io_dtype == M3_BF16;
+  if (bf16 && s->headdim % 8 != 0) return M3_ERR_UNSUPPORTED;
+  if (s->seqlen > 0 && (!x || !dt || !A || !lam || !theta || !B || !C || !y))
+    return M3_ERR_INVALID_ARGUMENT;
+  const void* v16[] = {x, B, C, y, h0, final_state, B_prev, x_prev};
+  for (const void* p : v16)
+    if (p && !aligned(p, 16)) return M3_ERR_ALIGNMENT;
+  const void* v4[] = {dt, A, lam, theta};
+  for (const void* p : v4)
+    if (p && !aligned(p, 4)) return M3_ERR_ALIGNMENT;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  if (s->seqlen == 0) {  // no token: the state is h0 (the left term waits for a token)
+    if (!final_state) return M3_OK;
+    const size_t nb = sizeof(float) * s->batch * s->nheads * s->dstate * s->headdim;
+    cudaError_t e = h0 ? cudaMemcpyAsync(final_state, h0, nb, cudaMemcpyDeviceToDevice, cs)
+                       : cudaMemsetAsync(final_state, 0, nb, cs);
+    return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+  }
+
+  ScanArgs a = make_scan_args(s);
+  const size_t need = simt_scan_workspace(a);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return M3_ERR_WORKSPACE;
+  a.x = x; a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.B = B; a.C = C;
+  a.h0 = h0; a.B_prev = B_prev; a.x_prev = x_prev; a.y = y; a.final_state = final_state;
+  a.ws = static_cast<char*>(workspace);
+  a.ws_bytes = workspace_bytes;
+  if (status_word(&a.status) != M3_OK) return M3_ERR_CUDA;
+  cudaError_t e = simt_scan_launch(a, cs);
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+M3_API int m3_decode_step(const m3_shape* s, const float* state_in, float* state_out,
+                          const void* x_t, const float* dt_t, const float* A_t,
+                          const float* lam_t, const float* theta_t, const void* B_t,
+                          const void* C_t, const void* B_prev, const void* x_prev, void* y_t,
+                          m3_stream_t stream) {
+  int st = check_common(s);
+  if (st != M3_OK) return st;
+  if ((B_prev == nullptr) != (x_prev == nullptr)) return M3_ERR_INVALID_ARGUMENT;
+  if (!state_in || !state_out || !x_t || !dt_t || !A_t || !lam_t || !theta_t || !B_t || !C_t ||
+      !y_t)
+    return M3_ERR_INVALID_ARGUMENT;
+  const bool bf16 = s->io_dtype == M3_BF16;
+  if (bf16 && s->headdim % 8 != 0) return M3_ERR_UNSUPPORTED;
+  const void* v16[] = {state_in, state_out, x_t, B_t, C_t, y_t, B_prev, x_prev};
+  for (const void* p : v16)
+    if (p && !aligned(p, 16)) return M3_ERR_ALIGNMENT;
+  const void* v4[] = {dt_t, A_t, lam_t, theta_t};
+  for (const void* p : v4)
+    if (!aligned(p, 4)) return M3_ERR_ALIGNMENT;
+  // in-place is allowed; a partial overlap is not
+  const size_t sb = sizeof(float) * s->batch * s->nheads * s->dstate * s->headdim;
+  const char* i0 = reinterpret_cast<const char*>(state_in);
+  const char* o0 = reinterpret_cast<const char*>(state_out);
+  if (i0 != o0 && i0 < o0 + sb && o0 < i0 + sb) return M3_ERR_INVALID_ARGUMENT;
+
+  DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.batch = s->batch; a.nheads = s->nheads; a.ngroups = s->ngroups;
+  a.P = s->headdim; a.N = s->dstate; a.R = s->rank; a.bf16 = bf16;
+  a.state_in = state_in; a.state_out = state_out; a.x = x_t; a.dt = dt_t; a.A = A_t;
+  a.lam = lam_t; a.theta = theta_t; a.B = B_t; a.C = C_t; a.B_prev = B_prev;
+  a.x_prev = x_prev; a.y = y_t;
+  cudaError_t e = decode_launch(a, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+M3_API int m3_stream_status(m3_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return M3_ERR_CUDA;
+  int* p = nullptr;
+  if (status_word(&p) != M3_OK) return M3_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return M3_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return M3_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+// m3_internal.cuh -- internal declarations shared by the library's .cu files.
+// Not part of the public ABI (include/m3.h is).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/m3.h"
+
+namespace m3 {
+
+// Element access for the io dtype (fp32 or bf16).
+__device__ __forceinline__ float io_load(const void* p, int64_t i, bool bf16) {
+  return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i])
+              : reinterpret_cast<const float*>(p)[i];
+}
+__device__ __forceinline__ void io_store(void* p, int64_t i, float v, bool bf16) {
+  if (bf16)
+    reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<float*>(p)[i] = v;
+}
+
+// Everything a prefill scan launch needs; pointers are device pointers.
+struct ScanArgs {
+  int64_t batch, seqlen, nheads, ngroups, P, N, R, Q, nchunks;
+  bool bf16;
+  const void* x;
+  const float* dt;
+  const float* A;
+  const float* lam;
+  const float* theta;
+  const void* B;
+  const void* C;
+  const float* h0;
+  const void* B_prev;
+  const void* x_prev;
+  void* y;
+  float* final_state;
+  char* ws;
+  size_t ws_bytes;
+  int* status;  // device-side error word
+};
+
+struct DecodeArgs {
+  int64_t batch, nheads, ngroups, P, N, R;
+  bool bf16;
+  const float* state_in;
+  float* state_out;
+  const void* x;
+  const float* dt;
+  const float* A;
+  const float* lam;
+  const float* theta;
+  const void* B;
+  const void* C;
+  const void* B_prev;
+  const void* x_prev;
+  void* y;
+};
+
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// CUDA-core fp32 scan (chunk state -> state passing -> chunk output).
+size_t simt_scan_workspace(const ScanArgs& a);
+cudaError_t simt_scan_launch(const ScanArgs& a, cudaStream_t s);
+
+// Decode step.
+cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t s);
+
+}  // namespace m3

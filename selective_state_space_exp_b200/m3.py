@@ -1,0 +1,170 @@
+"""Thin Python binding of libm3.so (the C ABI in include/m3.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  torch supplies device memory and the current stream.  There is no
+fallback: if the library is missing or the tensors are not on a CUDA device,
+the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libm3.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "m3.h")
+
+M3_F32, M3_BF16 = 0, 1
+M3_FLAG_SIMT = 1
+STATUS = {0: "M3_OK", -1: "M3_ERR_INVALID_ARGUMENT", -2: "M3_ERR_UNSUPPORTED",
+          -3: "M3_ERR_ALIGNMENT", -4: "M3_ERR_WORKSPACE", -5: "M3_ERR_CUDA",
+          -6: "M3_ERR_TIMEOUT"}
+
+
+class M3Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {status} ({STATUS.get(status, 'unknown')})")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    """m3_shape."""
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("nheads", ctypes.c_int64), ("ngroups", ctypes.c_int64),
+                ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64),
+                ("rank", ctypes.c_int64), ("chunk", ctypes.c_int64),
+                ("io_dtype", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load() -> ctypes.CDLL:
+    """Load libm3.so (built by __graft_entry__.build() or _build.py)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"libm3.so not built ({LIB_PATH}); run selective_state_space_exp_b200/_build.py")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, sp = ctypes.c_void_p, ctypes.POINTER(Shape)
+            L.m3_version.restype = ctypes.c_char_p
+            L.m3_status_string.restype = ctypes.c_char_p
+            L.m3_status_string.argtypes = [ctypes.c_int]
+            L.m3_check_shape.argtypes = [sp]
+            L.m3_check_shape.restype = ctypes.c_int
+            L.m3_scan_workspace_size.argtypes = [sp, ctypes.POINTER(ctypes.c_size_t)]
+            L.m3_scan_workspace_size.restype = ctypes.c_int
+            L.m3_scan_fwd.argtypes = [sp] + [vp] * 13 + [ctypes.c_size_t, vp]
+            L.m3_scan_fwd.restype = ctypes.c_int
+            L.m3_decode_step.argtypes = [sp] + [vp] * 13
+            L.m3_decode_step.restype = ctypes.c_int
+            L.m3_stream_status.argtypes = [vp]
+            L.m3_stream_status.restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def _check(fn: str, st: int):
+    if st != 0:
+        raise M3Error(fn, st)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _io_code(dtype: torch.dtype) -> int:
+    if dtype == torch.bfloat16:
+        return M3_BF16
+    if dtype == torch.float32:
+        return M3_F32
+    raise ValueError(f"unsupported io dtype {dtype}")
+
+
+def make_shape(batch, seqlen, nheads, ngroups, headdim, dstate, rank, chunk, io_dtype,
+               simt=False) -> Shape:
+    return Shape(batch, seqlen, nheads, ngroups, headdim, dstate, rank, chunk,
+                 _io_code(io_dtype) if isinstance(io_dtype, torch.dtype) else int(io_dtype),
+                 M3_FLAG_SIMT if simt else 0)
+
+
+def scan_shape(x: torch.Tensor, B: torch.Tensor, chunk: int, simt=False) -> Shape:
+    b, L, H, R, P = x.shape
+    G, N = B.shape[2], B.shape[4]
+    return make_shape(b, L, H, G, P, N, R, chunk, x.dtype, simt)
+
+
+def workspace_size(shape: Shape) -> int:
+    n = ctypes.c_size_t(0)
+    _check("m3_scan_workspace_size", load().m3_scan_workspace_size(ctypes.byref(shape),
+                                                                   ctypes.byref(n)))
+    return int(n.value)
+
+
+def m3_scan_fwd(x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None, B_prev=None,
+                x_prev=None, *, y=None, final_state=None, want_final=True, workspace=None,
+                simt=False, stream=None):
+    """Chunked prefill scan.  x [b][L][H][R][P] (io dtype), dt/A/lam [b][L][H],
+    theta [b][L][G][N/2] fp32, B/C [b][L][G][R][N] (io dtype).  R is x.shape[3].
+    Returns (y, final_state)."""
+    shape = scan_shape(x, B, chunk, simt)
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and want_final:
+        final_state = torch.empty((x.shape[0], x.shape[2], B.shape[4], x.shape[4]),
+                                  dtype=torch.float32, device=x.device)
+    need = workspace_size(shape)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    st = load().m3_scan_fwd(ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(lam),
+                            _ptr(theta), _ptr(B), _ptr(C), _ptr(h0), _ptr(B_prev),
+                            _ptr(x_prev), _ptr(y), _ptr(final_state), _ptr(workspace),
+                            ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check("m3_scan_fwd", st)
+    return y, final_state
+
+
+def m3_decode_step(state, x_t, dt, A, lam, theta, B_t, C_t, B_prev=None, x_prev=None, *,
+                   state_out=None, y=None, stream=None):
+    """One decode step.  state [b][H][N][P] fp32; x_t [b][H][R][P]; dt/A/lam [b][H];
+    theta [b][G][N/2]; B_t/C_t [b][G][R][N].  state_out defaults to `state`
+    (in place).  Returns (y_t, state_out)."""
+    b, H, R, P = x_t.shape
+    G, N = B_t.shape[1], B_t.shape[3]
+    shape = make_shape(b, 1, H, G, P, N, R, 64, x_t.dtype)
+    if state_out is None:
+        state_out = state
+    if y is None:
+        y = torch.empty_like(x_t)
+    st = load().m3_decode_step(ctypes.byref(shape), _ptr(state), _ptr(state_out), _ptr(x_t),
+                               _ptr(dt), _ptr(A), _ptr(lam), _ptr(theta), _ptr(B_t),
+                               _ptr(C_t), _ptr(B_prev), _ptr(x_prev), _ptr(y),
+                               _stream(stream))
+    _check("m3_decode_step", st)
+    return y, state_out
+
+
+def m3_stream_status(stream=None) -> int:
+    """Synchronise the stream and return the first device-side status."""
+    return int(load().m3_stream_status(_stream(stream)))
+
+
+def version() -> str:
+    return load().m3_version().decode()

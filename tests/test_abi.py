@@ -1,0 +1,124 @@
+"""The C ABI library: it builds, loads, exports every symbol include/m3.h
+declares, and rejects bad arguments on the host before touching the GPU.
+No test here launches a kernel."""
+import ctypes
+import re
+
+import pytest
+
+from selective_state_space_exp_b200 import _build, m3
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return m3.load()
+
+
+def declared_functions():
+    src = open(m3.HEADER).read()
+    return re.findall(r"M3_API\s+[\w\s\*]+?\b(m3_\w+)\s*\(", src)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    assert {"m3_scan_fwd", "m3_decode_step", "m3_scan_workspace_size", "m3_stream_status",
+            "m3_check_shape", "m3_status_string", "m3_version"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_version_and_status_strings(lib):
+    assert b"sm_100a" in lib.m3_version()
+    for code, name in m3.STATUS.items():
+        assert lib.m3_status_string(code).decode() == name
+
+
+def shape(**kw):
+    d = dict(batch=2, seqlen=100, nheads=4, ngroups=1, headdim=64, dstate=128, rank=1,
+             chunk=64, io_dtype=m3.M3_BF16, flags=0)
+    d.update(kw)
+    return m3.Shape(**d)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    ({}, 0),
+    (dict(rank=4), 0), (dict(rank=8, headdim=16, dstate=16), 0),
+    (dict(dstate=16, headdim=16, io_dtype=m3.M3_F32), 0),
+    (dict(seqlen=0), 0),
+    (dict(batch=0), -1), (dict(nheads=0), -1), (dict(seqlen=-1), -1),
+    (dict(dstate=127), -1), (dict(nheads=6, ngroups=4), -1), (dict(io_dtype=7), -1),
+    (dict(flags=2), -1), (dict(chunk=0), -1),
+    (dict(rank=3), -2), (dict(dstate=96), -2), (dict(headdim=48), -2),
+    (dict(headdim=256), -2), (dict(dstate=256, headdim=128), -2), (dict(chunk=48), -2),
+    (dict(chunk=128), -2), (dict(batch=70000), -2),
+])
+def test_check_shape(lib, kw, expect):
+    s = shape(**kw)
+    assert lib.m3_check_shape(ctypes.byref(s)) == expect
+
+
+def test_workspace_size(lib):
+    n = ctypes.c_size_t()
+    s = shape(seqlen=0)
+    assert lib.m3_scan_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0 and n.value == 0
+    s = shape(seqlen=130)  # 3 chunks, the last ragged
+    assert lib.m3_scan_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0
+    assert n.value >= 2 * 4 * 3 * 128 * 64 * 4  # one N x P fp32 state per chunk-head
+    assert lib.m3_scan_workspace_size(ctypes.byref(s), None) == -1
+    assert lib.m3_scan_workspace_size(None, ctypes.byref(n)) == -1
+
+
+# Fake, never dereferenced device addresses: every case below fails a host
+# check before any CUDA call is made.
+A16 = 0x7f0000000000
+P = [ctypes.c_void_p(A16 + 0x100000 * i) for i in range(16)]
+
+
+def scan_call(lib, s, **over):
+    args = dict(x=P[0], dt=P[1], A=P[2], lam=P[3], theta=P[4], B=P[5], C=P[6], h0=None,
+                B_prev=None, x_prev=None, y=P[7], fs=P[8], ws=P[9], wsb=0, stream=None)
+    args.update(over)
+    return lib.m3_scan_fwd(None if s is None else ctypes.byref(s), args["x"], args["dt"], args["A"], args["lam"],
+                           args["theta"], args["B"], args["C"], args["h0"], args["B_prev"],
+                           args["x_prev"], args["y"], args["fs"], args["ws"],
+                           ctypes.c_size_t(args["wsb"]), args["stream"])
+
+
+def test_scan_rejects_bad_arguments(lib):
+    s = shape()
+    assert scan_call(lib, s, x=None) == -1
+    assert scan_call(lib, s, y=None) == -1
+    assert scan_call(lib, s, theta=None) == -1
+    assert scan_call(lib, s, B_prev=P[10]) == -1           # B_prev without x_prev
+    assert scan_call(lib, s, x=ctypes.c_void_p(A16 + 8)) == -3
+    assert scan_call(lib, s, y=ctypes.c_void_p(A16 + 2)) == -3
+    assert scan_call(lib, s, dt=ctypes.c_void_p(A16 + 2)) == -3
+    assert scan_call(lib, s, ws=None) == -4
+    assert scan_call(lib, s, wsb=16) == -4
+    assert scan_call(lib, s, ws=ctypes.c_void_p(A16 + 16), wsb=1 << 40) == -4
+    assert scan_call(lib, shape(rank=3)) == -2
+    assert scan_call(lib, None) == -1
+
+
+def decode_call(lib, s, **over):
+    args = dict(si=P[0], so=P[0], x=P[1], dt=P[2], A=P[3], lam=P[4], theta=P[5], B=P[6],
+                C=P[7], Bp=None, xp=None, y=P[8], stream=None)
+    args.update(over)
+    return lib.m3_decode_step(ctypes.byref(s), args["si"], args["so"], args["x"], args["dt"],
+                              args["A"], args["lam"], args["theta"], args["B"], args["C"],
+                              args["Bp"], args["xp"], args["y"], args["stream"])
+
+
+def test_decode_rejects_bad_arguments(lib):
+    s = shape()
+    assert decode_call(lib, s, si=None) == -1
+    assert decode_call(lib, s, y=None) == -1
+    assert decode_call(lib, s, xp=P[9]) == -1                       # x_prev without B_prev
+    assert decode_call(lib, s, so=ctypes.c_void_p(A16 + 64)) == -1  # partial overlap
+    assert decode_call(lib, s, x=ctypes.c_void_p(A16 + 0x100000 + 4)) == -3
+    assert decode_call(lib, s, lam=ctypes.c_void_p(A16 + 1)) == -3
+    assert decode_call(lib, shape(headdim=24)) == -2

@@ -1,0 +1,237 @@
+"""Parity of the CUDA path (called through the C ABI) with the fp64 oracle.
+
+Bars (max |err| / max |ref|, y and final state separately): 1e-4 for fp32 io,
+2e-2 for bf16 io with fp32 accumulation and state.  Small cases compare every
+output; full-size workloads compare a seeded sample of (batch, head) chains,
+which the oracle computes independently of the others.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from selective_state_space_exp_b200 import inputs as I
+from selective_state_space_exp_b200 import m3
+from parity_helpers import (TOL, chain_rows, compare_scan, gpu_scan, need_gpu, oracle_scan,
+                            rel_err, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    need_gpu()
+
+
+def small(batch=2, L=250, H=4, P=16, N=16, R=1, G=1, chunk=64, io="f32", bc="normal",
+          decay="fast", h0=False, prev=False):
+    return I.Workload(I.Shape(batch, L, H, P, N, R, G, chunk, io), bc=bc, decay=decay,
+                      with_h0=h0, with_prev=prev)
+
+
+def check(errs, io):
+    ey, eh = errs
+    assert ey <= TOL[io] and eh <= TOL[io], f"err y {ey:.3e}, state {eh:.3e} (bar {TOL[io]})"
+
+
+# ---- prefill scan -----------------------------------------------------------
+
+def test_tiny_siso_fp32_full():
+    """The 256-token fp32 SISO case, every output against the oracle at 1e-4."""
+    w = I.TINY_SISO_F32
+    inp = I.make_scan_inputs(w, seed=1000)
+    check(compare_scan(inp, w.shape.chunk, "f32"), "f32")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("R", [1, 2, 4, 8])
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_ragged_small(io, R, chunk):
+    """L = 250 (ragged last chunk), several tiles, initial state and previous token."""
+    w = small(L=250, R=R, chunk=chunk, io=io, P=32, N=32, h0=True, prev=True,
+              bc="rmsnorm" if io == "bf16" else "normal")
+    inp = I.make_scan_inputs(w, seed=2000 + 10 * R + chunk)
+    check(compare_scan(inp, chunk, io), io)
+
+
+@pytest.mark.parametrize("N,P", [(16, 128), (256, 16), (64, 64), (128, 64)])
+def test_shapes_grouped(N, P):
+    """Groups G = H (per-head B, C, theta) and G = 2, slow decay so that every
+    chunk's state reaches the next one."""
+    for G in (2, 4):
+        w = small(batch=2, L=200, H=4, G=G, N=N, P=P, R=2, io="f32", decay="slow", h0=True,
+                  prev=True)
+        inp = I.make_scan_inputs(w, seed=3000 + N + P + G)
+        check(compare_scan(inp, 64, "f32"), "f32")
+
+
+@pytest.mark.parametrize("L", [1, 63, 64, 65, 129])
+def test_edge_lengths(L):
+    w = small(L=L, R=2, io="f32", h0=True, prev=True, decay="slow")
+    inp = I.make_scan_inputs(w, seed=4000 + L)
+    check(compare_scan(inp, 64, "f32"), "f32")
+
+
+def test_empty_sequence_returns_h0():
+    w = small(L=0, h0=True)
+    inp = to_dev(I.make_scan_inputs(w, seed=4100))
+    y, fs = m3.m3_scan_fwd(inp["x"], inp["dt"], inp["A"], inp["lam"], inp["theta"], inp["B"],
+                           inp["C"], 64, inp["h0"])
+    assert y.numel() == 0
+    assert torch.equal(fs, inp["h0"])
+    _, fs0 = m3.m3_scan_fwd(inp["x"], inp["dt"], inp["A"], inp["lam"], inp["theta"], inp["B"],
+                            inp["C"], 64)
+    assert torch.count_nonzero(fs0) == 0
+
+
+def test_chunk_invariance():
+    """The chunk length is a performance parameter only (fp32 io, slow decay)."""
+    w = small(L=300, R=4, P=32, N=64, io="f32", decay="slow", h0=True, prev=True)
+    inp = I.make_scan_inputs(w, seed=4200)
+    outs = [gpu_scan(inp, q) for q in (16, 32, 64)]
+    for y, h in outs[1:]:
+        assert rel_err(y, outs[0][0]) < 1e-5 and rel_err(h, outs[0][1]) < 1e-5
+
+
+def test_split_continuation_on_gpu():
+    """scan(L0) then scan(L1) seeded with (final state, last B, last x) equals
+    scan(L0 + L1)."""
+    w = small(L=200, R=2, P=32, N=32, io="f32", decay="slow", h0=True, prev=True)
+    inp = I.make_scan_inputs(w, seed=4300)
+    y, h = gpu_scan(inp, 64)
+    L0 = 77
+    seq = ("x", "dt", "A", "lam", "theta", "B", "C")
+    a = {k: (v[:, :L0].contiguous() if k in seq else v) for k, v in inp.items()}
+    ya, ha = gpu_scan(a, 64)
+    b = {k: (v[:, L0:].contiguous() if k in seq else v) for k, v in inp.items()}
+    b["h0"] = torch.from_numpy(ha)
+    b["B_prev"] = inp["B"][:, L0 - 1].contiguous()
+    b["x_prev"] = inp["x"][:, L0 - 1].contiguous()
+    yb, hb = gpu_scan(b, 64)
+    assert rel_err(np.concatenate([ya, yb], axis=1), y) < 1e-5
+    assert rel_err(hb, h) < 1e-5
+
+
+def test_slow_decay_siso_and_mimo():
+    """Config-1 shapes (two sequences) with slow decay, so the inter-chunk state
+    passing carries most of the output."""
+    for R in (1, 4):
+        w = I.Workload(I.Shape(2, 2048, 64, 64, 128, R, 1, 64, "bf16"), decay="slow",
+                       with_h0=True, with_prev=True)
+        inp = I.make_scan_inputs(w, seed=4400 + R)
+        check(compare_scan(inp, 64, "bf16", nsample=6), "bf16")
+
+
+@pytest.mark.parametrize("w,seed", [(I.SISO_PREFILL, 1001), (I.MIMO_PREFILL, 1002)],
+                         ids=["siso_prefill_b8_L2048", "mimo_r4_prefill_b8_L2048"])
+def test_full_size_prefill(w, seed):
+    inp = I.make_scan_inputs(w, seed=seed)
+    check(compare_scan(inp, w.shape.chunk, "bf16", nsample=6), "bf16")
+
+
+@pytest.mark.parametrize("w,seed", [(I.LONG_MIMO_16K, 1014), (I.LONG_MIMO_32K, 1004)],
+                         ids=["mimo_r4_L16384", "mimo_r4_L32768"])
+def test_long_context_prefill(w, seed):
+    inp = I.make_scan_inputs(w, seed=seed)
+    check(compare_scan(inp, w.shape.chunk, "bf16", nsample=3), "bf16")
+
+
+# ---- decode step ------------------------------------------------------------
+
+def gpu_decode(dec: dict, steps: int, in_place=True):
+    g = to_dev(dec)
+    state = g["state0"].clone()
+    ys = []
+    for t in range(steps):
+        Bp = g["B_prev"] if t == 0 else g["B"][t - 1]
+        xp = g["x_prev"] if t == 0 else g["x"][t - 1]
+        out = None if in_place else torch.empty_like(state)
+        y, state = m3.m3_decode_step(state, g["x"][t], g["dt"][t], g["A"][t], g["lam"][t],
+                                     g["theta"][t], g["B"][t], g["C"][t], Bp, xp,
+                                     state_out=out)
+        ys.append(y)
+    assert m3.m3_stream_status() == 0
+    return torch.stack(ys, 1).float().cpu().numpy(), state.cpu().numpy()
+
+
+def decode_as_scan(dec: dict) -> dict:
+    """Decode inputs [steps][b]... rearranged into scan layout [b][steps]..."""
+    out = {k: dec[k].transpose(0, 1).contiguous() for k in ("x", "dt", "A", "lam", "theta",
+                                                            "B", "C")}
+    out.update(h0=dec["state0"], B_prev=dec["B_prev"], x_prev=dec["x_prev"])
+    return out
+
+
+@pytest.mark.parametrize("w", [I.DECODE_SISO, I.DECODE_MIMO], ids=["R1", "R4"])
+def test_decode_full_batch(w):
+    """b = 128, H = 64 decode steps against the oracle on sampled chains."""
+    steps = 6
+    dec = I.make_decode_inputs(w, seed=1003 if w.shape.rank == 1 else 1013, steps=steps)
+    yg, hg = gpu_decode(dec, steps)
+    sc = decode_as_scan(dec)
+    b, H = w.shape.batch, w.shape.nheads
+    chains = I.sample_chains(b, H, 8)
+    yo, ho = oracle_scan(sc, chains)
+    gy, gh = chain_rows(yg, hg, chains, H)
+    oy, oh = chain_rows(yo, ho, chains, H)
+    check((rel_err(gy, oy), rel_err(gh, oh)), "bf16")
+
+
+def test_decode_1024_consecutive_steps():
+    """1024 consecutive steps (R = 4, two sequences) against the oracle."""
+    w = I.Workload(I.Shape(2, 1, 64, 64, 128, 4, 1, 64, "bf16"), with_h0=True, with_prev=True)
+    steps = 1024
+    dec = I.make_decode_inputs(w, seed=1023, steps=steps)
+    yg, hg = gpu_decode(dec, steps)
+    chains = I.sample_chains(2, 64, 6)
+    yo, ho = oracle_scan(decode_as_scan(dec), chains)
+    gy, gh = chain_rows(yg, hg, chains, 64)
+    oy, oh = chain_rows(yo, ho, chains, 64)
+    check((rel_err(gy, oy), rel_err(gh, oh)), "bf16")
+
+
+def test_decode_fp32_small_every_output():
+    w = I.Workload(I.Shape(3, 1, 4, 16, 32, 2, 2, 64, "f32"), bc="normal", with_h0=True,
+                   with_prev=True)
+    dec = I.make_decode_inputs(w, seed=5000, steps=40)
+    yg, hg = gpu_decode(dec, 40)
+    yo, ho = oracle_scan(decode_as_scan(dec))
+    check((rel_err(yg, yo), rel_err(hg, ho)), "f32")
+
+
+def test_decode_in_place_equals_out_of_place():
+    w = I.Workload(I.Shape(4, 1, 8, 64, 128, 4, 1, 64, "bf16"), with_h0=True, with_prev=True)
+    dec = I.make_decode_inputs(w, seed=5100, steps=3)
+    y1, h1 = gpu_decode(dec, 3, in_place=True)
+    y2, h2 = gpu_decode(dec, 3, in_place=False)
+    assert np.array_equal(y1, y2) and np.array_equal(h1, h2)
+
+
+def test_decode_equals_scan_on_gpu():
+    """Driving the decode kernel token by token reproduces the scan kernels
+    (fp32 io)."""
+    w = I.Workload(I.Shape(2, 1, 4, 32, 64, 2, 1, 64, "f32"), bc="normal", decay="slow",
+                   with_h0=True, with_prev=True)
+    dec = I.make_decode_inputs(w, seed=5200, steps=150)
+    yd, hd = gpu_decode(dec, 150)
+    ys, hs = gpu_scan(decode_as_scan(dec), 32)
+    assert rel_err(yd, ys) < 1e-5 and rel_err(hd, hs) < 1e-5
+
+
+def test_gpu_rejects_bad_pointers():
+    """Host-side checks with real device tensors: misaligned views and a small
+    workspace return errors and launch nothing."""
+    w = small(L=64, R=1, P=16, N=16, io="f32")
+    inp = to_dev(I.make_scan_inputs(w, seed=5300))
+    flat = torch.zeros(inp["x"].numel() + 4, device="cuda")
+    x_mis = flat[1:1 + inp["x"].numel()].view_as(inp["x"])
+    with pytest.raises(m3.M3Error) as e:
+        m3.m3_scan_fwd(x_mis, inp["dt"], inp["A"], inp["lam"], inp["theta"], inp["B"],
+                       inp["C"], 64)
+    assert e.value.status == -3
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(m3.M3Error) as e:
+        m3.m3_scan_fwd(inp["x"], inp["dt"], inp["A"], inp["lam"], inp["theta"], inp["B"],
+                       inp["C"], 64, workspace=ws)
+    assert e.value.status == -4
+    assert m3.m3_stream_status() == 0
