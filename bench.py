@@ -351,6 +351,8 @@ def main():
     ap.add_argument("--impl", default="m3", choices=["m3", "reference"])
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="run one part only (for profiling); prints its own line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     s = WORKLOADS[args.workload].shape
@@ -364,6 +366,25 @@ def main():
     m3.load()
     world, rank, local = dist_setup(args.gpus)
     peaks, psrc = load_peaks()
+
+    if args.only == "decode":
+        dw = I.DECODE_MIMO if s.rank > 1 else I.DECODE_SISO
+        dec = I.make_decode_inputs(dw, seed=1003, steps=args.decode_steps + args.warmup,
+                                   device="cuda")
+        t = time_decode(dec, dw.shape, args.decode_steps, args.warmup)
+        dflops, dbyt = decode_work(dw.shape)
+        print(json.dumps({"only": "decode", "us_per_step": round(t / args.decode_steps * 1e6, 2),
+                          "roofline": roofline(dflops, dbyt, t / args.decode_steps, peaks, psrc)}))
+        return
+    if args.only == "prefill":
+        inp = I.make_scan_inputs(I.Workload(s), seed=1001, device="cuda")
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        times = time_prefill(inp, s, args.steps, args.warmup, flush)
+        flops, byt = prefill_work(s)
+        per = sum(times) / len(times)
+        print(json.dumps({"only": "prefill", "ms_per_step": round(per * 1e3, 4),
+                          "roofline": roofline(flops, byt, per, peaks, psrc)}))
+        return
 
     # prefill: inputs generated on the device (seeded per rank)
     inp = I.make_scan_inputs(I.Workload(s), seed=1001 + 7919 * rank, device="cuda")
