@@ -161,6 +161,36 @@ M3_API int m3_decode_step(const m3_shape* shape, const float* state_in,
                           const void* C_t, const void* B_prev,
                           const void* x_prev, void* y_t, m3_stream_t stream);
 
+/* Size of the fixed device scratch array used by m3_scan_fwd_noalloc (16 MiB). */
+#define M3_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/* m3_scan_fwd for callers that cannot allocate device memory: for example a
+ * plugin whose host framework owns all device memory and offers it no
+ * allocator, or a caller on a path where a cudaMalloc (which may synchronise
+ * the device) is not acceptable.  The caller passes inputs and outputs only;
+ * the scratch memory that m3_scan_fwd takes as `workspace` comes from a
+ * library-owned static device array of M3_NOALLOC_SCRATCH_BYTES, which every
+ * GPU that loads the library holds until the process exits.  The paper has no
+ * counterpart to this call; it only changes where the scratch lives.
+ *
+ *   - Arguments, layouts, outputs and errors are those of m3_scan_fwd.
+ *   - Shapes whose workspace (m3_scan_workspace_size) exceeds
+ *     M3_NOALLOC_SCRATCH_BYTES return M3_ERR_WORKSPACE and launch nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
+ *     library routine.
+ *   - All calls on a device share the array, which keeps the last call's
+ *     contents; every scratch element is written before it is read, so
+ *     nothing needs clearing.  Calls that overlap on the GPU (unordered
+ *     streams or host threads) race on the array: order them on one stream. */
+M3_API int m3_scan_fwd_noalloc(const m3_shape* shape, const void* x, const float* dt,
+                               const float* A, const float* lam, const float* theta,
+                               const void* B, const void* C, const float* h0,
+                               const void* B_prev, const void* x_prev, void* y,
+                               float* final_state, m3_stream_t stream);
+
 /* Waits for `stream`, then reports the first error since the previous call:
  * M3_ERR_CUDA for a CUDA fault, M3_ERR_TIMEOUT if a bounded device-side wait
  * gave up, else M3_OK.  Clears the library's device-side error word. */

@@ -62,6 +62,8 @@ def load() -> ctypes.CDLL:
             L.m3_scan_workspace_size.restype = ctypes.c_int
             L.m3_scan_fwd.argtypes = [sp] + [vp] * 13 + [ctypes.c_size_t, vp]
             L.m3_scan_fwd.restype = ctypes.c_int
+            L.m3_scan_fwd_noalloc.argtypes = [sp] + [vp] * 13
+            L.m3_scan_fwd_noalloc.restype = ctypes.c_int
             L.m3_decode_step.argtypes = [sp] + [vp] * 13
             L.m3_decode_step.restype = ctypes.c_int
             L.m3_stream_status.argtypes = [vp]
@@ -138,6 +140,25 @@ def m3_scan_fwd(x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None, B_prev=Non
                             _ptr(x_prev), _ptr(y), _ptr(final_state), _ptr(workspace),
                             ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check("m3_scan_fwd", st)
+    return y, final_state
+
+
+def m3_scan_fwd_noalloc(x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None, B_prev=None,
+                        x_prev=None, *, y=None, final_state=None, want_final=True, simt=False,
+                        stream=None):
+    """m3_scan_fwd without a workspace argument: the library's fixed device
+    scratch (M3_NOALLOC_SCRATCH_BYTES) serves instead, for callers that cannot
+    allocate device memory.  Returns (y, final_state)."""
+    shape = scan_shape(x, B, chunk, simt)
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and want_final:
+        final_state = torch.empty((x.shape[0], x.shape[2], B.shape[4], x.shape[4]),
+                                  dtype=torch.float32, device=x.device)
+    st = load().m3_scan_fwd_noalloc(ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(lam),
+                                    _ptr(theta), _ptr(B), _ptr(C), _ptr(h0), _ptr(B_prev),
+                                    _ptr(x_prev), _ptr(y), _ptr(final_state), _stream(stream))
+    _check("m3_scan_fwd_noalloc", st)
     return y, final_state
 
 
