@@ -66,6 +66,14 @@ int status_word(int** out) {
   return M3_OK;
 }
 
+bool use_tc(const m3_shape* s, const ScanArgs& a) {
+  return (s->flags & M3_FLAG_SIMT) == 0 && tc_scan_supported(a);
+}
+
+size_t scan_workspace(const m3_shape* s, const ScanArgs& a) {
+  return use_tc(s, a) ? tc_scan_workspace(a) : simt_scan_workspace(a);
+}
+
 }  // namespace
 }  // namespace m3
 
@@ -99,7 +107,7 @@ M3_API int m3_scan_workspace_size(const m3_shape* s, size_t* bytes) {
     return M3_OK;
   }
   ScanArgs a = make_scan_args(s);
-  *bytes = simt_scan_workspace(a);
+  *bytes = scan_workspace(s, a);
   return M3_OK;
 }
 
@@ -132,14 +140,15 @@ M3_API int m3_scan_fwd(const m3_shape* s, const void* x, const float* dt, const 
   }
 
   ScanArgs a = make_scan_args(s);
-  const size_t need = simt_scan_workspace(a);
-  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return M3_ERR_WORKSPACE;
+  const size_t need = scan_workspace(s, a);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
+    return M3_ERR_WORKSPACE;
   a.x = x; a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.B = B; a.C = C;
   a.h0 = h0; a.B_prev = B_prev; a.x_prev = x_prev; a.y = y; a.final_state = final_state;
   a.ws = static_cast<char*>(workspace);
   a.ws_bytes = workspace_bytes;
   if (status_word(&a.status) != M3_OK) return M3_ERR_CUDA;
-  cudaError_t e = simt_scan_launch(a, cs);
+  cudaError_t e = use_tc(s, a) ? tc_scan_launch(a, cs) : simt_scan_launch(a, cs);
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 

@@ -66,6 +66,11 @@ __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a -
 size_t simt_scan_workspace(const ScanArgs& a);
 cudaError_t simt_scan_launch(const ScanArgs& a, cudaStream_t s);
 
+// Tensor-core (tcgen05) scan for bf16 io, N = 128, P = 64, Q*R in {64, 128, 256}.
+bool tc_scan_supported(const ScanArgs& a);
+size_t tc_scan_workspace(const ScanArgs& a);
+cudaError_t tc_scan_launch(const ScanArgs& a, cudaStream_t s);
+
 // Decode step.
 cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t s);
 

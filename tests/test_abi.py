@@ -65,9 +65,17 @@ def test_workspace_size(lib):
     n = ctypes.c_size_t()
     s = shape(seqlen=0)
     assert lib.m3_scan_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0 and n.value == 0
-    s = shape(seqlen=130)  # 3 chunks, the last ragged
+    # CUDA-core path: one N x P fp32 state per chunk-head (3 chunks, the last ragged)
+    s = shape(seqlen=130, flags=m3.M3_FLAG_SIMT)
     assert lib.m3_scan_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0
-    assert n.value >= 2 * 4 * 3 * 128 * 64 * 4  # one N x P fp32 state per chunk-head
+    assert n.value >= 2 * 4 * 3 * 128 * 64 * 4
+    # tensor-core path: 8 chains are cut into 3 segments -> 2 carried states per chain
+    s = shape(seqlen=130)
+    assert lib.m3_scan_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0
+    assert 2 * 4 * 2 * 128 * 64 * 4 <= n.value < 2 * 4 * 3 * 128 * 64 * 4
+    # many chains: one segment per chain, no workspace at all
+    s = shape(batch=8, nheads=64, seqlen=2048)
+    assert lib.m3_scan_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0 and n.value == 0
     assert lib.m3_scan_workspace_size(ctypes.byref(s), None) == -1
     assert lib.m3_scan_workspace_size(None, ctypes.byref(n)) == -1
 

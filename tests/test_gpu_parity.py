@@ -122,11 +122,44 @@ def test_slow_decay_siso_and_mimo():
         check(compare_scan(inp, 64, "bf16", nsample=6), "bf16")
 
 
+@pytest.mark.parametrize("simt", [False, True], ids=["tcgen05", "cuda_core"])
 @pytest.mark.parametrize("w,seed", [(I.SISO_PREFILL, 1001), (I.MIMO_PREFILL, 1002)],
                          ids=["siso_prefill_b8_L2048", "mimo_r4_prefill_b8_L2048"])
-def test_full_size_prefill(w, seed):
+def test_full_size_prefill(w, seed, simt):
     inp = I.make_scan_inputs(w, seed=seed)
-    check(compare_scan(inp, w.shape.chunk, "bf16", nsample=6), "bf16")
+    check(compare_scan(inp, w.shape.chunk, "bf16", nsample=6, simt=simt), "bf16")
+
+
+# ---- tensor-core path: every tile shape, segments, ragged tails ----------------
+
+@pytest.mark.parametrize("R,chunk", [(1, 64), (2, 64), (2, 32), (4, 64), (4, 32), (4, 16)])
+@pytest.mark.parametrize("L,batch,H", [(250, 1, 4), (700, 2, 8)])
+def test_tc_tiles_segments_ragged(R, chunk, L, batch, H):
+    """N = 128, P = 64 bf16: M = chunk * R rows of 64, 128 or 256; few chains,
+    so every chain is cut into several segments; ragged last chunk; initial
+    state and previous token; slow decay so the carried state matters."""
+    w = I.Workload(I.Shape(batch, L, H, 64, 128, R, 1, chunk, "bf16"), decay="slow",
+                   with_h0=True, with_prev=True)
+    inp = I.make_scan_inputs(w, seed=7000 + 10 * R + chunk + L)
+    check(compare_scan(inp, chunk, "bf16"), "bf16")
+
+
+@pytest.mark.parametrize("R", [1, 4])
+def test_tc_groups_and_fast_decay(R):
+    """G = H (per-head B, C, theta) and the workload's fast decay."""
+    w = I.Workload(I.Shape(2, 300, 4, 64, 128, R, 4, 64, "bf16"), with_h0=True, with_prev=True)
+    inp = I.make_scan_inputs(w, seed=7100 + R)
+    check(compare_scan(inp, 64, "bf16"), "bf16")
+
+
+def test_tc_matches_cuda_core_path():
+    """The two GPU paths agree with each other (bf16 io) to the bf16 bar."""
+    w = I.Workload(I.Shape(2, 512, 8, 64, 128, 4, 1, 64, "bf16"), decay="slow", with_h0=True,
+                   with_prev=True)
+    inp = I.make_scan_inputs(w, seed=7200)
+    y_tc, h_tc = gpu_scan(inp, 64, simt=False)
+    y_sc, h_sc = gpu_scan(inp, 64, simt=True)
+    assert rel_err(y_tc, y_sc) <= TOL["bf16"] and rel_err(h_tc, h_sc) <= TOL["bf16"]
 
 
 @pytest.mark.parametrize("w,seed", [(I.LONG_MIMO_16K, 1014), (I.LONG_MIMO_32K, 1004)],

@@ -52,7 +52,7 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     M3_ERR_WORKSPACE on the host and launches nothing."""
     _build.build()
     lib = m3.load()
-    s = m3.Shape(8, 2048, 64, 1, 64, 128, 1, 64, m3.M3_BF16, 0)
+    s = m3.Shape(8, 2048, 64, 1, 64, 128, 1, 64, m3.M3_BF16, m3.M3_FLAG_SIMT)
     n = ctypes.c_size_t()
     assert lib.m3_scan_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0
     assert n.value > 16 * 1024 * 1024
