@@ -37,8 +37,8 @@
  *     Head h reads group g = h / (nheads / ngroups).  theta is an angle RATE:
  *     the step angle of pair k is dt * theta_k.  State pairs are adjacent rows
  *     (2k, 2k+1); the rotation is [[cos, -sin], [sin, cos]].
- *   - io dtype tensors (x, y, B, C, B_prev, x_prev) must be 16-byte aligned;
- *     fp32 state tensors 16-byte aligned; dt, A, lam, theta 4-byte aligned.
+ *   - io dtype tensors (x, y, B, C, B_prev, x_prev), fp32 state tensors and
+ *     theta must be 16-byte aligned; dt, A, lam 4-byte aligned.
  *
  * Supported shapes (anything else returns M3_ERR_UNSUPPORTED):
  *   dstate N in {16, 32, 64, 128, 256}; headdim P in {16, 32, 64, 128};

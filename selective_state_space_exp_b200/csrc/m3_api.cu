@@ -123,10 +123,10 @@ M3_API int m3_scan_fwd(const m3_shape* s, const void* x, const float* dt, const 
   if (bf16 && s->headdim % 8 != 0) return M3_ERR_UNSUPPORTED;
   if (s->seqlen > 0 && (!x || !dt || !A || !lam || !theta || !B || !C || !y))
     return M3_ERR_INVALID_ARGUMENT;
-  const void* v16[] = {x, B, C, y, h0, final_state, B_prev, x_prev};
+  const void* v16[] = {x, B, C, y, h0, final_state, B_prev, x_prev, theta};
   for (const void* p : v16)
     if (p && !aligned(p, 16)) return M3_ERR_ALIGNMENT;
-  const void* v4[] = {dt, A, lam, theta};
+  const void* v4[] = {dt, A, lam};
   for (const void* p : v4)
     if (p && !aligned(p, 4)) return M3_ERR_ALIGNMENT;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);

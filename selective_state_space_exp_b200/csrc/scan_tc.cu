@@ -35,7 +35,6 @@ using namespace tc;
 constexpr int kN = 128;       // dstate
 constexpr int kP = 64;        // headdim
 constexpr int kPairs = kN / 2;
-constexpr int kThreads = 128;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded mbarrier wait (2 s)
 
 enum { MODE_FULL = 0, MODE_STATE = 1 };
@@ -43,6 +42,10 @@ enum { MODE_FULL = 0, MODE_STATE = 1 };
 template <int R, int Q>
 struct Cfg {
   static constexpr int M = Q * R;
+  // 256 threads and two CTAs per SM for 64-row chunks, else 512 threads
+  static constexpr int NTH = (Q * R == 64) ? 256 : 512;
+  static constexpr int MINB = (Q * R == 64) ? 2 : 1;
+  static constexpr int SLOTS_MAX = NTH / 16;    // token slots of the rotation pass
   static constexpr int MT = M < 128 ? M : 128;  // rows per MMA tile
   static constexpr int NT = M / MT;             // tiles per chunk
   static constexpr int OPB = M * 128;           // bytes of one [M][128 B] operand block
@@ -54,11 +57,15 @@ struct Cfg {
   static constexpr int P_OFF = B_OFF;           // masked scores reuse Bt + Xw
   static constexpr int G_OFF = XW_OFF + OPB;    // state, bf16 [N][128 B]
   static constexpr int SMALL_OFF = G_OFF + kN * 128;
-  static constexpr int SMALL_BYTES = 8 * Q * 4 + 2 * kPairs * 4 + 64;
+  // small region: per-token gates, chunk-end angles, the Q x Q decay table;
+  // the slot angle sums live in the x operand block (free until x is staged)
+  static constexpr int SMALL_BYTES = 6 * Q * 4 + kPairs * 4 + Q * Q * 4 + 64;
+  static_assert(SLOTS_MAX * kPairs * 4 <= OPB, "slot sums must fit in the x block");
   // + alignment slack; at least 80 KB so that no more than two CTAs (2 x 256
   // TMEM columns) share an SM
   static constexpr int SMEM_RAW = SMALL_OFF + SMALL_BYTES + 1024;
   static constexpr int SMEM = SMEM_RAW < 80 * 1024 ? 80 * 1024 : SMEM_RAW;
+  static_assert(MINB * (SMEM + 1024) <= 233472, "CTAs per SM must fit the SM's shared memory");
   // P tile mt: ((mt + 1) * MT / 64) blocks of [MT][128 B]
   __host__ __device__ static constexpr int p_tile_off(int mt) {
     return mt == 0 ? 0 : (MT / 64) * MT * 128;
@@ -89,7 +96,8 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 
-// Every thread polls; returns false on timeout (after recording it).
+// Polls an mbarrier (called by one thread); returns false on timeout after
+// recording it in the device status word.
 __device__ bool wait_bar(uint64_t* bar, uint32_t parity, int* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
@@ -102,30 +110,58 @@ __device__ bool wait_bar(uint64_t* bar, uint32_t parity, int* status) {
   return true;
 }
 
+__device__ __forceinline__ uint4 ldg_u128(const void* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// Thread layout (NTH = 256 or 512 threads).
+//  - TMEM work: warp w reads TMEM lanes 32*(w%4)..+31 ("quadrant" qd = w % 4)
+//    and takes column part cq = w / 4 of NTH / 128 parts; state row n =
+//    32*qd + lane is split over NTH / 128 threads.
+//  - Rotation: thread (kg = lane % 16, tq = 2*warp + lane / 16) rotates pairs
+//    4*kg..4*kg+3 for the TQ tokens of slot tq.  The 16 lanes of a half-warp
+//    cover one 256-byte row of B or C (coalesced 16-byte loads, conflict-free
+//    16-byte swizzled stores); the cumulative angles cross token slots
+//    through a small shared array.
 template <int R, int Q, int MODE>
-__global__ void __launch_bounds__(kThreads, 1) tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
+__global__ void __launch_bounds__(Cfg<R, Q>::NTH, Cfg<R, Q>::MINB)
+tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
   using C = Cfg<R, Q>;
   constexpr int M = C::M, MT = C::MT, NT = C::NT;
+  constexpr int NTH = C::NTH;
+  constexpr int CQN = NTH / 128;                          // column parts per TMEM lane
+  constexpr int TQ = Q >= C::SLOTS_MAX ? Q / C::SLOTS_MAX : 1;  // tokens per rotation slot
+  constexpr int SLOTS = Q / TQ;                           // active rotation slots
+  constexpr int CW = kP / CQN;                            // state / output columns per thread
+  constexpr float kL2E = 1.4426950408889634f;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(sm);
-  float* s_lam = reinterpret_cast<float*>(sm + C::SMALL_OFF);  // chunk-local Lam_t
-  float* s_gam = s_lam + Q;
+  float* s_l2 = reinterpret_cast<float*>(sm + C::SMALL_OFF);  // chunk-local Lam_t (prefix sum)
+  float* s_gam = s_l2 + Q;
   float* s_del = s_gam + Q;
   float* s_w = s_del + Q;
   float* s_dt = s_w + Q;
-  float* s_ph = s_dt + 3 * Q;                  // [2][kPairs] half-chunk angle sums
-  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_ph + 2 * kPairs);
+  float* s_lg = s_dt + Q;                       // Lam_t * log2(e)
+  float* s_phe = s_lg + Q;                      // [kPairs] chunk-end angles
+  float* s_D = s_phe + kPairs;                  // [Q][Q] decay x trapezoid weights
+  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_D + Q * Q);
+  float* s_part = reinterpret_cast<float*>(sm + C::X_OFF);  // [slots][kPairs], x block
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_bar + 1);
-  float* s_lend = reinterpret_cast<float*>(s_tmem + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, cq = warp >> 2;
+  const int kg = lane & 15, tq = (warp << 1) | (lane >> 4);
   const int64_t seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int64_t L = a.seqlen, H = a.nheads, G = a.ngroups;
   const int64_t g = h / (H / G);
-  const int64_t nseg = (MODE == MODE_FULL) ? pl.nseg : pl.nseg - 1;
-  (void)nseg;
+  const __nv_bfloat16* Bg = reinterpret_cast<const __nv_bfloat16*>(a.B);
+  const __nv_bfloat16* Cg = reinterpret_cast<const __nv_bfloat16*>(a.C);
+  const __nv_bfloat16* Xg = reinterpret_cast<const __nv_bfloat16*>(a.x);
+  const int64_t tokB = G * R * kN;   // element stride of one token in B, C
+  const int64_t tokT = G * kPairs;   // element stride of one token in theta
+  const int64_t tokX = H * R * kP;   // element stride of one token in x, y
 
   if (warp == 0) {
     tmem_alloc(s_tmem, C::TMEM_COLS);
@@ -139,46 +175,47 @@ __global__ void __launch_bounds__(kThreads, 1) tc_scan_kernel(const ScanArgs a, 
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *s_tmem;
-  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+  const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
   uint32_t phase = 0;
   bool aborted = false;
 
-  // ---- incoming state: thread n = tid owns state row n ---------------------
-  const int n = tid;
-  float gst[kP];
+  // ---- incoming state: thread (n, cq) owns columns [CW*cq, CW*cq + CW) of row n
+  const int n = 32 * qd + lane;
+  const int p0 = CW * cq;
+  float gst[CW];
   if (MODE == MODE_STATE) {
 #pragma unroll
-    for (int p = 0; p < kP; ++p) gst[p] = 0.f;
+    for (int p = 0; p < CW; ++p) gst[p] = 0.f;
   } else if (seg == 0) {
-    const int64_t so = ((b * H + h) * kN + n) * kP;
+    const int64_t so = ((b * H + h) * kN + n) * kP + p0;
 #pragma unroll
-    for (int p = 0; p < kP; ++p) gst[p] = a.h0 ? a.h0[so + p] : 0.f;
+    for (int p = 0; p < CW; ++p) gst[p] = a.h0 ? __ldg(a.h0 + so + p) : 0.f;
     if (a.B_prev) {
-      const float eps0 = (1.f - a.lam[(b * L) * H + h]) * a.dt[(b * L) * H + h];
+      const float eps0 = (1.f - __ldg(a.lam + (b * L) * H + h)) * __ldg(a.dt + (b * L) * H + h);
       for (int r = 0; r < R; ++r) {
         const float bp = eps0 * io_load(a.B_prev, ((b * G + g) * R + r) * kN + n, true);
-        const int64_t xo = ((b * H + h) * R + r) * kP;
+        const int64_t xo = ((b * H + h) * R + r) * kP + p0;
 #pragma unroll
-        for (int p = 0; p < kP; ++p) gst[p] = fmaf(bp, io_load(a.x_prev, xo + p, true), gst[p]);
+        for (int p = 0; p < CW; ++p) gst[p] = fmaf(bp, io_load(a.x_prev, xo + p, true), gst[p]);
       }
     }
   } else {
-    const float* src = pl.wsT + (((b * H + h) * (pl.nseg - 1) + (seg - 1)) * kN + n) * kP;
+    const float* src = pl.wsT + (((b * H + h) * (pl.nseg - 1) + (seg - 1)) * kN + n) * kP + p0;
 #pragma unroll
-    for (int p = 0; p < kP; p += 4) {
+    for (int p = 0; p < CW; p += 4) {
       const float4 v = *reinterpret_cast<const float4*>(src + p);
       gst[p] = v.x; gst[p + 1] = v.y; gst[p + 2] = v.z; gst[p + 3] = v.w;
     }
   }
   auto store_state_bf16 = [&]() {
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
+    for (int c2 = 0; c2 < CW / 8; ++c2) {
       uint4 v;
-      v.x = pack_bf16(gst[8 * ch + 0], gst[8 * ch + 1]);
-      v.y = pack_bf16(gst[8 * ch + 2], gst[8 * ch + 3]);
-      v.z = pack_bf16(gst[8 * ch + 4], gst[8 * ch + 5]);
-      v.w = pack_bf16(gst[8 * ch + 6], gst[8 * ch + 7]);
-      *reinterpret_cast<uint4*>(sm + C::G_OFF + sw128_off(n, ch)) = v;
+      v.x = pack_bf16(gst[8 * c2 + 0], gst[8 * c2 + 1]);
+      v.y = pack_bf16(gst[8 * c2 + 2], gst[8 * c2 + 3]);
+      v.z = pack_bf16(gst[8 * c2 + 4], gst[8 * c2 + 5]);
+      v.w = pack_bf16(gst[8 * c2 + 6], gst[8 * c2 + 7]);
+      *reinterpret_cast<uint4*>(sm + C::G_OFF + sw128_off(n, (CW / 8) * cq + c2)) = v;
     }
   };
   if (MODE == MODE_FULL) store_state_bf16();
@@ -190,98 +227,165 @@ __global__ void __launch_bounds__(kThreads, 1) tc_scan_kernel(const ScanArgs a, 
   for (int64_t c = c_begin; c < c_end && !aborted; ++c) {
     const int64_t c0 = c * Q;
     const int nt = (int)min((int64_t)Q, L - c0);
+    const __nv_bfloat16* Bc = Bg + ((b * L + c0) * G + g) * R * kN + 8 * kg;
+    const __nv_bfloat16* Cc = Cg + ((b * L + c0) * G + g) * R * kN + 8 * kg;
+    const float* Tc = a.theta + ((b * L + c0) * G + g) * kPairs + 4 * kg;
+    const __nv_bfloat16* Xc = Xg + ((b * L + c0) * H + h) * R * kP;
+    const bool slot_live = tq < SLOTS;
 
-    // ---- gates: dt, lam, gamma, delta, chunk-local Lam ----------------------
-    for (int t = tid; t < Q; t += kThreads) {
-      float dt = 0.f, lm = 0.f, av = 0.f, nx = 0.f;
-      if (t < nt) {
-        const int64_t bt = b * L + c0 + t;
-        dt = a.dt[bt * H + h];
-        lm = a.lam[bt * H + h];
-        av = a.A[bt * H + h];
-        if (c0 + t + 1 < L) nx = (1.f - a.lam[(bt + 1) * H + h]) * a.dt[(bt + 1) * H + h];
+    // ---- gate loads first, then this chunk's B / C / theta -------------------
+    const bool gate_warp = warp < (Q + 31) / 32;
+    float g_dt = 0.f, g_lm = 0.f, g_av = 0.f, g_nx = 0.f;
+    if (gate_warp && tid < nt) {
+      const int64_t bt = b * L + c0 + tid;
+      g_dt = __ldg(a.dt + bt * H + h);
+      g_lm = __ldg(a.lam + bt * H + h);
+      g_av = __ldg(a.A + bt * H + h);
+      if (c0 + tid + 1 < L)
+        g_nx = (1.f - __ldg(a.lam + (bt + 1) * H + h)) * __ldg(a.dt + (bt + 1) * H + h);
+    }
+    uint4 rb[TQ][R], rc[TQ][R];
+    float4 th[TQ];
+#pragma unroll
+    for (int u = 0; u < TQ; ++u) {
+      const int t = tq * TQ + u;
+      const bool ld = slot_live && t < nt;
+      th[u] = ld ? __ldg(reinterpret_cast<const float4*>(Tc + t * tokT)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        rb[u][r] = ld ? ldg_u128(Bc + t * tokB + r * kN) : make_uint4(0, 0, 0, 0);
+        rc[u][r] = (ld && MODE == MODE_FULL) ? ldg_u128(Cc + t * tokB + r * kN) : make_uint4(0, 0, 0, 0);
       }
-      s_dt[t] = dt;
-      s_gam[t] = lm * dt;
-      s_del[t] = lm * dt + nx;
-      s_lam[t] = dt * av;
     }
-    __syncthreads();
-    {  // half-chunk sums of the step angles, pair k = tid % 64, half = tid / 64
-      const int k = tid & (kPairs - 1), half = tid >> 6;
-      float acc = 0.f;
-      const int t1 = min(nt, (half + 1) * (Q / 2));
-      for (int t = half * (Q / 2); t < t1; ++t)
-        acc = fmaf(s_dt[t], a.theta[((b * L + c0 + t) * G + g) * kPairs + k], acc);
-      s_ph[half * kPairs + k] = acc;
-    }
-    if (tid == 0) {
-      float acc = 0.f;
-      for (int t = 0; t < nt; ++t) {
-        acc += s_lam[t];
-        s_lam[t] = acc;
-      }
-      *s_lend = acc;
-    }
-    __syncthreads();
-    const float lend = *s_lend;
-    for (int t = tid; t < Q; t += kThreads)
-      s_w[t] = (t < nt) ? __expf(lend - s_lam[t]) * s_del[t] : 0.f;
-    __syncthreads();
 
-    // ---- operands: Bt (and Ct) rotated by -Phi_t, x and w*x ------------------
-    {
-      const int k = tid & (kPairs - 1), half = tid >> 6;
-      float phi = half ? s_ph[k] : 0.f;
-      const int kb = k >> 5;                     // 64-element K block of element 2k
-      const int ch = (k & 31) >> 2;              // 16-byte chunk in the 128-byte row
-      const int cb = (k & 3) * 4;                // byte in the chunk
-      for (int tt = 0; tt < Q / 2; ++tt) {
-        const int t = half * (Q / 2) + tt;
-        float sn = 0.f, cs = 0.f;
-        const bool valid = t < nt;
-        if (valid) {
-          phi = fmaf(s_dt[t], a.theta[((b * L + c0 + t) * G + g) * kPairs + k], phi);
-          sincosf(phi, &sn, &cs);
-        }
+    // ---- gates and the chunk-local prefix sum of dt*A (warp shuffle scan) ----
+    if (gate_warp) {  // whole warps take part in the shuffle scan
+      const bool inq = tid < Q;
+      if (inq) {
+        s_dt[tid] = g_dt;
+        s_gam[tid] = g_lm * g_dt;
+        s_del[tid] = g_lm * g_dt + g_nx;
+      }
+      float v = g_dt * g_av;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += u;
+      }
+      if (inq) s_l2[tid] = v;
+    }
+    __syncthreads();
+    if (Q > 32 && tid >= 32 && tid < Q) s_l2[tid] += s_l2[31];  // second warp of tokens
+
+    // ---- cumulative angles of pairs 4kg..4kg+3 over this slot's tokens -------
+    float2 ang[TQ][2];
+    float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < TQ; ++u) {
+      const int t = tq * TQ + u;
+      const float d = (slot_live && t < nt) ? s_dt[t] : 0.f;
+      ang[u][0] = make_float2(d * th[u].x, d * th[u].y);
+      ang[u][1] = make_float2(d * th[u].z, d * th[u].w);
+      part[0] += ang[u][0].x; part[1] += ang[u][0].y;
+      part[2] += ang[u][1].x; part[3] += ang[u][1].y;
+    }
+    if (slot_live)
+      *reinterpret_cast<float4*>(s_part + tq * kPairs + 4 * kg) =
+          make_float4(part[0], part[1], part[2], part[3]);
+    __syncthreads();  // s_l2 complete, angle partial sums written
+    float phi[4] = {0.f, 0.f, 0.f, 0.f};
+    if (slot_live) {
+      for (int q2 = 0; q2 < tq; ++q2) {
+        const float4 o = *reinterpret_cast<const float4*>(s_part + q2 * kPairs + 4 * kg);
+        phi[0] += o.x; phi[1] += o.y; phi[2] += o.z; phi[3] += o.w;
+      }
+      if (tq == SLOTS - 1)
+        *reinterpret_cast<float4*>(s_phe + 4 * kg) =
+            make_float4(phi[0] + part[0], phi[1] + part[1], phi[2] + part[2], phi[3] + part[3]);
+    }
+    const float lend = s_l2[nt - 1];
+    const float l2end = lend * kL2E;
+    if (tid < Q) {
+      const float lg = s_l2[tid] * kL2E;
+      s_lg[tid] = lg;
+      s_w[tid] = (tid < nt) ? ex2(l2end - lg) * s_del[tid] : 0.f;
+    }
+
+    // ---- operands: Bt (and Ct) rotated by -Phi_t (16-byte row pieces) ---------
+    if (slot_live) {
+      const uint32_t kboff = (uint32_t)(kg >> 3) * C::OPB;
+      const uint32_t chk = (uint32_t)(kg & 7);
+#pragma unroll
+      for (int u = 0; u < TQ; ++u) {
+        const int t = tq * TQ + u;
+        phi[0] += ang[u][0].x; phi[1] += ang[u][0].y;
+        phi[2] += ang[u][1].x; phi[3] += ang[u][1].y;
+        float cs[4], sn[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) __sincosf(phi[j], &sn[j], &cs[j]);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          const uint32_t row = t * R + r;
-          const uint32_t off = kb * C::OPB + sw128_off(row, ch) + cb;
-          uint32_t vb = 0, vc = 0;
-          if (valid) {
-            const int64_t e = (((b * L + c0 + t) * G + g) * R + r) * kN + 2 * k;
-            const float2 bb = unpack_bf16(*reinterpret_cast<const uint32_t*>(
-                reinterpret_cast<const __nv_bfloat16*>(a.B) + e));
-            vb = pack_bf16(cs * bb.x + sn * bb.y, -sn * bb.x + cs * bb.y);
+          const uint32_t off = kboff + sw128_off(t * R + r, chk);
+          uint32_t ob[4], oc[4];
+          const uint32_t ib[4] = {rb[u][r].x, rb[u][r].y, rb[u][r].z, rb[u][r].w};
+          const uint32_t ic[4] = {rc[u][r].x, rc[u][r].y, rc[u][r].z, rc[u][r].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            // (b0, b1) -> (c b0 + s b1, c b1 - s b0)
+            const float2 v = make_float2(__uint_as_float(ib[j] << 16),
+                                         __uint_as_float(ib[j] & 0xffff0000u));
+            const float2 w = ffma2(make_float2(cs[j], cs[j]), v,
+                                   fmul2(make_float2(sn[j], -sn[j]), make_float2(v.y, v.x)));
+            ob[j] = pack_bf16(w.x, w.y);
             if (MODE == MODE_FULL) {
-              const float2 cc = unpack_bf16(*reinterpret_cast<const uint32_t*>(
-                  reinterpret_cast<const __nv_bfloat16*>(a.C) + e));
-              vc = pack_bf16(cs * cc.x + sn * cc.y, -sn * cc.x + cs * cc.y);
+              const float2 vc = make_float2(__uint_as_float(ic[j] << 16),
+                                            __uint_as_float(ic[j] & 0xffff0000u));
+              const float2 wc = ffma2(make_float2(cs[j], cs[j]), vc,
+                                      fmul2(make_float2(sn[j], -sn[j]), make_float2(vc.y, vc.x)));
+              oc[j] = pack_bf16(wc.x, wc.y);
             }
           }
-          *reinterpret_cast<uint32_t*>(sm + C::B_OFF + off) = vb;
-          if (MODE == MODE_FULL) *reinterpret_cast<uint32_t*>(sm + C::C_OFF + off) = vc;
+          *reinterpret_cast<uint4*>(sm + C::B_OFF + off) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+          if (MODE == MODE_FULL)
+            *reinterpret_cast<uint4*>(sm + C::C_OFF + off) = make_uint4(oc[0], oc[1], oc[2], oc[3]);
         }
       }
     }
-    for (int q = tid; q < M * 8; q += kThreads) {
-      const int row = q >> 3, ch = q & 7;
-      const int t = row / R, r = row % R;
-      uint4 v = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
-      if (t < nt) {
-        const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.x) +
-                                   (((b * L + c0 + t) * H + h) * R + r) * kP + ch * 8;
-        v = *reinterpret_cast<const uint4*>(src);
-        const float w = s_w[t];
-        float2 f;
-        f = unpack_bf16(v.x); vw.x = pack_bf16(w * f.x, w * f.y);
-        f = unpack_bf16(v.y); vw.y = pack_bf16(w * f.x, w * f.y);
-        f = unpack_bf16(v.z); vw.z = pack_bf16(w * f.x, w * f.y);
-        f = unpack_bf16(v.w); vw.w = pack_bf16(w * f.x, w * f.y);
+    // the x loads go out before the barrier so their latency overlaps it
+    constexpr int PER = M * 8 / NTH;
+    uint4 xv[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int q = tid + j * NTH;
+      const int row = q >> 3, chq = q & 7, t = row / R, r = row % R;
+      xv[j] = (t < nt) ? ldg_u128(Xc + t * tokX + r * kP + chq * 8) : make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();  // s_w ready for the x pass
+
+    // ---- w * x (chunk-state operand); x itself is copied after MMA issue ------
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int q = tid + j * NTH;
+      const int row = q >> 3, chq = q & 7, t = row / R;
+      const float w = s_w[t];
+      const uint32_t iv[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+      uint32_t ov[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = fmul2(make_float2(w, w), make_float2(__uint_as_float(iv[e] << 16),
+                                                              __uint_as_float(iv[e] & 0xffff0000u)));
+        ov[e] = pack_bf16(f.x, f.y);
       }
-      if (MODE == MODE_FULL) *reinterpret_cast<uint4*>(sm + C::X_OFF + sw128_off(row, ch)) = v;
-      *reinterpret_cast<uint4*>(sm + C::XW_OFF + sw128_off(row, ch)) = vw;
+      *reinterpret_cast<uint4*>(sm + C::XW_OFF + sw128_off(row, chq)) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+    }
+    if (MODE == MODE_FULL) {  // D[t][s] = [s <= t] exp(Lam_t - Lam_s) (s == t ? gamma_t : delta_s)
+#pragma unroll
+      for (int e = tid; e < Q * Q; e += NTH) {
+        const int t = e / Q, s2 = e % Q;
+        float d = 0.f;
+        if (t < nt && s2 <= t) d = ex2(s_lg[t] - s_lg[s2]) * ((s2 == t) ? s_gam[t] : s_del[s2]);
+        s_D[e] = d;
+      }
     }
     fence_async_smem();
     tc_fence_before();
@@ -313,7 +417,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_scan_kernel(const ScanArgs a, 
       }
       mma_commit(s_bar);
     }
-    const bool ok1 = wait_bar(s_bar, phase, a.status);
+    if (MODE == MODE_FULL) {  // x into the MMA2 operand while MMA1/MMA3 run
+#pragma unroll
+      for (int j = 0; j < PER; ++j) {
+        const int q = tid + j * NTH;
+        *reinterpret_cast<uint4*>(sm + C::X_OFF + sw128_off(q >> 3, q & 7)) = xv[j];
+      }
+    }
+    const bool ok1 = (tid == 0) ? wait_bar(s_bar, phase, a.status) : true;
     phase ^= 1;
     if (__syncthreads_or(!ok1)) { aborted = true; break; }
     tc_fence_after();
@@ -322,40 +433,35 @@ __global__ void __launch_bounds__(kThreads, 1) tc_scan_kernel(const ScanArgs a, 
       // ---- mask the scores into P (bf16, K-major, over Bt / Xw) -------------
 #pragma unroll
       for (int mt = 0; mt < NT; ++mt) {
-        const int rho = (MT == 64) ? 16 * warp + lane : tid;  // row within the tile
+        const int rho = (MT == 64) ? 16 * qd + lane : 32 * qd + lane;  // row in the tile
         const bool live = (MT == 64) ? lane < 16 : true;
-        const int i = mt * MT + rho;
-        const int t = i / R;
+        const int t = (mt * MT + rho) / R;
         const bool trow = live && t < nt;
-        const float lt = trow ? s_lam[t] : 0.f;
-        const int ncols = (mt + 1) * MT;
-        for (int cc = 0; cc < ncols / 32; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(tm + lane_base + C::s_col(mt) + cc * 32, v);
+        const int cpt = (mt + 1) * MT / CQN;  // columns per thread
+        for (int cc = cq * cpt / 16; cc < (cq + 1) * cpt / 16; ++cc) {
+          uint32_t v[16];
+          tmem_ld16(tm + lane_base + C::s_col(mt) + cc * 16, v);
           tmem_ld_wait();
           if (!live) continue;
-          uint32_t pk[16];
+          float mk[16 / R];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            float o[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int s = (cc * 32 + j + e) / R;
-              float m = 0.f;
-              if (trow && s <= t)
-                m = __expf(lt - s_lam[s]) * ((s == t) ? s_gam[t] : s_del[s]);
-              o[e] = __uint_as_float(v[j + e]) * m;
-            }
-            pk[j / 2] = pack_bf16(o[0], o[1]);
+          for (int q4 = 0; q4 < 16 / R / 4; ++q4) {
+            float4 d4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (trow) d4 = *reinterpret_cast<const float4*>(s_D + t * Q + cc * (16 / R) + 4 * q4);
+            mk[4 * q4] = d4.x; mk[4 * q4 + 1] = d4.y; mk[4 * q4 + 2] = d4.z; mk[4 * q4 + 3] = d4.w;
           }
-          const int kb = (cc * 32) / 64;
+          uint32_t pk[8];
+#pragma unroll
+          for (int j = 0; j < 16; j += 2) {
+            const float2 f = fmul2(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
+                                   make_float2(mk[j / R], mk[(j + 1) / R]));
+            pk[j / 2] = pack_bf16(f.x, f.y);
+          }
+          const int kb = (cc * 16) / 64;
           uint8_t* blk = sm + C::P_OFF + C::p_tile_off(mt) + kb * MT * 128;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int ch = ((cc * 32) % 64) / 8 + q;
-            *reinterpret_cast<uint4*>(blk + sw128_off(rho, ch)) =
-                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-          }
+          const int ch0 = ((cc * 16) % 64) / 8;
+          *reinterpret_cast<uint4*>(blk + sw128_off(rho, ch0)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(blk + sw128_off(rho, ch0 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
       fence_async_smem();
@@ -388,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_scan_kernel(const ScanArgs a, 
         }
         mma_commit(s_bar);
       }
-      const bool ok2 = wait_bar(s_bar, phase, a.status);
+      const bool ok2 = (tid == 0) ? wait_bar(s_bar, phase, a.status) : true;
       phase ^= 1;
       if (__syncthreads_or(!ok2)) { aborted = true; break; }
       tc_fence_after();
@@ -396,32 +502,33 @@ __global__ void __launch_bounds__(kThreads, 1) tc_scan_kernel(const ScanArgs a, 
       // ---- epilogue: y = P x + exp(Lam_t) Ct G ---------------------------------
 #pragma unroll
       for (int mt = 0; mt < NT; ++mt) {
-        const int rho = (MT == 64) ? 16 * warp + lane : tid;
+        const int rho = (MT == 64) ? 16 * qd + lane : 32 * qd + lane;
         const bool live = (MT == 64) ? lane < 16 : true;
         const int i = mt * MT + rho;
         const int t = i / R, r = i % R;
         const bool out = live && t < nt;
-        const float el = out ? __expf(s_lam[t]) : 0.f;
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.y) +
-                             (((b * L + c0 + (out ? t : 0)) * H + h) * R + r) * kP;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t yv[32], zv[32];
-          tmem_ld32(tm + lane_base + C::y_col(mt) + 32 * half, yv);
-          tmem_ld32(tm + lane_base + C::y2_col(mt) + 32 * half, zv);
+        for (int pc = 0; pc < CW / 16; ++pc) {
+          uint32_t yv[16], zv[16];
+          tmem_ld16(tm + lane_base + C::y_col(mt) + CW * cq + 16 * pc, yv);
+          tmem_ld16(tm + lane_base + C::y2_col(mt) + CW * cq + 16 * pc, zv);
           tmem_ld_wait();
           if (out) {
+            const float el = ex2(s_lg[t]);
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.y) +
+                                 ((b * L + c0 + t) * H + h) * R * kP + r * kP + CW * cq + 16 * pc;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
               uint32_t w4[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int j = q * 8 + 2 * e;
-                w4[e] = pack_bf16(fmaf(el, __uint_as_float(zv[j]), __uint_as_float(yv[j])),
-                                  fmaf(el, __uint_as_float(zv[j + 1]), __uint_as_float(yv[j + 1])));
+                const float2 f = ffma2(make_float2(el, el),
+                                       make_float2(__uint_as_float(zv[j]), __uint_as_float(zv[j + 1])),
+                                       make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1])));
+                w4[e] = pack_bf16(f.x, f.y);
               }
-              *reinterpret_cast<uint4*>(dst + 32 * half + q * 8) =
-                  make_uint4(w4[0], w4[1], w4[2], w4[3]);
+              *reinterpret_cast<uint4*>(dst + q * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
           }
         }
@@ -430,22 +537,27 @@ __global__ void __launch_bounds__(kThreads, 1) tc_scan_kernel(const ScanArgs a, 
 
     // ---- state update: G <- Rot(Phi_end) (exp(Lam_end) G + Sc) ---------------
     {
-      uint32_t s0[32], s1[32];
-      tmem_ld32(tm + lane_base + C::SC_COL, s0);
-      tmem_ld32(tm + lane_base + C::SC_COL + 32, s1);
-      tmem_ld_wait();
-      const int k = n >> 1;
-      const float phe = s_ph[k] + s_ph[kPairs + k];
+      const float phe = s_phe[n >> 1];
       float sn, cs;
       sincosf(phe, &sn, &cs);
-      const float el = __expf(lend);
-      const bool even = (n & 1) == 0;
+      const float el = ex2(l2end);
+      const float ss = (n & 1) ? sn : -sn;  // even row: c v - s o; odd row: c v + s o
 #pragma unroll
-      for (int p = 0; p < kP; ++p) {
-        const float sc = __uint_as_float(p < 32 ? s0[p] : s1[p - 32]);
-        const float v = fmaf(el, gst[p], sc);
-        const float o = __shfl_xor_sync(0xffffffffu, v, 1);
-        gst[p] = even ? (cs * v - sn * o) : (sn * o + cs * v);
+      for (int pc = 0; pc < CW / 16; ++pc) {
+        uint32_t sv[16];
+        tmem_ld16(tm + lane_base + C::SC_COL + CW * cq + 16 * pc, sv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int p = 0; p < 16; p += 2) {
+          const int pp = 16 * pc + p;
+          const float2 v = ffma2(make_float2(el, el), make_float2(gst[pp], gst[pp + 1]),
+                                 make_float2(__uint_as_float(sv[p]), __uint_as_float(sv[p + 1])));
+          const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, v.x, 1),
+                                       __shfl_xor_sync(0xffffffffu, v.y, 1));
+          const float2 w = ffma2(make_float2(cs, cs), v, fmul2(make_float2(ss, ss), o));
+          gst[pp] = w.x;
+          gst[pp + 1] = w.y;
+        }
       }
       if (MODE == MODE_STATE) {
         lam_seg += lend;
@@ -461,20 +573,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_scan_kernel(const ScanArgs a, 
   if (!aborted) {
     if (MODE == MODE_FULL) {
       if (seg == pl.nseg - 1 && a.final_state) {
-        float* dst = a.final_state + ((b * H + h) * kN + n) * kP;
+        float* dst = a.final_state + ((b * H + h) * kN + n) * kP + p0;
 #pragma unroll
-        for (int p = 0; p < kP; p += 4)
+        for (int p = 0; p < CW; p += 4)
           *reinterpret_cast<float4*>(dst + p) = make_float4(gst[p], gst[p + 1], gst[p + 2], gst[p + 3]);
       }
     } else {
       const int64_t slot = (b * H + h) * (pl.nseg - 1) + seg;
-      float* dst = pl.wsT + (slot * kN + n) * kP;
+      float* dst = pl.wsT + (slot * kN + n) * kP + p0;
 #pragma unroll
-      for (int p = 0; p < kP; p += 4)
+      for (int p = 0; p < CW; p += 4)
         *reinterpret_cast<float4*>(dst + p) = make_float4(gst[p], gst[p + 1], gst[p + 2], gst[p + 3]);
       float* su = pl.wsSum + slot * (1 + kPairs);
       if (tid == 0) su[0] = lam_seg;
-      if ((n & 1) == 0) su[1 + (n >> 1)] = phi_seg;
+      if (cq == 0 && (n & 1) == 0) su[1 + (n >> 1)] = phi_seg;
     }
   }
   tc_fence_before();
@@ -541,7 +653,7 @@ cudaError_t launch_kernel(const ScanArgs& a, const TcPlan& pl, int64_t nblocks, 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)nblocks, (unsigned)a.nheads, (unsigned)a.batch);
-  kern<<<grid, kThreads, C::SMEM, st>>>(a, pl);
+  kern<<<grid, C::NTH, C::SMEM, st>>>(a, pl);
   return cudaGetLastError();
 }
 

@@ -105,6 +105,7 @@ def test_scan_rejects_bad_arguments(lib):
     assert scan_call(lib, s, x=ctypes.c_void_p(A16 + 8)) == -3
     assert scan_call(lib, s, y=ctypes.c_void_p(A16 + 2)) == -3
     assert scan_call(lib, s, dt=ctypes.c_void_p(A16 + 2)) == -3
+    assert scan_call(lib, s, theta=ctypes.c_void_p(A16 + 4)) == -3
     assert scan_call(lib, s, ws=None) == -4
     assert scan_call(lib, s, wsb=16) == -4
     assert scan_call(lib, s, ws=ctypes.c_void_p(A16 + 16), wsb=1 << 40) == -4
