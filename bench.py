@@ -30,6 +30,7 @@ sys.path.insert(0, ROOT)
 
 from selective_state_space_exp_b200 import inputs as I  # noqa: E402
 from selective_state_space_exp_b200 import m3  # noqa: E402
+from selective_state_space_exp_b200.parallel import max_over_ranks as _max_ranks  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -185,12 +186,7 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
-    if world == 1:
-        return v
-    import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return _max_ranks(v, device="cuda") if world > 1 else v
 
 
 # ---- device timing ---------------------------------------------------------
@@ -417,7 +413,9 @@ def main():
     e2e_step, h2d, d2h = time_e2e_prefill(inp_host, s, max(3, args.steps // 4))
     e2e_step = max_over_ranks(e2e_step, world)
 
-    launches_per_call = 3
+    plan = m3.scan_plan(m3.scan_shape(inp_host["x"], inp_host["B"], s.chunk))
+    launches_per_call = plan["launches"]
+    kern = "tc_scan_kernel (tcgen05)" if plan["tensor_core"] else "CUDA-core scan kernels"
     line = {
         "metric": "prefill tokens/s",
         "value": round(world * tokens / per_step, 1),
@@ -432,9 +430,12 @@ def main():
         "config": {"workload": args.workload, **shape_cfg(s),
                    "parallelism": f"dp{world} (independent batches per rank)",
                    "l2": "flushed between timed steps (256 MiB write)",
-                   "path": "simt fp32 (3 launches per call)"},
+                   "path": f"{kern}, {launches_per_call} launch(es) per call, "
+                           f"{plan['segments']} segment(s) per sequence"},
         "roofline": {**roofline(flops, byt, per_step, peaks, psrc),
-                     "scope": "whole m3_scan_fwd call (chunk state + state pass + chunk output)",
+                     "scope": ("the one kernel launch of each m3_scan_fwd call, CUDA events on "
+                               "the launching stream" if launches_per_call == 1 else
+                               "whole m3_scan_fwd call (all launches), CUDA events"),
                      "traffic": None, "algorithmic_flops": flops, "algorithmic_bytes": byt},
         "decode": {
             "metric": "decode tokens/s", "value": round(world * ds.batch * dsteps / dt_total, 1),

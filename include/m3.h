@@ -108,6 +108,15 @@ M3_API int m3_check_shape(const m3_shape* shape);
  * Host-only; writes *bytes.  Returns M3_OK or the m3_check_shape error. */
 M3_API int m3_scan_workspace_size(const m3_shape* shape, size_t* bytes);
 
+/* How m3_scan_fwd will run `shape` (host-only): *tensor_core = 1 for the
+ * tcgen05 path (bf16 io, N = 128, P = 64, chunk * rank in {64, 128, 256},
+ * M3_FLAG_SIMT clear), 0 for the CUDA-core fp32 path; *segments = pieces
+ * each (batch, head) sequence is cut into (tensor-core path; 1 otherwise);
+ * *launches = kernel launches per call (0 when seqlen == 0).  Any output
+ * pointer may be NULL.  Returns M3_OK or the m3_check_shape error. */
+M3_API int m3_scan_plan(const m3_shape* shape, int* tensor_core, int64_t* segments,
+                        int* launches);
+
 /* Chunked prefill scan over a whole sequence batch: the recurrence above for
  * every (batch, head), y_t = C_t^T h_t for every token, and the state after
  * the last token.

@@ -111,6 +111,18 @@ M3_API int m3_scan_workspace_size(const m3_shape* s, size_t* bytes) {
   return M3_OK;
 }
 
+M3_API int m3_scan_plan(const m3_shape* s, int* tensor_core, int64_t* segments, int* launches) {
+  int st = check_common(s);
+  if (st != M3_OK) return st;
+  ScanArgs a = make_scan_args(s);
+  const bool tc = use_tc(s, a);
+  const int64_t nseg = (tc && s->seqlen > 0) ? tc_scan_segments(a) : 1;
+  if (tensor_core) *tensor_core = tc ? 1 : 0;
+  if (segments) *segments = nseg;
+  if (launches) *launches = s->seqlen == 0 ? 0 : (tc ? (nseg > 1 ? 3 : 1) : 3);
+  return M3_OK;
+}
+
 M3_API int m3_scan_fwd(const m3_shape* s, const void* x, const float* dt, const float* A,
                        const float* lam, const float* theta, const void* B, const void* C,
                        const float* h0, const void* B_prev, const void* x_prev, void* y,

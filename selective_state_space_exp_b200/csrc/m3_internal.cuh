@@ -69,6 +69,7 @@ cudaError_t simt_scan_launch(const ScanArgs& a, cudaStream_t s);
 // Tensor-core (tcgen05) scan for bf16 io, N = 128, P = 64, Q*R in {64, 128, 256}.
 bool tc_scan_supported(const ScanArgs& a);
 size_t tc_scan_workspace(const ScanArgs& a);
+int64_t tc_scan_segments(const ScanArgs& a);
 cudaError_t tc_scan_launch(const ScanArgs& a, cudaStream_t s);
 
 // Decode step.

@@ -678,6 +678,8 @@ bool tc_scan_supported(const ScanArgs& a) {
   return (a.R == 1 || a.R == 2 || a.R == 4) && (m == 64 || m == 128 || m == 256) && a.Q >= 16;
 }
 
+int64_t tc_scan_segments(const ScanArgs& a) { return make_plan(a).nseg; }
+
 size_t tc_scan_workspace(const ScanArgs& a) {
   const TcPlan pl = make_plan(a);
   if (pl.nseg <= 1) return 0;

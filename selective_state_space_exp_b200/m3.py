@@ -60,6 +60,10 @@ def load() -> ctypes.CDLL:
             L.m3_check_shape.restype = ctypes.c_int
             L.m3_scan_workspace_size.argtypes = [sp, ctypes.POINTER(ctypes.c_size_t)]
             L.m3_scan_workspace_size.restype = ctypes.c_int
+            L.m3_scan_plan.argtypes = [sp, ctypes.POINTER(ctypes.c_int),
+                                       ctypes.POINTER(ctypes.c_int64),
+                                       ctypes.POINTER(ctypes.c_int)]
+            L.m3_scan_plan.restype = ctypes.c_int
             L.m3_scan_fwd.argtypes = [sp] + [vp] * 13 + [ctypes.c_size_t, vp]
             L.m3_scan_fwd.restype = ctypes.c_int
             L.m3_scan_fwd_noalloc.argtypes = [sp] + [vp] * 13
@@ -118,6 +122,14 @@ def workspace_size(shape: Shape) -> int:
     _check("m3_scan_workspace_size", load().m3_scan_workspace_size(ctypes.byref(shape),
                                                                    ctypes.byref(n)))
     return int(n.value)
+
+
+def scan_plan(shape: Shape) -> dict:
+    """How m3_scan_fwd runs `shape`: tensor_core (bool), segments, launches."""
+    tc, seg, n = ctypes.c_int(), ctypes.c_int64(), ctypes.c_int()
+    _check("m3_scan_plan", load().m3_scan_plan(ctypes.byref(shape), ctypes.byref(tc),
+                                               ctypes.byref(seg), ctypes.byref(n)))
+    return {"tensor_core": bool(tc.value), "segments": int(seg.value), "launches": int(n.value)}
 
 
 def m3_scan_fwd(x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None, B_prev=None,

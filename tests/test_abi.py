@@ -131,3 +131,24 @@ def test_decode_rejects_bad_arguments(lib):
     assert decode_call(lib, s, x=ctypes.c_void_p(A16 + 0x100000 + 4)) == -3
     assert decode_call(lib, s, lam=ctypes.c_void_p(A16 + 1)) == -3
     assert decode_call(lib, shape(headdim=24)) == -2
+
+
+@pytest.mark.parametrize("kw,tc,seg,launches", [
+    (dict(batch=8, nheads=64, seqlen=2048), 1, 1, 1),            # many chains: one segment
+    (dict(batch=1, nheads=64, seqlen=32768, rank=4), 1, None, 3),  # few chains: segments
+    (dict(batch=8, nheads=64, seqlen=2048, flags=1), 0, 1, 3),     # forced CUDA-core path
+    (dict(io_dtype=0, dstate=16, headdim=16), 0, 1, 3),            # fp32 io
+    (dict(seqlen=0), 1, 1, 0),
+    (dict(rank=8), 0, 1, 3),                                       # R = 8: CUDA-core path
+])
+def test_scan_plan(lib, kw, tc, seg, launches):
+    s = shape(**kw)
+    t, g, n = ctypes.c_int(), ctypes.c_int64(), ctypes.c_int()
+    assert lib.m3_scan_plan(ctypes.byref(s), ctypes.byref(t), ctypes.byref(g), ctypes.byref(n)) == 0
+    assert t.value == tc and n.value == launches
+    if seg is None:
+        assert g.value > 1
+    else:
+        assert g.value == seg
+    assert lib.m3_scan_plan(ctypes.byref(s), None, None, None) == 0
+    assert lib.m3_scan_plan(None, None, None, None) == -1
