@@ -9,25 +9,39 @@
 // the rank-R MIMO update (section 2.3).  The step is HBM-bound (section 3.3:
 // decode is limited by state IO, not FLOPs): 2 * 4 * N * P bytes per head.
 //
-// Layout: one CTA of 128 threads per (b, h).  Thread (kslot, pv) owns float4
-// column pv of the state and the pairs k = kslot, kslot + nslots, ...  A row
-// of the state (P floats) is read by P/4 consecutive threads as float4, so
-// each warp access is a contiguous 256-512 byte segment.  The per-head
-// operands (B, C, B_prev, x, x_prev, the cos/sin table) are staged in shared
-// memory once; y is reduced over kslots through shared memory.
+// Layout: one CTA of 128 threads per (b, h) (whole state rows).
+// Thread (kslot, pv) owns float4 column pv of the block and the pairs
+// k = kslot, kslot + nslots, ...; a block row is read by consecutive threads
+// as float4 (a contiguous 128-byte segment per row).  The per-head operands
+// (B, C, B_prev, x, x_prev, the cos/sin table) are staged in shared memory;
+// y is reduced over kslots through shared memory.
 #include "m3_internal.cuh"
 
 namespace m3 {
 namespace {
 
 constexpr int kDecodeThreads = 128;
-constexpr int kPairsInFlight = 4;  // pairs loaded before any is computed
+constexpr int kMaxCols = 128;  // state columns per CTA (whole rows: P <= 128)
+constexpr int kPairsInFlight = 4;  // pairs whose state rows are loaded before any is computed
+
+// CTA (b, h, column block): columns [cb*CB, cb*CB + CB) of the head's state
+// and of y (columns are independent: y[r][p] only reads column p of h').
+// Whole rows per CTA (CB = P) read best: splitting a 256-byte state row
+// between CTAs that run at different times costs HBM locality.
+// Resident CTAs per SM the register budget is sized for (more state bytes in
+// flight for small R, room for the rank-R operands for large R).
+template <int R>
+struct DecodeOcc {
+  static constexpr int value = R == 1 ? 7 : (R == 2 ? 6 : (R == 4 ? 5 : 3));
+};
 
 template <int R>
-__global__ void __launch_bounds__(kDecodeThreads)
-decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kDecodeThreads, DecodeOcc<R>::value) decode_kernel(const DecodeArgs a) {
   const int P = (int)a.P, N = (int)a.N, K = N / 2;
-  const int64_t bh = blockIdx.x;
+  const int CB = P < kMaxCols ? P : kMaxCols;
+  const int nblk = P / CB;
+  const int64_t bh = blockIdx.x / nblk;
+  const int cb = blockIdx.x % nblk;
   const int64_t h = bh % a.nheads, b = bh / a.nheads;
   const int64_t g = h / (a.nheads / a.ngroups);
   const int64_t bg = b * a.ngroups + g;
@@ -39,14 +53,33 @@ decode_kernel(const DecodeArgs a) {
   float* s_Bp = s_as + K;         // B_prev                         [R][N]
   float* s_Bt = s_Bp + R * N;     // B_t                            [R][N]
   float* s_Ct = s_Bt + R * N;     // C_t                            [R][N]
-  float* s_xe = s_Ct + R * N;     // (1-lam) dt x_prev              [R][P]
-  float* s_xg = s_xe + R * P;     // lam dt x_t                     [R][P]
-  float* s_red = s_xg + R * P;    // partial y per kslot            [nslots][R][P]
+  float* s_xe = s_Ct + R * N;     // (1-lam) dt x_prev              [R][CB]
+  float* s_xg = s_xe + R * CB;    // lam dt x_t                     [R][CB]
+  float* s_red = s_xg + R * CB;   // partial y per kslot            [nslots][R][CB]
 
   const float dt = a.dt[bh], lamv = a.lam[bh];
   const float alpha = expf(dt * a.A[bh]);
   const float gamma = lamv * dt, eps = (1.f - lamv) * dt;
   const bool prev = a.B_prev != nullptr;
+
+  const int PV = CB / 4;  // float4 columns per state row in this block
+  const int nslots = kDecodeThreads / PV;
+  const int pv = tid % PV, kslot = tid / PV;
+  const int p0 = pv * 4;
+  const float4* src = reinterpret_cast<const float4*>(a.state_in + bh * (int64_t)N * P + cb * CB);
+  float4* dst = reinterpret_cast<float4*>(a.state_out + bh * (int64_t)N * P + cb * CB);
+  const int rowq = P / 4;  // float4 stride between state rows
+
+  // Issue the first pairs' state loads before staging the per-head operands.
+  float4 r0[kPairsInFlight], r1[kPairsInFlight];
+#pragma unroll
+  for (int u = 0; u < kPairsInFlight; ++u) {
+    const int k = kslot + u * nslots;
+    if (k < K) {
+      r0[u] = __ldcs(src + (2 * k) * rowq + pv);
+      r1[u] = __ldcs(src + (2 * k + 1) * rowq + pv);
+    }
+  }
 
   for (int k = tid; k < K; k += kDecodeThreads) {
     float sn, cs;
@@ -59,38 +92,33 @@ decode_kernel(const DecodeArgs a) {
     s_Ct[i] = io_load(a.C, bg * R * N + i, a.bf16);
     s_Bp[i] = prev ? io_load(a.B_prev, bg * R * N + i, a.bf16) : 0.f;
   }
-  for (int i = tid; i < R * P; i += kDecodeThreads) {
-    s_xg[i] = gamma * io_load(a.x, bh * R * P + i, a.bf16);
-    s_xe[i] = prev ? eps * io_load(a.x_prev, bh * R * P + i, a.bf16) : 0.f;
+  for (int i = tid; i < R * CB; i += kDecodeThreads) {
+    const int r = i / CB, c = i % CB;
+    const int64_t xi = bh * R * P + r * P + cb * CB + c;
+    s_xg[i] = gamma * io_load(a.x, xi, a.bf16);
+    s_xe[i] = prev ? eps * io_load(a.x_prev, xi, a.bf16) : 0.f;
   }
   __syncthreads();
-
-  const int PV = P / 4;              // float4 columns per state row
-  const int nslots = kDecodeThreads / PV;
-  const int pv = tid % PV, kslot = tid / PV;
-  const int p0 = pv * 4;
 
   float xg[R][4], xe[R][4], yacc[R][4];
 #pragma unroll
   for (int r = 0; r < R; ++r)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      xg[r][j] = s_xg[r * P + p0 + j];
-      xe[r][j] = s_xe[r * P + p0 + j];
+      xg[r][j] = s_xg[r * CB + p0 + j];
+      xe[r][j] = s_xe[r * CB + p0 + j];
       yacc[r][j] = 0.f;
     }
 
-  const float4* src = reinterpret_cast<const float4*>(a.state_in + bh * (int64_t)N * P);
-  float4* dst = reinterpret_cast<float4*>(a.state_out + bh * (int64_t)N * P);
-
   for (int kb = kslot; kb < K; kb += kPairsInFlight * nslots) {
-    float4 r0[kPairsInFlight], r1[kPairsInFlight];
+    if (kb != kslot) {
 #pragma unroll
-    for (int u = 0; u < kPairsInFlight; ++u) {
-      const int k = kb + u * nslots;
-      if (k < K) {
-        r0[u] = __ldcs(src + (2 * k) * PV + pv);
-        r1[u] = __ldcs(src + (2 * k + 1) * PV + pv);
+      for (int u = 0; u < kPairsInFlight; ++u) {
+        const int k = kb + u * nslots;
+        if (k < K) {
+          r0[u] = __ldcs(src + (2 * k) * rowq + pv);
+          r1[u] = __ldcs(src + (2 * k + 1) * rowq + pv);
+        }
       }
     }
 #pragma unroll
@@ -127,8 +155,8 @@ decode_kernel(const DecodeArgs a) {
           for (int r = 0; r < R; ++r)
             yacc[r][j] = fmaf(c0[r], o0[j], fmaf(c1[r], o1[j], yacc[r][j]));
         }
-        __stcs(dst + (2 * k) * PV + pv, make_float4(o0[0], o0[1], o0[2], o0[3]));
-        __stcs(dst + (2 * k + 1) * PV + pv, make_float4(o1[0], o1[1], o1[2], o1[3]));
+        __stcs(dst + (2 * k) * rowq + pv, make_float4(o0[0], o0[1], o0[2], o0[3]));
+        __stcs(dst + (2 * k + 1) * rowq + pv, make_float4(o1[0], o1[1], o1[2], o1[3]));
       }
     }
   }
@@ -136,26 +164,29 @@ decode_kernel(const DecodeArgs a) {
 #pragma unroll
   for (int r = 0; r < R; ++r)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) s_red[(kslot * R + r) * P + p0 + j] = yacc[r][j];
+    for (int j = 0; j < 4; ++j) s_red[(kslot * R + r) * CB + p0 + j] = yacc[r][j];
   __syncthreads();
-  for (int i = tid; i < R * P; i += kDecodeThreads) {
-    float s = 0.f;
-    for (int q = 0; q < nslots; ++q) s += s_red[q * R * P + i];
-    io_store(a.y, bh * R * P + i, s, a.bf16);
+  for (int i = tid; i < R * CB; i += kDecodeThreads) {
+    float acc = 0.f;
+    for (int q = 0; q < nslots; ++q) acc += s_red[q * R * CB + i];
+    const int r = i / CB, c = i % CB;
+    io_store(a.y, bh * R * P + r * P + cb * CB + c, acc, a.bf16);
   }
 }
 
 template <int R>
 cudaError_t launch_r(const DecodeArgs& a, cudaStream_t s) {
   const int P = (int)a.P, N = (int)a.N;
-  const int nslots = kDecodeThreads / (P / 4);
-  const size_t smem = sizeof(float) * (N + 3 * R * N + 2 * R * P + (size_t)nslots * R * P);
+  const int CB = P < kMaxCols ? P : kMaxCols;
+  const int nslots = kDecodeThreads / (CB / 4);
+  const size_t smem = sizeof(float) * (N + 3 * R * N + 2 * R * CB + (size_t)nslots * R * CB);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<R>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  decode_kernel<R><<<(unsigned)(a.batch * a.nheads), kDecodeThreads, smem, s>>>(a);
+  const int64_t blocks = a.batch * a.nheads * (P / CB);
+  decode_kernel<R><<<(unsigned)blocks, kDecodeThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -59,11 +59,17 @@ struct Cfg {
   static constexpr int SMALL_OFF = G_OFF + kN * 128;
   // small region: per-token gates, chunk-end angles, the Q x Q decay table;
   // the slot angle sums live in the x operand block (free until x is staged)
-  static constexpr int SMALL_BYTES = 6 * Q * 4 + kPairs * 4 + Q * Q * 4 + 64;
-  static_assert(SLOTS_MAX * kPairs * 4 <= OPB, "slot sums must fit in the x block");
-  // + alignment slack; at least 80 KB so that no more than two CTAs (2 x 256
-  // TMEM columns) share an SM
-  static constexpr int SMEM_RAW = SMALL_OFF + SMALL_BYTES + 1024;
+  // D table [Q][Q], also the staging area of the next chunk's theta [Q][N/2]
+  static constexpr int DT_FLOATS = (Q * Q > Q * kPairs) ? Q * Q : Q * kPairs;
+  static constexpr int SMALL_BYTES = 8 * Q * 4 + 3 * kPairs * 4 + DT_FLOATS * 4 + 64;
+  // the w*x block holds the slot angle sums at its start and the next chunk's
+  // gates (dt[Q+1], lam[Q+1], A[Q]) in its last KB while it is otherwise free
+  static constexpr int GST_OFF = XW_OFF + OPB - 1024;
+  static_assert(SLOTS_MAX * kPairs * 4 <= OPB - 1024, "slot sums must fit in the w*x block");
+  static_assert((3 * Q + 4) * 4 <= 1024, "gate staging must fit in 1 KB");
+  // at least 80 KB so that no more than two CTAs (2 x 256 TMEM columns) share
+  // an SM; the dynamic shared memory base is declared 1024-byte aligned
+  static constexpr int SMEM_RAW = SMALL_OFF + SMALL_BYTES;
   static constexpr int SMEM = SMEM_RAW < 80 * 1024 ? 80 * 1024 : SMEM_RAW;
   static_assert(MINB * (SMEM + 1024) <= 233472, "CTAs per SM must fit the SM's shared memory");
   // P tile mt: ((mt + 1) * MT / 64) blocks of [MT][128 B]
@@ -134,10 +140,13 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
   constexpr int SLOTS = Q / TQ;                           // active rotation slots
   constexpr int CW = kP / CQN;                            // state / output columns per thread
   constexpr float kL2E = 1.4426950408889634f;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw;
   const uint32_t sbase = smem_u32(sm);
+  if ((sbase & 1023u) != 0) {  // the swizzled operand layout needs 1 KB alignment
+    if (threadIdx.x == 0 && a.status) atomicCAS(a.status, 0, (int)M3_ERR_CUDA);
+    return;
+  }
   float* s_l2 = reinterpret_cast<float*>(sm + C::SMALL_OFF);  // chunk-local Lam_t (prefix sum)
   float* s_gam = s_l2 + Q;
   float* s_del = s_gam + Q;
@@ -145,9 +154,14 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
   float* s_dt = s_w + Q;
   float* s_lg = s_dt + Q;                       // Lam_t * log2(e)
   float* s_phe = s_lg + Q;                      // [kPairs] chunk-end angles
-  float* s_D = s_phe + kPairs;                  // [Q][Q] decay x trapezoid weights
-  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_D + Q * Q);
-  float* s_part = reinterpret_cast<float*>(sm + C::X_OFF);  // [slots][kPairs], x block
+  float* s_E = s_phe + kPairs;                  // exp(Lam_t - ref)             [Q]
+  float* s_F = s_E + Q;                         // exp(ref - Lam_s) * delta_s   [Q]
+  float2* s_pcs = reinterpret_cast<float2*>(s_F + Q);  // cos, sin of chunk-end angles [kPairs]
+  float* s_D = reinterpret_cast<float*>(s_pcs + kPairs);  // [Q][Q] decay x trapezoid weights
+  float* s_th = s_D;                            // next chunk's theta [Q][N/2] (same area)
+  float* s_gst = reinterpret_cast<float*>(sm + C::GST_OFF);  // next chunk's gates
+  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_D + C::DT_FLOATS);
+  float* s_part = reinterpret_cast<float*>(sm + C::XW_OFF);  // [slots][kPairs], w*x block
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_bar + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -160,8 +174,6 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
   const __nv_bfloat16* Cg = reinterpret_cast<const __nv_bfloat16*>(a.C);
   const __nv_bfloat16* Xg = reinterpret_cast<const __nv_bfloat16*>(a.x);
   const int64_t tokB = G * R * kN;   // element stride of one token in B, C
-  const int64_t tokT = G * kPairs;   // element stride of one token in theta
-  const int64_t tokX = H * R * kP;   // element stride of one token in x, y
 
   if (warp == 0) {
     tmem_alloc(s_tmem, C::TMEM_COLS);
@@ -224,33 +236,49 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
   const int64_t c_begin = seg * pl.cps;
   const int64_t c_end = min(c_begin + pl.cps, a.nchunks);
 
+  // Prefetch of a chunk's gates, theta and x with cp.async: gates into s_gst,
+  // theta into the decay-table area, x straight into its swizzled MMA tile.
+  // Issued while the previous chunk's epilogue and state update run.
+  auto prefetch = [&](int64_t cn) {
+    if (cn >= c_end) return;
+    const int64_t cn0 = cn * Q;
+    const int ntn = (int)min((int64_t)Q, L - cn0);
+    for (int i = tid; i < 3 * Q + 2; i += NTH) {
+      const int which = i < Q + 1 ? 0 : (i < 2 * Q + 2 ? 1 : 2);
+      const int t = which == 0 ? i : (which == 1 ? i - (Q + 1) : i - (2 * Q + 2));
+      const bool v = cn0 + t < L;
+      const float* base = which == 0 ? a.dt : (which == 1 ? a.lam : a.A);
+      cp_async4(s_gst + i, v ? base + (b * L + cn0 + t) * H + h : base, v);
+    }
+    for (int i = tid; i < Q * 16; i += NTH) {
+      const int t = i >> 4, gr = i & 15;
+      const bool v = t < ntn;
+      cp_async16(s_th + t * kPairs + 4 * gr,
+                 v ? a.theta + ((b * L + cn0 + t) * G + g) * kPairs + 4 * gr : a.theta, v);
+    }
+    for (int i = tid; i < M * 8; i += NTH) {
+      const int row = i >> 3, ch = i & 7, t = row / R, r = row % R;
+      const bool v = t < ntn;
+      cp_async16(sm + C::X_OFF + sw128_off(row, ch),
+                 v ? Xg + ((b * L + cn0 + t) * H + h) * R * kP + r * kP + ch * 8 : Xg, v);
+    }
+    cp_async_commit();
+  };
+  prefetch(c_begin);
+
   for (int64_t c = c_begin; c < c_end && !aborted; ++c) {
     const int64_t c0 = c * Q;
     const int nt = (int)min((int64_t)Q, L - c0);
     const __nv_bfloat16* Bc = Bg + ((b * L + c0) * G + g) * R * kN + 8 * kg;
     const __nv_bfloat16* Cc = Cg + ((b * L + c0) * G + g) * R * kN + 8 * kg;
-    const float* Tc = a.theta + ((b * L + c0) * G + g) * kPairs + 4 * kg;
-    const __nv_bfloat16* Xc = Xg + ((b * L + c0) * H + h) * R * kP;
     const bool slot_live = tq < SLOTS;
 
-    // ---- gate loads first, then this chunk's B / C / theta -------------------
-    const bool gate_warp = warp < (Q + 31) / 32;
-    float g_dt = 0.f, g_lm = 0.f, g_av = 0.f, g_nx = 0.f;
-    if (gate_warp && tid < nt) {
-      const int64_t bt = b * L + c0 + tid;
-      g_dt = __ldg(a.dt + bt * H + h);
-      g_lm = __ldg(a.lam + bt * H + h);
-      g_av = __ldg(a.A + bt * H + h);
-      if (c0 + tid + 1 < L)
-        g_nx = (1.f - __ldg(a.lam + (bt + 1) * H + h)) * __ldg(a.dt + (bt + 1) * H + h);
-    }
+    // ---- this chunk's B / C straight to registers; the rest was prefetched -----
     uint4 rb[TQ][R], rc[TQ][R];
-    float4 th[TQ];
 #pragma unroll
     for (int u = 0; u < TQ; ++u) {
       const int t = tq * TQ + u;
       const bool ld = slot_live && t < nt;
-      th[u] = ld ? __ldg(reinterpret_cast<const float4*>(Tc + t * tokT)) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         rb[u][r] = ld ? ldg_u128(Bc + t * tokB + r * kN) : make_uint4(0, 0, 0, 0);
@@ -259,6 +287,16 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
     }
 
     // ---- gates and the chunk-local prefix sum of dt*A (warp shuffle scan) ----
+    cp_async_wait_all();
+    __syncthreads();  // prefetched gates, theta and x visible to every thread
+    const bool gate_warp = warp < (Q + 31) / 32;
+    float g_dt = 0.f, g_lm = 0.f, g_av = 0.f, g_nx = 0.f;
+    if (gate_warp && tid < nt) {
+      g_dt = s_gst[tid];
+      g_lm = s_gst[Q + 1 + tid];
+      g_av = s_gst[2 * Q + 2 + tid];
+      g_nx = (1.f - s_gst[Q + 2 + tid]) * s_gst[tid + 1];  // zero-filled past the sequence end
+    }
     if (gate_warp) {  // whole warps take part in the shuffle scan
       const bool inq = tid < Q;
       if (inq) {
@@ -283,9 +321,12 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
 #pragma unroll
     for (int u = 0; u < TQ; ++u) {
       const int t = tq * TQ + u;
-      const float d = (slot_live && t < nt) ? s_dt[t] : 0.f;
-      ang[u][0] = make_float2(d * th[u].x, d * th[u].y);
-      ang[u][1] = make_float2(d * th[u].z, d * th[u].w);
+      const bool live_t = slot_live && t < nt;
+      const float d = live_t ? s_dt[t] : 0.f;
+      const float4 th = live_t ? *reinterpret_cast<const float4*>(s_th + t * kPairs + 4 * kg)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+      ang[u][0] = make_float2(d * th.x, d * th.y);
+      ang[u][1] = make_float2(d * th.z, d * th.w);
       part[0] += ang[u][0].x; part[1] += ang[u][0].y;
       part[2] += ang[u][1].x; part[3] += ang[u][1].y;
     }
@@ -305,10 +346,17 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
     }
     const float lend = s_l2[nt - 1];
     const float l2end = lend * kL2E;
+    // The decay table is built from per-token factors around the chunk's
+    // mid decay, exp(Lam_t - Lam_s) = E_t * F_s, while the chunk's total decay
+    // keeps both factors inside fp32 (|Lam_end| < 160); else entry by entry.
+    const float l2ref = 0.5f * l2end;
+    const bool fac_ok = l2end > -230.f;
     if (tid < Q) {
       const float lg = s_l2[tid] * kL2E;
       s_lg[tid] = lg;
       s_w[tid] = (tid < nt) ? ex2(l2end - lg) * s_del[tid] : 0.f;
+      s_E[tid] = fac_ok ? ex2(lg - l2ref) : 0.f;
+      s_F[tid] = fac_ok ? ex2(l2ref - lg) * s_del[tid] : 0.f;
     }
 
     // ---- operands: Bt (and Ct) rotated by -Phi_t (16-byte row pieces) ---------
@@ -351,24 +399,22 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
         }
       }
     }
-    // the x loads go out before the barrier so their latency overlaps it
-    constexpr int PER = M * 8 / NTH;
-    uint4 xv[PER];
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      const int q = tid + j * NTH;
-      const int row = q >> 3, chq = q & 7, t = row / R, r = row % R;
-      xv[j] = (t < nt) ? ldg_u128(Xc + t * tokX + r * kP + chq * 8) : make_uint4(0, 0, 0, 0);
+    __syncthreads();  // s_w ready; slot sums read, so the w*x block is free
+    if (tid < kPairs) {
+      float sn, cs;
+      sincosf(s_phe[tid], &sn, &cs);
+      s_pcs[tid] = make_float2(cs, sn);
     }
-    __syncthreads();  // s_w ready for the x pass
 
-    // ---- w * x (chunk-state operand); x itself is copied after MMA issue ------
+    // ---- w * x (chunk-state operand) from the prefetched x tile --------------
+    constexpr int PER = M * 8 / NTH;
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
       const int q = tid + j * NTH;
       const int row = q >> 3, chq = q & 7, t = row / R;
       const float w = s_w[t];
-      const uint32_t iv[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+      const uint4 xq = *reinterpret_cast<const uint4*>(sm + C::X_OFF + sw128_off(row, chq));
+      const uint32_t iv[4] = {xq.x, xq.y, xq.z, xq.w};
       uint32_t ov[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -377,15 +423,6 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
         ov[e] = pack_bf16(f.x, f.y);
       }
       *reinterpret_cast<uint4*>(sm + C::XW_OFF + sw128_off(row, chq)) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
-    }
-    if (MODE == MODE_FULL) {  // D[t][s] = [s <= t] exp(Lam_t - Lam_s) (s == t ? gamma_t : delta_s)
-#pragma unroll
-      for (int e = tid; e < Q * Q; e += NTH) {
-        const int t = e / Q, s2 = e % Q;
-        float d = 0.f;
-        if (t < nt && s2 <= t) d = ex2(s_lg[t] - s_lg[s2]) * ((s2 == t) ? s_gam[t] : s_del[s2]);
-        s_D[e] = d;
-      }
     }
     fence_async_smem();
     tc_fence_before();
@@ -417,17 +454,35 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
       }
       mma_commit(s_bar);
     }
-    if (MODE == MODE_FULL) {  // x into the MMA2 operand while MMA1/MMA3 run
+    if (MODE == MODE_FULL) {  // while MMA1/MMA3 run: D[t][s] = [s <= t] exp(Lam_t - Lam_s) w
 #pragma unroll
-      for (int j = 0; j < PER; ++j) {
-        const int q = tid + j * NTH;
-        *reinterpret_cast<uint4*>(sm + C::X_OFF + sw128_off(q >> 3, q & 7)) = xv[j];
+      for (int e4 = tid; e4 < Q * Q / 4; e4 += NTH) {
+        const int t = (4 * e4) / Q, s0 = (4 * e4) % Q;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        if (t < nt && s0 <= t) {
+          if (fac_ok) {
+            const float et = s_E[t];
+            const float4 fw = *reinterpret_cast<const float4*>(s_F + s0);
+            d[0] = et * fw.x; d[1] = et * fw.y; d[2] = et * fw.z; d[3] = et * fw.w;
+          } else {
+            const float lt = s_lg[t];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) d[j] = ex2(lt - s_lg[s0 + j]) * s_del[s0 + j];
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (s0 + j == t) d[j] = s_gam[t];
+            else if (s0 + j > t) d[j] = 0.f;
+          }
+        }
+        *reinterpret_cast<float4*>(s_D + 4 * e4) = make_float4(d[0], d[1], d[2], d[3]);
       }
     }
     const bool ok1 = (tid == 0) ? wait_bar(s_bar, phase, a.status) : true;
     phase ^= 1;
     if (__syncthreads_or(!ok1)) { aborted = true; break; }
     tc_fence_after();
+    if (MODE == MODE_STATE) prefetch(c + 1);
 
     if (MODE == MODE_FULL) {
       // ---- mask the scores into P (bf16, K-major, over Bt / Xw) -------------
@@ -498,6 +553,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
       phase ^= 1;
       if (__syncthreads_or(!ok2)) { aborted = true; break; }
       tc_fence_after();
+      prefetch(c + 1);  // x, theta and gate buffers are free from here on
 
       // ---- epilogue: y = P x + exp(Lam_t) Ct G ---------------------------------
 #pragma unroll
@@ -538,8 +594,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
     // ---- state update: G <- Rot(Phi_end) (exp(Lam_end) G + Sc) ---------------
     {
       const float phe = s_phe[n >> 1];
-      float sn, cs;
-      sincosf(phe, &sn, &cs);
+      const float2 pcs = s_pcs[n >> 1];
+      const float cs = pcs.x, sn = pcs.y;
       const float el = ex2(l2end);
       const float ss = (n & 1) ? sn : -sn;  // even row: c v - s o; odd row: c v + s o
 #pragma unroll
@@ -634,16 +690,35 @@ __global__ void __launch_bounds__(256) tc_seg_pass_kernel(const ScanArgs a, cons
   }
 }
 
+// Segments per chain: minimise the estimated time in chunk steps of one CTA,
+//   rounds(full pass) * cps + kStateCost * rounds(state pass) * cps,
+// where a round is one wave of CTAs over the SMs (148 SMs x CTAs per SM) and
+// the state-only pass costs about kStateCost of a full chunk step.
 TcPlan make_plan(const ScanArgs& a) {
-  TcPlan pl{};
+  constexpr double kStateCost = 0.4;
   const int64_t chains = a.batch * a.nheads;
-  const int64_t target = 2 * 148;  // CTAs for at least two waves of one CTA per SM
-  int64_t nseg = chains >= target ? 1 : (target + chains - 1) / chains;
-  if (nseg > a.nchunks) nseg = a.nchunks;
-  if (nseg < 1) nseg = 1;
-  pl.cps = (a.nchunks + nseg - 1) / nseg;
-  pl.nseg = (a.nchunks + pl.cps - 1) / pl.cps;
-  return pl;
+  const int64_t slots = 148 * ((a.Q * a.R == 64) ? 2 : 1);
+  TcPlan best{};
+  double best_cost = 0.0;
+  const int64_t max_seg = a.nchunks < 64 ? a.nchunks : 64;
+  for (int64_t ns = 1; ns <= (max_seg > 0 ? max_seg : 1); ++ns) {
+    const int64_t cps = (a.nchunks + ns - 1) / ns;
+    const int64_t nseg = (a.nchunks + cps - 1) / cps;
+    if (nseg != ns) continue;
+    const int64_t rounds_full = (chains * nseg + slots - 1) / slots;
+    const int64_t rounds_state = nseg > 1 ? (chains * (nseg - 1) + slots - 1) / slots : 0;
+    const double cost = (double)rounds_full * cps + kStateCost * (double)rounds_state * cps;
+    if (ns == 1 || cost < best_cost * 0.97) {  // more segments only for a clear gain
+      best_cost = cost;
+      best.nseg = nseg;
+      best.cps = cps;
+    }
+  }
+  if (best.nseg < 1) {
+    best.nseg = 1;
+    best.cps = a.nchunks;
+  }
+  return best;
 }
 
 template <int R, int Q, int MODE>

@@ -170,6 +170,25 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Asynchronous global -> shared copies (zero-filled when `valid` is false;
+// `gmem` must still be a valid address).
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem)), "l"(gmem),
+               "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Byte offset of 16-byte chunk `ch` (0..7) of row `row` in a 128-byte-swizzled
 // tile whose base is 1024-byte aligned.
 __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t ch) {
