@@ -16,11 +16,11 @@
 // (B, C, B_prev, x, x_prev, the cos/sin table) are staged in shared memory;
 // y is reduced over kslots through shared memory.
 #include "m3_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace m3 {
 namespace {
 
-constexpr int kDecodeThreads = 128;
 constexpr int kMaxCols = 128;  // state columns per CTA (whole rows: P <= 128)
 constexpr int kPairsInFlight = 4;  // pairs whose state rows are loaded before any is computed
 
@@ -30,13 +30,19 @@ constexpr int kPairsInFlight = 4;  // pairs whose state rows are loaded before a
 // between CTAs that run at different times costs HBM locality.
 // Resident CTAs per SM the register budget is sized for (more state bytes in
 // flight for small R, room for the rank-R operands for large R).
+// 128 threads per CTA; the register budget is sized for the resident CTAs
+// per SM (more state bytes in flight for small R, room for the rank-R
+// operands for large R).
 template <int R>
-struct DecodeOcc {
-  static constexpr int value = R == 1 ? 7 : (R == 2 ? 6 : (R == 4 ? 5 : 3));
+struct DecodeCfg {
+  static constexpr int threads = 128;
+  static constexpr int occupancy = R == 1 ? 7 : (R == 2 ? 5 : (R == 4 ? 4 : 3));
 };
 
 template <int R>
-__global__ void __launch_bounds__(kDecodeThreads, DecodeOcc<R>::value) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(DecodeCfg<R>::threads, DecodeCfg<R>::occupancy)
+decode_kernel(const DecodeArgs a) {
+  constexpr int kDecodeThreads = DecodeCfg<R>::threads;
   const int P = (int)a.P, N = (int)a.N, K = N / 2;
   const int CB = P < kMaxCols ? P : kMaxCols;
   const int nblk = P / CB;
@@ -50,9 +56,9 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeOcc<R>::value) decode_ke
   extern __shared__ float sm[];
   float* s_ac = sm;               // alpha cos(dt theta_k)          [K]
   float* s_as = s_ac + K;         // alpha sin(dt theta_k)          [K]
-  float* s_Bp = s_as + K;         // B_prev                         [R][N]
-  float* s_Bt = s_Bp + R * N;     // B_t                            [R][N]
-  float* s_Ct = s_Bt + R * N;     // C_t                            [R][N]
+  float* s_Bp = s_as + K;         // B_prev, transposed             [N][R]
+  float* s_Bt = s_Bp + R * N;     // B_t, transposed                [N][R]
+  float* s_Ct = s_Bt + R * N;     // C_t, transposed                [N][R]
   float* s_xe = s_Ct + R * N;     // (1-lam) dt x_prev              [R][CB]
   float* s_xg = s_xe + R * CB;    // lam dt x_t                     [R][CB]
   float* s_red = s_xg + R * CB;   // partial y per kslot            [nslots][R][CB]
@@ -87,10 +93,11 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeOcc<R>::value) decode_ke
     s_ac[k] = alpha * cs;
     s_as[k] = alpha * sn;
   }
-  for (int i = tid; i < R * N; i += kDecodeThreads) {
-    s_Bt[i] = io_load(a.B, bg * R * N + i, a.bf16);
-    s_Ct[i] = io_load(a.C, bg * R * N + i, a.bf16);
-    s_Bp[i] = prev ? io_load(a.B_prev, bg * R * N + i, a.bf16) : 0.f;
+  for (int i = tid; i < R * N; i += kDecodeThreads) {  // i = r * N + n -> [n][r]
+    const int r = i / N, nn = i % N, ti = nn * R + r;
+    s_Bt[ti] = io_load(a.B, bg * R * N + i, a.bf16);
+    s_Ct[ti] = io_load(a.C, bg * R * N + i, a.bf16);
+    s_Bp[ti] = prev ? io_load(a.B_prev, bg * R * N + i, a.bf16) : 0.f;
   }
   for (int i = tid; i < R * CB; i += kDecodeThreads) {
     const int r = i / CB, c = i % CB;
@@ -100,14 +107,15 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeOcc<R>::value) decode_ke
   }
   __syncthreads();
 
-  float xg[R][4], xe[R][4], yacc[R][4];
+  // column pairs (p0, p0+1) and (p0+2, p0+3) as packed fp32x2 operands
+  float2 xg[R][2], xe[R][2], yacc[R][2];
 #pragma unroll
   for (int r = 0; r < R; ++r)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      xg[r][j] = s_xg[r * CB + p0 + j];
-      xe[r][j] = s_xe[r * CB + p0 + j];
-      yacc[r][j] = 0.f;
+    for (int j = 0; j < 2; ++j) {
+      xg[r][j] = make_float2(s_xg[r * CB + p0 + 2 * j], s_xg[r * CB + p0 + 2 * j + 1]);
+      xe[r][j] = make_float2(s_xe[r * CB + p0 + 2 * j], s_xe[r * CB + p0 + 2 * j + 1]);
+      yacc[r][j] = make_float2(0.f, 0.f);
     }
 
   for (int kb = kslot; kb < K; kb += kPairsInFlight * nslots) {
@@ -128,32 +136,35 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeOcc<R>::value) decode_ke
         const float ac = s_ac[k], as = s_as[k];
         float bp0[R], bp1[R], bt0[R], bt1[R], c0[R], c1[R];
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const float2 vbp = *reinterpret_cast<const float2*>(s_Bp + r * N + 2 * k);
-          const float2 vbt = *reinterpret_cast<const float2*>(s_Bt + r * N + 2 * k);
-          const float2 vc = *reinterpret_cast<const float2*>(s_Ct + r * N + 2 * k);
-          bp0[r] = vbp.x; bp1[r] = vbp.y;
-          bt0[r] = vbt.x; bt1[r] = vbt.y;
-          c0[r] = vc.x; c1[r] = vc.y;
+        for (int r = 0; r < R; ++r) {  // rows 2k and 2k+1 are adjacent R-vectors
+          bp0[r] = s_Bp[(2 * k) * R + r]; bp1[r] = s_Bp[(2 * k + 1) * R + r];
+          bt0[r] = s_Bt[(2 * k) * R + r]; bt1[r] = s_Bt[(2 * k + 1) * R + r];
+          c0[r] = s_Ct[(2 * k) * R + r]; c1[r] = s_Ct[(2 * k + 1) * R + r];
         }
-        float in0[4] = {r0[u].x, r0[u].y, r0[u].z, r0[u].w};
-        float in1[4] = {r1[u].x, r1[u].y, r1[u].z, r1[u].w};
+        const float2 in0[2] = {make_float2(r0[u].x, r0[u].y), make_float2(r0[u].z, r0[u].w)};
+        const float2 in1[2] = {make_float2(r1[u].x, r1[u].y), make_float2(r1[u].z, r1[u].w)};
         float o0[4], o1[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float g0 = in0[j], g1 = in1[j], u0 = 0.f, u1 = 0.f;
+        for (int j = 0; j < 2; ++j) {
+          float2 g0 = in0[j], g1 = in1[j], u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
 #pragma unroll
           for (int r = 0; r < R; ++r) {
-            g0 = fmaf(bp0[r], xe[r][j], g0);
-            g1 = fmaf(bp1[r], xe[r][j], g1);
-            u0 = fmaf(bt0[r], xg[r][j], u0);
-            u1 = fmaf(bt1[r], xg[r][j], u1);
+            g0 = tc::ffma2(make_float2(bp0[r], bp0[r]), xe[r][j], g0);
+            g1 = tc::ffma2(make_float2(bp1[r], bp1[r]), xe[r][j], g1);
+            u0 = tc::ffma2(make_float2(bt0[r], bt0[r]), xg[r][j], u0);
+            u1 = tc::ffma2(make_float2(bt1[r], bt1[r]), xg[r][j], u1);
           }
-          o0[j] = fmaf(ac, g0, fmaf(-as, g1, u0));
-          o1[j] = fmaf(as, g0, fmaf(ac, g1, u1));
+          // (h'_{2k}, h'_{2k+1}) = alpha Rot(phi) (g_{2k}, g_{2k+1}) + (u_{2k}, u_{2k+1})
+          const float2 w0 = tc::ffma2(make_float2(ac, ac), g0,
+                                      tc::ffma2(make_float2(-as, -as), g1, u0));
+          const float2 w1 = tc::ffma2(make_float2(as, as), g0,
+                                      tc::ffma2(make_float2(ac, ac), g1, u1));
 #pragma unroll
           for (int r = 0; r < R; ++r)
-            yacc[r][j] = fmaf(c0[r], o0[j], fmaf(c1[r], o1[j], yacc[r][j]));
+            yacc[r][j] = tc::ffma2(make_float2(c0[r], c0[r]), w0,
+                                   tc::ffma2(make_float2(c1[r], c1[r]), w1, yacc[r][j]));
+          o0[2 * j] = w0.x; o0[2 * j + 1] = w0.y;
+          o1[2 * j] = w1.x; o1[2 * j + 1] = w1.y;
         }
         __stcs(dst + (2 * k) * rowq + pv, make_float4(o0[0], o0[1], o0[2], o0[3]));
         __stcs(dst + (2 * k + 1) * rowq + pv, make_float4(o1[0], o1[1], o1[2], o1[3]));
@@ -164,7 +175,10 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeOcc<R>::value) decode_ke
 #pragma unroll
   for (int r = 0; r < R; ++r)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) s_red[(kslot * R + r) * CB + p0 + j] = yacc[r][j];
+    for (int j = 0; j < 2; ++j) {
+      s_red[(kslot * R + r) * CB + p0 + 2 * j] = yacc[r][j].x;
+      s_red[(kslot * R + r) * CB + p0 + 2 * j + 1] = yacc[r][j].y;
+    }
   __syncthreads();
   for (int i = tid; i < R * CB; i += kDecodeThreads) {
     float acc = 0.f;
@@ -178,6 +192,7 @@ template <int R>
 cudaError_t launch_r(const DecodeArgs& a, cudaStream_t s) {
   const int P = (int)a.P, N = (int)a.N;
   const int CB = P < kMaxCols ? P : kMaxCols;
+  constexpr int kDecodeThreads = DecodeCfg<R>::threads;
   const int nslots = kDecodeThreads / (CB / 4);
   const size_t smem = sizeof(float) * (N + 3 * R * N + 2 * R * CB + (size_t)nslots * R * CB);
   if (smem > 48 * 1024) {

@@ -24,6 +24,8 @@
 // and are read by tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) issued by one
 // thread; accumulators live in TMEM and are read back with tcgen05.ld.
 // Supported: N = 128, P = 64, M = Q*R in {64, 128, 256}.
+#include <cuda.h>  // CUtensorMap (the encoder is reached through the runtime)
+
 #include "m3_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -62,6 +64,8 @@ struct Cfg {
   // D table [Q][Q], also the staging area of the next chunk's theta [Q][N/2]
   static constexpr int DT_FLOATS = (Q * Q > Q * kPairs) ? Q * Q : Q * kPairs;
   static constexpr int SMALL_BYTES = 8 * Q * 4 + 3 * kPairs * 4 + DT_FLOATS * 4 + 64;
+  // the D table / theta staging area is a TMA destination: 128-byte aligned
+  static_assert((SMALL_OFF + 8 * Q * 4 + 3 * kPairs * 4) % 128 == 0, "theta staging alignment");
   // the w*x block holds the slot angle sums at its start and the next chunk's
   // gates (dt[Q+1], lam[Q+1], A[Q]) in its last KB while it is otherwise free
   static constexpr int GST_OFF = XW_OFF + OPB - 1024;
@@ -87,6 +91,12 @@ struct Cfg {
   __host__ __device__ static constexpr int y_col(int mt) { return 64 * mt; }
   __host__ __device__ static constexpr int y2_col(int mt) { return 64 * (NT + mt); }
   static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+// TMA descriptors of one call: x, B, C (bf16, 128-byte swizzled boxes of
+// {64 elements, R rows, Q tokens}) and theta (fp32 boxes {N/2, 1, Q}).
+struct TcMaps {
+  CUtensorMap x, b, c, th;
 };
 
 struct TcPlan {
@@ -116,10 +126,6 @@ __device__ bool wait_bar(uint64_t* bar, uint32_t parity, int* status) {
   return true;
 }
 
-__device__ __forceinline__ uint4 ldg_u128(const void* p) {
-  return __ldg(reinterpret_cast<const uint4*>(p));
-}
-
 // Thread layout (NTH = 256 or 512 threads).
 //  - TMEM work: warp w reads TMEM lanes 32*(w%4)..+31 ("quadrant" qd = w % 4)
 //    and takes column part cq = w / 4 of NTH / 128 parts; state row n =
@@ -131,7 +137,7 @@ __device__ __forceinline__ uint4 ldg_u128(const void* p) {
 //    through a small shared array.
 template <int R, int Q, int MODE>
 __global__ void __launch_bounds__(Cfg<R, Q>::NTH, Cfg<R, Q>::MINB)
-tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
+tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps maps) {
   using C = Cfg<R, Q>;
   constexpr int M = C::M, MT = C::MT, NT = C::NT;
   constexpr int NTH = C::NTH;
@@ -160,9 +166,10 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
   float* s_D = reinterpret_cast<float*>(s_pcs + kPairs);  // [Q][Q] decay x trapezoid weights
   float* s_th = s_D;                            // next chunk's theta [Q][N/2] (same area)
   float* s_gst = reinterpret_cast<float*>(sm + C::GST_OFF);  // next chunk's gates
-  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_D + C::DT_FLOATS);
   float* s_part = reinterpret_cast<float*>(sm + C::XW_OFF);  // [slots][kPairs], w*x block
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_bar + 1);
+  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_D + C::DT_FLOATS);  // MMA completion
+  uint64_t* s_tbar = s_bar + 1;                                         // TMA completion
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_bar + 2);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, cq = warp >> 2;
@@ -170,10 +177,6 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
   const int64_t seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int64_t L = a.seqlen, H = a.nheads, G = a.ngroups;
   const int64_t g = h / (H / G);
-  const __nv_bfloat16* Bg = reinterpret_cast<const __nv_bfloat16*>(a.B);
-  const __nv_bfloat16* Cg = reinterpret_cast<const __nv_bfloat16*>(a.C);
-  const __nv_bfloat16* Xg = reinterpret_cast<const __nv_bfloat16*>(a.x);
-  const int64_t tokB = G * R * kN;   // element stride of one token in B, C
 
   if (warp == 0) {
     tmem_alloc(s_tmem, C::TMEM_COLS);
@@ -181,6 +184,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
   }
   if (tid == 0) {
     mbar_init(s_bar, 1);
+    mbar_init(s_tbar, 1);
     fence_mbar_init();
   }
   tc_fence_before();
@@ -188,8 +192,9 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
   tc_fence_after();
   const uint32_t tm = *s_tmem;
   const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
-  uint32_t phase = 0;
+  uint32_t phase = 0, tphase = 0;
   bool aborted = false;
+  bool tma_pending = false;  // thread 0: a prefetch is in flight on s_tbar
 
   // ---- incoming state: thread (n, cq) owns columns [CW*cq, CW*cq + CW) of row n
   const int n = 32 * qd + lane;
@@ -236,31 +241,34 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
   const int64_t c_begin = seg * pl.cps;
   const int64_t c_end = min(c_begin + pl.cps, a.nchunks);
 
-  // Prefetch of a chunk's gates, theta and x with cp.async: gates into s_gst,
-  // theta into the decay-table area, x straight into its swizzled MMA tile.
-  // Issued while the previous chunk's epilogue and state update run.
+  // Prefetch of a chunk's inputs while the previous chunk's epilogue and
+  // state update run: one thread issues TMA loads of raw B and C (straight
+  // into the swizzled operand tiles, rotated in place later), x (into its
+  // MMA tile) and theta (into the decay-table area); the gates go by cp.async.
   auto prefetch = [&](int64_t cn) {
     if (cn >= c_end) return;
     const int64_t cn0 = cn * Q;
-    const int ntn = (int)min((int64_t)Q, L - cn0);
+    if (tid == 0) {
+      constexpr uint32_t kTile = Q * R * 128;  // bytes of one {64, R, Q} bf16 box
+      const uint32_t bytes = kTile * (MODE == MODE_FULL ? 5 : 3) + Q * kPairs * 4;
+      mbar_expect_tx(s_tbar, bytes);
+      tma_pending = true;
+      const int tok = (int)(b * L + cn0);
+      tma_load_3d(sm + C::X_OFF, &maps.x, 0, (int)(h * R), tok, s_tbar);
+      tma_load_3d(sm + C::B_OFF, &maps.b, 0, (int)(g * R), tok, s_tbar);
+      tma_load_3d(sm + C::B_OFF + C::OPB, &maps.b, 64, (int)(g * R), tok, s_tbar);
+      if (MODE == MODE_FULL) {
+        tma_load_3d(sm + C::C_OFF, &maps.c, 0, (int)(g * R), tok, s_tbar);
+        tma_load_3d(sm + C::C_OFF + C::OPB, &maps.c, 64, (int)(g * R), tok, s_tbar);
+      }
+      tma_load_3d(s_th, &maps.th, 0, (int)g, tok, s_tbar);
+    }
     for (int i = tid; i < 3 * Q + 2; i += NTH) {
       const int which = i < Q + 1 ? 0 : (i < 2 * Q + 2 ? 1 : 2);
       const int t = which == 0 ? i : (which == 1 ? i - (Q + 1) : i - (2 * Q + 2));
       const bool v = cn0 + t < L;
       const float* base = which == 0 ? a.dt : (which == 1 ? a.lam : a.A);
       cp_async4(s_gst + i, v ? base + (b * L + cn0 + t) * H + h : base, v);
-    }
-    for (int i = tid; i < Q * 16; i += NTH) {
-      const int t = i >> 4, gr = i & 15;
-      const bool v = t < ntn;
-      cp_async16(s_th + t * kPairs + 4 * gr,
-                 v ? a.theta + ((b * L + cn0 + t) * G + g) * kPairs + 4 * gr : a.theta, v);
-    }
-    for (int i = tid; i < M * 8; i += NTH) {
-      const int row = i >> 3, ch = i & 7, t = row / R, r = row % R;
-      const bool v = t < ntn;
-      cp_async16(sm + C::X_OFF + sw128_off(row, ch),
-                 v ? Xg + ((b * L + cn0 + t) * H + h) * R * kP + r * kP + ch * 8 : Xg, v);
     }
     cp_async_commit();
   };
@@ -269,26 +277,12 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
   for (int64_t c = c_begin; c < c_end && !aborted; ++c) {
     const int64_t c0 = c * Q;
     const int nt = (int)min((int64_t)Q, L - c0);
-    const __nv_bfloat16* Bc = Bg + ((b * L + c0) * G + g) * R * kN + 8 * kg;
-    const __nv_bfloat16* Cc = Cg + ((b * L + c0) * G + g) * R * kN + 8 * kg;
     const bool slot_live = tq < SLOTS;
 
-    // ---- this chunk's B / C straight to registers; the rest was prefetched -----
-    uint4 rb[TQ][R], rc[TQ][R];
-#pragma unroll
-    for (int u = 0; u < TQ; ++u) {
-      const int t = tq * TQ + u;
-      const bool ld = slot_live && t < nt;
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        rb[u][r] = ld ? ldg_u128(Bc + t * tokB + r * kN) : make_uint4(0, 0, 0, 0);
-        rc[u][r] = (ld && MODE == MODE_FULL) ? ldg_u128(Cc + t * tokB + r * kN) : make_uint4(0, 0, 0, 0);
-      }
-    }
-
-    // ---- gates and the chunk-local prefix sum of dt*A (warp shuffle scan) ----
     cp_async_wait_all();
-    __syncthreads();  // prefetched gates, theta and x visible to every thread
+    const bool okt = (tid == 0) ? wait_bar(s_tbar, tphase, a.status) : true;
+    if (okt) { tma_pending = false; tphase ^= 1; }  // on a timeout the phase stays for the exit wait
+    if (__syncthreads_or(!okt)) { aborted = true; break; }  // prefetched inputs visible
     const bool gate_warp = warp < (Q + 31) / 32;
     float g_dt = 0.f, g_lm = 0.f, g_av = 0.f, g_nx = 0.f;
     if (gate_warp && tid < nt) {
@@ -366,6 +360,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
 #pragma unroll
       for (int u = 0; u < TQ; ++u) {
         const int t = tq * TQ + u;
+        const bool live_t = t < nt;  // rows past the chunk end become zeros
         phi[0] += ang[u][0].x; phi[1] += ang[u][0].y;
         phi[2] += ang[u][1].x; phi[3] += ang[u][1].y;
         float cs[4], sn[4];
@@ -375,8 +370,12 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
         for (int r = 0; r < R; ++r) {
           const uint32_t off = kboff + sw128_off(t * R + r, chk);
           uint32_t ob[4], oc[4];
-          const uint32_t ib[4] = {rb[u][r].x, rb[u][r].y, rb[u][r].z, rb[u][r].w};
-          const uint32_t ic[4] = {rc[u][r].x, rc[u][r].y, rc[u][r].z, rc[u][r].w};
+          uint4 rb = *reinterpret_cast<const uint4*>(sm + C::B_OFF + off);
+          uint4 rc = make_uint4(0, 0, 0, 0);
+          if (MODE == MODE_FULL) rc = *reinterpret_cast<const uint4*>(sm + C::C_OFF + off);
+          if (!live_t) { rb = make_uint4(0, 0, 0, 0); rc = make_uint4(0, 0, 0, 0); }
+          const uint32_t ib[4] = {rb.x, rb.y, rb.z, rb.w};
+          const uint32_t ic[4] = {rc.x, rc.y, rc.z, rc.w};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             // (b0, b1) -> (c b0 + s b1, c b1 - s b0)
@@ -645,6 +644,9 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl) {
       if (cq == 0 && (n & 1) == 0) su[1 + (n >> 1)] = phi_seg;
     }
   }
+  // an aborted run may leave a prefetch in flight: let it land (bounded wait)
+  cp_async_wait_all();
+  if (tid == 0 && tma_pending) wait_bar(s_tbar, tphase, a.status);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -721,28 +723,77 @@ TcPlan make_plan(const ScanArgs& a) {
   return best;
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D map over a row-major tensor [d2][d1][d0] of `esize`-byte elements.
+bool encode3d(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* base, uint64_t d0,
+              uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2,
+              CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * esize, d0 * d1 * esize};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_maps(const ScanArgs& a, TcMaps* m) {
+  const uint64_t tok = (uint64_t)(a.batch * a.seqlen);
+  const uint32_t R = (uint32_t)a.R, Q = (uint32_t)a.Q;
+  return encode3d(&m->x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.x, kP, a.nheads * a.R, tok, 64, R,
+                  Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         encode3d(&m->b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.B, kN, a.ngroups * a.R, tok, 64,
+                  R, Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         encode3d(&m->c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.C, kN, a.ngroups * a.R, tok, 64,
+                  R, Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         encode3d(&m->th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.theta, kPairs, a.ngroups, tok,
+                  kPairs, 1, Q, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 template <int R, int Q, int MODE>
-cudaError_t launch_kernel(const ScanArgs& a, const TcPlan& pl, int64_t nblocks, cudaStream_t st) {
+cudaError_t launch_kernel(const ScanArgs& a, const TcPlan& pl, const TcMaps& maps,
+                          int64_t nblocks, cudaStream_t st) {
   using C = Cfg<R, Q>;
   auto kern = tc_scan_kernel<R, Q, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)nblocks, (unsigned)a.nheads, (unsigned)a.batch);
-  kern<<<grid, C::NTH, C::SMEM, st>>>(a, pl);
+  kern<<<grid, C::NTH, C::SMEM, st>>>(a, pl, maps);
   return cudaGetLastError();
 }
 
 template <int R, int Q>
 cudaError_t launch_rq(const ScanArgs& a, TcPlan pl, cudaStream_t st) {
+  TcMaps maps;
+  if (!make_maps(a, &maps)) return cudaErrorInvalidValue;
   if (pl.nseg > 1) {
-    cudaError_t e = launch_kernel<R, Q, MODE_STATE>(a, pl, pl.nseg - 1, st);
+    cudaError_t e = launch_kernel<R, Q, MODE_STATE>(a, pl, maps, pl.nseg - 1, st);
     if (e != cudaSuccess) return e;
     dim3 pg((kPairs * kP + 255) / 256, (unsigned)a.nheads, (unsigned)a.batch);
     tc_seg_pass_kernel<<<pg, 256, 0, st>>>(a, pl);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  return launch_kernel<R, Q, MODE_FULL>(a, pl, pl.nseg, st);
+  return launch_kernel<R, Q, MODE_FULL>(a, pl, maps, pl.nseg, st);
 }
 
 }  // namespace
@@ -750,6 +801,8 @@ cudaError_t launch_rq(const ScanArgs& a, TcPlan pl, cudaStream_t st) {
 bool tc_scan_supported(const ScanArgs& a) {
   if (!a.bf16 || a.N != kN || a.P != kP) return false;
   const int64_t m = a.Q * a.R;
+  // TMA token coordinates are 32-bit
+  if (a.batch * a.seqlen > (int64_t)0x7fffffff - a.Q) return false;
   return (a.R == 1 || a.R == 2 || a.R == 4) && (m == 64 || m == 128 || m == 256) && a.Q >= 16;
 }
 

@@ -170,6 +170,23 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// TMA: 3-D tiled bulk tensor load global -> shared (no multicast), completing
+// `bytes` of transaction count on an mbarrier.  `map` is the generic address
+// of a CUtensorMap kernel parameter.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* map, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
 // Asynchronous global -> shared copies (zero-filled when `valid` is false;
 // `gmem` must still be a valid address).
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
