@@ -14,6 +14,7 @@ Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -349,9 +350,20 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one part only (for profiling); prints its own line")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="with --only: override the workload's batch (small profiling cases)")
+    ap.add_argument("--chunk", type=int, default=None,
+                    help="with --only: override the workload's chunk length")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     s = WORKLOADS[args.workload].shape
+    if args.batch is not None or args.chunk is not None:
+        if args.only is None:
+            raise SystemExit("--batch and --chunk are for the --only profiling modes")
+        if args.batch is not None:
+            s = dataclasses.replace(s, batch=args.batch)
+        if args.chunk is not None:
+            s = dataclasses.replace(s, chunk=args.chunk)
 
     if args.impl == "reference":
         run_reference(args, s, args.workload)
@@ -365,6 +377,8 @@ def main():
 
     if args.only == "decode":
         dw = I.DECODE_MIMO if s.rank > 1 else I.DECODE_SISO
+        if args.batch is not None:
+            dw = dataclasses.replace(dw, shape=dataclasses.replace(dw.shape, batch=args.batch))
         dec = I.make_decode_inputs(dw, seed=1003, steps=args.decode_steps + args.warmup,
                                    device="cuda")
         t = time_decode(dec, dw.shape, args.decode_steps, args.warmup)

@@ -59,18 +59,16 @@ struct Cfg {
   static constexpr int P_OFF = B_OFF;           // masked scores reuse Bt + Xw
   static constexpr int G_OFF = XW_OFF + OPB;    // state, bf16 [N][128 B]
   static constexpr int SMALL_OFF = G_OFF + kN * 128;
-  // small region: per-token gates, chunk-end angles, the Q x Q decay table;
-  // the slot angle sums live in the x operand block (free until x is staged)
-  // D table [Q][Q], also the staging area of the next chunk's theta [Q][N/2]
-  static constexpr int DT_FLOATS = (Q * Q > Q * kPairs) ? Q * Q : Q * kPairs;
-  static constexpr int SMALL_BYTES = 8 * Q * 4 + 3 * kPairs * 4 + DT_FLOATS * 4 + 64;
-  // the D table / theta staging area is a TMA destination: 128-byte aligned
-  static_assert((SMALL_OFF + 8 * Q * 4 + 3 * kPairs * 4) % 128 == 0, "theta staging alignment");
-  // the w*x block holds the slot angle sums at its start and the next chunk's
-  // gates (dt[Q+1], lam[Q+1], A[Q]) in its last KB while it is otherwise free
-  static constexpr int GST_OFF = XW_OFF + OPB - 1024;
-  static_assert(SLOTS_MAX * kPairs * 4 <= OPB - 1024, "slot sums must fit in the w*x block");
-  static_assert((3 * Q + 4) * 4 <= 1024, "gate staging must fit in 1 KB");
+  // small region: the chunk's theta [Q][N/2] (a TMA destination, first so it
+  // is 1 KB aligned), per-token gamma, delta, w, Lam (log2 units) and the
+  // decay factor F, chunk-end angles with their cos / sin, the staged gates
+  // (dt[Q+1], lam[Q+1], A[Q]) and the mbarriers.  The slot angle sums live in
+  // the w*x block, free during the angle pass.
+  static constexpr int TH_FLOATS = Q * kPairs;
+  static constexpr int GST_FLOATS = 3 * Q + 4;
+  static constexpr int SMALL_BYTES = (TH_FLOATS + 5 * Q + 3 * kPairs + GST_FLOATS) * 4 + 48;
+  static_assert(SLOTS_MAX * kPairs * 4 <= OPB, "slot sums must fit in the w*x block");
+  static_assert(((TH_FLOATS + 5 * Q + 3 * kPairs + GST_FLOATS) * 4) % 8 == 0, "mbarrier alignment");
   // at least 80 KB so that no more than two CTAs (2 x 256 TMEM columns) share
   // an SM; the dynamic shared memory base is declared 1024-byte aligned
   static constexpr int SMEM_RAW = SMALL_OFF + SMALL_BYTES;
@@ -85,18 +83,26 @@ struct Cfg {
   // TMEM columns
   static constexpr int S_COL1 = 0;                  // tile 1 scores (M = 256 only)
   static constexpr int S_COL0 = (NT == 2) ? 256 : 0;
-  static constexpr int SC_COL = (NT == 2) ? 384 : 128;  // chunk state N x P
+  // One tile per chunk: scores (MT columns; the MMA2 output reuses them once
+  // masked), MMA4 output and chunk state side by side, so MMA4 can run with
+  // MMA3 before the mask.  Two tiles: the scores take 384 columns, so MMA4
+  // runs after the mask and its output reuses score columns.
+  static constexpr bool EARLY4 = NT == 1;
+  static constexpr int SC_COL = (NT == 2) ? 384 : MT + 64;  // chunk state N x P
   static constexpr int TMEM_COLS = (NT == 2) ? 512 : 256;
   __host__ __device__ static constexpr int s_col(int mt) { return mt == 0 ? S_COL0 : S_COL1; }
   __host__ __device__ static constexpr int y_col(int mt) { return 64 * mt; }
-  __host__ __device__ static constexpr int y2_col(int mt) { return 64 * (NT + mt); }
+  __host__ __device__ static constexpr int y2_col(int mt) { return NT == 2 ? 64 * (2 + mt) : MT; }
+  static_assert(SC_COL + kP <= TMEM_COLS, "TMEM columns");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 // TMA descriptors of one call: x, B, C (bf16, 128-byte swizzled boxes of
-// {64 elements, R rows, Q tokens}) and theta (fp32 boxes {N/2, 1, Q}).
+// {64 elements, R rows, Q tokens}), theta (fp32 boxes {N/2, 1, Q}) and y
+// (bf16 stores of {64, R, Q, 1} over [batch][L][H*R][P], so a chunk's rows
+// past its sequence's end are clipped).
 struct TcMaps {
-  CUtensorMap x, b, c, th;
+  CUtensorMap x, b, c, th, y;
 };
 
 struct TcPlan {
@@ -146,6 +152,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   constexpr int SLOTS = Q / TQ;                           // active rotation slots
   constexpr int CW = kP / CQN;                            // state / output columns per thread
   constexpr float kL2E = 1.4426950408889634f;
+  constexpr float kLn2 = 0.6931471805599453f;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = smem_raw;
   const uint32_t sbase = smem_u32(sm);
@@ -153,23 +160,21 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     if (threadIdx.x == 0 && a.status) atomicCAS(a.status, 0, (int)M3_ERR_CUDA);
     return;
   }
-  float* s_l2 = reinterpret_cast<float*>(sm + C::SMALL_OFF);  // chunk-local Lam_t (prefix sum)
-  float* s_gam = s_l2 + Q;
-  float* s_del = s_gam + Q;
-  float* s_w = s_del + Q;
-  float* s_dt = s_w + Q;
-  float* s_lg = s_dt + Q;                       // Lam_t * log2(e)
-  float* s_phe = s_lg + Q;                      // [kPairs] chunk-end angles
-  float* s_E = s_phe + kPairs;                  // exp(Lam_t - ref)             [Q]
-  float* s_F = s_E + Q;                         // exp(ref - Lam_s) * delta_s   [Q]
-  float2* s_pcs = reinterpret_cast<float2*>(s_F + Q);  // cos, sin of chunk-end angles [kPairs]
-  float* s_D = reinterpret_cast<float*>(s_pcs + kPairs);  // [Q][Q] decay x trapezoid weights
-  float* s_th = s_D;                            // next chunk's theta [Q][N/2] (same area)
-  float* s_gst = reinterpret_cast<float*>(sm + C::GST_OFF);  // next chunk's gates
-  float* s_part = reinterpret_cast<float*>(sm + C::XW_OFF);  // [slots][kPairs], w*x block
-  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_D + C::DT_FLOATS);  // MMA completion
-  uint64_t* s_tbar = s_bar + 1;                                         // TMA completion
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_bar + 2);
+  float* s_th = reinterpret_cast<float*>(sm + C::SMALL_OFF);  // chunk theta [Q][N/2] (TMA)
+  float* s_gam = s_th + C::TH_FLOATS;           // gamma_t = lam_t dt_t                 [Q]
+  float* s_del = s_gam + Q;                     // delta_s, trapezoid weight of token s [Q]
+  float* s_w = s_del + Q;                       // exp(Lam_end - Lam_s) delta_s         [Q]
+  float* s_lg = s_w + Q;                        // Lam_t * log2(e)                      [Q]
+  float* s_F = s_lg + Q;                        // exp(ref - Lam_s) delta_s             [Q]
+  float* s_phe = s_F + Q;                       // chunk-end angles                     [kPairs]
+  float2* s_pcs = reinterpret_cast<float2*>(s_phe + kPairs);  // their cos, sin        [kPairs]
+  float* s_gst = reinterpret_cast<float*>(s_pcs + kPairs);    // staged gates of a chunk
+  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_gst + C::GST_FLOATS);  // MMA3+MMA4, MMA2
+  uint64_t* s_bar1 = s_bar + 1;                                         // MMA1
+  uint64_t* s_tbT = s_bar + 2;                                          // TMA of theta
+  uint64_t* s_tbM = s_bar + 3;                                          // TMA of B, C, x
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_bar + 4);
+  float* s_part = s_th;  // [slots][kPairs] slot angle sums, over the consumed theta rows
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, cq = warp >> 2;
@@ -184,7 +189,9 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   }
   if (tid == 0) {
     mbar_init(s_bar, 1);
-    mbar_init(s_tbar, 1);
+    mbar_init(s_bar1, 1);
+    mbar_init(s_tbT, 1);
+    mbar_init(s_tbM, 1);
     fence_mbar_init();
   }
   tc_fence_before();
@@ -192,9 +199,9 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   tc_fence_after();
   const uint32_t tm = *s_tmem;
   const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
-  uint32_t phase = 0, tphase = 0;
+  uint32_t phase = 0, phase1 = 0, tphT = 0, tphM = 0;
   bool aborted = false;
-  bool tma_pending = false;  // thread 0: a prefetch is in flight on s_tbar
+  bool tpendT = false, tpendM = false;  // thread 0: TMA bytes expected on s_tbT / s_tbM
 
   // ---- incoming state: thread (n, cq) owns columns [CW*cq, CW*cq + CW) of row n
   const int n = 32 * qd + lane;
@@ -237,31 +244,26 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   };
   if (MODE == MODE_FULL) store_state_bf16();
 
-  float lam_seg = 0.f, phi_seg = 0.f;  // MODE_STATE summaries (pair k = n / 2)
+  float l2seg = 0.f, phi_seg = 0.f;  // MODE_STATE summaries (pair k = n / 2), log2 units
   const int64_t c_begin = seg * pl.cps;
   const int64_t c_end = min(c_begin + pl.cps, a.nchunks);
 
-  // Prefetch of a chunk's inputs while the previous chunk's epilogue and
-  // state update run: one thread issues TMA loads of raw B and C (straight
-  // into the swizzled operand tiles, rotated in place later), x (into its
-  // MMA tile) and theta (into the decay-table area); the gates go by cp.async.
-  auto prefetch = [&](int64_t cn) {
+  // Prefetch of a chunk's inputs in three steps, each as soon as its buffer is
+  // free: theta (TMA, on s_tbT) and the gates (cp.async) once the previous
+  // chunk's angle prefix has been formed; raw C once MMA1 and MMA4 are done;
+  // raw B and x once MMA2 (MODE_FULL) or MMA3 (MODE_STATE) is done.  B and C
+  // land straight in the swizzled operand tiles and are rotated in place; x
+  // lands in its MMA tile.  C, B and x complete on s_tbM, whose byte count
+  // is declared by whichever of their steps comes first.
+  constexpr uint32_t kTileBytes = Q * R * 128;  // one {64, R, Q} bf16 box
+  constexpr uint32_t kMBytes = kTileBytes * (MODE == MODE_FULL ? 5 : 3);
+  auto prefetch_early = [&](int64_t cn) {
     if (cn >= c_end) return;
     const int64_t cn0 = cn * Q;
     if (tid == 0) {
-      constexpr uint32_t kTile = Q * R * 128;  // bytes of one {64, R, Q} bf16 box
-      const uint32_t bytes = kTile * (MODE == MODE_FULL ? 5 : 3) + Q * kPairs * 4;
-      mbar_expect_tx(s_tbar, bytes);
-      tma_pending = true;
-      const int tok = (int)(b * L + cn0);
-      tma_load_3d(sm + C::X_OFF, &maps.x, 0, (int)(h * R), tok, s_tbar);
-      tma_load_3d(sm + C::B_OFF, &maps.b, 0, (int)(g * R), tok, s_tbar);
-      tma_load_3d(sm + C::B_OFF + C::OPB, &maps.b, 64, (int)(g * R), tok, s_tbar);
-      if (MODE == MODE_FULL) {
-        tma_load_3d(sm + C::C_OFF, &maps.c, 0, (int)(g * R), tok, s_tbar);
-        tma_load_3d(sm + C::C_OFF + C::OPB, &maps.c, 64, (int)(g * R), tok, s_tbar);
-      }
-      tma_load_3d(s_th, &maps.th, 0, (int)g, tok, s_tbar);
+      mbar_expect_tx(s_tbT, Q * kPairs * 4);
+      tpendT = true;
+      tma_load_3d(s_th, &maps.th, 0, (int)g, (int)(b * L + cn0), s_tbT);
     }
     for (int i = tid; i < 3 * Q + 2; i += NTH) {
       const int which = i < Q + 1 ? 0 : (i < 2 * Q + 2 ? 1 : 2);
@@ -272,17 +274,45 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     }
     cp_async_commit();
   };
-  prefetch(c_begin);
+  auto arm_m = [&]() {  // thread 0
+    if (!tpendM) {
+      mbar_expect_tx(s_tbM, kMBytes);
+      tpendM = true;
+    }
+  };
+  auto prefetch_c = [&](int64_t cn) {
+    if (MODE != MODE_FULL || cn >= c_end || tid != 0) return;
+    arm_m();
+    const int tok = (int)(b * L + cn * Q);
+    tma_load_3d(sm + C::C_OFF, &maps.c, 0, (int)(g * R), tok, s_tbM);
+    tma_load_3d(sm + C::C_OFF + C::OPB, &maps.c, 64, (int)(g * R), tok, s_tbM);
+  };
+  auto prefetch_bx = [&](int64_t cn) {
+    if (cn >= c_end || tid != 0) return;
+    arm_m();
+    const int tok = (int)(b * L + cn * Q);
+    tma_load_3d(sm + C::X_OFF, &maps.x, 0, (int)(h * R), tok, s_tbM);
+    tma_load_3d(sm + C::B_OFF, &maps.b, 0, (int)(g * R), tok, s_tbM);
+    tma_load_3d(sm + C::B_OFF + C::OPB, &maps.b, 64, (int)(g * R), tok, s_tbM);
+  };
 
-  for (int64_t c = c_begin; c < c_end && !aborted; ++c) {
-    const int64_t c0 = c * Q;
-    const int nt = (int)min((int64_t)Q, L - c0);
+  // Chunk prologue: gates, the chunk-local log-decay prefix Lam_t (log2
+  // units) and the cumulative angles.  Leaves the angle increments `ang` and
+  // the slot prefix `phi` of this thread's rotation tokens in registers,
+  // gamma, delta, Lam, w, F and the chunk-end angles in shared memory, and
+  // the chunk's total decay in `l2end`.  Needs only theta and the gates, so it
+  // runs while the chunk's B, C and x are still in flight.
+  float2 ang[TQ][2];
+  float phi[4];
+  float l2end = 0.f;
+  auto prologue = [&](int64_t cc) -> bool {
+    const int nt = (int)min((int64_t)Q, L - cc * Q);
     const bool slot_live = tq < SLOTS;
-
     cp_async_wait_all();
-    const bool okt = (tid == 0) ? wait_bar(s_tbar, tphase, a.status) : true;
-    if (okt) { tma_pending = false; tphase ^= 1; }  // on a timeout the phase stays for the exit wait
-    if (__syncthreads_or(!okt)) { aborted = true; break; }  // prefetched inputs visible
+    const bool okt = (tid == 0) ? wait_bar(s_tbT, tphT, a.status) : true;
+    if (okt && tid == 0) { tpendT = false; tphT ^= 1; }  // on a timeout the phase stays
+    if (__syncthreads_or(!okt)) return false;            // theta and gates visible
+
     const bool gate_warp = warp < (Q + 31) / 32;
     float g_dt = 0.f, g_lm = 0.f, g_av = 0.f, g_nx = 0.f;
     if (gate_warp && tid < nt) {
@@ -294,29 +324,24 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     if (gate_warp) {  // whole warps take part in the shuffle scan
       const bool inq = tid < Q;
       if (inq) {
-        s_dt[tid] = g_dt;
         s_gam[tid] = g_lm * g_dt;
         s_del[tid] = g_lm * g_dt + g_nx;
       }
-      float v = g_dt * g_av;
+      float v = g_dt * g_av * kL2E;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const float u = __shfl_up_sync(0xffffffffu, v, off);
         if (lane >= off) v += u;
       }
-      if (inq) s_l2[tid] = v;
+      if (inq) s_lg[tid] = v;
     }
-    __syncthreads();
-    if (Q > 32 && tid >= 32 && tid < Q) s_l2[tid] += s_l2[31];  // second warp of tokens
-
-    // ---- cumulative angles of pairs 4kg..4kg+3 over this slot's tokens -------
-    float2 ang[TQ][2];
+    // cumulative angles of pairs 4kg..4kg+3 over this slot's tokens
     float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int u = 0; u < TQ; ++u) {
       const int t = tq * TQ + u;
       const bool live_t = slot_live && t < nt;
-      const float d = live_t ? s_dt[t] : 0.f;
+      const float d = live_t ? s_gst[t] : 0.f;
       const float4 th = live_t ? *reinterpret_cast<const float4*>(s_th + t * kPairs + 4 * kg)
                                : make_float4(0.f, 0.f, 0.f, 0.f);
       ang[u][0] = make_float2(d * th.x, d * th.y);
@@ -324,36 +349,71 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       part[0] += ang[u][0].x; part[1] += ang[u][0].y;
       part[2] += ang[u][1].x; part[3] += ang[u][1].y;
     }
+    __syncthreads();  // theta read; first-warp Lam written
+    if (Q > 32 && tid >= 32 && tid < Q) s_lg[tid] += s_lg[31];  // second warp of tokens
+    // slot sums: row = slot, 16-byte piece kg at position kg ^ (slot % 8)
+    auto part_at = [&](int slot, int k4) { return s_part + slot * kPairs + 4 * (k4 ^ (slot & 7)); };
     if (slot_live)
-      *reinterpret_cast<float4*>(s_part + tq * kPairs + 4 * kg) =
-          make_float4(part[0], part[1], part[2], part[3]);
-    __syncthreads();  // s_l2 complete, angle partial sums written
-    float phi[4] = {0.f, 0.f, 0.f, 0.f};
-    if (slot_live) {
-      for (int q2 = 0; q2 < tq; ++q2) {
-        const float4 o = *reinterpret_cast<const float4*>(s_part + q2 * kPairs + 4 * kg);
-        phi[0] += o.x; phi[1] += o.y; phi[2] += o.z; phi[3] += o.w;
+      *reinterpret_cast<float4*>(part_at(tq, kg)) = make_float4(part[0], part[1], part[2], part[3]);
+    __syncthreads();  // Lam complete, slot sums written
+    {  // exclusive prefix over the slots: warp w scans pieces kg of 32 / SLOTS groups,
+       // lane = slot within its group; the chunk-end angles are the group totals
+      static_assert(SLOTS == NTH / 16 && SLOTS <= 32, "one scan lane per slot and piece");
+      const int sl = lane % SLOTS;
+      const int k4 = warp * (32 / SLOTS) + lane / SLOTS;
+      float* pp = part_at(sl, k4);
+      const float4 o = *reinterpret_cast<const float4*>(pp);
+      float v[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+      for (int off = 1; off < SLOTS; off <<= 1) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float u = __shfl_up_sync(0xffffffffu, v[j], off, SLOTS);
+          if (sl >= off) v[j] += u;
+        }
       }
-      if (tq == SLOTS - 1)
-        *reinterpret_cast<float4*>(s_phe + 4 * kg) =
-            make_float4(phi[0] + part[0], phi[1] + part[1], phi[2] + part[2], phi[3] + part[3]);
+      *reinterpret_cast<float4*>(pp) = make_float4(v[0] - o.x, v[1] - o.y, v[2] - o.z, v[3] - o.w);
+      if (sl == SLOTS - 1) *reinterpret_cast<float4*>(s_phe + 4 * k4) = make_float4(v[0], v[1], v[2], v[3]);
     }
-    const float lend = s_l2[nt - 1];
-    const float l2end = lend * kL2E;
-    // The decay table is built from per-token factors around the chunk's
-    // mid decay, exp(Lam_t - Lam_s) = E_t * F_s, while the chunk's total decay
-    // keeps both factors inside fp32 (|Lam_end| < 160); else entry by entry.
+    __syncthreads();  // slot prefixes and chunk-end angles written
+    if (slot_live) {
+      const float4 o = *reinterpret_cast<const float4*>(part_at(tq, kg));
+      phi[0] = o.x; phi[1] = o.y; phi[2] = o.z; phi[3] = o.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) phi[j] = 0.f;
+    }
+    l2end = s_lg[nt - 1];
+    // The mask's decay is taken from per-token factors around the chunk's mid
+    // decay, exp(Lam_t - Lam_s) = E_t * F_s, while the chunk's total decay keeps
+    // both factors inside fp32 (|Lam_end| < 160); else entry by entry.
     const float l2ref = 0.5f * l2end;
     const bool fac_ok = l2end > -230.f;
     if (tid < Q) {
-      const float lg = s_l2[tid] * kL2E;
-      s_lg[tid] = lg;
+      const float lg = s_lg[tid];
       s_w[tid] = (tid < nt) ? ex2(l2end - lg) * s_del[tid] : 0.f;
-      s_E[tid] = fac_ok ? ex2(lg - l2ref) : 0.f;
       s_F[tid] = fac_ok ? ex2(l2ref - lg) * s_del[tid] : 0.f;
     }
+    return true;
+  };
 
-    // ---- operands: Bt (and Ct) rotated by -Phi_t (16-byte row pieces) ---------
+  prefetch_early(c_begin);
+  prefetch_c(c_begin);
+  prefetch_bx(c_begin);
+  if (c_begin < c_end && !prologue(c_begin)) aborted = true;
+
+  for (int64_t c = c_begin; c < c_end && !aborted; ++c) {
+    const int64_t c0 = c * Q;
+    const int nt = (int)min((int64_t)Q, L - c0);
+    const bool slot_live = tq < SLOTS;
+    const float l2ref = 0.5f * l2end;
+    const bool fac_ok = l2end > -230.f;
+
+    const bool okm = (tid == 0) ? wait_bar(s_tbM, tphM, a.status) : true;
+    if (okm && tid == 0) { tpendM = false; tphM ^= 1; }  // on a timeout the phase stays
+    if (__syncthreads_or(!okm)) { aborted = true; break; }  // B, C and x of this chunk visible
+
+    // ---- operands: Bt (and Ct) rotated by -Phi_t in place (16-byte pieces) -----
     if (slot_live) {
       const uint32_t kboff = (uint32_t)(kg >> 3) * C::OPB;
       const uint32_t chk = (uint32_t)(kg & 7);
@@ -398,14 +458,16 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         }
       }
     }
-    __syncthreads();  // s_w ready; slot sums read, so the w*x block is free
+    if (MODE == MODE_FULL && tid == 0) bulk_wait_read0();  // the last chunk's staged y is read
+    __syncthreads();  // s_w ready; slot sums read; the w*x block is free
+    prefetch_early(c + 1);  // theta and gate buffers are free
     if (tid < kPairs) {
       float sn, cs;
       sincosf(s_phe[tid], &sn, &cs);
       s_pcs[tid] = make_float2(cs, sn);
     }
 
-    // ---- w * x (chunk-state operand) from the prefetched x tile --------------
+    // ---- w * x (chunk-state operand) from the x tile ---------------------------
     constexpr int PER = M * 8 / NTH;
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
@@ -428,8 +490,30 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     __syncthreads();
     tc_fence_after();
 
-    // ---- MMA1 (scores) and MMA3 (chunk state) ---------------------------------
+    // ---- MMA3 (chunk state) and MMA4 (Ct G), then MMA1 (scores) ----------------
+    auto issue_mma4 = [&]() {  // y2 = Ct G, one thread
+      const uint32_t id4 = idesc_bf16(MT, kP, 0, 1);
+#pragma unroll
+      for (int mt = 0; mt < NT; ++mt)
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const uint64_t ad = sw128_desc(sbase + C::C_OFF + kb * C::OPB + mt * MT * 128 + k4 * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(sbase + C::G_OFF + (kb * 4 + k4) * 2048, kN * 128, 1024);
+            mma_bf16_ss(tm + C::y2_col(mt), ad, bd, id4, (kb | k4) != 0);
+          }
+    };
     if (tid == 0) {
+      const uint32_t id3 = idesc_bf16(kN, kP, 1, 1);
+#pragma unroll
+      for (int ks = 0; ks < M / 16; ++ks) {
+        const uint64_t ad = sw128_desc(sbase + C::B_OFF + ks * 2048, C::OPB, 1024);
+        const uint64_t bd = sw128_desc(sbase + C::XW_OFF + ks * 2048, C::OPB, 1024);
+        mma_bf16_ss(tm + C::SC_COL, ad, bd, id3, ks != 0);
+      }
+      if (MODE == MODE_FULL && C::EARLY4) issue_mma4();
+      mma_commit(s_bar);
       if (MODE == MODE_FULL) {
 #pragma unroll
         for (int mt = 0; mt < NT; ++mt) {
@@ -443,154 +527,16 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
               mma_bf16_ss(tm + C::s_col(mt), ad, bd, id, (kb | k4) != 0);
             }
         }
-      }
-      const uint32_t id3 = idesc_bf16(kN, kP, 1, 1);
-#pragma unroll
-      for (int ks = 0; ks < M / 16; ++ks) {
-        const uint64_t ad = sw128_desc(sbase + C::B_OFF + ks * 2048, C::OPB, 1024);
-        const uint64_t bd = sw128_desc(sbase + C::XW_OFF + ks * 2048, C::OPB, 1024);
-        mma_bf16_ss(tm + C::SC_COL, ad, bd, id3, ks != 0);
-      }
-      mma_commit(s_bar);
-    }
-    if (MODE == MODE_FULL) {  // while MMA1/MMA3 run: D[t][s] = [s <= t] exp(Lam_t - Lam_s) w
-#pragma unroll
-      for (int e4 = tid; e4 < Q * Q / 4; e4 += NTH) {
-        const int t = (4 * e4) / Q, s0 = (4 * e4) % Q;
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
-        if (t < nt && s0 <= t) {
-          if (fac_ok) {
-            const float et = s_E[t];
-            const float4 fw = *reinterpret_cast<const float4*>(s_F + s0);
-            d[0] = et * fw.x; d[1] = et * fw.y; d[2] = et * fw.z; d[3] = et * fw.w;
-          } else {
-            const float lt = s_lg[t];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) d[j] = ex2(lt - s_lg[s0 + j]) * s_del[s0 + j];
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (s0 + j == t) d[j] = s_gam[t];
-            else if (s0 + j > t) d[j] = 0.f;
-          }
-        }
-        *reinterpret_cast<float4*>(s_D + 4 * e4) = make_float4(d[0], d[1], d[2], d[3]);
+        mma_commit(s_bar1);
       }
     }
-    const bool ok1 = (tid == 0) ? wait_bar(s_bar, phase, a.status) : true;
+    const bool ok3 = (tid == 0) ? wait_bar(s_bar, phase, a.status) : true;
     phase ^= 1;
-    if (__syncthreads_or(!ok1)) { aborted = true; break; }
+    if (__syncthreads_or(!ok3)) { aborted = true; break; }
     tc_fence_after();
-    if (MODE == MODE_STATE) prefetch(c + 1);
+    if (MODE == MODE_STATE) prefetch_bx(c + 1);  // B and x are free once MMA3 is done
 
-    if (MODE == MODE_FULL) {
-      // ---- mask the scores into P (bf16, K-major, over Bt / Xw) -------------
-#pragma unroll
-      for (int mt = 0; mt < NT; ++mt) {
-        const int rho = (MT == 64) ? 16 * qd + lane : 32 * qd + lane;  // row in the tile
-        const bool live = (MT == 64) ? lane < 16 : true;
-        const int t = (mt * MT + rho) / R;
-        const bool trow = live && t < nt;
-        const int cpt = (mt + 1) * MT / CQN;  // columns per thread
-        for (int cc = cq * cpt / 16; cc < (cq + 1) * cpt / 16; ++cc) {
-          uint32_t v[16];
-          tmem_ld16(tm + lane_base + C::s_col(mt) + cc * 16, v);
-          tmem_ld_wait();
-          if (!live) continue;
-          float mk[16 / R];
-#pragma unroll
-          for (int q4 = 0; q4 < 16 / R / 4; ++q4) {
-            float4 d4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (trow) d4 = *reinterpret_cast<const float4*>(s_D + t * Q + cc * (16 / R) + 4 * q4);
-            mk[4 * q4] = d4.x; mk[4 * q4 + 1] = d4.y; mk[4 * q4 + 2] = d4.z; mk[4 * q4 + 3] = d4.w;
-          }
-          uint32_t pk[8];
-#pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            const float2 f = fmul2(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
-                                   make_float2(mk[j / R], mk[(j + 1) / R]));
-            pk[j / 2] = pack_bf16(f.x, f.y);
-          }
-          const int kb = (cc * 16) / 64;
-          uint8_t* blk = sm + C::P_OFF + C::p_tile_off(mt) + kb * MT * 128;
-          const int ch0 = ((cc * 16) % 64) / 8;
-          *reinterpret_cast<uint4*>(blk + sw128_off(rho, ch0)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(blk + sw128_off(rho, ch0 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
-      }
-      fence_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      tc_fence_after();
-
-      // ---- MMA2 (P x) and MMA4 (Ct G) ----------------------------------------
-      if (tid == 0) {
-        const uint32_t id2 = idesc_bf16(MT, kP, 0, 1);
-#pragma unroll
-        for (int mt = 0; mt < NT; ++mt) {
-          const int kblocks = (mt + 1) * MT / 64;
-          for (int kb = 0; kb < kblocks; ++kb)
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-              const uint64_t ad = sw128_desc(
-                  sbase + C::P_OFF + C::p_tile_off(mt) + kb * MT * 128 + k4 * 32, 16, 1024);
-              const uint64_t bd = sw128_desc(sbase + C::X_OFF + (kb * 4 + k4) * 2048, C::OPB, 1024);
-              mma_bf16_ss(tm + C::y_col(mt), ad, bd, id2, (kb | k4) != 0);
-            }
-#pragma unroll
-          for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-              const uint64_t ad = sw128_desc(sbase + C::C_OFF + kb * C::OPB + mt * MT * 128 + k4 * 32, 16, 1024);
-              const uint64_t bd = sw128_desc(sbase + C::G_OFF + (kb * 4 + k4) * 2048, kN * 128, 1024);
-              mma_bf16_ss(tm + C::y2_col(mt), ad, bd, id2, (kb | k4) != 0);
-            }
-        }
-        mma_commit(s_bar);
-      }
-      const bool ok2 = (tid == 0) ? wait_bar(s_bar, phase, a.status) : true;
-      phase ^= 1;
-      if (__syncthreads_or(!ok2)) { aborted = true; break; }
-      tc_fence_after();
-      prefetch(c + 1);  // x, theta and gate buffers are free from here on
-
-      // ---- epilogue: y = P x + exp(Lam_t) Ct G ---------------------------------
-#pragma unroll
-      for (int mt = 0; mt < NT; ++mt) {
-        const int rho = (MT == 64) ? 16 * qd + lane : 32 * qd + lane;
-        const bool live = (MT == 64) ? lane < 16 : true;
-        const int i = mt * MT + rho;
-        const int t = i / R, r = i % R;
-        const bool out = live && t < nt;
-#pragma unroll
-        for (int pc = 0; pc < CW / 16; ++pc) {
-          uint32_t yv[16], zv[16];
-          tmem_ld16(tm + lane_base + C::y_col(mt) + CW * cq + 16 * pc, yv);
-          tmem_ld16(tm + lane_base + C::y2_col(mt) + CW * cq + 16 * pc, zv);
-          tmem_ld_wait();
-          if (out) {
-            const float el = ex2(s_lg[t]);
-            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.y) +
-                                 ((b * L + c0 + t) * H + h) * R * kP + r * kP + CW * cq + 16 * pc;
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              uint32_t w4[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int j = q * 8 + 2 * e;
-                const float2 f = ffma2(make_float2(el, el),
-                                       make_float2(__uint_as_float(zv[j]), __uint_as_float(zv[j + 1])),
-                                       make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1])));
-                w4[e] = pack_bf16(f.x, f.y);
-              }
-              *reinterpret_cast<uint4*>(dst + q * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-            }
-          }
-        }
-      }
-    }
-
-    // ---- state update: G <- Rot(Phi_end) (exp(Lam_end) G + Sc) ---------------
+    // ---- state update G <- Rot(Phi_end) (exp(Lam_end) G + Sc), under MMA1 -------
     {
       const float phe = s_phe[n >> 1];
       const float2 pcs = s_pcs[n >> 1];
@@ -615,14 +561,167 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         }
       }
       if (MODE == MODE_STATE) {
-        lam_seg += lend;
+        l2seg += l2end;
         phi_seg += phe;
       }
     }
-    if (MODE == MODE_FULL) store_state_bf16();
+
+    if (MODE == MODE_FULL) {
+      if (C::EARLY4) store_state_bf16();  // MMA4 has read the previous state
+      const bool ok1 = (tid == 0) ? wait_bar(s_bar1, phase1, a.status) : true;
+      phase1 ^= 1;
+      if (__syncthreads_or(!ok1)) { aborted = true; break; }
+      tc_fence_after();
+      if (C::EARLY4) prefetch_c(c + 1);  // MMA1 and MMA4 have read Ct
+
+      // ---- mask the scores into P (bf16, K-major, over Bt / Xw) -------------
+      //   P[(t,r),(s,r')] = S * (s < t ? exp(Lam_t - Lam_s) delta_s : s == t ? gamma_t : 0)
+#pragma unroll
+      for (int mt = 0; mt < NT; ++mt) {
+        const int rho0 = (MT == 64) ? 16 * qd : 32 * qd;     // the warp's first row
+        const int rho = rho0 + lane;
+        const bool live = (MT == 64) ? lane < 16 : true;
+        const int t = live ? (mt * MT + rho) / R : 0;
+        const bool trow = live && t < nt;
+        const int t_hi = (mt * MT + rho0 + ((MT == 64) ? 15 : 31)) / R;  // the warp's last token
+        const float lgt = trow ? s_lg[t] : 0.f;
+        const float et = (trow && fac_ok) ? ex2(lgt - l2ref) : 0.f;
+        const float gmt = trow ? s_gam[t] : 0.f;
+        const int cpt = (mt + 1) * MT / CQN;  // columns per thread, a multiple of 32
+        static_assert((MT / CQN) % 32 == 0, "mask columns per thread");
+        // 16 masked columns (16 / R tokens from s0) of v, packed to bf16
+        auto mask16 = [&](const uint32_t* v, int s0, uint32_t* pk) {
+          float mk[16 / R];
+#pragma unroll
+          for (int q4 = 0; q4 < 16 / R / 4; ++q4) {
+            const int sb = s0 + 4 * q4;
+            float f[4];
+            if (fac_ok) {
+              const float4 fw = *reinterpret_cast<const float4*>(s_F + sb);
+              f[0] = et * fw.x; f[1] = et * fw.y; f[2] = et * fw.z; f[3] = et * fw.w;
+            } else {
+              const float4 l4 = *reinterpret_cast<const float4*>(s_lg + sb);
+              const float4 d4 = *reinterpret_cast<const float4*>(s_del + sb);
+              f[0] = ex2(lgt - l4.x) * d4.x; f[1] = ex2(lgt - l4.y) * d4.y;
+              f[2] = ex2(lgt - l4.z) * d4.z; f[3] = ex2(lgt - l4.w) * d4.w;
+            }
+            if (sb + 3 < t) {  // wholly below the diagonal
+#pragma unroll
+              for (int e = 0; e < 4; ++e) mk[4 * q4 + e] = f[e];
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                mk[4 * q4 + e] = sb + e < t ? f[e] : (sb + e == t ? gmt : 0.f);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 16; j += 2) {
+            const float2 fm = fmul2(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
+                                    make_float2(mk[j / R], mk[(j + 1) / R]));
+            pk[j / 2] = pack_bf16(fm.x, fm.y);
+          }
+        };
+        for (int cc = cq * cpt / 16; cc < (cq + 1) * cpt / 16; cc += 2) {
+          const int s0 = cc * 16 / R;  // first token of these 32 columns
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) pk[j] = 0u;
+          if (s0 <= t_hi) {  // warp-uniform: blocks wholly above the diagonal stay zero
+            uint32_t v[32];
+            tmem_ld32(tm + lane_base + C::s_col(mt) + cc * 16, v);
+            tmem_ld_wait();
+            if (trow) {
+              mask16(v, s0, pk);
+              mask16(v + 16, s0 + 16 / R, pk + 8);
+            }
+          }
+          if (live) {
+            const int kb = (cc * 16) / 64;
+            uint8_t* blk = sm + C::P_OFF + C::p_tile_off(mt) + kb * MT * 128;
+            const int ch0 = ((cc * 16) % 64) / 8;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<uint4*>(blk + sw128_off(rho, ch0 + q)) =
+                  make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+
+      // ---- MMA2 (P x) ----------------------------------------------------------
+      if (tid == 0) {
+        const uint32_t id2 = idesc_bf16(MT, kP, 0, 1);
+#pragma unroll
+        for (int mt = 0; mt < NT; ++mt) {
+          const int kblocks = (mt + 1) * MT / 64;
+          for (int kb = 0; kb < kblocks; ++kb)
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const uint64_t ad = sw128_desc(
+                  sbase + C::P_OFF + C::p_tile_off(mt) + kb * MT * 128 + k4 * 32, 16, 1024);
+              const uint64_t bd = sw128_desc(sbase + C::X_OFF + (kb * 4 + k4) * 2048, C::OPB, 1024);
+              mma_bf16_ss(tm + C::y_col(mt), ad, bd, id2, (kb | k4) != 0);
+            }
+        }
+        if (!C::EARLY4) issue_mma4();
+        mma_commit(s_bar);
+      }
+      const bool ok2 = (tid == 0) ? wait_bar(s_bar, phase, a.status) : true;
+      phase ^= 1;
+      if (__syncthreads_or(!ok2)) { aborted = true; break; }
+      tc_fence_after();
+      prefetch_bx(c + 1);  // MMA2 has read P (over Bt) and x
+      if (!C::EARLY4) {    // MMA4 has read Ct and the previous state
+        prefetch_c(c + 1);
+        store_state_bf16();
+      }
+
+      // ---- epilogue: y = P x + exp(Lam_t) Ct G, staged in the w*x block --------
+#pragma unroll
+      for (int mt = 0; mt < NT; ++mt) {
+        const int rho = (MT == 64) ? 16 * qd + lane : 32 * qd + lane;
+        const bool live = (MT == 64) ? lane < 16 : true;
+        const int i = mt * MT + rho;  // row (t, r) of the chunk
+        const int t = live ? i / R : 0;
+        const float el = (live && t < nt) ? ex2(s_lg[t]) : 0.f;
+#pragma unroll
+        for (int pc = 0; pc < CW / 16; ++pc) {
+          uint32_t yv[16], zv[16];
+          tmem_ld16(tm + lane_base + C::y_col(mt) + CW * cq + 16 * pc, yv);
+          tmem_ld16(tm + lane_base + C::y2_col(mt) + CW * cq + 16 * pc, zv);
+          tmem_ld_wait();
+          if (live) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              uint32_t w4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int j = q * 8 + 2 * e;
+                const float2 f = ffma2(make_float2(el, el),
+                                       make_float2(__uint_as_float(zv[j]), __uint_as_float(zv[j + 1])),
+                                       make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1])));
+                w4[e] = pack_bf16(f.x, f.y);
+              }
+              *reinterpret_cast<uint4*>(sm + C::XW_OFF + sw128_off(i, (CW * cq + 16 * pc) / 8 + q)) =
+                  make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+          }
+        }
+      }
+      fence_async_smem();  // staged y visible to the bulk store
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (MODE == MODE_FULL && tid == 0) {  // y of this chunk: one bulk tensor store
+      tma_store_4d(&maps.y, sm + C::XW_OFF, 0, (int)(h * R), (int)c0, (int)b);
+      bulk_commit();
+    }
+    // the next chunk's gates and angles overlap its B, C, x loads
+    if (c + 1 < c_end && !prologue(c + 1)) { aborted = true; break; }
   }
 
   if (!aborted) {
@@ -640,13 +739,15 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       for (int p = 0; p < CW; p += 4)
         *reinterpret_cast<float4*>(dst + p) = make_float4(gst[p], gst[p + 1], gst[p + 2], gst[p + 3]);
       float* su = pl.wsSum + slot * (1 + kPairs);
-      if (tid == 0) su[0] = lam_seg;
+      if (tid == 0) su[0] = l2seg * kLn2;
       if (cq == 0 && (n & 1) == 0) su[1 + (n >> 1)] = phi_seg;
     }
   }
   // an aborted run may leave a prefetch in flight: let it land (bounded wait)
   cp_async_wait_all();
-  if (tid == 0 && tma_pending) wait_bar(s_tbar, tphase, a.status);
+  if (tid == 0 && tpendT) wait_bar(s_tbT, tphT, a.status);
+  if (tid == 0 && tpendM) wait_bar(s_tbM, tphM, a.status);
+  if (MODE == MODE_FULL && tid == 0) bulk_wait0();  // y stores complete
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -741,24 +842,40 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D map over a row-major tensor [d2][d1][d0] of `esize`-byte elements.
+// Map over a row-major tensor of `rank` (<= 4) dimensions, dims[0] innermost,
+// of `esize`-byte elements.
+bool encode_nd(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* base, int rank,
+               const uint64_t* d, const uint32_t* bx, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4], estr[4];
+  uint64_t st = esize;
+  for (int i = 0; i < rank; ++i) {
+    dims[i] = d[i];
+    box[i] = bx[i];
+    estr[i] = 1;
+    if (i > 0) strides[i - 1] = st;
+    st *= d[i];
+  }
+  return fn(m, dt, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode3d(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* base, uint64_t d0,
               uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2,
               CUtensorMapSwizzle sw) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {d0, d1, d2};
-  const cuuint64_t strides[2] = {d0 * esize, d0 * d1 * esize};
-  const cuuint32_t box[3] = {b0, b1, b2};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const uint64_t d[3] = {d0, d1, d2};
+  const uint32_t bx[3] = {b0, b1, b2};
+  return encode_nd(m, dt, esize, base, 3, d, bx, sw);
 }
 
 bool make_maps(const ScanArgs& a, TcMaps* m) {
   const uint64_t tok = (uint64_t)(a.batch * a.seqlen);
   const uint32_t R = (uint32_t)a.R, Q = (uint32_t)a.Q;
+  const uint64_t yd[4] = {kP, (uint64_t)(a.nheads * a.R), (uint64_t)a.seqlen, (uint64_t)a.batch};
+  const uint32_t yb[4] = {64, R, Q, 1};
   return encode3d(&m->x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.x, kP, a.nheads * a.R, tok, 64, R,
                   Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
          encode3d(&m->b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.B, kN, a.ngroups * a.R, tok, 64,
@@ -766,7 +883,9 @@ bool make_maps(const ScanArgs& a, TcMaps* m) {
          encode3d(&m->c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.C, kN, a.ngroups * a.R, tok, 64,
                   R, Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
          encode3d(&m->th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.theta, kPairs, a.ngroups, tok,
-                  kPairs, 1, Q, CU_TENSOR_MAP_SWIZZLE_NONE);
+                  kPairs, 1, Q, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+         encode_nd(&m->y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.y, 4, yd, yb,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 template <int R, int Q, int MODE>
