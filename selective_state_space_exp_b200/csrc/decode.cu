@@ -9,205 +9,352 @@
 // the rank-R MIMO update (section 2.3).  The step is HBM-bound (section 3.3:
 // decode is limited by state IO, not FLOPs): 2 * 4 * N * P bytes per head.
 //
-// Layout: one CTA of 128 threads per (b, h) (whole state rows).
-// Thread (kslot, pv) owns float4 column pv of the block and the pairs
-// k = kslot, kslot + nslots, ...; a block row is read by consecutive threads
-// as float4 (a contiguous 128-byte segment per row).  The per-head operands
-// (B, C, B_prev, x, x_prev, the cos/sin table) are staged in shared memory;
-// y is reduced over kslots through shared memory.
+// Layout: CTAs of 256 threads, two or more per SM, each walking a contiguous
+// range of heads (so consecutive heads mostly share one (batch, group) and
+// its B, C, B_prev are converted once).  A head's state and its operands
+// arrive in shared memory by bulk async copies issued one head ahead into a
+// second buffer, so the state stream never waits on the arithmetic; h'
+// leaves by streaming 16-byte stores.
+// Thread (kslot, pv) owns float4 column pv of the state and the pairs
+// k = kslot, kslot + nslots, ...; y is reduced over kslots with warp
+// shuffles and then across warps through shared memory.
 #include "m3_internal.cuh"
 #include "tc_ptx.cuh"
 
 namespace m3 {
 namespace {
 
-constexpr int kMaxCols = 128;  // state columns per CTA (whole rows: P <= 128)
-constexpr int kPairsInFlight = 4;  // pairs whose state rows are loaded before any is computed
+using namespace tc;
 
-// CTA (b, h, column block): columns [cb*CB, cb*CB + CB) of the head's state
-// and of y (columns are independent: y[r][p] only reads column p of h').
-// Whole rows per CTA (CB = P) read best: splitting a 256-byte state row
-// between CTAs that run at different times costs HBM locality.
-// Resident CTAs per SM the register budget is sized for (more state bytes in
-// flight for small R, room for the rank-R operands for large R).
-// 128 threads per CTA; the register budget is sized for the resident CTAs
-// per SM (more state bytes in flight for small R, room for the rank-R
-// operands for large R).
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr unsigned long long kDecodeWaitNs = 2000000000ull;  // bounded mbarrier wait (2 s)
+
+__device__ __forceinline__ unsigned long long decode_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// One thread polls; false (and the status word set) after the time limit.
+__device__ bool decode_wait(uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = decode_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (decode_ns() - t0 > kDecodeWaitNs) {
+      if (status) atomicCAS(status, 0, (int)M3_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Bulk async copy global -> shared of `bytes` (a multiple of 16, both
+// addresses 16-byte aligned), completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* smem, const void* gmem, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem)),
+      "l"(gmem), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory plan of one CTA (byte offsets, all 128-byte aligned): the
+// state and raw operands of two heads (or one, for the largest shapes), the
+// fp32 B / C / B_prev of the current (batch, group), the per-head rotation
+// and x factors, and the per-warp partial sums of y.
+struct DecodeSmem {
+  int64_t st_bytes, ops_bytes;
+  int64_t st_off[2], ops_off[2], bc_off, head_off, red_off, bar_off, total;
+  int nbuf;  // 2: the next head streams in during this one; 1: the largest shapes
+};
+constexpr int64_t kMaxSmem = 232448;  // dynamic shared memory of one CTA
+
+__host__ __device__ inline DecodeSmem decode_smem(int64_t N, int64_t P, int64_t R, bool bf16) {
+  DecodeSmem m;
+  const int64_t es = bf16 ? 2 : 4;
+  const int64_t K = N / 2;
+  m.st_bytes = N * P * 4;
+  m.ops_bytes = (3 * R * N + 2 * R * P) * es + K * 4;  // B, C, B_prev, x, x_prev, theta
+  const int64_t bc = align_up(3 * R * N * 8, 128);            // [3][n][R] float pairs
+  const int64_t head = align_up((6 * K + 2 * R * P) * 4, 128);  // rot, sin pairs, xe, xg
+  const int64_t red = align_up(kWarps * R * P * 4, 128);
+  const int64_t buf = align_up(m.st_bytes, 128) + align_up(m.ops_bytes, 128);
+  m.nbuf = 2 * buf + bc + head + red + 16 <= kMaxSmem ? 2 : 1;
+  int64_t o = 0;
+  for (int i = 0; i < 2; ++i) {
+    m.st_off[i] = i < m.nbuf ? o : m.st_off[0];
+    if (i < m.nbuf) o += align_up(m.st_bytes, 128);
+  }
+  for (int i = 0; i < 2; ++i) {
+    m.ops_off[i] = i < m.nbuf ? o : m.ops_off[0];
+    if (i < m.nbuf) o += align_up(m.ops_bytes, 128);
+  }
+  m.bc_off = o; o += bc;
+  m.head_off = o; o += head;
+  m.red_off = o; o += red;
+  m.bar_off = o; o += 16;
+  m.total = o;
+  return m;
+}
+
+// CTAs per SM the register budget is sized for (three for R = 1: its shared
+// memory allows three)
 template <int R>
-struct DecodeCfg {
-  static constexpr int threads = 128;
-  static constexpr int occupancy = R == 1 ? 7 : (R == 2 ? 5 : (R == 4 ? 4 : 3));
+struct DecodeOcc {
+  static constexpr int value = R == 1 ? 3 : (R <= 4 ? 2 : 1);
 };
 
-template <int R>
-__global__ void __launch_bounds__(DecodeCfg<R>::threads, DecodeCfg<R>::occupancy)
-decode_kernel(const DecodeArgs a) {
-  constexpr int kDecodeThreads = DecodeCfg<R>::threads;
-  const int P = (int)a.P, N = (int)a.N, K = N / 2;
-  const int CB = P < kMaxCols ? P : kMaxCols;
-  const int nblk = P / CB;
-  const int64_t bh = blockIdx.x / nblk;
-  const int cb = blockIdx.x % nblk;
-  const int64_t h = bh % a.nheads, b = bh / a.nheads;
-  const int64_t g = h / (a.nheads / a.ngroups);
-  const int64_t bg = b * a.ngroups + g;
-  const int tid = threadIdx.x;
+// NC, PC: compile-time N and P (0: taken from the arguments), so that the
+// common state shape gets a fully unrolled pair loop.
+template <int R, int NC, int PC>
+__global__ void __launch_bounds__(kThreads, DecodeOcc<R>::value) decode_kernel(const DecodeArgs a) {
+  const int P = PC ? PC : (int)a.P, N = NC ? NC : (int)a.N, K = N / 2;
+  const int lgN = __ffs(N) - 1;  // N and P are powers of two
+  const int64_t H = a.nheads, G = a.ngroups, total = a.batch * H;
+  const int64_t es = a.bf16 ? 2 : 4;
+  const DecodeSmem sp = decode_smem(N, P, R, a.bf16);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  extern __shared__ float sm[];
-  float* s_ac = sm;               // alpha cos(dt theta_k)          [K]
-  float* s_as = s_ac + K;         // alpha sin(dt theta_k)          [K]
-  float* s_Bp = s_as + K;         // B_prev, transposed             [N][R]
-  float* s_Bt = s_Bp + R * N;     // B_t, transposed                [N][R]
-  float* s_Ct = s_Bt + R * N;     // C_t, transposed                [N][R]
-  float* s_xe = s_Ct + R * N;     // (1-lam) dt x_prev              [R][CB]
-  float* s_xg = s_xe + R * CB;    // lam dt x_t                     [R][CB]
-  float* s_red = s_xg + R * CB;   // partial y per kslot            [nslots][R][CB]
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + sp.bar_off);
+  // packed fp32x2 operands are staged with both halves equal, so the pair
+  // loop feeds them to the f32x2 FMAs as loaded
+  float2* s_Bp = reinterpret_cast<float2*>(sm + sp.bc_off);  // B_prev, [n][R] pairs
+  float2* s_Bt = s_Bp + R * N;                                // B_t,    [n][R] pairs
+  float2* s_Ct = s_Bt + R * N;                                // C_t,    [n][R] pairs
+  float4* s_rot = reinterpret_cast<float4*>(sm + sp.head_off);  // (a cos, a cos, -a sin, -a sin)
+  float2* s_as = reinterpret_cast<float2*>(s_rot + K);          // (a sin, a sin)      [K]
+  float* s_xe = reinterpret_cast<float*>(s_as + K);  // (1-lam) dt x_prev              [R][P]
+  float* s_xg = s_xe + R * P;                        // lam dt x_t                     [R][P]
+  float* s_red = reinterpret_cast<float*>(sm + sp.red_off);  // partial y [warps][R][P]
 
-  const float dt = a.dt[bh], lamv = a.lam[bh];
-  const float alpha = expf(dt * a.A[bh]);
-  const float gamma = lamv * dt, eps = (1.f - lamv) * dt;
   const bool prev = a.B_prev != nullptr;
+  const uint32_t opsB = (uint32_t)(R * N * es), opsX = (uint32_t)(R * P * es);
+  // bytes of one head: state, x (and x_prev), theta, plus B, C (and B_prev)
+  // whenever its (batch, group) differs from the previous head's
+  const uint32_t bytes_head = (uint32_t)sp.st_bytes + (prev ? 2 : 1) * opsX + (uint32_t)(K * 4);
+  const uint32_t bytes_bc = (prev ? 3 : 2) * opsB;
 
-  const int PV = CB / 4;  // float4 columns per state row in this block
-  const int nslots = kDecodeThreads / PV;
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int hpg = (int)(H / G);  // heads per group
+  // thread 0: bring head hd's state and operands into buffer bi
+  auto issue = [&](int64_t hd, int64_t bg, int bi, bool with_bc) {
+    uint8_t* st = sm + sp.st_off[bi];
+    uint8_t* ops = sm + sp.ops_off[bi];
+    fence_async_smem();
+    mbar_expect_tx(&bars[bi], bytes_head + (with_bc ? bytes_bc : 0u));
+    bulk_load(st, a.state_in + hd * (int64_t)N * P, (uint32_t)sp.st_bytes, &bars[bi]);
+    if (with_bc) {
+      bulk_load(ops, static_cast<const char*>(a.B) + bg * opsB, opsB, &bars[bi]);
+      bulk_load(ops + opsB, static_cast<const char*>(a.C) + bg * opsB, opsB, &bars[bi]);
+      if (prev) bulk_load(ops + 2 * opsB, static_cast<const char*>(a.B_prev) + bg * opsB, opsB, &bars[bi]);
+    }
+    bulk_load(ops + 3 * opsB, static_cast<const char*>(a.x) + hd * opsX, opsX, &bars[bi]);
+    if (prev) bulk_load(ops + 3 * opsB + opsX, static_cast<const char*>(a.x_prev) + hd * opsX, opsX, &bars[bi]);
+    bulk_load(ops + 3 * opsB + 2 * opsX, a.theta + bg * K, (uint32_t)(K * 4), &bars[bi]);
+  };
+
+  const int PV = P / 4;                     // float4 columns of a state row
+  const int nslots = kThreads / PV;
   const int pv = tid % PV, kslot = tid / PV;
   const int p0 = pv * 4;
-  const float4* src = reinterpret_cast<const float4*>(a.state_in + bh * (int64_t)N * P + cb * CB);
-  float4* dst = reinterpret_cast<float4*>(a.state_out + bh * (int64_t)N * P + cb * CB);
-  const int rowq = P / 4;  // float4 stride between state rows
+  const int rowq = P / 4;
 
-  // Issue the first pairs' state loads before staging the per-head operands.
-  float4 r0[kPairsInFlight], r1[kPairsInFlight];
-#pragma unroll
-  for (int u = 0; u < kPairsInFlight; ++u) {
-    const int k = kslot + u * nslots;
-    if (k < K) {
-      r0[u] = __ldcs(src + (2 * k) * rowq + pv);
-      r1[u] = __ldcs(src + (2 * k + 1) * rowq + pv);
+  // this CTA's heads: a contiguous range, so consecutive heads share B and C
+  const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+  const int64_t h_begin = (int64_t)blockIdx.x * per;
+  const int64_t h_end = min(total, h_begin + per);
+  int64_t hd = h_begin;
+  int64_t bg = (h_begin / H) * G + (int)(h_begin % H) / hpg;  // (batch, group) of head hd
+  int hh = (int)(h_begin % H);                                   // head index within the batch
+  if (tid == 0 && hd < h_end) issue(hd, bg, 0, true);
+  // per-head scalars of the current head, loaded one head ahead
+  float dt = 0.f, Av = 0.f, lamv = 0.f;
+  if (hd < h_end) { dt = a.dt[hd]; Av = a.A[hd]; lamv = a.lam[hd]; }
+  uint32_t pending = hd < h_end ? 1u : 0u;  // thread 0: bit i = bytes expected on bars[i]
+  uint32_t ph = 0u;                          // bit i = phase parity of bars[i]
+  bool aborted = false;
+
+  for (int j = 0; hd < h_end; ++hd, ++j) {
+    const int bi = sp.nbuf == 2 ? (j & 1) : 0;
+    const int64_t nhd = hd + 1;
+    const bool new_bc = hd == h_begin || hh % hpg == 0;  // first head of its (batch, group)
+    const int nh = hh + 1 == H ? 0 : hh + 1;             // the next head's index and group
+    const int64_t nbg = nh == 0 ? bg + 1 : (nh % hpg == 0 ? bg + 1 : bg);
+    if (sp.nbuf == 2 && tid == 0 && nhd < h_end) {  // buffer bi ^ 1 was released by the last head
+      issue(nhd, nbg, bi ^ 1, nbg != bg);
+      pending |= 1u << (bi ^ 1);
     }
-  }
+    float ndt = 0.f, nA = 0.f, nlam = 0.f;
+    if (nhd < h_end) { ndt = a.dt[nhd]; nA = a.A[nhd]; nlam = a.lam[nhd]; }
 
-  for (int k = tid; k < K; k += kDecodeThreads) {
-    float sn, cs;
-    sincosf(dt * a.theta[bg * K + k], &sn, &cs);
-    s_ac[k] = alpha * cs;
-    s_as[k] = alpha * sn;
-  }
-  for (int i = tid; i < R * N; i += kDecodeThreads) {  // i = r * N + n -> [n][r]
-    const int r = i / N, nn = i % N, ti = nn * R + r;
-    s_Bt[ti] = io_load(a.B, bg * R * N + i, a.bf16);
-    s_Ct[ti] = io_load(a.C, bg * R * N + i, a.bf16);
-    s_Bp[ti] = prev ? io_load(a.B_prev, bg * R * N + i, a.bf16) : 0.f;
-  }
-  for (int i = tid; i < R * CB; i += kDecodeThreads) {
-    const int r = i / CB, c = i % CB;
-    const int64_t xi = bh * R * P + r * P + cb * CB + c;
-    s_xg[i] = gamma * io_load(a.x, xi, a.bf16);
-    s_xe[i] = prev ? eps * io_load(a.x_prev, xi, a.bf16) : 0.f;
-  }
-  __syncthreads();
-
-  // column pairs (p0, p0+1) and (p0+2, p0+3) as packed fp32x2 operands
-  float2 xg[R][2], xe[R][2], yacc[R][2];
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      xg[r][j] = make_float2(s_xg[r * CB + p0 + 2 * j], s_xg[r * CB + p0 + 2 * j + 1]);
-      xe[r][j] = make_float2(s_xe[r * CB + p0 + 2 * j], s_xe[r * CB + p0 + 2 * j + 1]);
-      yacc[r][j] = make_float2(0.f, 0.f);
+    const bool ok = (tid == 0) ? decode_wait(&bars[bi], (ph >> bi) & 1u, a.status) : true;
+    if (tid == 0 && ok) {  // on a timeout the phase stays for the exit wait
+      pending &= ~(1u << bi);
+      ph ^= 1u << bi;
     }
+    if (__syncthreads_or(!ok)) { aborted = true; break; }
 
-  for (int kb = kslot; kb < K; kb += kPairsInFlight * nslots) {
-    if (kb != kslot) {
-#pragma unroll
-      for (int u = 0; u < kPairsInFlight; ++u) {
-        const int k = kb + u * nslots;
-        if (k < K) {
-          r0[u] = __ldcs(src + (2 * k) * rowq + pv);
-          r1[u] = __ldcs(src + (2 * k + 1) * rowq + pv);
-        }
+    const float alpha = expf(dt * Av);
+    const float gamma = lamv * dt, eps = (1.f - lamv) * dt;
+    const uint8_t* ops = sm + sp.ops_off[bi];
+    const void* ox = ops + 3 * opsB;
+    const void* oxp = ops + 3 * opsB + opsX;
+    const float* oth = reinterpret_cast<const float*>(ops + 3 * opsB + 2 * opsX);
+    if (new_bc) {  // fp32 pairs of B, C, B_prev of this (batch, group), [n][r] order
+      for (int i = tid; i < R * N; i += kThreads) {
+        const int nn = i / R, r = i % R, si = (r << lgN) + nn;
+        const float vb = io_load(ops, si, a.bf16), vc = io_load(ops + opsB, si, a.bf16);
+        const float vp = prev ? io_load(ops + 2 * opsB, si, a.bf16) : 0.f;
+        s_Bt[i] = make_float2(vb, vb);
+        s_Ct[i] = make_float2(vc, vc);
+        s_Bp[i] = make_float2(vp, vp);
       }
     }
-#pragma unroll
-    for (int u = 0; u < kPairsInFlight; ++u) {
-      const int k = kb + u * nslots;
-      if (k < K) {
-        const float ac = s_ac[k], as = s_as[k];
-        float bp0[R], bp1[R], bt0[R], bt1[R], c0[R], c1[R];
-#pragma unroll
-        for (int r = 0; r < R; ++r) {  // rows 2k and 2k+1 are adjacent R-vectors
-          bp0[r] = s_Bp[(2 * k) * R + r]; bp1[r] = s_Bp[(2 * k + 1) * R + r];
-          bt0[r] = s_Bt[(2 * k) * R + r]; bt1[r] = s_Bt[(2 * k + 1) * R + r];
-          c0[r] = s_Ct[(2 * k) * R + r]; c1[r] = s_Ct[(2 * k + 1) * R + r];
-        }
-        const float2 in0[2] = {make_float2(r0[u].x, r0[u].y), make_float2(r0[u].z, r0[u].w)};
-        const float2 in1[2] = {make_float2(r1[u].x, r1[u].y), make_float2(r1[u].z, r1[u].w)};
-        float o0[4], o1[4];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          float2 g0 = in0[j], g1 = in1[j], u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int r = 0; r < R; ++r) {
-            g0 = tc::ffma2(make_float2(bp0[r], bp0[r]), xe[r][j], g0);
-            g1 = tc::ffma2(make_float2(bp1[r], bp1[r]), xe[r][j], g1);
-            u0 = tc::ffma2(make_float2(bt0[r], bt0[r]), xg[r][j], u0);
-            u1 = tc::ffma2(make_float2(bt1[r], bt1[r]), xg[r][j], u1);
-          }
-          // (h'_{2k}, h'_{2k+1}) = alpha Rot(phi) (g_{2k}, g_{2k+1}) + (u_{2k}, u_{2k+1})
-          const float2 w0 = tc::ffma2(make_float2(ac, ac), g0,
-                                      tc::ffma2(make_float2(-as, -as), g1, u0));
-          const float2 w1 = tc::ffma2(make_float2(as, as), g0,
-                                      tc::ffma2(make_float2(ac, ac), g1, u1));
-#pragma unroll
-          for (int r = 0; r < R; ++r)
-            yacc[r][j] = tc::ffma2(make_float2(c0[r], c0[r]), w0,
-                                   tc::ffma2(make_float2(c1[r], c1[r]), w1, yacc[r][j]));
-          o0[2 * j] = w0.x; o0[2 * j + 1] = w0.y;
-          o1[2 * j] = w1.x; o1[2 * j + 1] = w1.y;
-        }
-        __stcs(dst + (2 * k) * rowq + pv, make_float4(o0[0], o0[1], o0[2], o0[3]));
-        __stcs(dst + (2 * k + 1) * rowq + pv, make_float4(o1[0], o1[1], o1[2], o1[3]));
-      }
+    for (int k = tid; k < K; k += kThreads) {
+      float sn, cs;
+      sincosf(dt * oth[k], &sn, &cs);
+      s_rot[k] = make_float4(alpha * cs, alpha * cs, -alpha * sn, -alpha * sn);
+      s_as[k] = make_float2(alpha * sn, alpha * sn);
     }
+    for (int i = tid; i < R * P; i += kThreads) {
+      s_xg[i] = gamma * io_load(ox, i, a.bf16);
+      s_xe[i] = prev ? eps * io_load(oxp, i, a.bf16) : 0.f;
+    }
+    __syncthreads();
+
+    // column pairs (p0, p0+1) and (p0+2, p0+3) as packed fp32x2 operands
+    float2 xg[R][2], xe[R][2], yacc[R][2];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        xg[r][jj] = make_float2(s_xg[r * P + p0 + 2 * jj], s_xg[r * P + p0 + 2 * jj + 1]);
+        xe[r][jj] = make_float2(s_xe[r * P + p0 + 2 * jj], s_xe[r * P + p0 + 2 * jj + 1]);
+        yacc[r][jj] = make_float2(0.f, 0.f);
+      }
+
+    const float4* src = reinterpret_cast<const float4*>(sm + sp.st_off[bi]);
+    float4* dst = reinterpret_cast<float4*>(a.state_out + hd * (int64_t)N * P);
+#pragma unroll
+    for (int k = kslot; k < K; k += nslots) {
+      const float4 r0 = src[(2 * k) * rowq + pv];
+      const float4 r1 = src[(2 * k + 1) * rowq + pv];
+      const float4 rot = s_rot[k];
+      const float2 AC = make_float2(rot.x, rot.y), NAS = make_float2(rot.z, rot.w);
+      const float2 AS = s_as[k];
+      float2 bp0[R], bp1[R], bt0[R], bt1[R], c0[R], c1[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {  // rows 2k and 2k+1 are adjacent R-vectors
+        bp0[r] = s_Bp[(2 * k) * R + r]; bp1[r] = s_Bp[(2 * k + 1) * R + r];
+        bt0[r] = s_Bt[(2 * k) * R + r]; bt1[r] = s_Bt[(2 * k + 1) * R + r];
+        c0[r] = s_Ct[(2 * k) * R + r]; c1[r] = s_Ct[(2 * k + 1) * R + r];
+      }
+      const float2 in0[2] = {make_float2(r0.x, r0.y), make_float2(r0.z, r0.w)};
+      const float2 in1[2] = {make_float2(r1.x, r1.y), make_float2(r1.z, r1.w)};
+      float o0[4], o1[4];
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        float2 g0 = in0[jj], g1 = in1[jj], u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          g0 = ffma2(bp0[r], xe[r][jj], g0);
+          g1 = ffma2(bp1[r], xe[r][jj], g1);
+          u0 = ffma2(bt0[r], xg[r][jj], u0);
+          u1 = ffma2(bt1[r], xg[r][jj], u1);
+        }
+        // (h'_{2k}, h'_{2k+1}) = alpha Rot(phi) (g_{2k}, g_{2k+1}) + (u_{2k}, u_{2k+1})
+        const float2 w0 = ffma2(AC, g0, ffma2(NAS, g1, u0));
+        const float2 w1 = ffma2(AS, g0, ffma2(AC, g1, u1));
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          yacc[r][jj] = ffma2(c0[r], w0, ffma2(c1[r], w1, yacc[r][jj]));
+        o0[2 * jj] = w0.x; o0[2 * jj + 1] = w0.y;
+        o1[2 * jj] = w1.x; o1[2 * jj + 1] = w1.y;
+      }
+      __stcs(dst + (2 * k) * rowq + pv, make_float4(o0[0], o0[1], o0[2], o0[3]));
+      __stcs(dst + (2 * k + 1) * rowq + pv, make_float4(o1[0], o1[1], o1[2], o1[3]));
+    }
+
+    // y: kslots of one warp share columns every PV lanes; then across warps
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj)
+        for (int off = PV; off < 32; off <<= 1) {
+          yacc[r][jj].x += __shfl_xor_sync(0xffffffffu, yacc[r][jj].x, off);
+          yacc[r][jj].y += __shfl_xor_sync(0xffffffffu, yacc[r][jj].y, off);
+        }
+    if (lane < PV) {  // PV = P / 4 <= 32: lanes below PV hold the warp's sums
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          s_red[(warp * R + r) * P + p0 + 2 * jj] = yacc[r][jj].x;
+          s_red[(warp * R + r) * P + p0 + 2 * jj + 1] = yacc[r][jj].y;
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < R * P; i += kThreads) {
+      float acc = 0.f;
+      for (int q = 0; q < kWarps; ++q) acc += s_red[q * R * P + i];
+      io_store(a.y, hd * R * P + i, acc, a.bf16);
+    }
+    __syncthreads();  // buffer bi, staging and partial sums free
+    if (sp.nbuf == 1 && tid == 0 && nhd < h_end) {  // one buffer: the next head starts now
+      issue(nhd, nbg, 0, nbg != bg);
+      pending |= 1u;
+    }
+    dt = ndt; Av = nA; lamv = nlam;
+    hh = nh;
+    bg = nbg;
   }
 
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      s_red[(kslot * R + r) * CB + p0 + 2 * j] = yacc[r][j].x;
-      s_red[(kslot * R + r) * CB + p0 + 2 * j + 1] = yacc[r][j].y;
-    }
-  __syncthreads();
-  for (int i = tid; i < R * CB; i += kDecodeThreads) {
-    float acc = 0.f;
-    for (int q = 0; q < nslots; ++q) acc += s_red[q * R * CB + i];
-    const int r = i / CB, c = i % CB;
-    io_store(a.y, bh * R * P + r * P + cb * CB + c, acc, a.bf16);
+  if (aborted && tid == 0) {  // let copies still in flight land (bounded) before exiting
+    for (int i = 0; i < 2; ++i)
+      if ((pending >> i) & 1u) decode_wait(&bars[i], (ph >> i) & 1u, a.status);
   }
+}
+
+template <int R, int NC, int PC>
+cudaError_t launch_shape(const DecodeArgs& a, cudaStream_t s) {
+  const DecodeSmem sp = decode_smem(a.N, a.P, R, a.bf16);
+  const size_t smem = (size_t)sp.total;
+  auto kern = decode_kernel<R, NC, PC>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const int64_t heads = a.batch * a.nheads;
+  const int64_t grid = heads < (int64_t)sms * per_sm ? heads : (int64_t)sms * per_sm;
+  kern<<<(unsigned)grid, kThreads, smem, s>>>(a);
+  return cudaGetLastError();
 }
 
 template <int R>
 cudaError_t launch_r(const DecodeArgs& a, cudaStream_t s) {
-  const int P = (int)a.P, N = (int)a.N;
-  const int CB = P < kMaxCols ? P : kMaxCols;
-  constexpr int kDecodeThreads = DecodeCfg<R>::threads;
-  const int nslots = kDecodeThreads / (CB / 4);
-  const size_t smem = sizeof(float) * (N + 3 * R * N + 2 * R * CB + (size_t)nslots * R * CB);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<R>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  const int64_t blocks = a.batch * a.nheads * (P / CB);
-  decode_kernel<R><<<(unsigned)blocks, kDecodeThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  if (a.N == 128 && a.P == 64) return launch_shape<R, 128, 64>(a, s);
+  return launch_shape<R, 0, 0>(a, s);
 }
 
 }  // namespace
 
 cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t s) {
+  if (a.batch * a.nheads == 0) return cudaSuccess;
   switch (a.R) {
     case 1: return launch_r<1>(a, s);
     case 2: return launch_r<2>(a, s);

@@ -196,6 +196,7 @@ M3_API int m3_decode_step(const m3_shape* s, const float* state_in, float* state
   a.state_in = state_in; a.state_out = state_out; a.x = x_t; a.dt = dt_t; a.A = A_t;
   a.lam = lam_t; a.theta = theta_t; a.B = B_t; a.C = C_t; a.B_prev = B_prev;
   a.x_prev = x_prev; a.y = y_t;
+  if (status_word(&a.status) != M3_OK) return M3_ERR_CUDA;
   cudaError_t e = decode_launch(a, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }

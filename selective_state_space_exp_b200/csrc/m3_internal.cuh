@@ -58,6 +58,7 @@ struct DecodeArgs {
   const void* B_prev;
   const void* x_prev;
   void* y;
+  int* status;  // device status word (timeouts)
 };
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }

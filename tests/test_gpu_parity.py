@@ -240,6 +240,36 @@ def test_decode_in_place_equals_out_of_place():
     assert np.array_equal(y1, y2) and np.array_equal(h1, h2)
 
 
+@pytest.mark.parametrize("N,P,R,io,prev", [(256, 32, 8, "f32", True), (16, 128, 1, "bf16", False),
+                                            (128, 128, 8, "f32", True), (64, 16, 4, "bf16", False),
+                                            (256, 64, 8, "f32", True)])
+def test_decode_shapes(N, P, R, io, prev):
+    """Decode over other state shapes (the largest N * P with R = 8 included,
+    one of them too large for two state buffers per CTA), two B/C groups,
+    with and without the previous token at step 0."""
+    w = I.Workload(I.Shape(3, 1, 4, P, N, R, 2, 64, io), bc="normal", with_h0=True,
+                   with_prev=True)
+    steps = 5
+    dec = I.make_decode_inputs(w, seed=5400 + N + P + R, steps=steps)
+    g = to_dev(dec)
+    state = g["state0"].clone()
+    ys = []
+    for t in range(steps):
+        Bp = (g["B_prev"] if prev else None) if t == 0 else g["B"][t - 1]
+        xp = (g["x_prev"] if prev else None) if t == 0 else g["x"][t - 1]
+        y, state = m3.m3_decode_step(state, g["x"][t], g["dt"][t], g["A"][t], g["lam"][t],
+                                     g["theta"][t], g["B"][t], g["C"][t], Bp, xp)
+        ys.append(y)
+    assert m3.m3_stream_status() == 0
+    yg = torch.stack(ys, 1).float().cpu().numpy()
+    sc = decode_as_scan(dec)
+    if not prev:
+        sc.pop("B_prev")
+        sc.pop("x_prev")
+    yo, ho = oracle_scan(sc)
+    check((rel_err(yg, yo), rel_err(state.cpu().numpy(), ho)), io)
+
+
 def test_decode_equals_scan_on_gpu():
     """Driving the decode kernel token by token reproduces the scan kernels
     (fp32 io)."""
