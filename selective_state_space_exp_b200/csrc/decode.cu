@@ -9,7 +9,8 @@
 // the rank-R MIMO update (section 2.3).  The step is HBM-bound (section 3.3:
 // decode is limited by state IO, not FLOPs): 2 * 4 * N * P bytes per head.
 //
-// Layout: CTAs of 256 threads, two or more per SM, each walking a contiguous
+// Rank R >= 2 (the arithmetic per element grows with R):
+// CTAs of 256 threads, two or more per SM, each walking a contiguous
 // range of heads (so consecutive heads mostly share one (batch, group) and
 // its B, C, B_prev are converted once).  A head's state and its operands
 // arrive in shared memory by bulk async copies issued one head ahead into a
@@ -18,6 +19,8 @@
 // Thread (kslot, pv) owns float4 column pv of the state and the pairs
 // k = kslot, kslot + nslots, ...; y is reduced over kslots with warp
 // shuffles and then across warps through shared memory.
+// Rank 1: one CTA per head streams the state through registers (see
+// stream_decode_kernel below).
 #include "m3_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -61,17 +64,22 @@ __device__ __forceinline__ void bulk_load(void* smem, const void* gmem, uint32_t
 }
 
 // Shared-memory plan of one CTA (byte offsets, all 128-byte aligned): the
-// state and raw operands of two heads (or one, for the largest shapes), the
-// fp32 B / C / B_prev of the current (batch, group), the per-head rotation
-// and x factors, and the per-warp partial sums of y.
+// state and raw operands of up to three heads in flight (one for the largest
+// shapes), the fp32 B / C / B_prev of the current (batch, group), the
+// per-head rotation and x factors, and the per-warp partial sums of y.
+constexpr int kMaxBuf = 3;
 struct DecodeSmem {
   int64_t st_bytes, ops_bytes;
-  int64_t st_off[2], ops_off[2], bc_off, head_off, red_off, bar_off, total;
-  int nbuf;  // 2: the next head streams in during this one; 1: the largest shapes
+  int64_t st_stride, ops_stride;  // buffer i: st at i * st_stride, ops at ops0 + i * ops_stride
+  int64_t ops0, bc_off, head_off, red_off, bar_off, total;
+  int nbuf;  // heads whose state is resident or in flight; nbuf - 1 stream in during one
 };
 constexpr int64_t kMaxSmem = 232448;  // dynamic shared memory of one CTA
 
-__host__ __device__ inline DecodeSmem decode_smem(int64_t N, int64_t P, int64_t R, bool bf16) {
+// want: buffers asked for (three when the arithmetic per head is light and
+// more bytes in flight pay, else two); fewer when they do not fit.
+__host__ __device__ inline DecodeSmem decode_smem(int64_t N, int64_t P, int64_t R, bool bf16,
+                                                  int want) {
   DecodeSmem m;
   const int64_t es = bf16 ? 2 : 4;
   const int64_t K = N / 2;
@@ -81,29 +89,25 @@ __host__ __device__ inline DecodeSmem decode_smem(int64_t N, int64_t P, int64_t 
   const int64_t head = align_up((6 * K + 2 * R * P) * 4, 128);  // rot, sin pairs, xe, xg
   const int64_t red = align_up(kWarps * R * P * 4, 128);
   const int64_t buf = align_up(m.st_bytes, 128) + align_up(m.ops_bytes, 128);
-  m.nbuf = 2 * buf + bc + head + red + 16 <= kMaxSmem ? 2 : 1;
-  int64_t o = 0;
-  for (int i = 0; i < 2; ++i) {
-    m.st_off[i] = i < m.nbuf ? o : m.st_off[0];
-    if (i < m.nbuf) o += align_up(m.st_bytes, 128);
-  }
-  for (int i = 0; i < 2; ++i) {
-    m.ops_off[i] = i < m.nbuf ? o : m.ops_off[0];
-    if (i < m.nbuf) o += align_up(m.ops_bytes, 128);
-  }
+  m.nbuf = want;
+  while (m.nbuf > 1 && m.nbuf * buf + bc + head + red + 32 > kMaxSmem) --m.nbuf;
+  m.st_stride = align_up(m.st_bytes, 128);
+  m.ops_stride = align_up(m.ops_bytes, 128);
+  m.ops0 = m.nbuf * m.st_stride;
+  int64_t o = m.ops0 + m.nbuf * m.ops_stride;
   m.bc_off = o; o += bc;
   m.head_off = o; o += head;
   m.red_off = o; o += red;
-  m.bar_off = o; o += 16;
+  m.bar_off = o; o += 32;
   m.total = o;
   return m;
 }
 
-// CTAs per SM the register budget is sized for (three for R = 1: its shared
-// memory allows three)
+// Buffers asked for, and the CTAs per SM the register budget is sized for.
 template <int R>
 struct DecodeOcc {
-  static constexpr int value = R == 1 ? 3 : (R <= 4 ? 2 : 1);
+  static constexpr int want = 2;
+  static constexpr int value = R <= 4 ? 2 : 1;
 };
 
 // NC, PC: compile-time N and P (0: taken from the arguments), so that the
@@ -114,7 +118,8 @@ __global__ void __launch_bounds__(kThreads, DecodeOcc<R>::value) decode_kernel(c
   const int lgN = __ffs(N) - 1;  // N and P are powers of two
   const int64_t H = a.nheads, G = a.ngroups, total = a.batch * H;
   const int64_t es = a.bf16 ? 2 : 4;
-  const DecodeSmem sp = decode_smem(N, P, R, a.bf16);
+  const DecodeSmem sp = decode_smem(N, P, R, a.bf16, DecodeOcc<R>::want);
+  const int nbuf = sp.nbuf;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   extern __shared__ __align__(128) uint8_t sm[];
@@ -138,8 +143,7 @@ __global__ void __launch_bounds__(kThreads, DecodeOcc<R>::value) decode_kernel(c
   const uint32_t bytes_bc = (prev ? 3 : 2) * opsB;
 
   if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    for (int i = 0; i < nbuf; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -147,8 +151,8 @@ __global__ void __launch_bounds__(kThreads, DecodeOcc<R>::value) decode_kernel(c
   const int hpg = (int)(H / G);  // heads per group
   // thread 0: bring head hd's state and operands into buffer bi
   auto issue = [&](int64_t hd, int64_t bg, int bi, bool with_bc) {
-    uint8_t* st = sm + sp.st_off[bi];
-    uint8_t* ops = sm + sp.ops_off[bi];
+    uint8_t* st = sm + bi * sp.st_stride;
+    uint8_t* ops = sm + sp.ops0 + bi * sp.ops_stride;
     fence_async_smem();
     mbar_expect_tx(&bars[bi], bytes_head + (with_bc ? bytes_bc : 0u));
     bulk_load(st, a.state_in + hd * (int64_t)N * P, (uint32_t)sp.st_bytes, &bars[bi]);
@@ -172,27 +176,38 @@ __global__ void __launch_bounds__(kThreads, DecodeOcc<R>::value) decode_kernel(c
   const int64_t per = (total + gridDim.x - 1) / gridDim.x;
   const int64_t h_begin = (int64_t)blockIdx.x * per;
   const int64_t h_end = min(total, h_begin + per);
+  uint32_t pending = 0u;  // thread 0: bit i = bytes expected on bars[i]
+  uint32_t ph = 0u;       // bit i = phase parity of bars[i]
+  // issue cursor (thread 0): the next head to bring in, its index within the
+  // batch, its (batch, group), the group of the head issued before it, its buffer
+  int64_t ihd = h_begin;
+  int ihh = (int)(h_begin % H);
+  int64_t ibg = (h_begin / H) * G + ihh / hpg, last_bg = -1;
+  int islot = 0;
+  auto issue_next = [&]() {
+    issue(ihd, ibg, islot, ibg != last_bg);
+    pending |= 1u << islot;
+    last_bg = ibg;
+    ++ihd;
+    ihh = ihh + 1 == H ? 0 : ihh + 1;
+    if (ihh % hpg == 0) ++ibg;
+    islot = islot + 1 == nbuf ? 0 : islot + 1;
+  };
+  if (tid == 0)
+    for (int i = 0; i < (nbuf > 1 ? nbuf - 1 : 1) && ihd < h_end; ++i) issue_next();
+
   int64_t hd = h_begin;
-  int64_t bg = (h_begin / H) * G + (int)(h_begin % H) / hpg;  // (batch, group) of head hd
-  int hh = (int)(h_begin % H);                                   // head index within the batch
-  if (tid == 0 && hd < h_end) issue(hd, bg, 0, true);
+  int hh = (int)(h_begin % H);  // head index within the batch
   // per-head scalars of the current head, loaded one head ahead
   float dt = 0.f, Av = 0.f, lamv = 0.f;
   if (hd < h_end) { dt = a.dt[hd]; Av = a.A[hd]; lamv = a.lam[hd]; }
-  uint32_t pending = hd < h_end ? 1u : 0u;  // thread 0: bit i = bytes expected on bars[i]
-  uint32_t ph = 0u;                          // bit i = phase parity of bars[i]
   bool aborted = false;
 
-  for (int j = 0; hd < h_end; ++hd, ++j) {
-    const int bi = sp.nbuf == 2 ? (j & 1) : 0;
+  for (int bi = 0; hd < h_end; ++hd, bi = bi + 1 == nbuf ? 0 : bi + 1) {
     const int64_t nhd = hd + 1;
     const bool new_bc = hd == h_begin || hh % hpg == 0;  // first head of its (batch, group)
-    const int nh = hh + 1 == H ? 0 : hh + 1;             // the next head's index and group
-    const int64_t nbg = nh == 0 ? bg + 1 : (nh % hpg == 0 ? bg + 1 : bg);
-    if (sp.nbuf == 2 && tid == 0 && nhd < h_end) {  // buffer bi ^ 1 was released by the last head
-      issue(nhd, nbg, bi ^ 1, nbg != bg);
-      pending |= 1u << (bi ^ 1);
-    }
+    // buffer (bi + nbuf - 1) % nbuf was released by the last head
+    if (nbuf > 1 && tid == 0 && ihd < h_end) issue_next();
     float ndt = 0.f, nA = 0.f, nlam = 0.f;
     if (nhd < h_end) { ndt = a.dt[nhd]; nA = a.A[nhd]; nlam = a.lam[nhd]; }
 
@@ -205,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, DecodeOcc<R>::value) decode_kernel(c
 
     const float alpha = expf(dt * Av);
     const float gamma = lamv * dt, eps = (1.f - lamv) * dt;
-    const uint8_t* ops = sm + sp.ops_off[bi];
+    const uint8_t* ops = sm + sp.ops0 + bi * sp.ops_stride;
     const void* ox = ops + 3 * opsB;
     const void* oxp = ops + 3 * opsB + opsX;
     const float* oth = reinterpret_cast<const float*>(ops + 3 * opsB + 2 * opsX);
@@ -242,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, DecodeOcc<R>::value) decode_kernel(c
         yacc[r][jj] = make_float2(0.f, 0.f);
       }
 
-    const float4* src = reinterpret_cast<const float4*>(sm + sp.st_off[bi]);
+    const float4* src = reinterpret_cast<const float4*>(sm + bi * sp.st_stride);
     float4* dst = reinterpret_cast<float4*>(a.state_out + hd * (int64_t)N * P);
 #pragma unroll
     for (int k = kslot; k < K; k += nslots) {
@@ -309,24 +324,20 @@ __global__ void __launch_bounds__(kThreads, DecodeOcc<R>::value) decode_kernel(c
       io_store(a.y, hd * R * P + i, acc, a.bf16);
     }
     __syncthreads();  // buffer bi, staging and partial sums free
-    if (sp.nbuf == 1 && tid == 0 && nhd < h_end) {  // one buffer: the next head starts now
-      issue(nhd, nbg, 0, nbg != bg);
-      pending |= 1u;
-    }
+    if (nbuf == 1 && tid == 0 && ihd < h_end) issue_next();  // one buffer: the next head now
     dt = ndt; Av = nA; lamv = nlam;
-    hh = nh;
-    bg = nbg;
+    hh = hh + 1 == H ? 0 : hh + 1;
   }
 
   if (aborted && tid == 0) {  // let copies still in flight land (bounded) before exiting
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < nbuf; ++i)
       if ((pending >> i) & 1u) decode_wait(&bars[i], (ph >> i) & 1u, a.status);
   }
 }
 
 template <int R, int NC, int PC>
 cudaError_t launch_shape(const DecodeArgs& a, cudaStream_t s) {
-  const DecodeSmem sp = decode_smem(a.N, a.P, R, a.bf16);
+  const DecodeSmem sp = decode_smem(a.N, a.P, R, a.bf16, DecodeOcc<R>::want);
   const size_t smem = (size_t)sp.total;
   auto kern = decode_kernel<R, NC, PC>;
   if (smem > 48 * 1024) {
@@ -351,12 +362,151 @@ cudaError_t launch_r(const DecodeArgs& a, cudaStream_t s) {
   return launch_shape<R, 0, 0>(a, s);
 }
 
+
+// ---- rank 1: one CTA per head, state streamed through registers -------------
+// With R = 1 the arithmetic per state element is small, and loads issued
+// straight into registers (four row pairs per thread in flight, seven CTAs
+// of 128 threads per SM) keep more bytes in flight than the shared-memory
+// pipeline above.  CTA (b, h); thread (kslot, pv) as above.
+constexpr int kStreamThreads = 128;
+constexpr int kStreamPairs = 4;  // row pairs whose loads are issued before any is used
+
+__global__ void __launch_bounds__(kStreamThreads, 7) stream_decode_kernel(const DecodeArgs a) {
+  const int P = (int)a.P, N = (int)a.N, K = N / 2;
+  const int64_t bh = blockIdx.x;
+  const int64_t h = bh % a.nheads, b = bh / a.nheads;
+  const int64_t bg = b * a.ngroups + h / (a.nheads / a.ngroups);
+  const int tid = threadIdx.x;
+
+  extern __shared__ float smf[];
+  float* s_ac = smf;              // alpha cos(dt theta_k)          [K]
+  float* s_as = s_ac + K;         // alpha sin(dt theta_k)          [K]
+  float* s_Bp = s_as + K;         // B_prev                         [N]
+  float* s_Bt = s_Bp + N;         // B_t                            [N]
+  float* s_Ct = s_Bt + N;         // C_t                            [N]
+  float* s_xe = s_Ct + N;         // (1-lam) dt x_prev              [P]
+  float* s_xg = s_xe + P;         // lam dt x_t                     [P]
+  float* s_red = s_xg + P;        // partial y per kslot            [nslots][P]
+
+  const float dt = a.dt[bh], lamv = a.lam[bh];
+  const float alpha = expf(dt * a.A[bh]);
+  const float gamma = lamv * dt, eps = (1.f - lamv) * dt;
+  const bool prev = a.B_prev != nullptr;
+
+  const int PV = P / 4;
+  const int nslots = kStreamThreads / PV;
+  const int pv = tid % PV, kslot = tid / PV;
+  const int p0 = pv * 4;
+  const float4* src = reinterpret_cast<const float4*>(a.state_in + bh * (int64_t)N * P);
+  float4* dst = reinterpret_cast<float4*>(a.state_out + bh * (int64_t)N * P);
+  const int rowq = P / 4;
+
+  // the first row pairs' loads go out before the per-head operands are staged
+  float4 r0[kStreamPairs], r1[kStreamPairs];
+#pragma unroll
+  for (int u = 0; u < kStreamPairs; ++u) {
+    const int k = kslot + u * nslots;
+    if (k < K) {
+      r0[u] = __ldcs(src + (2 * k) * rowq + pv);
+      r1[u] = __ldcs(src + (2 * k + 1) * rowq + pv);
+    }
+  }
+  for (int k = tid; k < K; k += kStreamThreads) {
+    float sn, cs;
+    sincosf(dt * a.theta[bg * K + k], &sn, &cs);
+    s_ac[k] = alpha * cs;
+    s_as[k] = alpha * sn;
+  }
+  for (int i = tid; i < N; i += kStreamThreads) {
+    s_Bt[i] = io_load(a.B, bg * N + i, a.bf16);
+    s_Ct[i] = io_load(a.C, bg * N + i, a.bf16);
+    s_Bp[i] = prev ? io_load(a.B_prev, bg * N + i, a.bf16) : 0.f;
+  }
+  for (int i = tid; i < P; i += kStreamThreads) {
+    s_xg[i] = gamma * io_load(a.x, bh * P + i, a.bf16);
+    s_xe[i] = prev ? eps * io_load(a.x_prev, bh * P + i, a.bf16) : 0.f;
+  }
+  __syncthreads();
+
+  float2 xg[2], xe[2], yacc[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    xg[j] = make_float2(s_xg[p0 + 2 * j], s_xg[p0 + 2 * j + 1]);
+    xe[j] = make_float2(s_xe[p0 + 2 * j], s_xe[p0 + 2 * j + 1]);
+    yacc[j] = make_float2(0.f, 0.f);
+  }
+  for (int kb = kslot; kb < K; kb += kStreamPairs * nslots) {
+    if (kb != kslot) {
+#pragma unroll
+      for (int u = 0; u < kStreamPairs; ++u) {
+        const int k = kb + u * nslots;
+        if (k < K) {
+          r0[u] = __ldcs(src + (2 * k) * rowq + pv);
+          r1[u] = __ldcs(src + (2 * k + 1) * rowq + pv);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kStreamPairs; ++u) {
+      const int k = kb + u * nslots;
+      if (k < K) {
+        const float ac = s_ac[k], as = s_as[k];
+        const float bp0 = s_Bp[2 * k], bp1 = s_Bp[2 * k + 1];
+        const float bt0 = s_Bt[2 * k], bt1 = s_Bt[2 * k + 1];
+        const float c0 = s_Ct[2 * k], c1 = s_Ct[2 * k + 1];
+        const float2 in0[2] = {make_float2(r0[u].x, r0[u].y), make_float2(r0[u].z, r0[u].w)};
+        const float2 in1[2] = {make_float2(r1[u].x, r1[u].y), make_float2(r1[u].z, r1[u].w)};
+        float o0[4], o1[4];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float2 g0 = ffma2(make_float2(bp0, bp0), xe[j], in0[j]);
+          const float2 g1 = ffma2(make_float2(bp1, bp1), xe[j], in1[j]);
+          const float2 u0 = fmul2(make_float2(bt0, bt0), xg[j]);
+          const float2 u1 = fmul2(make_float2(bt1, bt1), xg[j]);
+          // (h'_{2k}, h'_{2k+1}) = alpha Rot(phi) (g_{2k}, g_{2k+1}) + (u_{2k}, u_{2k+1})
+          const float2 w0 = ffma2(make_float2(ac, ac), g0, ffma2(make_float2(-as, -as), g1, u0));
+          const float2 w1 = ffma2(make_float2(as, as), g0, ffma2(make_float2(ac, ac), g1, u1));
+          yacc[j] = ffma2(make_float2(c0, c0), w0, ffma2(make_float2(c1, c1), w1, yacc[j]));
+          o0[2 * j] = w0.x; o0[2 * j + 1] = w0.y;
+          o1[2 * j] = w1.x; o1[2 * j + 1] = w1.y;
+        }
+        __stcs(dst + (2 * k) * rowq + pv, make_float4(o0[0], o0[1], o0[2], o0[3]));
+        __stcs(dst + (2 * k + 1) * rowq + pv, make_float4(o1[0], o1[1], o1[2], o1[3]));
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    s_red[kslot * P + p0 + 2 * j] = yacc[j].x;
+    s_red[kslot * P + p0 + 2 * j + 1] = yacc[j].y;
+  }
+  __syncthreads();
+  for (int i = tid; i < P; i += kStreamThreads) {
+    float acc = 0.f;
+    for (int q = 0; q < nslots; ++q) acc += s_red[q * P + i];
+    io_store(a.y, bh * P + i, acc, a.bf16);
+  }
+}
+
+cudaError_t launch_stream(const DecodeArgs& a, cudaStream_t s) {
+  const int P = (int)a.P, N = (int)a.N;
+  const int nslots = kStreamThreads / (P / 4);
+  const size_t smem = sizeof(float) * (N + 3 * N + 2 * P + (size_t)nslots * P);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(stream_decode_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  stream_decode_kernel<<<(unsigned)(a.batch * a.nheads), kStreamThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t s) {
   if (a.batch * a.nheads == 0) return cudaSuccess;
   switch (a.R) {
-    case 1: return launch_r<1>(a, s);
+    case 1: return launch_stream(a, s);
     case 2: return launch_r<2>(a, s);
     case 4: return launch_r<4>(a, s);
     case 8: return launch_r<8>(a, s);
