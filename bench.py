@@ -15,6 +15,7 @@ from __future__ import annotations
 
 import argparse
 import dataclasses
+import hashlib
 import json
 import math
 import os
@@ -86,6 +87,31 @@ def decode_work(s: I.Shape):
     byt = (2 * bh * N * P * 4 + 3 * bh * R * P * io + 3 * s.batch * s.ngroups * R * N * io
            + 3 * bh * 4 + s.batch * s.ngroups * (N // 2) * 4)
     return float(flops), float(byt)
+
+
+def profile_traffic(summary: str, key: str = "traffic_bytes_per_launch"):
+    """DRAM bytes per launch recorded in a committed ncu summary under profiles/,
+    or None when the kernel's sources changed since the counters were taken
+    (the summary names its source files and their combined sha256)."""
+    path = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith(("|", " ", "#")):
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+    try:
+        h = hashlib.sha256()
+        for rel in fields["source_files"].split():
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != fields["source_sha256"]:
+            return None
+        return int(fields[key])
+    except (KeyError, OSError, ValueError):
+        return None
 
 
 def roofline(flops, byt, seconds, peaks, src, sustained=False):
@@ -430,6 +456,18 @@ def main():
     plan = m3.scan_plan(m3.scan_shape(inp_host["x"], inp_host["B"], s.chunk))
     launches_per_call = plan["launches"]
     kern = "tc_scan_kernel (tcgen05)" if plan["tensor_core"] else "CUDA-core scan kernels"
+    # DRAM traffic per launch from the committed ncu summaries (None if stale
+    # or if the workload is not the one the summary was scaled to)
+    traffic, traffic_src = None, None
+    summary = {"siso_prefill": "tc_scan_kernel_siso_prefill.md",
+               "mimo_prefill": "tc_scan_kernel_mimo_prefill.md"}.get(args.workload)
+    if summary and plan["tensor_core"] and plan["segments"] == 1:
+        traffic = profile_traffic(summary)
+        traffic_src = f"profiles/{summary}" if traffic is not None else None
+    dkey = "traffic_bytes_per_launch_r1" if ds.rank == 1 else "traffic_bytes_per_launch_r4"
+    dtraffic = profile_traffic("decode_kernels_b128_h64_n128_p64.md", dkey) \
+        if ds.rank in (1, 4) and ds.batch == 128 else None
+    dtraffic_src = "profiles/decode_kernels_b128_h64_n128_p64.md" if dtraffic is not None else None
     line = {
         "metric": "prefill tokens/s",
         "value": round(world * tokens / per_step, 1),
@@ -450,13 +488,15 @@ def main():
                      "scope": ("the one kernel launch of each m3_scan_fwd call, CUDA events on "
                                "the launching stream" if launches_per_call == 1 else
                                "whole m3_scan_fwd call (all launches), CUDA events"),
-                     "traffic": None, "algorithmic_flops": flops, "algorithmic_bytes": byt},
+                     "traffic": traffic, "traffic_source": traffic_src,
+                     "algorithmic_flops": flops, "algorithmic_bytes": byt},
         "decode": {
             "metric": "decode tokens/s", "value": round(world * ds.batch * dsteps / dt_total, 1),
             "unit": "tokens/s", "steps": dsteps, "us_per_step": round(dt_total / dsteps * 1e6, 2),
             "config": {"workload": "decode_siso" if ds.rank == 1 else "decode_mimo",
                        **shape_cfg(ds)},
-            "roofline": roofline(dflops, dbyt, dt_total / dsteps, peaks, psrc),
+            "roofline": {**roofline(dflops, dbyt, dt_total / dsteps, peaks, psrc),
+                         "traffic": dtraffic, "traffic_source": dtraffic_src},
         },
         "e2e": {"value": round(world * tokens / e2e_step, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -170,7 +170,7 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// TMA: 3-D tiled bulk tensor load global -> shared (no multicast), completing
+// TMA: 3-D tiled bulk tensor load global -> this CTA's shared memory, completing
 // `bytes` of transaction count on an mbarrier.  `map` is the generic address
 // of a CUtensorMap kernel parameter.
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* map, int c0, int c1, int c2,
