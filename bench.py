@@ -120,9 +120,11 @@ def roofline(flops, byt, seconds, peaks, src, sustained=False):
     t_hbm = byt / (peaks["hbm_gbs"] * 1e9)
     if t_tensor >= t_hbm:
         ach = flops / seconds / 1e12
+        ts = peaks.get("bf16_tflops_sustained")
         return {"bound": "tensor", "achieved": round(ach, 2), "peak": tf, "unit": "TFLOP/s",
                 "frac": round(ach / tf, 4), "roofline_time_us": round(t_tensor * 1e6, 2),
-                "peak_source": f"{src} bf16 {'sustained' if sustained else 'burst'}"}
+                "peak_source": f"{src} bf16 {'sustained' if sustained else 'burst'}",
+                "frac_of_sustained": round(ach / ts, 4) if ts and not sustained else None}
     ach = byt / seconds / 1e9
     return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(ach / peaks["hbm_gbs"], 4), "roofline_time_us": round(t_hbm * 1e6, 2),
@@ -372,7 +374,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="siso_prefill", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="m3", choices=["m3", "reference"])
-    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--decode-steps", type=int, default=1024,
+                    help="consecutive decode steps timed (each with its own token's inputs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one part only (for profiling); prints its own line")

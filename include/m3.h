@@ -80,6 +80,13 @@ typedef enum {
 
 /* Flags (m3_shape.flags). */
 #define M3_FLAG_SIMT 1u /* force the CUDA-core fp32 scan (no tensor cores) */
+/* Diagnostic for the failure path of m3_scan_fwd on the tensor-core path:
+ * every CTA first waits, with a 1 ms limit, on an mbarrier that nothing
+ * completes, so the call computes nothing and the next m3_stream_status
+ * returns M3_ERR_TIMEOUT.  Lets a test check that a bounded device-side wait
+ * ends, reports its status and leaves the context usable.  Ignored by the
+ * CUDA-core path and by m3_decode_step. */
+#define M3_FLAG_TEST_TIMEOUT 2u
 
 typedef struct {
   int64_t batch;    /* b >= 1                                   */

@@ -23,7 +23,7 @@ int check_common(const m3_shape* s) {
     return M3_ERR_INVALID_ARGUMENT;
   if (s->dstate % 2 != 0 || s->nheads % s->ngroups != 0) return M3_ERR_INVALID_ARGUMENT;
   if (s->io_dtype != M3_F32 && s->io_dtype != M3_BF16) return M3_ERR_INVALID_ARGUMENT;
-  if ((s->flags & ~M3_FLAG_SIMT) != 0) return M3_ERR_INVALID_ARGUMENT;
+  if ((s->flags & ~(M3_FLAG_SIMT | M3_FLAG_TEST_TIMEOUT)) != 0) return M3_ERR_INVALID_ARGUMENT;
   // supported set
   if (!is_pow2(s->dstate) || s->dstate < 16 || s->dstate > 256) return M3_ERR_UNSUPPORTED;
   if (!is_pow2(s->headdim) || s->headdim < 16 || s->headdim > 128) return M3_ERR_UNSUPPORTED;
@@ -48,6 +48,7 @@ ScanArgs make_scan_args(const m3_shape* s) {
   a.Q = s->chunk;
   a.nchunks = (s->seqlen + s->chunk - 1) / s->chunk;
   a.bf16 = s->io_dtype == M3_BF16;
+  a.test_timeout = (s->flags & M3_FLAG_TEST_TIMEOUT) != 0;
   return a;
 }
 

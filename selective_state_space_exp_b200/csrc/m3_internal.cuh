@@ -40,7 +40,8 @@ struct ScanArgs {
   float* final_state;
   char* ws;
   size_t ws_bytes;
-  int* status;  // device-side error word
+  int* status;        // device-side error word
+  bool test_timeout;  // M3_FLAG_TEST_TIMEOUT
 };
 
 struct DecodeArgs {

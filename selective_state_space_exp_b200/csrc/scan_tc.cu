@@ -66,7 +66,7 @@ struct Cfg {
   // the w*x block, free during the angle pass.
   static constexpr int TH_FLOATS = Q * kPairs;
   static constexpr int GST_FLOATS = 3 * Q + 4;
-  static constexpr int SMALL_BYTES = (TH_FLOATS + 5 * Q + 3 * kPairs + GST_FLOATS) * 4 + 48;
+  static constexpr int SMALL_BYTES = (TH_FLOATS + 5 * Q + 3 * kPairs + GST_FLOATS) * 4 + 48;  // + 6 mbarrier slots
   static_assert(SLOTS_MAX * kPairs * 4 <= OPB, "slot sums must fit in the w*x block");
   static_assert(((TH_FLOATS + 5 * Q + 3 * kPairs + GST_FLOATS) * 4) % 8 == 0, "mbarrier alignment");
   // at least 80 KB so that no more than two CTAs (2 x 256 TMEM columns) share
@@ -120,11 +120,12 @@ __device__ __forceinline__ unsigned long long global_ns() {
 
 // Polls an mbarrier (called by one thread); returns false on timeout after
 // recording it in the device status word.
-__device__ bool wait_bar(uint64_t* bar, uint32_t parity, int* status) {
+__device__ bool wait_bar(uint64_t* bar, uint32_t parity, int* status,
+                         unsigned long long limit_ns = kWaitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > kWaitNs) {
+    if (global_ns() - t0 > limit_ns) {
       if (status) atomicCAS(status, 0, (int)M3_ERR_TIMEOUT);
       return false;
     }
@@ -174,6 +175,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   uint64_t* s_tbT = s_bar + 2;                                          // TMA of theta
   uint64_t* s_tbM = s_bar + 3;                                          // TMA of B, C, x
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_bar + 4);
+  uint64_t* s_never = s_bar + 5;  // M3_FLAG_TEST_TIMEOUT: a barrier nothing completes
   float* s_part = s_th;  // [slots][kPairs] slot angle sums, over the consumed theta rows
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -192,6 +194,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     mbar_init(s_bar1, 1);
     mbar_init(s_tbT, 1);
     mbar_init(s_tbM, 1);
+    mbar_init(s_never, 1);
     fence_mbar_init();
   }
   tc_fence_before();
@@ -397,10 +400,16 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     return true;
   };
 
-  prefetch_early(c_begin);
-  prefetch_c(c_begin);
-  prefetch_bx(c_begin);
-  if (c_begin < c_end && !prologue(c_begin)) aborted = true;
+  if (a.test_timeout) {  // diagnostics: this wait must end in M3_ERR_TIMEOUT after 1 ms
+    const bool okn = (tid == 0) ? wait_bar(s_never, 0, a.status, 1000000ull) : true;
+    if (__syncthreads_or(!okn)) aborted = true;
+  }
+  if (!aborted) {
+    prefetch_early(c_begin);
+    prefetch_c(c_begin);
+    prefetch_bx(c_begin);
+    if (c_begin < c_end && !prologue(c_begin)) aborted = true;
+  }
 
   for (int64_t c = c_begin; c < c_end && !aborted; ++c) {
     const int64_t c0 = c * Q;

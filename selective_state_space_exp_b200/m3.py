@@ -19,6 +19,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "m3.h")
 
 M3_F32, M3_BF16 = 0, 1
 M3_FLAG_SIMT = 1
+M3_FLAG_TEST_TIMEOUT = 2
 STATUS = {0: "M3_OK", -1: "M3_ERR_INVALID_ARGUMENT", -2: "M3_ERR_UNSUPPORTED",
           -3: "M3_ERR_ALIGNMENT", -4: "M3_ERR_WORKSPACE", -5: "M3_ERR_CUDA",
           -6: "M3_ERR_TIMEOUT"}
@@ -134,11 +135,12 @@ def scan_plan(shape: Shape) -> dict:
 
 def m3_scan_fwd(x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None, B_prev=None,
                 x_prev=None, *, y=None, final_state=None, want_final=True, workspace=None,
-                simt=False, stream=None):
+                simt=False, stream=None, extra_flags=0):
     """Chunked prefill scan.  x [b][L][H][R][P] (io dtype), dt/A/lam [b][L][H],
     theta [b][L][G][N/2] fp32, B/C [b][L][G][R][N] (io dtype).  R is x.shape[3].
-    Returns (y, final_state)."""
+    extra_flags: further M3_FLAG_* bits (diagnostics).  Returns (y, final_state)."""
     shape = scan_shape(x, B, chunk, simt)
+    shape.flags |= extra_flags
     if y is None:
         y = torch.empty_like(x)
     if final_state is None and want_final:

@@ -281,6 +281,22 @@ def test_decode_equals_scan_on_gpu():
     assert rel_err(yd, ys) < 1e-5 and rel_err(hd, hs) < 1e-5
 
 
+def test_bounded_wait_reports_timeout():
+    """Failure path: with M3_FLAG_TEST_TIMEOUT every CTA of the tensor-core scan
+    waits on an mbarrier that nothing completes; the wait gives up after its
+    1 ms limit, the call reports M3_ERR_TIMEOUT through m3_stream_status, and
+    the next call on the same context computes the right answer."""
+    w = I.Workload(I.Shape(1, 200, 4, 64, 128, 1, 1, 64, "bf16"), with_h0=True)
+    inp = I.make_scan_inputs(w, seed=5500)
+    g = to_dev(inp)
+    args = (g["x"], g["dt"], g["A"], g["lam"], g["theta"], g["B"], g["C"], 64, g["h0"])
+    assert m3.scan_plan(m3.scan_shape(g["x"], g["B"], 64))["tensor_core"]
+    m3.m3_scan_fwd(*args, extra_flags=m3.M3_FLAG_TEST_TIMEOUT)
+    assert m3.m3_stream_status() == -6  # M3_ERR_TIMEOUT, and the word is cleared
+    assert m3.m3_stream_status() == 0
+    check(compare_scan(inp, 64, "bf16"), "bf16")
+
+
 def test_gpu_rejects_bad_pointers():
     """Host-side checks with real device tensors: misaligned views and a small
     workspace return errors and launch nothing."""
