@@ -56,43 +56,48 @@ struct Cfg {
   static constexpr int X_OFF = C_OFF + 2 * OPB;
   static constexpr int B_OFF = X_OFF + OPB;     // Bt: 2 blocks
   static constexpr int XW_OFF = B_OFF + 2 * OPB;
-  static constexpr int P_OFF = B_OFF;           // masked scores reuse Bt + Xw
   static constexpr int G_OFF = XW_OFF + OPB;    // state, bf16 [N][128 B]
   static constexpr int SMALL_OFF = G_OFF + kN * 128;
   // small region: the chunk's theta [Q][N/2] (a TMA destination, first so it
-  // is 1 KB aligned), per-token gamma, delta, w, Lam (log2 units) and the
-  // decay factor F, chunk-end angles with their cos / sin, the staged gates
-  // (dt[Q+1], lam[Q+1], A[Q]) and the mbarriers.  The slot angle sums live in
-  // the w*x block, free during the angle pass.
+  // is 1 KB aligned; the slot angle sums go over it once it is read),
+  // per-token gamma, delta, w, Lam (log2 units) and the decay factor F,
+  // chunk-end angles with their cos / sin, and the mbarriers.
   static constexpr int TH_FLOATS = Q * kPairs;
-  static constexpr int GST_FLOATS = 3 * Q + 4;
-  static constexpr int SMALL_BYTES = (TH_FLOATS + 5 * Q + 3 * kPairs + GST_FLOATS) * 4 + 48;  // + 6 mbarrier slots
-  static_assert(SLOTS_MAX * kPairs * 4 <= OPB, "slot sums must fit in the w*x block");
-  static_assert(((TH_FLOATS + 5 * Q + 3 * kPairs + GST_FLOATS) * 4) % 8 == 0, "mbarrier alignment");
+  static constexpr int SMALL_BYTES = (TH_FLOATS + 6 * Q + 3 * kPairs) * 4 + 64;  // + 8 mbarrier slots
+  static_assert(((TH_FLOATS + 6 * Q + 3 * kPairs) * 4) % 8 == 0, "mbarrier alignment");
   // at least 80 KB so that no more than two CTAs (2 x 256 TMEM columns) share
   // an SM; the dynamic shared memory base is declared 1024-byte aligned
   static constexpr int SMEM_RAW = SMALL_OFF + SMALL_BYTES;
   static constexpr int SMEM = SMEM_RAW < 80 * 1024 ? 80 * 1024 : SMEM_RAW;
   static_assert(MINB * (SMEM + 1024) <= 233472, "CTAs per SM must fit the SM's shared memory");
-  // P tile mt: ((mt + 1) * MT / 64) blocks of [MT][128 B]
-  __host__ __device__ static constexpr int p_tile_off(int mt) {
-    return mt == 0 ? 0 : (MT / 64) * MT * 128;
+  // Masked scores P, tile mt: ((mt + 1) * MT / 64) K-blocks of [MT][128 B].
+  // One tile: over Bt (MMA1 and MMA3 are done when it is written).  Two
+  // tiles: tile 0 over w*x (MMA3 is done; tile 1's MMA1 still reads all of
+  // Bt), tile 1 over Bt once tile 1's scores are complete.
+  __host__ __device__ static constexpr int p_off(int mt) {
+    return (NT == 2 && mt == 0) ? XW_OFF : B_OFF;
   }
-  static constexpr int P_BYTES = p_tile_off(NT - 1) + (NT * MT / 64) * MT * 128;
-  static_assert(P_BYTES <= 3 * OPB, "masked scores must fit over Bt + Xw");
+  static_assert(NT == 1 ? (MT / 64) * MT * 128 <= 2 * OPB
+                        : (MT / 64) * MT * 128 <= OPB && 2 * (MT / 64) * MT * 128 <= 2 * OPB,
+                "masked scores must fit their regions");
   // TMEM columns
   static constexpr int S_COL1 = 0;                  // tile 1 scores (M = 256 only)
   static constexpr int S_COL0 = (NT == 2) ? 256 : 0;
   // One tile per chunk: scores (MT columns; the MMA2 output reuses them once
   // masked), MMA4 output and chunk state side by side, so MMA4 can run with
-  // MMA3 before the mask.  Two tiles: the scores take 384 columns, so MMA4
-  // runs after the mask and its output reuses score columns.
+  // MMA3 before the mask.  Two tiles: the scores take 384 columns, so a
+  // tile's MMA2 and MMA4 run after its mask and their outputs reuse that
+  // tile's score columns (tile 0's MMAs then overlap tile 1's mask).
   static constexpr bool EARLY4 = NT == 1;
   static constexpr int SC_COL = (NT == 2) ? 384 : MT + 64;  // chunk state N x P
   static constexpr int TMEM_COLS = (NT == 2) ? 512 : 256;
   __host__ __device__ static constexpr int s_col(int mt) { return mt == 0 ? S_COL0 : S_COL1; }
-  __host__ __device__ static constexpr int y_col(int mt) { return 64 * mt; }
-  __host__ __device__ static constexpr int y2_col(int mt) { return NT == 2 ? 64 * (2 + mt) : MT; }
+  __host__ __device__ static constexpr int y_col(int mt) {
+    return NT == 2 ? (mt == 0 ? 256 : 0) : 0;
+  }
+  __host__ __device__ static constexpr int y2_col(int mt) {
+    return NT == 2 ? (mt == 0 ? 320 : 64) : MT;
+  }
   static_assert(SC_COL + kP <= TMEM_COLS, "TMEM columns");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
@@ -167,15 +172,16 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   float* s_w = s_del + Q;                       // exp(Lam_end - Lam_s) delta_s         [Q]
   float* s_lg = s_w + Q;                        // Lam_t * log2(e)                      [Q]
   float* s_F = s_lg + Q;                        // exp(ref - Lam_s) delta_s             [Q]
-  float* s_phe = s_F + Q;                       // chunk-end angles                     [kPairs]
+  float* s_dtv = s_F + Q;                       // dt_t                                 [Q]
+  float* s_phe = s_dtv + Q;                     // chunk-end angles                     [kPairs]
   float2* s_pcs = reinterpret_cast<float2*>(s_phe + kPairs);  // their cos, sin        [kPairs]
-  float* s_gst = reinterpret_cast<float*>(s_pcs + kPairs);    // staged gates of a chunk
-  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_gst + C::GST_FLOATS);  // MMA3+MMA4, MMA2
+  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_pcs + kPairs);  // MMA3+MMA4, MMA2
   uint64_t* s_bar1 = s_bar + 1;                                         // MMA1
   uint64_t* s_tbT = s_bar + 2;                                          // TMA of theta
   uint64_t* s_tbM = s_bar + 3;                                          // TMA of B, C, x
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_bar + 4);
   uint64_t* s_never = s_bar + 5;  // M3_FLAG_TEST_TIMEOUT: a barrier nothing completes
+  uint64_t* s_bar1b = s_bar + 6;  // MMA1 of tile 1 (two-tile chunks)
   float* s_part = s_th;  // [slots][kPairs] slot angle sums, over the consumed theta rows
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -195,6 +201,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     mbar_init(s_tbT, 1);
     mbar_init(s_tbM, 1);
     mbar_init(s_never, 1);
+    mbar_init(s_bar1b, 1);
     fence_mbar_init();
   }
   tc_fence_before();
@@ -202,7 +209,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   tc_fence_after();
   const uint32_t tm = *s_tmem;
   const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
-  uint32_t phase = 0, phase1 = 0, tphT = 0, tphM = 0;
+  uint32_t phase = 0, phase1 = 0, phase1b = 0, tphT = 0, tphM = 0;
   bool aborted = false;
   bool tpendT = false, tpendM = false;  // thread 0: TMA bytes expected on s_tbT / s_tbM
 
@@ -261,21 +268,26 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   constexpr uint32_t kTileBytes = Q * R * 128;  // one {64, R, Q} bf16 box
   constexpr uint32_t kMBytes = kTileBytes * (MODE == MODE_FULL ? 5 : 3);
   auto prefetch_early = [&](int64_t cn) {
-    if (cn >= c_end) return;
+    if (cn >= c_end || tid != 0) return;
+    mbar_expect_tx(s_tbT, Q * kPairs * 4);
+    tpendT = true;
+    tma_load_3d(s_th, &maps.th, 0, (int)g, (int)(b * L + cn * Q), s_tbT);
+  };
+  // The gates go to registers of the gate threads one chunk ahead (plain
+  // loads: the prologue that uses them runs a whole chunk later): token tid's
+  // dt, lam, A and the next token's dt, lam.
+  float gr_dt = 0.f, gr_lm = 0.f, gr_av = 0.f, gr_dt1 = 0.f, gr_lm1 = 0.f;
+  auto load_gates = [&](int64_t cn) {
     const int64_t cn0 = cn * Q;
-    if (tid == 0) {
-      mbar_expect_tx(s_tbT, Q * kPairs * 4);
-      tpendT = true;
-      tma_load_3d(s_th, &maps.th, 0, (int)g, (int)(b * L + cn0), s_tbT);
+    if (tid < Q) {
+      const int64_t t0 = cn0 + tid, i0 = (b * L + t0) * H + h;
+      const bool v0 = cn < c_end && t0 < L, v1 = cn < c_end && t0 + 1 < L;
+      gr_dt = v0 ? __ldg(a.dt + i0) : 0.f;
+      gr_lm = v0 ? __ldg(a.lam + i0) : 0.f;
+      gr_av = v0 ? __ldg(a.A + i0) : 0.f;
+      gr_dt1 = v1 ? __ldg(a.dt + i0 + H) : 0.f;
+      gr_lm1 = v1 ? __ldg(a.lam + i0 + H) : 0.f;
     }
-    for (int i = tid; i < 3 * Q + 2; i += NTH) {
-      const int which = i < Q + 1 ? 0 : (i < 2 * Q + 2 ? 1 : 2);
-      const int t = which == 0 ? i : (which == 1 ? i - (Q + 1) : i - (2 * Q + 2));
-      const bool v = cn0 + t < L;
-      const float* base = which == 0 ? a.dt : (which == 1 ? a.lam : a.A);
-      cp_async4(s_gst + i, v ? base + (b * L + cn0 + t) * H + h : base, v);
-    }
-    cp_async_commit();
   };
   auto arm_m = [&]() {  // thread 0
     if (!tpendM) {
@@ -311,24 +323,15 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   auto prologue = [&](int64_t cc) -> bool {
     const int nt = (int)min((int64_t)Q, L - cc * Q);
     const bool slot_live = tq < SLOTS;
-    cp_async_wait_all();
-    const bool okt = (tid == 0) ? wait_bar(s_tbT, tphT, a.status) : true;
-    if (okt && tid == 0) { tpendT = false; tphT ^= 1; }  // on a timeout the phase stays
-    if (__syncthreads_or(!okt)) return false;            // theta and gates visible
-
     const bool gate_warp = warp < (Q + 31) / 32;
-    float g_dt = 0.f, g_lm = 0.f, g_av = 0.f, g_nx = 0.f;
-    if (gate_warp && tid < nt) {
-      g_dt = s_gst[tid];
-      g_lm = s_gst[Q + 1 + tid];
-      g_av = s_gst[2 * Q + 2 + tid];
-      g_nx = (1.f - s_gst[Q + 2 + tid]) * s_gst[tid + 1];  // zero-filled past the sequence end
-    }
-    if (gate_warp) {  // whole warps take part in the shuffle scan
+    if (gate_warp) {  // whole warps take part in the shuffle scan of Lam
+      // loaded as zeros past the sequence end
+      const float g_dt = gr_dt, g_lm = gr_lm, g_av = gr_av, g_nx = (1.f - gr_lm1) * gr_dt1;
       const bool inq = tid < Q;
       if (inq) {
         s_gam[tid] = g_lm * g_dt;
         s_del[tid] = g_lm * g_dt + g_nx;
+        s_dtv[tid] = g_dt;
       }
       float v = g_dt * g_av * kL2E;
 #pragma unroll
@@ -338,13 +341,17 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       }
       if (inq) s_lg[tid] = v;
     }
+    const bool okt = (tid == 0) ? wait_bar(s_tbT, tphT, a.status) : true;
+    if (okt && tid == 0) { tpendT = false; tphT ^= 1; }  // on a timeout the phase stays
+    if (__syncthreads_or(!okt)) return false;  // theta, gates and each warp's Lam visible
+    if (Q > 32 && tid >= 32 && tid < Q) s_lg[tid] += s_lg[31];  // second warp of tokens
     // cumulative angles of pairs 4kg..4kg+3 over this slot's tokens
     float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int u = 0; u < TQ; ++u) {
       const int t = tq * TQ + u;
       const bool live_t = slot_live && t < nt;
-      const float d = live_t ? s_gst[t] : 0.f;
+      const float d = live_t ? s_dtv[t] : 0.f;
       const float4 th = live_t ? *reinterpret_cast<const float4*>(s_th + t * kPairs + 4 * kg)
                                : make_float4(0.f, 0.f, 0.f, 0.f);
       ang[u][0] = make_float2(d * th.x, d * th.y);
@@ -352,8 +359,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       part[0] += ang[u][0].x; part[1] += ang[u][0].y;
       part[2] += ang[u][1].x; part[3] += ang[u][1].y;
     }
-    __syncthreads();  // theta read; first-warp Lam written
-    if (Q > 32 && tid >= 32 && tid < Q) s_lg[tid] += s_lg[31];  // second warp of tokens
+    __syncthreads();  // theta read (the slot sums go over it); Lam complete
     // slot sums: row = slot, 16-byte piece kg at position kg ^ (slot % 8)
     auto part_at = [&](int slot, int k4) { return s_part + slot * kPairs + 4 * (k4 ^ (slot & 7)); };
     if (slot_live)
@@ -396,6 +402,10 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       const float lg = s_lg[tid];
       s_w[tid] = (tid < nt) ? ex2(l2end - lg) * s_del[tid] : 0.f;
       s_F[tid] = fac_ok ? ex2(l2ref - lg) * s_del[tid] : 0.f;
+    } else if (tid < Q + kPairs) {  // cos, sin of the chunk-end angles (state update)
+      float sn, cs;
+      sincosf(s_phe[tid - Q], &sn, &cs);
+      s_pcs[tid - Q] = make_float2(cs, sn);
     }
     return true;
   };
@@ -408,6 +418,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     prefetch_early(c_begin);
     prefetch_c(c_begin);
     prefetch_bx(c_begin);
+    load_gates(c_begin);
     if (c_begin < c_end && !prologue(c_begin)) aborted = true;
   }
 
@@ -418,6 +429,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     const float l2ref = 0.5f * l2end;
     const bool fac_ok = l2end > -230.f;
 
+    load_gates(c + 1);  // consumed by the next chunk's prologue, at the end of this one
     const bool okm = (tid == 0) ? wait_bar(s_tbM, tphM, a.status) : true;
     if (okm && tid == 0) { tpendM = false; tphM ^= 1; }  // on a timeout the phase stays
     if (__syncthreads_or(!okm)) { aborted = true; break; }  // B, C and x of this chunk visible
@@ -469,12 +481,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     }
     if (MODE == MODE_FULL && tid == 0) bulk_wait_read0();  // the last chunk's staged y is read
     __syncthreads();  // s_w ready; slot sums read; the w*x block is free
-    prefetch_early(c + 1);  // theta and gate buffers are free
-    if (tid < kPairs) {
-      float sn, cs;
-      sincosf(s_phe[tid], &sn, &cs);
-      s_pcs[tid] = make_float2(cs, sn);
-    }
+    prefetch_early(c + 1);  // the theta buffer is free
 
     // ---- w * x (chunk-state operand) from the x tile ---------------------------
     constexpr int PER = M * 8 / NTH;
@@ -500,10 +507,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     tc_fence_after();
 
     // ---- MMA3 (chunk state) and MMA4 (Ct G), then MMA1 (scores) ----------------
-    auto issue_mma4 = [&]() {  // y2 = Ct G, one thread
+    auto issue_mma4 = [&](int mt) {  // y2 = Ct G for tile mt, one thread
       const uint32_t id4 = idesc_bf16(MT, kP, 0, 1);
-#pragma unroll
-      for (int mt = 0; mt < NT; ++mt)
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
@@ -521,7 +526,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         const uint64_t bd = sw128_desc(sbase + C::XW_OFF + ks * 2048, C::OPB, 1024);
         mma_bf16_ss(tm + C::SC_COL, ad, bd, id3, ks != 0);
       }
-      if (MODE == MODE_FULL && C::EARLY4) issue_mma4();
+      if (MODE == MODE_FULL && C::EARLY4) issue_mma4(0);
       mma_commit(s_bar);
       if (MODE == MODE_FULL) {
 #pragma unroll
@@ -535,8 +540,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
               const uint64_t bd = sw128_desc(sbase + C::B_OFF + kb * C::OPB + k4 * 32, 16, 1024);
               mma_bf16_ss(tm + C::s_col(mt), ad, bd, id, (kb | k4) != 0);
             }
+          mma_commit(mt == 0 ? s_bar1 : s_bar1b);  // each tile's scores on their own barrier
         }
-        mma_commit(s_bar1);
       }
     }
     const bool ok3 = (tid == 0) ? wait_bar(s_bar, phase, a.status) : true;
@@ -583,10 +588,17 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       tc_fence_after();
       if (C::EARLY4) prefetch_c(c + 1);  // MMA1 and MMA4 have read Ct
 
-      // ---- mask the scores into P (bf16, K-major, over Bt / Xw) -------------
+      // ---- per score tile: mask into P (bf16, K-major), then its MMA2 (P x) -----
       //   P[(t,r),(s,r')] = S * (s < t ? exp(Lam_t - Lam_s) delta_s : s == t ? gamma_t : 0)
+      // With two tiles, tile 1's mask runs while tile 0's MMA2 and MMA4 run.
 #pragma unroll
       for (int mt = 0; mt < NT; ++mt) {
+        if (mt == 1) {  // tile 1's scores
+          const bool okb = (tid == 0) ? wait_bar(s_bar1b, phase1b, a.status) : true;
+          phase1b ^= 1;
+          if (__syncthreads_or(!okb)) { aborted = true; break; }
+          tc_fence_after();
+        }
         const int rho0 = (MT == 64) ? 16 * qd : 32 * qd;     // the warp's first row
         const int rho = rho0 + lane;
         const bool live = (MT == 64) ? lane < 16 : true;
@@ -646,7 +658,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
           }
           if (live) {
             const int kb = (cc * 16) / 64;
-            uint8_t* blk = sm + C::P_OFF + C::p_tile_off(mt) + kb * MT * 128;
+            uint8_t* blk = sm + C::p_off(mt) + kb * MT * 128;
             const int ch0 = ((cc * 16) % 64) / 8;
 #pragma unroll
             for (int q = 0; q < 4; ++q)
@@ -654,30 +666,25 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
                   make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           }
         }
-      }
-      fence_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      tc_fence_after();
-
-      // ---- MMA2 (P x) ----------------------------------------------------------
-      if (tid == 0) {
-        const uint32_t id2 = idesc_bf16(MT, kP, 0, 1);
-#pragma unroll
-        for (int mt = 0; mt < NT; ++mt) {
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0) {  // MMA2 for this tile (and MMA4 for two-tile chunks)
+          const uint32_t id2 = idesc_bf16(MT, kP, 0, 1);
           const int kblocks = (mt + 1) * MT / 64;
           for (int kb = 0; kb < kblocks; ++kb)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
-              const uint64_t ad = sw128_desc(
-                  sbase + C::P_OFF + C::p_tile_off(mt) + kb * MT * 128 + k4 * 32, 16, 1024);
+              const uint64_t ad = sw128_desc(sbase + C::p_off(mt) + kb * MT * 128 + k4 * 32, 16, 1024);
               const uint64_t bd = sw128_desc(sbase + C::X_OFF + (kb * 4 + k4) * 2048, C::OPB, 1024);
               mma_bf16_ss(tm + C::y_col(mt), ad, bd, id2, (kb | k4) != 0);
             }
+          if (!C::EARLY4) issue_mma4(mt);
+          if (mt == NT - 1) mma_commit(s_bar);
         }
-        if (!C::EARLY4) issue_mma4();
-        mma_commit(s_bar);
       }
+      if (aborted) break;
       const bool ok2 = (tid == 0) ? wait_bar(s_bar, phase, a.status) : true;
       phase ^= 1;
       if (__syncthreads_or(!ok2)) { aborted = true; break; }
@@ -753,7 +760,6 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     }
   }
   // an aborted run may leave a prefetch in flight: let it land (bounded wait)
-  cp_async_wait_all();
   if (tid == 0 && tpendT) wait_bar(s_tbT, tphT, a.status);
   if (tid == 0 && tpendM) wait_bar(s_tbM, tphM, a.status);
   if (MODE == MODE_FULL && tid == 0) bulk_wait0();  // y stores complete
