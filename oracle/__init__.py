@@ -24,8 +24,10 @@ _lib = None
 
 
 class Dims(ctypes.Structure):
+    # tgroups: theta groups (its third dimension: G like B and C, or H)
     _fields_ = [(n, ctypes.c_int64) for n in
-                ("batch", "seqlen", "nheads", "ngroups", "headdim", "dstate", "rank")]
+                ("batch", "seqlen", "nheads", "ngroups", "headdim", "dstate", "rank",
+                 "tgroups")]
 
 
 def build(force: bool = False) -> str:
@@ -84,7 +86,7 @@ def _dims(x, B, theta):
     # x: [b][L][H][R][P], B: [b][L][G][R][N]
     b, L, H, R, P = x.shape
     G, N = B.shape[2], B.shape[4]
-    return Dims(b, L, H, G, P, N, R)
+    return Dims(b, L, H, G, P, N, R, theta.shape[2])
 
 
 def scan(x, dt, A, lam, theta, B, C, h0=None, B_prev=None, x_prev=None,
@@ -121,7 +123,7 @@ def decode_step(state, x_t, dt, A, lam, theta, B_t, C_t, B_prev=None, x_prev=Non
     arrs = [_np(v, dt_) for v in (x_t, dt, A, lam, theta, B_t, C_t, B_prev, x_prev)]
     b, H, R, P = arrs[0].shape
     G, N = arrs[5].shape[1], arrs[5].shape[3]
-    d = Dims(b, 1, H, G, P, N, R)
+    d = Dims(b, 1, H, G, P, N, R, arrs[4].shape[1])
     y = np.zeros((b, H, R, P), dtype=np.float64)
     rc = lib().m3o_decode_step(ctypes.byref(d), 1 if f64 else 0,
                                st.ctypes.data_as(ctypes.c_void_p),

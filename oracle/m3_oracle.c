@@ -38,14 +38,16 @@
  *
  * Readings where the pages are silent (not stated on the pages):
  *   - pairs are adjacent rows (2k, 2k+1); rotation e^{+i phi};
- *   - theta is an angle rate [b][L][G][N/2]; the step angle is dt * theta;
+ *   - theta is an angle rate [b][L][Gt][N/2]; the step angle is dt * theta;
+ *     Gt (tgroups) is the B/C group count G by default, or H for per-head
+ *     angle rates (a layout variant: head h reads theta group h / (H / Gt));
  *   - B, C are shared by the H/G heads of a group; A is per token and head;
  *   - the left-endpoint term is carried through the rotation and decay;
  *   - initial conditions: z = h0 (else 0); B_{-1} x_{-1} = B_prev x_prev (else 0).
  *
  * Layouts (row-major, contiguous) are the library's:
  *   x, y: [b][L][H][R][P]   B, C: [b][L][G][R][N]   dt, A, lam: [b][L][H]
- *   theta: [b][L][G][N/2]   h0, hL: [b][H][N][P]   B_prev: [b][G][R][N]
+ *   theta: [b][L][Gt][N/2]  h0, hL: [b][H][N][P]   B_prev: [b][G][R][N]
  *   x_prev: [b][H][R][P]
  */
 #include <complex.h>
@@ -57,7 +59,15 @@
 
 typedef struct {
   int64_t batch, seqlen, nheads, ngroups, headdim, dstate, rank;
+  int64_t tgroups; /* theta groups: 0 or ngroups (shared like B, C) or nheads */
 } m3o_dims;
+
+/* theta group of head h */
+static int64_t tgroup(const m3o_dims* d, int64_t h) {
+  int64_t Gt = d->tgroups > 0 ? d->tgroups : d->ngroups;
+  return h / (d->nheads / Gt);
+}
+static int64_t tgroups(const m3o_dims* d) { return d->tgroups > 0 ? d->tgroups : d->ngroups; }
 
 /* ---- test-only fault planting (0 = exact method) -------------------------
  * Tests set a mutation to prove that the pins catch plausible mistakes.
@@ -176,7 +186,8 @@ static void gather_chain(const scan_job* j, int64_t b, int64_t h, chain_buf* cb)
     cb->A[t] = ld(j->A, bt * H + h, j->f64);
     cb->lam[t] = ld(j->lam, bt * H + h, j->f64);
     for (int64_t k = 0; k < N / 2; ++k)
-      cb->theta[t * (N / 2) + k] = ld(j->theta, (bt * G + g) * (N / 2) + k, j->f64);
+      cb->theta[t * (N / 2) + k] =
+          ld(j->theta, (bt * tgroups(d) + tgroup(d, h)) * (N / 2) + k, j->f64);
     for (int64_t i = 0; i < R * N; ++i) {
       cb->B[t * R * N + i] = ld(j->B, (bt * G + g) * R * N + i, j->f64);
       cb->C[t * R * N + i] = ld(j->C, (bt * G + g) * R * N + i, j->f64);
@@ -252,6 +263,7 @@ static int check_dims(const m3o_dims* d) {
       d->headdim < 1 || d->dstate < 2 || d->rank < 1)
     return -1;
   if (d->dstate % 2 || d->nheads % d->ngroups) return -1;
+  if (d->tgroups < 0 || (d->tgroups > 0 && d->nheads % d->tgroups)) return -1;
   return 0;
 }
 
@@ -313,7 +325,8 @@ int m3o_decode_step(const m3o_dims* d, int in_f64, double* state,
   for (int64_t b = 0; b < Bn; ++b)
     for (int64_t h = 0; h < H; ++h) {
       int64_t g = h / (H / G), bh = b * H + h, bg = b * G + g;
-      for (int64_t k = 0; k < N / 2; ++k) th[k] = ld(theta, bg * (N / 2) + k, in_f64);
+      for (int64_t k = 0; k < N / 2; ++k)
+        th[k] = ld(theta, (b * tgroups(d) + tgroup(d, h)) * (N / 2) + k, in_f64);
       for (int64_t i = 0; i < R * N; ++i) {
         Bt[i] = ld(B_t, bg * R * N + i, in_f64);
         Ct[i] = ld(C_t, bg * R * N + i, in_f64);
@@ -379,7 +392,7 @@ int m3o_scan_mask(const m3o_dims* d, const double* x, const double* dt,
     for (int64_t h = 0; h < H; ++h) {
       int64_t g = h / (H / G);
 #define MU(tok) (dt[(b * L + (tok)) * H + h] * (A[(b * L + (tok)) * H + h] + \
-                 I * theta[((b * L + (tok)) * G + g) * (N / 2) + k]))
+                 I * theta[((b * L + (tok)) * tgroups(d) + tgroup(d, h)) * (N / 2) + k]))
       if (y)
         for (int64_t t = 0; t < L; ++t)
           for (int64_t i = 0; i < R * P; ++i) y[((b * L + t) * H + h) * R * P + i] = 0.0;
@@ -500,7 +513,8 @@ int m3o_scan_rope(const m3o_dims* d, const double* x, const double* dt,
         Lam[t] = lsum;
         for (int64_t k = 0; k < N / 2; ++k) {
           double prev = t ? Phi[(t - 1) * (N / 2) + k] : 0.0;
-          Phi[t * (N / 2) + k] = prev + dt[bt * H + h] * theta[(bt * G + g) * (N / 2) + k];
+          Phi[t * (N / 2) + k] =
+              prev + dt[bt * H + h] * theta[(bt * tgroups(d) + tgroup(d, h)) * (N / 2) + k];
         }
         for (int64_t r = 0; r < R; ++r)
           for (int64_t k = 0; k < N / 2; ++k) {

@@ -386,3 +386,59 @@ def test_pins_catch_planted_mistake(m):
             if not err <= tol:
                 failed.append(name)
     assert failed, f"mutation {m} ({MUTATIONS[m]}) passed every pin"
+
+
+# ---- per-head angle rates (theta [b][L][H][N/2], a layout variant) ----------
+
+def test_per_head_theta_equal_across_group_matches_grouped():
+    """theta given per head, but equal for the heads of each group, gives the
+    grouped result exactly (the two layouts index the same rates)."""
+    d = rand_problem(901, H=4, G=2)
+    y0, h0 = run(d)
+    per_head = dict(d, theta=np.repeat(d["theta"], 2, axis=2))  # head h -> group h // 2
+    y1, h1 = run(per_head)
+    assert np.array_equal(y0, y1) and np.array_equal(h0, h1)
+
+
+def test_per_head_theta_each_head_matches_its_own_problem():
+    """With distinct per-head rates, every head equals an independent one-head
+    problem that takes that head's rates as its (shared) theta."""
+    d = rand_problem(902, H=4, G=1)
+    rng = np.random.default_rng(903)
+    d["theta"] = rng.uniform(-np.pi, np.pi, (2, 11, 4, 3))
+    y, hL = run(d)
+    for h in range(4):
+        one = dict(x=d["x"][:, :, h:h + 1], dt=d["dt"][:, :, h:h + 1],
+                   A=d["A"][:, :, h:h + 1], lam=d["lam"][:, :, h:h + 1],
+                   theta=d["theta"][:, :, h:h + 1], B=d["B"], C=d["C"],
+                   h0=d["h0"][:, h:h + 1], B_prev=d["B_prev"], x_prev=d["x_prev"][:, h:h + 1])
+        y1, h1 = run(one)
+        assert rel(y[:, :, h:h + 1], y1) < 1e-13 and rel(hL[:, h:h + 1], h1) < 1e-13
+
+
+def test_per_head_theta_forms_agree():
+    """The mask form and the RoPE form read per-head rates the same way."""
+    d = rand_problem(904, H=4, G=2, L=9)
+    rng = np.random.default_rng(905)
+    d["theta"] = rng.uniform(-np.pi, np.pi, (2, 9, 4, 3))
+    y, hL = run(d)
+    for name in ("scan_mask", "scan_rope"):
+        yf, hf = getattr(oracle, name)(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"],
+                                       d["C"], d["h0"], d["B_prev"], d["x_prev"])
+        assert rel(yf, y) < 1e-11 and rel(hf, hL) < 1e-11, name
+
+
+def test_per_head_theta_decode_matches_scan():
+    d = rand_problem(906, H=4, G=2, L=5)
+    rng = np.random.default_rng(907)
+    d["theta"] = rng.uniform(-np.pi, np.pi, (2, 5, 4, 3))
+    y, hL = run(d)
+    st = d["h0"]
+    for t in range(5):
+        Bp = d["B_prev"] if t == 0 else d["B"][:, t - 1]
+        xp = d["x_prev"] if t == 0 else d["x"][:, t - 1]
+        yt, st = oracle.decode_step(st, d["x"][:, t], d["dt"][:, t], d["A"][:, t],
+                                    d["lam"][:, t], d["theta"][:, t], d["B"][:, t],
+                                    d["C"][:, t], Bp, xp, f64=True)
+        assert rel(yt, y[:, t]) < 1e-12
+    assert rel(st, hL) < 1e-12
