@@ -31,6 +31,7 @@
  *       B, C              [batch][seqlen][ngroups][rank][dstate]   io dtype
  *       dt, A, lam        [batch][seqlen][nheads]                  fp32
  *       theta             [batch][seqlen][ngroups][dstate/2]       fp32
+ *                         ([batch][seqlen][nheads][dstate/2] with M3_FLAG_THETA_PER_HEAD)
  *       h0, final_state   [batch][nheads][dstate][headdim]         fp32
  *       B_prev            [batch][ngroups][rank][dstate]           io dtype
  *       x_prev            [batch][nheads][rank][headdim]           io dtype
@@ -87,6 +88,9 @@ typedef enum {
  * ends, reports its status and leaves the context usable.  Ignored by the
  * CUDA-core path and by m3_decode_step. */
 #define M3_FLAG_TEST_TIMEOUT 2u
+/* theta holds one angle-rate vector per head: [b][L][H][N/2] for the scan,
+ * [b][H][N/2] for the decode step (default: per group, like B and C). */
+#define M3_FLAG_THETA_PER_HEAD 4u
 
 typedef struct {
   int64_t batch;    /* b >= 1                                   */
@@ -164,7 +168,8 @@ M3_API int m3_scan_fwd(const m3_shape* shape, const void* x, const float* dt,
  *   state_out  [b][H][N][P] fp32; may equal state_in (in-place update), but
  *              must not partially overlap it.
  *   x_t        [b][H][R][P] io dtype;  dt_t, A_t, lam_t [b][H] fp32;
- *   theta_t    [b][G][N/2] fp32;      B_t, C_t [b][G][R][N] io dtype.
+ *   theta_t    [b][G][N/2] fp32 ([b][H][N/2] with M3_FLAG_THETA_PER_HEAD);
+ *   B_t, C_t [b][G][R][N] io dtype.
  *   B_prev,
  *   x_prev     previous token's B [b][G][R][N] and x [b][H][R][P]; both NULL
  *              for a zero left endpoint.

@@ -163,7 +163,8 @@ __global__ void __launch_bounds__(kThreads, DecodeOcc<R>::value) decode_kernel(c
     }
     bulk_load(ops + 3 * opsB, static_cast<const char*>(a.x) + hd * opsX, opsX, &bars[bi]);
     if (prev) bulk_load(ops + 3 * opsB + opsX, static_cast<const char*>(a.x_prev) + hd * opsX, opsX, &bars[bi]);
-    bulk_load(ops + 3 * opsB + 2 * opsX, a.theta + bg * K, (uint32_t)(K * 4), &bars[bi]);
+    const int64_t tgi = (hd / H) * a.tgroups + (hd % H) / (H / a.tgroups);  // theta group
+    bulk_load(ops + 3 * opsB + 2 * opsX, a.theta + tgi * K, (uint32_t)(K * 4), &bars[bi]);
   };
 
   const int PV = P / 4;                     // float4 columns of a state row
@@ -376,6 +377,7 @@ __global__ void __launch_bounds__(kStreamThreads, 7) stream_decode_kernel(const 
   const int64_t bh = blockIdx.x;
   const int64_t h = bh % a.nheads, b = bh / a.nheads;
   const int64_t bg = b * a.ngroups + h / (a.nheads / a.ngroups);
+  const int64_t tgi = b * a.tgroups + h / (a.nheads / a.tgroups);  // theta group
   const int tid = threadIdx.x;
 
   extern __shared__ float smf[];
@@ -413,7 +415,7 @@ __global__ void __launch_bounds__(kStreamThreads, 7) stream_decode_kernel(const 
   }
   for (int k = tid; k < K; k += kStreamThreads) {
     float sn, cs;
-    sincosf(dt * a.theta[bg * K + k], &sn, &cs);
+    sincosf(dt * a.theta[tgi * K + k], &sn, &cs);
     s_ac[k] = alpha * cs;
     s_as[k] = alpha * sn;
   }

@@ -23,7 +23,8 @@ int check_common(const m3_shape* s) {
     return M3_ERR_INVALID_ARGUMENT;
   if (s->dstate % 2 != 0 || s->nheads % s->ngroups != 0) return M3_ERR_INVALID_ARGUMENT;
   if (s->io_dtype != M3_F32 && s->io_dtype != M3_BF16) return M3_ERR_INVALID_ARGUMENT;
-  if ((s->flags & ~(M3_FLAG_SIMT | M3_FLAG_TEST_TIMEOUT)) != 0) return M3_ERR_INVALID_ARGUMENT;
+  if ((s->flags & ~(M3_FLAG_SIMT | M3_FLAG_TEST_TIMEOUT | M3_FLAG_THETA_PER_HEAD)) != 0)
+    return M3_ERR_INVALID_ARGUMENT;
   // supported set
   if (!is_pow2(s->dstate) || s->dstate < 16 || s->dstate > 256) return M3_ERR_UNSUPPORTED;
   if (!is_pow2(s->headdim) || s->headdim < 16 || s->headdim > 128) return M3_ERR_UNSUPPORTED;
@@ -49,6 +50,7 @@ ScanArgs make_scan_args(const m3_shape* s) {
   a.nchunks = (s->seqlen + s->chunk - 1) / s->chunk;
   a.bf16 = s->io_dtype == M3_BF16;
   a.test_timeout = (s->flags & M3_FLAG_TEST_TIMEOUT) != 0;
+  a.tgroups = (s->flags & M3_FLAG_THETA_PER_HEAD) ? s->nheads : s->ngroups;
   return a;
 }
 
@@ -194,6 +196,7 @@ M3_API int m3_decode_step(const m3_shape* s, const float* state_in, float* state
   memset(&a, 0, sizeof(a));
   a.batch = s->batch; a.nheads = s->nheads; a.ngroups = s->ngroups;
   a.P = s->headdim; a.N = s->dstate; a.R = s->rank; a.bf16 = bf16;
+  a.tgroups = (s->flags & M3_FLAG_THETA_PER_HEAD) ? s->nheads : s->ngroups;
   a.state_in = state_in; a.state_out = state_out; a.x = x_t; a.dt = dt_t; a.A = A_t;
   a.lam = lam_t; a.theta = theta_t; a.B = B_t; a.C = C_t; a.B_prev = B_prev;
   a.x_prev = x_prev; a.y = y_t;

@@ -42,6 +42,7 @@ struct ScanArgs {
   size_t ws_bytes;
   int* status;        // device-side error word
   bool test_timeout;  // M3_FLAG_TEST_TIMEOUT
+  int64_t tgroups;    // theta groups: ngroups, or nheads (M3_FLAG_THETA_PER_HEAD)
 };
 
 struct DecodeArgs {
@@ -60,6 +61,7 @@ struct DecodeArgs {
   const void* x_prev;
   void* y;
   int* status;  // device status word (timeouts)
+  int64_t tgroups;  // theta groups: ngroups, or nheads (M3_FLAG_THETA_PER_HEAD)
 };
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }

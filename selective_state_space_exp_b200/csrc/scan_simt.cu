@@ -32,7 +32,7 @@ constexpr int kTileRows = 64;  // (token, rank) rows of B / x per staged tile
 constexpr int kOutRows = 32;   // (token, rank) output rows per chunk-output CTA
 
 struct Geo {
-  int64_t b, h, g, c, t0;  // t0: first token of the chunk
+  int64_t b, h, g, tg, c, t0;  // g: B/C group, tg: theta group, t0: first token of the chunk
   int nt;                  // valid tokens in the chunk
 };
 
@@ -41,6 +41,7 @@ __device__ __forceinline__ Geo chunk_geo(const ScanArgs& a, int64_t c) {
   q.b = blockIdx.z;
   q.h = blockIdx.y;
   q.g = q.h / (a.nheads / a.ngroups);
+  q.tg = q.h / (a.nheads / a.tgroups);
   q.c = c;
   q.t0 = c * a.Q;
   int64_t rem = a.seqlen - q.t0;
@@ -75,7 +76,7 @@ __device__ void chunk_prep(const ScanArgs& a, const Geo& q, float* lcum, float* 
   for (int k = threadIdx.x; k < K; k += blockDim.x) {
     float acc = 0.f;
     for (int i = 0; i < q.nt; ++i) {
-      acc += dts[i] * a.theta[((q.b * L + q.t0 + i) * a.ngroups + q.g) * K + k];
+      acc += dts[i] * a.theta[((q.b * L + q.t0 + i) * a.tgroups + q.tg) * K + k];
       phi[i * K + k] = acc;
     }
   }

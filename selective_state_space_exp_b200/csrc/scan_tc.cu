@@ -190,6 +190,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   const int64_t seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int64_t L = a.seqlen, H = a.nheads, G = a.ngroups;
   const int64_t g = h / (H / G);
+  const int64_t tg = h / (H / a.tgroups);  // theta group
 
   if (warp == 0) {
     tmem_alloc(s_tmem, C::TMEM_COLS);
@@ -271,7 +272,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     if (cn >= c_end || tid != 0) return;
     mbar_expect_tx(s_tbT, Q * kPairs * 4);
     tpendT = true;
-    tma_load_3d(s_th, &maps.th, 0, (int)g, (int)(b * L + cn * Q), s_tbT);
+    tma_load_3d(s_th, &maps.th, 0, (int)tg, (int)(b * L + cn * Q), s_tbT);
   };
   // The gates go to registers of the gate threads one chunk ahead (plain
   // loads: the prologue that uses them runs a whole chunk later): token tid's
@@ -897,7 +898,7 @@ bool make_maps(const ScanArgs& a, TcMaps* m) {
                   R, Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
          encode3d(&m->c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.C, kN, a.ngroups * a.R, tok, 64,
                   R, Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         encode3d(&m->th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.theta, kPairs, a.ngroups, tok,
+         encode3d(&m->th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.theta, kPairs, a.tgroups, tok,
                   kPairs, 1, Q, CU_TENSOR_MAP_SWIZZLE_NONE) &&
          encode_nd(&m->y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.y, 4, yd, yb,
                    CU_TENSOR_MAP_SWIZZLE_128B);

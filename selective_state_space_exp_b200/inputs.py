@@ -55,6 +55,7 @@ class Workload:
     decay: str = "fast"      # "fast" or "slow"
     with_h0: bool = False
     with_prev: bool = False
+    theta_per_head: bool = False  # theta [..][H][N/2] instead of [..][G][N/2]
 
 
 # The five workloads the layer is measured and checked on.
@@ -98,8 +99,9 @@ def _bc(g, s: Shape, lead: tuple, kind: str, device, bias=None):
     return v + bias
 
 
-def draw_token_gates(g, s: Shape, lead: tuple, decay: str, device):
-    """dt, A, lam with shape lead + (H,), theta with shape lead + (G, N/2)."""
+def draw_token_gates(g, s: Shape, lead: tuple, decay: str, device, theta_per_head=False):
+    """dt, A, lam with shape lead + (H,), theta with shape lead + (G, N/2)
+    (lead + (H, N/2) for per-head angle rates)."""
     H = s.nheads
     dt = torch.nn.functional.softplus(_normal(g, lead + (H,), -2.0, 0.5, device))
     if decay == "slow":
@@ -107,7 +109,8 @@ def draw_token_gates(g, s: Shape, lead: tuple, decay: str, device):
     else:
         A = -torch.exp(_uniform(g, lead + (H,), 0.0, math.log(16.0), device))
     lam = torch.sigmoid(_normal(g, lead + (H,), 0.0, 1.0, device))
-    theta = _uniform(g, lead + (s.ngroups, s.dstate // 2), -math.pi, math.pi, device)
+    tg = s.nheads if theta_per_head else s.ngroups
+    theta = _uniform(g, lead + (tg, s.dstate // 2), -math.pi, math.pi, device)
     return dt.contiguous(), A.contiguous(), lam.contiguous(), theta.contiguous()
 
 
@@ -122,7 +125,7 @@ def make_scan_inputs(w: Workload, seed: int, device: str | torch.device = "cpu")
     if w.bc == "rmsnorm":
         bias = _normal(g, (s.ngroups, s.rank, s.dstate), 0.0, 0.1, device)
     x = _normal(g, lead + (s.nheads, s.rank, s.headdim), 0.0, 1.0, device)
-    dt, A, lam, theta = draw_token_gates(g, s, lead, w.decay, device)
+    dt, A, lam, theta = draw_token_gates(g, s, lead, w.decay, device, w.theta_per_head)
     B = _bc(g, s, lead, w.bc, device, bias)
     C = _bc(g, s, lead, w.bc, device, bias)
     out = dict(x=_round_io(x, s.io), B=_round_io(B, s.io), C=_round_io(C, s.io),
@@ -151,7 +154,7 @@ def make_decode_inputs(w: Workload, seed: int, steps: int,
     state0 = _normal(g, (s.batch, s.nheads, s.dstate, s.headdim), 0.0, 1.0, device)
     lead = (steps, s.batch)
     x = _normal(g, lead + (s.nheads, s.rank, s.headdim), 0.0, 1.0, device)
-    dt, A, lam, theta = draw_token_gates(g, s, lead, w.decay, device)
+    dt, A, lam, theta = draw_token_gates(g, s, lead, w.decay, device, w.theta_per_head)
     B = _bc(g, s, lead, w.bc, device, bias)
     C = _bc(g, s, lead, w.bc, device, bias)
     B_prev = _bc(g, s, (s.batch,), w.bc, device, bias)

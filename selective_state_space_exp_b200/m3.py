@@ -20,6 +20,17 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "m3.h")
 M3_F32, M3_BF16 = 0, 1
 M3_FLAG_SIMT = 1
 M3_FLAG_TEST_TIMEOUT = 2
+M3_FLAG_THETA_PER_HEAD = 4
+
+
+def theta_flag(theta_groups: int, ngroups: int, nheads: int) -> int:
+    """M3_FLAG_THETA_PER_HEAD when theta's group dimension is the head count
+    (and differs from the B/C group count), 0 when it is the group count."""
+    if theta_groups == ngroups:
+        return 0
+    if theta_groups == nheads:
+        return M3_FLAG_THETA_PER_HEAD
+    raise ValueError(f"theta has {theta_groups} groups: expected {ngroups} or {nheads}")
 STATUS = {0: "M3_OK", -1: "M3_ERR_INVALID_ARGUMENT", -2: "M3_ERR_UNSUPPORTED",
           -3: "M3_ERR_ALIGNMENT", -4: "M3_ERR_WORKSPACE", -5: "M3_ERR_CUDA",
           -6: "M3_ERR_TIMEOUT"}
@@ -112,10 +123,14 @@ def make_shape(batch, seqlen, nheads, ngroups, headdim, dstate, rank, chunk, io_
                  M3_FLAG_SIMT if simt else 0)
 
 
-def scan_shape(x: torch.Tensor, B: torch.Tensor, chunk: int, simt=False) -> Shape:
+def scan_shape(x: torch.Tensor, B: torch.Tensor, chunk: int, simt=False, theta=None) -> Shape:
+    """Shape of a scan call; theta (if given) decides grouped or per-head rates."""
     b, L, H, R, P = x.shape
     G, N = B.shape[2], B.shape[4]
-    return make_shape(b, L, H, G, P, N, R, chunk, x.dtype, simt)
+    s = make_shape(b, L, H, G, P, N, R, chunk, x.dtype, simt)
+    if theta is not None:
+        s.flags |= theta_flag(theta.shape[2], G, H)
+    return s
 
 
 def workspace_size(shape: Shape) -> int:
@@ -139,7 +154,7 @@ def m3_scan_fwd(x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None, B_prev=Non
     """Chunked prefill scan.  x [b][L][H][R][P] (io dtype), dt/A/lam [b][L][H],
     theta [b][L][G][N/2] fp32, B/C [b][L][G][R][N] (io dtype).  R is x.shape[3].
     extra_flags: further M3_FLAG_* bits (diagnostics).  Returns (y, final_state)."""
-    shape = scan_shape(x, B, chunk, simt)
+    shape = scan_shape(x, B, chunk, simt, theta)
     shape.flags |= extra_flags
     if y is None:
         y = torch.empty_like(x)
@@ -163,7 +178,7 @@ def m3_scan_fwd_noalloc(x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None, B_
     """m3_scan_fwd without a workspace argument: the library's fixed device
     scratch (M3_NOALLOC_SCRATCH_BYTES) serves instead, for callers that cannot
     allocate device memory.  Returns (y, final_state)."""
-    shape = scan_shape(x, B, chunk, simt)
+    shape = scan_shape(x, B, chunk, simt, theta)
     if y is None:
         y = torch.empty_like(x)
     if final_state is None and want_final:
@@ -179,11 +194,12 @@ def m3_scan_fwd_noalloc(x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None, B_
 def m3_decode_step(state, x_t, dt, A, lam, theta, B_t, C_t, B_prev=None, x_prev=None, *,
                    state_out=None, y=None, stream=None):
     """One decode step.  state [b][H][N][P] fp32; x_t [b][H][R][P]; dt/A/lam [b][H];
-    theta [b][G][N/2]; B_t/C_t [b][G][R][N].  state_out defaults to `state`
-    (in place).  Returns (y_t, state_out)."""
+    theta [b][G][N/2] (or [b][H][N/2], per head); B_t/C_t [b][G][R][N].
+    state_out defaults to `state` (in place).  Returns (y_t, state_out)."""
     b, H, R, P = x_t.shape
     G, N = B_t.shape[1], B_t.shape[3]
     shape = make_shape(b, 1, H, G, P, N, R, 64, x_t.dtype)
+    shape.flags |= theta_flag(theta.shape[1], G, H)
     if state_out is None:
         state_out = state
     if y is None:

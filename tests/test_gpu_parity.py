@@ -314,3 +314,40 @@ def test_gpu_rejects_bad_pointers():
                        inp["C"], 64, workspace=ws)
     assert e.value.status == -4
     assert m3.m3_stream_status() == 0
+
+
+# ---- per-head angle rates (theta [b][L][H][N/2]) -----------------------------
+
+@pytest.mark.parametrize("R,chunk,L,batch,H,G,simt", [
+    (1, 64, 300, 2, 8, 1, False),    # tensor-core path, one tile per chunk
+    (4, 64, 200, 1, 4, 1, False),    # tensor-core path, two tiles, several segments
+    (2, 32, 130, 2, 4, 2, False),    # tensor-core path, two groups
+    (2, 32, 130, 2, 4, 2, True),     # CUDA-core path
+])
+def test_per_head_theta_scan(R, chunk, L, batch, H, G, simt):
+    """Per-head angle rates through both prefill paths against the oracle."""
+    io = "bf16"
+    w = I.Workload(I.Shape(batch, L, H, 64, 128, R, G, chunk, io), decay="slow", with_h0=True,
+                   with_prev=True, theta_per_head=True)
+    inp = I.make_scan_inputs(w, seed=8000 + 10 * R + L + (1 if simt else 0))
+    assert inp["theta"].shape[2] == H
+    check(compare_scan(inp, chunk, io, simt=simt), io)
+
+
+def test_per_head_theta_scan_fp32_small():
+    w = I.Workload(I.Shape(2, 150, 4, 16, 32, 2, 2, 32, "f32"), bc="normal", with_h0=True,
+                   with_prev=True, theta_per_head=True)
+    inp = I.make_scan_inputs(w, seed=8100)
+    check(compare_scan(inp, 32, "f32"), "f32")
+
+
+@pytest.mark.parametrize("R", [1, 4])
+def test_per_head_theta_decode(R):
+    """Both decode kernels (rank 1 streams, rank 4 pipelines) with per-head rates."""
+    w = I.Workload(I.Shape(4, 1, 8, 64, 128, R, 2, 64, "bf16"), with_h0=True, with_prev=True,
+                   theta_per_head=True)
+    dec = I.make_decode_inputs(w, seed=8200 + R, steps=4)
+    assert dec["theta"].shape[2] == 8
+    yg, hg = gpu_decode(dec, 4)
+    yo, ho = oracle_scan(decode_as_scan(dec))
+    check((rel_err(yg, yo), rel_err(hg, ho)), "bf16")
