@@ -212,6 +212,49 @@ M3_API int m3_scan_fwd_noalloc(const m3_shape* shape, const void* x, const float
                                const void* B_prev, const void* x_prev, void* y,
                                float* final_state, m3_stream_t stream);
 
+/* ---- sequence split across ranks (context parallel) -------------------------
+ * Over a segment of tokens the recurrence unrolls (PaperWeekly page section
+ * 2.2, exponential-trapezoidal step; section 2.1, rotation) to
+ *   h_end = exp(Lam_seg) Rot(Phi_seg) h_start + T,
+ * Lam_seg = sum_t dt_t A_t, Phi_seg,k = sum_t dt_t theta_{t,k}, and T the
+ * segment's end state from a zero start.  A rank holding one segment of every
+ * sequence calls m3_scan_state (T), m3_segment_totals (Lam_seg, Phi_seg),
+ * exchanges them, folds the earlier segments' summaries into its incoming
+ * state with m3_state_fold and calls m3_scan_fwd from that state.  These
+ * calls have no counterpart on the pages beyond that identity. */
+
+/* Workspace of m3_scan_state (may differ from m3_scan_fwd's). */
+M3_API int m3_scan_state_workspace_size(const m3_shape* shape, size_t* bytes);
+
+/* The state after the last token of every sequence, final_state
+ * [b][H][N][P] fp32 (required), from h0 (nullable: zero) and
+ * B_prev / x_prev (nullable), without computing y.  Arguments, layouts,
+ * alignment and errors as m3_scan_fwd; y is not taken. */
+M3_API int m3_scan_state(const m3_shape* shape, const void* x, const float* dt, const float* A,
+                         const float* lam, const float* theta, const void* B, const void* C,
+                         const float* h0, const void* B_prev, const void* x_prev,
+                         float* final_state, void* workspace, size_t workspace_bytes,
+                         m3_stream_t stream);
+
+/* Segment totals: lam_tot [b][H] = sum_t dt_t A_t and phi_tot [b][H][N/2] =
+ * sum_t dt_t theta_{t,k} over the shape's seqlen tokens, accumulated in fp64
+ * and written fp32.  dt, A, theta as for m3_scan_fwd (4-byte aligned device
+ * pointers); outputs 4-byte aligned device arrays owned by the caller. */
+M3_API int m3_segment_totals(const m3_shape* shape, const float* dt, const float* A,
+                             const float* theta, float* lam_tot, float* phi_tot,
+                             m3_stream_t stream);
+
+/* Fold nseg >= 0 segment summaries in order:
+ *   h = h0 (nullable: zero);  for s < nseg: h = Rot(phi_tot[s]) exp(lam_tot[s]) h + T[s];
+ *   out = h.
+ * T [nseg][b][H][N][P], lam_tot [nseg][b][H], phi_tot [nseg][b][H][N/2], h0
+ * and out [b][H][N][P], all fp32 device arrays, 16-byte aligned (T, h0,
+ * out) or 4-byte aligned (the totals); out must not overlap the inputs.
+ * shape->seqlen and shape->chunk are ignored. */
+M3_API int m3_state_fold(const m3_shape* shape, int64_t nseg, const float* h0, const float* T,
+                         const float* lam_tot, const float* phi_tot, float* out,
+                         m3_stream_t stream);
+
 /* Waits for `stream`, then reports the first error since the previous call:
  * M3_ERR_CUDA for a CUDA fault, M3_ERR_TIMEOUT if a bounded device-side wait
  * gave up, else M3_OK.  Clears the library's device-side error word. */

@@ -101,7 +101,9 @@ M3_API const char* m3_status_string(int st) {
 
 M3_API int m3_check_shape(const m3_shape* s) { return check_common(s); }
 
-M3_API int m3_scan_workspace_size(const m3_shape* s, size_t* bytes) {
+namespace {
+
+int workspace_query(const m3_shape* s, size_t* bytes, bool state_only) {
   int st = check_common(s);
   if (st != M3_OK) return st;
   if (!bytes) return M3_ERR_INVALID_ARGUMENT;
@@ -110,8 +112,19 @@ M3_API int m3_scan_workspace_size(const m3_shape* s, size_t* bytes) {
     return M3_OK;
   }
   ScanArgs a = make_scan_args(s);
+  a.state_only = state_only;
   *bytes = scan_workspace(s, a);
   return M3_OK;
+}
+
+}  // namespace
+
+M3_API int m3_scan_workspace_size(const m3_shape* s, size_t* bytes) {
+  return workspace_query(s, bytes, false);
+}
+
+M3_API int m3_scan_state_workspace_size(const m3_shape* s, size_t* bytes) {
+  return workspace_query(s, bytes, true);
 }
 
 M3_API int m3_scan_plan(const m3_shape* s, int* tensor_core, int64_t* segments, int* launches) {
@@ -126,19 +139,23 @@ M3_API int m3_scan_plan(const m3_shape* s, int* tensor_core, int64_t* segments, 
   return M3_OK;
 }
 
-M3_API int m3_scan_fwd(const m3_shape* s, const void* x, const float* dt, const float* A,
-                       const float* lam, const float* theta, const void* B, const void* C,
-                       const float* h0, const void* B_prev, const void* x_prev, void* y,
-                       float* final_state, void* workspace, size_t workspace_bytes,
-                       m3_stream_t stream) {
+namespace {
+
+// m3_scan_fwd and m3_scan_state: state_only skips y (and needs final_state).
+int scan_call(const m3_shape* s, const void* x, const float* dt, const float* A,
+              const float* lam, const float* theta, const void* B, const void* C,
+              const float* h0, const void* B_prev, const void* x_prev, void* y,
+              float* final_state, void* workspace, size_t workspace_bytes, m3_stream_t stream,
+              bool state_only) {
   int st = check_common(s);
   if (st != M3_OK) return st;
   if ((B_prev == nullptr) != (x_prev == nullptr)) return M3_ERR_INVALID_ARGUMENT;
+  if (state_only && !final_state) return M3_ERR_INVALID_ARGUMENT;
   const bool bf16 = s->io_dtype == M3_BF16;
   if (bf16 && s->headdim % 8 != 0) return M3_ERR_UNSUPPORTED;
-  if (s->seqlen > 0 && (!x || !dt || !A || !lam || !theta || !B || !C || !y))
+  if (s->seqlen > 0 && (!x || !dt || !A || !lam || !theta || !B || !C || (!y && !state_only)))
     return M3_ERR_INVALID_ARGUMENT;
-  const void* v16[] = {x, B, C, y, h0, final_state, B_prev, x_prev, theta};
+  const void* v16[] = {x, B, C, state_only ? nullptr : y, h0, final_state, B_prev, x_prev, theta};
   for (const void* p : v16)
     if (p && !aligned(p, 16)) return M3_ERR_ALIGNMENT;
   const void* v4[] = {dt, A, lam};
@@ -155,15 +172,78 @@ M3_API int m3_scan_fwd(const m3_shape* s, const void* x, const float* dt, const 
   }
 
   ScanArgs a = make_scan_args(s);
+  a.state_only = state_only;
   const size_t need = scan_workspace(s, a);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
     return M3_ERR_WORKSPACE;
   a.x = x; a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.B = B; a.C = C;
-  a.h0 = h0; a.B_prev = B_prev; a.x_prev = x_prev; a.y = y; a.final_state = final_state;
+  a.h0 = h0; a.B_prev = B_prev; a.x_prev = x_prev; a.y = state_only ? nullptr : y;
+  a.final_state = final_state;
   a.ws = static_cast<char*>(workspace);
   a.ws_bytes = workspace_bytes;
   if (status_word(&a.status) != M3_OK) return M3_ERR_CUDA;
   cudaError_t e = use_tc(s, a) ? tc_scan_launch(a, cs) : simt_scan_launch(a, cs);
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+}  // namespace
+
+M3_API int m3_scan_fwd(const m3_shape* s, const void* x, const float* dt, const float* A,
+                       const float* lam, const float* theta, const void* B, const void* C,
+                       const float* h0, const void* B_prev, const void* x_prev, void* y,
+                       float* final_state, void* workspace, size_t workspace_bytes,
+                       m3_stream_t stream) {
+  return scan_call(s, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev, y, final_state, workspace,
+                   workspace_bytes, stream, false);
+}
+
+M3_API int m3_scan_state(const m3_shape* s, const void* x, const float* dt, const float* A,
+                         const float* lam, const float* theta, const void* B, const void* C,
+                         const float* h0, const void* B_prev, const void* x_prev,
+                         float* final_state, void* workspace, size_t workspace_bytes,
+                         m3_stream_t stream) {
+  return scan_call(s, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev, nullptr, final_state,
+                   workspace, workspace_bytes, stream, true);
+}
+
+M3_API int m3_segment_totals(const m3_shape* s, const float* dt, const float* A,
+                             const float* theta, float* lam_tot, float* phi_tot,
+                             m3_stream_t stream) {
+  int st = check_common(s);
+  if (st != M3_OK) return st;
+  if (!lam_tot || !phi_tot) return M3_ERR_INVALID_ARGUMENT;
+  if (s->seqlen > 0 && (!dt || !A || !theta)) return M3_ERR_INVALID_ARGUMENT;
+  const void* v4[] = {dt, A, theta, lam_tot, phi_tot};
+  for (const void* p : v4)
+    if (p && !aligned(p, 4)) return M3_ERR_ALIGNMENT;
+  ScanArgs a = make_scan_args(s);
+  a.dt = dt; a.A = A; a.theta = theta;
+  cudaError_t e = segment_totals_launch(a, lam_tot, phi_tot, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+M3_API int m3_state_fold(const m3_shape* s, int64_t nseg, const float* h0, const float* T,
+                         const float* lam_tot, const float* phi_tot, float* out,
+                         m3_stream_t stream) {
+  int st = check_common(s);
+  if (st != M3_OK) return st;
+  if (nseg < 0 || !out || (nseg > 0 && (!T || !lam_tot || !phi_tot))) return M3_ERR_INVALID_ARGUMENT;
+  const void* v16[] = {h0, T, out};
+  for (const void* p : v16)
+    if (p && !aligned(p, 16)) return M3_ERR_ALIGNMENT;
+  const void* v4[] = {lam_tot, phi_tot};
+  for (const void* p : v4)
+    if (p && !aligned(p, 4)) return M3_ERR_ALIGNMENT;
+  // out must not overlap the inputs
+  const size_t sb = sizeof(float) * s->batch * s->nheads * s->dstate * s->headdim;
+  const char* o0 = reinterpret_cast<const char*>(out);
+  auto overlaps = [&](const void* p, size_t n) {
+    const char* c = reinterpret_cast<const char*>(p);
+    return p && c < o0 + sb && o0 < c + n;
+  };
+  if (overlaps(h0, sb) || overlaps(T, sb * (size_t)nseg)) return M3_ERR_INVALID_ARGUMENT;
+  cudaError_t e = state_fold_launch(nseg, s->batch, s->nheads, s->dstate, s->headdim, h0, T,
+                                    lam_tot, phi_tot, out, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 

@@ -43,6 +43,7 @@ struct ScanArgs {
   int* status;        // device-side error word
   bool test_timeout;  // M3_FLAG_TEST_TIMEOUT
   int64_t tgroups;    // theta groups: ngroups, or nheads (M3_FLAG_THETA_PER_HEAD)
+  bool state_only;    // m3_scan_state: the final state only, no y
 };
 
 struct DecodeArgs {
@@ -78,5 +79,12 @@ cudaError_t tc_scan_launch(const ScanArgs& a, cudaStream_t s);
 
 // Decode step.
 cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t s);
+
+// Sequence split across ranks: segment totals and the fold of summaries.
+cudaError_t segment_totals_launch(const ScanArgs& a, float* lam_tot, float* phi_tot,
+                                  cudaStream_t s);
+cudaError_t state_fold_launch(int64_t nseg, int64_t batch, int64_t nheads, int64_t N, int64_t P,
+                              const float* h0, const float* T, const float* lam_tot,
+                              const float* phi_tot, float* out, cudaStream_t s);
 
 }  // namespace m3

@@ -391,7 +391,7 @@ cudaError_t launch_all(const ScanArgs& a, cudaStream_t st) {
              (unsigned)a.batch);
   state_pass_kernel<<<pgrid, kThreads, 0, st>>>(a);
   e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || a.state_only) return e;
 
   const int64_t ypt = (kOutRows * a.P) / kThreads;  // P / 8
   if (ypt <= 2) return launch_output<R, 2>(a, st);

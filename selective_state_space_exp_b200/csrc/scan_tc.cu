@@ -111,8 +111,9 @@ struct TcMaps {
 };
 
 struct TcPlan {
-  int64_t nseg;  // segments per (b, h) chain
-  int64_t cps;   // chunks per segment
+  int64_t nseg;   // segments per (b, h) chain
+  int64_t cps;    // chunks per segment
+  int64_t slots;  // segment summaries per chain: nseg - 1, or nseg for the state only
   float* wsT;    // [b][H][nseg-1][N][P]: local end states, then incoming states
   float* wsSum;  // [b][H][nseg-1][1 + N/2]: segment log-decay and angles
 };
@@ -235,7 +236,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       }
     }
   } else {
-    const float* src = pl.wsT + (((b * H + h) * (pl.nseg - 1) + (seg - 1)) * kN + n) * kP + p0;
+    const float* src = pl.wsT + (((b * H + h) * pl.slots + (seg - 1)) * kN + n) * kP + p0;
 #pragma unroll
     for (int p = 0; p < CW; p += 4) {
       const float4 v = *reinterpret_cast<const float4*>(src + p);
@@ -750,7 +751,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
           *reinterpret_cast<float4*>(dst + p) = make_float4(gst[p], gst[p + 1], gst[p + 2], gst[p + 3]);
       }
     } else {
-      const int64_t slot = (b * H + h) * (pl.nseg - 1) + seg;
+      const int64_t slot = (b * H + h) * pl.slots + seg;
       float* dst = pl.wsT + (slot * kN + n) * kP + p0;
 #pragma unroll
       for (int p = 0; p < CW; p += 4)
@@ -773,6 +774,9 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
 // Combine segment summaries into each segment's incoming state (fp32).
 // Thread (k, p) of chain (b, h): G_0 = h0 + (1 - lam_0) dt_0 B_prev x_prev^T,
 // G_{s+1} = Rot(Phi_s) exp(Lam_s) G_s + T_s, stored over T_s.
+// TO_FINAL: fold every segment and write the chain's final state (state-only
+// calls) instead of the incoming state of each later segment.
+template <bool TO_FINAL>
 __global__ void __launch_bounds__(256) tc_seg_pass_kernel(const ScanArgs a, const TcPlan pl) {
   const int64_t b = blockIdx.z, h = blockIdx.y;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
@@ -792,8 +796,8 @@ __global__ void __launch_bounds__(256) tc_seg_pass_kernel(const ScanArgs a, cons
       g1 = fmaf(eps * io_load(a.B_prev, bb + 2 * k + 1, true), xv, g1);
     }
   }
-  for (int64_t s = 0; s + 1 < pl.nseg; ++s) {
-    const int64_t slot = (b * H + h) * (pl.nseg - 1) + s;
+  for (int64_t s = 0; s < (TO_FINAL ? pl.nseg : pl.nseg - 1); ++s) {
+    const int64_t slot = (b * H + h) * pl.slots + s;
     float* T = pl.wsT + slot * kN * kP;
     const float* su = pl.wsSum + slot * (1 + kPairs);
     const float e = expf(su[0]);
@@ -802,10 +806,16 @@ __global__ void __launch_bounds__(256) tc_seg_pass_kernel(const ScanArgs a, cons
     const float u0 = e * g0, u1 = e * g1;
     const float n0 = cs * u0 - sn * u1 + T[(2 * k) * kP + p];
     const float n1 = sn * u0 + cs * u1 + T[(2 * k + 1) * kP + p];
-    T[(2 * k) * kP + p] = n0;
-    T[(2 * k + 1) * kP + p] = n1;
+    if (!TO_FINAL) {
+      T[(2 * k) * kP + p] = n0;
+      T[(2 * k + 1) * kP + p] = n1;
+    }
     g0 = n0;
     g1 = n1;
+  }
+  if (TO_FINAL && a.final_state) {
+    a.final_state[so + (2 * k) * kP + p] = g0;
+    a.final_state[so + (2 * k + 1) * kP + p] = g1;
   }
 }
 
@@ -900,8 +910,9 @@ bool make_maps(const ScanArgs& a, TcMaps* m) {
                   R, Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
          encode3d(&m->th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.theta, kPairs, a.tgroups, tok,
                   kPairs, 1, Q, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-         encode_nd(&m->y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.y, 4, yd, yb,
-                   CU_TENSOR_MAP_SWIZZLE_128B);
+         (a.state_only ||  // no y in a state-only call
+          encode_nd(&m->y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.y, 4, yd, yb,
+                    CU_TENSOR_MAP_SWIZZLE_128B));
 }
 
 template <int R, int Q, int MODE>
@@ -919,12 +930,19 @@ cudaError_t launch_kernel(const ScanArgs& a, const TcPlan& pl, const TcMaps& map
 template <int R, int Q>
 cudaError_t launch_rq(const ScanArgs& a, TcPlan pl, cudaStream_t st) {
   TcMaps maps;
+  memset(&maps, 0, sizeof(maps));
   if (!make_maps(a, &maps)) return cudaErrorInvalidValue;
+  dim3 pg((kPairs * kP + 255) / 256, (unsigned)a.nheads, (unsigned)a.batch);
+  if (a.state_only) {  // every segment's local end state, then the fold into final_state
+    cudaError_t e = launch_kernel<R, Q, MODE_STATE>(a, pl, maps, pl.nseg, st);
+    if (e != cudaSuccess) return e;
+    tc_seg_pass_kernel<true><<<pg, 256, 0, st>>>(a, pl);
+    return cudaGetLastError();
+  }
   if (pl.nseg > 1) {
     cudaError_t e = launch_kernel<R, Q, MODE_STATE>(a, pl, maps, pl.nseg - 1, st);
     if (e != cudaSuccess) return e;
-    dim3 pg((kPairs * kP + 255) / 256, (unsigned)a.nheads, (unsigned)a.batch);
-    tc_seg_pass_kernel<<<pg, 256, 0, st>>>(a, pl);
+    tc_seg_pass_kernel<false><<<pg, 256, 0, st>>>(a, pl);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -945,16 +963,18 @@ int64_t tc_scan_segments(const ScanArgs& a) { return make_plan(a).nseg; }
 
 size_t tc_scan_workspace(const ScanArgs& a) {
   const TcPlan pl = make_plan(a);
-  if (pl.nseg <= 1) return 0;
-  const size_t slots = (size_t)a.batch * a.nheads * (pl.nseg - 1);
+  const int64_t per = a.state_only ? pl.nseg : pl.nseg - 1;
+  if (per <= 0) return 0;
+  const size_t slots = (size_t)a.batch * a.nheads * per;
   return align_up(sizeof(float) * slots * kN * kP, 256) +
          align_up(sizeof(float) * slots * (1 + kPairs), 256);
 }
 
 cudaError_t tc_scan_launch(const ScanArgs& a, cudaStream_t st) {
   TcPlan pl = make_plan(a);
-  if (pl.nseg > 1) {
-    const size_t slots = (size_t)a.batch * a.nheads * (pl.nseg - 1);
+  pl.slots = a.state_only ? pl.nseg : pl.nseg - 1;
+  if (pl.slots > 0) {
+    const size_t slots = (size_t)a.batch * a.nheads * pl.slots;
     pl.wsT = reinterpret_cast<float*>(a.ws);
     pl.wsSum = reinterpret_cast<float*>(a.ws + align_up(sizeof(float) * slots * kN * kP, 256));
   }

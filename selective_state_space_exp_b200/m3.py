@@ -84,6 +84,14 @@ def load() -> ctypes.CDLL:
             L.m3_decode_step.restype = ctypes.c_int
             L.m3_stream_status.argtypes = [vp]
             L.m3_stream_status.restype = ctypes.c_int
+            L.m3_scan_state_workspace_size.argtypes = [sp, ctypes.POINTER(ctypes.c_size_t)]
+            L.m3_scan_state_workspace_size.restype = ctypes.c_int
+            L.m3_scan_state.argtypes = [sp] + [vp] * 12 + [ctypes.c_size_t, vp]
+            L.m3_scan_state.restype = ctypes.c_int
+            L.m3_segment_totals.argtypes = [sp] + [vp] * 6
+            L.m3_segment_totals.restype = ctypes.c_int
+            L.m3_state_fold.argtypes = [sp, ctypes.c_int64] + [vp] * 6
+            L.m3_state_fold.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -189,6 +197,54 @@ def m3_scan_fwd_noalloc(x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None, B_
                                     _ptr(x_prev), _ptr(y), _ptr(final_state), _stream(stream))
     _check("m3_scan_fwd_noalloc", st)
     return y, final_state
+
+
+def m3_scan_state(x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None, B_prev=None,
+                  x_prev=None, *, final_state=None, workspace=None, simt=False, stream=None):
+    """The state after every sequence's last token, [b][H][N][P] fp32, without y."""
+    shape = scan_shape(x, B, chunk, simt, theta)
+    if final_state is None:
+        final_state = torch.empty((x.shape[0], x.shape[2], B.shape[4], x.shape[4]),
+                                  dtype=torch.float32, device=x.device)
+    n = ctypes.c_size_t(0)
+    _check("m3_scan_state_workspace_size",
+           load().m3_scan_state_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
+    if workspace is None:
+        workspace = torch.empty(max(int(n.value), 1), dtype=torch.uint8, device=x.device)
+    st = load().m3_scan_state(ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(lam),
+                              _ptr(theta), _ptr(B), _ptr(C), _ptr(h0), _ptr(B_prev),
+                              _ptr(x_prev), _ptr(final_state), _ptr(workspace),
+                              ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check("m3_scan_state", st)
+    return final_state
+
+
+def m3_segment_totals(x, dt, A, theta, B, chunk: int = 64, *, stream=None):
+    """(lam_tot [b][H], phi_tot [b][H][N/2]): sum over the tokens of dt*A and
+    of dt*theta for every (batch, head)."""
+    shape = scan_shape(x, B, chunk, False, theta)
+    b, _, H = dt.shape
+    K = B.shape[4] // 2
+    lam_tot = torch.empty((b, H), dtype=torch.float32, device=dt.device)
+    phi_tot = torch.empty((b, H, K), dtype=torch.float32, device=dt.device)
+    _check("m3_segment_totals", load().m3_segment_totals(
+        ctypes.byref(shape), _ptr(dt), _ptr(A), _ptr(theta), _ptr(lam_tot), _ptr(phi_tot),
+        _stream(stream)))
+    return lam_tot, phi_tot
+
+
+def m3_state_fold(h0, T, lam_tot, phi_tot, *, out=None, stream=None):
+    """Fold segment summaries: h = h0 (None: zero); for each s:
+    h = Rot(phi_tot[s]) exp(lam_tot[s]) h + T[s].  T [nseg][b][H][N][P]."""
+    nseg, b, H, N, P = T.shape
+    shape = make_shape(b, 1, H, 1, P, N, 1, 64, torch.float32)
+    if out is None:
+        out = torch.empty((b, H, N, P), dtype=torch.float32, device=T.device)
+    _check("m3_state_fold", load().m3_state_fold(
+        ctypes.byref(shape), ctypes.c_int64(nseg), _ptr(h0), _ptr(T) if nseg else None,
+        _ptr(lam_tot) if nseg else None, _ptr(phi_tot) if nseg else None, _ptr(out),
+        _stream(stream)))
+    return out
 
 
 def m3_decode_step(state, x_t, dt, A, lam, theta, B_t, C_t, B_prev=None, x_prev=None, *,

@@ -351,3 +351,77 @@ def test_per_head_theta_decode(R):
     yg, hg = gpu_decode(dec, 4)
     yo, ho = oracle_scan(decode_as_scan(dec))
     check((rel_err(yg, yo), rel_err(hg, ho)), "bf16")
+
+
+# ---- sequence split across ranks: state-only scan, totals, fold ----------------
+
+@pytest.mark.parametrize("R,chunk,L,batch,H,io,simt", [
+    (1, 64, 700, 1, 8, "bf16", False),   # tensor-core path, several segments per chain
+    (4, 64, 300, 2, 4, "bf16", False),   # two tiles per chunk
+    (2, 32, 250, 2, 4, "f32", True),     # CUDA-core path
+])
+def test_scan_state_matches_oracle_final_state(R, chunk, L, batch, H, io, simt):
+    N, P = (128, 64) if io == "bf16" else (32, 16)
+    w = I.Workload(I.Shape(batch, L, H, P, N, R, 1, chunk, io), decay="slow", with_h0=True,
+                   with_prev=True)
+    inp = I.make_scan_inputs(w, seed=9000 + L)
+    g = to_dev(inp)
+    hs = m3.m3_scan_state(g["x"], g["dt"], g["A"], g["lam"], g["theta"], g["B"], g["C"], chunk,
+                          g["h0"], g["B_prev"], g["x_prev"], simt=simt)
+    assert m3.m3_stream_status() == 0
+    _, ho = oracle_scan(inp)
+    assert rel_err(hs.cpu().numpy(), ho) <= TOL[io]
+
+
+def test_segment_totals_and_fold_match_numpy():
+    w = I.Workload(I.Shape(2, 300, 4, 64, 128, 2, 2, 64, "bf16"), theta_per_head=True)
+    inp = I.make_scan_inputs(w, seed=9100)
+    g = to_dev(inp)
+    lam, phi = m3.m3_segment_totals(g["x"], g["dt"], g["A"], g["theta"], g["B"], 64)
+    dt, A, th = (inp[k].double().numpy() for k in ("dt", "A", "theta"))
+    assert np.allclose(lam.cpu().numpy(), (dt * A).sum(1), rtol=1e-5, atol=1e-5)
+    assert np.allclose(phi.cpu().numpy(), (dt[..., None] * th).sum(1), rtol=1e-5, atol=1e-5)
+    rng = np.random.default_rng(9101)
+    nseg, b, H, N, P = 3, 2, 4, 128, 64
+    T = rng.standard_normal((nseg, b, H, N, P)).astype(np.float32)
+    lt = rng.uniform(-2.0, 0.0, (nseg, b, H)).astype(np.float32)
+    pt = rng.uniform(-20.0, 20.0, (nseg, b, H, N // 2)).astype(np.float32)
+    h0 = rng.standard_normal((b, H, N, P)).astype(np.float32)
+    out = m3.m3_state_fold(*(torch.from_numpy(a).cuda() for a in (h0, T, lt, pt)))
+    h = h0.astype(np.float64)
+    for s in range(nseg):
+        e = np.exp(lt[s].astype(np.float64))[:, :, None, None]
+        c, sn = np.cos(pt[s].astype(np.float64))[..., None], np.sin(pt[s].astype(np.float64))[..., None]
+        u0, u1 = e * h[:, :, 0::2], e * h[:, :, 1::2]
+        n0, n1 = c * u0 - sn * u1 + T[s][:, :, 0::2], sn * u0 + c * u1 + T[s][:, :, 1::2]
+        h = np.empty_like(h)
+        h[:, :, 0::2], h[:, :, 1::2] = n0, n1
+    assert rel_err(out.cpu().numpy(), h) <= 1e-5
+
+
+@pytest.mark.parametrize("R,world", [(1, 4), (4, 3)])
+def test_sequence_split_emulated_on_one_gpu(R, world):
+    """The sequence split driven rank by rank with the library's kernels on one
+    device; the ranks' y, in token order, and the last end state against one
+    oracle scan of the whole sequence."""
+    from selective_state_space_exp_b200.parallel import M3Ops, seq_boundary, seq_finish, seq_summary
+    L = 192 * world
+    w = I.Workload(I.Shape(1, L, 8, 64, 128, R, 1, 64, "bf16"), decay="slow", with_h0=True,
+                   with_prev=True)
+    inp = I.make_scan_inputs(w, seed=9200 + R)
+    g = to_dev(inp)
+    seq_keys = ("x", "dt", "A", "lam", "theta", "B", "C")
+    segs = [{k: (g[k][:, r * L // world:(r + 1) * L // world].contiguous() if k in seq_keys
+                 else g[k]) for k in g} for r in range(world)]
+    ops = M3Ops()
+    lasts = [seq_boundary(s["x"], s["B"]) for s in segs]
+    prevs = [(g["B_prev"], g["x_prev"])] + [lasts[r - 1] for r in range(1, world)]
+    sums = [seq_summary(ops, s["x"], s["dt"], s["A"], s["lam"], s["theta"], s["B"], s["C"], 64,
+                        *prevs[r]) for r, s in enumerate(segs)]
+    Ts, lams, phis = [t[0] for t in sums], [t[1] for t in sums], [t[2] for t in sums]
+    outs = [seq_finish(ops, r, s["x"], s["dt"], s["A"], s["lam"], s["theta"], s["B"], s["C"], 64,
+                       g["h0"], Ts, lams, phis, *prevs[r]) for r, s in enumerate(segs)]
+    assert m3.m3_stream_status() == 0
+    y = torch.cat([o[0] for o in outs], dim=1).float().cpu().numpy()
+    yo, ho = oracle_scan(inp)
+    check((rel_err(y, yo), rel_err(outs[-1][1].cpu().numpy(), ho)), "bf16")

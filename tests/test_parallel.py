@@ -59,3 +59,116 @@ def test_gloo_two_ranks():
 
 def test_single_process_reductions_are_identity():
     assert max_over_ranks(3.5) == 3.5 and sum_over_ranks(2.0) == 2.0
+
+
+# ---- sequence split across ranks (context parallel) ---------------------------
+# The host orchestration with the oracle standing in for the per-rank kernels:
+# the ranks' y, concatenated in token order, and the last rank's end state
+# must equal one oracle scan over the whole sequence.
+
+import numpy as np  # noqa: E402
+
+import oracle  # noqa: E402
+from selective_state_space_exp_b200.parallel import (seq_boundary, seq_finish,  # noqa: E402
+                                                     seq_parallel_scan, seq_summary)
+
+
+class OracleOps:
+    """Per-rank steps computed by the fp64 oracle and numpy (test stand-in)."""
+
+    def scan_state(self, x, dt, A, lam, theta, B, C, chunk, B_prev, x_prev):
+        _, hL = oracle.scan(x, dt, A, lam, theta, B, C, None, B_prev, x_prev, f64=True)
+        return torch.from_numpy(hL)
+
+    def segment_totals(self, x, dt, A, theta, B, chunk):
+        dtn, An, thn = dt.numpy(), A.numpy(), theta.numpy()
+        H, Gt = dtn.shape[2], thn.shape[2]
+        th_h = thn[:, :, np.arange(H) // (H // Gt)]
+        return (torch.from_numpy((dtn * An).sum(axis=1)),
+                torch.from_numpy((dtn[..., None] * th_h).sum(axis=1)))
+
+    def state_fold(self, h0, T, lam, phi):
+        h = np.zeros(T.shape[1:]) if h0 is None else h0.numpy().copy()
+        for s in range(T.shape[0]):
+            e = np.exp(lam[s].numpy())[:, :, None, None]
+            c = np.cos(phi[s].numpy())[..., None]
+            sn = np.sin(phi[s].numpy())[..., None]
+            u0, u1 = e * h[:, :, 0::2], e * h[:, :, 1::2]
+            n0 = c * u0 - sn * u1 + T[s].numpy()[:, :, 0::2]
+            n1 = sn * u0 + c * u1 + T[s].numpy()[:, :, 1::2]
+            h = np.empty_like(h)
+            h[:, :, 0::2], h[:, :, 1::2] = n0, n1
+        return torch.from_numpy(h)
+
+    def scan_fwd(self, x, dt, A, lam, theta, B, C, chunk, h0, B_prev, x_prev):
+        y, hL = oracle.scan(x, dt, A, lam, theta, B, C, h0, B_prev, x_prev, f64=True)
+        return torch.from_numpy(y), torch.from_numpy(hL)
+
+
+def _seq_problem(L=24, theta_per_head=False):
+    rng = np.random.default_rng(77)
+    b, H, G, P, N, R = 2, 4, 2, 3, 6, 2
+    Gt = H if theta_per_head else G
+    d = dict(x=rng.standard_normal((b, L, H, R, P)),
+             dt=np.log1p(np.exp(rng.normal(-1.0, 0.5, (b, L, H)))),
+             A=-np.exp(rng.uniform(0.0, 1.0, (b, L, H))),
+             lam=1 / (1 + np.exp(-rng.standard_normal((b, L, H)))),
+             theta=rng.uniform(-np.pi, np.pi, (b, L, Gt, N // 2)),
+             B=rng.standard_normal((b, L, G, R, N)), C=rng.standard_normal((b, L, G, R, N)),
+             h0=rng.standard_normal((b, H, N, P)), B_prev=rng.standard_normal((b, G, R, N)),
+             x_prev=rng.standard_normal((b, H, R, P)))
+    return {k: torch.from_numpy(v) for k, v in d.items()}
+
+
+def _segment(d, rank, world):
+    L = d["x"].shape[1]
+    a, b = rank * L // world, (rank + 1) * L // world
+    return {k: (v[:, a:b].contiguous() if k in ("x", "dt", "A", "lam", "theta", "B", "C") else v)
+            for k, v in d.items()}
+
+
+def _seq_worker(rank, world, port, out, theta_per_head):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        s = _segment(_seq_problem(theta_per_head=theta_per_head), rank, world)
+        y, hL = seq_parallel_scan(s["x"], s["dt"], s["A"], s["lam"], s["theta"], s["B"], s["C"],
+                                  64, s["h0"], s["B_prev"], s["x_prev"], ops=OracleOps())
+        out[rank] = (y, hL)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,theta_per_head", [(2, False), (3, True)])
+def test_gloo_sequence_split_matches_one_scan(world, theta_per_head):
+    port = _free_port()
+    out = mp.Manager().dict()
+    mp.spawn(_seq_worker, args=(world, port, out, theta_per_head), nprocs=world, join=True)
+    d = _seq_problem(theta_per_head=theta_per_head)
+    y_ref, h_ref = oracle.scan(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"], d["C"],
+                               d["h0"], d["B_prev"], d["x_prev"], f64=True)
+    y = np.concatenate([out[r][0].numpy() for r in range(world)], axis=1)
+    assert np.max(np.abs(y - y_ref)) <= 1e-10 * np.max(np.abs(y_ref))
+    hL = out[world - 1][1].numpy()
+    assert np.max(np.abs(hL - h_ref)) <= 1e-10 * np.max(np.abs(h_ref))
+
+
+def test_sequence_split_phases_in_one_process():
+    """The same phases driven rank by rank in one process (the exchange is a
+    list), as a one-device emulation does."""
+    world = 4
+    d = _seq_problem(L=20)
+    segs = [_segment(d, r, world) for r in range(world)]
+    ops = OracleOps()
+    lasts = [seq_boundary(s["x"], s["B"]) for s in segs]
+    prevs = [(d["B_prev"], d["x_prev"])] + [(lasts[r - 1][0], lasts[r - 1][1]) for r in range(1, world)]
+    sums = [seq_summary(ops, s["x"], s["dt"], s["A"], s["lam"], s["theta"], s["B"], s["C"], 64,
+                        *prevs[r]) for r, s in enumerate(segs)]
+    Ts, lams, phis = [t[0] for t in sums], [t[1] for t in sums], [t[2] for t in sums]
+    ys = [seq_finish(ops, r, s["x"], s["dt"], s["A"], s["lam"], s["theta"], s["B"], s["C"], 64,
+                     d["h0"], Ts, lams, phis, *prevs[r])[0] for r, s in enumerate(segs)]
+    y_ref, _ = oracle.scan(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"], d["C"],
+                           d["h0"], d["B_prev"], d["x_prev"], f64=True)
+    y = np.concatenate([t.numpy() for t in ys], axis=1)
+    assert np.max(np.abs(y - y_ref)) <= 1e-10 * np.max(np.abs(y_ref))
