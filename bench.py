@@ -327,10 +327,20 @@ def cpu_oracle_prefill(inp_host, s, budget_s=12.0):
         elapsed += time.perf_counter() - t0
         done += len(chains)
     tokens = done / s.nheads * s.seqlen
+    # the same oracle on one thread, on a smaller sample of the same chains
+    one = min(max(1, done // max(cores, 1)), total)
+    t0 = time.perf_counter()
+    oracle.scan(inp_host["x"], inp_host["dt"], inp_host["A"], inp_host["lam"],
+                inp_host["theta"], inp_host["B"], inp_host["C"], chains=list(range(one)),
+                nthreads=1)
+    t1 = time.perf_counter() - t0
     return {"value": round(tokens / elapsed, 1), "unit": "tokens/s", "cores": cores,
             "kind": "oracle",
             "sample": f"{done} of {total} (batch, head) chains, all {s.seqlen} tokens each, "
-                      f"{elapsed:.1f} s on {cores} threads"}
+                      f"{elapsed:.1f} s on {cores} threads",
+            "single_thread": {"value": round(one / s.nheads * s.seqlen / t1, 1),
+                              "unit": "tokens/s", "cores": 1,
+                              "sample": f"{one} chains, {t1:.1f} s"}}
 
 
 # ---- main -------------------------------------------------------------------
@@ -439,6 +449,22 @@ def main():
     tokens = s.batch * s.seqlen
     flops, byt = prefill_work(s)
 
+    # secondary line: the SISO workload with B and C per head (G = H), which
+    # moves 0.5 GB more through HBM per call
+    secondary = None
+    if args.workload == "siso_prefill":
+        s2 = dataclasses.replace(s, ngroups=s.nheads)
+        inp2 = I.make_scan_inputs(I.Workload(s2), seed=1011 + 7919 * rank, device="cuda")
+        barrier(world)
+        t2 = max_over_ranks(sum(time_prefill(inp2, s2, max(3, args.steps // 2), args.warmup,
+                                             flush)), world) / max(3, args.steps // 2)
+        f2, b2 = prefill_work(s2)
+        secondary = {"workload": "siso_prefill, B and C per head (ngroups = nheads = 64)",
+                     "value": round(world * s2.batch * s2.seqlen / t2, 1), "unit": "tokens/s",
+                     "ms_per_step": round(t2 * 1e3, 4),
+                     "roofline": roofline(f2, b2, t2, peaks, psrc)}
+        del inp2
+
     # decode (b = 128, H = 64, R as the prefill workload)
     dw = I.DECODE_MIMO if s.rank > 1 else I.DECODE_SISO
     ds = dw.shape
@@ -507,6 +533,8 @@ def main():
         "gpu_launches": args.steps * launches_per_call,
         "clocks": clk.summary(),
     }
+    if secondary is not None:
+        line["secondary"] = secondary
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_prefill(inp_host, s)
     if rank == 0:
