@@ -601,11 +601,13 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
           if (__syncthreads_or(!okb)) { aborted = true; break; }
           tc_fence_after();
         }
+        // 64-row tiles fill lanes 0-15 of each warp's TMEM quadrant: both
+        // half-warps take those 16 rows, each half 16 of the warp's columns
         const int rho0 = (MT == 64) ? 16 * qd : 32 * qd;     // the warp's first row
-        const int rho = rho0 + lane;
-        const bool live = (MT == 64) ? lane < 16 : true;
-        const int t = live ? (mt * MT + rho) / R : 0;
-        const bool trow = live && t < nt;
+        const int rho = rho0 + ((MT == 64) ? (lane & 15) : lane);
+        const int hsel = (MT == 64) ? (lane >> 4) : 0;        // column half (64-row tiles)
+        const int t = (mt * MT + rho) / R;
+        const bool trow = t < nt;
         const int t_hi = (mt * MT + rho0 + ((MT == 64) ? 15 : 31)) / R;  // the warp's last token
         const float lgt = trow ? s_lg[t] : 0.f;
         const float et = (trow && fac_ok) ? ex2(lgt - l2ref) : 0.f;
@@ -644,21 +646,37 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
             pk[j / 2] = pack_bf16(fm.x, fm.y);
           }
         };
-        for (int cc = cq * cpt / 16; cc < (cq + 1) * cpt / 16; cc += 2) {
-          const int s0 = cc * 16 / R;  // first token of these 32 columns
-          uint32_t pk[16];
+        if (MT == 64) {  // one 32-column block per warp; each half-warp masks 16 of them
+          const int c0 = cq * cpt;             // the warp's first column
+          const int cth = c0 + 16 * hsel;      // this thread's first column
+          uint32_t pk[8];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) pk[j] = 0u;
-          if (s0 <= t_hi) {  // warp-uniform: blocks wholly above the diagonal stay zero
-            uint32_t v[32];
-            tmem_ld32(tm + lane_base + C::s_col(mt) + cc * 16, v);
+          for (int j = 0; j < 8; ++j) pk[j] = 0u;
+          if (c0 / R <= t_hi) {  // warp-uniform: blocks wholly above the diagonal stay zero
+            uint32_t v[16];
+            tmem_ld16x2<16>(tm + lane_base + C::s_col(mt) + c0, v);
             tmem_ld_wait();
-            if (trow) {
-              mask16(v, s0, pk);
-              mask16(v + 16, s0 + 16 / R, pk + 8);
-            }
+            if (trow) mask16(v, cth / R, pk);
           }
-          if (live) {
+          uint8_t* blk = sm + C::p_off(mt);  // K = 64: one block
+          const int ch0 = cth / 8;
+          *reinterpret_cast<uint4*>(blk + sw128_off(rho, ch0)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(blk + sw128_off(rho, ch0 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else {
+          for (int cc = cq * cpt / 16; cc < (cq + 1) * cpt / 16; cc += 2) {
+            const int s0 = cc * 16 / R;  // first token of these 32 columns
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pk[j] = 0u;
+            if (s0 <= t_hi) {  // warp-uniform: blocks wholly above the diagonal stay zero
+              uint32_t v[32];
+              tmem_ld32(tm + lane_base + C::s_col(mt) + cc * 16, v);
+              tmem_ld_wait();
+              if (trow) {
+                mask16(v, s0, pk);
+                mask16(v + 16, s0 + 16 / R, pk + 8);
+              }
+            }
             const int kb = (cc * 16) / 64;
             uint8_t* blk = sm + C::p_off(mt) + kb * MT * 128;
             const int ch0 = ((cc * 16) % 64) / 8;
@@ -700,18 +718,29 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       // ---- epilogue: y = P x + exp(Lam_t) Ct G, staged in the w*x block --------
 #pragma unroll
       for (int mt = 0; mt < NT; ++mt) {
-        const int rho = (MT == 64) ? 16 * qd + lane : 32 * qd + lane;
-        const bool live = (MT == 64) ? lane < 16 : true;
+        // 64-row tiles: both half-warps take the warp's 16 rows, each half
+        // 16 of the thread group's columns (see the mask)
+        const int rho = (MT == 64) ? 16 * qd + (lane & 15) : 32 * qd + lane;
         const int i = mt * MT + rho;  // row (t, r) of the chunk
-        const int t = live ? i / R : 0;
-        const float el = (live && t < nt) ? ex2(s_lg[t]) : 0.f;
+        const int t = i / R;
+        const float el = (t < nt) ? ex2(s_lg[t]) : 0.f;
+        constexpr int NPC = (MT == 64) ? CW / 32 : CW / 16;  // 16-column pieces per thread
+        static_assert(MT != 64 || CW % 32 == 0, "64-row tiles: 32 columns per thread group");
 #pragma unroll
-        for (int pc = 0; pc < CW / 16; ++pc) {
+        for (int pc = 0; pc < NPC; ++pc) {
           uint32_t yv[16], zv[16];
-          tmem_ld16(tm + lane_base + C::y_col(mt) + CW * cq + 16 * pc, yv);
-          tmem_ld16(tm + lane_base + C::y2_col(mt) + CW * cq + 16 * pc, zv);
+          int col;  // this thread's first column
+          if (MT == 64) {
+            col = CW * cq + 32 * pc + 16 * (lane >> 4);
+            tmem_ld16x2<16>(tm + lane_base + C::y_col(mt) + CW * cq + 32 * pc, yv);
+            tmem_ld16x2<16>(tm + lane_base + C::y2_col(mt) + CW * cq + 32 * pc, zv);
+          } else {
+            col = CW * cq + 16 * pc;
+            tmem_ld16(tm + lane_base + C::y_col(mt) + col, yv);
+            tmem_ld16(tm + lane_base + C::y2_col(mt) + col, zv);
+          }
           tmem_ld_wait();
-          if (live) {
+          {
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
               uint32_t w4[4];
@@ -723,7 +752,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
                                        make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1])));
                 w4[e] = pack_bf16(f.x, f.y);
               }
-              *reinterpret_cast<uint4*>(sm + C::XW_OFF + sw128_off(i, (CW * cq + 16 * pc) / 8 + q)) =
+              *reinterpret_cast<uint4*>(sm + C::XW_OFF + sw128_off(i, col / 8 + q)) =
                   make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
           }
