@@ -211,6 +211,16 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   tc_fence_after();
   const uint32_t tm = *s_tmem;
   const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
+  // Operand descriptors at each region's start; an MMA's descriptor adds its
+  // byte offset / 16 to the 14-bit start-address field (shared addresses stay
+  // below 256 KB, so the field never carries).
+  const uint64_t dC = sw128_desc(sbase + C::C_OFF, 16, 1024);         // Ct, K-major
+  const uint64_t dB = sw128_desc(sbase + C::B_OFF, 16, 1024);         // Bt, K-major
+  const uint64_t dBmn = sw128_desc(sbase + C::B_OFF, C::OPB, 1024);   // Bt, MN-major
+  const uint64_t dXW = sw128_desc(sbase + C::XW_OFF, C::OPB, 1024);   // w*x, MN-major
+  const uint64_t dX = sw128_desc(sbase + C::X_OFF, C::OPB, 1024);     // x, MN-major
+  const uint64_t dG = sw128_desc(sbase + C::G_OFF, kN * 128, 1024);   // state, MN-major
+  auto dadd = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
   uint32_t phase = 0, phase1 = 0, phase1b = 0, tphT = 0, tphM = 0;
   bool aborted = false;
   bool tpendT = false, tpendM = false;  // thread 0: TMA bytes expected on s_tbT / s_tbM
@@ -515,8 +525,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4) {
-            const uint64_t ad = sw128_desc(sbase + C::C_OFF + kb * C::OPB + mt * MT * 128 + k4 * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(sbase + C::G_OFF + (kb * 4 + k4) * 2048, kN * 128, 1024);
+            const uint64_t ad = dadd(dC, kb * C::OPB + mt * MT * 128 + k4 * 32);
+            const uint64_t bd = dadd(dG, (kb * 4 + k4) * 2048);
             mma_bf16_ss(tm + C::y2_col(mt), ad, bd, id4, (kb | k4) != 0);
           }
     };
@@ -524,8 +534,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       const uint32_t id3 = idesc_bf16(kN, kP, 1, 1);
 #pragma unroll
       for (int ks = 0; ks < M / 16; ++ks) {
-        const uint64_t ad = sw128_desc(sbase + C::B_OFF + ks * 2048, C::OPB, 1024);
-        const uint64_t bd = sw128_desc(sbase + C::XW_OFF + ks * 2048, C::OPB, 1024);
+        const uint64_t ad = dadd(dBmn, ks * 2048);
+        const uint64_t bd = dadd(dXW, ks * 2048);
         mma_bf16_ss(tm + C::SC_COL, ad, bd, id3, ks != 0);
       }
       if (MODE == MODE_FULL && C::EARLY4) issue_mma4(0);
@@ -538,8 +548,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
           for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
-              const uint64_t ad = sw128_desc(sbase + C::C_OFF + kb * C::OPB + mt * MT * 128 + k4 * 32, 16, 1024);
-              const uint64_t bd = sw128_desc(sbase + C::B_OFF + kb * C::OPB + k4 * 32, 16, 1024);
+              const uint64_t ad = dadd(dC, kb * C::OPB + mt * MT * 128 + k4 * 32);
+              const uint64_t bd = dadd(dB, kb * C::OPB + k4 * 32);
               mma_bf16_ss(tm + C::s_col(mt), ad, bd, id, (kb | k4) != 0);
             }
           mma_commit(mt == 0 ? s_bar1 : s_bar1b);  // each tile's scores on their own barrier
@@ -696,8 +706,9 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
           for (int kb = 0; kb < kblocks; ++kb)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
-              const uint64_t ad = sw128_desc(sbase + C::p_off(mt) + kb * MT * 128 + k4 * 32, 16, 1024);
-              const uint64_t bd = sw128_desc(sbase + C::X_OFF + (kb * 4 + k4) * 2048, C::OPB, 1024);
+              const uint64_t ad = dadd(mt == 0 && NT == 2 ? dadd(dC, C::XW_OFF - C::C_OFF) : dB,
+                                       kb * MT * 128 + k4 * 32);  // P over w*x or Bt
+              const uint64_t bd = dadd(dX, (kb * 4 + k4) * 2048);
               mma_bf16_ss(tm + C::y_col(mt), ad, bd, id2, (kb | k4) != 0);
             }
           if (!C::EARLY4) issue_mma4(mt);
