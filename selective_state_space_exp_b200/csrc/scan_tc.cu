@@ -459,6 +459,25 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         float cs[4], sn[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) __sincosf(phi[j], &sn[j], &cs[j]);
+        // two pairs at a time as (even elements, odd elements) fp32x2 vectors:
+        // (b0, b1) -> (c b0 + s b1, c b1 - s b0) for each pair
+        const float2 c2[2] = {make_float2(cs[0], cs[1]), make_float2(cs[2], cs[3])};
+        const float2 s2[2] = {make_float2(sn[0], sn[1]), make_float2(sn[2], sn[3])};
+        const float2 n2[2] = {make_float2(-sn[0], -sn[1]), make_float2(-sn[2], -sn[3])};
+        auto rot4 = [&](const uint4 in, uint32_t (&o)[4]) {
+          const uint32_t iw[4] = {in.x, in.y, in.z, in.w};
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const float2 e = make_float2(__uint_as_float(iw[2 * q] << 16),
+                                         __uint_as_float(iw[2 * q + 1] << 16));
+            const float2 d = make_float2(__uint_as_float(iw[2 * q] & 0xffff0000u),
+                                         __uint_as_float(iw[2 * q + 1] & 0xffff0000u));
+            const float2 oe = ffma2(c2[q], e, fmul2(s2[q], d));
+            const float2 od = ffma2(c2[q], d, fmul2(n2[q], e));
+            o[2 * q] = pack_bf16(oe.x, od.x);
+            o[2 * q + 1] = pack_bf16(oe.y, od.y);
+          }
+        };
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           const uint32_t off = kboff + sw128_off(t * R + r, chk);
@@ -467,24 +486,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
           uint4 rc = make_uint4(0, 0, 0, 0);
           if (MODE == MODE_FULL) rc = *reinterpret_cast<const uint4*>(sm + C::C_OFF + off);
           if (!live_t) { rb = make_uint4(0, 0, 0, 0); rc = make_uint4(0, 0, 0, 0); }
-          const uint32_t ib[4] = {rb.x, rb.y, rb.z, rb.w};
-          const uint32_t ic[4] = {rc.x, rc.y, rc.z, rc.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            // (b0, b1) -> (c b0 + s b1, c b1 - s b0)
-            const float2 v = make_float2(__uint_as_float(ib[j] << 16),
-                                         __uint_as_float(ib[j] & 0xffff0000u));
-            const float2 w = ffma2(make_float2(cs[j], cs[j]), v,
-                                   fmul2(make_float2(sn[j], -sn[j]), make_float2(v.y, v.x)));
-            ob[j] = pack_bf16(w.x, w.y);
-            if (MODE == MODE_FULL) {
-              const float2 vc = make_float2(__uint_as_float(ic[j] << 16),
-                                            __uint_as_float(ic[j] & 0xffff0000u));
-              const float2 wc = ffma2(make_float2(cs[j], cs[j]), vc,
-                                      fmul2(make_float2(sn[j], -sn[j]), make_float2(vc.y, vc.x)));
-              oc[j] = pack_bf16(wc.x, wc.y);
-            }
-          }
+          rot4(rb, ob);
+          if (MODE == MODE_FULL) rot4(rc, oc);
           *reinterpret_cast<uint4*>(sm + C::B_OFF + off) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
           if (MODE == MODE_FULL)
             *reinterpret_cast<uint4*>(sm + C::C_OFF + off) = make_uint4(oc[0], oc[1], oc[2], oc[3]);
