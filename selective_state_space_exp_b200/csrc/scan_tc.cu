@@ -294,11 +294,11 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     if (tid < Q) {
       const int64_t t0 = cn0 + tid, i0 = (b * L + t0) * H + h;
       const bool v0 = cn < c_end && t0 < L, v1 = cn < c_end && t0 + 1 < L;
-      gr_dt = v0 ? __ldg(a.dt + i0) : 0.f;
-      gr_lm = v0 ? __ldg(a.lam + i0) : 0.f;
-      gr_av = v0 ? __ldg(a.A + i0) : 0.f;
-      gr_dt1 = v1 ? __ldg(a.dt + i0 + H) : 0.f;
-      gr_lm1 = v1 ? __ldg(a.lam + i0 + H) : 0.f;
+      gr_dt = v0 ? ldg_early(a.dt + i0) : 0.f;
+      gr_lm = v0 ? ldg_early(a.lam + i0) : 0.f;
+      gr_av = v0 ? ldg_early(a.A + i0) : 0.f;
+      gr_dt1 = v1 ? ldg_early(a.dt + i0 + H) : 0.f;
+      gr_lm1 = v1 ? ldg_early(a.lam + i0 + H) : 0.f;
     }
   };
   auto arm_m = [&]() {  // thread 0
@@ -442,9 +442,14 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     const bool fac_ok = l2end > -230.f;
 
     load_gates(c + 1);  // consumed by the next chunk's prologue, at the end of this one
+    // the last chunk's staged y must be read before w*x reuses its tile
+    if (MODE == MODE_FULL && tid == 0) bulk_wait_read0();
     const bool okm = (tid == 0) ? wait_bar(s_tbM, tphM, a.status) : true;
     if (okm && tid == 0) { tpendM = false; tphM ^= 1; }  // on a timeout the phase stays
     if (__syncthreads_or(!okm)) { aborted = true; break; }  // B, C and x of this chunk visible
+    // every thread has read theta and the slot sums over it (the prologue): the
+    // theta buffer takes the next chunk's
+    prefetch_early(c + 1);
 
     // ---- operands: Bt (and Ct) rotated by -Phi_t in place (16-byte pieces) -----
     if (slot_live) {
@@ -494,9 +499,6 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         }
       }
     }
-    if (MODE == MODE_FULL && tid == 0) bulk_wait_read0();  // the last chunk's staged y is read
-    __syncthreads();  // s_w ready; slot sums read; the w*x block is free
-    prefetch_early(c + 1);  // the theta buffer is free
 
     // ---- w * x (chunk-state operand) from the x tile ---------------------------
     constexpr int PER = M * 8 / NTH;

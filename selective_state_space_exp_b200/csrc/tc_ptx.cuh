@@ -222,6 +222,14 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
+// A read-only global load that stays where it is written (volatile: not moved
+// towards its first use), for values fetched well ahead of need.
+__device__ __forceinline__ float ldg_early(const float* p) {
+  float v;
+  asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
+}
+
 // Asynchronous global -> shared copies (zero-filled when `valid` is false;
 // `gmem` must still be a valid address).
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
