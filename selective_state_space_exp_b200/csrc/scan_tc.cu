@@ -63,8 +63,14 @@ struct Cfg {
   // per-token gamma, delta, w, Lam (log2 units) and the decay factor F,
   // chunk-end angles with their cos / sin, and the mbarriers.
   static constexpr int TH_FLOATS = Q * kPairs;
-  static constexpr int SMALL_BYTES = (TH_FLOATS + 6 * Q + 3 * kPairs) * 4 + 64;  // + 8 mbarrier slots
-  static_assert(((TH_FLOATS + 6 * Q + 3 * kPairs) * 4) % 8 == 0, "mbarrier alignment");
+  // The slot angle sums have their own buffer when shared memory allows (one
+  // tile per chunk), else they go over theta once it is read (a barrier more).
+  static constexpr bool PART_OWN = NT == 1;
+  static constexpr int PART_FLOATS = PART_OWN ? SLOTS_MAX * kPairs : 0;
+  static constexpr int SMALL_BYTES =
+      (TH_FLOATS + PART_FLOATS + 6 * Q + 3 * kPairs) * 4 + 64;  // + 8 mbarrier slots
+  static_assert(((TH_FLOATS + PART_FLOATS + 6 * Q + 3 * kPairs) * 4) % 8 == 0,
+                "mbarrier alignment");
   // at least 80 KB so that no more than two CTAs (2 x 256 TMEM columns) share
   // an SM; the dynamic shared memory base is declared 1024-byte aligned
   static constexpr int SMEM_RAW = SMALL_OFF + SMALL_BYTES;
@@ -168,7 +174,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     return;
   }
   float* s_th = reinterpret_cast<float*>(sm + C::SMALL_OFF);  // chunk theta [Q][N/2] (TMA)
-  float* s_gam = s_th + C::TH_FLOATS;           // gamma_t = lam_t dt_t                 [Q]
+  float* s_gam = s_th + C::TH_FLOATS + C::PART_FLOATS;  // gamma_t = lam_t dt_t         [Q]
   float* s_del = s_gam + Q;                     // delta_s, trapezoid weight of token s [Q]
   float* s_w = s_del + Q;                       // exp(Lam_end - Lam_s) delta_s         [Q]
   float* s_lg = s_w + Q;                        // Lam_t * log2(e)                      [Q]
@@ -183,7 +189,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_bar + 4);
   uint64_t* s_never = s_bar + 5;  // M3_FLAG_TEST_TIMEOUT: a barrier nothing completes
   uint64_t* s_bar1b = s_bar + 6;  // MMA1 of tile 1 (two-tile chunks)
-  float* s_part = s_th;  // [slots][kPairs] slot angle sums, over the consumed theta rows
+  // [slots][kPairs] slot angle sums: their own buffer, or over the consumed theta rows
+  float* s_part = C::PART_OWN ? s_th + C::TH_FLOATS : s_th;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, cq = warp >> 2;
@@ -371,7 +378,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       part[0] += ang[u][0].x; part[1] += ang[u][0].y;
       part[2] += ang[u][1].x; part[3] += ang[u][1].y;
     }
-    __syncthreads();  // theta read (the slot sums go over it); Lam complete
+    if (!C::PART_OWN) __syncthreads();  // theta read: the slot sums go over it
     // slot sums: row = slot, 16-byte piece kg at position kg ^ (slot % 8)
     auto part_at = [&](int slot, int k4) { return s_part + slot * kPairs + 4 * (k4 ^ (slot & 7)); };
     if (slot_live)
