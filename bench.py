@@ -79,6 +79,66 @@ def prefill_work(s: I.Shape):
     return float(flops), float(byt)
 
 
+def varlen_work(s: I.Shape, lengths):
+    """Algorithmic FLOPs and bytes of a packed batch: the sum over its
+    sequences of one-sequence scans (each sequence's last chunk counted like a
+    whole causal chunk, as for a ragged batch row)."""
+    f = b = 0.0
+    for n in lengths:
+        fi, bi = prefill_work(dataclasses.replace(s, batch=1, seqlen=int(n)))
+        f, b = f + fi, b + bi
+    return f, b
+
+
+VARLEN_SEQS = 16   # sequences in the packed-batch line: the length mix of
+VARLEN_MAX = 2048  # inputs.varlen_lengths (edges 0, 1, Q-1, Q, Q+1, max; rest uniform)
+
+
+def time_varlen(inp, s, max_len, steps, warmup, flush):
+    shape = m3.make_shape(len(inp["cu_seqlens"]) - 1, max_len, s.nheads, s.ngroups, s.headdim,
+                          s.dstate, s.rank, s.chunk, inp["x"].dtype)
+    ws = torch.empty(max(m3.workspace_size(shape), 1), dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(inp["x"])
+    fs = torch.empty((len(inp["cu_seqlens"]) - 1, s.nheads, s.dstate, s.headdim),
+                     dtype=torch.float32, device="cuda")
+
+    def step():
+        m3.m3_scan_fwd_varlen(inp["cu_seqlens"], inp["x"], inp["dt"], inp["A"], inp["lam"],
+                              inp["theta"], inp["B"], inp["C"], s.chunk, max_seqlen=max_len,
+                              y=y, final_state=fs, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    st = m3.m3_stream_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st}")
+    return [a.elapsed_time(b) * 1e-3 for a, b in ev]
+
+
+def varlen_line(s, rank, world, steps, warmup, flush, peaks, psrc):
+    """The packed variable-length batch of the workload's layer shape."""
+    lengths = I.varlen_lengths(VARLEN_SEQS, VARLEN_MAX, s.chunk, seed=1021)
+    inp = I.make_varlen_inputs(I.Workload(s), lengths, seed=1021 + 7919 * rank, device="cuda")
+    barrier(world)
+    t = max_over_ranks(sum(time_varlen(inp, s, VARLEN_MAX, steps, warmup, flush)),
+                       world) / steps
+    f, b = varlen_work(s, lengths)
+    return {"workload": f"packed batch of {len(lengths)} sequences, lengths 0..{VARLEN_MAX} "
+                        f"({sum(lengths)} tokens), layer shape as the main line",
+            "value": round(world * sum(lengths) / t, 1), "unit": "tokens/s",
+            "ms_per_step": round(t * 1e3, 4), "lengths": lengths,
+            "roofline": roofline(f, b, t, peaks, psrc)}
+
+
 def decode_work(s: I.Shape):
     R, N, P = s.rank, s.dstate, s.headdim
     bh = s.batch * s.nheads
@@ -387,7 +447,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1024,
                     help="consecutive decode steps timed (each with its own token's inputs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "varlen"], default=None,
                     help="run one part only (for profiling); prints its own line")
     ap.add_argument("--batch", type=int, default=None,
                     help="with --only: override the workload's batch (small profiling cases)")
@@ -424,6 +484,11 @@ def main():
         dflops, dbyt = decode_work(dw.shape)
         print(json.dumps({"only": "decode", "us_per_step": round(t / args.decode_steps * 1e6, 2),
                           "roofline": roofline(dflops, dbyt, t / args.decode_steps, peaks, psrc)}))
+        return
+    if args.only == "varlen":
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        line = varlen_line(s, 0, 1, args.steps, args.warmup, flush, peaks, psrc)
+        print(json.dumps({"only": "varlen", **line}))
         return
     if args.only == "prefill":
         inp = I.make_scan_inputs(I.Workload(s), seed=1001, device="cuda")
@@ -464,6 +529,10 @@ def main():
                      "ms_per_step": round(t2 * 1e3, 4),
                      "roofline": roofline(f2, b2, t2, peaks, psrc)}
         del inp2
+
+    # a packed batch of mixed lengths with the same layer shape
+    varlen = varlen_line(s, rank, world, max(3, args.steps // 2), args.warmup, flush, peaks,
+                         psrc)
 
     # decode (b = 128, H = 64, R as the prefill workload)
     dw = I.DECODE_MIMO if s.rank > 1 else I.DECODE_SISO
@@ -535,6 +604,7 @@ def main():
     }
     if secondary is not None:
         line["secondary"] = secondary
+    line["varlen"] = varlen
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_prefill(inp_host, s)
     if rank == 0:

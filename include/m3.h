@@ -212,6 +212,44 @@ M3_API int m3_scan_fwd_noalloc(const m3_shape* shape, const void* x, const float
                                const void* B_prev, const void* x_prev, void* y,
                                float* final_state, m3_stream_t stream);
 
+/* ---- packed variable-length batch -------------------------------------------
+ * Several sequences of different lengths in one call, stored back to back
+ * along the token dimension (no padding): sequence i is tokens
+ * [cu_seqlens[i], cu_seqlens[i+1]).  Each sequence is scanned exactly as
+ * m3_scan_fwd scans one batch row, with its own h0 / B_prev / x_prev and
+ * final state; no state crosses a sequence boundary.  The pages describe no
+ * packed layout (the wmrh blog, section 4.3, only discusses deployment in
+ * production): this is the serving layout of independent sequences that the
+ * recurrence itself allows.
+ *
+ *   shape->batch   number of sequences S >= 1.
+ *   shape->seqlen  an upper bound on every sequence's length (the longest);
+ *                  the workspace and launch grid are sized from it.
+ *   cu_seqlens     DEVICE array of S + 1 int32 offsets, cu_seqlens[0] = 0,
+ *                  nondecreasing, cu_seqlens[S] <= total_tokens; a sequence
+ *                  may be empty (its final state is then h0, or zeros).
+ *                  Read by the kernels: a pair that breaks these rules or a
+ *                  sequence longer than shape->seqlen is not read from; it
+ *                  sets M3_ERR_INVALID_ARGUMENT in the device error word
+ *                  (m3_stream_status) and that sequence's outputs are
+ *                  undefined.
+ *   total_tokens   rows T >= 0 of the token dimension of every packed tensor.
+ *   x, y           [T][H][R][P] io dtype;  dt, A, lam [T][H] fp32;
+ *   theta          [T][G][N/2] fp32 ([T][H][N/2] with M3_FLAG_THETA_PER_HEAD);
+ *   B, C           [T][G][R][N] io dtype.
+ *   h0, final_state [S][H][N][P] fp32 (nullable, as in m3_scan_fwd);
+ *   B_prev [S][G][R][N], x_prev [S][H][R][P] (both NULL or both non-NULL).
+ *   workspace      at least m3_scan_workspace_size(shape) bytes.
+ * Alignment, aliasing and errors otherwise as m3_scan_fwd; cu_seqlens must
+ * be 4-byte aligned. */
+M3_API int m3_scan_fwd_varlen(const m3_shape* shape, const int32_t* cu_seqlens,
+                              int64_t total_tokens, const void* x, const float* dt,
+                              const float* A, const float* lam, const float* theta,
+                              const void* B, const void* C, const float* h0,
+                              const void* B_prev, const void* x_prev, void* y,
+                              float* final_state, void* workspace,
+                              size_t workspace_bytes, m3_stream_t stream);
+
 /* ---- sequence split across ranks (context parallel) -------------------------
  * Over a segment of tokens the recurrence unrolls (PaperWeekly page section
  * 2.2, exponential-trapezoidal step; section 2.1, rotation) to

@@ -114,6 +114,32 @@ def scan(x, dt, A, lam, theta, B, C, h0=None, B_prev=None, x_prev=None,
     return y, hL
 
 
+def scan_varlen(cu_seqlens, x, dt, A, lam, theta, B, C, h0=None, B_prev=None, x_prev=None,
+                nthreads=None):
+    """Packed batch of independent sequences: sequence i is rows
+    cu_seqlens[i]:cu_seqlens[i+1] of the token dimension of x [T][H][R][P],
+    dt/A/lam [T][H], theta [T][G][N/2], B/C [T][G][R][N], with its own h0[i],
+    B_prev[i], x_prev[i].  No state crosses a boundary, so this is `scan`
+    (the token recurrence) applied to each sequence alone.  Returns y
+    [T][H][R][P] (rows outside every sequence stay NaN) and the final states
+    [S][H][N][P], float64."""
+    cu = [int(v) for v in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    x, dt, A, lam, theta, B, C = (_np(v, np.float32) for v in (x, dt, A, lam, theta, B, C))
+    h0, B_prev, x_prev = (_np(v, np.float32) for v in (h0, B_prev, x_prev))
+    S = len(cu) - 1
+    y = np.full(x.shape, np.nan, dtype=np.float64)
+    hL = np.empty((S, x.shape[1], B.shape[3], x.shape[3]), dtype=np.float64)
+    for i in range(S):
+        a, e = cu[i], cu[i + 1]
+        one = lambda v: None if v is None else v[i:i + 1]
+        yi, hi = scan(x[None, a:e], dt[None, a:e], A[None, a:e], lam[None, a:e],
+                      theta[None, a:e], B[None, a:e], C[None, a:e], h0=one(h0),
+                      B_prev=one(B_prev), x_prev=one(x_prev), nthreads=nthreads)
+        y[a:e] = yi[0]
+        hL[i] = hi[0]
+    return y, hL
+
+
 def decode_step(state, x_t, dt, A, lam, theta, B_t, C_t, B_prev=None, x_prev=None,
                 f64=False):
     """One decode step for every (b, h).  state [b][H][N][P] is copied and

@@ -146,14 +146,18 @@ int scan_call(const m3_shape* s, const void* x, const float* dt, const float* A,
               const float* lam, const float* theta, const void* B, const void* C,
               const float* h0, const void* B_prev, const void* x_prev, void* y,
               float* final_state, void* workspace, size_t workspace_bytes, m3_stream_t stream,
-              bool state_only) {
+              bool state_only, const int32_t* cu_seqlens = nullptr, int64_t total_tokens = 0) {
   int st = check_common(s);
   if (st != M3_OK) return st;
+  const bool varlen = cu_seqlens != nullptr;
+  if (varlen && (total_tokens < 0 || !aligned(cu_seqlens, 4))) return M3_ERR_INVALID_ARGUMENT;
+  // tokens of the call: none when L == 0 (or a packed batch holds none)
+  const bool empty = s->seqlen == 0 || (varlen && total_tokens == 0);
   if ((B_prev == nullptr) != (x_prev == nullptr)) return M3_ERR_INVALID_ARGUMENT;
   if (state_only && !final_state) return M3_ERR_INVALID_ARGUMENT;
   const bool bf16 = s->io_dtype == M3_BF16;
   if (bf16 && s->headdim % 8 != 0) return M3_ERR_UNSUPPORTED;
-  if (s->seqlen > 0 && (!x || !dt || !A || !lam || !theta || !B || !C || (!y && !state_only)))
+  if (!empty && (!x || !dt || !A || !lam || !theta || !B || !C || (!y && !state_only)))
     return M3_ERR_INVALID_ARGUMENT;
   const void* v16[] = {x, B, C, state_only ? nullptr : y, h0, final_state, B_prev, x_prev, theta};
   for (const void* p : v16)
@@ -163,7 +167,7 @@ int scan_call(const m3_shape* s, const void* x, const float* dt, const float* A,
     if (p && !aligned(p, 4)) return M3_ERR_ALIGNMENT;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
-  if (s->seqlen == 0) {  // no token: the state is h0 (the left term waits for a token)
+  if (empty) {  // no token: the state is h0 (the left term waits for a token)
     if (!final_state) return M3_OK;
     const size_t nb = sizeof(float) * s->batch * s->nheads * s->dstate * s->headdim;
     cudaError_t e = h0 ? cudaMemcpyAsync(final_state, h0, nb, cudaMemcpyDeviceToDevice, cs)
@@ -181,6 +185,8 @@ int scan_call(const m3_shape* s, const void* x, const float* dt, const float* A,
   a.final_state = final_state;
   a.ws = static_cast<char*>(workspace);
   a.ws_bytes = workspace_bytes;
+  a.cu_seqlens = cu_seqlens;
+  a.total_tokens = varlen ? total_tokens : s->batch * s->seqlen;
   if (status_word(&a.status) != M3_OK) return M3_ERR_CUDA;
   cudaError_t e = use_tc(s, a) ? tc_scan_launch(a, cs) : simt_scan_launch(a, cs);
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
@@ -195,6 +201,18 @@ M3_API int m3_scan_fwd(const m3_shape* s, const void* x, const float* dt, const 
                        m3_stream_t stream) {
   return scan_call(s, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev, y, final_state, workspace,
                    workspace_bytes, stream, false);
+}
+
+M3_API int m3_scan_fwd_varlen(const m3_shape* s, const int32_t* cu_seqlens,
+                              int64_t total_tokens, const void* x, const float* dt,
+                              const float* A, const float* lam, const float* theta,
+                              const void* B, const void* C, const float* h0,
+                              const void* B_prev, const void* x_prev, void* y,
+                              float* final_state, void* workspace, size_t workspace_bytes,
+                              m3_stream_t stream) {
+  if (!cu_seqlens) return M3_ERR_INVALID_ARGUMENT;
+  return scan_call(s, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev, y, final_state, workspace,
+                   workspace_bytes, stream, false, cu_seqlens, total_tokens);
 }
 
 M3_API int m3_scan_state(const m3_shape* s, const void* x, const float* dt, const float* A,

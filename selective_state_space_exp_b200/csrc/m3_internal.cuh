@@ -44,7 +44,29 @@ struct ScanArgs {
   bool test_timeout;  // M3_FLAG_TEST_TIMEOUT
   int64_t tgroups;    // theta groups: ngroups, or nheads (M3_FLAG_THETA_PER_HEAD)
   bool state_only;    // m3_scan_state: the final state only, no y
+  // Packed variable-length batch (m3_scan_fwd_varlen): sequence i is tokens
+  // [cu_seqlens[i], cu_seqlens[i+1]) of tensors with total_tokens rows, and
+  // seqlen is the longest sequence.  nullptr: batch x seqlen, fixed length.
+  const int32_t* cu_seqlens;
+  int64_t total_tokens;
 };
+
+// Token range of chain b's sequence in the token dimension of its tensors.
+struct Chain {
+  int64_t base, len;
+};
+
+// Sequence b's first token and length.  Packed batches are read from
+// cu_seqlens and checked: an offset pair outside [0, total_tokens], a
+// decreasing pair or a sequence longer than seqlen records
+// M3_ERR_INVALID_ARGUMENT and yields an empty sequence (nothing is read).
+__device__ __forceinline__ Chain chain_of(const ScanArgs& a, int64_t b) {
+  if (!a.cu_seqlens) return Chain{b * a.seqlen, a.seqlen};
+  const int64_t s0 = __ldg(a.cu_seqlens + b), s1 = __ldg(a.cu_seqlens + b + 1);
+  if (s0 >= 0 && s1 >= s0 && s1 <= a.total_tokens && s1 - s0 <= a.seqlen) return Chain{s0, s1 - s0};
+  if (a.status) atomicCAS(a.status, 0, (int)M3_ERR_INVALID_ARGUMENT);
+  return Chain{0, 0};
+}
 
 struct DecodeArgs {
   int64_t batch, nheads, ngroups, P, N, R;

@@ -33,7 +33,8 @@ constexpr int kOutRows = 32;   // (token, rank) output rows per chunk-output CTA
 
 struct Geo {
   int64_t b, h, g, tg, c, t0;  // g: B/C group, tg: theta group, t0: first token of the chunk
-  int nt;                  // valid tokens in the chunk
+  int64_t base, len;           // the sequence's first token (token dimension) and length
+  int nt;                      // valid tokens in the chunk (0 past a short packed sequence)
 };
 
 __device__ __forceinline__ Geo chunk_geo(const ScanArgs& a, int64_t c) {
@@ -44,8 +45,11 @@ __device__ __forceinline__ Geo chunk_geo(const ScanArgs& a, int64_t c) {
   q.tg = q.h / (a.nheads / a.tgroups);
   q.c = c;
   q.t0 = c * a.Q;
-  int64_t rem = a.seqlen - q.t0;
-  q.nt = (int)(rem < a.Q ? rem : a.Q);
+  const Chain ch = chain_of(a, q.b);
+  q.base = ch.base;
+  q.len = ch.len;
+  int64_t rem = ch.len - q.t0;
+  q.nt = (int)(rem < 0 ? 0 : rem < a.Q ? rem : a.Q);
   return q;
 }
 
@@ -54,12 +58,12 @@ __device__ __forceinline__ Geo chunk_geo(const ScanArgs& a, int64_t c) {
 __device__ void chunk_prep(const ScanArgs& a, const Geo& q, float* lcum, float* gam,
                            float* del, float* dts, float* phi) {
   const int K = (int)(a.N / 2);
-  const int64_t H = a.nheads, L = a.seqlen;
+  const int64_t H = a.nheads;
   for (int i = threadIdx.x; i < q.nt; i += blockDim.x) {
-    const int64_t bt = q.b * L + q.t0 + i;
+    const int64_t bt = q.base + q.t0 + i;
     const float dt = a.dt[bt * H + q.h], lam = a.lam[bt * H + q.h];
     float nxt = 0.f;
-    if (q.t0 + i + 1 < L) nxt = (1.f - a.lam[(bt + 1) * H + q.h]) * a.dt[(bt + 1) * H + q.h];
+    if (q.t0 + i + 1 < q.len) nxt = (1.f - a.lam[(bt + 1) * H + q.h]) * a.dt[(bt + 1) * H + q.h];
     dts[i] = dt;
     gam[i] = lam * dt;
     del[i] = lam * dt + nxt;
@@ -76,7 +80,7 @@ __device__ void chunk_prep(const ScanArgs& a, const Geo& q, float* lcum, float* 
   for (int k = threadIdx.x; k < K; k += blockDim.x) {
     float acc = 0.f;
     for (int i = 0; i < q.nt; ++i) {
-      acc += dts[i] * a.theta[((q.b * L + q.t0 + i) * a.tgroups + q.tg) * K + k];
+      acc += dts[i] * a.theta[((q.base + q.t0 + i) * a.tgroups + q.tg) * K + k];
       phi[i * K + k] = acc;
     }
   }
@@ -90,13 +94,12 @@ template <int R>
 __device__ void stage_tile(const ScanArgs& a, const Geo& q, int s0, const float* phi,
                            const float* wts, float* Bs, int ldb, float* Xs) {
   const int K = (int)(a.N / 2), N = (int)a.N, P = (int)a.P;
-  const int64_t L = a.seqlen;
   for (int e = threadIdx.x; e < kTileRows * K; e += blockDim.x) {
     const int ri = e / K, k = e % K;
     const int s = s0 + ri / R, r = ri % R;
     float v0 = 0.f, v1 = 0.f;
     if (s < q.nt) {
-      const int64_t base = ((q.b * L + q.t0 + s) * a.ngroups + q.g) * R * N + (int64_t)r * N;
+      const int64_t base = ((q.base + q.t0 + s) * a.ngroups + q.g) * R * N + (int64_t)r * N;
       const float b0 = io_load(a.B, base + 2 * k, a.bf16);
       const float b1 = io_load(a.B, base + 2 * k + 1, a.bf16);
       float sn, cs;
@@ -113,7 +116,7 @@ __device__ void stage_tile(const ScanArgs& a, const Geo& q, int s0, const float*
     const int s = s0 + ri / R, r = ri % R;
     float v = 0.f;
     if (s < q.nt)
-      v = io_load(a.x, ((q.b * L + q.t0 + s) * a.nheads + q.h) * R * P + (int64_t)r * P + p,
+      v = io_load(a.x, ((q.base + q.t0 + s) * a.nheads + q.h) * R * P + (int64_t)r * P + p,
                   a.bf16);
     Xs[ri * P + p] = v;
   }
@@ -180,9 +183,11 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(const ScanArgs a)
     const int n = n0 + i * NS;
     if (n < N) S[n * P + p] = acc[i];
   }
+  // an empty chunk (past a short packed sequence) passes the state unchanged
   float* sm_out = w.sum + cidx * (1 + K);
-  if (threadIdx.x == 0) sm_out[0] = lcum[q.nt - 1];
-  for (int k = threadIdx.x; k < K; k += blockDim.x) sm_out[1 + k] = phi[(q.nt - 1) * K + k];
+  if (threadIdx.x == 0) sm_out[0] = q.nt > 0 ? lcum[q.nt - 1] : 0.f;
+  for (int k = threadIdx.x; k < K; k += blockDim.x)
+    sm_out[1 + k] = q.nt > 0 ? phi[(q.nt - 1) * K + k] : 0.f;
 }
 
 // ---- 2. state passing -------------------------------------------------------
@@ -192,16 +197,17 @@ __global__ void __launch_bounds__(kThreads) state_pass_kernel(const ScanArgs a) 
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= K * P) return;
   const int k = idx / P, p = idx % P;
-  const int64_t H = a.nheads, L = a.seqlen, R = a.R;
+  const int64_t H = a.nheads, R = a.R;
   const int64_t g = h / (H / a.ngroups);
+  const Chain ch = chain_of(a, b);
   float g0 = 0.f, g1 = 0.f;
   const int64_t so = ((b * H + h) * N) * P;
   if (a.h0) {
     g0 = a.h0[so + (2 * k) * P + p];
     g1 = a.h0[so + (2 * k + 1) * P + p];
   }
-  if (a.B_prev) {
-    const float eps = (1.f - a.lam[(b * L) * H + h]) * a.dt[(b * L) * H + h];
+  if (a.B_prev && ch.len > 0) {  // the left endpoint term waits for a token
+    const float eps = (1.f - a.lam[ch.base * H + h]) * a.dt[ch.base * H + h];
     for (int r = 0; r < R; ++r) {
       const int64_t bb = ((b * a.ngroups + g) * R + r) * N;
       const float xv = io_load(a.x_prev, ((b * H + h) * R + r) * P + p, a.bf16);
@@ -256,13 +262,12 @@ __global__ void __launch_bounds__(kThreads) chunk_output_kernel(const ScanArgs a
   float* Sc = Xs + kTileRows * P;        // [kOutRows][kTileRows+1] masked scores
 
   chunk_prep(a, q, lcum, gam, del, dts, phi);
-  const int64_t L = a.seqlen;
   for (int e = threadIdx.x; e < kOutRows * K; e += blockDim.x) {
     const int ro = e / K, k = e % K;
     const int t = tt0 + ro / R, r = ro % R;
     float v0 = 0.f, v1 = 0.f;
     if (t < tt1) {
-      const int64_t base = ((q.b * L + q.t0 + t) * a.ngroups + q.g) * R * N + (int64_t)r * N;
+      const int64_t base = ((q.base + q.t0 + t) * a.ngroups + q.g) * R * N + (int64_t)r * N;
       const float c0 = io_load(a.C, base + 2 * k, a.bf16);
       const float c1 = io_load(a.C, base + 2 * k + 1, a.bf16);
       float sn, cs;
@@ -337,7 +342,7 @@ __global__ void __launch_bounds__(kThreads) chunk_output_kernel(const ScanArgs a
     const int ro = ro0 + i * RS;
     const int t = tt0 + ro / R, r = ro % R;
     if (t < tt1)
-      io_store(a.y, ((q.b * L + q.t0 + t) * a.nheads + q.h) * R * P + (int64_t)r * P + p,
+      io_store(a.y, ((q.base + q.t0 + t) * a.nheads + q.h) * R * P + (int64_t)r * P + p,
                acc[i], a.bf16);
   }
 }

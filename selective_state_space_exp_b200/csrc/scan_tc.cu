@@ -196,7 +196,10 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   const int qd = warp & 3, cq = warp >> 2;
   const int kg = lane & 15, tq = (warp << 1) | (lane >> 4);
   const int64_t seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int64_t L = a.seqlen, H = a.nheads, G = a.ngroups;
+  const int64_t H = a.nheads, G = a.ngroups;
+  // this chain's sequence: tokens [tokb, tokb + L) of the token dimension
+  const Chain chn = chain_of(a, b);
+  const int64_t L = chn.len, tokb = chn.base;
   const int64_t g = h / (H / G);
   const int64_t tg = h / (H / a.tgroups);  // theta group
 
@@ -243,8 +246,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     const int64_t so = ((b * H + h) * kN + n) * kP + p0;
 #pragma unroll
     for (int p = 0; p < CW; ++p) gst[p] = a.h0 ? __ldg(a.h0 + so + p) : 0.f;
-    if (a.B_prev) {
-      const float eps0 = (1.f - __ldg(a.lam + (b * L) * H + h)) * __ldg(a.dt + (b * L) * H + h);
+    if (a.B_prev && L > 0) {  // the left endpoint term waits for a token
+      const float eps0 = (1.f - __ldg(a.lam + tokb * H + h)) * __ldg(a.dt + tokb * H + h);
       for (int r = 0; r < R; ++r) {
         const float bp = eps0 * io_load(a.B_prev, ((b * G + g) * R + r) * kN + n, true);
         const int64_t xo = ((b * H + h) * R + r) * kP + p0;
@@ -275,7 +278,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
 
   float l2seg = 0.f, phi_seg = 0.f;  // MODE_STATE summaries (pair k = n / 2), log2 units
   const int64_t c_begin = seg * pl.cps;
-  const int64_t c_end = min(c_begin + pl.cps, a.nchunks);
+  const int64_t c_end = min(c_begin + pl.cps, (L + Q - 1) / Q);
 
   // Prefetch of a chunk's inputs in three steps, each as soon as its buffer is
   // free: theta (TMA, on s_tbT) and the gates (cp.async) once the previous
@@ -290,7 +293,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     if (cn >= c_end || tid != 0) return;
     mbar_expect_tx(s_tbT, Q * kPairs * 4);
     tpendT = true;
-    tma_load_3d(s_th, &maps.th, 0, (int)tg, (int)(b * L + cn * Q), s_tbT);
+    tma_load_3d(s_th, &maps.th, 0, (int)tg, (int)(tokb + cn * Q), s_tbT);
   };
   // The gates go to registers of the gate threads one chunk ahead (plain
   // loads: the prologue that uses them runs a whole chunk later): token tid's
@@ -299,7 +302,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   auto load_gates = [&](int64_t cn) {
     const int64_t cn0 = cn * Q;
     if (tid < Q) {
-      const int64_t t0 = cn0 + tid, i0 = (b * L + t0) * H + h;
+      const int64_t t0 = cn0 + tid, i0 = (tokb + t0) * H + h;
       const bool v0 = cn < c_end && t0 < L, v1 = cn < c_end && t0 + 1 < L;
       gr_dt = v0 ? ldg_early(a.dt + i0) : 0.f;
       gr_lm = v0 ? ldg_early(a.lam + i0) : 0.f;
@@ -317,14 +320,14 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   auto prefetch_c = [&](int64_t cn) {
     if (MODE != MODE_FULL || cn >= c_end || tid != 0) return;
     arm_m();
-    const int tok = (int)(b * L + cn * Q);
+    const int tok = (int)(tokb + cn * Q);
     tma_load_3d(sm + C::C_OFF, &maps.c, 0, (int)(g * R), tok, s_tbM);
     tma_load_3d(sm + C::C_OFF + C::OPB, &maps.c, 64, (int)(g * R), tok, s_tbM);
   };
   auto prefetch_bx = [&](int64_t cn) {
     if (cn >= c_end || tid != 0) return;
     arm_m();
-    const int tok = (int)(b * L + cn * Q);
+    const int tok = (int)(tokb + cn * Q);
     tma_load_3d(sm + C::X_OFF, &maps.x, 0, (int)(h * R), tok, s_tbM);
     tma_load_3d(sm + C::B_OFF, &maps.b, 0, (int)(g * R), tok, s_tbM);
     tma_load_3d(sm + C::B_OFF + C::OPB, &maps.b, 64, (int)(g * R), tok, s_tbM);
@@ -786,9 +789,28 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (MODE == MODE_FULL && tid == 0) {  // y of this chunk: one bulk tensor store
-      tma_store_4d(&maps.y, sm + C::XW_OFF, 0, (int)(h * R), (int)c0, (int)b);
-      bulk_commit();
+    if (MODE == MODE_FULL) {
+      if (!a.cu_seqlens) {  // y of this chunk: one bulk tensor store, clipped at the sequence end
+        if (tid == 0) {
+          tma_store_4d(&maps.y, sm + C::XW_OFF, 0, (int)(h * R), (int)c0, (int)b);
+          bulk_commit();
+        }
+      } else if (nt == Q) {  // packed batch: a whole chunk by the bulk store
+        if (tid == 0) {
+          tma_store_4d(&maps.y, sm + C::XW_OFF, 0, (int)(h * R), (int)(tokb + c0), 0);
+          bulk_commit();
+        }
+      } else {  // packed batch, a sequence's last partial chunk: the next sequence's rows
+                // follow, so only its nt * R rows are written (16-byte pieces)
+        const int pieces = nt * R * 8;
+        for (int e = tid; e < pieces; e += NTH) {
+          const int i = e >> 3, j = e & 7, t = i / R, r = i % R;
+          const uint4 v = *reinterpret_cast<const uint4*>(sm + C::XW_OFF + sw128_off(i, j));
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.y) +
+                               (((tokb + c0 + t) * H + h) * R + r) * kP + 8 * j;
+          *reinterpret_cast<uint4*>(dst) = v;
+        }
+      }
     }
     // the next chunk's gates and angles overlap its B, C, x loads
     if (c + 1 < c_end && !prologue(c + 1)) { aborted = true; break; }
@@ -834,13 +856,14 @@ __global__ void __launch_bounds__(256) tc_seg_pass_kernel(const ScanArgs a, cons
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= kPairs * kP) return;
   const int k = idx / kP, p = idx % kP;
-  const int64_t H = a.nheads, L = a.seqlen, R = a.R, G = a.ngroups;
+  const int64_t H = a.nheads, R = a.R, G = a.ngroups;
   const int64_t g = h / (H / G);
+  const Chain chn = chain_of(a, b);
   const int64_t so = (b * H + h) * kN * kP;
   float g0 = a.h0 ? a.h0[so + (2 * k) * kP + p] : 0.f;
   float g1 = a.h0 ? a.h0[so + (2 * k + 1) * kP + p] : 0.f;
-  if (a.B_prev) {
-    const float eps = (1.f - a.lam[(b * L) * H + h]) * a.dt[(b * L) * H + h];
+  if (a.B_prev && chn.len > 0) {  // the left endpoint term waits for a token
+    const float eps = (1.f - a.lam[chn.base * H + h]) * a.dt[chn.base * H + h];
     for (int r = 0; r < R; ++r) {
       const int64_t bb = ((b * G + g) * R + r) * kN;
       const float xv = io_load(a.x_prev, ((b * H + h) * R + r) * kP + p, true);
@@ -949,10 +972,18 @@ bool encode3d(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* 
   return encode_nd(m, dt, esize, base, 3, d, bx, sw);
 }
 
+// Rows of the token dimension: batch x seqlen, or a packed batch's total.
+int64_t token_rows(const ScanArgs& a) {
+  return a.cu_seqlens ? a.total_tokens : a.batch * a.seqlen;
+}
+
 bool make_maps(const ScanArgs& a, TcMaps* m) {
-  const uint64_t tok = (uint64_t)(a.batch * a.seqlen);
+  const uint64_t tok = (uint64_t)token_rows(a);
   const uint32_t R = (uint32_t)a.R, Q = (uint32_t)a.Q;
-  const uint64_t yd[4] = {kP, (uint64_t)(a.nheads * a.R), (uint64_t)a.seqlen, (uint64_t)a.batch};
+  // y as [batch][L][H*R][P], or a packed batch as [1][total][H*R][P]
+  const uint64_t yd[4] = {kP, (uint64_t)(a.nheads * a.R),
+                          a.cu_seqlens ? tok : (uint64_t)a.seqlen,
+                          a.cu_seqlens ? 1u : (uint64_t)a.batch};
   const uint32_t yb[4] = {64, R, Q, 1};
   return encode3d(&m->x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.x, kP, a.nheads * a.R, tok, 64, R,
                   Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -1007,7 +1038,7 @@ bool tc_scan_supported(const ScanArgs& a) {
   if (!a.bf16 || a.N != kN || a.P != kP) return false;
   const int64_t m = a.Q * a.R;
   // TMA token coordinates are 32-bit
-  if (a.batch * a.seqlen > (int64_t)0x7fffffff - a.Q) return false;
+  if (token_rows(a) > (int64_t)0x7fffffff - a.Q) return false;
   return (a.R == 1 || a.R == 2 || a.R == 4) && (m == 64 || m == 128 || m == 256) && a.Q >= 16;
 }
 

@@ -26,7 +26,7 @@ Tensor layouts are the library's (row-major):
 from __future__ import annotations
 
 import math
-from dataclasses import dataclass
+from dataclasses import dataclass, replace
 
 import torch
 
@@ -162,6 +162,43 @@ def make_decode_inputs(w: Workload, seed: int, steps: int,
     return dict(state0=state0, x=_round_io(x, s.io), B=_round_io(B, s.io),
                 C=_round_io(C, s.io), dt=dt, A=A, lam=lam, theta=theta,
                 B_prev=_round_io(B_prev, s.io), x_prev=_round_io(x_prev, s.io))
+
+
+def varlen_lengths(count: int, max_len: int, chunk: int, seed: int) -> list[int]:
+    """A seeded length mix for a packed batch of `count` sequences: the edge
+    lengths 0, 1, chunk - 1, chunk, chunk + 1 and max_len first (those that fit
+    in `count`), the rest uniform in [1, max_len]."""
+    edges = [v for v in (0, 1, chunk - 1, chunk, chunk + 1, max_len) if 0 <= v <= max_len]
+    g = torch.Generator().manual_seed(int(seed))
+    rest = torch.randint(1, max_len + 1, (max(0, count - len(edges)),), generator=g).tolist()
+    return (edges + rest)[:count]
+
+
+def make_varlen_inputs(w: Workload, lengths: list[int], seed: int,
+                       device: str | torch.device = "cpu") -> dict:
+    """Inputs of a packed batch of len(lengths) sequences stored back to back:
+    the per-token tensors of make_scan_inputs without the batch dimension
+    (x [T][H][R][P], dt [T][H], ...; T = sum(lengths)), drawn with the
+    workload's distributions; cu_seqlens [S+1] int32; and, per sequence, h0
+    [S][H][N][P] and B_prev, x_prev [S][..] when the workload asks for them.
+    w.shape.batch and w.shape.seqlen are ignored."""
+    s = w.shape
+    T, S = int(sum(lengths)), len(lengths)
+    packed = replace(w, shape=replace(s, batch=1, seqlen=T), with_h0=False, with_prev=False)
+    out = {k: v[0].contiguous() for k, v in make_scan_inputs(packed, seed, device).items()}
+    g = _gen(seed + 1, device)
+    if w.with_h0:
+        out["h0"] = _normal(g, (S, s.nheads, s.dstate, s.headdim), 0.0, 1.0, device)
+    if w.with_prev:
+        bias = _normal(g, (s.ngroups, s.rank, s.dstate), 0.0, 0.1, device)
+        out["B_prev"] = _round_io(_bc(g, s, (S,), w.bc, device, bias), s.io)
+        out["x_prev"] = _round_io(_normal(g, (S, s.nheads, s.rank, s.headdim), 0.0, 1.0, device),
+                                  s.io)
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + int(n))
+    out["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32, device=device)
+    return out
 
 
 def sample_chains(batch: int, nheads: int, count: int, seed: int = 7) -> list[int]:

@@ -21,6 +21,7 @@ M3_F32, M3_BF16 = 0, 1
 M3_FLAG_SIMT = 1
 M3_FLAG_TEST_TIMEOUT = 2
 M3_FLAG_THETA_PER_HEAD = 4
+M3_OK, M3_ERR_INVALID_ARGUMENT, M3_ERR_TIMEOUT = 0, -1, -6
 
 
 def theta_flag(theta_groups: int, ngroups: int, nheads: int) -> int:
@@ -31,6 +32,8 @@ def theta_flag(theta_groups: int, ngroups: int, nheads: int) -> int:
     if theta_groups == nheads:
         return M3_FLAG_THETA_PER_HEAD
     raise ValueError(f"theta has {theta_groups} groups: expected {ngroups} or {nheads}")
+
+
 STATUS = {0: "M3_OK", -1: "M3_ERR_INVALID_ARGUMENT", -2: "M3_ERR_UNSUPPORTED",
           -3: "M3_ERR_ALIGNMENT", -4: "M3_ERR_WORKSPACE", -5: "M3_ERR_CUDA",
           -6: "M3_ERR_TIMEOUT"}
@@ -92,6 +95,9 @@ def load() -> ctypes.CDLL:
             L.m3_segment_totals.restype = ctypes.c_int
             L.m3_state_fold.argtypes = [sp, ctypes.c_int64] + [vp] * 6
             L.m3_state_fold.restype = ctypes.c_int
+            L.m3_scan_fwd_varlen.argtypes = [sp, vp, ctypes.c_int64] + [vp] * 13 + \
+                [ctypes.c_size_t, vp]
+            L.m3_scan_fwd_varlen.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -177,6 +183,40 @@ def m3_scan_fwd(x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None, B_prev=Non
                             _ptr(x_prev), _ptr(y), _ptr(final_state), _ptr(workspace),
                             ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check("m3_scan_fwd", st)
+    return y, final_state
+
+
+def m3_scan_fwd_varlen(cu_seqlens, x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None,
+                       B_prev=None, x_prev=None, *, max_seqlen=None, y=None, final_state=None,
+                       want_final=True, workspace=None, simt=False, stream=None):
+    """Packed batch of S independent sequences: cu_seqlens [S+1] int32 on the
+    device (sequence i is token rows cu_seqlens[i]:cu_seqlens[i+1]); x [T][H][R][P],
+    dt/A/lam [T][H], theta [T][G][N/2], B/C [T][G][R][N]; h0 [S][H][N][P],
+    B_prev [S][G][R][N], x_prev [S][H][R][P].  max_seqlen bounds every
+    sequence's length (read from cu_seqlens, with a device sync, when None).
+    Returns (y [T][H][R][P], final_state [S][H][N][P])."""
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    S = cu_seqlens.numel() - 1
+    T, H, R, P = x.shape
+    G, N = B.shape[1], B.shape[3]
+    if max_seqlen is None:
+        max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item()) if S > 0 else 0
+    shape = make_shape(S, max_seqlen, H, G, P, N, R, chunk, x.dtype, simt)
+    shape.flags |= theta_flag(theta.shape[1], G, H)
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and want_final:
+        final_state = torch.empty((S, H, N, P), dtype=torch.float32, device=x.device)
+    need = workspace_size(shape)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    st = load().m3_scan_fwd_varlen(ctypes.byref(shape), _ptr(cu_seqlens), ctypes.c_int64(T),
+                                   _ptr(x), _ptr(dt), _ptr(A), _ptr(lam), _ptr(theta), _ptr(B),
+                                   _ptr(C), _ptr(h0), _ptr(B_prev), _ptr(x_prev), _ptr(y),
+                                   _ptr(final_state), _ptr(workspace),
+                                   ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check("m3_scan_fwd_varlen", st)
     return y, final_state
 
 
