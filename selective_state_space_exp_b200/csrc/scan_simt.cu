@@ -23,69 +23,18 @@
 // Workspace: S / G [b][H][nc][N][P] fp32 (G overwrites S in place) and the
 // chunk summaries [b][H][nc][1 + N/2] fp32 (Lam_end, Phi_end[k]).
 #include "m3_internal.cuh"
+#include "simt_chunk.cuh"
 
 namespace m3 {
 namespace {
 
+using simt::Geo;
+using simt::chunk_geo;
+using simt::chunk_prep;
+
 constexpr int kThreads = 256;
 constexpr int kTileRows = 64;  // (token, rank) rows of B / x per staged tile
 constexpr int kOutRows = 32;   // (token, rank) output rows per chunk-output CTA
-
-struct Geo {
-  int64_t b, h, g, tg, c, t0;  // g: B/C group, tg: theta group, t0: first token of the chunk
-  int64_t base, len;           // the sequence's first token (token dimension) and length
-  int nt;                      // valid tokens in the chunk (0 past a short packed sequence)
-};
-
-__device__ __forceinline__ Geo chunk_geo(const ScanArgs& a, int64_t c) {
-  Geo q;
-  q.b = blockIdx.z;
-  q.h = blockIdx.y;
-  q.g = q.h / (a.nheads / a.ngroups);
-  q.tg = q.h / (a.nheads / a.tgroups);
-  q.c = c;
-  q.t0 = c * a.Q;
-  const Chain ch = chain_of(a, q.b);
-  q.base = ch.base;
-  q.len = ch.len;
-  int64_t rem = ch.len - q.t0;
-  q.nt = (int)(rem < 0 ? 0 : rem < a.Q ? rem : a.Q);
-  return q;
-}
-
-// Chunk-local prefix sums and trapezoid weights into shared memory:
-// lcum[Q], gam[Q], del[Q], dts[Q], phi[Q][K].
-__device__ void chunk_prep(const ScanArgs& a, const Geo& q, float* lcum, float* gam,
-                           float* del, float* dts, float* phi) {
-  const int K = (int)(a.N / 2);
-  const int64_t H = a.nheads;
-  for (int i = threadIdx.x; i < q.nt; i += blockDim.x) {
-    const int64_t bt = q.base + q.t0 + i;
-    const float dt = a.dt[bt * H + q.h], lam = a.lam[bt * H + q.h];
-    float nxt = 0.f;
-    if (q.t0 + i + 1 < q.len) nxt = (1.f - a.lam[(bt + 1) * H + q.h]) * a.dt[(bt + 1) * H + q.h];
-    dts[i] = dt;
-    gam[i] = lam * dt;
-    del[i] = lam * dt + nxt;
-    lcum[i] = dt * a.A[bt * H + q.h];
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {  // <= 64 sequential adds: the plain prefix sum
-    float acc = 0.f;
-    for (int i = 0; i < q.nt; ++i) {
-      acc += lcum[i];
-      lcum[i] = acc;
-    }
-  }
-  for (int k = threadIdx.x; k < K; k += blockDim.x) {
-    float acc = 0.f;
-    for (int i = 0; i < q.nt; ++i) {
-      acc += dts[i] * a.theta[((q.base + q.t0 + i) * a.tgroups + q.tg) * K + k];
-      phi[i * K + k] = acc;
-    }
-  }
-  __syncthreads();
-}
 
 // Stage rows (s, r) of Rot(-Phi_s) B_s (scaled per token by wts[s] if given)
 // and of x_s for tokens [s0, s0 + kTileRows / R) into shared memory.
