@@ -139,6 +139,96 @@ def varlen_line(s, rank, world, steps, warmup, flush, peaks, psrc):
             "roofline": roofline(f, b, t, peaks, psrc)}
 
 
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz
+# (the nominal unit count and maximum SM clock; nothing here measures it)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def bwd_rows(s: I.Shape):
+    """Rows per chunk the backward picks (the library's rule for N = 128,
+    P = 64 and smaller: 64 rows, 32 for N = 256)."""
+    return 64 if (s.dstate // 2) * 64 <= 4096 else 32
+
+
+def bwd_work(s: I.Shape):
+    """Algorithmic FLOPs and bytes of one m3_scan_bwd.
+
+    Per chunk-head of the backward's chunking (M = Qb * R rows, causal token
+    blocks Qb(Qb+1)/2 * R^2): the score and dY X^T products (2 * causal * (N + P)),
+    dCt and dBt (2 * causal * N each), dX (2 * causal * P), and five N x P x M
+    state products (the forward chunk state it recomputes, D_c, dY G^T,
+    dGhat x, dGhat^T Bt): 10 * M * N * P.  Bytes: every input and dy read
+    once, every gradient (fp32) and the final-state adjoint written once."""
+    R, N, P = s.rank, s.dstate, s.headdim
+    M = bwd_rows(s)
+    Qb = M // R
+    causal = Qb * (Qb + 1) // 2 * R * R
+    nc = math.ceil(s.seqlen / Qb)
+    flops = (causal * (2 * (N + P) + 4 * N + 2 * P) + 10 * M * N * P) * nc * s.batch * s.nheads
+    io = 2 if s.io == "bf16" else 4
+    tok = s.batch * s.seqlen
+    byt = (3 * tok * s.nheads * R * P * io                 # x, dy in; (y is not read)
+           + tok * s.nheads * R * P * 4 - tok * s.nheads * R * P * io  # dx out (fp32)
+           + 2 * tok * s.ngroups * R * N * (io + 4)        # B, C in; dB, dC out
+           + 3 * tok * s.nheads * 4 * 2                    # dt, A, lam in; their grads out
+           + tok * s.ngroups * (N // 2) * 4 * 2            # theta in, dtheta out
+           + 2 * s.batch * s.nheads * N * P * 4)           # d_final in, dh0 out
+    return float(flops), float(byt)
+
+
+def alu_roofline(flops, byt, seconds, peaks):
+    t_alu = flops / (FP32_ALU_TFLOPS * 1e12)
+    t_hbm = byt / (peaks["hbm_gbs"] * 1e9)
+    if t_alu >= t_hbm:
+        ach = flops / seconds / 1e12
+        return {"bound": "alu", "achieved": round(ach, 2), "peak": round(FP32_ALU_TFLOPS, 1),
+                "unit": "TFLOP/s", "frac": round(ach / FP32_ALU_TFLOPS, 4),
+                "roofline_time_us": round(t_alu * 1e6, 2),
+                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x 1.965 GHz (nominal)"}
+    ach = byt / seconds / 1e9
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(ach / peaks["hbm_gbs"], 4), "roofline_time_us": round(t_hbm * 1e6, 2)}
+
+
+def time_bwd(inp, s, steps, warmup, flush):
+    gen = torch.Generator(device="cuda").manual_seed(77)
+    dy = torch.randn(inp["x"].shape, generator=gen, device="cuda").to(inp["x"].dtype)
+    dfin = torch.randn((s.batch, s.nheads, s.dstate, s.headdim), generator=gen, device="cuda")
+    ws = torch.empty(max(m3.bwd_workspace_size(m3.scan_shape(inp["x"], inp["B"], s.chunk)), 1),
+                     dtype=torch.uint8, device="cuda")
+
+    def step():
+        m3.m3_scan_bwd(inp["x"], inp["dt"], inp["A"], inp["lam"], inp["theta"], inp["B"],
+                       inp["C"], dy, s.chunk, d_final=dfin, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    st = m3.m3_stream_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st}")
+    return [a.elapsed_time(b) * 1e-3 for a, b in ev]
+
+
+def bwd_line(inp, s, world, steps, warmup, flush, peaks):
+    barrier(world)
+    t = max_over_ranks(sum(time_bwd(inp, s, steps, warmup, flush)), world) / steps
+    f, b = bwd_work(s)
+    return {"metric": "backward tokens/s", "value": round(world * s.batch * s.seqlen / t, 1),
+            "unit": "tokens/s", "ms_per_step": round(t * 1e3, 4),
+            "path": "m3_scan_bwd: state-only forward recompute + 3 backward launches, "
+                    "CUDA cores fp32",
+            "roofline": alu_roofline(f, b, t, peaks)}
+
+
 def decode_work(s: I.Shape):
     R, N, P = s.rank, s.dstate, s.headdim
     bh = s.batch * s.nheads
@@ -447,7 +537,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1024,
                     help="consecutive decode steps timed (each with its own token's inputs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode", "varlen"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "varlen", "bwd"], default=None,
                     help="run one part only (for profiling); prints its own line")
     ap.add_argument("--batch", type=int, default=None,
                     help="with --only: override the workload's batch (small profiling cases)")
@@ -484,6 +574,12 @@ def main():
         dflops, dbyt = decode_work(dw.shape)
         print(json.dumps({"only": "decode", "us_per_step": round(t / args.decode_steps * 1e6, 2),
                           "roofline": roofline(dflops, dbyt, t / args.decode_steps, peaks, psrc)}))
+        return
+    if args.only == "bwd":
+        inp = I.make_scan_inputs(I.Workload(s), seed=1001, device="cuda")
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        print(json.dumps({"only": "bwd", **bwd_line(inp, s, 1, args.steps, args.warmup, flush,
+                                                    peaks)}))
         return
     if args.only == "varlen":
         flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")

@@ -212,6 +212,40 @@ M3_API int m3_scan_fwd_noalloc(const m3_shape* shape, const void* x, const float
                                const void* B_prev, const void* x_prev, void* y,
                                float* final_state, m3_stream_t stream);
 
+/* ---- backward pass ------------------------------------------------------------
+ * Gradients of a scalar loss with respect to every input of m3_scan_fwd,
+ * given its gradients dy with respect to y and d_final with respect to the
+ * final state.  The recurrence is the one of m3_scan_fwd (PaperWeekly page
+ * sections 2.1-2.3); the gradients are those of its token-by-token form,
+ * evaluated chunk by chunk: the forward's chunk-start states are recomputed,
+ * the adjoint of the state is passed backwards over the chunks, and each
+ * chunk's gradients follow from its masked quadratic form.  Computed on CUDA
+ * cores in fp32 for both io dtypes; every gradient is written in fp32.
+ *
+ *   inputs      as m3_scan_fwd (same layouts, dtypes and nullability).
+ *   dy          [b][L][H][R][P] io dtype (required when L > 0).
+ *   d_final     [b][H][N][P] fp32, or NULL for zero.
+ *   dx          [b][L][H][R][P] fp32;  ddt, dA, dlam [b][L][H] fp32;
+ *   dtheta      fp32, theta's layout;  dB, dC [b][L][G][R][N] fp32 (summed
+ *               over the heads of a group).  All required when L > 0.
+ *   dh0         [b][H][N][P] fp32, or NULL to skip (computed whether or not
+ *               h0 was given: the gradient with respect to the initial state).
+ *   dB_prev,
+ *   dx_prev     [b][G][R][N] and [b][H][R][P] fp32, both NULL or both
+ *               non-NULL; zeros when B_prev is NULL.
+ *   workspace   at least m3_scan_bwd_workspace_size() bytes, 256-byte aligned.
+ * Packed variable-length batches are not supported by this call.  Returns
+ * M3_OK when the work was enqueued, M3_ERR_UNSUPPORTED for shapes whose
+ * chunk tiles do not fit one CTA's shared memory. */
+M3_API int m3_scan_bwd_workspace_size(const m3_shape* shape, size_t* bytes);
+M3_API int m3_scan_bwd(const m3_shape* shape, const void* x, const float* dt, const float* A,
+                       const float* lam, const float* theta, const void* B, const void* C,
+                       const float* h0, const void* B_prev, const void* x_prev, const void* dy,
+                       const float* d_final, float* dx, float* ddt, float* dA, float* dlam,
+                       float* dtheta, float* dB, float* dC, float* dh0, float* dB_prev,
+                       float* dx_prev, void* workspace, size_t workspace_bytes,
+                       m3_stream_t stream);
+
 /* ---- packed variable-length batch -------------------------------------------
  * Several sequences of different lengths in one call, stored back to back
  * along the token dimension (no padding): sequence i is tokens

@@ -215,6 +215,83 @@ M3_API int m3_scan_fwd_varlen(const m3_shape* s, const int32_t* cu_seqlens,
                    workspace_bytes, stream, false, cu_seqlens, total_tokens);
 }
 
+M3_API int m3_scan_bwd_workspace_size(const m3_shape* s, size_t* bytes) {
+  int st = check_common(s);
+  if (st != M3_OK) return st;
+  if (!bytes) return M3_ERR_INVALID_ARGUMENT;
+  ScanArgs a = make_scan_args(s);
+  if (!bwd_supported(a)) return M3_ERR_UNSUPPORTED;
+  *bytes = s->seqlen == 0 ? 0 : bwd_workspace(a);
+  return M3_OK;
+}
+
+M3_API int m3_scan_bwd(const m3_shape* s, const void* x, const float* dt, const float* A,
+                       const float* lam, const float* theta, const void* B, const void* C,
+                       const float* h0, const void* B_prev, const void* x_prev, const void* dy,
+                       const float* d_final, float* dx, float* ddt, float* dA, float* dlam,
+                       float* dtheta, float* dB, float* dC, float* dh0, float* dB_prev,
+                       float* dx_prev, void* workspace, size_t workspace_bytes,
+                       m3_stream_t stream) {
+  int st = check_common(s);
+  if (st != M3_OK) return st;
+  if ((B_prev == nullptr) != (x_prev == nullptr)) return M3_ERR_INVALID_ARGUMENT;
+  if ((dB_prev == nullptr) != (dx_prev == nullptr)) return M3_ERR_INVALID_ARGUMENT;
+  const bool bf16 = s->io_dtype == M3_BF16;
+  if (bf16 && s->headdim % 8 != 0) return M3_ERR_UNSUPPORTED;
+  ScanArgs a = make_scan_args(s);
+  if (!bwd_supported(a)) return M3_ERR_UNSUPPORTED;
+  if (s->seqlen > 0 && (!x || !dt || !A || !lam || !theta || !B || !C || !dy || !dx || !ddt ||
+                        !dA || !dlam || !dtheta || !dB || !dC))
+    return M3_ERR_INVALID_ARGUMENT;
+  const void* v16[] = {x, B, C, dy, h0, d_final, B_prev, x_prev, theta, dx, dtheta, dB, dC,
+                       dh0, dB_prev, dx_prev};
+  for (const void* p : v16)
+    if (p && !aligned(p, 16)) return M3_ERR_ALIGNMENT;
+  const void* v4[] = {dt, A, lam, ddt, dA, dlam};
+  for (const void* p : v4)
+    if (p && !aligned(p, 4)) return M3_ERR_ALIGNMENT;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const size_t sb = sizeof(float) * s->batch * s->nheads * s->dstate * s->headdim;
+
+  if (s->seqlen == 0) {  // no token: the state is h0, so dh0 = d_final; nothing else
+    if (dh0) {
+      cudaError_t e = d_final ? cudaMemcpyAsync(dh0, d_final, sb, cudaMemcpyDeviceToDevice, cs)
+                              : cudaMemsetAsync(dh0, 0, sb, cs);
+      if (e != cudaSuccess) return M3_ERR_CUDA;
+    }
+    if (dB_prev) {
+      const size_t nb = sizeof(float) * s->batch * s->ngroups * s->rank * s->dstate;
+      const size_t nx = sizeof(float) * s->batch * s->nheads * s->rank * s->headdim;
+      if (cudaMemsetAsync(dB_prev, 0, nb, cs) != cudaSuccess ||
+          cudaMemsetAsync(dx_prev, 0, nx, cs) != cudaSuccess)
+        return M3_ERR_CUDA;
+    }
+    return M3_OK;
+  }
+  const size_t need = bwd_workspace(a);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return M3_ERR_WORKSPACE;
+  a.x = x; a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.B = B; a.C = C;
+  a.h0 = h0; a.B_prev = B_prev; a.x_prev = x_prev;
+  a.ws = static_cast<char*>(workspace);
+  a.ws_bytes = workspace_bytes;
+  a.total_tokens = s->batch * s->seqlen;
+  if (status_word(&a.status) != M3_OK) return M3_ERR_CUDA;
+  BwdArgs g;
+  g.dy = dy; g.d_final = d_final; g.dx = dx; g.ddt = ddt; g.dA = dA; g.dlam = dlam;
+  g.dtheta = dtheta; g.dB = dB; g.dC = dC; g.dh0 = dh0;
+  g.dB_prev = B_prev ? dB_prev : nullptr;
+  g.dx_prev = B_prev ? dx_prev : nullptr;
+  if (dB_prev && !B_prev) {  // no previous token: its gradients are zero
+    const size_t nb = sizeof(float) * s->batch * s->ngroups * s->rank * s->dstate;
+    const size_t nx = sizeof(float) * s->batch * s->nheads * s->rank * s->headdim;
+    if (cudaMemsetAsync(dB_prev, 0, nb, cs) != cudaSuccess ||
+        cudaMemsetAsync(dx_prev, 0, nx, cs) != cudaSuccess)
+      return M3_ERR_CUDA;
+  }
+  cudaError_t e = bwd_launch(a, g, cs);
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
 M3_API int m3_scan_state(const m3_shape* s, const void* x, const float* dt, const float* A,
                          const float* lam, const float* theta, const void* B, const void* C,
                          const float* h0, const void* B_prev, const void* x_prev,

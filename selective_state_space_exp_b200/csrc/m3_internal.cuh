@@ -99,6 +99,30 @@ size_t tc_scan_workspace(const ScanArgs& a);
 int64_t tc_scan_segments(const ScanArgs& a);
 cudaError_t tc_scan_launch(const ScanArgs& a, cudaStream_t s);
 
+// Where the CUDA-core pass keeps its chunk states (one N x P fp32 matrix per
+// chunk-head, [b][H][nc][N][P]; the chunk-start states once state passing has
+// run) and its chunk totals ([b][H][nc][1 + N/2]: Lam_end, Phi_end).
+void simt_state_views(const ScanArgs& a, float** states, float** sums);
+
+// Backward pass of the scan (CUDA cores, fp32): outputs and incoming adjoints.
+struct BwdArgs {
+  const void* dy;         // [b][L][H][R][P] io dtype
+  const float* d_final;   // [b][H][N][P] or nullptr
+  float* dx;              // [b][L][H][R][P]
+  float* ddt;             // [b][L][H]
+  float* dA;              // [b][L][H]
+  float* dlam;            // [b][L][H]
+  float* dtheta;          // [b][L][Gt][N/2]
+  float* dB;              // [b][L][G][R][N]
+  float* dC;              // [b][L][G][R][N]
+  float* dh0;             // [b][H][N][P] or nullptr
+  float* dB_prev;         // [b][G][R][N] or nullptr (with dx_prev)
+  float* dx_prev;         // [b][H][R][P] or nullptr
+};
+size_t bwd_workspace(const ScanArgs& a);
+bool bwd_supported(const ScanArgs& a);
+cudaError_t bwd_launch(const ScanArgs& a, const BwdArgs& g, cudaStream_t s);
+
 // Decode step.
 cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t s);
 

@@ -76,7 +76,7 @@ struct WsView {
   float* sum;  // [b][H][nc][1 + K]
 };
 
-__device__ __forceinline__ WsView ws_view(const ScanArgs& a) {
+__host__ __device__ __forceinline__ WsView ws_view(const ScanArgs& a) {
   WsView w;
   const size_t sbytes = align_up(sizeof(float) * a.batch * a.nheads * a.nchunks * a.N * a.P, 256);
   w.S = reinterpret_cast<float*>(a.ws);
@@ -361,6 +361,12 @@ size_t simt_scan_workspace(const ScanArgs& a) {
   const size_t mbytes =
       align_up(sizeof(float) * a.batch * a.nheads * a.nchunks * (1 + a.N / 2), 256);
   return sbytes + mbytes;
+}
+
+void simt_state_views(const ScanArgs& a, float** states, float** sums) {
+  const WsView w = ws_view(a);
+  *states = w.S;
+  *sums = w.sum;
 }
 
 cudaError_t simt_scan_launch(const ScanArgs& a, cudaStream_t st) {

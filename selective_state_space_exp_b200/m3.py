@@ -98,6 +98,10 @@ def load() -> ctypes.CDLL:
             L.m3_scan_fwd_varlen.argtypes = [sp, vp, ctypes.c_int64] + [vp] * 13 + \
                 [ctypes.c_size_t, vp]
             L.m3_scan_fwd_varlen.restype = ctypes.c_int
+            L.m3_scan_bwd_workspace_size.argtypes = [sp, ctypes.POINTER(ctypes.c_size_t)]
+            L.m3_scan_bwd_workspace_size.restype = ctypes.c_int
+            L.m3_scan_bwd.argtypes = [sp] + [vp] * 23 + [ctypes.c_size_t, vp]
+            L.m3_scan_bwd.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -218,6 +222,47 @@ def m3_scan_fwd_varlen(cu_seqlens, x, dt, A, lam, theta, B, C, chunk: int = 64, 
                                    ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check("m3_scan_fwd_varlen", st)
     return y, final_state
+
+
+def bwd_workspace_size(shape: Shape) -> int:
+    n = ctypes.c_size_t(0)
+    _check("m3_scan_bwd_workspace_size",
+           load().m3_scan_bwd_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
+    return int(n.value)
+
+
+def m3_scan_bwd(x, dt, A, lam, theta, B, C, dy, chunk: int = 64, h0=None, B_prev=None,
+                x_prev=None, d_final=None, *, want_dh0=True, workspace=None, stream=None):
+    """Backward of m3_scan_fwd: gradients of sum(y * dy) + sum(final * d_final)
+    with respect to every input.  Returns a dict of fp32 tensors: x, dt, A, lam,
+    theta, B, C, and h0 (when want_dh0), B_prev and x_prev (when B_prev is given),
+    each in its input's layout."""
+    shape = scan_shape(x, B, chunk, False, theta)
+    dev, f32 = x.device, torch.float32
+    g = {"x": torch.empty(x.shape, dtype=f32, device=dev),
+         "dt": torch.empty(dt.shape, dtype=f32, device=dev),
+         "A": torch.empty(A.shape, dtype=f32, device=dev),
+         "lam": torch.empty(lam.shape, dtype=f32, device=dev),
+         "theta": torch.empty(theta.shape, dtype=f32, device=dev),
+         "B": torch.empty(B.shape, dtype=f32, device=dev),
+         "C": torch.empty(C.shape, dtype=f32, device=dev)}
+    if want_dh0:
+        g["h0"] = torch.empty((x.shape[0], x.shape[2], B.shape[4], x.shape[4]), dtype=f32,
+                              device=dev)
+    if B_prev is not None:
+        g["B_prev"] = torch.empty(B_prev.shape, dtype=f32, device=dev)
+        g["x_prev"] = torch.empty(x_prev.shape, dtype=f32, device=dev)
+    need = bwd_workspace_size(shape)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    st = load().m3_scan_bwd(ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(lam),
+                            _ptr(theta), _ptr(B), _ptr(C), _ptr(h0), _ptr(B_prev), _ptr(x_prev),
+                            _ptr(dy), _ptr(d_final), _ptr(g["x"]), _ptr(g["dt"]), _ptr(g["A"]),
+                            _ptr(g["lam"]), _ptr(g["theta"]), _ptr(g["B"]), _ptr(g["C"]),
+                            _ptr(g.get("h0")), _ptr(g.get("B_prev")), _ptr(g.get("x_prev")),
+                            _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check("m3_scan_bwd", st)
+    return g
 
 
 def m3_scan_fwd_noalloc(x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None, B_prev=None,

@@ -1,0 +1,115 @@
+"""Parity of the backward pass (m3_scan_bwd, through the C ABI) with the
+gradient oracle (fp64 autograd through the token recurrence, pinned in
+test_grad_oracle.py).
+
+Bar, for every gradient tensor separately: max |err| / max |ref| <= 1e-4 for
+fp32 io.  bf16 io shares the rounded inputs with the oracle and computes in
+fp32 as well, so it is held to the same 1e-4 (the io bar of 2e-2 applies to
+rounded outputs; these gradients are fp32).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import m3_grad
+from selective_state_space_exp_b200 import inputs as I
+from selective_state_space_exp_b200 import m3
+from parity_helpers import need_gpu, rel_err, to_dev
+
+pytestmark = pytest.mark.gpu
+BAR = 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    need_gpu()
+
+
+def case(batch=2, L=150, H=4, P=16, N=16, R=1, G=1, io="f32", decay="slow", h0=True,
+         prev=True, tph=False, seed=0):
+    w = I.Workload(I.Shape(batch, L, H, P, N, R, G, 64, io),
+                   bc="rmsnorm" if io == "bf16" else "normal", decay=decay, with_h0=h0,
+                   with_prev=prev, theta_per_head=tph)
+    inp = I.make_scan_inputs(w, seed=seed)
+    gen = torch.Generator().manual_seed(seed + 1)
+    dy = torch.randn(inp["x"].shape, generator=gen)
+    inp["dy"] = dy.to(inp["x"].dtype)
+    inp["d_final"] = torch.randn((batch, H, N, P), generator=gen)
+    return inp
+
+
+def compare(inp, chunk=64, with_final=True):
+    g = to_dev(inp)
+    got = m3.m3_scan_bwd(g["x"], g["dt"], g["A"], g["lam"], g["theta"], g["B"], g["C"],
+                         g["dy"], chunk, g.get("h0"), g.get("B_prev"), g.get("x_prev"),
+                         g["d_final"] if with_final else None)
+    assert m3.m3_stream_status() == 0
+    _, _, ref = m3_grad.scan_grads(*[inp.get(k) for k in m3_grad.NAMES], dy=inp["dy"],
+                                   d_final=inp["d_final"] if with_final else None)
+    errs = {}
+    for name, r in ref.items():
+        if name == "h0" and "h0" not in inp:
+            continue
+        a = got[name].cpu().numpy()
+        assert np.isfinite(a).all(), name
+        errs[name] = rel_err(a, r)
+    if "h0" not in inp:  # dh0 is the gradient with respect to a zero initial state
+        _, _, r0 = m3_grad.scan_grads(*[inp.get(k) for k in m3_grad.NAMES[:7]],
+                                      h0=np.zeros(tuple(got["h0"].shape)), dy=inp["dy"],
+                                      d_final=inp["d_final"] if with_final else None)
+        errs["h0"] = rel_err(got["h0"].cpu().numpy(), r0["h0"])
+    bad = {k: v for k, v in errs.items() if not v <= BAR}
+    assert not bad, f"errors above {BAR}: {bad} (all: {errs})"
+    return errs
+
+
+@pytest.mark.parametrize("R", [1, 2, 4, 8])
+def test_bwd_ranks(R):
+    """Ragged length (150 is not a multiple of any backward chunk), h0, previous
+    token, d_final; slow decay so that the adjoint crosses many chunks."""
+    compare(case(R=R, seed=100 + R))
+
+
+@pytest.mark.parametrize("G,tph", [(2, False), (4, False), (1, True), (2, True)])
+def test_bwd_groups_and_angle_rates(G, tph):
+    compare(case(R=2, G=G, tph=tph, seed=200 + G + 10 * tph))
+
+
+@pytest.mark.parametrize("N,P", [(32, 32), (64, 16), (16, 128), (256, 32), (128, 64)])
+def test_bwd_shapes(N, P):
+    compare(case(batch=1, L=90, H=2, N=N, P=P, R=2, seed=300 + N + P))
+
+
+def test_bwd_fast_decay_no_prev_no_final():
+    compare(case(R=4, decay="fast", h0=False, prev=False, seed=400), with_final=False)
+
+
+@pytest.mark.parametrize("L", [1, 2, 64, 65])
+def test_bwd_edge_lengths(L):
+    compare(case(batch=1, L=L, H=2, R=2, seed=500 + L))
+
+
+def test_bwd_bf16_layer_shape():
+    """bf16 io at the layer's N = 128, P = 64 (a few chains)."""
+    compare(case(batch=1, L=200, H=2, N=128, P=64, R=4, io="bf16", seed=600))
+
+
+def test_bwd_empty_sequence():
+    inp = to_dev(case(batch=1, L=0, H=2, R=1, seed=700))
+    got = m3.m3_scan_bwd(inp["x"], inp["dt"], inp["A"], inp["lam"], inp["theta"], inp["B"],
+                         inp["C"], inp["dy"], 64, inp["h0"], inp["B_prev"], inp["x_prev"],
+                         inp["d_final"])
+    assert m3.m3_stream_status() == 0
+    assert torch.equal(got["h0"], inp["d_final"])
+    assert float(got["B_prev"].abs().max()) == 0.0
+
+
+def test_bwd_chunk_invariant():
+    """The backward picks its own chunk; the caller's chunk changes nothing."""
+    g = to_dev(case(R=2, seed=800))
+    outs = [m3.m3_scan_bwd(g["x"], g["dt"], g["A"], g["lam"], g["theta"], g["B"], g["C"],
+                           g["dy"], c, g["h0"], g["B_prev"], g["x_prev"], g["d_final"])
+            for c in (16, 64)]
+    for k in outs[0]:
+        assert torch.equal(outs[0][k], outs[1][k]) or \
+            rel_err(outs[0][k].cpu().numpy(), outs[1][k].cpu().numpy()) < 1e-6, k
