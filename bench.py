@@ -145,9 +145,9 @@ FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def bwd_rows(s: I.Shape):
-    """Rows per chunk the backward picks (the library's rule for N = 128,
-    P = 64 and smaller: 64 rows, 32 for N = 256)."""
-    return 64 if (s.dstate // 2) * 64 <= 4096 else 32
+    """Rows per chunk the backward picks (the library's rule: 32 rows, two
+    CTAs per SM)."""
+    return 32
 
 
 def bwd_work(s: I.Shape):
@@ -630,6 +630,9 @@ def main():
     varlen = varlen_line(s, rank, world, max(3, args.steps // 2), args.warmup, flush, peaks,
                          psrc)
 
+    # backward of the same scan (gradients of every input), CUDA cores fp32
+    backward = bwd_line(inp, s, world, 3, args.warmup, flush, peaks)
+
     # decode (b = 128, H = 64, R as the prefill workload)
     dw = I.DECODE_MIMO if s.rank > 1 else I.DECODE_SISO
     ds = dw.shape
@@ -701,6 +704,7 @@ def main():
     if secondary is not None:
         line["secondary"] = secondary
     line["varlen"] = varlen
+    line["backward"] = backward
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_prefill(inp_host, s)
     if rank == 0:

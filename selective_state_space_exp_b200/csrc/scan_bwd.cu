@@ -39,8 +39,8 @@ using simt::Geo;
 
 constexpr int kThreads = 256;
 constexpr int kTileRows = 64;  // (token, rank) rows staged per pass of step 2
-constexpr int kMaxPairs = 16;  // accumulator pairs per thread in step 4 (N/2 * M <= 4096)
-constexpr int kMaxCols = 32;   // dX columns per thread in step 4 (P * M <= 8192)
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
 struct BwdWs {
   float* G;     // [b][H][nc][N][P] chunk-start states (forward)
@@ -60,12 +60,14 @@ ScanArgs fwd_args(const ScanArgs& a, int64_t Qb) {
 }
 
 // ---- step 2: D_c -------------------------------------------------------------
-template <int R, int OPT>
+// Thread tiles of 4 x 4 (n, p) outputs, TPT tiles per thread (as the forward's
+// chunk-state kernel).
+template <int R, int TPT>
 __global__ void __launch_bounds__(kThreads) bwd_dstate_kernel(const ScanArgs a, const BwdArgs g,
                                                               const BwdWs w) {
   const Geo q = chunk_geo(a, blockIdx.x);
   const int N = (int)a.N, P = (int)a.P, K = N / 2, Q = (int)a.Q;
-  extern __shared__ float sm[];
+  extern __shared__ __align__(16) float sm[];
   float* lcum = sm;
   float* gam = lcum + Q;
   float* del = gam + Q;
@@ -75,10 +77,14 @@ __global__ void __launch_bounds__(kThreads) bwd_dstate_kernel(const ScanArgs a, 
   float* Ys = Cs + kTileRows * N;   // [kTileRows][P] dy
   chunk_prep(a, q, lcum, gam, del, dts, phi);
 
-  const int p = threadIdx.x % P, n0 = threadIdx.x / P, NS = kThreads / P;
-  float acc[OPT];
+  const int PG = P / 4, ntiles = (N / 4) * PG;
+  float acc[TPT][4][4];
 #pragma unroll
-  for (int i = 0; i < OPT; ++i) acc[i] = 0.f;
+  for (int m = 0; m < TPT; ++m)
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[m][u][v] = 0.f;
   const int TS = kTileRows / R;
   for (int s0 = 0; s0 < q.nt; s0 += TS) {
     for (int e = threadIdx.x; e < kTileRows * K; e += blockDim.x) {
@@ -105,20 +111,33 @@ __global__ void __launch_bounds__(kThreads) bwd_dstate_kernel(const ScanArgs a, 
     __syncthreads();
     const int rows = min(kTileRows, (q.nt - s0) * R);
     for (int ri = 0; ri < rows; ++ri) {
-      const float yv = Ys[ri * P + p];
 #pragma unroll
-      for (int i = 0; i < OPT; ++i) {
-        const int n = n0 + i * NS;
-        if (n < N) acc[i] = fmaf(Cs[ri * N + n], yv, acc[i]);
+      for (int m = 0; m < TPT; ++m) {
+        const int ti = threadIdx.x + kThreads * m;
+        if (ti < ntiles) {
+          const float4 cv = ld4(Cs + ri * N + 4 * (ti / PG));
+          const float4 yv = ld4(Ys + ri * P + 4 * (ti % PG));
+          const float c4[4] = {cv.x, cv.y, cv.z, cv.w}, y4[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) acc[m][u][v] = fmaf(c4[u], y4[v], acc[m][u][v]);
+        }
       }
     }
     __syncthreads();
   }
   float* D = w.D + ((q.b * a.nheads + q.h) * a.nchunks + q.c) * (int64_t)N * P;
 #pragma unroll
-  for (int i = 0; i < OPT; ++i) {
-    const int n = n0 + i * NS;
-    if (n < N) D[n * P + p] = acc[i];
+  for (int m = 0; m < TPT; ++m) {
+    const int ti = threadIdx.x + kThreads * m;
+    if (ti < ntiles) {
+      const int n0 = 4 * (ti / PG), p0 = 4 * (ti % PG);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<float4*>(D + (n0 + u) * P + p0) =
+            make_float4(acc[m][u][0], acc[m][u][1], acc[m][u][2], acc[m][u][3]);
+    }
   }
 }
 
@@ -133,20 +152,35 @@ __global__ void __launch_bounds__(kThreads) bwd_state_pass_kernel(const ScanArgs
   const int64_t so = (b * H + h) * (int64_t)N * P;
   float d0 = g.d_final ? g.d_final[so + (2 * k) * P + p] : 0.f;
   float d1 = g.d_final ? g.d_final[so + (2 * k + 1) * P + p] : 0.f;
-  for (int64_t c = a.nchunks - 1; c >= 0; --c) {
-    const int64_t cidx = (b * H + h) * a.nchunks + c;
-    float* Dc = w.D + cidx * (int64_t)N * P;
-    const float* su = w.sums + cidx * (1 + K);
-    const float e0 = Dc[(2 * k) * P + p], e1 = Dc[(2 * k + 1) * P + p];
-    Dc[(2 * k) * P + p] = d0;  // adjoint of chunk c's outgoing state
-    Dc[(2 * k + 1) * P + p] = d1;
-    const float dec = expf(su[0]);
-    float sn, cs;
-    sincosf(su[1 + k], &sn, &cs);
-    const float n0 = fmaf(dec, cs * d0 + sn * d1, e0);  // D_c + exp(Lam) Rot(-Phi) dG
-    const float n1 = fmaf(dec, -sn * d0 + cs * d1, e1);
-    d0 = n0;
-    d1 = n1;
+  // chunks in batches of kPipe, all of a batch's loads issued before its
+  // dependent updates (the chain waits on arithmetic, not on each load)
+  constexpr int kPipe = 8;
+  for (int64_t c0 = a.nchunks - 1; c0 >= 0; c0 -= kPipe) {
+    float e0[kPipe], e1[kPipe], dec[kPipe], sn[kPipe], cs[kPipe];
+#pragma unroll
+    for (int j = 0; j < kPipe; ++j) {
+      const int64_t c = c0 - j;
+      if (c < 0) break;
+      const int64_t cidx = (b * H + h) * a.nchunks + c;
+      const float* Dc = w.D + cidx * (int64_t)N * P;
+      const float* su = w.sums + cidx * (1 + K);
+      e0[j] = Dc[(2 * k) * P + p];
+      e1[j] = Dc[(2 * k + 1) * P + p];
+      dec[j] = expf(su[0]);
+      sincosf(su[1 + k], &sn[j], &cs[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < kPipe; ++j) {
+      const int64_t c = c0 - j;
+      if (c < 0) break;
+      float* Dc = w.D + ((b * H + h) * a.nchunks + c) * (int64_t)N * P;
+      Dc[(2 * k) * P + p] = d0;  // adjoint of chunk c's outgoing state
+      Dc[(2 * k + 1) * P + p] = d1;
+      const float n0 = fmaf(dec[j], cs[j] * d0 + sn[j] * d1, e0[j]);  // D_c + exp(Lam) Rot(-Phi) dG
+      const float n1 = fmaf(dec[j], -sn[j] * d0 + cs[j] * d1, e1[j]);
+      d0 = n0;
+      d1 = n1;
+    }
   }
   if (g.dh0) {
     g.dh0[so + (2 * k) * P + p] = d0;
@@ -181,48 +215,128 @@ __global__ void __launch_bounds__(kThreads) bwd_state_pass_kernel(const ScanArgs
 }
 
 // ---- step 4: per-chunk gradients ---------------------------------------------
-// Shared memory (floats), M = Q * R rows, rows of Ct / Bt padded to N + 1 and
-// of X / dY to P + 1 (conflict-free column walks).
+// One CTA per chunk-head, M = Q * R <= 64 rows.  The products are register
+// tiles over shared-memory operands: the thread grid is 16 x 16, a thread
+// owns rows ty + 16 a and, per product, columns tx + 16 c (score-shaped
+// outputs) or 4-wide column groups 4 (tx + 16 c) (N-wide outputs).  Row
+// strides are padded by 4 floats so 16 consecutive rows of a float4 column
+// fall on distinct banks.
 struct ChunkSmem {
-  int lcum, gam, del, dts, phi, Ct, Bt, X, dY, S, DX, dMt, dPhi, dLam, dgam, ddel, beta, wv, ecs,
+  int lcum, gam, del, dts, phi, Ct, Bt, X, dY, S, DX, Gt, dPhi, dLam, dgam, ddel, beta, wv, ecs,
       thT, red, total;
+  int ldn, ldp, ldm;
   __host__ __device__ ChunkSmem(int M, int N, int P, int Q) {
     const int K = N / 2;
+    ldn = N + 4; ldp = P + 4; ldm = M + 4;
     int o = 0;
     lcum = o; o += Q;
     gam = o; o += Q;
     del = o; o += Q;
     dts = o; o += Q;
-    phi = o; o += Q * K;  // chunk_prep's layout ends here
-    Ct = o; o += M * (N + 1);
-    Bt = o; o += M * (N + 1);
-    X = o; o += M * (P + 1);
-    dY = o; o += M * (P + 1);
-    S = o; o += M * M;
-    DX = o; o += M * M;
-    dMt = o; o += Q * Q;
+    phi = o; o += Q * K;
+    o = (o + 3) & ~3;  // float4 alignment of the operand tiles
+    Ct = o; o += M * ldn;
+    Bt = o; o += M * ldn;
+    X = o; o += M * ldp;
+    dY = o; o += M * ldp;
+    S = o; o += M * ldm;
+    DX = o; o += M * ldm;
+    Gt = o;  // G_c^T, then dGhat^T ([p][n]); first the token-pair dL/dM [Q][Q]
+    o += (P * ldn > Q * Q ? P * ldn : ((Q * Q + 3) & ~3));
     dPhi = o; o += Q * K;
     dLam = o; o += Q;
     dgam = o; o += Q;
     ddel = o; o += Q;
     beta = o; o += Q;
     wv = o; o += Q;
-    ecs = o; o += 2 * K;
     thT = o; o += Q;
+    ecs = o; o += 2 * K;
     red = o; o += 32;
     total = o;
   }
 };
 
-template <int R>
+
+// sum over the 16 lanes of a half-warp (tx = lane % 16)
+__device__ __forceinline__ float sum16(float v) {
+#pragma unroll
+  for (int off = 1; off < 16; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+__device__ __forceinline__ float f4c(const float4& v, int k) {
+  return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
+}
+
+// acc[i][c][:] += sum_kk a4[i].kk * B[kk][4 gi .. 4 gi + 3], gi = tx + 16 c:
+// four k-steps of an N-wide product whose A operand was loaded 4 k wide.
+template <int TI, int NGT>
+__device__ __forceinline__ void nn4(float (&acc)[TI][NGT][4], const float4 (&a4)[TI],
+                                    const float* B, int ldb, int tx, int NG) {
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+    for (int c = 0; c < NGT; ++c) {
+      const int gi = tx + 16 * c;
+      if (gi < NG) {
+        const float4 bv = ld4(B + kk * ldb + 4 * gi);
+#pragma unroll
+        for (int i = 0; i < TI; ++i) {
+          const float av = f4c(a4[i], kk);
+          acc[i][c][0] = fmaf(av, bv.x, acc[i][c][0]);
+          acc[i][c][1] = fmaf(av, bv.y, acc[i][c][1]);
+          acc[i][c][2] = fmaf(av, bv.z, acc[i][c][2]);
+          acc[i][c][3] = fmaf(av, bv.w, acc[i][c][3]);
+        }
+      }
+    }
+}
+
+// TI consecutive floats (the thread's rows of a column of a transposed operand)
+template <int TI>
+__device__ __forceinline__ void ld_rows(const float* p, float (&v)[TI]) {
+  if constexpr (TI == 4) {
+    const float4 t = ld4(p);
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  } else {
+    const float2 t = *reinterpret_cast<const float2*>(p);
+    v[0] = t.x; v[1] = t.y;
+  }
+}
+
+// acc[i][c][:] += av[i] * B[4 gi .. 4 gi + 3]: one k-step of an N-wide product
+template <int TI, int NGT>
+__device__ __forceinline__ void tn1(float (&acc)[TI][NGT][4], const float (&av)[TI],
+                                    const float* B, int tx, int NG) {
+#pragma unroll
+  for (int c = 0; c < NGT; ++c) {
+    const int gi = tx + 16 * c;
+    if (gi < NG) {
+      const float4 bv = ld4(B + 4 * gi);
+#pragma unroll
+      for (int i = 0; i < TI; ++i) {
+        acc[i][c][0] = fmaf(av[i], bv.x, acc[i][c][0]);
+        acc[i][c][1] = fmaf(av[i], bv.y, acc[i][c][1]);
+        acc[i][c][2] = fmaf(av[i], bv.z, acc[i][c][2]);
+        acc[i][c][3] = fmaf(av[i], bv.w, acc[i][c][3]);
+      }
+    }
+  }
+}
+
+template <int R, int M>
 __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(const ScanArgs a, const BwdArgs g,
                                                              const BwdWs w) {
+  constexpr int Q = M / R;
+  constexpr int TI = M / 16;           // rows per thread
+  constexpr int NGT = 8 / TI;          // N-wide products: 4-column groups per thread (N <= 64 NGT)
+  constexpr int PCT = 128 / 16;        // dX columns per thread at most (P <= 128)
   const Geo q = chunk_geo(a, blockIdx.x);
-  const int N = (int)a.N, P = (int)a.P, K = N / 2, Q = (int)a.Q, M = Q * R;
-  const int ldn = N + 1, ldp = P + 1;
+  const int N = (int)a.N, P = (int)a.P, K = N / 2;
   const int64_t H = a.nheads;
   const ChunkSmem L(M, N, P, Q);
-  extern __shared__ float sm[];
+  const int ldn = L.ldn, ldp = L.ldp, ldm = L.ldm;
+  extern __shared__ __align__(16) float sm[];
   float* lcum = sm + L.lcum;
   float* gam = sm + L.gam;
   float* del = sm + L.del;
@@ -234,17 +348,18 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(const ScanArgs a, c
   float* dY = sm + L.dY;
   float* S = sm + L.S;
   float* DX = sm + L.DX;
-  float* dMt = sm + L.dMt;
+  float* Gt = sm + L.Gt;
+  float* dMt = Gt;  // token-pair dL/dM until G_c^T is staged
   float* dPhi = sm + L.dPhi;
   float* dLam = sm + L.dLam;
   float* dgam = sm + L.dgam;
   float* ddel = sm + L.ddel;
   float* beta = sm + L.beta;
   float* wv = sm + L.wv;
-  float* ecs = sm + L.ecs;
   float* thT = sm + L.thT;
+  float* ecs = sm + L.ecs;
   float* red = sm + L.red;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const int nt = q.nt;
   if (nt <= 0) return;  // uniform over the block
 
@@ -291,16 +406,46 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(const ScanArgs a, c
   }
   __syncthreads();
 
-  // scores S = Ct Bt^T and DX = dY X^T on the causal token blocks
-  for (int e = tid; e < M * M; e += kThreads) {
-    const int i = e / M, j = e % M;
-    float sv = 0.f, dv = 0.f;
-    if (j / R <= i / R && i / R < nt) {
-      for (int n = 0; n < N; ++n) sv = fmaf(Ct[i * ldn + n], Bt[j * ldn + n], sv);
-      for (int p = 0; p < P; ++p) dv = fmaf(dY[i * ldp + p], X[j * ldp + p], dv);
+  // S = Ct Bt^T and DX = dY X^T: rows ty + 16 a, columns tx + 16 c
+  {
+    float s_acc[TI][TI], d_acc[TI][TI];
+#pragma unroll
+    for (int i = 0; i < TI; ++i)
+#pragma unroll
+      for (int j = 0; j < TI; ++j) s_acc[i][j] = d_acc[i][j] = 0.f;
+    for (int n = 0; n < N; n += 4) {
+      float4 av[TI], bv[TI];
+#pragma unroll
+      for (int i = 0; i < TI; ++i) av[i] = ld4(Ct + (ty + 16 * i) * ldn + n);
+#pragma unroll
+      for (int j = 0; j < TI; ++j) bv[j] = ld4(Bt + (tx + 16 * j) * ldn + n);
+#pragma unroll
+      for (int i = 0; i < TI; ++i)
+#pragma unroll
+        for (int j = 0; j < TI; ++j)
+          s_acc[i][j] = fmaf(av[i].x, bv[j].x, fmaf(av[i].y, bv[j].y,
+                        fmaf(av[i].z, bv[j].z, fmaf(av[i].w, bv[j].w, s_acc[i][j]))));
     }
-    S[e] = sv;
-    DX[e] = dv;
+    for (int p = 0; p < P; p += 4) {
+      float4 av[TI], bv[TI];
+#pragma unroll
+      for (int i = 0; i < TI; ++i) av[i] = ld4(dY + (ty + 16 * i) * ldp + p);
+#pragma unroll
+      for (int j = 0; j < TI; ++j) bv[j] = ld4(X + (tx + 16 * j) * ldp + p);
+#pragma unroll
+      for (int i = 0; i < TI; ++i)
+#pragma unroll
+        for (int j = 0; j < TI; ++j)
+          d_acc[i][j] = fmaf(av[i].x, bv[j].x, fmaf(av[i].y, bv[j].y,
+                        fmaf(av[i].z, bv[j].z, fmaf(av[i].w, bv[j].w, d_acc[i][j]))));
+    }
+#pragma unroll
+    for (int i = 0; i < TI; ++i)
+#pragma unroll
+      for (int j = 0; j < TI; ++j) {
+        S[(ty + 16 * i) * ldm + tx + 16 * j] = s_acc[i][j];
+        DX[(ty + 16 * i) * ldm + tx + 16 * j] = d_acc[i][j];
+      }
   }
   __syncthreads();
   // dL/dM per token pair, summed over the ranks of both tokens
@@ -308,9 +453,11 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(const ScanArgs a, c
     const int t = e / Q, s = e % Q;
     float v = 0.f;
     if (s <= t && t < nt)
+#pragma unroll
       for (int r = 0; r < R; ++r)
+#pragma unroll
         for (int r2 = 0; r2 < R; ++r2) {
-          const int o = (t * R + r) * M + s * R + r2;
+          const int o = (t * R + r) * ldm + s * R + r2;
           v = fmaf(S[o], DX[o], v);
         }
     dMt[e] = v;
@@ -319,165 +466,249 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(const ScanArgs a, c
   auto mtok = [&](int t, int s) {  // mask entry M_ts, s <= t < nt
     return s == t ? gam[t] : expf(lcum[t] - lcum[s]) * del[s];
   };
-  // S <- M o S,  DX <- M o DX
+  // S <- M o S,  DX <- M o DX  (zero above the diagonal and past the chunk end)
   for (int e = tid; e < M * M; e += kThreads) {
-    const int t = (e / M) / R, s = (e % M) / R;
+    const int i = e / M, j = e % M, t = i / R, s = j / R;
     const float m = (s <= t && t < nt) ? mtok(t, s) : 0.f;
-    S[e] *= m;
-    DX[e] *= m;
+    S[i * ldm + j] *= m;
+    DX[i * ldm + j] *= m;
   }
-  // the mask's own gradients: Lam (row minus column), gamma, delta
+  // the mask's own gradients.  With F_ts = dM_ts exp(Lam_t - Lam_s) (s < t):
+  // dLam_u = sum_s<u F_us delta_s - delta_u sum_t>u F_tu (the diagonal's row
+  // and column terms cancel), d delta_u = sum_t>u F_tu, d gamma_u = dM_uu.
+  for (int u = tid; u < nt; u += kThreads) dgam[u] += dMt[u * Q + u];
+  __syncthreads();
+  for (int e = tid; e < Q * Q; e += kThreads) {
+    const int t = e / Q, s = e % Q;
+    dMt[e] = (s < t && t < nt) ? dMt[e] * expf(lcum[t] - lcum[s]) : 0.f;
+  }
+  __syncthreads();
   for (int u = tid; u < nt; u += kThreads) {
-    float dl = 0.f, dd = 0.f;
-    for (int s = 0; s <= u; ++s) dl = fmaf(dMt[u * Q + s], mtok(u, s), dl);
-    for (int t = u; t < nt; ++t) dl -= dMt[t * Q + u] * mtok(t, u);
-    for (int t = u + 1; t < nt; ++t) dd = fmaf(dMt[t * Q + u], expf(lcum[t] - lcum[u]), dd);
-    dLam[u] += dl;
-    dgam[u] += dMt[u * Q + u];
-    ddel[u] += dd;
+    float row = 0.f, col = 0.f;
+    for (int s = 0; s < u; ++s) row = fmaf(dMt[u * Q + s], del[s], row);
+    for (int t = u + 1; t < nt; ++t) col += dMt[t * Q + u];
+    dLam[u] += row - del[u] * col;
+    ddel[u] += col;
   }
   __syncthreads();
 
-  const int TPR = kThreads / M;  // threads per row
-  const int row = tid / TPR, qq = tid % TPR;
   const int64_t cidx = (q.b * H + q.h) * a.nchunks + q.c;
   const float* Gc = w.G + cidx * (int64_t)N * P;  // state entering the chunk
   const float* Do = w.D + cidx * (int64_t)N * P;  // adjoint of the state leaving it
-  const int np = (K - qq + TPR - 1) / TPR;        // pairs of this thread: k = qq + TPR * m
-
-  // dCt rows -> dC, dPhi (C's rotation), dLam (the exp(Lam_t) term)
-  if (row < M && row / R < nt) {
-    const int i = row, t = i / R, r = i % R;
-    float acc[2 * kMaxPairs];
-#pragma unroll
-    for (int m = 0; m < 2 * kMaxPairs; ++m) acc[m] = 0.f;
-    for (int j = 0; j < (t + 1) * R; ++j) {
-      const float pij = DX[i * M + j];
-#pragma unroll
-      for (int m = 0; m < kMaxPairs; ++m)
-        if (m < np) {
-          const int k = qq + TPR * m;
-          acc[2 * m] = fmaf(pij, Bt[j * ldn + 2 * k], acc[2 * m]);
-          acc[2 * m + 1] = fmaf(pij, Bt[j * ldn + 2 * k + 1], acc[2 * m + 1]);
-        }
-    }
-    const float el = expf(lcum[t]);
-    float dl = 0.f;
-    const int64_t base = ((q.base + q.t0 + t) * a.ngroups + q.g) * R * N + (int64_t)r * N;
-#pragma unroll
-    for (int m = 0; m < kMaxPairs; ++m)
-      if (m < np) {
-        const int k = qq + TPR * m;
-        float g0 = 0.f, g1 = 0.f;
-        for (int p = 0; p < P; ++p) {
-          const float yv = dY[i * ldp + p];
-          g0 = fmaf(yv, __ldg(Gc + (2 * k) * P + p), g0);
-          g1 = fmaf(yv, __ldg(Gc + (2 * k + 1) * P + p), g1);
-        }
-        const float c0 = Ct[i * ldn + 2 * k], c1 = Ct[i * ldn + 2 * k + 1];
-        dl = fmaf(c0, g0, fmaf(c1, g1, dl));
-        const float d0 = fmaf(el, g0, acc[2 * m]), d1 = fmaf(el, g1, acc[2 * m + 1]);
-        atomicAdd(dPhi + t * K + k, d0 * c1 - d1 * c0);
-        float sn, cs;
-        sincosf(phi[t * K + k], &sn, &cs);
-        atomicAdd(g.dC + base + 2 * k, cs * d0 - sn * d1);  // Rot(Phi_t) dCt
-        atomicAdd(g.dC + base + 2 * k + 1, sn * d0 + cs * d1);
-      }
-    atomicAdd(dLam + t, el * dl);
+  // G_c^T into Gt ([p][n])
+  for (int e = tid; e < N * P; e += kThreads) {
+    const int n = e / P, p = e % P;
+    Gt[p * ldn + n] = __ldg(Gc + e);
   }
+  __syncthreads();
 
-  // dBt rows -> dB, dPhi (B's rotation), beta_s = Bt_s^T dGhat x_s
-  if (row < M && row / R < nt) {
-    const int j = row, s = j / R, r = j % R;
-    float acc[2 * kMaxPairs];
+  const int NG = N / 4;  // 4-column groups of an N-wide row
+  // dCt = exp(Lam_t) dY G_c^T + (M o DX) Bt -> dC, dPhi (C's rotation), dLam
+  {
+    float acc[TI][NGT][4];
 #pragma unroll
-    for (int m = 0; m < 2 * kMaxPairs; ++m) acc[m] = 0.f;
-    for (int i = s * R; i < nt * R; ++i) {
-      const float pij = DX[i * M + j];
+    for (int i = 0; i < TI; ++i)
 #pragma unroll
-      for (int m = 0; m < kMaxPairs; ++m)
-        if (m < np) {
-          const int k = qq + TPR * m;
-          acc[2 * m] = fmaf(pij, Ct[i * ldn + 2 * k], acc[2 * m]);
-          acc[2 * m + 1] = fmaf(pij, Ct[i * ldn + 2 * k + 1], acc[2 * m + 1]);
-        }
+      for (int c = 0; c < NGT; ++c)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[i][c][v] = 0.f;
+    for (int p = 0; p < P; p += 4) {
+      float4 a4[TI];
+#pragma unroll
+      for (int i = 0; i < TI; ++i) a4[i] = ld4(dY + (ty + 16 * i) * ldp + p);
+      nn4<TI, NGT>(acc, a4, Gt + p * ldn, ldn, tx, NG);
     }
-    const float ws = wv[s];
-    float bt = 0.f;
-    const int64_t base = ((q.base + q.t0 + s) * a.ngroups + q.g) * R * N + (int64_t)r * N;
+    // dLam_t += exp(Lam_t) Ct_t . (dY G_c^T)_t, then scale by exp(Lam_t)
 #pragma unroll
-    for (int m = 0; m < kMaxPairs; ++m)
-      if (m < np) {
-        const int k = qq + TPR * m;
-        float a0 = 0.f, a1 = 0.f;
-        for (int p = 0; p < P; ++p) {
-          const float xv = X[j * ldp + p];
-          a0 = fmaf(__ldg(Do + (2 * k) * P + p), xv, a0);
-          a1 = fmaf(__ldg(Do + (2 * k + 1) * P + p), xv, a1);
+    for (int i = 0; i < TI; ++i) {
+      const int row = ty + 16 * i, t = row / R;
+      const float el = (t < nt) ? expf(lcum[t]) : 0.f;
+      float dl = 0.f;
+#pragma unroll
+      for (int c = 0; c < NGT; ++c) {
+        const int gi = tx + 16 * c;
+        if (gi < NG) {
+          const float4 cv = ld4(Ct + row * ldn + 4 * gi);
+          dl += cv.x * acc[i][c][0] + cv.y * acc[i][c][1] + cv.z * acc[i][c][2] + cv.w * acc[i][c][3];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[i][c][v] *= el;
         }
-        const float ce = ecs[2 * k], se = ecs[2 * k + 1];
-        const float v0 = ce * a0 + se * a1, v1 = -se * a0 + ce * a1;  // (dGhat x_j) pair
-        const float b0 = Bt[j * ldn + 2 * k], b1 = Bt[j * ldn + 2 * k + 1];
-        bt = fmaf(b0, v0, fmaf(b1, v1, bt));
-        const float d0 = fmaf(ws, v0, acc[2 * m]), d1 = fmaf(ws, v1, acc[2 * m + 1]);
-        atomicAdd(dPhi + s * K + k, d0 * b1 - d1 * b0);
-        float sn, cs;
-        sincosf(phi[s * K + k], &sn, &cs);
-        atomicAdd(g.dB + base + 2 * k, cs * d0 - sn * d1);  // Rot(Phi_s) dBt
-        atomicAdd(g.dB + base + 2 * k + 1, sn * d0 + cs * d1);
       }
-    atomicAdd(beta + s, bt);
-  }
-
-  // dX rows
-  if (row < M && row / R < nt) {
-    const int j = row, s = j / R, r = j % R;
-    const int nc = (P - qq + TPR - 1) / TPR;  // columns p = qq + TPR * m
-    float acc[kMaxCols];
-#pragma unroll
-    for (int m = 0; m < kMaxCols; ++m) acc[m] = 0.f;
-    for (int i = s * R; i < nt * R; ++i) {
-      const float pij = S[i * M + j];
-#pragma unroll
-      for (int m = 0; m < kMaxCols; ++m)
-        if (m < nc) acc[m] = fmaf(pij, dY[i * ldp + qq + TPR * m], acc[m]);
+      dl = sum16(dl);
+      if (tx == 0 && t < nt) atomicAdd(dLam + t, el * dl);
     }
-    const float ws = wv[s];
-    float* dxo = g.dx + ((q.base + q.t0 + s) * H + q.h) * R * P + (int64_t)r * P;
+    for (int j = 0; j < M; j += 4) {
+      float4 a4[TI];
 #pragma unroll
-    for (int m = 0; m < kMaxCols; ++m)
-      if (m < nc) {
-        const int p = qq + TPR * m;
-        float v = 0.f;  // (dGhat^T Bt_j)_p = sum_k Do_pair . Rot(Phi_end) Bt_pair
-        for (int k = 0; k < K; ++k) {
-          const float b0 = Bt[j * ldn + 2 * k], b1 = Bt[j * ldn + 2 * k + 1];
-          const float ce = ecs[2 * k], se = ecs[2 * k + 1];
-          v = fmaf(__ldg(Do + (2 * k) * P + p), ce * b0 - se * b1,
-                   fmaf(__ldg(Do + (2 * k + 1) * P + p), se * b0 + ce * b1, v));
+      for (int i = 0; i < TI; ++i) a4[i] = ld4(DX + (ty + 16 * i) * ldm + j);
+      nn4<TI, NGT>(acc, a4, Bt + j * ldn, ldn, tx, NG);
+    }
+#pragma unroll
+    for (int i = 0; i < TI; ++i) {
+      const int row = ty + 16 * i, t = row / R, r = row % R;
+      if (t >= nt) continue;
+      const int64_t base = ((q.base + q.t0 + t) * a.ngroups + q.g) * R * N + (int64_t)r * N;
+#pragma unroll
+      for (int c = 0; c < NGT; ++c) {
+        const int gi = tx + 16 * c;
+        if (gi < NG) {
+          const float4 cv = ld4(Ct + row * ldn + 4 * gi);
+          const float* d = acc[i][c];
+          const int k0 = 2 * gi;  // pairs k0, k0 + 1
+          atomicAdd(dPhi + t * K + k0, d[0] * cv.y - d[1] * cv.x);
+          atomicAdd(dPhi + t * K + k0 + 1, d[2] * cv.w - d[3] * cv.z);
+          float s0, c0, s1, c1;
+          sincosf(phi[t * K + k0], &s0, &c0);
+          sincosf(phi[t * K + k0 + 1], &s1, &c1);
+          atomicAdd(reinterpret_cast<float4*>(g.dC + base + 4 * gi),  // Rot(Phi_t) dCt
+                    make_float4(c0 * d[0] - s0 * d[1], s0 * d[0] + c0 * d[1],
+                                c1 * d[2] - s1 * d[3], s1 * d[2] + c1 * d[3]));
         }
-        dxo[p] = fmaf(ws, v, acc[m]);
       }
+    }
   }
+  __syncthreads();
 
-  // <dGhat, G_c> and the outgoing rotation's angle gradient
+  // dGhat^T = (Rot(-Phi_end) dG_c+1)^T into Gt, with <dGhat, G_c> and the
+  // outgoing rotation's angle gradient sum_p (dG_1 G'_0 - dG_0 G'_1)
   {
     const float* Gn = (q.c + 1 < a.nchunks) ? Gc + (int64_t)N * P   // next chunk's start state
                                             : w.fin + (q.b * H + q.h) * (int64_t)N * P;
     float part = 0.f;
+    const int pw = P < 32 ? P : 32;  // lanes sharing one pair k
     for (int e = tid; e < K * P; e += kThreads) {
       const int k = e / P, p = e % P;
       const float o0 = __ldg(Do + (2 * k) * P + p), o1 = __ldg(Do + (2 * k + 1) * P + p);
       const float ce = ecs[2 * k], se = ecs[2 * k + 1];
       const float h0v = ce * o0 + se * o1, h1v = -se * o0 + ce * o1;  // dGhat pair
+      Gt[p * ldn + 2 * k] = h0v;
+      Gt[p * ldn + 2 * k + 1] = h1v;
       part = fmaf(h0v, __ldg(Gc + (2 * k) * P + p), fmaf(h1v, __ldg(Gc + (2 * k + 1) * P + p), part));
-      atomicAdd(dPhi + t1 * K + k,
-                o1 * __ldg(Gn + (2 * k) * P + p) - o0 * __ldg(Gn + (2 * k + 1) * P + p));
+      float cr = o1 * __ldg(Gn + (2 * k) * P + p) - o0 * __ldg(Gn + (2 * k + 1) * P + p);
+      for (int off = 1; off < pw; off <<= 1) cr += __shfl_xor_sync(0xffffffffu, cr, off);
+      if ((tid & (pw - 1)) == 0) atomicAdd(dPhi + t1 * K + k, cr);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
     if ((tid & 31) == 0) red[tid >> 5] = part;
   }
   __syncthreads();
+
+  // dBt = (M o DX)^T Ct + w X dGhat^T -> dB, dPhi (B's rotation), beta
+  {
+    float acc[TI][NGT][4];
+#pragma unroll
+    for (int i = 0; i < TI; ++i)
+#pragma unroll
+      for (int c = 0; c < NGT; ++c)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[i][c][v] = 0.f;
+    for (int p = 0; p < P; p += 4) {  // X dGhat^T first: beta_s reads it unscaled
+      float4 a4[TI];
+#pragma unroll
+      for (int i = 0; i < TI; ++i) a4[i] = ld4(X + (TI * ty + i) * ldp + p);
+      nn4<TI, NGT>(acc, a4, Gt + p * ldn, ldn, tx, NG);
+    }
+#pragma unroll
+    for (int i = 0; i < TI; ++i) {
+      const int row = TI * ty + i, s = row / R;  // this product's rows are contiguous
+      const float ws = (s < nt) ? wv[s] : 0.f;
+      float bt = 0.f;
+#pragma unroll
+      for (int c = 0; c < NGT; ++c) {
+        const int gi = tx + 16 * c;
+        if (gi < NG) {
+          const float4 bv = ld4(Bt + row * ldn + 4 * gi);
+          bt += bv.x * acc[i][c][0] + bv.y * acc[i][c][1] + bv.z * acc[i][c][2] + bv.w * acc[i][c][3];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[i][c][v] *= ws;
+        }
+      }
+      bt = sum16(bt);
+      if (tx == 0 && s < nt) atomicAdd(beta + s, bt);
+    }
+    for (int i2 = 0; i2 < M; ++i2) {
+      float av[TI];
+      ld_rows<TI>(DX + i2 * ldm + TI * ty, av);
+      tn1<TI, NGT>(acc, av, Ct + i2 * ldn, tx, NG);
+    }
+#pragma unroll
+    for (int i = 0; i < TI; ++i) {
+      const int row = TI * ty + i, s = row / R, r = row % R;
+      if (s >= nt) continue;
+      const int64_t base = ((q.base + q.t0 + s) * a.ngroups + q.g) * R * N + (int64_t)r * N;
+#pragma unroll
+      for (int c = 0; c < NGT; ++c) {
+        const int gi = tx + 16 * c;
+        if (gi < NG) {
+          const float4 bv = ld4(Bt + row * ldn + 4 * gi);
+          const float* d = acc[i][c];
+          const int k0 = 2 * gi;
+          atomicAdd(dPhi + s * K + k0, d[0] * bv.y - d[1] * bv.x);
+          atomicAdd(dPhi + s * K + k0 + 1, d[2] * bv.w - d[3] * bv.z);
+          float s0, c0, s1, c1;
+          sincosf(phi[s * K + k0], &s0, &c0);
+          sincosf(phi[s * K + k0 + 1], &s1, &c1);
+          atomicAdd(reinterpret_cast<float4*>(g.dB + base + 4 * gi),  // Rot(Phi_s) dBt
+                    make_float4(c0 * d[0] - s0 * d[1], s0 * d[0] + c0 * d[1],
+                                c1 * d[2] - s1 * d[3], s1 * d[2] + c1 * d[3]));
+        }
+      }
+    }
+  }
+
+  // dX = (M o S)^T dY + w Bt dGhat: rows TI ty + a, columns tx + 16 c
+  {
+    const int npc = P / 16;
+    float acc[TI][PCT];
+#pragma unroll
+    for (int i = 0; i < TI; ++i)
+#pragma unroll
+      for (int c = 0; c < PCT; ++c) acc[i][c] = 0.f;
+    for (int n = 0; n < N; n += 4) {  // Bt dGhat (dGhat^T rows are p)
+      float4 av[TI];
+#pragma unroll
+      for (int i = 0; i < TI; ++i) av[i] = ld4(Bt + (TI * ty + i) * ldn + n);
+#pragma unroll
+      for (int c = 0; c < PCT; ++c)
+        if (c < npc) {
+          const float4 bv = ld4(Gt + (tx + 16 * c) * ldn + n);
+#pragma unroll
+          for (int i = 0; i < TI; ++i)
+            acc[i][c] = fmaf(av[i].x, bv.x, fmaf(av[i].y, bv.y,
+                        fmaf(av[i].z, bv.z, fmaf(av[i].w, bv.w, acc[i][c]))));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < TI; ++i) {
+      const int s = (TI * ty + i) / R;
+      const float ws = (s < nt) ? wv[s] : 0.f;
+#pragma unroll
+      for (int c = 0; c < PCT; ++c) acc[i][c] *= ws;
+    }
+    for (int i2 = 0; i2 < M; ++i2) {
+      float av[TI];
+      ld_rows<TI>(S + i2 * ldm + TI * ty, av);
+#pragma unroll
+      for (int c = 0; c < PCT; ++c)
+        if (c < npc) {
+          const float bv = dY[i2 * ldp + tx + 16 * c];
+#pragma unroll
+          for (int i = 0; i < TI; ++i) acc[i][c] = fmaf(av[i], bv, acc[i][c]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < TI; ++i) {
+      const int row = TI * ty + i, s = row / R, r = row % R;
+      if (s >= nt) continue;
+      float* dxo = g.dx + ((q.base + q.t0 + s) * H + q.h) * R * P + (int64_t)r * P;
+#pragma unroll
+      for (int c = 0; c < PCT; ++c)
+        if (c < npc) dxo[tx + 16 * c] = acc[i][c];
+    }
+  }
+  __syncthreads();
+
   // w_s = exp(Lam_end - Lam_s) delta_s and the exp(Lam_end) G_c term of Ghat
   for (int u = tid; u < nt; u += kThreads) {
     float dl = -wv[u] * beta[u];
@@ -492,14 +723,36 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(const ScanArgs a, c
   }
   __syncthreads();
 
-  // through the prefix sums: d(dt theta) and theta's gradient, per pair
+  // through the prefix sums: suffix sums of dPhi over the chunk's tokens are
+  // d(dt theta); then theta's gradient and the dt term sum_k theta_k d(dt theta)_k
   for (int k = tid; k < K; k += kThreads) {
     float run = 0.f;
     for (int u = nt - 1; u >= 0; --u) {
       run += dPhi[u * K + k];
-      const int64_t to = ((q.base + q.t0 + u) * a.tgroups + q.tg) * K + k;
-      atomicAdd(g.dtheta + to, dts[u] * run);
-      atomicAdd(thT + u, __ldg(a.theta + to) * run);
+      dPhi[u * K + k] = run;
+    }
+  }
+  __syncthreads();
+  {
+    const int K4 = K / 4;                // float4 groups per token (2..32)
+    const int seg = K4 < 32 ? K4 : 32;   // lanes sharing a token
+    for (int e0 = 0; e0 < nt * K4; e0 += kThreads) {
+      const int e = e0 + tid;
+      float part = 0.f;
+      int u = 0;
+      if (e < nt * K4) {
+        u = e / K4;
+        const int k4 = e % K4;
+        const int64_t to = ((q.base + q.t0 + u) * a.tgroups + q.tg) * K + 4 * k4;
+        const float4 dp = ld4(dPhi + u * K + 4 * k4);
+        const float d = dts[u];
+        atomicAdd(reinterpret_cast<float4*>(g.dtheta + to),
+                  make_float4(d * dp.x, d * dp.y, d * dp.z, d * dp.w));
+        const float4 th = __ldg(reinterpret_cast<const float4*>(a.theta + to));
+        part = th.x * dp.x + th.y * dp.y + th.z * dp.z + th.w * dp.w;
+      }
+      for (int off = 1; off < seg; off <<= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      if (e < nt * K4 && (tid & (seg - 1)) == 0) atomicAdd(thT + u, part);
     }
   }
   __syncthreads();
@@ -531,17 +784,14 @@ cudaError_t set_smem(Kern k, size_t smem) {
 
 constexpr size_t kSmemMax = 227 * 1024;
 
-// Rows per chunk of the backward (M = Qb * R): the largest of 64, 32, 16 whose
-// shared memory and per-thread accumulators fit.
+// Rows per chunk of the backward (M = Qb * R): 64, or 32 when N = 256 (the
+// register tiles hold M/16 rows x N/4 columns, at most 32 values), if the
+// shared memory fits.
 int64_t bwd_rows(const ScanArgs& a) {
-  for (int64_t M = 64; M >= 16; M /= 2) {
-    if (M < a.R || M % a.R != 0) continue;
-    const int64_t Qb = M / a.R;
-    const ChunkSmem L((int)M, (int)a.N, (int)a.P, (int)Qb);
-    const int64_t tpr = kThreads / M;
-    if ((size_t)L.total * 4 <= kSmemMax && (a.N / 2) <= kMaxPairs * tpr &&
-        a.P <= kMaxCols * tpr)
-      return M;
+  for (int64_t M = 32; M <= 64; M *= 2) {
+    if (M < a.R || (M / 16) * (a.N / 64) > 8 || a.P > 128) continue;
+    const ChunkSmem L((int)M, (int)a.N, (int)a.P, (int)(M / a.R));
+    if ((size_t)L.total * 4 <= kSmemMax) return M;
   }
   return 0;
 }
@@ -553,19 +803,18 @@ size_t dstate_smem(const ScanArgs& f) {
 template <int R>
 cudaError_t launch_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaStream_t st) {
   cudaError_t e;
-  const int64_t opt = (f.N * f.P + kThreads - 1) / kThreads;
+  const int64_t tiles = (f.N / 4) * (f.P / 4);
   const size_t sm1 = dstate_smem(f);
   dim3 grid((unsigned)f.nchunks, (unsigned)f.nheads, (unsigned)f.batch);
-#define M3_DSTATE(O)                                                  \
+#define M3_DSTATE(T)                                                  \
   do {                                                                \
-    e = set_smem(bwd_dstate_kernel<R, O>, sm1);                       \
+    e = set_smem(bwd_dstate_kernel<R, T>, sm1);                       \
     if (e != cudaSuccess) return e;                                   \
-    bwd_dstate_kernel<R, O><<<grid, kThreads, sm1, st>>>(f, g, w);    \
+    bwd_dstate_kernel<R, T><<<grid, kThreads, sm1, st>>>(f, g, w);    \
   } while (0)
-  if (opt <= 8) M3_DSTATE(8);
-  else if (opt <= 16) M3_DSTATE(16);
-  else if (opt <= 32) M3_DSTATE(32);
-  else M3_DSTATE(64);
+  if (tiles <= kThreads) M3_DSTATE(1);
+  else if (tiles <= 2 * kThreads) M3_DSTATE(2);
+  else M3_DSTATE(4);
 #undef M3_DSTATE
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -576,11 +825,18 @@ cudaError_t launch_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaSt
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  const ChunkSmem L((int)(f.Q * R), (int)f.N, (int)f.P, (int)f.Q);
+  const int M = (int)(f.Q * R);
+  const ChunkSmem L(M, (int)f.N, (int)f.P, (int)f.Q);
   const size_t sm3 = sizeof(float) * (size_t)L.total;
-  e = set_smem(bwd_chunk_kernel<R>, sm3);
-  if (e != cudaSuccess) return e;
-  bwd_chunk_kernel<R><<<grid, kThreads, sm3, st>>>(f, g, w);
+  if (M == 64) {
+    e = set_smem(bwd_chunk_kernel<R, 64>, sm3);
+    if (e != cudaSuccess) return e;
+    bwd_chunk_kernel<R, 64><<<grid, kThreads, sm3, st>>>(f, g, w);
+  } else {
+    e = set_smem(bwd_chunk_kernel<R, 32>, sm3);
+    if (e != cudaSuccess) return e;
+    bwd_chunk_kernel<R, 32><<<grid, kThreads, sm3, st>>>(f, g, w);
+  }
   return cudaGetLastError();
 }
 

@@ -85,11 +85,13 @@ __host__ __device__ __forceinline__ WsView ws_view(const ScanArgs& a) {
 }
 
 // ---- 1. chunk state ---------------------------------------------------------
-template <int R, int OPT>
+// Thread tiles of 4 x 4 (n, p) outputs; per staged row a thread reads one float4
+// of the rotated B row and one of x (TPT tiles per thread).
+template <int R, int TPT>
 __global__ void __launch_bounds__(kThreads) chunk_state_kernel(const ScanArgs a) {
   const Geo q = chunk_geo(a, blockIdx.x);
   const int N = (int)a.N, P = (int)a.P, K = N / 2, Q = (int)a.Q;
-  extern __shared__ float sm[];
+  extern __shared__ __align__(16) float sm[];
   float* lcum = sm;
   float* gam = lcum + Q;
   float* del = gam + Q;
@@ -104,10 +106,14 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(const ScanArgs a)
     wts[i] = expf(lcum[q.nt - 1] - lcum[i]) * del[i];
   __syncthreads();
 
-  const int p = threadIdx.x % P, n0 = threadIdx.x / P, NS = kThreads / P;
-  float acc[OPT];
+  const int PG = P / 4, ntiles = (N / 4) * PG;
+  float acc[TPT][4][4];
 #pragma unroll
-  for (int i = 0; i < OPT; ++i) acc[i] = 0.f;
+  for (int m = 0; m < TPT; ++m)
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[m][u][v] = 0.f;
 
   const int TS = kTileRows / R;
   for (int s0 = 0; s0 < q.nt; s0 += TS) {
@@ -115,11 +121,18 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(const ScanArgs a)
     __syncthreads();
     const int rows = min(kTileRows, (q.nt - s0) * R);
     for (int ri = 0; ri < rows; ++ri) {
-      const float xv = Xs[ri * P + p];
 #pragma unroll
-      for (int i = 0; i < OPT; ++i) {
-        const int n = n0 + i * NS;
-        if (n < N) acc[i] = fmaf(Bs[ri * N + n], xv, acc[i]);
+      for (int m = 0; m < TPT; ++m) {
+        const int ti = threadIdx.x + kThreads * m;
+        if (ti < ntiles) {
+          const float4 bv = *reinterpret_cast<const float4*>(Bs + ri * N + 4 * (ti / PG));
+          const float4 xv = *reinterpret_cast<const float4*>(Xs + ri * P + 4 * (ti % PG));
+          const float b4[4] = {bv.x, bv.y, bv.z, bv.w}, x4[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) acc[m][u][v] = fmaf(b4[u], x4[v], acc[m][u][v]);
+        }
       }
     }
     __syncthreads();
@@ -128,9 +141,15 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(const ScanArgs a)
   const int64_t cidx = (q.b * a.nheads + q.h) * a.nchunks + q.c;
   float* S = w.S + cidx * N * P;
 #pragma unroll
-  for (int i = 0; i < OPT; ++i) {
-    const int n = n0 + i * NS;
-    if (n < N) S[n * P + p] = acc[i];
+  for (int m = 0; m < TPT; ++m) {
+    const int ti = threadIdx.x + kThreads * m;
+    if (ti < ntiles) {
+      const int n0 = 4 * (ti / PG), p0 = 4 * (ti % PG);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<float4*>(S + (n0 + u) * P + p0) =
+            make_float4(acc[m][u][0], acc[m][u][1], acc[m][u][2], acc[m][u][3]);
+    }
   }
   // an empty chunk (past a short packed sequence) passes the state unchanged
   float* sm_out = w.sum + cidx * (1 + K);
@@ -165,19 +184,34 @@ __global__ void __launch_bounds__(kThreads) state_pass_kernel(const ScanArgs a) 
     }
   }
   const WsView w = ws_view(a);
-  for (int64_t c = 0; c < a.nchunks; ++c) {
-    const int64_t cidx = (b * H + h) * a.nchunks + c;
-    float* S = w.S + cidx * N * P;
-    const float* su = w.sum + cidx * (1 + K);
-    const float s0 = S[(2 * k) * P + p], s1 = S[(2 * k + 1) * P + p];
-    S[(2 * k) * P + p] = g0;  // chunk-start state, true frame
-    S[(2 * k + 1) * P + p] = g1;
-    const float dec = expf(su[0]);
-    float sn, cs;
-    sincosf(su[1 + k], &sn, &cs);
-    const float v0 = fmaf(dec, g0, s0), v1 = fmaf(dec, g1, s1);
-    g0 = cs * v0 - sn * v1;
-    g1 = sn * v0 + cs * v1;
+  // chunks in batches of kPipe, all of a batch's loads issued before its
+  // dependent updates (the chain waits on arithmetic, not on each load)
+  constexpr int kPipe = 8;
+  for (int64_t c0 = 0; c0 < a.nchunks; c0 += kPipe) {
+    float s0[kPipe], s1[kPipe], dec[kPipe], sn[kPipe], cs[kPipe];
+#pragma unroll
+    for (int j = 0; j < kPipe; ++j) {
+      const int64_t c = c0 + j;
+      if (c >= a.nchunks) break;
+      const int64_t cidx = (b * H + h) * a.nchunks + c;
+      const float* S = w.S + cidx * N * P;
+      const float* su = w.sum + cidx * (1 + K);
+      s0[j] = S[(2 * k) * P + p];
+      s1[j] = S[(2 * k + 1) * P + p];
+      dec[j] = expf(su[0]);
+      sincosf(su[1 + k], &sn[j], &cs[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < kPipe; ++j) {
+      const int64_t c = c0 + j;
+      if (c >= a.nchunks) break;
+      float* S = w.S + ((b * H + h) * a.nchunks + c) * N * P;
+      S[(2 * k) * P + p] = g0;  // chunk-start state, true frame
+      S[(2 * k + 1) * P + p] = g1;
+      const float v0 = fmaf(dec[j], g0, s0[j]), v1 = fmaf(dec[j], g1, s1[j]);
+      g0 = cs[j] * v0 - sn[j] * v1;
+      g1 = sn[j] * v0 + cs[j] * v1;
+    }
   }
   if (a.final_state) {
     a.final_state[so + (2 * k) * P + p] = g0;
@@ -198,7 +232,7 @@ __global__ void __launch_bounds__(kThreads) chunk_output_kernel(const ScanArgs a
   if (tt0 >= q.nt) return;
   const int tt1 = min(tt0 + TT, q.nt);  // one past the last valid token
 
-  extern __shared__ float sm[];
+  extern __shared__ __align__(16) float sm[];
   float* lcum = sm;
   float* gam = lcum + Q;
   float* del = gam + Q;
@@ -302,13 +336,13 @@ cudaError_t set_smem(Kern k, size_t smem) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
 }
 
-template <int R, int OPT>
+template <int R, int TPT>
 cudaError_t launch_state(const ScanArgs& a, cudaStream_t st) {
   const size_t smem = sizeof(float) * (5 * a.Q + a.Q * (a.N / 2) + kTileRows * (a.N + a.P));
-  cudaError_t e = set_smem(chunk_state_kernel<R, OPT>, smem);
+  cudaError_t e = set_smem(chunk_state_kernel<R, TPT>, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)a.nchunks, (unsigned)a.nheads, (unsigned)a.batch);
-  chunk_state_kernel<R, OPT><<<grid, kThreads, smem, st>>>(a);
+  chunk_state_kernel<R, TPT><<<grid, kThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -330,14 +364,10 @@ cudaError_t launch_output(const ScanArgs& a, cudaStream_t st) {
 template <int R>
 cudaError_t launch_all(const ScanArgs& a, cudaStream_t st) {
   cudaError_t e;
-  const int64_t opt = (a.N * a.P + kThreads - 1) / kThreads;
-  if (opt <= 1) e = launch_state<R, 1>(a, st);
-  else if (opt <= 2) e = launch_state<R, 2>(a, st);
-  else if (opt <= 4) e = launch_state<R, 4>(a, st);
-  else if (opt <= 8) e = launch_state<R, 8>(a, st);
-  else if (opt <= 16) e = launch_state<R, 16>(a, st);
-  else if (opt <= 32) e = launch_state<R, 32>(a, st);
-  else e = launch_state<R, 64>(a, st);
+  const int64_t tiles = (a.N / 4) * (a.P / 4);  // 4 x 4 output tiles
+  if (tiles <= kThreads) e = launch_state<R, 1>(a, st);
+  else if (tiles <= 2 * kThreads) e = launch_state<R, 2>(a, st);
+  else e = launch_state<R, 4>(a, st);
   if (e != cudaSuccess) return e;
 
   const int K = (int)(a.N / 2);

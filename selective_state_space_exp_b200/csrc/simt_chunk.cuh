@@ -45,6 +45,12 @@ __device__ __forceinline__ void chunk_prep(const ScanArgs& a, const Geo& q, floa
     del[i] = lam * dt + nxt;
     lcum[i] = dt * a.A[bt * H + q.h];
   }
+  // the chunk's angle rates, one coalesced pass (the scan below reads them
+  // from shared memory)
+  for (int e = threadIdx.x; e < q.nt * K; e += blockDim.x) {
+    const int i = e / K, k = e % K;
+    phi[e] = a.theta[((q.base + q.t0 + i) * a.tgroups + q.tg) * K + k];
+  }
   __syncthreads();
   if (threadIdx.x == 0) {  // <= 64 sequential adds: the plain prefix sum
     float acc = 0.f;
@@ -53,10 +59,14 @@ __device__ __forceinline__ void chunk_prep(const ScanArgs& a, const Geo& q, floa
       lcum[i] = acc;
     }
   }
-  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+  // angle prefix sums, one pair per thread (threads from the second warp on,
+  // beside thread 0's decay sum)
+  const int first = blockDim.x > 32 ? 32 : 0;
+  for (int k = (int)threadIdx.x - first; k < K; k += (int)blockDim.x - first) {
+    if (k < 0) break;
     float acc = 0.f;
     for (int i = 0; i < q.nt; ++i) {
-      acc += dts[i] * a.theta[((q.base + q.t0 + i) * a.tgroups + q.tg) * K + k];
+      acc = fmaf(dts[i], phi[i * K + k], acc);
       phi[i * K + k] = acc;
     }
   }
