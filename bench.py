@@ -229,6 +229,43 @@ def bwd_line(inp, s, world, steps, warmup, flush, peaks):
             "roofline": alu_roofline(f, b, t, peaks)}
 
 
+def prep_line(s, world, steps, warmup, flush, peaks, psrc):
+    """m3_bc_prep (QK-norm + scale + bias of B and C) on the layer's tokens
+    with B and C per head (G = H): HBM-bound, every raw value read once and
+    every output written once."""
+    G, R, N = s.nheads, s.rank, s.dstate
+    gen = torch.Generator(device="cuda").manual_seed(1031)
+    shp = (s.batch, s.seqlen, G, R, N)
+    Br = torch.randn(shp, generator=gen, device="cuda").to(torch.bfloat16)
+    Cr = torch.randn(shp, generator=gen, device="cuda").to(torch.bfloat16)
+    prm = [torch.randn((G, R, N), generator=gen, device="cuda") for _ in range(4)]
+    Bo, Co = torch.empty_like(Br), torch.empty_like(Cr)
+
+    def step():
+        m3.m3_bc_prep(Br, Cr, *prm, B=Bo, C=Co)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    if m3.m3_stream_status() != 0:
+        raise RuntimeError("device status")
+    barrier(world)
+    t = max_over_ranks(sum(a.elapsed_time(b) * 1e-3 for a, b in ev), world) / steps
+    byt = 4.0 * Br.numel() * 2 + 4 * G * R * N * 4
+    return {"workload": f"B and C per head: [{s.batch}][{s.seqlen}][{G}][{R}][{N}] bf16 each",
+            "value": round(world * s.batch * s.seqlen / t, 1), "unit": "tokens/s",
+            "us_per_step": round(t * 1e6, 2),
+            "roofline": roofline(0.0, byt, t, peaks, psrc)}
+
+
 def decode_work(s: I.Shape):
     R, N, P = s.rank, s.dstate, s.headdim
     bh = s.batch * s.nheads
@@ -537,7 +574,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1024,
                     help="consecutive decode steps timed (each with its own token's inputs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode", "varlen", "bwd"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "varlen", "bwd", "prep"], default=None,
                     help="run one part only (for profiling); prints its own line")
     ap.add_argument("--batch", type=int, default=None,
                     help="with --only: override the workload's batch (small profiling cases)")
@@ -574,6 +611,11 @@ def main():
         dflops, dbyt = decode_work(dw.shape)
         print(json.dumps({"only": "decode", "us_per_step": round(t / args.decode_steps * 1e6, 2),
                           "roofline": roofline(dflops, dbyt, t / args.decode_steps, peaks, psrc)}))
+        return
+    if args.only == "prep":
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        print(json.dumps({"only": "prep", **prep_line(s, 1, args.steps, args.warmup, flush, peaks,
+                                                      psrc)}))
         return
     if args.only == "bwd":
         inp = I.make_scan_inputs(I.Workload(s), seed=1001, device="cuda")
@@ -629,6 +671,9 @@ def main():
     # a packed batch of mixed lengths with the same layer shape
     varlen = varlen_line(s, rank, world, max(3, args.steps // 2), args.warmup, flush, peaks,
                          psrc)
+
+    # QK-norm + bias prep of B and C (block-level step before the scan)
+    bc_prep = prep_line(s, world, 10, args.warmup, flush, peaks, psrc)
 
     # backward of the same scan (gradients of every input), CUDA cores fp32
     backward = bwd_line(inp, s, world, 3, args.warmup, flush, peaks)
@@ -705,6 +750,7 @@ def main():
         line["secondary"] = secondary
     line["varlen"] = varlen
     line["backward"] = backward
+    line["bc_prep"] = bc_prep
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_prefill(inp_host, s)
     if rank == 0:

@@ -246,6 +246,28 @@ M3_API int m3_scan_bwd(const m3_shape* shape, const void* x, const float* dt, co
                        float* dx_prev, void* workspace, size_t workspace_bytes,
                        m3_stream_t stream);
 
+/* ---- B / C projection prep ------------------------------------------------------
+ * QK-norm and learnable bias after the B and C projections (PaperWeekly page
+ * section 2.4, "normalisation and bias"; Figure 4).  For every row of N values
+ * (one per token, group and rank):
+ *   out[n] = raw[n] / sqrt(mean_m raw[m]^2 + eps) * weight[n] + bias[n],
+ * computed in fp32 and rounded to the io dtype (nearest even for bf16).  The
+ * outputs are the B and C that m3_scan_fwd and m3_decode_step take.
+ *
+ *   shape      batch, seqlen (tokens = batch * seqlen; 1 for a decode step),
+ *              ngroups, rank, dstate, io_dtype; the other fields are checked
+ *              as usual but not used.
+ *   B_raw, B   [tokens][G][R][N] io dtype; both NULL to skip B.
+ *   C_raw, C   the same for C.
+ *   *_weight,
+ *   *_bias     [G][R][N] fp32, or NULL for 1 and 0.
+ *   eps        >= 0.
+ * All pointers are 16-byte aligned device pointers.  An output may be its
+ * own input (in place); any other overlap returns M3_ERR_INVALID_ARGUMENT. */
+M3_API int m3_bc_prep(const m3_shape* shape, const void* B_raw, const void* C_raw,
+                      const float* B_weight, const float* B_bias, const float* C_weight,
+                      const float* C_bias, float eps, void* B, void* C, m3_stream_t stream);
+
 /* ---- packed variable-length batch -------------------------------------------
  * Several sequences of different lengths in one call, stored back to back
  * along the token dimension (no padding): sequence i is tokens

@@ -292,6 +292,35 @@ M3_API int m3_scan_bwd(const m3_shape* s, const void* x, const float* dt, const 
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 
+M3_API int m3_bc_prep(const m3_shape* s, const void* B_raw, const void* C_raw,
+                      const float* B_weight, const float* B_bias, const float* C_weight,
+                      const float* C_bias, float eps, void* B, void* C, m3_stream_t stream) {
+  int st = check_common(s);
+  if (st != M3_OK) return st;
+  if ((B_raw == nullptr) != (B == nullptr) || (C_raw == nullptr) != (C == nullptr))
+    return M3_ERR_INVALID_ARGUMENT;
+  if (!(eps >= 0.f) || !(eps < 1e30f)) return M3_ERR_INVALID_ARGUMENT;
+  const void* v16[] = {B_raw, C_raw, B_weight, B_bias, C_weight, C_bias, B, C};
+  for (const void* p : v16)
+    if (p && !aligned(p, 16)) return M3_ERR_ALIGNMENT;
+  // an output may be its own input (in place); other overlaps are not allowed
+  const size_t esz = s->io_dtype == M3_BF16 ? 2 : 4;
+  const int64_t rows = s->batch * s->seqlen * s->ngroups * s->rank;
+  const size_t nb = esz * (size_t)rows * (size_t)s->dstate;
+  auto overlap = [&](const void* a, const void* b) {
+    const char* x = static_cast<const char*>(a);
+    const char* y = static_cast<const char*>(b);
+    return a && b && x != y && x < y + nb && y < x + nb;
+  };
+  if (overlap(B, B_raw) || overlap(C, C_raw) || overlap(B, C) || overlap(B, C_raw) ||
+      overlap(C, B_raw) || (B && B == C))
+    return M3_ERR_INVALID_ARGUMENT;
+  cudaError_t e = bc_prep_launch(s->batch * s->seqlen, s->dstate, s->ngroups * s->rank,
+                                 s->io_dtype == M3_BF16, B_raw, C_raw, B_weight, B_bias, C_weight,
+                                 C_bias, eps, B, C, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
 M3_API int m3_scan_state(const m3_shape* s, const void* x, const float* dt, const float* A,
                          const float* lam, const float* theta, const void* B, const void* C,
                          const float* h0, const void* B_prev, const void* x_prev,

@@ -123,6 +123,12 @@ size_t bwd_workspace(const ScanArgs& a);
 bool bwd_supported(const ScanArgs& a);
 cudaError_t bwd_launch(const ScanArgs& a, const BwdArgs& g, cudaStream_t s);
 
+// B / C prep: QK-norm, per-channel scale and bias over rows of N values,
+// tensors [tokens][gr][N] with gr = G * R channel rows.
+cudaError_t bc_prep_launch(int64_t tokens, int64_t N, int64_t gr, bool bf16, const void* Braw,
+                           const void* Craw, const float* wB, const float* bB, const float* wC,
+                           const float* bC, float eps, void* Bo, void* Co, cudaStream_t s);
+
 // Decode step.
 cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t s);
 

@@ -102,6 +102,8 @@ def load() -> ctypes.CDLL:
             L.m3_scan_bwd_workspace_size.restype = ctypes.c_int
             L.m3_scan_bwd.argtypes = [sp] + [vp] * 23 + [ctypes.c_size_t, vp]
             L.m3_scan_bwd.restype = ctypes.c_int
+            L.m3_bc_prep.argtypes = [sp] + [vp] * 6 + [ctypes.c_float, vp, vp, vp]
+            L.m3_bc_prep.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -222,6 +224,28 @@ def m3_scan_fwd_varlen(cu_seqlens, x, dt, A, lam, theta, B, C, chunk: int = 64, 
                                    ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check("m3_scan_fwd_varlen", st)
     return y, final_state
+
+
+def m3_bc_prep(B_raw=None, C_raw=None, B_weight=None, B_bias=None, C_weight=None, C_bias=None,
+               eps: float = 1e-6, *, B=None, C=None, stream=None):
+    """QK-norm + per-channel scale + bias of raw B / C projections, either
+    [b][L][G][R][N] (scan layout) or [b][G][R][N] (decode layout), io dtype.
+    weight / bias [G][R][N] fp32 or None.  Returns (B, C) (None for a skipped one)."""
+    ref = B_raw if B_raw is not None else C_raw
+    if ref.dim() == 5:
+        b, L, G, R, N = ref.shape
+    else:
+        (b, G, R, N), L = ref.shape, 1
+    if B_raw is not None and B is None:
+        B = torch.empty_like(B_raw)
+    if C_raw is not None and C is None:
+        C = torch.empty_like(C_raw)
+    shape = make_shape(b, L, G, G, 16, N, R, 64, ref.dtype)
+    st = load().m3_bc_prep(ctypes.byref(shape), _ptr(B_raw), _ptr(C_raw), _ptr(B_weight),
+                           _ptr(B_bias), _ptr(C_weight), _ptr(C_bias), ctypes.c_float(eps),
+                           _ptr(B), _ptr(C), _stream(stream))
+    _check("m3_bc_prep", st)
+    return B, C
 
 
 def bwd_workspace_size(shape: Shape) -> int:

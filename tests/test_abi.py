@@ -152,3 +152,24 @@ def test_scan_plan(lib, kw, tc, seg, launches):
         assert g.value == seg
     assert lib.m3_scan_plan(ctypes.byref(s), None, None, None) == 0
     assert lib.m3_scan_plan(None, None, None, None) == -1
+
+
+def prep_call(lib, s, **over):
+    args = dict(Br=P[0], Cr=P[1], wB=None, bB=None, wC=None, bC=None, eps=1e-6, B=P[2], C=P[3])
+    args.update(over)
+    return lib.m3_bc_prep(ctypes.byref(s), args["Br"], args["Cr"], args["wB"], args["bB"],
+                          args["wC"], args["bC"], ctypes.c_float(args["eps"]), args["B"],
+                          args["C"], None)
+
+
+def test_bc_prep_rejects_bad_arguments(lib):
+    s = shape()  # 200 tokens x 128 bf16: 51200 bytes per tensor
+    assert prep_call(lib, s, B=None) == -1                         # raw B without output
+    assert prep_call(lib, s, Cr=None) == -1                        # C output without raw C
+    assert prep_call(lib, s, eps=-1.0) == -1
+    assert prep_call(lib, s, eps=float("nan")) == -1
+    assert prep_call(lib, s, B=ctypes.c_void_p(A16 + 0x100000 + 4096)) == -1   # B overlaps raw C
+    assert prep_call(lib, s, B=P[3], C=P[3]) == -1                 # one output for both
+    assert prep_call(lib, s, B=ctypes.c_void_p(A16 + 0x200000 + 8)) == -3
+    assert prep_call(lib, s, wB=ctypes.c_void_p(A16 + 0x500000 + 4)) == -3
+    assert prep_call(lib, shape(rank=3)) == -2
