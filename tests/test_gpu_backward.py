@@ -113,3 +113,39 @@ def test_bwd_chunk_invariant():
     for k in outs[0]:
         assert torch.equal(outs[0][k], outs[1][k]) or \
             rel_err(outs[0][k].cpu().numpy(), outs[1][k].cpu().numpy()) < 1e-6, k
+
+
+@pytest.mark.parametrize("R", [1, 4])
+def test_bwd_full_size_sampled_chains(R):
+    """The bench's backward workload (b=8, L=2048, H=64, N=128, P=64, bf16 io,
+    the workload's input recipe), gradients of a seeded sample of (batch, head)
+    chains: everything a chain owns (dx, d dt, dA, d lam, dh0) against the
+    gradient oracle run on that chain alone.  B, C and theta are shared by all
+    64 heads (G = 1), so their gradients are sums over chains; they are covered
+    by the small cases above."""
+    w = I.Workload(I.Shape(8, 2048, 64, 64, 128, R, 1, 64, "bf16"), with_h0=True)
+    inp = I.make_scan_inputs(w, seed=1001 + R)
+    gen = torch.Generator().manual_seed(900 + R)
+    dy = torch.randn(inp["x"].shape, generator=gen).to(torch.bfloat16)
+    dfin = torch.randn(inp["h0"].shape, generator=gen)
+    g = to_dev(inp)
+    got = m3.m3_scan_bwd(g["x"], g["dt"], g["A"], g["lam"], g["theta"], g["B"], g["C"],
+                         dy.cuda(), 64, g["h0"], None, None, dfin.cuda())
+    assert m3.m3_stream_status() == 0
+    got = {k: v.cpu().numpy() for k, v in got.items()}
+    for c in I.sample_chains(8, 64, 3, seed=11 + R):
+        b, h = divmod(c, 64)
+        one = {"x": inp["x"][b:b + 1, :, h:h + 1], "dt": inp["dt"][b:b + 1, :, h:h + 1],
+               "A": inp["A"][b:b + 1, :, h:h + 1], "lam": inp["lam"][b:b + 1, :, h:h + 1],
+               "theta": inp["theta"][b:b + 1], "B": inp["B"][b:b + 1], "C": inp["C"][b:b + 1],
+               "h0": inp["h0"][b:b + 1, h:h + 1]}
+        _, _, ref = m3_grad.scan_grads(*[one.get(k) for k in m3_grad.NAMES],
+                                       dy=dy[b:b + 1, :, h:h + 1],
+                                       d_final=dfin[b:b + 1, h:h + 1])
+        errs = {"x": rel_err(got["x"][b, :, h], ref["x"][0, :, 0]),
+                "dt": rel_err(got["dt"][b, :, h], ref["dt"][0, :, 0]),
+                "A": rel_err(got["A"][b, :, h], ref["A"][0, :, 0]),
+                "lam": rel_err(got["lam"][b, :, h], ref["lam"][0, :, 0]),
+                "h0": rel_err(got["h0"][b, h], ref["h0"][0, 0])}
+        bad = {k: v for k, v in errs.items() if not v <= BAR}
+        assert not bad, (c, errs)

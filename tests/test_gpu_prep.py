@@ -101,3 +101,28 @@ def test_prep_then_scan_matches_oracle():
                          Bref.float().bfloat16(), Cref.float().bfloat16(), inp["h0"])
     assert rel_err(y.float().cpu().numpy(), yo) <= TOL["bf16"]
     assert rel_err(fs.cpu().numpy(), ho) <= TOL["bf16"]
+
+
+def test_prep_bench_workload_sampled_rows():
+    """The bench's prep line (per-head B and C: [8][2048][64][1][128] bf16 each),
+    a seeded sample of 4096 rows of each output against the oracle."""
+    G, N = 64, 128
+    gen = torch.Generator(device="cuda").manual_seed(1031)
+    shp = (8, 2048, G, 1, N)
+    Br = torch.randn(shp, generator=gen, device="cuda").to(torch.bfloat16)
+    Cr = torch.randn(shp, generator=gen, device="cuda").to(torch.bfloat16)
+    prm = [torch.randn((G, 1, N), generator=gen, device="cuda") for _ in range(4)]
+    Bo, Co = m3.m3_bc_prep(Br, Cr, *prm)
+    assert m3.m3_stream_status() == 0
+    rows = np.random.default_rng(7).choice(8 * 2048 * G, size=4096, replace=False)
+    for raw, out, w, b in ((Br, Bo, prm[0], prm[1]), (Cr, Co, prm[2], prm[3])):
+        r2 = raw.reshape(-1, N)[torch.from_numpy(rows).cuda()].cpu()
+        o2 = out.reshape(-1, N)[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+        ch = torch.from_numpy(rows % G)
+        wr, br = w.reshape(G, N).cpu()[ch], b.reshape(G, N).cpu()[ch]
+        wr4 = wr.double().numpy()[:, None, None, :]
+        br4 = br.double().numpy()[:, None, None, :]
+        ref = m3_prep.qk_norm_bias(r2[:, None, None, :], wr4, br4)[:, 0, 0, :]
+        mag = (np.abs(m3_prep.qk_norm_bias(r2[:, None, None, :], wr4, None))
+               + np.abs(br4))[:, 0, 0, :]
+        assert ulp_check(o2, ref, mag) == 0

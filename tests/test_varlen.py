@@ -189,3 +189,20 @@ def test_varlen_bad_offsets_reported(simt):
     yo, ho = oracle_varlen(ref)
     assert rel_err(yg[:220], yo[:220]) <= TOL["bf16"]
     assert rel_err(hg[:2], ho) <= TOL["bf16"]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("R", [1, 4])
+def test_varlen_bench_workload(R):
+    """The bench's packed-batch line exactly: 16 sequences of the seeded length
+    mix up to 2048 tokens, the layer shape (H=64, N=128, P=64, bf16), every
+    output against the oracle."""
+    need_gpu()
+    s = I.Shape(1, 1, 64, 64, 128, R, 1, 64, "bf16")
+    lengths = I.varlen_lengths(16, 2048, 64, seed=1021)
+    inp = I.make_varlen_inputs(I.Workload(s), lengths, seed=1021)
+    yg, hg, st = gpu_varlen(inp, 64, max_seqlen=2048)
+    assert st == 0
+    yo, ho = oracle_varlen(inp)
+    assert np.isfinite(yg).all()
+    assert rel_err(yg, yo) <= TOL["bf16"] and rel_err(hg, ho) <= TOL["bf16"]
