@@ -784,9 +784,10 @@ cudaError_t set_smem(Kern k, size_t smem) {
 
 constexpr size_t kSmemMax = 227 * 1024;
 
-// Rows per chunk of the backward (M = Qb * R): 64, or 32 when N = 256 (the
-// register tiles hold M/16 rows x N/4 columns, at most 32 values), if the
-// shared memory fits.
+// Rows per chunk of the backward (M = Qb * R): 32 (about 110 KB of shared
+// memory at N = 128, P = 64, so two CTAs share an SM, and half the quadratic
+// work of 64-row chunks), 64 only if 32 rows do not fit; the register tiles
+// hold M/16 rows x N/4 columns, at most 32 values.
 int64_t bwd_rows(const ScanArgs& a) {
   for (int64_t M = 32; M <= 64; M *= 2) {
     if (M < a.R || (M / 16) * (a.N / 64) > 8 || a.P > 128) continue;
