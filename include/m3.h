@@ -234,9 +234,17 @@ M3_API int m3_scan_fwd_noalloc(const m3_shape* shape, const void* x, const float
  *   dx_prev     [b][G][R][N] and [b][H][R][P] fp32, both NULL or both
  *               non-NULL; zeros when B_prev is NULL.
  *   workspace   at least m3_scan_bwd_workspace_size() bytes, 256-byte aligned.
- * Packed variable-length batches are not supported by this call.  Returns
- * M3_OK when the work was enqueued, M3_ERR_UNSUPPORTED for shapes whose
- * chunk tiles do not fit one CTA's shared memory. */
+ * Returns M3_OK when the work was enqueued, M3_ERR_UNSUPPORTED for shapes
+ * whose chunk tiles do not fit one CTA's shared memory.
+ *
+ * m3_scan_bwd_varlen is the same for a packed variable-length batch, with
+ * cu_seqlens / total_tokens / layouts as m3_scan_fwd_varlen: dy and dx
+ * [T][H][R][P], ddt, dA, dlam [T][H], dtheta [T][Gt][N/2], dB, dC
+ * [T][G][R][N]; d_final, dh0 [S][H][N][P]; dB_prev, dx_prev per sequence.
+ * Rows of the token dimension outside every sequence are left undefined
+ * in dx and dA (zero in the others).  The workspace size is
+ * m3_scan_bwd_workspace_size(shape) with shape->batch = S and
+ * shape->seqlen = the longest sequence. */
 M3_API int m3_scan_bwd_workspace_size(const m3_shape* shape, size_t* bytes);
 M3_API int m3_scan_bwd(const m3_shape* shape, const void* x, const float* dt, const float* A,
                        const float* lam, const float* theta, const void* B, const void* C,
@@ -245,6 +253,15 @@ M3_API int m3_scan_bwd(const m3_shape* shape, const void* x, const float* dt, co
                        float* dtheta, float* dB, float* dC, float* dh0, float* dB_prev,
                        float* dx_prev, void* workspace, size_t workspace_bytes,
                        m3_stream_t stream);
+M3_API int m3_scan_bwd_varlen(const m3_shape* shape, const int32_t* cu_seqlens,
+                              int64_t total_tokens, const void* x, const float* dt,
+                              const float* A, const float* lam, const float* theta,
+                              const void* B, const void* C, const float* h0,
+                              const void* B_prev, const void* x_prev, const void* dy,
+                              const float* d_final, float* dx, float* ddt, float* dA,
+                              float* dlam, float* dtheta, float* dB, float* dC, float* dh0,
+                              float* dB_prev, float* dx_prev, void* workspace,
+                              size_t workspace_bytes, m3_stream_t stream);
 
 /* ---- B / C projection prep ------------------------------------------------------
  * QK-norm and learnable bias after the B and C projections (PaperWeekly page

@@ -92,3 +92,33 @@ def scan_grads(x, dt, A, lam, theta, B, C, h0=None, B_prev=None, x_prev=None, dy
     grads = {n: (np.zeros(tuple(leaves[n].shape)) if g is None else g.numpy())
              for n, g in zip(names, gs)}
     return y.detach().numpy(), zL.detach().numpy(), grads
+
+
+def scan_grads_varlen(cu_seqlens, x, dt, A, lam, theta, B, C, h0=None, B_prev=None,
+                      x_prev=None, dy=None, d_final=None):
+    """Gradients for a packed batch (layouts of the packed scan: token
+    dimension first, no batch dimension; h0, B_prev, x_prev, d_final per
+    sequence).  No state or input is shared between sequences, so each
+    sequence's gradients are scan_grads of that sequence alone; they are
+    written into packed arrays (rows outside every sequence stay zero)."""
+    cu = [int(v) for v in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    packed = {"x": x, "dt": dt, "A": A, "lam": lam, "theta": theta, "B": B, "C": C}
+    per_seq = {"h0": h0, "B_prev": B_prev, "x_prev": x_prev}
+    out = {k: np.zeros(tuple(v.shape)) for k, v in packed.items()}
+    for k, v in per_seq.items():
+        if v is not None:
+            out[k] = np.zeros(tuple(v.shape))
+    for i in range(len(cu) - 1):
+        a, e = cu[i], cu[i + 1]
+        one = {k: v[None, a:e] for k, v in packed.items()}
+        for k, v in per_seq.items():
+            one[k] = None if v is None else v[i:i + 1]
+        _, _, g = scan_grads(*[one[k] for k in NAMES],
+                             dy=None if dy is None else dy[None, a:e],
+                             d_final=None if d_final is None else d_final[i:i + 1])
+        for k in packed:
+            out[k][a:e] = g[k][0]
+        for k in per_seq:
+            if k in g:
+                out[k][i] = g[k][0]
+    return out

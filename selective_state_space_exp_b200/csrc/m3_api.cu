@@ -225,23 +225,28 @@ M3_API int m3_scan_bwd_workspace_size(const m3_shape* s, size_t* bytes) {
   return M3_OK;
 }
 
-M3_API int m3_scan_bwd(const m3_shape* s, const void* x, const float* dt, const float* A,
-                       const float* lam, const float* theta, const void* B, const void* C,
-                       const float* h0, const void* B_prev, const void* x_prev, const void* dy,
-                       const float* d_final, float* dx, float* ddt, float* dA, float* dlam,
-                       float* dtheta, float* dB, float* dC, float* dh0, float* dB_prev,
-                       float* dx_prev, void* workspace, size_t workspace_bytes,
-                       m3_stream_t stream) {
+namespace {
+
+int bwd_call(const m3_shape* s, const int32_t* cu_seqlens, int64_t total_tokens, const void* x,
+             const float* dt, const float* A, const float* lam, const float* theta,
+             const void* B, const void* C, const float* h0, const void* B_prev,
+             const void* x_prev, const void* dy, const float* d_final, float* dx, float* ddt,
+             float* dA, float* dlam, float* dtheta, float* dB, float* dC, float* dh0,
+             float* dB_prev, float* dx_prev, void* workspace, size_t workspace_bytes,
+             m3_stream_t stream) {
   int st = check_common(s);
   if (st != M3_OK) return st;
+  const bool varlen = cu_seqlens != nullptr;
+  if (varlen && (total_tokens < 0 || !aligned(cu_seqlens, 4))) return M3_ERR_INVALID_ARGUMENT;
   if ((B_prev == nullptr) != (x_prev == nullptr)) return M3_ERR_INVALID_ARGUMENT;
   if ((dB_prev == nullptr) != (dx_prev == nullptr)) return M3_ERR_INVALID_ARGUMENT;
   const bool bf16 = s->io_dtype == M3_BF16;
   if (bf16 && s->headdim % 8 != 0) return M3_ERR_UNSUPPORTED;
   ScanArgs a = make_scan_args(s);
   if (!bwd_supported(a)) return M3_ERR_UNSUPPORTED;
-  if (s->seqlen > 0 && (!x || !dt || !A || !lam || !theta || !B || !C || !dy || !dx || !ddt ||
-                        !dA || !dlam || !dtheta || !dB || !dC))
+  const bool empty = s->seqlen == 0 || (varlen && total_tokens == 0);
+  if (!empty && (!x || !dt || !A || !lam || !theta || !B || !C || !dy || !dx || !ddt ||
+                 !dA || !dlam || !dtheta || !dB || !dC))
     return M3_ERR_INVALID_ARGUMENT;
   const void* v16[] = {x, B, C, dy, h0, d_final, B_prev, x_prev, theta, dx, dtheta, dB, dC,
                        dh0, dB_prev, dx_prev};
@@ -253,7 +258,7 @@ M3_API int m3_scan_bwd(const m3_shape* s, const void* x, const float* dt, const 
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const size_t sb = sizeof(float) * s->batch * s->nheads * s->dstate * s->headdim;
 
-  if (s->seqlen == 0) {  // no token: the state is h0, so dh0 = d_final; nothing else
+  if (empty) {  // no token: the state is h0, so dh0 = d_final; nothing else
     if (dh0) {
       cudaError_t e = d_final ? cudaMemcpyAsync(dh0, d_final, sb, cudaMemcpyDeviceToDevice, cs)
                               : cudaMemsetAsync(dh0, 0, sb, cs);
@@ -274,7 +279,8 @@ M3_API int m3_scan_bwd(const m3_shape* s, const void* x, const float* dt, const 
   a.h0 = h0; a.B_prev = B_prev; a.x_prev = x_prev;
   a.ws = static_cast<char*>(workspace);
   a.ws_bytes = workspace_bytes;
-  a.total_tokens = s->batch * s->seqlen;
+  a.cu_seqlens = cu_seqlens;
+  a.total_tokens = varlen ? total_tokens : s->batch * s->seqlen;
   if (status_word(&a.status) != M3_OK) return M3_ERR_CUDA;
   BwdArgs g;
   g.dy = dy; g.d_final = d_final; g.dx = dx; g.ddt = ddt; g.dA = dA; g.dlam = dlam;
@@ -290,6 +296,34 @@ M3_API int m3_scan_bwd(const m3_shape* s, const void* x, const float* dt, const 
   }
   cudaError_t e = bwd_launch(a, g, cs);
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+}  // namespace
+
+M3_API int m3_scan_bwd(const m3_shape* s, const void* x, const float* dt, const float* A,
+                       const float* lam, const float* theta, const void* B, const void* C,
+                       const float* h0, const void* B_prev, const void* x_prev, const void* dy,
+                       const float* d_final, float* dx, float* ddt, float* dA, float* dlam,
+                       float* dtheta, float* dB, float* dC, float* dh0, float* dB_prev,
+                       float* dx_prev, void* workspace, size_t workspace_bytes,
+                       m3_stream_t stream) {
+  return bwd_call(s, nullptr, 0, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev, dy, d_final,
+                  dx, ddt, dA, dlam, dtheta, dB, dC, dh0, dB_prev, dx_prev, workspace,
+                  workspace_bytes, stream);
+}
+
+M3_API int m3_scan_bwd_varlen(const m3_shape* s, const int32_t* cu_seqlens, int64_t total_tokens,
+                              const void* x, const float* dt, const float* A, const float* lam,
+                              const float* theta, const void* B, const void* C, const float* h0,
+                              const void* B_prev, const void* x_prev, const void* dy,
+                              const float* d_final, float* dx, float* ddt, float* dA,
+                              float* dlam, float* dtheta, float* dB, float* dC, float* dh0,
+                              float* dB_prev, float* dx_prev, void* workspace,
+                              size_t workspace_bytes, m3_stream_t stream) {
+  if (!cu_seqlens) return M3_ERR_INVALID_ARGUMENT;
+  return bwd_call(s, cu_seqlens, total_tokens, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev,
+                  dy, d_final, dx, ddt, dA, dlam, dtheta, dB, dC, dh0, dB_prev, dx_prev,
+                  workspace, workspace_bytes, stream);
 }
 
 M3_API int m3_bc_prep(const m3_shape* s, const void* B_raw, const void* C_raw,

@@ -186,9 +186,10 @@ __global__ void __launch_bounds__(kThreads) bwd_state_pass_kernel(const ScanArgs
     g.dh0[so + (2 * k) * P + p] = d0;
     g.dh0[so + (2 * k + 1) * P + p] = d1;
   }
-  if (a.B_prev && a.seqlen > 0) {  // G_0 = h0 + eps_0 B_prev x_prev^T
+  const Chain chn = chain_of(a, b);
+  if (a.B_prev && chn.len > 0) {  // G_0 = h0 + eps_0 B_prev x_prev^T
     const int64_t grp = h / (H / a.ngroups);
-    const int64_t t0 = (b * a.seqlen) * H + h;  // token 0 of this chain
+    const int64_t t0 = chn.base * H + h;  // token 0 of this chain
     const float lam0 = a.lam[t0], dt0 = a.dt[t0], eps0 = (1.f - lam0) * dt0;
     float part = 0.f;
     for (int r = 0; r < R; ++r) {
@@ -853,7 +854,7 @@ BwdWs carve(const ScanArgs& f) {
 
 }  // namespace
 
-bool bwd_supported(const ScanArgs& a) { return bwd_rows(a) > 0 && a.cu_seqlens == nullptr; }
+bool bwd_supported(const ScanArgs& a) { return bwd_rows(a) > 0; }
 
 size_t bwd_workspace(const ScanArgs& a) {
   const int64_t M = bwd_rows(a);
@@ -871,7 +872,7 @@ cudaError_t bwd_launch(const ScanArgs& a, const BwdArgs& g, cudaStream_t st) {
   BwdWs w = carve(f);
   f.final_state = w.fin;
   // outputs accumulated with atomic adds start from zero
-  const int64_t tok = a.batch * a.seqlen;
+  const int64_t tok = a.total_tokens;  // batch x seqlen, or a packed batch's rows
   const int64_t K = a.N / 2;
   struct Z { float* p; int64_t n; } zs[] = {
       {g.ddt, tok * a.nheads}, {g.dlam, tok * a.nheads}, {g.dtheta, tok * a.tgroups * K},

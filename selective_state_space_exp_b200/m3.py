@@ -102,6 +102,9 @@ def load() -> ctypes.CDLL:
             L.m3_scan_bwd_workspace_size.restype = ctypes.c_int
             L.m3_scan_bwd.argtypes = [sp] + [vp] * 23 + [ctypes.c_size_t, vp]
             L.m3_scan_bwd.restype = ctypes.c_int
+            L.m3_scan_bwd_varlen.argtypes = [sp, vp, ctypes.c_int64] + [vp] * 23 + \
+                [ctypes.c_size_t, vp]
+            L.m3_scan_bwd_varlen.restype = ctypes.c_int
             L.m3_bc_prep.argtypes = [sp] + [vp] * 6 + [ctypes.c_float, vp, vp, vp]
             L.m3_bc_prep.restype = ctypes.c_int
             _lib = L
@@ -286,6 +289,43 @@ def m3_scan_bwd(x, dt, A, lam, theta, B, C, dy, chunk: int = 64, h0=None, B_prev
                             _ptr(g.get("h0")), _ptr(g.get("B_prev")), _ptr(g.get("x_prev")),
                             _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check("m3_scan_bwd", st)
+    return g
+
+
+def m3_scan_bwd_varlen(cu_seqlens, x, dt, A, lam, theta, B, C, dy, chunk: int = 64, h0=None,
+                       B_prev=None, x_prev=None, d_final=None, *, max_seqlen=None,
+                       want_dh0=True, workspace=None, stream=None):
+    """Backward of m3_scan_fwd_varlen (packed tensors without a batch
+    dimension, as there).  Returns the gradient dict of m3_scan_bwd."""
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    S = cu_seqlens.numel() - 1
+    T, H, R, P = x.shape
+    G, N = B.shape[1], B.shape[3]
+    if max_seqlen is None:
+        max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item()) if S > 0 else 0
+    shape = make_shape(S, max_seqlen, H, G, P, N, R, chunk, x.dtype, False)
+    shape.flags |= theta_flag(theta.shape[1], G, H)
+    dev, f32 = x.device, torch.float32
+    g = {k: torch.empty(v.shape, dtype=f32, device=dev)
+         for k, v in (("x", x), ("dt", dt), ("A", A), ("lam", lam), ("theta", theta), ("B", B),
+                      ("C", C))}
+    if want_dh0:
+        g["h0"] = torch.empty((S, H, N, P), dtype=f32, device=dev)
+    if B_prev is not None:
+        g["B_prev"] = torch.empty(B_prev.shape, dtype=f32, device=dev)
+        g["x_prev"] = torch.empty(x_prev.shape, dtype=f32, device=dev)
+    need = bwd_workspace_size(shape)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    st = load().m3_scan_bwd_varlen(
+        ctypes.byref(shape), _ptr(cu_seqlens), ctypes.c_int64(T), _ptr(x), _ptr(dt), _ptr(A),
+        _ptr(lam), _ptr(theta), _ptr(B), _ptr(C), _ptr(h0), _ptr(B_prev), _ptr(x_prev), _ptr(dy),
+        _ptr(d_final), _ptr(g["x"]), _ptr(g["dt"]), _ptr(g["A"]), _ptr(g["lam"]),
+        _ptr(g["theta"]), _ptr(g["B"]), _ptr(g["C"]), _ptr(g.get("h0")), _ptr(g.get("B_prev")),
+        _ptr(g.get("x_prev")), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+        _stream(stream))
+    _check("m3_scan_bwd_varlen", st)
     return g
 
 

@@ -77,3 +77,30 @@ def test_gradient_of_y_only_and_final_only_add_up():
     _, _, g_f = m3_grad.scan_grads(*args, d_final=dfin)
     for n in m3_grad.NAMES:
         assert np.allclose(g_both[n], g_y[n] + g_f[n], rtol=1e-12, atol=1e-12)
+
+
+def test_varlen_gradients_are_the_batched_ones():
+    """Packed sequences of one length: the per-sequence gradients placed back in
+    the packed layout are the batched call's (a misplaced slice or a gradient
+    leaking across a boundary fails)."""
+    S, L = 3, 11
+    inp = tiny(L=S * L, H=2, G=1, R=2, N=4, P=3, seed=41)
+    rng = np.random.default_rng(8)
+    flat = {k: inp[k][0] for k in ("x", "dt", "A", "lam", "theta", "B", "C")}
+    per = {"h0": rng.standard_normal((S,) + inp["h0"].shape[1:]),
+           "B_prev": rng.standard_normal((S,) + inp["B_prev"].shape[1:]),
+           "x_prev": rng.standard_normal((S,) + inp["x_prev"].shape[1:])}
+    dy = rng.standard_normal(flat["x"].shape)
+    dfin = rng.standard_normal(per["h0"].shape)
+    got = m3_grad.scan_grads_varlen([0, L, 2 * L, 3 * L], *[flat[k] for k in
+                                    ("x", "dt", "A", "lam", "theta", "B", "C")],
+                                    per["h0"], per["B_prev"], per["x_prev"], dy=dy,
+                                    d_final=dfin)
+    bat = {k: v.reshape((S, L) + v.shape[1:]) for k, v in flat.items()}
+    _, _, ref = m3_grad.scan_grads(*[bat[k] for k in ("x", "dt", "A", "lam", "theta", "B", "C")],
+                                   per["h0"], per["B_prev"], per["x_prev"],
+                                   dy=dy.reshape((S, L) + dy.shape[1:]), d_final=dfin)
+    for k in ("x", "dt", "A", "lam", "theta", "B", "C"):
+        assert np.allclose(got[k], ref[k].reshape(got[k].shape), rtol=1e-12, atol=1e-13), k
+    for k in ("h0", "B_prev", "x_prev"):
+        assert np.allclose(got[k], ref[k], rtol=1e-12, atol=1e-13), k
