@@ -234,6 +234,10 @@ M3_API int m3_scan_fwd_noalloc(const m3_shape* shape, const void* x, const float
  *   dx_prev     [b][G][R][N] and [b][H][R][P] fp32, both NULL or both
  *               non-NULL; zeros when B_prev is NULL.
  *   workspace   at least m3_scan_bwd_workspace_size() bytes, 256-byte aligned.
+ * dB, dC and dtheta sum contributions of all heads of a group, and ddt, dlam
+ * of a chunk's first token also receive the previous chunk's term; these sums
+ * are floating-point atomic adds, so those outputs can differ in the last
+ * bits from run to run (dx, dA, dh0 are written once and are reproducible).
  * Returns M3_OK when the work was enqueued, M3_ERR_UNSUPPORTED for shapes
  * whose chunk tiles do not fit one CTA's shared memory.
  *
