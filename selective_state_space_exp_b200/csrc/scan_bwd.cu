@@ -12,13 +12,15 @@
 // G_c the state entering chunk c (its first token's left endpoint included).
 //
 // Steps (one launch each):
-//  1. the forward's chunk-start states G_c and chunk totals (the CUDA-core
-//     forward pass run without its output step);
-//  2. D_c = sum_t exp(Lam_t) Ct_t dy_t^T, the adjoint y sends to G_c;
-//  3. reverse state passing: dG_c = D_c + exp(Lam_end) Rot(-Phi_end) dG_c+1,
-//     from dG_nc = d_final; each chunk keeps dG_c+1, the adjoint of its
-//     outgoing state; dG_0 gives dh0 and the previous token's gradients;
-//  4. per chunk: dCt = (M o dY X^T) Bt + diag(exp Lam) dY G_c^T,
+//  1. per chunk, the forward's chunk state S_c = sum_s w_s Bt_s x_s^T and
+//     D_c = sum_t exp(Lam_t) Ct_t dy_t^T, the adjoint y sends to G_c, with
+//     the chunk totals;
+//  2. both state passes: forward, G_c+1 = Rot(Phi_end) (exp(Lam_end) G_c + S_c)
+//     from h0 and the previous token; reverse, dG_c = D_c + exp(Lam_end)
+//     Rot(-Phi_end) dG_c+1 from dG_nc = d_final, each chunk keeping dG_c+1,
+//     the adjoint of its outgoing state; dG_0 gives dh0 and the previous
+//     token's gradients;
+//  3. per chunk: dCt = (M o dY X^T) Bt + diag(exp Lam) dY G_c^T,
 //     dBt = (M o dY X^T)^T Ct + diag(w) X dGhat^T,
 //     dX = (M o Ct Bt^T)^T dY + diag(w) Bt dGhat  (dGhat = Rot(-Phi_end) dG_c+1),
 //     the gradients of Lam (mask decay, exp(Lam_t) term, w_s), of Phi (the
@@ -38,7 +40,6 @@ using simt::chunk_prep;
 using simt::Geo;
 
 constexpr int kThreads = 256;
-constexpr int kTileRows = 64;  // (token, rank) rows staged per pass of step 2
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
@@ -59,113 +60,208 @@ ScanArgs fwd_args(const ScanArgs& a, int64_t Qb) {
   return f;
 }
 
-// ---- step 2: D_c -------------------------------------------------------------
-// Thread tiles of 4 x 4 (n, p) outputs, TPT tiles per thread (as the forward's
-// chunk-state kernel).
+// ---- step 1: per-chunk sums (S_c and D_c) ---------------------------------------
+// One pass over a chunk's rows gives both N x P products it contributes:
+//   S_c = sum_s w_s Bt_s x_s^T          (the forward's chunk state, recomputed)
+//   D_c = sum_t exp(Lam_t) Ct_t dy_t^T  (the adjoint y sends to the chunk's start state)
+// and the chunk totals (Lam_end, Phi_end).  Rows are staged kSumRows at a time;
+// each (token, pair) angle's sincos serves B and C of all R ranks.  Thread
+// tiles of 4 x 4 (n, p) outputs, TPT tiles of each product per thread.
+constexpr int kSumRows = 32;
+
 template <int R, int TPT>
-__global__ void __launch_bounds__(kThreads) bwd_dstate_kernel(const ScanArgs a, const BwdArgs g,
-                                                              const BwdWs w) {
+__global__ void __launch_bounds__(512) bwd_sums_kernel(const ScanArgs a, const BwdArgs g,
+                                                       const BwdWs w) {
   const Geo q = chunk_geo(a, blockIdx.x);
   const int N = (int)a.N, P = (int)a.P, K = N / 2, Q = (int)a.Q;
+  const int tid = threadIdx.x, nth = blockDim.x;
   extern __shared__ __align__(16) float sm[];
   float* lcum = sm;
   float* gam = lcum + Q;
   float* del = gam + Q;
   float* dts = del + Q;
-  float* phi = dts + Q;
-  float* Cs = phi + Q * K;          // [kTileRows][N] exp(Lam_t) Rot(-Phi_t) C_t
-  float* Ys = Cs + kTileRows * N;   // [kTileRows][P] dy
+  float* wts = dts + Q;
+  float* phi = wts + Q;
+  float* Bs = phi + Q * K;           // [kSumRows][N]  w_s Rot(-Phi_s) B_s
+  float* Cs = Bs + kSumRows * N;     // [kSumRows][N]  exp(Lam_t) Rot(-Phi_t) C_t
+  float* Xs = Cs + kSumRows * N;     // [kSumRows][P]  x
+  float* Ys = Xs + kSumRows * P;     // [kSumRows][P]  dy
+
   chunk_prep(a, q, lcum, gam, del, dts, phi);
+  for (int i = tid; i < q.nt; i += nth) wts[i] = expf(lcum[q.nt - 1] - lcum[i]) * del[i];
+  __syncthreads();
 
   const int PG = P / 4, ntiles = (N / 4) * PG;
-  float acc[TPT][4][4];
+  float accS[TPT][4][4], accD[TPT][4][4];
 #pragma unroll
   for (int m = 0; m < TPT; ++m)
 #pragma unroll
     for (int u = 0; u < 4; ++u)
 #pragma unroll
-      for (int v = 0; v < 4; ++v) acc[m][u][v] = 0.f;
-  const int TS = kTileRows / R;
+      for (int v = 0; v < 4; ++v) accS[m][u][v] = accD[m][u][v] = 0.f;
+
+  const int TS = kSumRows / R;  // tokens per staged round
   for (int s0 = 0; s0 < q.nt; s0 += TS) {
-    for (int e = threadIdx.x; e < kTileRows * K; e += blockDim.x) {
-      const int ri = e / K, k = e % K, s = s0 + ri / R, r = ri % R;
-      float v0 = 0.f, v1 = 0.f;
+    for (int e = tid; e < TS * K; e += nth) {
+      const int sl = e / K, k = e % K, s = s0 + sl;
+      float sn = 0.f, cs = 0.f, ws = 0.f, el = 0.f;
       if (s < q.nt) {
-        const int64_t base = ((q.base + q.t0 + s) * a.ngroups + q.g) * R * N + (int64_t)r * N;
-        const float c0 = io_load(a.C, base + 2 * k, a.bf16), c1 = io_load(a.C, base + 2 * k + 1, a.bf16);
-        float sn, cs;
         sincosf(phi[s * K + k], &sn, &cs);
-        const float el = expf(lcum[s]);
-        v0 = el * (cs * c0 + sn * c1);
-        v1 = el * (-sn * c0 + cs * c1);
+        ws = wts[s];
+        el = expf(lcum[s]);
       }
-      Cs[ri * N + 2 * k] = v0;
-      Cs[ri * N + 2 * k + 1] = v1;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int ri = sl * R + r;
+        float b0 = 0.f, b1 = 0.f, c0 = 0.f, c1 = 0.f;
+        if (s < q.nt) {
+          const int64_t base = ((q.base + q.t0 + s) * a.ngroups + q.g) * R * N + (int64_t)r * N;
+          const float br0 = io_load(a.B, base + 2 * k, a.bf16), br1 = io_load(a.B, base + 2 * k + 1, a.bf16);
+          const float cr0 = io_load(a.C, base + 2 * k, a.bf16), cr1 = io_load(a.C, base + 2 * k + 1, a.bf16);
+          b0 = ws * (cs * br0 + sn * br1); b1 = ws * (-sn * br0 + cs * br1);
+          c0 = el * (cs * cr0 + sn * cr1); c1 = el * (-sn * cr0 + cs * cr1);
+        }
+        Bs[ri * N + 2 * k] = b0; Bs[ri * N + 2 * k + 1] = b1;
+        Cs[ri * N + 2 * k] = c0; Cs[ri * N + 2 * k + 1] = c1;
+      }
     }
-    for (int e = threadIdx.x; e < kTileRows * P; e += blockDim.x) {
-      const int ri = e / P, pp = e % P, s = s0 + ri / R, r = ri % R;
-      Ys[ri * P + pp] = (s < q.nt) ? io_load(g.dy, ((q.base + q.t0 + s) * a.nheads + q.h) * R * P +
-                                                        (int64_t)r * P + pp, a.bf16)
-                                   : 0.f;
+    for (int e = tid; e < kSumRows * P; e += nth) {
+      const int ri = e / P, p = e % P, s = s0 + ri / R, r = ri % R;
+      float xv = 0.f, yv = 0.f;
+      if (s < q.nt) {
+        const int64_t o = ((q.base + q.t0 + s) * a.nheads + q.h) * R * P + (int64_t)r * P + p;
+        xv = io_load(a.x, o, a.bf16);
+        yv = io_load(g.dy, o, a.bf16);
+      }
+      Xs[ri * P + p] = xv;
+      Ys[ri * P + p] = yv;
     }
     __syncthreads();
-    const int rows = min(kTileRows, (q.nt - s0) * R);
+    const int rows = min(kSumRows, (q.nt - s0) * R);
     for (int ri = 0; ri < rows; ++ri) {
 #pragma unroll
       for (int m = 0; m < TPT; ++m) {
-        const int ti = threadIdx.x + kThreads * m;
+        const int ti = tid + nth * m;
         if (ti < ntiles) {
-          const float4 cv = ld4(Cs + ri * N + 4 * (ti / PG));
-          const float4 yv = ld4(Ys + ri * P + 4 * (ti % PG));
-          const float c4[4] = {cv.x, cv.y, cv.z, cv.w}, y4[4] = {yv.x, yv.y, yv.z, yv.w};
+          const int n4 = 4 * (ti / PG), p4 = 4 * (ti % PG);
+          const float4 bv = ld4(Bs + ri * N + n4), cv = ld4(Cs + ri * N + n4);
+          const float4 xv = ld4(Xs + ri * P + p4), yv = ld4(Ys + ri * P + p4);
+          const float b4[4] = {bv.x, bv.y, bv.z, bv.w}, c4[4] = {cv.x, cv.y, cv.z, cv.w};
+          const float x4[4] = {xv.x, xv.y, xv.z, xv.w}, y4[4] = {yv.x, yv.y, yv.z, yv.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u)
 #pragma unroll
-            for (int v = 0; v < 4; ++v) acc[m][u][v] = fmaf(c4[u], y4[v], acc[m][u][v]);
+            for (int v = 0; v < 4; ++v) {
+              accS[m][u][v] = fmaf(b4[u], x4[v], accS[m][u][v]);
+              accD[m][u][v] = fmaf(c4[u], y4[v], accD[m][u][v]);
+            }
         }
       }
     }
     __syncthreads();
   }
-  float* D = w.D + ((q.b * a.nheads + q.h) * a.nchunks + q.c) * (int64_t)N * P;
+  const int64_t cidx = (q.b * a.nheads + q.h) * a.nchunks + q.c;
+  float* S = w.G + cidx * (int64_t)N * P;  // turned into G_c by the state pass
+  float* D = w.D + cidx * (int64_t)N * P;
 #pragma unroll
   for (int m = 0; m < TPT; ++m) {
-    const int ti = threadIdx.x + kThreads * m;
+    const int ti = tid + nth * m;
     if (ti < ntiles) {
       const int n0 = 4 * (ti / PG), p0 = 4 * (ti % PG);
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < 4; ++u) {
+        *reinterpret_cast<float4*>(S + (n0 + u) * P + p0) =
+            make_float4(accS[m][u][0], accS[m][u][1], accS[m][u][2], accS[m][u][3]);
         *reinterpret_cast<float4*>(D + (n0 + u) * P + p0) =
-            make_float4(acc[m][u][0], acc[m][u][1], acc[m][u][2], acc[m][u][3]);
+            make_float4(accD[m][u][0], accD[m][u][1], accD[m][u][2], accD[m][u][3]);
+      }
     }
   }
+  // an empty chunk (past a short packed sequence) passes both states unchanged
+  float* su = w.sums + cidx * (1 + K);
+  if (tid == 0) su[0] = q.nt > 0 ? lcum[q.nt - 1] : 0.f;
+  for (int k = tid; k < K; k += nth) su[1 + k] = q.nt > 0 ? phi[(q.nt - 1) * K + k] : 0.f;
 }
 
-// ---- step 3: reverse state passing ------------------------------------------
-__global__ void __launch_bounds__(kThreads) bwd_state_pass_kernel(const ScanArgs a, const BwdArgs g,
-                                                                  const BwdWs w) {
+// ---- step 2: both state passes ---------------------------------------------------
+// Thread (k, p) of chain (b, h) holds the pair (2k, 2k+1) of column p.
+// Forward: G_0 = h0 + eps_0 B_prev x_prev^T, G_c+1 = Rot(Phi_c) (exp(Lam_c) G_c + S_c),
+// each G_c written over S_c, the last one is the final state.  Reverse: from
+// dG_nc = d_final, dG_c = D_c + exp(Lam_c) Rot(-Phi_c) dG_c+1, each chunk keeping
+// dG_c+1 (its outgoing state's adjoint) over D_c; dG_0 gives dh0 and the
+// previous token's gradients.  Chunks go in batches of kPipe whose loads are
+// all issued before the batch's dependent updates.
+__global__ void __launch_bounds__(kThreads) bwd_pass_kernel(const ScanArgs a, const BwdArgs g,
+                                                            const BwdWs w) {
   const int N = (int)a.N, P = (int)a.P, K = N / 2, R = (int)a.R;
   const int64_t b = blockIdx.z, h = blockIdx.y, H = a.nheads;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= K * P) return;  // K * P is a multiple of 32: whole warps leave
   const int k = idx / P, p = idx % P;
   const int64_t so = (b * H + h) * (int64_t)N * P;
-  float d0 = g.d_final ? g.d_final[so + (2 * k) * P + p] : 0.f;
-  float d1 = g.d_final ? g.d_final[so + (2 * k + 1) * P + p] : 0.f;
-  // chunks in batches of kPipe, all of a batch's loads issued before its
-  // dependent updates (the chain waits on arithmetic, not on each load)
+  const int64_t grp = h / (H / a.ngroups);
+  const Chain chn = chain_of(a, b);
+  const int64_t i0 = (2 * k) * P + p, i1 = (2 * k + 1) * P + p;
   constexpr int kPipe = 8;
+  const int64_t chain0 = (b * H + h) * a.nchunks;
+
+  // forward
+  float g0 = a.h0 ? a.h0[so + i0] : 0.f, g1 = a.h0 ? a.h0[so + i1] : 0.f;
+  float eps0 = 0.f, lam0 = 0.f, dt0 = 0.f;
+  int64_t t0 = 0;
+  if (a.B_prev && chn.len > 0) {  // the left endpoint term waits for a token
+    t0 = chn.base * H + h;
+    lam0 = a.lam[t0];
+    dt0 = a.dt[t0];
+    eps0 = (1.f - lam0) * dt0;
+    for (int r = 0; r < R; ++r) {
+      const int64_t bb = ((b * a.ngroups + grp) * R + r) * N;
+      const float xv = io_load(a.x_prev, ((b * H + h) * R + r) * P + p, a.bf16);
+      g0 = fmaf(eps0 * io_load(a.B_prev, bb + 2 * k, a.bf16), xv, g0);
+      g1 = fmaf(eps0 * io_load(a.B_prev, bb + 2 * k + 1, a.bf16), xv, g1);
+    }
+  }
+  for (int64_t c0 = 0; c0 < a.nchunks; c0 += kPipe) {
+    float s0[kPipe], s1[kPipe], dec[kPipe], sn[kPipe], cs[kPipe];
+#pragma unroll
+    for (int j = 0; j < kPipe; ++j) {
+      const int64_t c = c0 + j;
+      if (c >= a.nchunks) break;
+      const float* S = w.G + (chain0 + c) * (int64_t)N * P;
+      const float* su = w.sums + (chain0 + c) * (1 + K);
+      s0[j] = S[i0];
+      s1[j] = S[i1];
+      dec[j] = expf(su[0]);
+      sincosf(su[1 + k], &sn[j], &cs[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < kPipe; ++j) {
+      const int64_t c = c0 + j;
+      if (c >= a.nchunks) break;
+      float* S = w.G + (chain0 + c) * (int64_t)N * P;
+      S[i0] = g0;  // chunk-start state, true frame
+      S[i1] = g1;
+      const float v0 = fmaf(dec[j], g0, s0[j]), v1 = fmaf(dec[j], g1, s1[j]);
+      g0 = cs[j] * v0 - sn[j] * v1;
+      g1 = sn[j] * v0 + cs[j] * v1;
+    }
+  }
+  w.fin[so + i0] = g0;
+  w.fin[so + i1] = g1;
+
+  // reverse
+  float d0 = g.d_final ? g.d_final[so + i0] : 0.f;
+  float d1 = g.d_final ? g.d_final[so + i1] : 0.f;
   for (int64_t c0 = a.nchunks - 1; c0 >= 0; c0 -= kPipe) {
     float e0[kPipe], e1[kPipe], dec[kPipe], sn[kPipe], cs[kPipe];
 #pragma unroll
     for (int j = 0; j < kPipe; ++j) {
       const int64_t c = c0 - j;
       if (c < 0) break;
-      const int64_t cidx = (b * H + h) * a.nchunks + c;
-      const float* Dc = w.D + cidx * (int64_t)N * P;
-      const float* su = w.sums + cidx * (1 + K);
-      e0[j] = Dc[(2 * k) * P + p];
-      e1[j] = Dc[(2 * k + 1) * P + p];
+      const float* Dc = w.D + (chain0 + c) * (int64_t)N * P;
+      const float* su = w.sums + (chain0 + c) * (1 + K);
+      e0[j] = Dc[i0];
+      e1[j] = Dc[i1];
       dec[j] = expf(su[0]);
       sincosf(su[1 + k], &sn[j], &cs[j]);
     }
@@ -173,9 +269,9 @@ __global__ void __launch_bounds__(kThreads) bwd_state_pass_kernel(const ScanArgs
     for (int j = 0; j < kPipe; ++j) {
       const int64_t c = c0 - j;
       if (c < 0) break;
-      float* Dc = w.D + ((b * H + h) * a.nchunks + c) * (int64_t)N * P;
-      Dc[(2 * k) * P + p] = d0;  // adjoint of chunk c's outgoing state
-      Dc[(2 * k + 1) * P + p] = d1;
+      float* Dc = w.D + (chain0 + c) * (int64_t)N * P;
+      Dc[i0] = d0;  // adjoint of chunk c's outgoing state
+      Dc[i1] = d1;
       const float n0 = fmaf(dec[j], cs[j] * d0 + sn[j] * d1, e0[j]);  // D_c + exp(Lam) Rot(-Phi) dG
       const float n1 = fmaf(dec[j], -sn[j] * d0 + cs[j] * d1, e1[j]);
       d0 = n0;
@@ -183,14 +279,10 @@ __global__ void __launch_bounds__(kThreads) bwd_state_pass_kernel(const ScanArgs
     }
   }
   if (g.dh0) {
-    g.dh0[so + (2 * k) * P + p] = d0;
-    g.dh0[so + (2 * k + 1) * P + p] = d1;
+    g.dh0[so + i0] = d0;
+    g.dh0[so + i1] = d1;
   }
-  const Chain chn = chain_of(a, b);
   if (a.B_prev && chn.len > 0) {  // G_0 = h0 + eps_0 B_prev x_prev^T
-    const int64_t grp = h / (H / a.ngroups);
-    const int64_t t0 = chn.base * H + h;  // token 0 of this chain
-    const float lam0 = a.lam[t0], dt0 = a.dt[t0], eps0 = (1.f - lam0) * dt0;
     float part = 0.f;
     for (int r = 0; r < R; ++r) {
       const int64_t bb = ((b * a.ngroups + grp) * R + r) * N;
@@ -215,7 +307,7 @@ __global__ void __launch_bounds__(kThreads) bwd_state_pass_kernel(const ScanArgs
   }
 }
 
-// ---- step 4: per-chunk gradients ---------------------------------------------
+// ---- step 3: per-chunk gradients ---------------------------------------------
 // One CTA per chunk-head, M = Q * R <= 64 rows.  The products are register
 // tiles over shared-memory operands: the thread grid is 16 x 16, a thread
 // owns rows ty + 16 a and, per product, columns tx + 16 c (score-shaped
@@ -798,32 +890,33 @@ int64_t bwd_rows(const ScanArgs& a) {
   return 0;
 }
 
-size_t dstate_smem(const ScanArgs& f) {
-  return sizeof(float) * (4 * f.Q + f.Q * (f.N / 2) + kTileRows * (f.N + f.P));
+size_t sums_smem(const ScanArgs& f) {
+  return sizeof(float) * (5 * f.Q + f.Q * (f.N / 2) + 2 * kSumRows * (f.N + f.P));
 }
 
 template <int R>
 cudaError_t launch_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaStream_t st) {
   cudaError_t e;
   const int64_t tiles = (f.N / 4) * (f.P / 4);
-  const size_t sm1 = dstate_smem(f);
+  const size_t sm1 = sums_smem(f);
   dim3 grid((unsigned)f.nchunks, (unsigned)f.nheads, (unsigned)f.batch);
-#define M3_DSTATE(T)                                                  \
-  do {                                                                \
-    e = set_smem(bwd_dstate_kernel<R, T>, sm1);                       \
-    if (e != cudaSuccess) return e;                                   \
-    bwd_dstate_kernel<R, T><<<grid, kThreads, sm1, st>>>(f, g, w);    \
-  } while (0)
-  if (tiles <= kThreads) M3_DSTATE(1);
-  else if (tiles <= 2 * kThreads) M3_DSTATE(2);
-  else M3_DSTATE(4);
-#undef M3_DSTATE
+  // 256 threads for up to 256 output tiles per product, else 512 (two tiles each)
+  const int nth = tiles <= kThreads ? kThreads : 2 * kThreads;
+  if (tiles <= kThreads) {
+    e = set_smem(bwd_sums_kernel<R, 1>, sm1);
+    if (e != cudaSuccess) return e;
+    bwd_sums_kernel<R, 1><<<grid, nth, sm1, st>>>(f, g, w);
+  } else {
+    e = set_smem(bwd_sums_kernel<R, 2>, sm1);
+    if (e != cudaSuccess) return e;
+    bwd_sums_kernel<R, 2><<<grid, nth, sm1, st>>>(f, g, w);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
   dim3 pgrid((unsigned)(((f.N / 2) * f.P + kThreads - 1) / kThreads), (unsigned)f.nheads,
              (unsigned)f.batch);
-  bwd_state_pass_kernel<<<pgrid, kThreads, 0, st>>>(f, g, w);
+  bwd_pass_kernel<<<pgrid, kThreads, 0, st>>>(f, g, w);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -883,8 +976,6 @@ cudaError_t bwd_launch(const ScanArgs& a, const BwdArgs& g, cudaStream_t st) {
       cudaError_t e = cudaMemsetAsync(z.p, 0, sizeof(float) * z.n, st);
       if (e != cudaSuccess) return e;
     }
-  cudaError_t e = simt_scan_launch(f, st);  // chunk-start states, totals, final state
-  if (e != cudaSuccess) return e;
   switch (a.R) {
     case 1: return launch_r<1>(f, g, w, st);
     case 2: return launch_r<2>(f, g, w, st);
