@@ -224,8 +224,8 @@ def bwd_line(inp, s, world, steps, warmup, flush, peaks):
     f, b = bwd_work(s)
     return {"metric": "backward tokens/s", "value": round(world * s.batch * s.seqlen / t, 1),
             "unit": "tokens/s", "ms_per_step": round(t * 1e3, 4),
-            "path": "m3_scan_bwd: state-only forward recompute + 3 backward launches, "
-                    "CUDA cores fp32",
+            "path": "m3_scan_bwd: 3 launches (per-chunk sums, both state passes, "
+                    "per-chunk gradients), CUDA cores fp32",
             "roofline": alu_roofline(f, b, t, peaks)}
 
 
