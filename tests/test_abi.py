@@ -173,3 +173,66 @@ def test_bc_prep_rejects_bad_arguments(lib):
     assert prep_call(lib, s, B=ctypes.c_void_p(A16 + 0x200000 + 8)) == -3
     assert prep_call(lib, s, wB=ctypes.c_void_p(A16 + 0x500000 + 4)) == -3
     assert prep_call(lib, shape(rank=3)) == -2
+
+
+def varlen_call(lib, s, **over):
+    args = dict(cu=P[11], T=200, x=P[0], dt=P[1], A=P[2], lam=P[3], theta=P[4], B=P[5], C=P[6],
+                h0=None, Bp=None, xp=None, y=P[7], fs=None, ws=P[9], wsb=1 << 30, stream=None)
+    args.update(over)
+    return lib.m3_scan_fwd_varlen(ctypes.byref(s), args["cu"], ctypes.c_int64(args["T"]),
+                                  args["x"], args["dt"], args["A"], args["lam"], args["theta"],
+                                  args["B"], args["C"], args["h0"], args["Bp"], args["xp"],
+                                  args["y"], args["fs"], args["ws"], ctypes.c_size_t(args["wsb"]),
+                                  args["stream"])
+
+
+def test_varlen_rejects_bad_arguments(lib):
+    s = shape()
+    assert varlen_call(lib, s, cu=None) == -1
+    assert varlen_call(lib, s, T=-1) == -1
+    assert varlen_call(lib, s, cu=ctypes.c_void_p(A16 + 0xB00000 + 2)) == -1  # not 4-byte aligned
+    assert varlen_call(lib, s, x=None) == -1
+    assert varlen_call(lib, s, Bp=P[10]) == -1                               # B_prev alone
+    assert varlen_call(lib, s, y=ctypes.c_void_p(A16 + 0x700000 + 8)) == -3
+    need = ctypes.c_size_t()
+    s_long = shape(batch=1, nheads=1, seqlen=4096)  # one chain: cut into segments
+    assert lib.m3_scan_workspace_size(ctypes.byref(s_long), ctypes.byref(need)) == 0
+    assert need.value > 0 and varlen_call(lib, s_long, T=4096, ws=None, wsb=0) == -4
+    assert varlen_call(lib, shape(rank=3)) == -2
+
+
+def bwd_call(lib, s, varlen=False, **over):
+    args = dict(x=P[0], dt=P[1], A=P[2], lam=P[3], theta=P[4], B=P[5], C=P[6], h0=None, Bp=None,
+                xp=None, dy=P[7], dfin=None, dx=P[8], ddt=P[9], dA=P[10], dlam=P[11], dth=P[12],
+                dB=P[13], dC=P[14], dh0=None, dBp=None, dxp=None, ws=P[15], wsb=1 << 40,
+                stream=None, cu=P[11], T=200)
+    args.update(over)
+    rest = [args[k] for k in ("x", "dt", "A", "lam", "theta", "B", "C", "h0", "Bp", "xp", "dy",
+                              "dfin", "dx", "ddt", "dA", "dlam", "dth", "dB", "dC", "dh0",
+                              "dBp", "dxp", "ws")] + [ctypes.c_size_t(args["wsb"]), args["stream"]]
+    if varlen:
+        return lib.m3_scan_bwd_varlen(ctypes.byref(s), args["cu"], ctypes.c_int64(args["T"]),
+                                      *rest)
+    return lib.m3_scan_bwd(ctypes.byref(s), *rest)
+
+
+def test_bwd_workspace_and_bad_arguments(lib):
+    n = ctypes.c_size_t()
+    s = shape(batch=2, seqlen=130, io_dtype=m3.M3_F32, dstate=16, headdim=16)
+    assert lib.m3_scan_bwd_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0
+    # 32-row chunks (R = 1): 5 per sequence; chunk states and adjoints, totals, final states
+    assert n.value >= 2 * (2 * 4 * 5 * 16 * 16 * 4) + 2 * 4 * 16 * 16 * 4
+    assert lib.m3_scan_bwd_workspace_size(None, ctypes.byref(n)) == -1
+    for varlen in (False, True):
+        assert bwd_call(lib, s, varlen, dy=None) == -1
+        assert bwd_call(lib, s, varlen, dth=None) == -1
+        assert bwd_call(lib, s, varlen, dC=None) == -1
+        assert bwd_call(lib, s, varlen, Bp=P[10]) == -1                  # B_prev without x_prev
+        assert bwd_call(lib, s, varlen, dBp=P[10]) == -1                 # dB_prev without dx_prev
+        assert bwd_call(lib, s, varlen, dx=ctypes.c_void_p(A16 + 0x800000 + 4)) == -3
+        assert bwd_call(lib, s, varlen, ddt=ctypes.c_void_p(A16 + 0x900000 + 2)) == -3
+        assert bwd_call(lib, s, varlen, ws=None) == -4
+        assert bwd_call(lib, s, varlen, wsb=16) == -4
+        assert bwd_call(lib, shape(rank=3), varlen) == -2
+    assert bwd_call(lib, s, True, cu=None) == -1
+    assert bwd_call(lib, s, True, T=-5) == -1
