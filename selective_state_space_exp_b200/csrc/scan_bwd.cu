@@ -417,13 +417,15 @@ __device__ __forceinline__ void tn1(float (&acc)[TI][NGT][4], const float (&av)[
   }
 }
 
-template <int R, int M>
+// NGT_: 4-column groups per thread in the N-wide products (ceil(N / 64)),
+// PCT_: dX columns per thread (P / 16); 0 picks the widest supported shape.
+template <int R, int M, int NGT_, int PCT_>
 __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(const ScanArgs a, const BwdArgs g,
                                                              const BwdWs w) {
   constexpr int Q = M / R;
   constexpr int TI = M / 16;           // rows per thread
-  constexpr int NGT = 8 / TI;          // N-wide products: 4-column groups per thread (N <= 64 NGT)
-  constexpr int PCT = 128 / 16;        // dX columns per thread at most (P <= 128)
+  constexpr int NGT = NGT_ ? NGT_ : 8 / TI;  // N-wide products: 4-column groups per thread
+  constexpr int PCT = PCT_ ? PCT_ : 128 / 16;  // dX columns per thread
   const Geo q = chunk_geo(a, blockIdx.x);
   const int N = (int)a.N, P = (int)a.P, K = N / 2;
   const int64_t H = a.nheads;
@@ -923,15 +925,23 @@ cudaError_t launch_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaSt
   const int M = (int)(f.Q * R);
   const ChunkSmem L(M, (int)f.N, (int)f.P, (int)f.Q);
   const size_t sm3 = sizeof(float) * (size_t)L.total;
+  // N = 128, P = 64 (the layer's shape) has exact register tiles; other shapes
+  // take the widest ones, with the unused groups predicated off
+  const bool layer = f.N == 128 && f.P == 64;
+#define M3_CHUNK(MM, NG_, PC_)                                        \
+  do {                                                                \
+    e = set_smem(bwd_chunk_kernel<R, MM, NG_, PC_>, sm3);             \
+    if (e != cudaSuccess) return e;                                   \
+    bwd_chunk_kernel<R, MM, NG_, PC_><<<grid, kThreads, sm3, st>>>(f, g, w); \
+  } while (0)
   if (M == 64) {
-    e = set_smem(bwd_chunk_kernel<R, 64>, sm3);
-    if (e != cudaSuccess) return e;
-    bwd_chunk_kernel<R, 64><<<grid, kThreads, sm3, st>>>(f, g, w);
+    if (layer) M3_CHUNK(64, 2, 4);
+    else M3_CHUNK(64, 0, 0);
   } else {
-    e = set_smem(bwd_chunk_kernel<R, 32>, sm3);
-    if (e != cudaSuccess) return e;
-    bwd_chunk_kernel<R, 32><<<grid, kThreads, sm3, st>>>(f, g, w);
+    if (layer) M3_CHUNK(32, 2, 4);
+    else M3_CHUNK(32, 0, 0);
   }
+#undef M3_CHUNK
   return cudaGetLastError();
 }
 
