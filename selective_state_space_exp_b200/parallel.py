@@ -14,6 +14,17 @@ rank folds the earlier segments' summaries into its incoming state and scans
 its segment from it.  The steps run in the library's kernels (m3_scan_state,
 m3_segment_totals, m3_state_fold, m3_scan_fwd); the per-rank phases are plain
 functions so that one process can also drive every rank in turn.
+
+The backward of the split needs one more exchange.  The adjoint of segment r's
+end state is dG_end(r) = d_final for the last segment, else
+dG_end(r) = exp(Lam_{r+1}) Rot(-Phi_{r+1}) dG_end(r+1) + D_{r+1}, the transpose
+of segment r+1's state transition applied to its own end adjoint plus D_{r+1},
+the adjoint that segment r+1's outputs send to its incoming state (the dh0 of
+its backward with no final-state gradient).  So each rank computes D_r, the
+ranks all-gather them, each folds the later segments' (D, Lam, -Phi) into its
+end adjoint with the forward's fold, and runs its backward from it; the
+gradients of a segment's first-token left endpoint (its B_prev, x_prev: the
+previous segment's last token) go back to the previous rank.
 """
 from __future__ import annotations
 
@@ -70,6 +81,12 @@ class M3Ops:
         from . import m3
         return m3.m3_scan_fwd(x, dt, A, lam, theta, B, C, chunk, h0, B_prev, x_prev)
 
+    def scan_bwd(self, x, dt, A, lam, theta, B, C, chunk, h0, B_prev, x_prev, dy, d_final):
+        """Gradient dict of m3_scan_bwd (keys x, dt, A, lam, theta, B, C, h0 and,
+        with a previous token, B_prev, x_prev)."""
+        from . import m3
+        return m3.m3_scan_bwd(x, dt, A, lam, theta, B, C, dy, chunk, h0, B_prev, x_prev, d_final)
+
 
 def seq_boundary(x: torch.Tensor, B: torch.Tensor):
     """This segment's last token: (B [b][G][R][N], x [b][H][R][P]), the next
@@ -119,3 +136,68 @@ def seq_parallel_scan(x, dt, A, lam, theta, B, C, chunk=64, h0=None, B_prev=None
     T, lam_tot, phi_tot = seq_summary(ops, x, dt, A, lam, theta, B, C, chunk, Bp, xp)
     Ts, lams, phis = _all_gather(T, group), _all_gather(lam_tot, group), _all_gather(phi_tot, group)
     return seq_finish(ops, r, x, dt, A, lam, theta, B, C, chunk, h0, Ts, lams, phis, Bp, xp)
+
+
+# ---- backward of the sequence split --------------------------------------------
+
+def seq_incoming_state(ops, rank, h0, Ts, lams, phis):
+    """The state entering segment `rank`: segments 0..rank-1 folded from h0."""
+    if rank == 0:
+        return h0
+    return ops.state_fold(h0, torch.stack(Ts[:rank]), torch.stack(lams[:rank]),
+                          torch.stack(phis[:rank]))
+
+
+def seq_end_adjoint(ops, rank, world, d_final, Ds, lams, phis):
+    """The adjoint of segment `rank`'s end state: d_final (None: zero) carried
+    back through segments world-1 .. rank+1, each step
+    d <- exp(Lam_s) Rot(-Phi_s) d + D_s (the forward's fold with the angles
+    negated).  Returns None for a zero adjoint."""
+    later = list(range(world - 1, rank, -1))
+    if not later:
+        return d_final
+    return ops.state_fold(d_final, torch.stack([Ds[s] for s in later]),
+                          torch.stack([lams[s] for s in later]),
+                          torch.stack([-phis[s] for s in later]))
+
+
+def seq_parallel_scan_bwd(x, dt, A, lam, theta, B, C, dy, chunk=64, h0=None, B_prev=None,
+                          x_prev=None, d_final=None, *, group=None, ops=None):
+    """Gradients of the split scan (the layout of seq_parallel_scan): this
+    rank's dy [b][Ls][H][R][P]; d_final, h0, B_prev, x_prev the same on every
+    rank (only the last rank uses d_final, only rank 0 h0 and the previous
+    token).  The forward's exchange is repeated to get each segment's incoming
+    state.  Returns this rank's gradient dict: x, dt, A, lam, theta, B, C of
+    its segment (its last token's B and x including the next segment's
+    left-endpoint terms), "h_in" (the adjoint of its incoming state: the
+    sequences' dh0 on rank 0) and, on rank 0 with a previous token, B_prev and
+    x_prev."""
+    ops = ops or M3Ops()
+    r, world = dist.get_rank(group), dist.get_world_size(group)
+    B_last, x_last = seq_boundary(x, B)
+    gB, gx = _all_gather(B_last, group), _all_gather(x_last, group)
+    Bp, xp = (B_prev, x_prev) if r == 0 else (gB[r - 1], gx[r - 1])
+    T, lam_tot, phi_tot = seq_summary(ops, x, dt, A, lam, theta, B, C, chunk, Bp, xp)
+    Ts, lams, phis = _all_gather(T, group), _all_gather(lam_tot, group), _all_gather(phi_tot, group)
+    h_in = seq_incoming_state(ops, r, h0, Ts, lams, phis)
+    if h_in is None:
+        h_in = torch.zeros_like(T)
+    D = ops.scan_bwd(x, dt, A, lam, theta, B, C, chunk, h_in, Bp, xp, dy, None)["h0"]
+    Ds = _all_gather(D, group)
+    d_end = seq_end_adjoint(ops, r, world, d_final, Ds, lams, phis)
+    g = ops.scan_bwd(x, dt, A, lam, theta, B, C, chunk, h_in, Bp, xp, dy, d_end)
+    # the next segment's first token used this segment's last B and x
+    zB = torch.zeros_like(B_last, dtype=g["B"].dtype)
+    zx = torch.zeros_like(x_last, dtype=g["x"].dtype)
+    gBp = _all_gather(g["B_prev"] if Bp is not None else zB, group)
+    gxp = _all_gather(g["x_prev"] if Bp is not None else zx, group)
+    out = {k: g[k] for k in ("x", "dt", "A", "lam", "theta", "B", "C")}
+    if r + 1 < world:
+        out["B"] = out["B"].clone()
+        out["x"] = out["x"].clone()
+        out["B"][:, -1] += gBp[r + 1]
+        out["x"][:, -1] += gxp[r + 1]
+    out["h_in"] = g["h0"]
+    if r == 0 and B_prev is not None:
+        out["B_prev"], out["x_prev"] = g["B_prev"], g["x_prev"]
+    return out

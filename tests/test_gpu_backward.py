@@ -149,3 +149,47 @@ def test_bwd_full_size_sampled_chains(R):
                 "h0": rel_err(got["h0"][b, h], ref["h0"][0, 0])}
         bad = {k: v for k, v in errs.items() if not v <= BAR}
         assert not bad, (c, errs)
+
+
+@pytest.mark.parametrize("world,io", [(2, "f32"), (3, "bf16")])
+def test_bwd_sequence_split_emulated_on_one_gpu(world, io):
+    """The backward of the sequence split driven rank by rank with the
+    library's kernels on one device: every input's gradient, in token order,
+    against the gradient oracle on the whole sequence.  With bf16 io the
+    segments' incoming states come from the tensor-core state-only pass
+    (bf16 operands), so that case is held to the bf16 io bar."""
+    from selective_state_space_exp_b200.parallel import (M3Ops, seq_boundary, seq_end_adjoint,
+                                                         seq_incoming_state, seq_summary)
+    N, P = (16, 16) if io == "f32" else (128, 64)
+    inp = case(batch=1, L=60 * world, H=2, N=N, P=P, R=2, io=io, seed=1200 + world)
+    g = to_dev(inp)
+    L = inp["x"].shape[1]
+    keys = ("x", "dt", "A", "lam", "theta", "B", "C", "dy")
+    segs = [{k: g[k][:, r * L // world:(r + 1) * L // world].contiguous() for k in keys}
+            for r in range(world)]
+    ops = M3Ops()
+    lasts = [seq_boundary(s["x"], s["B"]) for s in segs]
+    prevs = [(g["B_prev"], g["x_prev"])] + [lasts[r - 1] for r in range(1, world)]
+    sums = [seq_summary(ops, s["x"], s["dt"], s["A"], s["lam"], s["theta"], s["B"], s["C"], 64,
+                        *prevs[r]) for r, s in enumerate(segs)]
+    Ts, lams, phis = [t[0] for t in sums], [t[1] for t in sums], [t[2] for t in sums]
+    h_ins = [seq_incoming_state(ops, r, g["h0"], Ts, lams, phis) for r in range(world)]
+    args = lambda r: (segs[r]["x"], segs[r]["dt"], segs[r]["A"], segs[r]["lam"],
+                      segs[r]["theta"], segs[r]["B"], segs[r]["C"], 64, h_ins[r], *prevs[r])
+    Ds = [ops.scan_bwd(*args(r), segs[r]["dy"], None)["h0"] for r in range(world)]
+    parts = [ops.scan_bwd(*args(r), segs[r]["dy"],
+                          seq_end_adjoint(ops, r, world, g["d_final"], Ds, lams, phis))
+             for r in range(world)]
+    for r in range(world - 1):
+        parts[r]["B"][:, -1] += parts[r + 1]["B_prev"]
+        parts[r]["x"][:, -1] += parts[r + 1]["x_prev"]
+    assert m3.m3_stream_status() == 0
+    _, _, ref = m3_grad.scan_grads(*[inp.get(k) for k in m3_grad.NAMES], dy=inp["dy"],
+                                   d_final=inp["d_final"])
+    errs = {k: rel_err(torch.cat([p[k] for p in parts], dim=1).cpu().numpy(), ref[k])
+            for k in ("x", "dt", "A", "lam", "theta", "B", "C")}
+    errs["h0"] = rel_err(parts[0]["h0"].cpu().numpy(), ref["h0"])
+    errs["B_prev"] = rel_err(parts[0]["B_prev"].cpu().numpy(), ref["B_prev"])
+    bar = BAR if io == "f32" else 2e-2
+    bad = {k: v for k, v in errs.items() if not v <= bar}
+    assert not bad, errs

@@ -69,6 +69,7 @@ def test_single_process_reductions_are_identity():
 import numpy as np  # noqa: E402
 
 import oracle  # noqa: E402
+from oracle import m3_grad  # noqa: E402
 from selective_state_space_exp_b200.parallel import (seq_boundary, seq_finish,  # noqa: E402
                                                      seq_parallel_scan, seq_summary)
 
@@ -103,6 +104,11 @@ class OracleOps:
     def scan_fwd(self, x, dt, A, lam, theta, B, C, chunk, h0, B_prev, x_prev):
         y, hL = oracle.scan(x, dt, A, lam, theta, B, C, h0, B_prev, x_prev, f64=True)
         return torch.from_numpy(y), torch.from_numpy(hL)
+
+    def scan_bwd(self, x, dt, A, lam, theta, B, C, chunk, h0, B_prev, x_prev, dy, d_final):
+        _, _, g = m3_grad.scan_grads(x, dt, A, lam, theta, B, C, h0, B_prev, x_prev, dy=dy,
+                                     d_final=d_final)
+        return {k: torch.from_numpy(v) for k, v in g.items()}
 
 
 def _seq_problem(L=24, theta_per_head=False):
@@ -172,3 +178,89 @@ def test_sequence_split_phases_in_one_process():
                            d["h0"], d["B_prev"], d["x_prev"], f64=True)
     y = np.concatenate([t.numpy() for t in ys], axis=1)
     assert np.max(np.abs(y - y_ref)) <= 1e-10 * np.max(np.abs(y_ref))
+
+
+# ---- backward of the sequence split ----------------------------------------------
+
+def _seq_bwd_problem(L=24, theta_per_head=False):
+    d = _seq_problem(L=L, theta_per_head=theta_per_head)
+    rng = np.random.default_rng(78)
+    d["dy"] = torch.from_numpy(rng.standard_normal(tuple(d["x"].shape)))
+    d["d_final"] = torch.from_numpy(rng.standard_normal(tuple(d["h0"].shape)))
+    return d
+
+
+def _bwd_reference(d):
+    _, _, g = m3_grad.scan_grads(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"], d["C"],
+                                 d["h0"], d["B_prev"], d["x_prev"], dy=d["dy"],
+                                 d_final=d["d_final"])
+    return g
+
+
+def _check_split_grads(parts, ref, world):
+    for k in ("x", "dt", "A", "lam", "theta", "B", "C"):
+        got = np.concatenate([parts[r][k].numpy() for r in range(world)], axis=1)
+        assert np.max(np.abs(got - ref[k])) <= 1e-10 * np.max(np.abs(ref[k])), k
+    for k_got, k_ref in (("h_in", "h0"), ("B_prev", "B_prev"), ("x_prev", "x_prev")):
+        got = parts[0][k_got].numpy()
+        assert np.max(np.abs(got - ref[k_ref])) <= 1e-10 * np.max(np.abs(ref[k_ref])), k_got
+
+
+def _seq_bwd_worker(rank, world, port, out, theta_per_head):
+    from selective_state_space_exp_b200.parallel import seq_parallel_scan_bwd
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        d = _seq_bwd_problem(theta_per_head=theta_per_head)
+        s = _segment(d, rank, world)
+        L = d["x"].shape[1]
+        dy = d["dy"][:, rank * L // world:(rank + 1) * L // world].contiguous()
+        g = seq_parallel_scan_bwd(s["x"], s["dt"], s["A"], s["lam"], s["theta"], s["B"], s["C"],
+                                  dy, 64, s["h0"], s["B_prev"], s["x_prev"], d["d_final"],
+                                  ops=OracleOps())
+        out[rank] = g
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,theta_per_head", [(2, False), (3, True)])
+def test_gloo_sequence_split_backward_matches_one_backward(world, theta_per_head):
+    """Gradients of the split scan, ranks as gloo processes with the oracle
+    standing in for the kernels: every input's gradient, in token order, equals
+    the gradient oracle's on the whole sequence (the last token of each
+    segment carries the next segment's left-endpoint terms)."""
+    port = _free_port()
+    out = mp.Manager().dict()
+    mp.spawn(_seq_bwd_worker, args=(world, port, out, theta_per_head), nprocs=world, join=True)
+    _check_split_grads(out, _bwd_reference(_seq_bwd_problem(theta_per_head=theta_per_head)), world)
+
+
+def test_sequence_split_backward_phases_in_one_process():
+    """The backward's phases rank by rank in one process (4 ranks)."""
+    from selective_state_space_exp_b200.parallel import seq_end_adjoint, seq_incoming_state
+    world = 4
+    d = _seq_bwd_problem(L=20)
+    L = d["x"].shape[1]
+    segs = [_segment(d, r, world) for r in range(world)]
+    dys = [d["dy"][:, r * L // world:(r + 1) * L // world] for r in range(world)]
+    ops = OracleOps()
+    lasts = [seq_boundary(s["x"], s["B"]) for s in segs]
+    prevs = [(d["B_prev"], d["x_prev"])] + [lasts[r - 1] for r in range(1, world)]
+    sums = [seq_summary(ops, s["x"], s["dt"], s["A"], s["lam"], s["theta"], s["B"], s["C"], 64,
+                        *prevs[r]) for r, s in enumerate(segs)]
+    Ts, lams, phis = [t[0] for t in sums], [t[1] for t in sums], [t[2] for t in sums]
+    h_ins = [seq_incoming_state(ops, r, d["h0"], Ts, lams, phis) for r in range(world)]
+    args = lambda r: (segs[r]["x"], segs[r]["dt"], segs[r]["A"], segs[r]["lam"],
+                      segs[r]["theta"], segs[r]["B"], segs[r]["C"], 64, h_ins[r], *prevs[r])
+    Ds = [ops.scan_bwd(*args(r), dys[r], None)["h0"] for r in range(world)]
+    parts = []
+    for r in range(world):
+        d_end = seq_end_adjoint(ops, r, world, d["d_final"], Ds, lams, phis)
+        g = ops.scan_bwd(*args(r), dys[r], d_end)
+        parts.append({k: v.clone() for k, v in g.items()})
+    for r in range(world - 1):  # the next segment's left-endpoint gradients
+        parts[r]["B"][:, -1] += parts[r + 1]["B_prev"]
+        parts[r]["x"][:, -1] += parts[r + 1]["x_prev"]
+    parts[0]["h_in"] = parts[0]["h0"]
+    _check_split_grads(parts, _bwd_reference(d), world)
