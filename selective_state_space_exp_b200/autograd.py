@@ -1,0 +1,50 @@
+"""torch.autograd binding of the scan: the forward is m3_scan_fwd, the backward
+m3_scan_bwd (both through the C ABI).  Argument marshalling only; every step
+runs in the library's kernels.
+
+    y, final_state = m3_scan(x, dt, A, lam, theta, B, C, chunk=64, h0=None,
+                             B_prev=None, x_prev=None)
+
+Layouts as m3_scan_fwd.  Gradients flow to every tensor argument that
+requires them; they are computed in fp32 and returned in each input's dtype
+(bf16 inputs get bf16 gradients).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import m3
+
+_NAMES = ("x", "dt", "A", "lam", "theta", "B", "C", "h0", "B_prev", "x_prev")
+
+
+class M3Scan(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, chunk, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev):
+        y, fs = m3.m3_scan_fwd(x, dt, A, lam, theta, B, C, chunk, h0, B_prev, x_prev)
+        ctx.chunk = chunk
+        ctx.save_for_backward(x, dt, A, lam, theta, B, C, h0, B_prev, x_prev)
+        return y, fs
+
+    @staticmethod
+    def backward(ctx, dy, d_final):
+        x, dt, A, lam, theta, B, C, h0, B_prev, x_prev = ctx.saved_tensors
+        if dy is None:
+            dy = torch.zeros_like(x)
+        g = m3.m3_scan_bwd(x, dt, A, lam, theta, B, C, dy.contiguous().to(x.dtype), ctx.chunk,
+                           h0, B_prev, x_prev,
+                           None if d_final is None else d_final.contiguous().float())
+        inputs = dict(zip(_NAMES, (x, dt, A, lam, theta, B, C, h0, B_prev, x_prev)))
+        out = [None]  # chunk
+        for i, name in enumerate(_NAMES):
+            t = inputs[name]
+            if t is None or not ctx.needs_input_grad[i + 1] or name not in g:
+                out.append(None)
+            else:
+                out.append(g[name].to(t.dtype))
+        return tuple(out)
+
+
+def m3_scan(x, dt, A, lam, theta, B, C, chunk: int = 64, h0=None, B_prev=None, x_prev=None):
+    """Differentiable chunked scan: (y, final_state), gradients by m3_scan_bwd."""
+    return M3Scan.apply(chunk, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev)
