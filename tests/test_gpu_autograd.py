@@ -65,3 +65,27 @@ def test_autograd_only_requested_gradients():
                                                             "C")],
                                    dy=np.ones(tuple(inp["x"].shape)))
     assert rel_err(x.grad.cpu().numpy(), ref["x"]) <= 1e-4
+
+
+def test_autograd_varlen():
+    """The packed-batch binding against the gradient oracle run per sequence."""
+    from selective_state_space_exp_b200.autograd import m3_scan_varlen
+    w = I.Workload(I.Shape(1, 1, 2, 64, 128, 2, 1, 64, "bf16"), decay="slow", with_h0=True,
+                   with_prev=True)
+    lengths = I.varlen_lengths(6, 150, 64, seed=1330)
+    inp = I.make_varlen_inputs(w, lengths, seed=1331)
+    gen = torch.Generator().manual_seed(1332)
+    dy = torch.randn(inp["x"].shape, generator=gen).to(torch.bfloat16)
+    dfin = torch.randn(inp["h0"].shape, generator=gen)
+    leaves = {k: v.cuda().requires_grad_(k != "cu_seqlens") for k, v in inp.items()}
+    y, fs = m3_scan_varlen(leaves["cu_seqlens"], leaves["x"], leaves["dt"], leaves["A"],
+                           leaves["lam"], leaves["theta"], leaves["B"], leaves["C"], 64,
+                           leaves["h0"], leaves["B_prev"], leaves["x_prev"])
+    ((y.float() * dy.cuda().float()).sum() + (fs * dfin.cuda()).sum()).backward()
+    assert m3.m3_stream_status() == 0
+    ref = m3_grad.scan_grads_varlen(inp["cu_seqlens"], inp["x"], inp["dt"], inp["A"],
+                                    inp["lam"], inp["theta"], inp["B"], inp["C"], inp["h0"],
+                                    inp["B_prev"], inp["x_prev"], dy=dy, d_final=dfin)
+    errs = {k: rel_err(leaves[k].grad.float().cpu().numpy(), ref[k]) for k in ref}
+    bad = {k: v for k, v in errs.items() if not v <= 2e-2}
+    assert not bad, errs
