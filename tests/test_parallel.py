@@ -264,3 +264,41 @@ def test_sequence_split_backward_phases_in_one_process():
         parts[r]["x"][:, -1] += parts[r + 1]["x_prev"]
     parts[0]["h_in"] = parts[0]["h0"]
     _check_split_grads(parts, _bwd_reference(d), world)
+
+
+def test_sequence_split_backward_without_h0_or_previous_token():
+    """The zero paths: no initial state, no previous token, no final-state
+    gradient (4 ranks in one process, oracle stand-ins)."""
+    from selective_state_space_exp_b200.parallel import seq_end_adjoint, seq_incoming_state
+    world = 4
+    d = _seq_bwd_problem(L=16)
+    for k in ("h0", "B_prev", "x_prev", "d_final"):
+        d[k] = None
+    L = d["x"].shape[1]
+    segs = [_segment(d, r, world) for r in range(world)]
+    dys = [d["dy"][:, r * L // world:(r + 1) * L // world] for r in range(world)]
+    ops = OracleOps()
+    lasts = [seq_boundary(s["x"], s["B"]) for s in segs]
+    prevs = [(None, None)] + [lasts[r - 1] for r in range(1, world)]
+    sums = [seq_summary(ops, s["x"], s["dt"], s["A"], s["lam"], s["theta"], s["B"], s["C"], 64,
+                        *prevs[r]) for r, s in enumerate(segs)]
+    Ts, lams, phis = [t[0] for t in sums], [t[1] for t in sums], [t[2] for t in sums]
+    h_ins = [seq_incoming_state(ops, r, None, Ts, lams, phis) for r in range(world)]
+    h_ins[0] = torch.zeros_like(Ts[0])
+    args = lambda r: (segs[r]["x"], segs[r]["dt"], segs[r]["A"], segs[r]["lam"],
+                      segs[r]["theta"], segs[r]["B"], segs[r]["C"], 64, h_ins[r], *prevs[r])
+    Ds = [ops.scan_bwd(*args(r), dys[r], None)["h0"] for r in range(world)]
+    assert seq_end_adjoint(ops, world - 1, world, None, Ds, lams, phis) is None
+    parts = [{k: v.clone() for k, v in
+              ops.scan_bwd(*args(r), dys[r], seq_end_adjoint(ops, r, world, None, Ds, lams,
+                                                               phis)).items()}
+             for r in range(world)]
+    for r in range(world - 1):
+        parts[r]["B"][:, -1] += parts[r + 1]["B_prev"]
+        parts[r]["x"][:, -1] += parts[r + 1]["x_prev"]
+    _, _, ref = m3_grad.scan_grads(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"], d["C"],
+                                   np.zeros(tuple(Ts[0].shape)), dy=d["dy"])
+    for k in ("x", "dt", "A", "lam", "theta", "B", "C"):
+        got = np.concatenate([parts[r][k].numpy() for r in range(world)], axis=1)
+        assert np.max(np.abs(got - ref[k])) <= 1e-10 * np.max(np.abs(ref[k])), k
+    assert np.max(np.abs(parts[0]["h0"].numpy() - ref["h0"])) <= 1e-10 * np.max(np.abs(ref["h0"]))
