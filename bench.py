@@ -526,10 +526,11 @@ def time_e2e_prefill(inp_host, s, steps):
 
 # ---- CPU oracle baseline ----------------------------------------------------
 
-def cpu_oracle_prefill(inp_host, s, budget_s=12.0):
+def cpu_oracle_prefill(inp_host, s, budget_s=12.0, single_thread=True):
     """Time the oracle (as it stands) on whole (batch, head) chains of the same
     workload until about `budget_s` seconds of CPU work; tokens/s counts the
-    tokens those chains cover (chains / nheads * seqlen)."""
+    tokens those chains cover (chains / nheads * seqlen).  With single_thread,
+    also the same oracle on one thread on a smaller sample."""
     import oracle
     cores = len(os.sched_getaffinity(0))
     total = s.batch * s.nheads
@@ -544,6 +545,12 @@ def cpu_oracle_prefill(inp_host, s, budget_s=12.0):
         elapsed += time.perf_counter() - t0
         done += len(chains)
     tokens = done / s.nheads * s.seqlen
+    res = {"value": round(tokens / elapsed, 1), "unit": "tokens/s", "cores": cores,
+           "kind": "oracle",
+           "sample": f"{done} of {total} (batch, head) chains, all {s.seqlen} tokens each, "
+                     f"{elapsed:.1f} s on {cores} threads"}
+    if not single_thread:
+        return res
     # the same oracle on one thread, on a smaller sample of the same chains
     one = min(max(1, done // max(cores, 1)), total)
     t0 = time.perf_counter()
@@ -551,13 +558,9 @@ def cpu_oracle_prefill(inp_host, s, budget_s=12.0):
                 inp_host["theta"], inp_host["B"], inp_host["C"], chains=list(range(one)),
                 nthreads=1)
     t1 = time.perf_counter() - t0
-    return {"value": round(tokens / elapsed, 1), "unit": "tokens/s", "cores": cores,
-            "kind": "oracle",
-            "sample": f"{done} of {total} (batch, head) chains, all {s.seqlen} tokens each, "
-                      f"{elapsed:.1f} s on {cores} threads",
-            "single_thread": {"value": round(one / s.nheads * s.seqlen / t1, 1),
-                              "unit": "tokens/s", "cores": 1,
-                              "sample": f"{one} chains, {t1:.1f} s"}}
+    res["single_thread"] = {"value": round(one / s.nheads * s.seqlen / t1, 1),
+                            "unit": "tokens/s", "cores": 1, "sample": f"{one} chains, {t1:.1f} s"}
+    return res
 
 
 # ---- main -------------------------------------------------------------------
@@ -573,7 +576,7 @@ def run_reference(args, s, wname):
     vals = []
     budget = max(2.0, 120.0 / max(args.steps + args.warmup, 1))
     for i in range(args.warmup + args.steps):
-        r = cpu_oracle_prefill(inp, s, budget_s=budget)
+        r = cpu_oracle_prefill(inp, s, budget_s=budget, single_thread=False)
         if i >= args.warmup:
             vals.append(r)
     v = statistics.mean(r["value"] for r in vals)
