@@ -9,7 +9,6 @@ import numpy as np
 import pytest
 import torch
 
-import oracle
 from selective_state_space_exp_b200 import inputs as I
 from selective_state_space_exp_b200 import m3
 from parity_helpers import (TOL, chain_rows, compare_scan, gpu_scan, need_gpu, oracle_scan,

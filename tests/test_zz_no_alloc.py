@@ -12,7 +12,6 @@ import ctypes
 
 import numpy as np
 import pytest
-import torch
 
 from selective_state_space_exp_b200 import _build, m3
 from selective_state_space_exp_b200 import inputs as I
