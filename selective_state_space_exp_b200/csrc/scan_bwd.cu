@@ -902,8 +902,9 @@ cudaError_t launch_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaSt
   const int64_t tiles = (f.N / 4) * (f.P / 4);
   const size_t sm1 = sums_smem(f);
   dim3 grid((unsigned)f.nchunks, (unsigned)f.nheads, (unsigned)f.batch);
-  // 256 threads for up to 256 output tiles per product, else 512 (two tiles each)
-  const int nth = tiles <= kThreads ? kThreads : 2 * kThreads;
+  // 256 threads with one or two output tiles each (two CTAs share an SM),
+  // 512 threads with two tiles each beyond that
+  const int nth = tiles <= 2 * kThreads ? kThreads : 2 * kThreads;
   if (tiles <= kThreads) {
     e = set_smem(bwd_sums_kernel<R, 1>, sm1);
     if (e != cudaSuccess) return e;
