@@ -17,6 +17,15 @@
  *   - output y_t = C_t^T h_t (R x P per token and head), the real part of the
  *     complex state read by C (section 2.1).
  *
+ * Calls: the chunked prefill scan (m3_scan_fwd; its packed variable-length
+ * form m3_scan_fwd_varlen; m3_scan_fwd_noalloc without a workspace argument;
+ * m3_scan_state for the final state only), the single-token decode step
+ * (m3_decode_step), the backward pass (m3_scan_bwd, m3_scan_bwd_varlen), the
+ * B / C projection prep (m3_bc_prep), the pieces of a sequence split across
+ * ranks (m3_segment_totals, m3_state_fold), and sizing, planning and status
+ * (m3_*_workspace_size, m3_scan_plan, m3_check_shape, m3_stream_status,
+ * m3_status_string, m3_version).
+ *
  * Conventions for every call:
  *   - Every data pointer is a DEVICE pointer owned by the caller.  The library
  *     never allocates, frees or retains memory; it writes only the outputs
