@@ -79,3 +79,36 @@ def test_split_continuation(sh, frac):
     y2, h2 = oracle.scan(*[second[k] for k in ORDER], f64=True)
     assert rel(np.concatenate([y1, y2], axis=1), y) < 1e-10
     assert rel(h2, h) < 1e-10
+
+
+@settings(max_examples=12, deadline=None)
+@given(st.integers(0, 10 ** 6), st.integers(1, 6), st.sampled_from([(1, 1), (2, 1), (2, 2)]),
+       st.integers(1, 2), st.sampled_from([2, 4]), st.integers(1, 3), st.booleans())
+def test_gradient_oracle_matches_finite_differences(seed, L, HG, R, N, P, per_head):
+    """Random shapes: three random coordinates of every input, central
+    differences of the C oracle against the autograd gradient oracle."""
+    from oracle import m3_grad
+    H, G = HG
+    d = problem(seed, L, H, G, R, N, P, per_head)
+    rng = np.random.default_rng(seed + 2)
+    dy = rng.standard_normal(d["x"].shape)
+    dfin = rng.standard_normal(d["h0"].shape)
+    _, _, grads = m3_grad.scan_grads(*[d[k] for k in ORDER], dy=dy, d_final=dfin)
+
+    def loss():
+        yo, ho = oracle.scan(*[d[k] for k in ORDER], f64=True)
+        return float(np.sum(yo * dy) + np.sum(ho * dfin))
+
+    hstep = 1e-5
+    for name in ORDER:
+        flat = d[name].reshape(-1)
+        g = grads[name].reshape(-1)
+        scale = max(np.max(np.abs(g)), 1e-12)
+        for i in rng.choice(flat.size, size=min(3, flat.size), replace=False):
+            keep = flat[i]
+            flat[i] = keep + hstep
+            lp = loss()
+            flat[i] = keep - hstep
+            lm = loss()
+            flat[i] = keep
+            assert abs((lp - lm) / (2 * hstep) - g[i]) <= 1e-6 * scale, (name, int(i))
