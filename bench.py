@@ -1,6 +1,10 @@
-"""Benchmark of the Mamba-3 SSM layer on B200: prefill tokens/s (headline) and
-decode tokens/s, with roofline fractions, an end-to-end number through host
-buffers, and the fp64 CPU oracle timed on a bounded sample as a baseline.
+"""Benchmark of the Mamba-3 SSM layer on B200: prefill tokens/s (headline: the
+MIMO rank-4 layer, b = 8, L = 2048, H = 64, P = 64, N = 128, chunk 64) and, as
+lines of their own, the SISO layer, the long-context MIMO layer at L = 32768
+and 16384, and decode tokens/s at rank 1 and rank 4 (b = 128, 1024 consecutive
+steps), each with its roofline fraction and the fp64 CPU oracle timed on a
+bounded sample as a baseline; an end-to-end number through host buffers for
+the headline.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--impl m3|reference]
@@ -526,7 +530,7 @@ def time_e2e_prefill(inp_host, s, steps):
 
 # ---- CPU oracle baseline ----------------------------------------------------
 
-def cpu_oracle_prefill(inp_host, s, budget_s=12.0, single_thread=True):
+def cpu_oracle_prefill(inp_host, s, budget_s=10.0, single_thread=False):
     """Time the oracle (as it stands) on whole (batch, head) chains of the same
     workload until about `budget_s` seconds of CPU work; tokens/s counts the
     tokens those chains cover (chains / nheads * seqlen).  With single_thread,
@@ -563,6 +567,130 @@ def cpu_oracle_prefill(inp_host, s, budget_s=12.0, single_thread=True):
     return res
 
 
+DECODE_CPU_STEPS = 64
+
+
+def cpu_oracle_decode(dec, s, budget_s=10.0, steps=DECODE_CPU_STEPS):
+    """The oracle's decode driver (m3o_decode_step as it stands, one thread) on
+    the first `steps` decode steps of whole batch rows (every head), one row
+    after another until about `budget_s` seconds.  tokens/s = rows x steps /
+    time.  A step's cost does not depend on its index, so this is also the
+    rate of the full 1024-step run: the figure is extrapolated from the first
+    `steps` steps, and the sample says so."""
+    import oracle
+    rows, elapsed = 0, 0.0
+    host = {k: v.cpu() for k, v in dec.items()}
+    while rows < s.batch and elapsed < budget_s:
+        i = rows
+        st = host["state0"][i:i + 1].double().numpy()
+        t0 = time.perf_counter()
+        for t in range(steps):
+            Bp = host["B_prev"][i:i + 1] if t == 0 else host["B"][t - 1, i:i + 1]
+            xp = host["x_prev"][i:i + 1] if t == 0 else host["x"][t - 1, i:i + 1]
+            _, st = oracle.decode_step(st, host["x"][t, i:i + 1], host["dt"][t, i:i + 1],
+                                       host["A"][t, i:i + 1], host["lam"][t, i:i + 1],
+                                       host["theta"][t, i:i + 1], host["B"][t, i:i + 1],
+                                       host["C"][t, i:i + 1], Bp, xp)
+        elapsed += time.perf_counter() - t0
+        rows += 1
+    return {"value": round(rows * steps / elapsed, 1), "unit": "tokens/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{rows} of {s.batch} sequences (all {s.nheads} heads), the first "
+                      f"{steps} of the workload's steps, {elapsed:.1f} s on one thread; "
+                      f"tokens/s extrapolated to the full run (constant cost per step)"}
+
+
+# ---- one bench line per workload ---------------------------------------------
+
+SEEDS = {"siso_prefill": 1001, "mimo_prefill": 1002, "long_mimo_32k": 1004,
+         "long_mimo_16k": 1014, "decode_r1": 1003, "decode_r4": 1013}
+PROFILE = {"siso_prefill": "tc_scan_kernel_siso_prefill.md",
+           "mimo_prefill": "tc_scan_kernel_mimo_prefill.md"}
+
+
+def prefill_traffic(name, plan):
+    """DRAM bytes per launch of the scan kernel from its committed ncu summary
+    (one-launch calls only), and where it came from."""
+    summary = PROFILE.get(name)
+    if not summary or not plan["tensor_core"] or plan["segments"] != 1:
+        return None, None
+    t = profile_traffic(summary)
+    return t, (f"profiles/{summary}" if t is not None else None)
+
+
+def prefill_line(name, rank, world, steps, warmup, flush, peaks, psrc, cpu=True):
+    """Device throughput of m3_scan_fwd on one workload (inputs resident in HBM,
+    L2 flushed between timed steps), its roofline and the oracle baseline.
+    Returns (line, device inputs)."""
+    w = WORKLOADS[name]
+    s = w.shape
+    inp = I.make_scan_inputs(w, seed=SEEDS[name] + 7919 * rank, device="cuda")
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        times = time_prefill(inp, s, steps, warmup, flush)
+    barrier(world)
+    per_step = max_over_ranks(sum(times), world) / steps
+    flops, byt = prefill_work(s)
+    plan = m3.scan_plan(m3.scan_shape(inp["x"], inp["B"], s.chunk))
+    kern = "tc_scan_kernel (tcgen05)" if plan["tensor_core"] else "CUDA-core scan kernels"
+    traffic, traffic_src = prefill_traffic(name, plan)
+    line = {
+        "metric": "prefill tokens/s",
+        "value": round(world * s.batch * s.seqlen / per_step, 1),
+        "unit": "tokens/s", "steps": steps, "warmup": warmup,
+        "ms_per_step": round(per_step * 1e3, 4),
+        "config": {"workload": name, **shape_cfg(s),
+                   "l2": "flushed between timed steps (256 MiB write)",
+                   "path": f"{kern}, {plan['launches']} launch(es) per call, "
+                           f"{plan['segments']} segment(s) per sequence"},
+        "roofline": {**roofline(flops, byt, per_step, peaks, psrc),
+                     "scope": ("the one kernel launch of each m3_scan_fwd call, CUDA events on "
+                               "the launching stream" if plan["launches"] == 1 else
+                               "whole m3_scan_fwd call (all its launches), CUDA events on the "
+                               "launching stream"),
+                     "traffic": traffic, "traffic_source": traffic_src,
+                     "algorithmic_flops": flops, "algorithmic_bytes": byt},
+        "gpu_launches": steps * plan["launches"],
+        "clocks": clk.summary(),
+    }
+    if cpu and rank == 0 and world == 1:
+        host = {k: v.cpu() for k, v in inp.items()}
+        line["cpu_baseline"] = cpu_oracle_prefill(host, s)
+    return line, inp
+
+
+def decode_line(name, rank, world, dsteps, warmup, peaks, psrc, cpu=True):
+    """1024 consecutive decode steps (b = 128, H = 64), state updated in place."""
+    dw = I.DECODE_SISO if name == "decode_r1" else I.DECODE_MIMO
+    ds = dw.shape
+    dec = I.make_decode_inputs(dw, seed=SEEDS[name] + 7919 * rank, steps=dsteps + warmup,
+                               device="cuda")
+    barrier(world)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t = time_decode(dec, ds, dsteps, warmup)
+    dt_total = max_over_ranks(t, world)
+    dflops, dbyt = decode_work(ds)
+    dkey = "traffic_bytes_per_launch_r1" if ds.rank == 1 else "traffic_bytes_per_launch_r4"
+    dtraffic = profile_traffic("decode_kernels_b128_h64_n128_p64.md", dkey)
+    line = {
+        "metric": "decode tokens/s", "value": round(world * ds.batch * dsteps / dt_total, 1),
+        "unit": "tokens/s", "steps": dsteps, "us_per_step": round(dt_total / dsteps * 1e6, 2),
+        "config": {"workload": name, **shape_cfg(ds),
+                   "l2": "not flushed: each step streams the 268 MB state, twice L2"},
+        "roofline": {**roofline(dflops, dbyt, dt_total / dsteps, peaks, psrc),
+                     "scope": "one m3_decode_step launch, averaged over the consecutive steps",
+                     "traffic": dtraffic,
+                     "traffic_source": ("profiles/decode_kernels_b128_h64_n128_p64.md"
+                                        if dtraffic is not None else None)},
+        "gpu_launches": dsteps,
+        "clocks": clk.summary(),
+    }
+    if cpu and rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_oracle_decode(dec, ds)
+    return line
+
+
 # ---- main -------------------------------------------------------------------
 
 def run_reference(args, s, wname):
@@ -572,7 +700,7 @@ def run_reference(args, s, wname):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    inp = I.make_scan_inputs(I.Workload(s), seed=1001)
+    inp = I.make_scan_inputs(WORKLOADS[wname], seed=SEEDS[wname])
     vals = []
     budget = max(2.0, 120.0 / max(args.steps + args.warmup, 1))
     for i in range(args.warmup + args.steps):
@@ -597,12 +725,16 @@ def shape_cfg(s: I.Shape):
             "io": s.io}
 
 
+HEADLINE = "mimo_prefill"
+SUBLINES = ("siso_prefill", "long_mimo_32k", "long_mimo_16k")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="siso_prefill", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="m3", choices=["m3", "reference"])
     ap.add_argument("--decode-steps", type=int, default=1024,
                     help="consecutive decode steps timed (each with its own token's inputs)")
@@ -671,123 +803,84 @@ def main():
                           "roofline": roofline(flops, byt, per, peaks, psrc)}))
         return
 
-    # prefill: inputs generated on the device (seeded per rank)
-    inp = I.make_scan_inputs(I.Workload(s), seed=1001 + 7919 * rank, device="cuda")
+    cpu = not args.no_cpu_baseline
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        times = time_prefill(inp, s, args.steps, args.warmup, flush)
-    torch.cuda.synchronize()
-    barrier(world)
-    total = max_over_ranks(sum(times), world)
-    per_step = total / args.steps
-    tokens = s.batch * s.seqlen
-    flops, byt = prefill_work(s)
-
-    # secondary line: the SISO workload with B and C per head (G = H), which
-    # moves 0.5 GB more through HBM per call
-    secondary = None
-    if args.workload == "siso_prefill":
-        s2 = dataclasses.replace(s, ngroups=s.nheads)
-        inp2 = I.make_scan_inputs(I.Workload(s2), seed=1011 + 7919 * rank, device="cuda")
-        barrier(world)
-        t2 = max_over_ranks(sum(time_prefill(inp2, s2, max(3, args.steps // 2), args.warmup,
-                                             flush)), world) / max(3, args.steps // 2)
-        f2, b2 = prefill_work(s2)
-        secondary = {"workload": "siso_prefill, B and C per head (ngroups = nheads = 64)",
-                     "value": round(world * s2.batch * s2.seqlen / t2, 1), "unit": "tokens/s",
-                     "ms_per_step": round(t2 * 1e3, 4),
-                     "roofline": roofline(f2, b2, t2, peaks, psrc)}
-        del inp2
-
-    # a packed batch of mixed lengths with the same layer shape
-    varlen = varlen_line(s, rank, world, max(3, args.steps // 2), args.warmup, flush, peaks,
-                         psrc)
-
-    # QK-norm + bias prep of B and C (block-level step before the scan)
-    bc_prep = prep_line(s, world, 10, args.warmup, flush, peaks, psrc)
-
-    # backward of the same scan (gradients of every input), CUDA cores fp32
-    backward = bwd_line(inp, s, world, 3, args.warmup, flush, peaks)
-
-    # decode (b = 128, H = 64, R as the prefill workload)
-    dw = I.DECODE_MIMO if s.rank > 1 else I.DECODE_SISO
-    ds = dw.shape
-    dsteps = args.decode_steps
-    dec = I.make_decode_inputs(dw, seed=1003 + 7919 * rank, steps=dsteps + args.warmup,
-                               device="cuda")
-    barrier(world)
-    dt_total = max_over_ranks(time_decode(dec, ds, dsteps, args.warmup), world)
-    dflops, dbyt = decode_work(ds)
-    del dec
-
-    # end to end through host buffers (inputs drawn on the host)
+    # the headline workload (inputs drawn on the device, seeded per rank)
+    head, inp = prefill_line(args.workload, rank, world, args.steps, args.warmup, flush, peaks,
+                             psrc, cpu=False)
     inp_host = {k: v.cpu() for k, v in inp.items()}
     del inp
+    # end to end through host buffers (the same inputs, copied from pinned host memory)
     e2e_step, h2d, d2h = time_e2e_prefill(inp_host, s, max(3, args.steps // 4))
     e2e_step = max_over_ranks(e2e_step, world)
-
-    plan = m3.scan_plan(m3.scan_shape(inp_host["x"], inp_host["B"], s.chunk))
-    launches_per_call = plan["launches"]
-    kern = "tc_scan_kernel (tcgen05)" if plan["tensor_core"] else "CUDA-core scan kernels"
-    # DRAM traffic per launch from the committed ncu summaries (None if stale
-    # or if the workload is not the one the summary was scaled to)
-    traffic, traffic_src = None, None
-    summary = {"siso_prefill": "tc_scan_kernel_siso_prefill.md",
-               "mimo_prefill": "tc_scan_kernel_mimo_prefill.md"}.get(args.workload)
-    if summary and plan["tensor_core"] and plan["segments"] == 1:
-        traffic = profile_traffic(summary)
-        traffic_src = f"profiles/{summary}" if traffic is not None else None
-    dkey = "traffic_bytes_per_launch_r1" if ds.rank == 1 else "traffic_bytes_per_launch_r4"
-    dtraffic = profile_traffic("decode_kernels_b128_h64_n128_p64.md", dkey) \
-        if ds.rank in (1, 4) and ds.batch == 128 else None
-    dtraffic_src = "profiles/decode_kernels_b128_h64_n128_p64.md" if dtraffic is not None else None
+    tokens = s.batch * s.seqlen
     line = {
         "metric": "prefill tokens/s",
-        "value": round(world * tokens / per_step, 1),
-        "unit": "tokens/s",
+        "value": head["value"], "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(per_step * 1e3, 4),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": s.io,
-        "data": "synthetic",
-        "config": {"workload": args.workload, **shape_cfg(s),
-                   "parallelism": f"dp{world} (independent batches per rank)",
-                   "l2": "flushed between timed steps (256 MiB write)",
-                   "path": f"{kern}, {launches_per_call} launch(es) per call, "
-                           f"{plan['segments']} segment(s) per sequence"},
-        "roofline": {**roofline(flops, byt, per_step, peaks, psrc),
-                     "scope": ("the one kernel launch of each m3_scan_fwd call, CUDA events on "
-                               "the launching stream" if launches_per_call == 1 else
-                               "whole m3_scan_fwd call (all launches), CUDA events"),
-                     "traffic": traffic, "traffic_source": traffic_src,
-                     "algorithmic_flops": flops, "algorithmic_bytes": byt},
-        "decode": {
-            "metric": "decode tokens/s", "value": round(world * ds.batch * dsteps / dt_total, 1),
-            "unit": "tokens/s", "steps": dsteps, "us_per_step": round(dt_total / dsteps * 1e6, 2),
-            "config": {"workload": "decode_siso" if ds.rank == 1 else "decode_mimo",
-                       **shape_cfg(ds)},
-            "roofline": {**roofline(dflops, dbyt, dt_total / dsteps, peaks, psrc),
-                         "traffic": dtraffic, "traffic_source": dtraffic_src},
-        },
+        "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": s.io, "data": "synthetic",
+        "config": {**head["config"], "parallelism": f"dp{world} (independent batches per rank)"},
+        "roofline": head["roofline"],
         "e2e": {"value": round(world * tokens / e2e_step, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_step * 1e3, 3),
                 "mode": "pinned host buffers; copies in, scan, copies out on three streams "
                         "with two buffer sets (step i's copy out overlaps step i+1)"},
-        "gpu_launches": args.steps * launches_per_call,
-        "clocks": clk.summary(),
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
     }
-    if secondary is not None:
-        line["secondary"] = secondary
-    line["varlen"] = varlen
-    line["backward"] = backward
-    line["bc_prep"] = bc_prep
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_oracle_prefill(inp_host, s)
+    if cpu and rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_oracle_prefill(inp_host, s, single_thread=True)
+    del inp_host
+
+    # the other prefill workloads and both decode ranks, each a line of its own
+    siso_inp = None
+    for name in SUBLINES:
+        if name == args.workload:
+            continue
+        sub, sub_inp = prefill_line(name, rank, world, args.steps, args.warmup, flush, peaks,
+                                    psrc, cpu=cpu)
+        line[name] = sub
+        if name == "siso_prefill":
+            siso_inp = sub_inp
+        del sub_inp
+    for name in ("decode_r1", "decode_r4"):
+        line[name] = decode_line(name, rank, world, args.decode_steps, args.warmup, peaks, psrc,
+                                 cpu=cpu)
+
+    # the SISO layer with B and C per head (G = H), which moves 0.5 GB more
+    # through HBM per call
+    ss = I.SISO_PREFILL.shape
+    s2 = dataclasses.replace(ss, ngroups=ss.nheads)
+    inp2 = I.make_scan_inputs(I.Workload(s2), seed=1011 + 7919 * rank, device="cuda")
+    barrier(world)
+    t2 = max_over_ranks(sum(time_prefill(inp2, s2, max(3, args.steps // 2), args.warmup,
+                                         flush)), world) / max(3, args.steps // 2)
+    f2, b2 = prefill_work(s2)
+    line["siso_per_head_bc"] = {
+        "workload": "siso_prefill, B and C per head (ngroups = nheads = 64)",
+        "value": round(world * s2.batch * s2.seqlen / t2, 1), "unit": "tokens/s",
+        "ms_per_step": round(t2 * 1e3, 4), "roofline": roofline(f2, b2, t2, peaks, psrc)}
+    del inp2
+
+    # a packed batch of mixed lengths with the SISO layer shape
+    line["varlen"] = varlen_line(ss, rank, world, max(3, args.steps // 2), args.warmup, flush,
+                                 peaks, psrc)
+    # QK-norm + bias prep of B and C (block-level step before the scan)
+    line["bc_prep"] = prep_line(ss, world, 10, args.warmup, flush, peaks, psrc)
+    # backward of the SISO and MIMO scans (gradients of every input)
+    if siso_inp is None:
+        siso_inp = I.make_scan_inputs(I.SISO_PREFILL, seed=SEEDS["siso_prefill"] + 7919 * rank,
+                                      device="cuda")
+    line["backward"] = bwd_line(siso_inp, ss, world, 3, args.warmup, flush, peaks)
+    del siso_inp
+    ms = I.MIMO_PREFILL.shape
+    mimo_inp = I.make_scan_inputs(I.MIMO_PREFILL, seed=SEEDS["mimo_prefill"] + 7919 * rank,
+                                  device="cuda")
+    line["backward_mimo"] = bwd_line(mimo_inp, ms, world, 3, args.warmup, flush, peaks)
+    del mimo_inp
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
