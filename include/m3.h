@@ -100,6 +100,10 @@ typedef enum {
 /* theta holds one angle-rate vector per head: [b][L][H][N/2] for the scan,
  * [b][H][N/2] for the decode step (default: per group, like B and C). */
 #define M3_FLAG_THETA_PER_HEAD 4u
+/* m3_scan_bwd, m3_scan_bwd_varlen: dy is fp32 whatever the io dtype (a bf16
+ * layer trained with fp32 output gradients keeps them unrounded).  Ignored
+ * by every other call. */
+#define M3_FLAG_DY_F32 8u
 
 typedef struct {
   int64_t batch;    /* b >= 1                                   */
@@ -208,7 +212,9 @@ M3_API int m3_decode_step(const m3_shape* shape, const float* state_in,
  *     M3_NOALLOC_SCRATCH_BYTES return M3_ERR_WORKSPACE and launch nothing.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept with the identity of
+ *     the device's context and looked up again when that changes (after a
+ *     cudaDeviceReset, say), so it never outlives the module it points into.
  *   - Nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
  *     library routine.
  *   - All calls on a device share the array, which keeps the last call's
@@ -232,7 +238,8 @@ M3_API int m3_scan_fwd_noalloc(const m3_shape* shape, const void* x, const float
  * cores in fp32 for both io dtypes; every gradient is written in fp32.
  *
  *   inputs      as m3_scan_fwd (same layouts, dtypes and nullability).
- *   dy          [b][L][H][R][P] io dtype (required when L > 0).
+ *   dy          [b][L][H][R][P] io dtype, or fp32 with M3_FLAG_DY_F32 (required
+ *               when L > 0).
  *   d_final     [b][H][N][P] fp32, or NULL for zero.
  *   dx          [b][L][H][R][P] fp32;  ddt, dA, dlam [b][L][H] fp32;
  *   dtheta      fp32, theta's layout;  dB, dC [b][L][G][R][N] fp32 (summed
@@ -362,7 +369,8 @@ M3_API int m3_scan_state(const m3_shape* shape, const void* x, const float* dt, 
 
 /* Segment totals: lam_tot [b][H] = sum_t dt_t A_t and phi_tot [b][H][N/2] =
  * sum_t dt_t theta_{t,k} over the shape's seqlen tokens, accumulated in fp64
- * and written fp32.  dt, A, theta as for m3_scan_fwd (4-byte aligned device
+ * and written fp32; phi_tot is reduced to [-pi, pi] first (the angle acts only
+ * through its cosine and sine).  dt, A, theta as for m3_scan_fwd (4-byte aligned device
  * pointers); outputs 4-byte aligned device arrays owned by the caller. */
 M3_API int m3_segment_totals(const m3_shape* shape, const float* dt, const float* A,
                              const float* theta, float* lam_tot, float* phi_tot,

@@ -7,8 +7,15 @@ library's kernels.
                              B_prev=None, x_prev=None)
 
 Layouts as m3_scan_fwd.  Gradients flow to every tensor argument that
-requires them; they are computed in fp32 and returned in each input's dtype
-(bf16 inputs get bf16 gradients).
+requires them.  Precision: the incoming gradient of y is handed to the
+backward as it arrives, never rounded here.  torch's engine delivers the
+gradient of an output in that output's dtype, so for a bf16 layer dy is
+already bf16 when it gets here; callers that hold fp32 output gradients and
+want them used unrounded call m3.m3_scan_bwd directly with an fp32 dy (the
+C ABI's M3_FLAG_DY_F32).  The final-state gradient is fp32.  The backward
+computes every gradient in fp32; each is returned in its input's dtype, as
+torch requires (bf16 x, B, C, B_prev, x_prev receive bf16 gradients, rounded
+to nearest even once, at the end; dt, A, lam, theta, h0 are fp32).
 """
 from __future__ import annotations
 
@@ -17,6 +24,14 @@ import torch
 from . import m3
 
 _NAMES = ("x", "dt", "A", "lam", "theta", "B", "C", "h0", "B_prev", "x_prev")
+
+
+def _dy(dy, x):
+    """dy as the backward reads it: x's dtype, or fp32 unrounded (anything else
+    is converted to fp32 first, which is exact for every narrower float)."""
+    if dy.dtype != x.dtype and dy.dtype != torch.float32:
+        dy = dy.float()
+    return dy.contiguous()
 
 
 class M3Scan(torch.autograd.Function):
@@ -32,7 +47,7 @@ class M3Scan(torch.autograd.Function):
         x, dt, A, lam, theta, B, C, h0, B_prev, x_prev = ctx.saved_tensors
         if dy is None:
             dy = torch.zeros_like(x)
-        g = m3.m3_scan_bwd(x, dt, A, lam, theta, B, C, dy.contiguous().to(x.dtype), ctx.chunk,
+        g = m3.m3_scan_bwd(x, dt, A, lam, theta, B, C, _dy(dy, x), ctx.chunk,
                            h0, B_prev, x_prev,
                            None if d_final is None else d_final.contiguous().float())
         inputs = dict(zip(_NAMES, (x, dt, A, lam, theta, B, C, h0, B_prev, x_prev)))
@@ -66,7 +81,7 @@ class M3ScanVarlen(torch.autograd.Function):
         cu, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev = ctx.saved_tensors
         if dy is None:
             dy = torch.zeros_like(x)
-        g = m3.m3_scan_bwd_varlen(cu, x, dt, A, lam, theta, B, C, dy.contiguous().to(x.dtype),
+        g = m3.m3_scan_bwd_varlen(cu, x, dt, A, lam, theta, B, C, _dy(dy, x),
                                   ctx.chunk, h0, B_prev, x_prev,
                                   None if d_final is None else d_final.contiguous().float(),
                                   max_seqlen=ctx.max_seqlen)

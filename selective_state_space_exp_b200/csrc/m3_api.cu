@@ -1,7 +1,10 @@
 // m3_api.cu -- the C ABI declared in include/m3.h: argument checks, workspace
 // sizing, dispatch to the kernels, and the device-side error word.
+#include <cuda.h>  // CUcontext (the driver calls are reached through the runtime)
+
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "m3_internal.cuh"
 
@@ -9,6 +12,30 @@ namespace m3 {
 
 // First device-side error raised by a kernel (M3_ERR_*), 0 if none.
 __device__ int g_device_status = 0;
+
+unsigned long long current_context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+  });
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&c) != CUDA_SUCCESS || !c ||
+      get_id(c, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 namespace {
 
@@ -23,7 +50,8 @@ int check_common(const m3_shape* s) {
     return M3_ERR_INVALID_ARGUMENT;
   if (s->dstate % 2 != 0 || s->nheads % s->ngroups != 0) return M3_ERR_INVALID_ARGUMENT;
   if (s->io_dtype != M3_F32 && s->io_dtype != M3_BF16) return M3_ERR_INVALID_ARGUMENT;
-  if ((s->flags & ~(M3_FLAG_SIMT | M3_FLAG_TEST_TIMEOUT | M3_FLAG_THETA_PER_HEAD)) != 0)
+  if ((s->flags & ~(M3_FLAG_SIMT | M3_FLAG_TEST_TIMEOUT | M3_FLAG_THETA_PER_HEAD |
+                    M3_FLAG_DY_F32)) != 0)
     return M3_ERR_INVALID_ARGUMENT;
   // supported set
   if (!is_pow2(s->dstate) || s->dstate < 16 || s->dstate > 256) return M3_ERR_UNSUPPORTED;
@@ -55,15 +83,20 @@ ScanArgs make_scan_args(const m3_shape* s) {
 }
 
 int status_word(int** out) {
-  // Device address of g_device_status, looked up once per device.
+  // Device address of g_device_status, looked up once per device and context.
   constexpr int kMaxDevices = 64;
+  static std::mutex mu;
   static int* cache[kMaxDevices] = {};
+  static unsigned long long cache_ctx[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return M3_ERR_CUDA;
-  if (!cache[dev]) {
+  std::lock_guard<std::mutex> lock(mu);
+  const unsigned long long ctx = current_context_id();
+  if (!cache[dev] || ctx == 0 || ctx != cache_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return M3_ERR_CUDA;
     cache[dev] = static_cast<int*>(p);
+    cache_ctx[dev] = current_context_id();  // the lookup made a context current if none was
   }
   *out = cache[dev];
   return M3_OK;
@@ -283,7 +316,8 @@ int bwd_call(const m3_shape* s, const int32_t* cu_seqlens, int64_t total_tokens,
   a.total_tokens = varlen ? total_tokens : s->batch * s->seqlen;
   if (status_word(&a.status) != M3_OK) return M3_ERR_CUDA;
   BwdArgs g;
-  g.dy = dy; g.d_final = d_final; g.dx = dx; g.ddt = ddt; g.dA = dA; g.dlam = dlam;
+  g.dy = dy; g.dy_f32 = (s->flags & M3_FLAG_DY_F32) != 0;
+  g.d_final = d_final; g.dx = dx; g.ddt = ddt; g.dA = dA; g.dlam = dlam;
   g.dtheta = dtheta; g.dB = dB; g.dC = dC; g.dh0 = dh0;
   g.dB_prev = B_prev ? dB_prev : nullptr;
   g.dx_prev = B_prev ? dx_prev : nullptr;

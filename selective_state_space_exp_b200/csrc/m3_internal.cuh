@@ -89,6 +89,12 @@ struct DecodeArgs {
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// A process-unique identity of the calling thread's current CUDA context
+// (0 when there is none yet or the driver cannot say).  Device addresses of
+// the library's __device__ variables are cached with it: a device reset
+// replaces the context and reloads the module, which may move them.
+unsigned long long current_context_id();
+
 // CUDA-core fp32 scan (chunk state -> state passing -> chunk output).
 size_t simt_scan_workspace(const ScanArgs& a);
 cudaError_t simt_scan_launch(const ScanArgs& a, cudaStream_t s);
@@ -106,7 +112,8 @@ void simt_state_views(const ScanArgs& a, float** states, float** sums);
 
 // Backward pass of the scan (CUDA cores, fp32): outputs and incoming adjoints.
 struct BwdArgs {
-  const void* dy;         // [b][L][H][R][P] io dtype
+  const void* dy;         // [b][L][H][R][P] io dtype (fp32 when dy_f32)
+  bool dy_f32;            // M3_FLAG_DY_F32
   const float* d_final;   // [b][H][N][P] or nullptr
   float* dx;              // [b][L][H][R][P]
   float* ddt;             // [b][L][H]

@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(512) bwd_sums_kernel(const ScanArgs a, const B
       if (s < q.nt) {
         const int64_t o = ((q.base + q.t0 + s) * a.nheads + q.h) * R * P + (int64_t)r * P + p;
         xv = io_load(a.x, o, a.bf16);
-        yv = io_load(g.dy, o, a.bf16);
+        yv = io_load(g.dy, o, a.bf16 && !g.dy_f32);
       }
       Xs[ri * P + p] = xv;
       Ys[ri * P + p] = yv;
@@ -494,7 +494,7 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(const ScanArgs a, c
     if (s < nt) {
       const int64_t o = ((q.base + q.t0 + s) * H + q.h) * R * P + (int64_t)r * P + p;
       xv = io_load(a.x, o, a.bf16);
-      yv = io_load(g.dy, o, a.bf16);
+      yv = io_load(g.dy, o, a.bf16 && !g.dy_f32);
     }
     X[ri * ldp + p] = xv;
     dY[ri * ldp + p] = yv;

@@ -7,8 +7,10 @@
 // the process exits.  Host code cannot use the array's name as a device
 // address (on the host it is only a stand-in symbol), so the first call on
 // each device looks up the real address with cudaGetSymbolAddress while that
-// device is current, caches it, and every call hands that address to the
-// scan as its workspace.
+// device is current, caches it with the identity of the device's context, and
+// every call hands that address to the scan as its workspace.  A new context
+// on the device (after a cudaDeviceReset) triggers a fresh lookup, since the
+// reloaded module may put the array elsewhere.
 //
 // All calls on a device share the one array.  The scan writes every scratch
 // element before it reads it (chunk states and chunk summaries), so nothing
@@ -28,17 +30,21 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[M3_NOALLOC_SCRA
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up once).
+// Device address of the scratch array on the current device (looked up once
+// per device and context).
 int scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return M3_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (!g_scratch_addr[dev]) {
+  const unsigned long long ctx = current_context_id();
+  if (!g_scratch_addr[dev] || ctx == 0 || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return M3_ERR_CUDA;
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = current_context_id();  // the lookup made a context current if none was
   }
   *out = g_scratch_addr[dev];
   return M3_OK;

@@ -276,7 +276,10 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   };
   if (MODE == MODE_FULL) store_state_bf16();
 
-  float l2seg = 0.f, phi_seg = 0.f;  // MODE_STATE summaries (pair k = n / 2), log2 units
+  // MODE_STATE summaries (pair k = n / 2): log-decay in log2 units, and the
+  // angle in fp64 (thousands of radians over a long segment), stored mod 2 pi
+  float l2seg = 0.f;
+  double phi_seg = 0.0;
   const int64_t c_begin = seg * pl.cps;
   const int64_t c_end = min(c_begin + pl.cps, (L + Q - 1) / Q);
 
@@ -473,7 +476,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         phi[2] += ang[u][1].x; phi[3] += ang[u][1].y;
         float cs[4], sn[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) __sincosf(phi[j], &sn[j], &cs[j]);
+        for (int j = 0; j < 4; ++j) __sincosf(reduce_2pi(phi[j]), &sn[j], &cs[j]);
         // two pairs at a time as (even elements, odd elements) fp32x2 vectors:
         // (b0, b1) -> (c b0 + s b1, c b1 - s b0) for each pair
         const float2 c2[2] = {make_float2(cs[0], cs[1]), make_float2(cs[2], cs[3])};
@@ -603,7 +606,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       }
       if (MODE == MODE_STATE) {
         l2seg += l2end;
-        phi_seg += phe;
+        phi_seg += (double)phe;
       }
     }
 
@@ -832,7 +835,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         *reinterpret_cast<float4*>(dst + p) = make_float4(gst[p], gst[p + 1], gst[p + 2], gst[p + 3]);
       float* su = pl.wsSum + slot * (1 + kPairs);
       if (tid == 0) su[0] = l2seg * kLn2;
-      if (cq == 0 && (n & 1) == 0) su[1 + (n >> 1)] = phi_seg;
+      if (cq == 0 && (n & 1) == 0) su[1 + (n >> 1)] = (float)remainder(phi_seg, 6.283185307179586);
     }
   }
   // an aborted run may leave a prefetch in flight: let it land (bounded wait)

@@ -16,7 +16,10 @@
 namespace m3 {
 namespace {
 
-// Lam_seg[b][H] and Phi_seg[b][H][N/2], accumulated in fp64 over the segment.
+// Lam_seg[b][H] and Phi_seg[b][H][N/2], accumulated in fp64 over the segment;
+// the angle is stored reduced to [-pi, pi] (it only enters through its sine and
+// cosine, and a long segment's total reaches thousands of radians, where an
+// fp32 value would have lost its fraction).
 // Block (b, h); thread k < K sums pair k's angles, thread K the log-decay.
 __global__ void segment_totals_kernel(const float* dt, const float* A, const float* theta,
                                       int64_t L, int64_t H, int64_t tgroups, int K,
@@ -28,7 +31,7 @@ __global__ void segment_totals_kernel(const float* dt, const float* A, const flo
     if (k < K) {
       for (int64_t t = 0; t < L; ++t)
         acc += (double)dt[(b * L + t) * H + h] * (double)theta[((b * L + t) * tgroups + tg) * K + k];
-      phi_tot[(b * H + h) * K + k] = (float)acc;
+      phi_tot[(b * H + h) * K + k] = (float)remainder(acc, 6.283185307179586);
     } else {
       for (int64_t t = 0; t < L; ++t)
         acc += (double)dt[(b * L + t) * H + h] * (double)A[(b * L + t) * H + h];

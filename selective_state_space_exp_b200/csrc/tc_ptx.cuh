@@ -184,6 +184,17 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// x minus the nearest multiple of 2 pi (about [-pi, pi]), so that the fast
+// sin / cos below get arguments inside the range their accuracy is stated
+// for.  Cody and Waite's two-part reduction: 2 pi = 6.28125 + 1.9353...e-3,
+// whose first part has 8 significant bits, so n * 6.28125 is exact for
+// |n| < 2^16 and the fused steps lose nothing before the small correction.
+__device__ __forceinline__ float reduce_2pi(float x) {
+  const float n = rintf(x * 0.15915494309189535f);
+  const float r = fmaf(-n, 6.28125f, x);
+  return fmaf(-n, 1.9353071795864769e-3f, r);
+}
+
 // TMA: 3-D tiled bulk tensor load global -> this CTA's shared memory, completing
 // `bytes` of transaction count on an mbarrier.  `map` is the generic address
 // of a CUtensorMap kernel parameter.

@@ -21,6 +21,7 @@ M3_F32, M3_BF16 = 0, 1
 M3_FLAG_SIMT = 1
 M3_FLAG_TEST_TIMEOUT = 2
 M3_FLAG_THETA_PER_HEAD = 4
+M3_FLAG_DY_F32 = 8
 M3_OK, M3_ERR_INVALID_ARGUMENT, M3_ERR_TIMEOUT = 0, -1, -6
 
 
@@ -251,6 +252,16 @@ def m3_bc_prep(B_raw=None, C_raw=None, B_weight=None, B_bias=None, C_weight=None
     return B, C
 
 
+def dy_flag(dy: torch.Tensor, x: torch.Tensor) -> int:
+    """M3_FLAG_DY_F32 when dy is fp32 and the io dtype is not; otherwise dy
+    must have x's dtype."""
+    if dy.dtype == x.dtype:
+        return 0
+    if dy.dtype == torch.float32:
+        return M3_FLAG_DY_F32
+    raise TypeError(f"dy is {dy.dtype}: expected {x.dtype} or torch.float32")
+
+
 def bwd_workspace_size(shape: Shape) -> int:
     n = ctypes.c_size_t(0)
     _check("m3_scan_bwd_workspace_size",
@@ -261,10 +272,12 @@ def bwd_workspace_size(shape: Shape) -> int:
 def m3_scan_bwd(x, dt, A, lam, theta, B, C, dy, chunk: int = 64, h0=None, B_prev=None,
                 x_prev=None, d_final=None, *, want_dh0=True, workspace=None, stream=None):
     """Backward of m3_scan_fwd: gradients of sum(y * dy) + sum(final * d_final)
-    with respect to every input.  Returns a dict of fp32 tensors: x, dt, A, lam,
-    theta, B, C, and h0 (when want_dh0), B_prev and x_prev (when B_prev is given),
-    each in its input's layout."""
+    with respect to every input.  dy has x's dtype, or fp32 (read unrounded).
+    Returns a dict of fp32 tensors: x, dt, A, lam, theta, B, C, and h0 (when
+    want_dh0), B_prev and x_prev (when B_prev is given), each in its input's
+    layout."""
     shape = scan_shape(x, B, chunk, False, theta)
+    shape.flags |= dy_flag(dy, x)
     dev, f32 = x.device, torch.float32
     g = {"x": torch.empty(x.shape, dtype=f32, device=dev),
          "dt": torch.empty(dt.shape, dtype=f32, device=dev),
@@ -305,7 +318,7 @@ def m3_scan_bwd_varlen(cu_seqlens, x, dt, A, lam, theta, B, C, dy, chunk: int = 
     if max_seqlen is None:
         max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item()) if S > 0 else 0
     shape = make_shape(S, max_seqlen, H, G, P, N, R, chunk, x.dtype, False)
-    shape.flags |= theta_flag(theta.shape[1], G, H)
+    shape.flags |= theta_flag(theta.shape[1], G, H) | dy_flag(dy, x)
     dev, f32 = x.device, torch.float32
     g = {k: torch.empty(v.shape, dtype=f32, device=dev)
          for k, v in (("x", x), ("dt", dt), ("A", A), ("lam", lam), ("theta", theta), ("B", B),

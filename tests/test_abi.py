@@ -51,7 +51,7 @@ def shape(**kw):
     (dict(seqlen=0), 0),
     (dict(batch=0), -1), (dict(nheads=0), -1), (dict(seqlen=-1), -1),
     (dict(dstate=127), -1), (dict(nheads=6, ngroups=4), -1), (dict(io_dtype=7), -1),
-    (dict(flags=8), -1), (dict(chunk=0), -1),
+    (dict(flags=8), 0), (dict(flags=16), -1), (dict(chunk=0), -1),
     (dict(rank=3), -2), (dict(dstate=96), -2), (dict(headdim=48), -2),
     (dict(headdim=256), -2), (dict(dstate=256, headdim=128), -2), (dict(chunk=48), -2),
     (dict(chunk=128), -2), (dict(batch=70000), -2),

@@ -94,6 +94,24 @@ def test_bwd_bf16_layer_shape():
     compare(case(batch=1, L=200, H=2, N=128, P=64, R=4, io="bf16", seed=600))
 
 
+def test_bwd_bf16_inputs_fp32_dy():
+    """bf16 inputs with an fp32 output gradient (M3_FLAG_DY_F32): dy is read
+    unrounded, so the gradients meet the 1e-4 bar against the oracle run with
+    the same fp32 dy; the same dy rounded to bf16 first misses that bar, so
+    the flag is what keeps the extra precision."""
+    inp = case(batch=1, L=200, H=2, N=128, P=64, R=4, io="bf16", seed=610)
+    gen = torch.Generator().manual_seed(611)
+    inp["dy"] = torch.randn(inp["x"].shape, generator=gen)  # fp32, not rounded
+    compare(inp)
+    g = to_dev(inp)
+    rounded = m3.m3_scan_bwd(g["x"], g["dt"], g["A"], g["lam"], g["theta"], g["B"], g["C"],
+                             g["dy"].to(torch.bfloat16), 64, g["h0"], g["B_prev"], g["x_prev"],
+                             g["d_final"])
+    _, _, ref = m3_grad.scan_grads(*[inp.get(k) for k in m3_grad.NAMES], dy=inp["dy"],
+                                   d_final=inp["d_final"])
+    assert rel_err(rounded["x"].cpu().numpy(), ref["x"]) > BAR
+
+
 def test_bwd_empty_sequence():
     inp = to_dev(case(batch=1, L=0, H=2, R=1, seed=700))
     got = m3.m3_scan_bwd(inp["x"], inp["dt"], inp["A"], inp["lam"], inp["theta"], inp["B"],
