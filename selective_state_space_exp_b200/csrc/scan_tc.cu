@@ -6,13 +6,27 @@
 // section 2.3 -- rank-R MIMO), per (batch b, head h) and chunk of Q tokens
 // with M = Q*R rows (token, rank):
 //
-//   S   = Ct Bt^T                       M x M,  K = N     (MMA1, tcgen05)
-//   P   = S o mask,  mask[(t,r),(s,r')] = [s<=t] exp(Lam_t - Lam_s) (s==t ? gamma_t : delta_s)
-//   Y   = P X  +  diag(exp(Lam_t)) Ct G  M x P            (MMA2 + MMA4)
-//   Sc  = Bt^T diag(w) X,  w_s = exp(Lam_end - Lam_s) delta_s   (MMA3)
-//   G  <- Rot(Phi_end) (exp(Lam_end) G + Sc)                     (fp32, registers)
+//   y_t = sum_{s<=t} exp(Lam_t - Lam_s) c_ts (Ct_t . Bt_s) x_s + exp(Lam_t) Ct_t G,
+//   c_tt = gamma_t, c_ts = delta_s (s < t);   G <- Rot(Phi_end)(exp(Lam_end) G + Sc),
+//   Sc = sum_s exp(Lam_end - Lam_s) delta_s Bt_s x_s^T,
 //
-// with Bt = Rot(-Phi) B, Ct = Rot(-Phi) C rotated in the chunk-local frame.
+// with Bt = Rot(-Phi) B, Ct = Rot(-Phi) C rotated in the chunk-local frame.  The
+// decay matrix exp(Lam_t - Lam_s) is factored around a reference ref = Lam_end / 2:
+// B is staged as Bh_s = u_s Bt_s with u_s = exp(ref - Lam_s) delta_s, so that
+//
+//   S'  = Ct Bh^T                         M x M,  K = N     (MMA1, tcgen05)
+//   P'  = S' o M',  M'[(t,r),(s,r')] = 1 (s < t), gamma_t / delta_t (s = t), 0 (s > t)
+//   Y'  = P' X + Ct (exp(ref) G)          M x P, one accumulator (MMA2 + MMA4)
+//   y_t = exp(Lam_t - ref) Y'_t                               (epilogue)
+//   Sc  = exp(Lam_end - ref) Bh^T X                           (MMA3)
+//
+// so the mask is a plain causal mask and no weighted copy of x is made.  The
+// factors stay inside fp32 / bf16 range while the chunk's total decay does
+// (|Lam_end| below about 100 nats, every chunk of the usual inputs); a chunk
+// that decays further is done exactly the plain way: Bh_s = delta_s Bt_s for
+// the scores, P[t,s] = S'[t,s] exp(Lam_t - Lam_s), a separate Ct G
+// accumulator scaled by exp(Lam_t), and Bh rescaled in place to
+// exp(Lam_end - Lam_s) delta_s Bt_s before MMA3 reads it.
 // One CTA owns a run of consecutive chunks ("segment") of one (b, h) and
 // carries the fp32 state G across them in registers (thread n holds state
 // row n).  When there are too few (b, h) chains to fill the GPU, each chain is
@@ -38,6 +52,10 @@ constexpr int kN = 128;       // dstate
 constexpr int kP = 64;        // headdim
 constexpr int kPairs = kN / 2;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded mbarrier wait (2 s)
+// A chunk whose total log-decay (log2 units) is at or below this (about -100
+// nats) is done in the plain form: the factored one would need factors beyond
+// e^+-50, where bf16 state and scaled-B values lose their low-order bits.
+constexpr float kPlainL2 = -144.f;
 
 enum { MODE_FULL = 0, MODE_STATE = 1 };
 
@@ -55,8 +73,8 @@ struct Cfg {
   static constexpr int C_OFF = 0;               // Ct: K = N split in 2 blocks of 64
   static constexpr int X_OFF = C_OFF + 2 * OPB;
   static constexpr int B_OFF = X_OFF + OPB;     // Bt: 2 blocks
-  static constexpr int XW_OFF = B_OFF + 2 * OPB;
-  static constexpr int G_OFF = XW_OFF + OPB;    // state, bf16 [N][128 B]
+  static constexpr int ST_OFF = B_OFF + 2 * OPB;  // staging: masked scores of tile 0, y
+  static constexpr int G_OFF = ST_OFF + OPB;    // scaled state, bf16 [N][128 B]
   static constexpr int SMALL_OFF = G_OFF + kN * 128;
   // small region: the chunk's theta [Q][N/2] (a TMA destination, first so it
   // is 1 KB aligned; the slot angle sums go over it once it is read),
@@ -77,11 +95,11 @@ struct Cfg {
   static constexpr int SMEM = SMEM_RAW < 80 * 1024 ? 80 * 1024 : SMEM_RAW;
   static_assert(MINB * (SMEM + 1024) <= 233472, "CTAs per SM must fit the SM's shared memory");
   // Masked scores P, tile mt: ((mt + 1) * MT / 64) K-blocks of [MT][128 B].
-  // One tile: over Bt (MMA1 and MMA3 are done when it is written).  Two
-  // tiles: tile 0 over w*x (MMA3 is done; tile 1's MMA1 still reads all of
-  // Bt), tile 1 over Bt once tile 1's scores are complete.
+  // One tile: over Bh (MMA1 and MMA3 are done when it is written).  Two
+  // tiles: tile 0 in the staging block (tile 1's MMA1 still reads all of Bh),
+  // tile 1 over Bh once tile 1's scores and MMA3 are complete.
   __host__ __device__ static constexpr int p_off(int mt) {
-    return (NT == 2 && mt == 0) ? XW_OFF : B_OFF;
+    return (NT == 2 && mt == 0) ? ST_OFF : B_OFF;
   }
   static_assert(NT == 1 ? (MT / 64) * MT * 128 <= 2 * OPB
                         : (MT / 64) * MT * 128 <= OPB && 2 * (MT / 64) * MT * 128 <= 2 * OPB,
@@ -89,11 +107,13 @@ struct Cfg {
   // TMEM columns
   static constexpr int S_COL1 = 0;                  // tile 1 scores (M = 256 only)
   static constexpr int S_COL0 = (NT == 2) ? 256 : 0;
-  // One tile per chunk: scores (MT columns; the MMA2 output reuses them once
-  // masked), MMA4 output and chunk state side by side, so MMA4 can run with
-  // MMA3 before the mask.  Two tiles: the scores take 384 columns, so a
-  // tile's MMA2 and MMA4 run after its mask and their outputs reuse that
-  // tile's score columns (tile 0's MMAs then overlap tile 1's mask).
+  // One tile per chunk: scores (MT columns), output accumulator and chunk
+  // state side by side, so MMA4 can run with MMA3 before the mask.  Two
+  // tiles: the scores take 384 columns, so a tile's MMA2 and MMA4 run after
+  // its mask and their accumulators reuse that tile's score columns (tile 0's
+  // MMAs then overlap tile 1's mask).  y_col / y2_col: the two accumulators
+  // of the plain (large-decay) form; the factored form accumulates both
+  // products in acc_col.
   static constexpr bool EARLY4 = NT == 1;
   static constexpr int SC_COL = (NT == 2) ? 384 : MT + 64;  // chunk state N x P
   static constexpr int TMEM_COLS = (NT == 2) ? 512 : 256;
@@ -104,6 +124,7 @@ struct Cfg {
   __host__ __device__ static constexpr int y2_col(int mt) {
     return NT == 2 ? (mt == 0 ? 320 : 64) : MT;
   }
+  __host__ __device__ static constexpr int acc_col(int mt) { return NT == 2 ? y_col(mt) : MT; }
   static_assert(SC_COL + kP <= TMEM_COLS, "TMEM columns");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
@@ -176,10 +197,10 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   float* s_th = reinterpret_cast<float*>(sm + C::SMALL_OFF);  // chunk theta [Q][N/2] (TMA)
   float* s_gam = s_th + C::TH_FLOATS + C::PART_FLOATS;  // gamma_t = lam_t dt_t         [Q]
   float* s_del = s_gam + Q;                     // delta_s, trapezoid weight of token s [Q]
-  float* s_w = s_del + Q;                       // exp(Lam_end - Lam_s) delta_s         [Q]
-  float* s_lg = s_w + Q;                        // Lam_t * log2(e)                      [Q]
-  float* s_F = s_lg + Q;                        // exp(ref - Lam_s) delta_s             [Q]
-  float* s_dtv = s_F + Q;                       // dt_t                                 [Q]
+  float* s_u = s_del + Q;                       // row scale u_s of Bh                  [Q]
+  float* s_lg = s_u + Q;                        // Lam_t * log2(e)                      [Q]
+  float* s_d = s_lg + Q;                        // gamma_t / delta_t (mask diagonal)    [Q]
+  float* s_dtv = s_d + Q;                       // dt_t                                 [Q]
   float* s_phe = s_dtv + Q;                     // chunk-end angles                     [kPairs]
   float2* s_pcs = reinterpret_cast<float2*>(s_phe + kPairs);  // their cos, sin        [kPairs]
   uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_pcs + kPairs);  // MMA3+MMA4, MMA2
@@ -225,9 +246,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   // byte offset / 16 to the 14-bit start-address field (shared addresses stay
   // below 256 KB, so the field never carries).
   const uint64_t dC = sw128_desc(sbase + C::C_OFF, 16, 1024);         // Ct, K-major
-  const uint64_t dB = sw128_desc(sbase + C::B_OFF, 16, 1024);         // Bt, K-major
-  const uint64_t dBmn = sw128_desc(sbase + C::B_OFF, C::OPB, 1024);   // Bt, MN-major
-  const uint64_t dXW = sw128_desc(sbase + C::XW_OFF, C::OPB, 1024);   // w*x, MN-major
+  const uint64_t dB = sw128_desc(sbase + C::B_OFF, 16, 1024);         // Bh, K-major
+  const uint64_t dBmn = sw128_desc(sbase + C::B_OFF, C::OPB, 1024);   // Bh, MN-major
   const uint64_t dX = sw128_desc(sbase + C::X_OFF, C::OPB, 1024);     // x, MN-major
   const uint64_t dG = sw128_desc(sbase + C::G_OFF, kN * 128, 1024);   // state, MN-major
   auto dadd = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
@@ -263,18 +283,18 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       gst[p] = v.x; gst[p + 1] = v.y; gst[p + 2] = v.z; gst[p + 3] = v.w;
     }
   }
-  auto store_state_bf16 = [&]() {
+  // The MMA4 operand: the chunk-start state times `scale`, bf16.
+  auto store_state_bf16 = [&](float scale) {
 #pragma unroll
     for (int c2 = 0; c2 < CW / 8; ++c2) {
       uint4 v;
-      v.x = pack_bf16(gst[8 * c2 + 0], gst[8 * c2 + 1]);
-      v.y = pack_bf16(gst[8 * c2 + 2], gst[8 * c2 + 3]);
-      v.z = pack_bf16(gst[8 * c2 + 4], gst[8 * c2 + 5]);
-      v.w = pack_bf16(gst[8 * c2 + 6], gst[8 * c2 + 7]);
+      v.x = pack_bf16(scale * gst[8 * c2 + 0], scale * gst[8 * c2 + 1]);
+      v.y = pack_bf16(scale * gst[8 * c2 + 2], scale * gst[8 * c2 + 3]);
+      v.z = pack_bf16(scale * gst[8 * c2 + 4], scale * gst[8 * c2 + 5]);
+      v.w = pack_bf16(scale * gst[8 * c2 + 6], scale * gst[8 * c2 + 7]);
       *reinterpret_cast<uint4*>(sm + C::G_OFF + sw128_off(n, (CW / 8) * cq + c2)) = v;
     }
   };
-  if (MODE == MODE_FULL) store_state_bf16();
 
   // MODE_STATE summaries (pair k = n / 2): log-decay in log2 units, and the
   // angle in fp64 (thousands of radians over a long segment), stored mod 2 pi
@@ -339,8 +359,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   // Chunk prologue: gates, the chunk-local log-decay prefix Lam_t (log2
   // units) and the cumulative angles.  Leaves the angle increments `ang` and
   // the slot prefix `phi` of this thread's rotation tokens in registers,
-  // gamma, delta, Lam, w, F and the chunk-end angles in shared memory, and
-  // the chunk's total decay in `l2end`.  Needs only theta and the gates, so it
+  // gamma, delta, Lam, u, the diagonal factor and the chunk-end angles in
+  // shared memory, and the chunk's total decay in `l2end`.  Needs only theta and the gates, so it
   // runs while the chunk's B, C and x are still in flight.
   float2 ang[TQ][2];
   float phi[4];
@@ -418,15 +438,18 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       for (int j = 0; j < 4; ++j) phi[j] = 0.f;
     }
     l2end = s_lg[nt - 1];
-    // The mask's decay is taken from per-token factors around the chunk's mid
-    // decay, exp(Lam_t - Lam_s) = E_t * F_s, while the chunk's total decay keeps
-    // both factors inside fp32 (|Lam_end| < 160); else entry by entry.
-    const float l2ref = 0.5f * l2end;
-    const bool fac_ok = l2end > -230.f;
+    // Row scale of Bh: exp(ref - Lam_s) delta_s in the factored form,
+    // delta_s in the plain one; a state-only pass has no scores, so its Bh
+    // carries the chunk-state weights exp(Lam_end - Lam_s) delta_s directly
+    // (a weight that underflows belongs to a negligible term).
     if (tid < Q) {
-      const float lg = s_lg[tid];
-      s_w[tid] = (tid < nt) ? ex2(l2end - lg) * s_del[tid] : 0.f;
-      s_F[tid] = fac_ok ? ex2(l2ref - lg) * s_del[tid] : 0.f;
+      const float lg = s_lg[tid], del = s_del[tid];
+      float u;
+      if (MODE == MODE_STATE) u = ex2(l2end - lg) * del;
+      else if (l2end > kPlainL2) u = ex2(0.5f * l2end - lg) * del;
+      else u = del;
+      s_u[tid] = (tid < nt) ? u : 0.f;
+      s_d[tid] = (tid < nt && del > 0.f) ? s_gam[tid] / del : 0.f;
     } else if (tid < Q + kPairs) {  // cos, sin of the chunk-end angles (state update)
       float sn, cs;
       sincosf(s_phe[tid - Q], &sn, &cs);
@@ -451,11 +474,11 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     const int64_t c0 = c * Q;
     const int nt = (int)min((int64_t)Q, L - c0);
     const bool slot_live = tq < SLOTS;
-    const float l2ref = 0.5f * l2end;
-    const bool fac_ok = l2end > -230.f;
+    const float l2ref = 0.5f * l2end;  // the factored form's reference (log2 units)
+    const bool plain = MODE == MODE_FULL && l2end <= kPlainL2;  // chunk-uniform
 
     load_gates(c + 1);  // consumed by the next chunk's prologue, at the end of this one
-    // the last chunk's staged y must be read before w*x reuses its tile
+    // the last chunk's staged y must be read before the staging block is reused
     if (MODE == MODE_FULL && tid == 0) bulk_wait_read0();
     const bool okm = (tid == 0) ? wait_bar(s_tbM, tphM, a.status) : true;
     if (okm && tid == 0) { tpendM = false; tphM ^= 1; }  // on a timeout the phase stays
@@ -464,7 +487,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     // theta buffer takes the next chunk's
     prefetch_early(c + 1);
 
-    // ---- operands: Bt (and Ct) rotated by -Phi_t in place (16-byte pieces) -----
+    // ---- operands: Bh = u Bt (and Ct) rotated by -Phi_t in place (16-byte pieces)
     if (slot_live) {
       const uint32_t kboff = (uint32_t)(kg >> 3) * C::OPB;
       const uint32_t chk = (uint32_t)(kg & 7);
@@ -478,11 +501,18 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
 #pragma unroll
         for (int j = 0; j < 4; ++j) __sincosf(reduce_2pi(phi[j]), &sn[j], &cs[j]);
         // two pairs at a time as (even elements, odd elements) fp32x2 vectors:
-        // (b0, b1) -> (c b0 + s b1, c b1 - s b0) for each pair
+        // (b0, b1) -> (c b0 + s b1, c b1 - s b0) for each pair; B's rows also
+        // take their scale u_t
+        const float us = live_t ? s_u[t] : 0.f;
         const float2 c2[2] = {make_float2(cs[0], cs[1]), make_float2(cs[2], cs[3])};
         const float2 s2[2] = {make_float2(sn[0], sn[1]), make_float2(sn[2], sn[3])};
         const float2 n2[2] = {make_float2(-sn[0], -sn[1]), make_float2(-sn[2], -sn[3])};
-        auto rot4 = [&](const uint4 in, uint32_t (&o)[4]) {
+        const float2 u2 = make_float2(us, us);
+        const float2 cb2[2] = {fmul2(u2, c2[0]), fmul2(u2, c2[1])};
+        const float2 sb2[2] = {fmul2(u2, s2[0]), fmul2(u2, s2[1])};
+        const float2 nb2[2] = {fmul2(u2, n2[0]), fmul2(u2, n2[1])};
+        auto rot4 = [&](const uint4 in, uint32_t (&o)[4], const float2 (&cv)[2],
+                        const float2 (&sv)[2], const float2 (&nv)[2]) {
           const uint32_t iw[4] = {in.x, in.y, in.z, in.w};
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
@@ -490,8 +520,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
                                          __uint_as_float(iw[2 * q + 1] << 16));
             const float2 d = make_float2(__uint_as_float(iw[2 * q] & 0xffff0000u),
                                          __uint_as_float(iw[2 * q + 1] & 0xffff0000u));
-            const float2 oe = ffma2(c2[q], e, fmul2(s2[q], d));
-            const float2 od = ffma2(c2[q], d, fmul2(n2[q], e));
+            const float2 oe = ffma2(cv[q], e, fmul2(sv[q], d));
+            const float2 od = ffma2(cv[q], d, fmul2(nv[q], e));
             o[2 * q] = pack_bf16(oe.x, od.x);
             o[2 * q + 1] = pack_bf16(oe.y, od.y);
           }
@@ -504,8 +534,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
           uint4 rc = make_uint4(0, 0, 0, 0);
           if (MODE == MODE_FULL) rc = *reinterpret_cast<const uint4*>(sm + C::C_OFF + off);
           if (!live_t) { rb = make_uint4(0, 0, 0, 0); rc = make_uint4(0, 0, 0, 0); }
-          rot4(rb, ob);
-          if (MODE == MODE_FULL) rot4(rc, oc);
+          rot4(rb, ob, cb2, sb2, nb2);
+          if (MODE == MODE_FULL) rot4(rc, oc, c2, s2, n2);
           *reinterpret_cast<uint4*>(sm + C::B_OFF + off) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
           if (MODE == MODE_FULL)
             *reinterpret_cast<uint4*>(sm + C::C_OFF + off) = make_uint4(oc[0], oc[1], oc[2], oc[3]);
@@ -513,31 +543,18 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       }
     }
 
-    // ---- w * x (chunk-state operand) from the x tile ---------------------------
-    constexpr int PER = M * 8 / NTH;
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      const int q = tid + j * NTH;
-      const int row = q >> 3, chq = q & 7, t = row / R;
-      const float w = s_w[t];
-      const uint4 xq = *reinterpret_cast<const uint4*>(sm + C::X_OFF + sw128_off(row, chq));
-      const uint32_t iv[4] = {xq.x, xq.y, xq.z, xq.w};
-      uint32_t ov[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = fmul2(make_float2(w, w), make_float2(__uint_as_float(iv[e] << 16),
-                                                              __uint_as_float(iv[e] & 0xffff0000u)));
-        ov[e] = pack_bf16(f.x, f.y);
-      }
-      *reinterpret_cast<uint4*>(sm + C::XW_OFF + sw128_off(row, chq)) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
-    }
+    // ---- the MMA4 operand: the chunk-start state, times exp(ref) when factored
+    // (every MMA of the previous chunk is complete, so its tile is free)
+    if (MODE == MODE_FULL) store_state_bf16(plain ? 1.f : ex2(l2ref));
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
     // ---- MMA3 (chunk state) and MMA4 (Ct G), then MMA1 (scores) ----------------
-    auto issue_mma4 = [&](int mt) {  // y2 = Ct G for tile mt, one thread
+    // MMA4: Ct G' for tile mt into TMEM column `col` (one thread); `acc`: add
+    // to what the column holds
+    auto issue_mma4 = [&](int mt, int col, bool acc) {
       const uint32_t id4 = idesc_bf16(MT, kP, 0, 1);
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb)
@@ -545,33 +562,78 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
           for (int k4 = 0; k4 < 4; ++k4) {
             const uint64_t ad = dadd(dC, kb * C::OPB + mt * MT * 128 + k4 * 32);
             const uint64_t bd = dadd(dG, (kb * 4 + k4) * 2048);
-            mma_bf16_ss(tm + C::y2_col(mt), ad, bd, id4, (kb | k4) != 0);
+            mma_bf16_ss(tm + col, ad, bd, id4, acc || (kb | k4) != 0);
           }
     };
-    if (tid == 0) {
+    auto issue_mma3 = [&]() {  // Sc' = Bh^T x (one thread)
       const uint32_t id3 = idesc_bf16(kN, kP, 1, 1);
 #pragma unroll
       for (int ks = 0; ks < M / 16; ++ks) {
         const uint64_t ad = dadd(dBmn, ks * 2048);
-        const uint64_t bd = dadd(dXW, ks * 2048);
+        const uint64_t bd = dadd(dX, ks * 2048);
         mma_bf16_ss(tm + C::SC_COL, ad, bd, id3, ks != 0);
       }
-      if (MODE == MODE_FULL && C::EARLY4) issue_mma4(0);
-      mma_commit(s_bar);
-      if (MODE == MODE_FULL) {
+    };
+    auto issue_mma1 = [&]() {  // S' = Ct Bh^T per tile, each on its own barrier (one thread)
 #pragma unroll
-        for (int mt = 0; mt < NT; ++mt) {
-          const uint32_t id = idesc_bf16(MT, (mt + 1) * MT, 0, 0);
+      for (int mt = 0; mt < NT; ++mt) {
+        const uint32_t id = idesc_bf16(MT, (mt + 1) * MT, 0, 0);
 #pragma unroll
-          for (int kb = 0; kb < 2; ++kb)
+        for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-              const uint64_t ad = dadd(dC, kb * C::OPB + mt * MT * 128 + k4 * 32);
-              const uint64_t bd = dadd(dB, kb * C::OPB + k4 * 32);
-              mma_bf16_ss(tm + C::s_col(mt), ad, bd, id, (kb | k4) != 0);
-            }
-          mma_commit(mt == 0 ? s_bar1 : s_bar1b);  // each tile's scores on their own barrier
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const uint64_t ad = dadd(dC, kb * C::OPB + mt * MT * 128 + k4 * 32);
+            const uint64_t bd = dadd(dB, kb * C::OPB + k4 * 32);
+            mma_bf16_ss(tm + C::s_col(mt), ad, bd, id, (kb | k4) != 0);
+          }
+        mma_commit(mt == 0 ? s_bar1 : s_bar1b);
+      }
+    };
+    if (tid == 0) {
+      if (MODE == MODE_STATE) {
+        issue_mma3();
+        mma_commit(s_bar);
+      } else if (!plain) {  // MMA3 (and MMA4 for one-tile chunks) first, then the scores
+        issue_mma3();
+        if (C::EARLY4) issue_mma4(0, C::acc_col(0), false);
+        mma_commit(s_bar);
+        issue_mma1();
+      } else {  // plain form: the scores read Bh before it is rescaled for MMA3
+        if (C::EARLY4) issue_mma4(0, C::y2_col(0), false);
+        issue_mma1();
+      }
+    }
+    if (plain) {  // chunk-uniform branch
+      bool okp = true;
+      if (tid == 0) {  // both score tiles done (waited again, same phase, below)
+        okp = wait_bar(s_bar1, phase1, a.status);
+        if (okp && NT == 2) okp = wait_bar(s_bar1b, phase1b, a.status);
+      }
+      if (__syncthreads_or(!okp)) { aborted = true; break; }
+      // Bh_s <- exp(Lam_end - Lam_s) Bh_s = w_s Bt_s, the chunk-state weights
+      for (int q = tid; q < M * 16; q += NTH) {
+        const int row = q >> 4, t = row / R;
+        if (t >= nt) continue;  // rows past the end are zero
+        const float f = ex2(l2end - s_lg[t]);
+        uint8_t* pq = sm + C::B_OFF + ((q >> 3) & 1) * C::OPB + sw128_off(row, q & 7);
+        const uint4 v = *reinterpret_cast<const uint4*>(pq);
+        const uint32_t iv[4] = {v.x, v.y, v.z, v.w};
+        uint32_t ov[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 g = fmul2(make_float2(f, f), make_float2(__uint_as_float(iv[e] << 16),
+                                                                __uint_as_float(iv[e] & 0xffff0000u)));
+          ov[e] = pack_bf16(g.x, g.y);
         }
+        *reinterpret_cast<uint4*>(pq) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (tid == 0) {
+        issue_mma3();
+        mma_commit(s_bar);
       }
     }
     const bool ok3 = (tid == 0) ? wait_bar(s_bar, phase, a.status) : true;
@@ -581,11 +643,13 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     if (MODE == MODE_STATE) prefetch_bx(c + 1);  // B and x are free once MMA3 is done
 
     // ---- state update G <- Rot(Phi_end) (exp(Lam_end) G + Sc), under MMA1 -------
+    //      (Sc = exp(Lam_end - ref) Sc' when factored)
     {
       const float phe = s_phe[n >> 1];
       const float2 pcs = s_pcs[n >> 1];
       const float cs = pcs.x, sn = pcs.y;
       const float el = ex2(l2end);
+      const float sc = (MODE == MODE_FULL && !plain) ? ex2(l2end - l2ref) : 1.f;
       const float ss = (n & 1) ? sn : -sn;  // even row: c v - s o; odd row: c v + s o
 #pragma unroll
       for (int pc = 0; pc < CW / 16; ++pc) {
@@ -596,7 +660,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         for (int p = 0; p < 16; p += 2) {
           const int pp = 16 * pc + p;
           const float2 v = ffma2(make_float2(el, el), make_float2(gst[pp], gst[pp + 1]),
-                                 make_float2(__uint_as_float(sv[p]), __uint_as_float(sv[p + 1])));
+                                 fmul2(make_float2(sc, sc), make_float2(__uint_as_float(sv[p]),
+                                                                        __uint_as_float(sv[p + 1]))));
           const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, v.x, 1),
                                        __shfl_xor_sync(0xffffffffu, v.y, 1));
           const float2 w = ffma2(make_float2(cs, cs), v, fmul2(make_float2(ss, ss), o));
@@ -611,7 +676,6 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     }
 
     if (MODE == MODE_FULL) {
-      if (C::EARLY4) store_state_bf16();  // MMA4 has read the previous state
       const bool ok1 = (tid == 0) ? wait_bar(s_bar1, phase1, a.status) : true;
       phase1 ^= 1;
       if (__syncthreads_or(!ok1)) { aborted = true; break; }
@@ -619,7 +683,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       if (C::EARLY4) prefetch_c(c + 1);  // MMA1 and MMA4 have read Ct
 
       // ---- per score tile: mask into P (bf16, K-major), then its MMA2 (P x) -----
-      //   P[(t,r),(s,r')] = S * (s < t ? exp(Lam_t - Lam_s) delta_s : s == t ? gamma_t : 0)
+      //   factored: P'[(t,r),(s,r')] = S' * (s < t ? 1 : s == t ? gamma_t / delta_t : 0)
+      //   plain:    P [(t,r),(s,r')] = S' * (s < t ? exp(Lam_t - Lam_s) : s == t ? gamma_t / delta_t : 0)
       // With two tiles, tile 1's mask runs while tile 0's MMA2 and MMA4 run.
 #pragma unroll
       for (int mt = 0; mt < NT; ++mt) {
@@ -638,34 +703,30 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         const bool trow = t < nt;
         const int t_hi = (mt * MT + rho0 + ((MT == 64) ? 15 : 31)) / R;  // the warp's last token
         const float lgt = trow ? s_lg[t] : 0.f;
-        const float et = (trow && fac_ok) ? ex2(lgt - l2ref) : 0.f;
-        const float gmt = trow ? s_gam[t] : 0.f;
+        const float dgt = trow ? s_d[t] : 0.f;
         const int cpt = (mt + 1) * MT / CQN;  // columns per thread, a multiple of 32
         static_assert((MT / CQN) % 32 == 0, "mask columns per thread");
         // 16 masked columns (16 / R tokens from s0) of v, packed to bf16
         auto mask16 = [&](const uint32_t* v, int s0, uint32_t* pk) {
+          if (!plain && s0 + 16 / R - 1 < t) {  // wholly below the diagonal: S' as it is
+#pragma unroll
+            for (int j = 0; j < 16; j += 2)
+              pk[j / 2] = pack_bf16(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+            return;
+          }
           float mk[16 / R];
 #pragma unroll
           for (int q4 = 0; q4 < 16 / R / 4; ++q4) {
             const int sb = s0 + 4 * q4;
-            float f[4];
-            if (fac_ok) {
-              const float4 fw = *reinterpret_cast<const float4*>(s_F + sb);
-              f[0] = et * fw.x; f[1] = et * fw.y; f[2] = et * fw.z; f[3] = et * fw.w;
-            } else {
+            float f[4] = {1.f, 1.f, 1.f, 1.f};
+            if (plain) {
               const float4 l4 = *reinterpret_cast<const float4*>(s_lg + sb);
-              const float4 d4 = *reinterpret_cast<const float4*>(s_del + sb);
-              f[0] = ex2(lgt - l4.x) * d4.x; f[1] = ex2(lgt - l4.y) * d4.y;
-              f[2] = ex2(lgt - l4.z) * d4.z; f[3] = ex2(lgt - l4.w) * d4.w;
+              f[0] = ex2(lgt - l4.x); f[1] = ex2(lgt - l4.y);
+              f[2] = ex2(lgt - l4.z); f[3] = ex2(lgt - l4.w);
             }
-            if (sb + 3 < t) {  // wholly below the diagonal
 #pragma unroll
-              for (int e = 0; e < 4; ++e) mk[4 * q4 + e] = f[e];
-            } else {
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                mk[4 * q4 + e] = sb + e < t ? f[e] : (sb + e == t ? gmt : 0.f);
-            }
+            for (int e = 0; e < 4; ++e)
+              mk[4 * q4 + e] = sb + e < t ? f[e] : (sb + e == t ? dgt : 0.f);
           }
 #pragma unroll
           for (int j = 0; j < 16; j += 2) {
@@ -721,15 +782,23 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         if (tid == 0) {  // MMA2 for this tile (and MMA4 for two-tile chunks)
           const uint32_t id2 = idesc_bf16(MT, kP, 0, 1);
           const int kblocks = (mt + 1) * MT / 64;
+          // factored: one accumulator, Ct G' (MMA4) first; plain: P x alone
+          int col = C::y_col(mt);
+          bool acc = false;
+          if (!plain) {
+            col = C::acc_col(mt);
+            if (!C::EARLY4) issue_mma4(mt, col, false);
+            acc = true;
+          }
           for (int kb = 0; kb < kblocks; ++kb)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
-              const uint64_t ad = dadd(mt == 0 && NT == 2 ? dadd(dC, C::XW_OFF - C::C_OFF) : dB,
-                                       kb * MT * 128 + k4 * 32);  // P over w*x or Bt
+              const uint64_t ad = dadd(mt == 0 && NT == 2 ? dadd(dC, C::ST_OFF - C::C_OFF) : dB,
+                                       kb * MT * 128 + k4 * 32);  // P in the staging block or over Bh
               const uint64_t bd = dadd(dX, (kb * 4 + k4) * 2048);
-              mma_bf16_ss(tm + C::y_col(mt), ad, bd, id2, (kb | k4) != 0);
+              mma_bf16_ss(tm + col, ad, bd, id2, acc || (kb | k4) != 0);
             }
-          if (!C::EARLY4) issue_mma4(mt);
+          if (plain && !C::EARLY4) issue_mma4(mt, C::y2_col(mt), false);
           if (mt == NT - 1) mma_commit(s_bar);
         }
       }
@@ -738,13 +807,11 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       phase ^= 1;
       if (__syncthreads_or(!ok2)) { aborted = true; break; }
       tc_fence_after();
-      prefetch_bx(c + 1);  // MMA2 has read P (over Bt) and x
-      if (!C::EARLY4) {    // MMA4 has read Ct and the previous state
-        prefetch_c(c + 1);
-        store_state_bf16();
-      }
+      prefetch_bx(c + 1);                 // MMA2 has read P (over Bh) and x
+      if (!C::EARLY4) prefetch_c(c + 1);  // MMA4 has read Ct
 
-      // ---- epilogue: y = P x + exp(Lam_t) Ct G, staged in the w*x block --------
+      // ---- epilogue, staged in the staging block: y = exp(Lam_t - ref) Y'
+      //      (factored), y = Y + exp(Lam_t) Y2 (plain) --------------------------
 #pragma unroll
       for (int mt = 0; mt < NT; ++mt) {
         // 64-row tiles: both half-warps take the warp's 16 rows, each half
@@ -752,7 +819,9 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         const int rho = (MT == 64) ? 16 * qd + (lane & 15) : 32 * qd + lane;
         const int i = mt * MT + rho;  // row (t, r) of the chunk
         const int t = i / R;
-        const float el = (t < nt) ? ex2(s_lg[t]) : 0.f;
+        // plain: (1, exp(Lam_t)) on (Y, Y2); factored: exp(Lam_t - ref) on Y'
+        const float el = (t < nt) ? ex2(plain ? s_lg[t] : s_lg[t] - l2ref) : 0.f;
+        const int ycol = plain ? C::y_col(mt) : C::acc_col(mt);
         constexpr int NPC = (MT == 64) ? CW / 32 : CW / 16;  // 16-column pieces per thread
         static_assert(MT != 64 || CW % 32 == 0, "64-row tiles: 32 columns per thread group");
 #pragma unroll
@@ -761,12 +830,12 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
           int col;  // this thread's first column
           if (MT == 64) {
             col = CW * cq + 32 * pc + 16 * (lane >> 4);
-            tmem_ld16x2<16>(tm + lane_base + C::y_col(mt) + CW * cq + 32 * pc, yv);
-            tmem_ld16x2<16>(tm + lane_base + C::y2_col(mt) + CW * cq + 32 * pc, zv);
+            tmem_ld16x2<16>(tm + lane_base + ycol + CW * cq + 32 * pc, yv);
+            if (plain) tmem_ld16x2<16>(tm + lane_base + C::y2_col(mt) + CW * cq + 32 * pc, zv);
           } else {
             col = CW * cq + 16 * pc;
-            tmem_ld16(tm + lane_base + C::y_col(mt) + col, yv);
-            tmem_ld16(tm + lane_base + C::y2_col(mt) + col, zv);
+            tmem_ld16(tm + lane_base + ycol + col, yv);
+            if (plain) tmem_ld16(tm + lane_base + C::y2_col(mt) + col, zv);
           }
           tmem_ld_wait();
           {
@@ -776,12 +845,14 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int j = q * 8 + 2 * e;
-                const float2 f = ffma2(make_float2(el, el),
-                                       make_float2(__uint_as_float(zv[j]), __uint_as_float(zv[j + 1])),
-                                       make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1])));
+                const float2 yy = make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1]));
+                const float2 f =
+                    plain ? ffma2(make_float2(el, el),
+                                  make_float2(__uint_as_float(zv[j]), __uint_as_float(zv[j + 1])), yy)
+                          : fmul2(make_float2(el, el), yy);
                 w4[e] = pack_bf16(f.x, f.y);
               }
-              *reinterpret_cast<uint4*>(sm + C::XW_OFF + sw128_off(i, col / 8 + q)) =
+              *reinterpret_cast<uint4*>(sm + C::ST_OFF + sw128_off(i, col / 8 + q)) =
                   make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
           }
@@ -795,12 +866,12 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     if (MODE == MODE_FULL) {
       if (!a.cu_seqlens) {  // y of this chunk: one bulk tensor store, clipped at the sequence end
         if (tid == 0) {
-          tma_store_4d(&maps.y, sm + C::XW_OFF, 0, (int)(h * R), (int)c0, (int)b);
+          tma_store_4d(&maps.y, sm + C::ST_OFF, 0, (int)(h * R), (int)c0, (int)b);
           bulk_commit();
         }
       } else if (nt == Q) {  // packed batch: a whole chunk by the bulk store
         if (tid == 0) {
-          tma_store_4d(&maps.y, sm + C::XW_OFF, 0, (int)(h * R), (int)(tokb + c0), 0);
+          tma_store_4d(&maps.y, sm + C::ST_OFF, 0, (int)(h * R), (int)(tokb + c0), 0);
           bulk_commit();
         }
       } else {  // packed batch, a sequence's last partial chunk: the next sequence's rows
@@ -808,7 +879,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         const int pieces = nt * R * 8;
         for (int e = tid; e < pieces; e += NTH) {
           const int i = e >> 3, j = e & 7, t = i / R, r = i % R;
-          const uint4 v = *reinterpret_cast<const uint4*>(sm + C::XW_OFF + sw128_off(i, j));
+          const uint4 v = *reinterpret_cast<const uint4*>(sm + C::ST_OFF + sw128_off(i, j));
           __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.y) +
                                (((tokb + c0 + t) * H + h) * R + r) * kP + 8 * j;
           *reinterpret_cast<uint4*>(dst) = v;

@@ -148,6 +148,36 @@ def test_tc_tiles_segments_ragged(R, chunk, L, batch, H):
     check(compare_scan(inp, chunk, "bf16"), "bf16")
 
 
+@pytest.mark.parametrize("R,chunk", [(1, 64), (2, 32), (2, 64), (4, 64), (4, 32)])
+def test_tc_large_decay_chunks(R, chunk):
+    """Every other chunk decays by hundreds of nats (dt ten times larger and
+    A = -16 there), so the tensor-core path does those chunks in its plain
+    form and the slow-decay chunks between in its factored form; few chains,
+    so segments and the state-only pass are used too; ragged tail."""
+    w = I.Workload(I.Shape(2, 700, 4, 64, 128, R, 1, chunk, "bf16"), decay="slow",
+                   with_h0=True, with_prev=True)
+    inp = I.make_scan_inputs(w, seed=7300 + 10 * R + chunk)
+    odd = ((torch.arange(700) // chunk) % 2 == 1)[None, :, None]
+    inp["dt"] = torch.where(odd, inp["dt"] * 10.0, inp["dt"]).contiguous()
+    inp["A"] = torch.where(odd, torch.full_like(inp["A"], -16.0), inp["A"]).contiguous()
+    lam_chunk = (inp["dt"] * inp["A"])[:, :chunk * (700 // chunk)].reshape(2, -1, chunk, 4).sum(2)
+    assert float(lam_chunk.min()) < -300.0 and float(lam_chunk.max()) > -5.0
+    check(compare_scan(inp, chunk, "bf16"), "bf16")
+
+
+@pytest.mark.parametrize("nats", [95.0, 105.0])
+@pytest.mark.parametrize("R", [1, 4])
+def test_tc_decay_at_the_form_switch(nats, R):
+    """Every chunk decays by the same total, just inside (95 nats: the
+    factored form, factors up to e^47.5) or just outside (105 nats: the plain
+    form) the switch between the two forms."""
+    w = I.Workload(I.Shape(2, 640, 4, 64, 128, R, 1, 64, "bf16"), with_h0=True, with_prev=True)
+    inp = I.make_scan_inputs(w, seed=7400 + R + int(nats))
+    inp["dt"] = torch.ones_like(inp["dt"])
+    inp["A"] = torch.full_like(inp["A"], -nats / 64.0)
+    check(compare_scan(inp, 64, "bf16"), "bf16")
+
+
 @pytest.mark.parametrize("R", [1, 4])
 def test_tc_groups_and_fast_decay(R):
     """G = H (per-head B, C, theta) and the workload's fast decay."""
