@@ -270,6 +270,69 @@ def prep_line(s, world, steps, warmup, flush, peaks, psrc):
             "roofline": roofline(0.0, byt, t, peaks, psrc)}
 
 
+def time_calls(fn, steps, warmup, flush):
+    """Mean device time of fn() over `steps` calls (CUDA events on the current
+    stream, L2 flushed before each timed call)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        fn()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    if m3.m3_stream_status() != 0:
+        raise RuntimeError("device status")
+    return sum(a.elapsed_time(b) * 1e-3 for a, b in ev) / steps
+
+
+def block_line(world, steps, warmup, flush, peaks, psrc):
+    """The block projections around the layer at the 1.5B-scale width
+    (D = 2048, H * P = 4096, G * N / 2 = 64 angle rates) on the SISO workload's
+    16384 tokens: the gate projection z = u W_z (m3_linear, tcgen05), the angle
+    projection theta = u W_theta (fp32 out), and the rank-4 MIMO up- and
+    down-projections with the output gate (HBM-bound)."""
+    T, D, HP, NTH, H, P, R = 8 * 2048, 2048, 4096, 64, 64, 64, 4
+    gen = torch.Generator(device="cuda").manual_seed(1041)
+    u = torch.randn((T, D), generator=gen, device="cuda").to(torch.bfloat16)
+    Wz = (torch.randn((HP, D), generator=gen, device="cuda") / D ** 0.5).to(torch.bfloat16)
+    Wt = (torch.randn((NTH, D), generator=gen, device="cuda") / D ** 0.5).to(torch.bfloat16)
+    z = torch.empty((T, HP), dtype=torch.bfloat16, device="cuda")
+    th = torch.empty((T, NTH), dtype=torch.float32, device="cuda")
+    x = torch.randn((T, H, P), generator=gen, device="cuda").to(torch.bfloat16)
+    w_up = torch.randn((H, R, P), generator=gen, device="cuda")
+    w_dn = torch.randn((H, R, P), generator=gen, device="cuda")
+    X = torch.empty((T, H, R, P), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((T, H, P), dtype=torch.bfloat16, device="cuda")
+    zz = z.view(T, H, P)
+    t_z = time_calls(lambda: m3.m3_linear(u, Wz, out=z), steps, warmup, flush)
+    t_t = time_calls(lambda: m3.m3_linear(u, Wt, out=th), steps, warmup, flush)
+    t_u = time_calls(lambda: m3.m3_mimo_up(x, w_up, X=X), steps, warmup, flush)
+    t_d = time_calls(lambda: m3.m3_mimo_down_gate(X, w_dn, zz, out=out), steps, warmup, flush)
+    barrier(world)
+    t_z, t_t, t_u, t_d = (max_over_ranks(v, world) for v in (t_z, t_t, t_u, t_d))
+    fz, bz = 2.0 * T * HP * D, 2.0 * (T * D + HP * D + T * HP)
+    ft, bt = 2.0 * T * NTH * D, 2.0 * (T * D + NTH * D) + 4.0 * T * NTH
+    bu = 2.0 * T * H * P * (1 + R) + 4.0 * H * R * P
+    bd = 2.0 * T * H * P * (R + 2) + 4.0 * H * R * P
+    return {
+        "workload": f"{T} tokens, D = {D}, H * P = {HP}, angle rates {NTH}, rank {R}, bf16",
+        "gate_projection": {"kernel": "gemm_tc_kernel (tcgen05, 128 x 256 tiles)",
+                            "us_per_call": round(t_z * 1e6, 2),
+                            "roofline": roofline(fz, bz, t_z, peaks, psrc)},
+        "angle_projection": {"kernel": "gemm_tc_kernel (tcgen05, 128 x 64 tiles), fp32 out",
+                             "us_per_call": round(t_t * 1e6, 2),
+                             "roofline": roofline(ft, bt, t_t, peaks, psrc)},
+        "mimo_up": {"us_per_call": round(t_u * 1e6, 2),
+                    "roofline": roofline(0.0, bu, t_u, peaks, psrc)},
+        "mimo_down_gate": {"us_per_call": round(t_d * 1e6, 2),
+                           "roofline": roofline(0.0, bd, t_d, peaks, psrc)},
+    }
+
+
 def decode_work(s: I.Shape):
     R, N, P = s.rank, s.dstate, s.headdim
     bh = s.batch * s.nheads
@@ -739,7 +802,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1024,
                     help="consecutive decode steps timed (each with its own token's inputs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode", "varlen", "bwd", "prep"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "varlen", "bwd", "prep", "block"],
+                    default=None,
                     help="run one part only (for profiling); prints its own line")
     ap.add_argument("--batch", type=int, default=None,
                     help="with --only: override the workload's batch (small profiling cases)")
@@ -781,6 +845,11 @@ def main():
         flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
         print(json.dumps({"only": "prep", **prep_line(s, 1, args.steps, args.warmup, flush, peaks,
                                                       psrc)}))
+        return
+    if args.only == "block":
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        print(json.dumps({"only": "block", **block_line(1, args.steps, args.warmup, flush, peaks,
+                                                        psrc)}))
         return
     if args.only == "bwd":
         inp = I.make_scan_inputs(I.Workload(s), seed=1001, device="cuda")
@@ -876,6 +945,8 @@ def main():
                                       device="cuda")
     line["backward"] = bwd_line(siso_inp, ss, world, 3, args.warmup, flush, peaks)
     del siso_inp
+    # the block projections around the layer (tensor-core GEMMs, MIMO up / down, gate)
+    line["block"] = block_line(world, 10, args.warmup, flush, peaks, psrc)
     ms = I.MIMO_PREFILL.shape
     mimo_inp = I.make_scan_inputs(I.MIMO_PREFILL, seed=SEEDS["mimo_prefill"] + 7919 * rank,
                                   device="cuda")

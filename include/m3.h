@@ -21,7 +21,8 @@
  * form m3_scan_fwd_varlen; m3_scan_fwd_noalloc without a workspace argument;
  * m3_scan_state for the final state only), the single-token decode step
  * (m3_decode_step), the backward pass (m3_scan_bwd, m3_scan_bwd_varlen), the
- * B / C projection prep (m3_bc_prep), the pieces of a sequence split across
+ * B / C projection prep (m3_bc_prep), the block projections around the
+ * layer (m3_linear, m3_mimo_up, m3_mimo_down_gate), the pieces of a sequence split across
  * ranks (m3_segment_totals, m3_state_fold), and sizing, planning and status
  * (m3_*_workspace_size, m3_scan_plan, m3_check_shape, m3_stream_status,
  * m3_status_string, m3_version).
@@ -304,6 +305,54 @@ M3_API int m3_scan_bwd_varlen(const m3_shape* shape, const int32_t* cu_seqlens,
 M3_API int m3_bc_prep(const m3_shape* shape, const void* B_raw, const void* C_raw,
                       const float* B_weight, const float* B_bias, const float* C_weight,
                       const float* C_bias, float eps, void* B, void* C, m3_stream_t stream);
+
+/* ---- block projections around the layer ----------------------------------------
+ * The dense maps of a Mamba-3 block that feed the layer and read its output
+ * (PaperWeekly page section 2.4 and Figure 4: the input projections, the
+ * data-dependent RoPE angles theta, the MIMO projection; the output gate).
+ * The pages name these steps but print no formula for them; the readings are
+ * the plainest ones the rest supports:
+ *   - every projection is a linear map of the token's features,
+ *     out = A W^T (+ bias), with the angle rates theta one such projection
+ *     (no nonlinearity);
+ *   - the MIMO up-projection gives each rank r of head h a learned copy of
+ *     the head's input, X[r][p] = x[p] w_up[h][r][p], and the down-projection
+ *     sums the ranks back, y[p] = sum_r Y[r][p] w_down[h][r][p];
+ *   - the output gate multiplies by silu(z) = z / (1 + exp(-z)), z a
+ *     projection of the block input (the gate of the Mamba block family).
+ *
+ * m3_linear: out[M][N] = A[M][K] W[N][K]^T (+ bias[N]) on the tensor cores
+ * (tcgen05, bf16 operands, fp32 accumulation).
+ *   A          [M][K] bf16 (one token per row); W [N][K] bf16 (a weight in
+ *              the [out][in] layout); bias [N] fp32 or NULL.
+ *   out        [M][N], out_dtype M3_BF16 (rounded to nearest even) or M3_F32.
+ *   M >= 0; N >= 1; K >= 8 with K % 8 == 0; N % 8 == 0 (bf16 out) or
+ *   N % 4 == 0 (fp32 out); M, N < 2^31 - 256.
+ *   A, W, out 16-byte aligned, bias 4-byte aligned; out must not overlap A,
+ *   W or bias.  Errors as elsewhere; a device-side wait that gives up is
+ *   reported by m3_stream_status (M3_ERR_TIMEOUT). */
+M3_API int m3_linear(int64_t M, int64_t N, int64_t K, const void* A, const void* W,
+                     const float* bias, void* out, int32_t out_dtype, m3_stream_t stream);
+
+/* MIMO up-projection: X[t][h][r][p] = x[t][h][p] * w_up[h][r][p].
+ *   shape      batch, seqlen (tokens = batch * seqlen), nheads, rank,
+ *              headdim, io_dtype; the other fields are checked as usual but
+ *              not used.
+ *   x          [tokens][H][P] io dtype;  w_up [H][R][P] fp32;
+ *   X          [tokens][H][R][P] io dtype (the layer's x).
+ *   x, X 16-byte aligned, w_up 4-byte aligned; P % 8 == 0 for bf16 io. */
+M3_API int m3_mimo_up(const m3_shape* shape, const void* x, const float* w_up, void* X,
+                      m3_stream_t stream);
+
+/* MIMO down-projection and output gate:
+ *   out[t][h][p] = (sum_r Y[t][h][r][p] * w_down[h][r][p]) * silu(z[t][h][p]),
+ * fp32 arithmetic, rounded to the io dtype.
+ *   Y          [tokens][H][R][P] io dtype (the layer's y);  w_down [H][R][P] fp32;
+ *   z          [tokens][H][P] io dtype, or NULL for no gate;
+ *   out        [tokens][H][P] io dtype.
+ *   Shape, alignment and size rules as m3_mimo_up. */
+M3_API int m3_mimo_down_gate(const m3_shape* shape, const void* Y, const float* w_down,
+                             const void* z, void* out, m3_stream_t stream);
 
 /* ---- packed variable-length batch -------------------------------------------
  * Several sequences of different lengths in one call, stored back to back

@@ -389,6 +389,82 @@ M3_API int m3_bc_prep(const m3_shape* s, const void* B_raw, const void* C_raw,
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 
+M3_API int m3_linear(int64_t M, int64_t N, int64_t K, const void* A, const void* W,
+                     const float* bias, void* out, int32_t out_dtype, m3_stream_t stream) {
+  if (out_dtype != M3_BF16 && out_dtype != M3_F32) return M3_ERR_INVALID_ARGUMENT;
+  const bool f32 = out_dtype == M3_F32;
+  if (M < 0 || N < 1 || K < 8) return M3_ERR_INVALID_ARGUMENT;
+  if (K % 8 != 0 || N % (f32 ? 4 : 8) != 0) return M3_ERR_UNSUPPORTED;
+  if (M >= ((int64_t)1 << 31) - 256 || N >= ((int64_t)1 << 31) - 256) return M3_ERR_UNSUPPORTED;
+  if (M == 0) return M3_OK;
+  if (!A || !W || !out) return M3_ERR_INVALID_ARGUMENT;
+  if (!aligned(A, 16) || !aligned(W, 16) || !aligned(out, 16) || (bias && !aligned(bias, 4)))
+    return M3_ERR_ALIGNMENT;
+  const size_t nout = (size_t)M * (size_t)N * (f32 ? 4 : 2);
+  auto overlaps = [&](const void* p, size_t n) {
+    const char* c = static_cast<const char*>(p);
+    const char* o = static_cast<const char*>(out);
+    return p && c < o + nout && o < c + n;
+  };
+  if (overlaps(A, (size_t)M * K * 2) || overlaps(W, (size_t)N * K * 2) ||
+      overlaps(bias, (size_t)N * 4))
+    return M3_ERR_INVALID_ARGUMENT;
+  int* status = nullptr;
+  if (status_word(&status) != M3_OK) return M3_ERR_CUDA;
+  cudaError_t e = gemm_launch(M, N, K, A, W, bias, out, f32, status,
+                              reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+namespace {
+int mimo_check(const m3_shape* s, const void* in, const float* w, const void* extra,
+               const void* out) {
+  int st = check_common(s);
+  if (st != M3_OK) return st;
+  const bool bf16 = s->io_dtype == M3_BF16;
+  if (s->headdim % (bf16 ? 8 : 4) != 0) return M3_ERR_UNSUPPORTED;
+  if (s->batch * s->seqlen == 0) return M3_OK;
+  if (!in || !w || !out) return M3_ERR_INVALID_ARGUMENT;
+  if (!aligned(in, 16) || !aligned(out, 16) || (extra && !aligned(extra, 16)) || !aligned(w, 4))
+    return M3_ERR_ALIGNMENT;
+  return M3_OK;
+}
+}  // namespace
+
+M3_API int m3_mimo_up(const m3_shape* s, const void* x, const float* w_up, void* X,
+                      m3_stream_t stream) {
+  int st = mimo_check(s, x, w_up, nullptr, X);
+  if (st != M3_OK || s->batch * s->seqlen == 0) return st;
+  const size_t es = s->io_dtype == M3_BF16 ? 2 : 4;
+  const int64_t T = s->batch * s->seqlen;
+  const char* xi = static_cast<const char*>(x);
+  const char* xo = static_cast<const char*>(X);
+  const size_t nin = es * T * s->nheads * s->headdim, nout = nin * s->rank;
+  if (xi < xo + nout && xo < xi + nin) return M3_ERR_INVALID_ARGUMENT;  // no overlap
+  cudaError_t e = mimo_up_launch(T, s->nheads, s->rank, s->headdim, s->io_dtype == M3_BF16, x,
+                                 w_up, X, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+M3_API int m3_mimo_down_gate(const m3_shape* s, const void* Y, const float* w_down,
+                             const void* z, void* out, m3_stream_t stream) {
+  int st = mimo_check(s, Y, w_down, z, out);
+  if (st != M3_OK || s->batch * s->seqlen == 0) return st;
+  const size_t es = s->io_dtype == M3_BF16 ? 2 : 4;
+  const int64_t T = s->batch * s->seqlen;
+  const size_t nout = es * T * s->nheads * s->headdim, nY = nout * s->rank;
+  auto overlaps = [&](const void* p, size_t n) {
+    const char* c = static_cast<const char*>(p);
+    const char* o = static_cast<const char*>(out);
+    return p && c < o + nout && o < c + n;
+  };
+  if (overlaps(Y, nY) || overlaps(z, nout)) return M3_ERR_INVALID_ARGUMENT;
+  cudaError_t e = mimo_down_gate_launch(T, s->nheads, s->rank, s->headdim,
+                                        s->io_dtype == M3_BF16, Y, w_down, z, out,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
 M3_API int m3_scan_state(const m3_shape* s, const void* x, const float* dt, const float* A,
                          const float* lam, const float* theta, const void* B, const void* C,
                          const float* h0, const void* B_prev, const void* x_prev,

@@ -136,6 +136,16 @@ cudaError_t bc_prep_launch(int64_t tokens, int64_t N, int64_t gr, bool bf16, con
                            const void* Craw, const float* wB, const float* bB, const float* wC,
                            const float* bC, float eps, void* Bo, void* Co, cudaStream_t s);
 
+// Block projections: out = A W^T (+ bias) on the tensor cores; the MIMO up-
+// projection; the MIMO down-projection with the output gate.
+cudaError_t gemm_launch(int64_t M, int64_t N, int64_t K, const void* A, const void* W,
+                        const float* bias, void* out, bool out_f32, int* status, cudaStream_t st);
+cudaError_t mimo_up_launch(int64_t T, int64_t H, int64_t R, int64_t P, bool bf16, const void* x,
+                           const float* w, void* X, cudaStream_t s);
+cudaError_t mimo_down_gate_launch(int64_t T, int64_t H, int64_t R, int64_t P, bool bf16,
+                                  const void* Y, const float* w, const void* z, void* out,
+                                  cudaStream_t s);
+
 // Decode step.
 cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t s);
 

@@ -108,6 +108,13 @@ def load() -> ctypes.CDLL:
             L.m3_scan_bwd_varlen.restype = ctypes.c_int
             L.m3_bc_prep.argtypes = [sp] + [vp] * 6 + [ctypes.c_float, vp, vp, vp]
             L.m3_bc_prep.restype = ctypes.c_int
+            L.m3_linear.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64] + [vp] * 4 + \
+                [ctypes.c_int32, vp]
+            L.m3_linear.restype = ctypes.c_int
+            L.m3_mimo_up.argtypes = [sp] + [vp] * 4
+            L.m3_mimo_up.restype = ctypes.c_int
+            L.m3_mimo_down_gate.argtypes = [sp] + [vp] * 5
+            L.m3_mimo_down_gate.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -437,3 +444,59 @@ def m3_stream_status(stream=None) -> int:
 
 def version() -> str:
     return load().m3_version().decode()
+
+
+# ---- block projections around the layer ---------------------------------------
+
+def m3_linear(A, W, bias=None, *, out=None, out_dtype=torch.bfloat16, stream=None):
+    """out = A W^T (+ bias) on the tensor cores: A [..][K] bf16 (rows are
+    tokens), W [N][K] bf16, bias [N] fp32; returns out [..][N] in out_dtype
+    (bf16 or fp32)."""
+    if A.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
+        raise TypeError("m3_linear takes bf16 A and W")
+    K = A.shape[-1]
+    M = A.numel() // K if K else 0
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError(f"W is {tuple(W.shape)}, expected [N][{K}]")
+    if out is None:
+        out = torch.empty(A.shape[:-1] + (N,), dtype=out_dtype, device=A.device)
+    code = M3_F32 if out.dtype == torch.float32 else M3_BF16
+    st = load().m3_linear(ctypes.c_int64(M), ctypes.c_int64(N), ctypes.c_int64(K), _ptr(A),
+                          _ptr(W), _ptr(bias), _ptr(out), ctypes.c_int32(code), _stream(stream))
+    _check("m3_linear", st)
+    return out
+
+
+def _tokens_shape(T, H, R, P, dtype):
+    """m3_shape of a block step over T tokens (one sequence of T tokens; the
+    scan-only fields get admissible placeholders)."""
+    return make_shape(1, T, H, 1, P, 16, R, 64, dtype, False)
+
+
+def m3_mimo_up(x, w_up, *, X=None, stream=None):
+    """X[..][h][r][p] = x[..][h][p] * w_up[h][r][p]: x [..][H][P] io dtype,
+    w_up [H][R][P] fp32; returns X [..][H][R][P]."""
+    H, R, P = w_up.shape
+    T = x.numel() // (H * P)
+    if X is None:
+        X = torch.empty(x.shape[:-1] + (R, P), dtype=x.dtype, device=x.device)
+    shape = _tokens_shape(T, H, R, P, x.dtype)
+    st = load().m3_mimo_up(ctypes.byref(shape), _ptr(x), _ptr(w_up), _ptr(X), _stream(stream))
+    _check("m3_mimo_up", st)
+    return X
+
+
+def m3_mimo_down_gate(Y, w_down, z=None, *, out=None, stream=None):
+    """out[..][h][p] = (sum_r Y[..][h][r][p] w_down[h][r][p]) * silu(z[..][h][p]):
+    Y [..][H][R][P] io dtype, w_down [H][R][P] fp32, z [..][H][P] io dtype or
+    None (no gate); returns out [..][H][P]."""
+    H, R, P = w_down.shape
+    T = Y.numel() // (H * R * P)
+    if out is None:
+        out = torch.empty(Y.shape[:-2] + (P,), dtype=Y.dtype, device=Y.device)
+    shape = _tokens_shape(T, H, R, P, Y.dtype)
+    st = load().m3_mimo_down_gate(ctypes.byref(shape), _ptr(Y), _ptr(w_down), _ptr(z), _ptr(out),
+                                  _stream(stream))
+    _check("m3_mimo_down_gate", st)
+    return out
