@@ -340,7 +340,7 @@ M3_API int m3_linear(int64_t M, int64_t N, int64_t K, const void* A, const void*
  *              not used.
  *   x          [tokens][H][P] io dtype;  w_up [H][R][P] fp32;
  *   X          [tokens][H][R][P] io dtype (the layer's x).
- *   x, X 16-byte aligned, w_up 4-byte aligned; P % 8 == 0 for bf16 io. */
+ *   x, X, w_up 16-byte aligned; P % 8 == 0 for bf16 io. */
 M3_API int m3_mimo_up(const m3_shape* shape, const void* x, const float* w_up, void* X,
                       m3_stream_t stream);
 

@@ -50,35 +50,47 @@ struct Vec {
   }
 };
 
-// one thread per V-wide piece of X: piece q covers (t, h, r, p .. p+V-1)
-template <bool BF16>
-__global__ void __launch_bounds__(kThreads) mimo_up_kernel(int64_t T, int H, int R, int P,
-                                                           const void* x, const float* w,
-                                                           void* X) {
-  using Vc = Vec<BF16>;
-  constexpr int V = Vc::V;
-  const int pv = P / V;
-  const int64_t pieces = T * H * R * pv;
-  for (int64_t q = (int64_t)blockIdx.x * kThreads + threadIdx.x; q < pieces;
-       q += (int64_t)gridDim.x * kThreads) {
-    const int p = (int)(q % pv) * V;
-    int64_t rest = q / pv;
-    const int r = (int)(rest % R);
-    rest /= R;
-    const int h = (int)(rest % H);
-    const int64_t t = rest / H;
-    float xv[V], o[V];
-    Vc::load(x, (t * H + h) * P + p, xv);
-    const float* wr = w + ((int64_t)h * R + r) * P + p;
+// V consecutive fp32 weights (two or one float4 loads through the read-only path).
+template <int V>
+__device__ __forceinline__ void load_w(const float* w, float (&f)[V]) {
 #pragma unroll
-    for (int e = 0; e < V; ++e) o[e] = xv[e] * __ldg(wr + e);
-    Vc::store(X, ((t * H + h) * R + r) * P + p, o);
+  for (int e = 0; e < V; e += 4) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(w + e));
+    f[e] = v.x; f[e + 1] = v.y; f[e + 2] = v.z; f[e + 3] = v.w;
   }
 }
 
-// one thread per V-wide piece of out: piece q covers (t, h, p .. p+V-1)
-template <bool BF16>
-__global__ void __launch_bounds__(kThreads) mimo_down_gate_kernel(int64_t T, int H, int R, int P,
+// one thread per V-wide piece of x: piece q covers (t, h, p .. p+V-1) and
+// writes that piece of all R ranks of X
+template <bool BF16, int R>
+__global__ void __launch_bounds__(kThreads) mimo_up_kernel(int64_t T, int H, int P, const void* x,
+                                                           const float* w, void* X) {
+  using Vc = Vec<BF16>;
+  constexpr int V = Vc::V;
+  const int pv = P / V;
+  const int64_t pieces = T * H * pv;
+  for (int64_t q = (int64_t)blockIdx.x * kThreads + threadIdx.x; q < pieces;
+       q += (int64_t)gridDim.x * kThreads) {
+    const int p = (int)(q % pv) * V;
+    const int64_t th = q / pv;  // t * H + h
+    const int h = (int)(th % H);
+    float xv[V];
+    Vc::load(x, th * P + p, xv);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float wv[V], o[V];
+      load_w<V>(w + ((int64_t)h * R + r) * P + p, wv);
+#pragma unroll
+      for (int e = 0; e < V; ++e) o[e] = xv[e] * wv[e];
+      Vc::store(X, (th * R + r) * P + p, o);
+    }
+  }
+}
+
+// one thread per V-wide piece of out: piece q covers (t, h, p .. p+V-1); the
+// R pieces of Y are all loaded before any is used
+template <bool BF16, int R>
+__global__ void __launch_bounds__(kThreads) mimo_down_gate_kernel(int64_t T, int H, int P,
                                                                   const void* Y, const float* w,
                                                                   const void* z, void* out) {
   using Vc = Vec<BF16>;
@@ -90,21 +102,23 @@ __global__ void __launch_bounds__(kThreads) mimo_down_gate_kernel(int64_t T, int
     const int p = (int)(q % pv) * V;
     const int64_t th = q / pv;  // t * H + h
     const int h = (int)(th % H);
+    float yv[R][V], zv[V];
+#pragma unroll
+    for (int r = 0; r < R; ++r) Vc::load(Y, (th * R + r) * P + p, yv[r]);
+    if (z) Vc::load(z, th * P + p, zv);
     float acc[V];
 #pragma unroll
     for (int e = 0; e < V; ++e) acc[e] = 0.f;
-    for (int r = 0; r < R; ++r) {
-      float yv[V];
-      Vc::load(Y, (th * R + r) * P + p, yv);
-      const float* wr = w + ((int64_t)h * R + r) * P + p;
 #pragma unroll
-      for (int e = 0; e < V; ++e) acc[e] = fmaf(yv[e], __ldg(wr + e), acc[e]);
+    for (int r = 0; r < R; ++r) {
+      float wv[V];
+      load_w<V>(w + ((int64_t)h * R + r) * P + p, wv);
+#pragma unroll
+      for (int e = 0; e < V; ++e) acc[e] = fmaf(yv[r][e], wv[e], acc[e]);
     }
     if (z) {
-      float zv[V];
-      Vc::load(z, th * P + p, zv);
 #pragma unroll
-      for (int e = 0; e < V; ++e) acc[e] *= zv[e] / (1.f + expf(-zv[e]));
+      for (int e = 0; e < V; ++e) acc[e] *= zv[e] / (1.f + __expf(-zv[e]));
     }
     Vc::store(out, th * P + p, acc);
   }
@@ -119,31 +133,62 @@ int grid_for(int64_t pieces) {
   return (int)(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
 }
 
+template <bool BF16, int R>
+cudaError_t up_r(int64_t T, int64_t H, int64_t P, const void* x, const float* w, void* X,
+                 cudaStream_t s) {
+  const int64_t pieces = T * H * (P / Vec<BF16>::V);
+  mimo_up_kernel<BF16, R><<<grid_for(pieces), kThreads, 0, s>>>(T, (int)H, (int)P, x, w, X);
+  return cudaGetLastError();
+}
+
+template <bool BF16, int R>
+cudaError_t down_r(int64_t T, int64_t H, int64_t P, const void* Y, const float* w, const void* z,
+                   void* out, cudaStream_t s) {
+  const int64_t pieces = T * H * (P / Vec<BF16>::V);
+  mimo_down_gate_kernel<BF16, R><<<grid_for(pieces), kThreads, 0, s>>>(T, (int)H, (int)P, Y, w,
+                                                                        z, out);
+  return cudaGetLastError();
+}
+
+template <bool BF16>
+cudaError_t up_dispatch(int64_t T, int64_t H, int64_t R, int64_t P, const void* x, const float* w,
+                        void* X, cudaStream_t s) {
+  switch (R) {
+    case 1: return up_r<BF16, 1>(T, H, P, x, w, X, s);
+    case 2: return up_r<BF16, 2>(T, H, P, x, w, X, s);
+    case 4: return up_r<BF16, 4>(T, H, P, x, w, X, s);
+    case 8: return up_r<BF16, 8>(T, H, P, x, w, X, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <bool BF16>
+cudaError_t down_dispatch(int64_t T, int64_t H, int64_t R, int64_t P, const void* Y,
+                          const float* w, const void* z, void* out, cudaStream_t s) {
+  switch (R) {
+    case 1: return down_r<BF16, 1>(T, H, P, Y, w, z, out, s);
+    case 2: return down_r<BF16, 2>(T, H, P, Y, w, z, out, s);
+    case 4: return down_r<BF16, 4>(T, H, P, Y, w, z, out, s);
+    case 8: return down_r<BF16, 8>(T, H, P, Y, w, z, out, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 }  // namespace
 
 cudaError_t mimo_up_launch(int64_t T, int64_t H, int64_t R, int64_t P, bool bf16, const void* x,
                            const float* w, void* X, cudaStream_t s) {
-  const int64_t pieces = T * H * R * (P / (bf16 ? 8 : 4));
-  if (pieces == 0) return cudaSuccess;
-  if (bf16)
-    mimo_up_kernel<true><<<grid_for(pieces), kThreads, 0, s>>>(T, (int)H, (int)R, (int)P, x, w, X);
-  else
-    mimo_up_kernel<false><<<grid_for(pieces), kThreads, 0, s>>>(T, (int)H, (int)R, (int)P, x, w, X);
-  return cudaGetLastError();
+  if (T * H == 0) return cudaSuccess;
+  return bf16 ? up_dispatch<true>(T, H, R, P, x, w, X, s)
+              : up_dispatch<false>(T, H, R, P, x, w, X, s);
 }
 
 cudaError_t mimo_down_gate_launch(int64_t T, int64_t H, int64_t R, int64_t P, bool bf16,
                                   const void* Y, const float* w, const void* z, void* out,
                                   cudaStream_t s) {
-  const int64_t pieces = T * H * (P / (bf16 ? 8 : 4));
-  if (pieces == 0) return cudaSuccess;
-  if (bf16)
-    mimo_down_gate_kernel<true><<<grid_for(pieces), kThreads, 0, s>>>(T, (int)H, (int)R, (int)P,
-                                                                       Y, w, z, out);
-  else
-    mimo_down_gate_kernel<false><<<grid_for(pieces), kThreads, 0, s>>>(T, (int)H, (int)R, (int)P,
-                                                                        Y, w, z, out);
-  return cudaGetLastError();
+  if (T * H == 0) return cudaSuccess;
+  return bf16 ? down_dispatch<true>(T, H, R, P, Y, w, z, out, s)
+              : down_dispatch<false>(T, H, R, P, Y, w, z, out, s);
 }
 
 }  // namespace m3

@@ -425,7 +425,7 @@ int mimo_check(const m3_shape* s, const void* in, const float* w, const void* ex
   if (s->headdim % (bf16 ? 8 : 4) != 0) return M3_ERR_UNSUPPORTED;
   if (s->batch * s->seqlen == 0) return M3_OK;
   if (!in || !w || !out) return M3_ERR_INVALID_ARGUMENT;
-  if (!aligned(in, 16) || !aligned(out, 16) || (extra && !aligned(extra, 16)) || !aligned(w, 4))
+  if (!aligned(in, 16) || !aligned(out, 16) || (extra && !aligned(extra, 16)) || !aligned(w, 16))
     return M3_ERR_ALIGNMENT;
   return M3_OK;
 }
