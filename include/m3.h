@@ -133,6 +133,12 @@ M3_API int m3_check_shape(const m3_shape* shape);
  * Host-only; writes *bytes.  Returns M3_OK or the m3_check_shape error. */
 M3_API int m3_scan_workspace_size(const m3_shape* shape, size_t* bytes);
 
+/* The same query as a single value: the workspace bytes m3_scan_fwd needs for
+ * `shape` (0 when L == 0 or when the shape needs none), or SIZE_MAX when the
+ * shape fails m3_check_shape (the status itself is not reported; call
+ * m3_check_shape for it).  Host-only, never touches the GPU. */
+M3_API size_t m3_scan_workspace_bytes(const m3_shape* shape);
+
 /* How m3_scan_fwd will run `shape` (host-only): *tensor_core = 1 for the
  * tcgen05 path (bf16 io, N = 128, P = 64, chunk * rank in {64, 128, 256},
  * M3_FLAG_SIMT clear), 0 for the CUDA-core fp32 path; *segments = pieces

@@ -1,7 +1,9 @@
 // m3_api.cu -- the C ABI declared in include/m3.h: argument checks, workspace
 // sizing, dispatch to the kernels, and the device-side error word.
 #include <cuda.h>  // CUcontext (the driver calls are reached through the runtime)
+#include <nvtx3/nvToolsExt.h>  // header-only; ranges cost a pointer check with no tool attached
 
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -9,6 +11,16 @@
 #include "m3_internal.cuh"
 
 namespace m3 {
+
+// An NVTX range named after the C-ABI call for the duration of the call (host
+// side: argument checks and launches), so a timeline tool attached to the
+// process shows each call around its kernels.
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 // First device-side error raised by a kernel (M3_ERR_*), 0 if none.
 __device__ int g_device_status = 0;
@@ -156,6 +168,11 @@ M3_API int m3_scan_workspace_size(const m3_shape* s, size_t* bytes) {
   return workspace_query(s, bytes, false);
 }
 
+M3_API size_t m3_scan_workspace_bytes(const m3_shape* s) {
+  size_t n = 0;
+  return workspace_query(s, &n, false) == M3_OK ? n : SIZE_MAX;
+}
+
 M3_API int m3_scan_state_workspace_size(const m3_shape* s, size_t* bytes) {
   return workspace_query(s, bytes, true);
 }
@@ -232,6 +249,7 @@ M3_API int m3_scan_fwd(const m3_shape* s, const void* x, const float* dt, const 
                        const float* h0, const void* B_prev, const void* x_prev, void* y,
                        float* final_state, void* workspace, size_t workspace_bytes,
                        m3_stream_t stream) {
+  m3::CallRange range_("m3_scan_fwd");
   return scan_call(s, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev, y, final_state, workspace,
                    workspace_bytes, stream, false);
 }
@@ -243,6 +261,7 @@ M3_API int m3_scan_fwd_varlen(const m3_shape* s, const int32_t* cu_seqlens,
                               const void* B_prev, const void* x_prev, void* y,
                               float* final_state, void* workspace, size_t workspace_bytes,
                               m3_stream_t stream) {
+  m3::CallRange range_("m3_scan_fwd_varlen");
   if (!cu_seqlens) return M3_ERR_INVALID_ARGUMENT;
   return scan_call(s, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev, y, final_state, workspace,
                    workspace_bytes, stream, false, cu_seqlens, total_tokens);
@@ -341,6 +360,7 @@ M3_API int m3_scan_bwd(const m3_shape* s, const void* x, const float* dt, const 
                        float* dtheta, float* dB, float* dC, float* dh0, float* dB_prev,
                        float* dx_prev, void* workspace, size_t workspace_bytes,
                        m3_stream_t stream) {
+  m3::CallRange range_("m3_scan_bwd");
   return bwd_call(s, nullptr, 0, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev, dy, d_final,
                   dx, ddt, dA, dlam, dtheta, dB, dC, dh0, dB_prev, dx_prev, workspace,
                   workspace_bytes, stream);
@@ -354,6 +374,7 @@ M3_API int m3_scan_bwd_varlen(const m3_shape* s, const int32_t* cu_seqlens, int6
                               float* dlam, float* dtheta, float* dB, float* dC, float* dh0,
                               float* dB_prev, float* dx_prev, void* workspace,
                               size_t workspace_bytes, m3_stream_t stream) {
+  m3::CallRange range_("m3_scan_bwd_varlen");
   if (!cu_seqlens) return M3_ERR_INVALID_ARGUMENT;
   return bwd_call(s, cu_seqlens, total_tokens, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev,
                   dy, d_final, dx, ddt, dA, dlam, dtheta, dB, dC, dh0, dB_prev, dx_prev,
@@ -363,6 +384,7 @@ M3_API int m3_scan_bwd_varlen(const m3_shape* s, const int32_t* cu_seqlens, int6
 M3_API int m3_bc_prep(const m3_shape* s, const void* B_raw, const void* C_raw,
                       const float* B_weight, const float* B_bias, const float* C_weight,
                       const float* C_bias, float eps, void* B, void* C, m3_stream_t stream) {
+  m3::CallRange range_("m3_bc_prep");
   int st = check_common(s);
   if (st != M3_OK) return st;
   if ((B_raw == nullptr) != (B == nullptr) || (C_raw == nullptr) != (C == nullptr))
@@ -391,6 +413,7 @@ M3_API int m3_bc_prep(const m3_shape* s, const void* B_raw, const void* C_raw,
 
 M3_API int m3_linear(int64_t M, int64_t N, int64_t K, const void* A, const void* W,
                      const float* bias, void* out, int32_t out_dtype, m3_stream_t stream) {
+  m3::CallRange range_("m3_linear");
   if (out_dtype != M3_BF16 && out_dtype != M3_F32) return M3_ERR_INVALID_ARGUMENT;
   const bool f32 = out_dtype == M3_F32;
   if (M < 0 || N < 1 || K < 8) return M3_ERR_INVALID_ARGUMENT;
@@ -433,6 +456,7 @@ int mimo_check(const m3_shape* s, const void* in, const float* w, const void* ex
 
 M3_API int m3_mimo_up(const m3_shape* s, const void* x, const float* w_up, void* X,
                       m3_stream_t stream) {
+  m3::CallRange range_("m3_mimo_up");
   int st = mimo_check(s, x, w_up, nullptr, X);
   if (st != M3_OK || s->batch * s->seqlen == 0) return st;
   const size_t es = s->io_dtype == M3_BF16 ? 2 : 4;
@@ -448,6 +472,7 @@ M3_API int m3_mimo_up(const m3_shape* s, const void* x, const float* w_up, void*
 
 M3_API int m3_mimo_down_gate(const m3_shape* s, const void* Y, const float* w_down,
                              const void* z, void* out, m3_stream_t stream) {
+  m3::CallRange range_("m3_mimo_down_gate");
   int st = mimo_check(s, Y, w_down, z, out);
   if (st != M3_OK || s->batch * s->seqlen == 0) return st;
   const size_t es = s->io_dtype == M3_BF16 ? 2 : 4;
@@ -470,6 +495,7 @@ M3_API int m3_scan_state(const m3_shape* s, const void* x, const float* dt, cons
                          const float* h0, const void* B_prev, const void* x_prev,
                          float* final_state, void* workspace, size_t workspace_bytes,
                          m3_stream_t stream) {
+  m3::CallRange range_("m3_scan_state");
   return scan_call(s, x, dt, A, lam, theta, B, C, h0, B_prev, x_prev, nullptr, final_state,
                    workspace, workspace_bytes, stream, true);
 }
@@ -477,6 +503,7 @@ M3_API int m3_scan_state(const m3_shape* s, const void* x, const float* dt, cons
 M3_API int m3_segment_totals(const m3_shape* s, const float* dt, const float* A,
                              const float* theta, float* lam_tot, float* phi_tot,
                              m3_stream_t stream) {
+  m3::CallRange range_("m3_segment_totals");
   int st = check_common(s);
   if (st != M3_OK) return st;
   if (!lam_tot || !phi_tot) return M3_ERR_INVALID_ARGUMENT;
@@ -493,6 +520,7 @@ M3_API int m3_segment_totals(const m3_shape* s, const float* dt, const float* A,
 M3_API int m3_state_fold(const m3_shape* s, int64_t nseg, const float* h0, const float* T,
                          const float* lam_tot, const float* phi_tot, float* out,
                          m3_stream_t stream) {
+  m3::CallRange range_("m3_state_fold");
   int st = check_common(s);
   if (st != M3_OK) return st;
   if (nseg < 0 || !out || (nseg > 0 && (!T || !lam_tot || !phi_tot))) return M3_ERR_INVALID_ARGUMENT;
@@ -520,6 +548,7 @@ M3_API int m3_decode_step(const m3_shape* s, const float* state_in, float* state
                           const float* lam_t, const float* theta_t, const void* B_t,
                           const void* C_t, const void* B_prev, const void* x_prev, void* y_t,
                           m3_stream_t stream) {
+  m3::CallRange range_("m3_decode_step");
   int st = check_common(s);
   if (st != M3_OK) return st;
   if ((B_prev == nullptr) != (x_prev == nullptr)) return M3_ERR_INVALID_ARGUMENT;

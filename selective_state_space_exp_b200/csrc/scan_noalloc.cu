@@ -59,7 +59,7 @@ extern "C" M3_API int m3_scan_fwd_noalloc(const m3_shape* s, const void* x, cons
                                           const float* h0, const void* B_prev,
                                           const void* x_prev, void* y, float* final_state,
                                           m3_stream_t stream) {
-  size_t need = 0;
+  size_t need = 0;  // (m3_scan_fwd below opens this call's NVTX range)
   const int st = m3_scan_workspace_size(s, &need);
   if (st != M3_OK) return st;
   if (need > (size_t)M3_NOALLOC_SCRATCH_BYTES) return M3_ERR_WORKSPACE;

@@ -76,6 +76,8 @@ def load() -> ctypes.CDLL:
             L.m3_check_shape.restype = ctypes.c_int
             L.m3_scan_workspace_size.argtypes = [sp, ctypes.POINTER(ctypes.c_size_t)]
             L.m3_scan_workspace_size.restype = ctypes.c_int
+            L.m3_scan_workspace_bytes.argtypes = [sp]
+            L.m3_scan_workspace_bytes.restype = ctypes.c_size_t
             L.m3_scan_plan.argtypes = [sp, ctypes.POINTER(ctypes.c_int),
                                        ctypes.POINTER(ctypes.c_int64),
                                        ctypes.POINTER(ctypes.c_int)]

@@ -60,6 +60,33 @@ def sum_over_ranks(value: float, device: torch.device | str = "cpu") -> float:
     return float(t.item())
 
 
+def batch_shard(tensors: dict, world: int, rank: int) -> dict:
+    """This rank's contiguous share (shard_range over dim 0) of every batched
+    tensor of a layer call; None entries pass through."""
+    n = next(v.shape[0] for v in tensors.values() if v is not None)
+    a, b = shard_range(n, world, rank)
+    return {k: (None if v is None else v[a:b]) for k, v in tensors.items()}
+
+
+def batch_gather(local: torch.Tensor, n: int, group=None) -> torch.Tensor:
+    """Assemble the ranks' batch shards (in rank order, as batch_shard cut
+    them) into the whole batch of n rows on every rank.  Not part of the
+    layer's data path, which needs no exchange; a caller that wants one rank
+    to hold every output uses it after the step."""
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    rows = max(b - a for a, b in (shard_range(n, world, r) for r in range(world)))
+    a, b = shard_range(n, world, rank)
+    if local.shape[0] != b - a:
+        raise ValueError(f"rank {rank} holds {local.shape[0]} rows, its share is {b - a}")
+    pad = local.new_zeros((rows,) + tuple(local.shape[1:]))
+    pad[: b - a] = local
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad.contiguous(), group=group)
+    return torch.cat([parts[r][: e - s] for r, (s, e) in
+                      enumerate(shard_range(n, world, r) for r in range(world))])
+
+
 # ---- sequence split across ranks (context parallel) ---------------------------
 
 class M3Ops:

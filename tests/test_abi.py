@@ -22,8 +22,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = set(declared_functions())
-    assert {"m3_scan_fwd", "m3_decode_step", "m3_scan_workspace_size", "m3_stream_status",
-            "m3_check_shape", "m3_status_string", "m3_version"} <= names
+    assert {"m3_scan_fwd", "m3_decode_step", "m3_scan_workspace_size", "m3_scan_workspace_bytes",
+            "m3_stream_status", "m3_check_shape", "m3_status_string", "m3_version"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -78,6 +78,23 @@ def test_workspace_size(lib):
     assert lib.m3_scan_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0 and n.value == 0
     assert lib.m3_scan_workspace_size(ctypes.byref(s), None) == -1
     assert lib.m3_scan_workspace_size(None, ctypes.byref(n)) == -1
+
+
+def test_workspace_bytes_matches_the_status_form(lib):
+    """m3_scan_workspace_bytes returns the value m3_scan_workspace_size writes,
+    and SIZE_MAX where the status form returns an error."""
+    size_max = ctypes.c_size_t(-1).value
+    for kw in (dict(seqlen=0), dict(seqlen=130, flags=m3.M3_FLAG_SIMT), dict(seqlen=130),
+               dict(batch=8, nheads=64, seqlen=2048), dict(seqlen=4096, flags=m3.M3_FLAG_SIMT)):
+        s = shape(**kw)
+        n = ctypes.c_size_t()
+        assert lib.m3_scan_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0
+        assert lib.m3_scan_workspace_bytes(ctypes.byref(s)) == n.value
+    for kw in (dict(nheads=0), dict(headdim=0), dict(chunk=48), dict(io_dtype=7)):
+        s = shape(**kw)
+        assert lib.m3_check_shape(ctypes.byref(s)) != 0
+        assert lib.m3_scan_workspace_bytes(ctypes.byref(s)) == size_max
+    assert lib.m3_scan_workspace_bytes(None) == size_max
 
 
 # Fake, never dereferenced device addresses: every case below fails a host

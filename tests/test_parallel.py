@@ -302,3 +302,75 @@ def test_sequence_split_backward_without_h0_or_previous_token():
         got = np.concatenate([parts[r][k].numpy() for r in range(world)], axis=1)
         assert np.max(np.abs(got - ref[k])) <= 1e-10 * np.max(np.abs(ref[k])), k
     assert np.max(np.abs(parts[0]["h0"].numpy() - ref["h0"])) <= 1e-10 * np.max(np.abs(ref["h0"]))
+
+
+# ---- batch sharding, assembled ------------------------------------------------
+# Each rank scans its shard_range share of one seeded batch (the oracle standing
+# in for the rank's kernels); batch_gather assembles the shares, which must
+# equal one oracle scan of the whole batch.
+
+from selective_state_space_exp_b200.parallel import batch_gather, batch_shard  # noqa: E402
+
+
+def _batch_problem(b=5):
+    rng = np.random.default_rng(91)
+    L, H, G, P, N, R = 12, 2, 1, 3, 4, 2
+    d = dict(x=rng.standard_normal((b, L, H, R, P)),
+             dt=np.log1p(np.exp(rng.normal(-1.0, 0.5, (b, L, H)))),
+             A=-np.exp(rng.uniform(0.0, 1.0, (b, L, H))),
+             lam=1 / (1 + np.exp(-rng.standard_normal((b, L, H)))),
+             theta=rng.uniform(-np.pi, np.pi, (b, L, G, N // 2)),
+             B=rng.standard_normal((b, L, G, R, N)), C=rng.standard_normal((b, L, G, R, N)),
+             h0=rng.standard_normal((b, H, N, P)), B_prev=rng.standard_normal((b, G, R, N)),
+             x_prev=rng.standard_normal((b, H, R, P)))
+    return {k: torch.from_numpy(v) for k, v in d.items()}
+
+
+def _batch_worker(rank, world, port, out, b):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        d = batch_shard(_batch_problem(b), world, rank)
+        if d["x"].shape[0]:
+            y, hL = OracleOps().scan_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"],
+                                         d["C"], 4, d["h0"], d["B_prev"], d["x_prev"])
+        else:  # more ranks than rows: this rank launches nothing (batch 0 is not a shape)
+            y = torch.zeros(d["x"].shape, dtype=torch.float64)
+            hL = torch.zeros(d["h0"].shape, dtype=torch.float64)
+        out[rank] = (batch_gather(y, b).numpy(), batch_gather(hL, b).numpy(), y.shape[0])
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,b", [(2, 5), (3, 5), (2, 1)])
+def test_gloo_batch_shards_assemble_to_the_whole_batch(world, b):
+    out = mp.Manager().dict()
+    mp.spawn(_batch_worker, args=(world, _free_port(), out, b), nprocs=world, join=True)
+    d = _batch_problem(b)
+    y_ref, h_ref = OracleOps().scan_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"],
+                                        d["C"], 4, d["h0"], d["B_prev"], d["x_prev"])
+    assert sum(out[r][2] for r in range(world)) == b  # every batch row scanned once
+    for r in range(world):
+        y, hL, _ = out[r]
+        assert y.shape == tuple(y_ref.shape) and hL.shape == tuple(h_ref.shape)
+        np.testing.assert_allclose(y, y_ref.numpy(), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(hL, h_ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_batch_gather_rejects_a_wrong_share():
+    out = mp.Manager().dict()
+    mp.spawn(_bad_share_worker, args=(2, _free_port(), out), nprocs=2, join=True)
+    assert out[0] == "ValueError" and out[1] == "ValueError"
+
+
+def _bad_share_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        try:
+            batch_gather(torch.zeros(4, 3), 5)  # shares of 5 rows are 3 and 2
+            out[rank] = "ok"
+        except ValueError:
+            out[rank] = "ValueError"
+    finally:
+        dist.destroy_process_group()
