@@ -17,7 +17,7 @@ OBJ = os.path.join(PKG, "_build")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libm3.so")
 SOURCES = ["m3_api.cu", "decode.cu", "scan_simt.cu", "scan_tc.cu", "scan_noalloc.cu",
-           "seqpar.cu", "scan_bwd.cu", "bc_prep.cu", "gemm_tc.cu", "block_ops.cu"]
+           "seqpar.cu", "scan_bwd.cu", "scan_bwd_tc.cu", "bc_prep.cu", "gemm_tc.cu", "block_ops.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
          "-Xptxas", "-warn-spills", "--expt-relaxed-constexpr"]

@@ -273,7 +273,7 @@ M3_API int m3_scan_bwd_workspace_size(const m3_shape* s, size_t* bytes) {
   if (!bytes) return M3_ERR_INVALID_ARGUMENT;
   ScanArgs a = make_scan_args(s);
   if (!bwd_supported(a)) return M3_ERR_UNSUPPORTED;
-  *bytes = s->seqlen == 0 ? 0 : bwd_workspace(a);
+  *bytes = s->seqlen == 0 ? 0 : bwd_workspace(a, (s->flags & M3_FLAG_SIMT) == 0);
   return M3_OK;
 }
 
@@ -325,7 +325,8 @@ int bwd_call(const m3_shape* s, const int32_t* cu_seqlens, int64_t total_tokens,
     }
     return M3_OK;
   }
-  const size_t need = bwd_workspace(a);
+  const bool tc = (s->flags & M3_FLAG_SIMT) == 0;
+  const size_t need = bwd_workspace(a, tc);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return M3_ERR_WORKSPACE;
   a.x = x; a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.B = B; a.C = C;
   a.h0 = h0; a.B_prev = B_prev; a.x_prev = x_prev;
@@ -347,7 +348,7 @@ int bwd_call(const m3_shape* s, const int32_t* cu_seqlens, int64_t total_tokens,
         cudaMemsetAsync(dx_prev, 0, nx, cs) != cudaSuccess)
       return M3_ERR_CUDA;
   }
-  cudaError_t e = bwd_launch(a, g, cs);
+  cudaError_t e = bwd_launch(a, g, tc, cs);
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 

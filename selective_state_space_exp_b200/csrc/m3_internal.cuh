@@ -126,9 +126,12 @@ struct BwdArgs {
   float* dB_prev;         // [b][G][R][N] or nullptr (with dx_prev)
   float* dx_prev;         // [b][H][R][P] or nullptr
 };
-size_t bwd_workspace(const ScanArgs& a);
+// tc: the tensor-core form where the shape allows it (bf16 io, N = 128,
+// P = 64), else the CUDA-core one; the workspace depends on the form.
+size_t bwd_workspace(const ScanArgs& a, bool tc);
 bool bwd_supported(const ScanArgs& a);
-cudaError_t bwd_launch(const ScanArgs& a, const BwdArgs& g, cudaStream_t s);
+bool bwd_use_tc(const ScanArgs& a, bool allow);
+cudaError_t bwd_launch(const ScanArgs& a, const BwdArgs& g, bool tc, cudaStream_t s);
 
 // B / C prep: QK-norm, per-channel scale and bias over rows of N values,
 // tensors [tokens][gr][N] with gr = G * R channel rows.

@@ -30,9 +30,20 @@
 // lam also receive the next chunk's left-endpoint term, so those gradients
 // are accumulated with atomic adds into zeroed outputs.
 #include "m3_internal.cuh"
+#include "scan_bwd.cuh"
 #include "simt_chunk.cuh"
 
 namespace m3 {
+
+ScanArgs bwd_fwd_args(const ScanArgs& a, int64_t Qb) {
+  ScanArgs f = a;
+  f.Q = Qb;
+  f.nchunks = (a.seqlen + Qb - 1) / Qb;
+  f.state_only = true;
+  f.y = nullptr;
+  return f;
+}
+
 namespace {
 
 using simt::chunk_geo;
@@ -42,23 +53,6 @@ using simt::Geo;
 constexpr int kThreads = 256;
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
-
-struct BwdWs {
-  float* G;     // [b][H][nc][N][P] chunk-start states (forward)
-  float* sums;  // [b][H][nc][1 + K] chunk totals (forward)
-  float* D;     // [b][H][nc][N][P] D_c, then the adjoint of chunk c's outgoing state
-  float* fin;   // [b][H][N][P] final state (forward)
-};
-
-// Forward args of the backward's own chunking (chunk Qb, state only).
-ScanArgs fwd_args(const ScanArgs& a, int64_t Qb) {
-  ScanArgs f = a;
-  f.Q = Qb;
-  f.nchunks = (a.seqlen + Qb - 1) / Qb;
-  f.state_only = true;
-  f.y = nullptr;
-  return f;
-}
 
 // ---- step 1: per-chunk sums (S_c and D_c) ---------------------------------------
 // One pass over a chunk's rows gives both N x P products it contributes:
@@ -917,10 +911,7 @@ cudaError_t launch_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaSt
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  dim3 pgrid((unsigned)(((f.N / 2) * f.P + kThreads - 1) / kThreads), (unsigned)f.nheads,
-             (unsigned)f.batch);
-  bwd_pass_kernel<<<pgrid, kThreads, 0, st>>>(f, g, w);
-  e = cudaGetLastError();
+  e = bwd_pass_launch(f, g, w, st);
   if (e != cudaSuccess) return e;
 
   const int M = (int)(f.Q * R);
@@ -946,7 +937,9 @@ cudaError_t launch_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaSt
   return cudaGetLastError();
 }
 
-BwdWs carve(const ScanArgs& f) {
+}  // namespace
+
+BwdWs bwd_carve(const ScanArgs& f) {
   BwdWs w;
   simt_state_views(f, &w.G, &w.sums);
   const size_t fwd = simt_scan_workspace(f);
@@ -956,25 +949,35 @@ BwdWs carve(const ScanArgs& f) {
   return w;
 }
 
-}  // namespace
-
-bool bwd_supported(const ScanArgs& a) { return bwd_rows(a) > 0; }
-
-size_t bwd_workspace(const ScanArgs& a) {
-  const int64_t M = bwd_rows(a);
-  if (M == 0 || a.seqlen == 0) return 0;
-  const ScanArgs f = fwd_args(a, M / a.R);
+size_t bwd_ws_bytes(const ScanArgs& f) {
   return simt_scan_workspace(f) +
          align_up(sizeof(float) * f.batch * f.nheads * f.nchunks * f.N * f.P, 256) +
          align_up(sizeof(float) * f.batch * f.nheads * f.N * f.P, 256);
 }
 
-cudaError_t bwd_launch(const ScanArgs& a, const BwdArgs& g, cudaStream_t st) {
-  const int64_t M = bwd_rows(a);
-  if (M == 0) return cudaErrorInvalidValue;
-  ScanArgs f = fwd_args(a, M / a.R);
-  BwdWs w = carve(f);
-  f.final_state = w.fin;
+cudaError_t bwd_pass_launch(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaStream_t st) {
+  dim3 pgrid((unsigned)(((f.N / 2) * f.P + kThreads - 1) / kThreads), (unsigned)f.nheads,
+             (unsigned)f.batch);
+  bwd_pass_kernel<<<pgrid, kThreads, 0, st>>>(f, g, w);
+  return cudaGetLastError();
+}
+
+bool bwd_supported(const ScanArgs& a) { return bwd_rows(a) > 0; }
+
+// Rows per backward chunk: 64 on the tensor cores, else bwd_rows.
+static int64_t chunk_rows(const ScanArgs& a, bool tc) {
+  return tc && bwd_tc_shape(a) ? kBwdTcRows : bwd_rows(a);
+}
+
+bool bwd_use_tc(const ScanArgs& a, bool allow) { return allow && bwd_tc_shape(a); }
+
+size_t bwd_workspace(const ScanArgs& a, bool tc) {
+  const int64_t M = chunk_rows(a, tc);
+  if (M == 0 || a.seqlen == 0) return 0;
+  return bwd_ws_bytes(bwd_fwd_args(a, M / a.R));
+}
+
+cudaError_t bwd_zero_outputs(const ScanArgs& a, const BwdArgs& g, cudaStream_t st) {
   // outputs accumulated with atomic adds start from zero
   const int64_t tok = a.total_tokens;  // batch x seqlen, or a packed batch's rows
   const int64_t K = a.N / 2;
@@ -987,6 +990,24 @@ cudaError_t bwd_launch(const ScanArgs& a, const BwdArgs& g, cudaStream_t st) {
       cudaError_t e = cudaMemsetAsync(z.p, 0, sizeof(float) * z.n, st);
       if (e != cudaSuccess) return e;
     }
+  return cudaSuccess;
+}
+
+cudaError_t bwd_launch(const ScanArgs& a, const BwdArgs& g, bool tc, cudaStream_t st) {
+  const int64_t M = chunk_rows(a, tc);
+  if (M == 0) return cudaErrorInvalidValue;
+  ScanArgs f = bwd_fwd_args(a, M / a.R);
+  BwdWs w = bwd_carve(f);
+  f.final_state = w.fin;
+  cudaError_t e = bwd_zero_outputs(a, g, st);
+  if (e != cudaSuccess) return e;
+  if (tc && bwd_tc_shape(a)) {
+    e = bwd_tc_sums_launch(f, g, w, st);
+    if (e != cudaSuccess) return e;
+    e = bwd_pass_launch(f, g, w, st);
+    if (e != cudaSuccess) return e;
+    return bwd_tc_chunk_launch(f, g, w, st);
+  }
   switch (a.R) {
     case 1: return launch_r<1>(f, g, w, st);
     case 2: return launch_r<2>(f, g, w, st);

@@ -1,0 +1,782 @@
+// scan_bwd_tc.cu -- steps 1 and 3 of the backward pass on the tensor cores
+// (tcgen05.mma kind::f16: bf16 operands in 128-byte-swizzled shared memory,
+// fp32 accumulators in TMEM), for the layer's shape: bf16 io, N = 128,
+// P = 64, chunks of M = Q R = 64 rows (token, rank).
+//
+// The quantities and notation are those of the CUDA-core backward
+// (scan_bwd.cu), which follows the chunked form of the exponential-
+// trapezoidal recurrence (PaperWeekly page sections 2.1-2.3):
+//   Bt = Rot(-Phi) B, Ct = Rot(-Phi) C        (chunk-local angles Phi)
+//   M_ts = exp(Lam_t - Lam_s) delta_s (s < t), gamma_t (s = t), 0 (s > t)
+//   w_s  = exp(Lam_end - Lam_s) delta_s
+//   G_c  = the state entering chunk c,  dGhat = Rot(-Phi_end) dG_c+1.
+//
+// Step 1, per chunk: S_c = (w Bt)^T X and D_c = (exp(Lam) Ct)^T dY, two
+// N x P products with K = M, each one MMA chain (M = 128 state rows).
+//
+// Step 3, per chunk, in two MMA phases around the mask:
+//   phase A   S  = Ct Bt^T,  DX = dY X^T          (M x M, K = N and P)
+//             AX = Bt dGhat                       (M x P, K = N)
+//             AC = dY G_c^T, AB = X dGhat^T       (M x N, K = P)
+//   between   the masked scores M o S, M o DX (bf16, to shared memory); the
+//             mask's gradients (token pair t, s: dL/dM_ts summed over both
+//             ranks, F_ts = dL/dM_ts exp(Lam_t - Lam_s)); beta_s = x_s . AX_s;
+//             the exp(Lam_t) term of dLam, Ct_t . AC_t exp(Lam_t); then AC,
+//             AB, AX scaled in TMEM by exp(Lam_t), w_s, w_s
+//   phase B   AC += (M o DX) Bt      -> dCt = exp(Lam) dY G^T + (M o DX) Bt
+//             AB += (M o DX)^T Ct    -> dBt = (M o DX)^T Ct + w X dGhat^T
+//             AX += (M o S)^T dY     -> dX  = (M o S)^T dY + w Bt dGhat
+// then the rotations back to B and C, the angle gradients and the backward
+// of the chunk-local prefix sums, as on the CUDA cores.  TMEM holds 448 of
+// its 512 columns; the global loads of a chunk are staged before its TMEM is
+// allocated, so a second CTA on the SM prepares its chunk while the first
+// one computes.
+#include <cuda_bf16.h>
+
+#include "m3_internal.cuh"
+#include "scan_bwd.cuh"
+#include "simt_chunk.cuh"
+#include "tc_ptx.cuh"
+
+namespace m3 {
+namespace {
+
+using namespace tc;
+using simt::chunk_geo;
+using simt::chunk_prep;
+using simt::Geo;
+
+constexpr int kN = 128;                 // dstate
+constexpr int kP = 64;                  // headdim
+constexpr int kK = kN / 2;              // rotation pairs
+constexpr int kM = (int)kBwdTcRows;     // rows per chunk
+constexpr int kTh = 256;
+constexpr int kOPB = kM * 128;          // one [64 rows][128 B] operand block
+constexpr float kL2E = 1.4426950408889634f;
+constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded mbarrier wait (2 s)
+
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Polls an mbarrier (one thread); false after recording M3_ERR_TIMEOUT.
+__device__ bool wait_mma(uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = now_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (now_ns() - t0 > kWaitNs) {
+      if (status) atomicCAS(status, 0, (int)M3_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t bytes) {
+  return d + (uint64_t)(bytes >> 4);
+}
+
+// 8 consecutive bf16 values (16 bytes) as floats.
+__device__ __forceinline__ void ld8_bf16(const void* base, int64_t idx, float (&v)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + idx));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = unpack_bf16(w[j]);
+    v[2 * j] = f.x;
+    v[2 * j + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void ld8_f32(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
+  return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                    pack_bf16(v[6], v[7]));
+}
+// 16 consecutive bf16 values of row `row` from column c0 (a multiple of 16)
+// of a [rows][64] swizzled block, as floats.
+__device__ __forceinline__ void ld16_sw(const uint8_t* blk, int row, int c0, float (&v)[16]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint4 u = *reinterpret_cast<const uint4*>(blk + sw128_off(row, c0 / 8 + h));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = unpack_bf16(w[j]);
+      v[8 * h + 2 * j] = f.x;
+      v[8 * h + 2 * j + 1] = f.y;
+    }
+  }
+}
+
+// Sine and cosine of an angle of any size (reduced to about [-pi, pi] first).
+__device__ __forceinline__ void sincos_r(float x, float* s, float* c) {
+  __sincosf(reduce_2pi(x), s, c);
+}
+
+// Rows (token, rank) of a chunk: row i is token i / R, rank i % R.  Stages
+// Rot(-Phi_t) of B and C (times the per-token scales sb, sc) for rows i with
+// token t < nt, zeros beyond, as 2 K-major blocks of [64 rows][64 columns].
+template <int R>
+__device__ __forceinline__ void stage_bc(const ScanArgs& a, const Geo& q, const float* phi,
+                                         const float* sb, const float* sc, uint8_t* bt,
+                                         uint8_t* ct) {
+  for (int e = threadIdx.x; e < kM * 16; e += blockDim.x) {
+    const int i = e >> 4, c16 = e & 15, t = i / R, r = i % R;
+    float bv[8], cv[8];
+    if (t < q.nt) {
+      const int64_t base = ((q.base + q.t0 + t) * a.ngroups + q.g) * R * kN + (int64_t)r * kN + 8 * c16;
+      ld8_bf16(a.B, base, bv);
+      ld8_bf16(a.C, base, cv);
+      const float fb = sb ? sb[t] : 1.f, fc = sc ? sc[t] : 1.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float sn, cs;
+        sincos_r(phi[t * kK + 4 * c16 + j], &sn, &cs);
+        const float b0 = bv[2 * j], b1 = bv[2 * j + 1], c0 = cv[2 * j], c1 = cv[2 * j + 1];
+        bv[2 * j] = fb * (cs * b0 + sn * b1);
+        bv[2 * j + 1] = fb * (-sn * b0 + cs * b1);
+        cv[2 * j] = fc * (cs * c0 + sn * c1);
+        cv[2 * j + 1] = fc * (-sn * c0 + cs * c1);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) bv[j] = cv[j] = 0.f;
+    }
+    const uint32_t off = (c16 >> 3) * kOPB + sw128_off(i, c16 & 7);
+    *reinterpret_cast<uint4*>(bt + off) = pack8(bv);
+    *reinterpret_cast<uint4*>(ct + off) = pack8(cv);
+  }
+}
+
+// x and dy rows as one K-major [64 rows][64 columns] block each.
+template <int R>
+__device__ __forceinline__ void stage_xdy(const ScanArgs& a, const BwdArgs& g, const Geo& q,
+                                          uint8_t* xs, uint8_t* dys) {
+  for (int e = threadIdx.x; e < kM * 8; e += blockDim.x) {
+    const int i = e >> 3, c8 = e & 7, t = i / R, r = i % R;
+    float xv[8], yv[8];
+    if (t < q.nt) {
+      const int64_t o = ((q.base + q.t0 + t) * a.nheads + q.h) * R * kP + (int64_t)r * kP + 8 * c8;
+      ld8_bf16(a.x, o, xv);
+      if (g.dy_f32) ld8_f32(static_cast<const float*>(g.dy) + o, yv);
+      else ld8_bf16(g.dy, o, yv);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xv[j] = yv[j] = 0.f;
+    }
+    *reinterpret_cast<uint4*>(xs + sw128_off(i, c8)) = pack8(xv);
+    *reinterpret_cast<uint4*>(dys + sw128_off(i, c8)) = pack8(yv);
+  }
+}
+
+// ---- step 1: S_c and D_c ----------------------------------------------------
+// Shared memory: w Bt (2 blocks), exp(Lam) Ct (2 blocks), x, dy (1 block
+// each), then the prefix sums.  TMEM: S_c in columns 0-63, D_c in 64-127,
+// lane n = state row n.
+struct SumsSmem {
+  static constexpr int WB = 0, EC = 2 * kOPB, XS = 4 * kOPB, DYS = 5 * kOPB;
+  static constexpr int SMALL = 6 * kOPB;
+  static constexpr int bytes(int Q) { return SMALL + (Q * kK + 6 * Q) * 4 + 32; }
+};
+
+template <int R>
+__global__ void __launch_bounds__(kTh) bwd_tc_sums_kernel(const ScanArgs a, const BwdArgs g,
+                                                          const BwdWs w) {
+  constexpr int Q = kM / R;
+  using L = SumsSmem;
+  extern __shared__ __align__(1024) uint8_t sm[];
+  const uint32_t sbase = smem_u32(sm);
+  const Geo q = chunk_geo(a, blockIdx.x);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t cidx = (q.b * a.nheads + q.h) * a.nchunks + q.c;
+  float* S = w.G + cidx * (int64_t)kN * kP;  // turned into G_c by the state pass
+  float* D = w.D + cidx * (int64_t)kN * kP;
+  float* su = w.sums + cidx * (1 + kK);
+  if (q.nt <= 0) {  // past a short packed sequence: both states pass unchanged
+    for (int e = tid; e < kN * kP / 4; e += kTh) {
+      reinterpret_cast<float4*>(S)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      reinterpret_cast<float4*>(D)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int k = tid; k < 1 + kK; k += kTh) su[k] = 0.f;
+    return;
+  }
+  if ((sbase & 1023u) != 0) {
+    if (tid == 0 && a.status) atomicCAS(a.status, 0, (int)M3_ERR_CUDA);
+    return;
+  }
+  float* phi = reinterpret_cast<float*>(sm + L::SMALL);
+  float* lcum = phi + Q * kK;
+  float* gam = lcum + Q;
+  float* del = gam + Q;
+  float* dts = del + Q;
+  float* s_w = dts + Q;  // w_s, the row scale of Bt
+  float* s_e = s_w + Q;  // exp(Lam_t), the row scale of Ct
+  uint64_t* bar = reinterpret_cast<uint64_t*>(s_e + Q);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar + 1);
+
+  chunk_prep(a, q, lcum, gam, del, dts, phi);
+  const float lend = lcum[q.nt - 1];
+  for (int i = tid; i < Q; i += kTh) {
+    s_w[i] = i < q.nt ? expf(lend - lcum[i]) * del[i] : 0.f;
+    s_e[i] = i < q.nt ? expf(lcum[i]) : 0.f;
+  }
+  __syncthreads();
+  stage_bc<R>(a, q, phi, s_w, s_e, sm + L::WB, sm + L::EC);
+  stage_xdy<R>(a, g, q, sm + L::XS, sm + L::DYS);
+  fence_async_smem();
+  if (warp == 0) {
+    tmem_alloc(s_tmem, 128);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *s_tmem;
+  if (tid == 0) {
+    // M = 128 state rows (MN-major A: rows i of the chunk are K), N = 64
+    const uint32_t id = idesc_bf16(kN, kP, 1, 1);
+    const uint64_t dWB = sw128_desc(sbase + L::WB, kOPB, 1024);
+    const uint64_t dEC = sw128_desc(sbase + L::EC, kOPB, 1024);
+    const uint64_t dXS = sw128_desc(sbase + L::XS, kOPB, 1024);
+    const uint64_t dDY = sw128_desc(sbase + L::DYS, kOPB, 1024);
+#pragma unroll
+    for (int ks = 0; ks < kM / 16; ++ks)
+      mma_bf16_ss(tm, dadd(dWB, ks * 2048), dadd(dXS, ks * 2048), id, ks != 0);
+#pragma unroll
+    for (int ks = 0; ks < kM / 16; ++ks)
+      mma_bf16_ss(tm + kP, dadd(dEC, ks * 2048), dadd(dDY, ks * 2048), id, ks != 0);
+    mma_commit(bar);
+  }
+  const bool ok = (tid == 0) ? wait_mma(bar, 0, a.status) : true;
+  const bool aborted = __syncthreads_or(!ok);
+  tc_fence_after();
+  if (!aborted) {
+    // warps 0-3: S_c, warps 4-7: D_c; thread row n = 32 (warp % 4) + lane
+    const int qd = warp & 3, which = warp >> 2;
+    const int n = 32 * qd + lane;
+    float* dst = (which ? D : S) + (int64_t)n * kP;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t v[32];
+      tmem_ld32(tm + ((uint32_t)(32 * qd) << 16) + which * kP + 32 * half, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4*>(dst + 32 * half + j) =
+            make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                        __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+    }
+    if (tid == 0) su[0] = lend;
+    for (int k = tid; k < kK; k += kTh) su[1 + k] = phi[(q.nt - 1) * kK + k];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tm, 128);
+}
+
+// ---- step 3: per-chunk gradients ---------------------------------------------
+// Shared memory (bytes):
+//   CT, BT   Ct, Bt: 2 K-major blocks each
+//   XS, DYS  x, dy: 1 block each
+//   GM       G_c in bf16, [128 rows n][64 p]; after phase A: M o S, M o DX
+//   DG       dGhat in bf16, [128 rows n][64 p]; after phase A: dPhi, fp32 [Q][K]
+//   SMALL    Phi [Q][K], per-token arrays, end-angle cos / sin, barriers
+struct ChunkTc {
+  static constexpr int CT = 0, BT = 2 * kOPB, XS = 4 * kOPB, DYS = 5 * kOPB;
+  static constexpr int GM = 6 * kOPB, MS = GM, MD = GM + kOPB;
+  static constexpr int DG = GM + kN * 128;
+  static constexpr int SMALL = DG + kN * 128;
+  static constexpr int NTOK = 12;  // per-token float arrays
+  static constexpr int bytes(int Q) {
+    return SMALL + (Q * kK + NTOK * Q + kK + 2 * kK + 32) * 4 + 32;
+  }
+  // TMEM columns
+  static constexpr int S_COL = 0, DX_COL = 64, AX_COL = 128, AC_COL = 192, AB_COL = 320;
+  static constexpr int TMEM_COLS = 512;
+};
+
+template <int R>
+__global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, const BwdArgs g,
+                                                              const BwdWs w) {
+  constexpr int Q = kM / R;
+  using L = ChunkTc;
+  extern __shared__ __align__(1024) uint8_t sm[];
+  const uint32_t sbase = smem_u32(sm);
+  const Geo q = chunk_geo(a, blockIdx.x);
+  const int nt = q.nt;
+  if (nt <= 0) return;  // uniform over the block
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if ((sbase & 1023u) != 0) {
+    if (tid == 0 && a.status) atomicCAS(a.status, 0, (int)M3_ERR_CUDA);
+    return;
+  }
+  const int64_t H = a.nheads;
+  float* phi = reinterpret_cast<float*>(sm + L::SMALL);
+  float* lcum = phi + Q * kK;
+  float* gam = lcum + Q;
+  float* del = gam + Q;
+  float* dts = del + Q;
+  float* lg = dts + Q;     // Lam_t log2(e)
+  float* wv = lg + Q;      // w_s
+  float* beta = wv + Q;    // x_s . (Bt dGhat)_s over the ranks
+  float* dLam = beta + Q;
+  float* dgam = dLam + Q;
+  float* ddel = dgam + Q;
+  float* colF = ddel + Q;  // sum over t > s of F_ts
+  float* thT = colF + Q;   // sum_k theta_k d(dt theta)_k
+  float* s_pe = thT + Q;   // the outgoing rotation's angle gradient, [K]
+  float* ecs = s_pe + kK;  // cos, sin of Phi_end, [K][2]
+  float* red = ecs + 2 * kK;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 32);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2);
+  float* dPhi = reinterpret_cast<float*>(sm + L::DG);  // after phase A
+
+  // ---- prologue: prefix sums, operands (before TMEM is taken) ----------------
+  chunk_prep(a, q, lcum, gam, del, dts, phi);
+  const int t1 = nt - 1;
+  const float lam_end = lcum[t1];
+  for (int i = tid; i < Q; i += kTh) {
+    wv[i] = (i < nt) ? expf(lam_end - lcum[i]) * del[i] : 0.f;
+    lg[i] = (i < nt) ? lcum[i] * kL2E : 0.f;
+    beta[i] = dLam[i] = dgam[i] = ddel[i] = colF[i] = thT[i] = 0.f;
+  }
+  for (int k = tid; k < kK; k += kTh) {
+    float sn, cs;
+    sincos_r(phi[t1 * kK + k], &sn, &cs);
+    ecs[2 * k] = cs;
+    ecs[2 * k + 1] = sn;
+  }
+  __syncthreads();
+  stage_bc<R>(a, q, phi, nullptr, nullptr, sm + L::BT, sm + L::CT);
+  stage_xdy<R>(a, g, q, sm + L::XS, sm + L::DYS);
+  const int64_t cidx = (q.b * H + q.h) * a.nchunks + q.c;
+  const float* Gc = w.G + cidx * (int64_t)kN * kP;  // state entering the chunk
+  const float* Do = w.D + cidx * (int64_t)kN * kP;  // adjoint of the state leaving it
+  const float* Gn = (q.c + 1 < a.nchunks) ? Gc + (int64_t)kN * kP  // next chunk's start state
+                                          : w.fin + (q.b * H + q.h) * (int64_t)kN * kP;
+  // G_c and dGhat = Rot(-Phi_end) dG_c+1 by row pairs (2k, 2k+1) and 8 columns;
+  // <dGhat, G_c> and the outgoing rotation's angle gradient in fp32
+  float dgg = 0.f;
+  for (int e = tid; e < kK * 8; e += kTh) {
+    const int k = e >> 3, c8 = e & 7;
+    float g0[8], g1[8], o0[8], o1[8], n0[8], n1[8];
+    ld8_f32(Gc + (2 * k) * kP + 8 * c8, g0);
+    ld8_f32(Gc + (2 * k + 1) * kP + 8 * c8, g1);
+    ld8_f32(Do + (2 * k) * kP + 8 * c8, o0);
+    ld8_f32(Do + (2 * k + 1) * kP + 8 * c8, o1);
+    ld8_f32(Gn + (2 * k) * kP + 8 * c8, n0);
+    ld8_f32(Gn + (2 * k + 1) * kP + 8 * c8, n1);
+    const float ce = ecs[2 * k], se = ecs[2 * k + 1];
+    float h0[8], h1[8], cr = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      h0[j] = ce * o0[j] + se * o1[j];
+      h1[j] = -se * o0[j] + ce * o1[j];
+      dgg = fmaf(h0[j], g0[j], fmaf(h1[j], g1[j], dgg));
+      cr = fmaf(o1[j], n0[j], fmaf(-o0[j], n1[j], cr));
+    }
+    *reinterpret_cast<uint4*>(sm + L::GM + sw128_off(2 * k, c8)) = pack8(g0);
+    *reinterpret_cast<uint4*>(sm + L::GM + sw128_off(2 * k + 1, c8)) = pack8(g1);
+    *reinterpret_cast<uint4*>(sm + L::DG + sw128_off(2 * k, c8)) = pack8(h0);
+    *reinterpret_cast<uint4*>(sm + L::DG + sw128_off(2 * k + 1, c8)) = pack8(h1);
+    // the 8 column groups of pair k are 8 consecutive lanes
+    cr += __shfl_xor_sync(0xffffffffu, cr, 1);
+    cr += __shfl_xor_sync(0xffffffffu, cr, 2);
+    cr += __shfl_xor_sync(0xffffffffu, cr, 4);
+    if (c8 == 0) s_pe[k] = cr;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) dgg += __shfl_xor_sync(0xffffffffu, dgg, off);
+  if (lane == 0) red[warp] = dgg;
+  fence_async_smem();
+  if (warp == 0) {
+    tmem_alloc(s_tmem, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bars, 1);
+    mbar_init(bars + 1, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *s_tmem;
+
+  const uint64_t kCT = sw128_desc(sbase + L::CT, 16, 1024), mCT = sw128_desc(sbase + L::CT, kOPB, 1024);
+  const uint64_t kBT = sw128_desc(sbase + L::BT, 16, 1024), mBT = sw128_desc(sbase + L::BT, kOPB, 1024);
+  const uint64_t kXS = sw128_desc(sbase + L::XS, 16, 1024);
+  const uint64_t kDY = sw128_desc(sbase + L::DYS, 16, 1024), mDY = sw128_desc(sbase + L::DYS, kOPB, 1024);
+  const uint64_t kGM = sw128_desc(sbase + L::GM, 16, 1024);
+  const uint64_t kDG = sw128_desc(sbase + L::DG, 16, 1024), mDG = sw128_desc(sbase + L::DG, kN * 128, 1024);
+  const uint64_t kMD = sw128_desc(sbase + L::MD, 16, 1024), mMD = sw128_desc(sbase + L::MD, kOPB, 1024);
+  const uint64_t mMS = sw128_desc(sbase + L::MS, kOPB, 1024);
+
+  // ---- phase A ----------------------------------------------------------------
+  if (tid == 0) {
+    const uint32_t id64 = idesc_bf16(kM, 64, 0, 0), id128 = idesc_bf16(kM, 128, 0, 0);
+    const uint32_t idAX = idesc_bf16(kM, kP, 0, 1);
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {  // S = Ct Bt^T, K = N
+        const uint32_t o = kb * kOPB + k4 * 32;
+        mma_bf16_ss(tm + L::S_COL, dadd(kCT, o), dadd(kBT, o), id64, (kb | k4) != 0);
+      }
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4)  // DX = dY X^T, K = P
+      mma_bf16_ss(tm + L::DX_COL, dadd(kDY, k4 * 32), dadd(kXS, k4 * 32), id64, k4 != 0);
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4)  // AX = Bt dGhat, K = N (dGhat MN-major)
+        mma_bf16_ss(tm + L::AX_COL, dadd(kBT, kb * kOPB + k4 * 32), dadd(mDG, (kb * 4 + k4) * 2048),
+                    idAX, (kb | k4) != 0);
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) {  // AC = dY G^T, AB = X dGhat^T, K = P
+      mma_bf16_ss(tm + L::AC_COL, dadd(kDY, k4 * 32), dadd(kGM, k4 * 32), id128, k4 != 0);
+      mma_bf16_ss(tm + L::AB_COL, dadd(kXS, k4 * 32), dadd(kDG, k4 * 32), id128, k4 != 0);
+    }
+    mma_commit(bars);
+  }
+  bool ok = (tid == 0) ? wait_mma(bars, 0, a.status) : true;
+  bool aborted = __syncthreads_or(!ok);
+  tc_fence_after();
+
+  // Thread layout over 64-row accumulators: warp w reads TMEM lanes
+  // 32 (w % 4) .. +15 (rows 16 (w % 4) .. +15); warps w and w + 4 split the
+  // columns (hh = w / 4), and the half-warps split a warp's columns again.
+  const int qd = warp & 3, hh = warp >> 2, hl = lane >> 4;
+  const int rho = 16 * qd + (lane & 15);
+  const int tr = rho / R, rr = rho % R;
+  const bool trow = tr < nt;
+  const uint32_t lb = tm + ((uint32_t)(32 * qd) << 16);
+  const int c64 = 32 * hh + 16 * hl;  // this thread's 16 columns of a 64-column accumulator
+
+  if (!aborted) {
+    // (1) the mask, its gradients and the masked scores
+    {
+      uint32_t sv[16], dv[16];
+      tmem_ld16x2<16>(lb + L::S_COL + 32 * hh, sv);
+      tmem_ld16x2<16>(lb + L::DX_COL + 32 * hh, dv);
+      tmem_ld_wait();
+      const float lgt = trow ? lg[tr] : 0.f;
+      float rowacc = 0.f, dg = 0.f, colv[16];
+      uint32_t pks[8], pkd[8];
+#pragma unroll
+      for (int jj = 0; jj < 16; jj += 2) {
+        float msv[2], mdv[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int s = (c64 + jj + u) / R;
+          const float sv_ = __uint_as_float(sv[jj + u]), dv_ = __uint_as_float(dv[jj + u]);
+          const float p = sv_ * dv_;
+          float m = 0.f, F = 0.f;
+          if (trow) {
+            if (s < tr) {
+              const float e = ex2(lgt - lg[s]);
+              F = p * e;
+              rowacc = fmaf(F, del[s], rowacc);
+              m = e * del[s];
+            } else if (s == tr) {
+              dg += p;
+              m = gam[tr];
+            }
+          }
+          colv[jj + u] = F;
+          msv[u] = sv_ * m;
+          mdv[u] = dv_ * m;
+        }
+        pks[jj / 2] = pack_bf16(msv[0], msv[1]);
+        pkd[jj / 2] = pack_bf16(mdv[0], mdv[1]);
+      }
+      *reinterpret_cast<uint4*>(sm + L::MS + sw128_off(rho, c64 / 8)) = make_uint4(pks[0], pks[1], pks[2], pks[3]);
+      *reinterpret_cast<uint4*>(sm + L::MS + sw128_off(rho, c64 / 8 + 1)) = make_uint4(pks[4], pks[5], pks[6], pks[7]);
+      *reinterpret_cast<uint4*>(sm + L::MD + sw128_off(rho, c64 / 8)) = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+      *reinterpret_cast<uint4*>(sm + L::MD + sw128_off(rho, c64 / 8 + 1)) = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
+      // row terms: the two half-warps hold the same rows
+      rowacc += __shfl_xor_sync(0xffffffffu, rowacc, 16);
+      dg += __shfl_xor_sync(0xffffffffu, dg, 16);
+      if (hl == 0 && trow) {
+        if (rowacc != 0.f) atomicAdd(dLam + tr, rowacc);
+        if (dg != 0.f) atomicAdd(dgam + tr, dg);
+      }
+      // column terms: reduce the 16 rows of a half-warp, one column per lane
+#pragma unroll
+      for (int off = 8; off >= 1; off >>= 1) {
+        const bool up = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < off; ++i) {
+          const float send = up ? colv[i] : colv[i + off];
+          const float keep = up ? colv[i + off] : colv[i];
+          colv[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      const int sc_ = (c64 + (lane & 15)) / R;
+      if (sc_ < nt && colv[0] != 0.f) atomicAdd(colF + sc_, colv[0]);
+    }
+    // (2) beta from AX = Bt dGhat; AX *= w_s
+    {
+      uint32_t v[16];
+      tmem_ld16x2<16>(lb + L::AX_COL + 32 * hh, v);
+      tmem_ld_wait();
+      float xr[16];
+      ld16_sw(sm + L::XS, rho, c64, xr);
+      float bt = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) bt = fmaf(xr[j], __uint_as_float(v[j]), bt);
+      bt += __shfl_xor_sync(0xffffffffu, bt, 16);
+      if (hl == 0 && trow) atomicAdd(beta + tr, bt);
+      const float ws = trow ? wv[tr] : 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * ws);
+      tmem_st16x2<16>(lb + L::AX_COL + 32 * hh, v);
+    }
+    // (3) AC = dY G^T: the exp(Lam_t) term of dLam; AC *= exp(Lam_t).
+    // (4) AB = X dGhat^T: AB *= w_s.  128 columns: two 32-column loads per warp.
+    {
+      const float el = trow ? ex2(lg[tr]) : 0.f;
+      const float ws = trow ? wv[tr] : 0.f;
+      float cdot = 0.f;
+#pragma unroll
+      for (int pc = 0; pc < 2; ++pc) {
+        const int col = 64 * hh + 32 * pc;  // the warp's 32 columns; this thread's 16 from col + 16 hl
+        const int n0 = col + 16 * hl;
+        uint32_t v[16];
+        tmem_ld16x2<16>(lb + L::AC_COL + col, v);
+        tmem_ld_wait();
+        float cr[16];
+        ld16_sw(sm + L::CT + (n0 >> 6) * kOPB, rho, n0 & 63, cr);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float x = __uint_as_float(v[j]);
+          cdot = fmaf(cr[j], x, cdot);
+          v[j] = __float_as_uint(x * el);
+        }
+        tmem_st16x2<16>(lb + L::AC_COL + col, v);
+        uint32_t u[16];
+        tmem_ld16x2<16>(lb + L::AB_COL + col, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) u[j] = __float_as_uint(__uint_as_float(u[j]) * ws);
+        tmem_st16x2<16>(lb + L::AB_COL + col, u);
+      }
+      cdot += __shfl_xor_sync(0xffffffffu, cdot, 16);
+      if (hl == 0 && trow) atomicAdd(dLam + tr, el * cdot);
+    }
+    // dPhi goes over dGhat, which phase A has read
+    for (int i = tid; i < Q * kK; i += kTh) dPhi[i] = 0.f;
+    tmem_st_wait();
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  // ---- phase B ----------------------------------------------------------------
+  if (!aborted && tid == 0) {
+    const uint32_t idC = idesc_bf16(kM, 128, 0, 1), idB = idesc_bf16(kM, 128, 1, 1);
+    const uint32_t idX = idesc_bf16(kM, kP, 1, 1);
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) {  // K = the chunk's 64 rows
+      // AC += (M o DX) Bt: A K-major [t][s], B MN-major (rows s, N = n)
+      mma_bf16_ss(tm + L::AC_COL, dadd(kMD, k4 * 32), dadd(mBT, k4 * 2048), idC, 1);
+      // AB += (M o DX)^T Ct: A MN-major (rows t, M = s), B MN-major (rows t, N = n)
+      mma_bf16_ss(tm + L::AB_COL, dadd(mMD, k4 * 2048), dadd(mCT, k4 * 2048), idB, 1);
+      // AX += (M o S)^T dY
+      mma_bf16_ss(tm + L::AX_COL, dadd(mMS, k4 * 2048), dadd(mDY, k4 * 2048), idX, 1);
+    }
+    mma_commit(bars + 1);
+  }
+  if (!aborted) {
+    ok = (tid == 0) ? wait_mma(bars + 1, 0, a.status) : true;
+    aborted = __syncthreads_or(!ok);
+    tc_fence_after();
+  }
+
+  // ---- epilogue: dC, dB (rotated back), their angle gradients, dx ----------------
+  if (!aborted) {
+    const int64_t tok = q.base + q.t0 + tr;
+    const int64_t bcb = (tok * a.ngroups + q.g) * R * kN + (int64_t)rr * kN;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {  // 0: AC -> dC with Ct, 1: AB -> dB with Bt
+      const int acol = which ? L::AB_COL : L::AC_COL;
+      const uint8_t* opnd = sm + (which ? L::BT : L::CT);
+      float* gout = which ? g.dB : g.dC;
+#pragma unroll
+      for (int pc = 0; pc < 2; ++pc) {
+        const int col = 64 * hh + 32 * pc;
+        const int n0 = col + 16 * hl;
+        uint32_t v[16];
+        tmem_ld16x2<16>(lb + acol + col, v);
+        tmem_ld_wait();
+        if (trow) {
+          float ov[16];
+          ld16_sw(opnd + (n0 >> 6) * kOPB, rho, n0 & 63, ov);
+          float res[16];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int k = n0 / 2 + j;
+            const float d0 = __uint_as_float(v[2 * j]), d1 = __uint_as_float(v[2 * j + 1]);
+            atomicAdd(dPhi + tr * kK + k, d0 * ov[2 * j + 1] - d1 * ov[2 * j]);
+            float sn, cs;
+            sincos_r(phi[tr * kK + k], &sn, &cs);
+            res[2 * j] = cs * d0 - sn * d1;  // Rot(Phi_t) of the rotated-frame gradient
+            res[2 * j + 1] = sn * d0 + cs * d1;
+          }
+#pragma unroll
+          for (int j = 0; j < 16; j += 4)
+            atomicAdd(reinterpret_cast<float4*>(gout + bcb + n0 + j),
+                      make_float4(res[j], res[j + 1], res[j + 2], res[j + 3]));
+        }
+      }
+    }
+    {  // dX
+      uint32_t v[16];
+      tmem_ld16x2<16>(lb + L::AX_COL + 32 * hh, v);
+      tmem_ld_wait();
+      if (trow) {
+        float* dxo = g.dx + ((q.base + q.t0 + tr) * H + q.h) * R * kP + (int64_t)rr * kP + c64;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+          *reinterpret_cast<float4*>(dxo + j) =
+              make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                          __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tm, L::TMEM_COLS);
+  if (aborted) return;
+
+  // ---- the scalar gradients (as on the CUDA cores) ----------------------------
+  for (int k = tid; k < kK; k += kTh) dPhi[t1 * kK + k] += s_pe[k];
+  for (int u = tid; u < nt; u += kTh) {
+    float dl = -wv[u] * beta[u] - del[u] * colF[u];
+    if (u == t1) {
+      float dsum = 0.f, wb = 0.f;
+      for (int i = 0; i < kTh / 32; ++i) dsum += red[i];
+      for (int s = 0; s < nt; ++s) wb = fmaf(wv[s], beta[s], wb);
+      dl += wb + expf(lam_end) * dsum;
+    }
+    dLam[u] += dl;
+    ddel[u] += expf(lam_end - lcum[u]) * beta[u] + colF[u];
+  }
+  __syncthreads();
+  // suffix sums of dPhi over the chunk's tokens are d(dt theta)
+  for (int k = tid; k < kK; k += kTh) {
+    float run = 0.f;
+    for (int u = nt - 1; u >= 0; --u) {
+      run += dPhi[u * kK + k];
+      dPhi[u * kK + k] = run;
+    }
+  }
+  __syncthreads();
+  {
+    constexpr int K4 = kK / 4;  // 16 float4 groups per token
+    for (int e0 = 0; e0 < nt * K4; e0 += kTh) {
+      const int e = e0 + tid;
+      float part = 0.f;
+      int u = 0;
+      if (e < nt * K4) {
+        u = e / K4;
+        const int k4 = e % K4;
+        const int64_t to = ((q.base + q.t0 + u) * a.tgroups + q.tg) * kK + 4 * k4;
+        const float4 dp = *reinterpret_cast<const float4*>(dPhi + u * kK + 4 * k4);
+        const float d = dts[u];
+        atomicAdd(reinterpret_cast<float4*>(g.dtheta + to),
+                  make_float4(d * dp.x, d * dp.y, d * dp.z, d * dp.w));
+        const float4 th = __ldg(reinterpret_cast<const float4*>(a.theta + to));
+        part = th.x * dp.x + th.y * dp.y + th.z * dp.z + th.w * dp.w;
+      }
+#pragma unroll
+      for (int off = 1; off < K4; off <<= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      if (e < nt * K4 && (tid & (K4 - 1)) == 0) atomicAdd(thT + u, part);
+    }
+  }
+  __syncthreads();
+  // per token: dt, A, lam (gamma = lam dt, eps = (1 - lam) dt, delta_s = gamma_s + eps_s+1)
+  for (int u = tid; u < nt; u += kTh) {
+    float run = 0.f;
+    for (int t = u; t < nt; ++t) run += dLam[t];
+    const int64_t o = (q.base + q.t0 + u) * H + q.h;
+    const float dt = dts[u], lam = __ldg(a.lam + o), Av = __ldg(a.A + o);
+    const float dgv = dgam[u] + ddel[u];
+    const float de = (u > 0) ? ddel[u - 1] : 0.f;  // eps_u through delta_u-1 (this chunk)
+    g.dA[o] = dt * run;
+    atomicAdd(g.ddt + o, Av * run + thT[u] + lam * dgv + (1.f - lam) * de);
+    atomicAdd(g.dlam + o, dt * (dgv - de));
+    if (u == t1 && q.t0 + nt < q.len) {  // the next token's eps, through delta_end
+      const int64_t on = o + H;
+      const float lamn = __ldg(a.lam + on), dtn = __ldg(a.dt + on);
+      atomicAdd(g.ddt + on, (1.f - lamn) * ddel[u]);
+      atomicAdd(g.dlam + on, -dtn * ddel[u]);
+    }
+  }
+}
+
+template <typename Kern>
+cudaError_t set_smem(Kern k, size_t smem) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+}
+
+template <int R>
+cudaError_t sums_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaStream_t st) {
+  const size_t smem = SumsSmem::bytes(kM / R);
+  cudaError_t e = set_smem(bwd_tc_sums_kernel<R>, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)f.nchunks, (unsigned)f.nheads, (unsigned)f.batch);
+  bwd_tc_sums_kernel<R><<<grid, kTh, smem, st>>>(f, g, w);
+  return cudaGetLastError();
+}
+
+template <int R>
+cudaError_t chunk_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaStream_t st) {
+  const size_t smem = ChunkTc::bytes(kM / R);
+  cudaError_t e = set_smem(bwd_tc_chunk_kernel<R>, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)f.nchunks, (unsigned)f.nheads, (unsigned)f.batch);
+  bwd_tc_chunk_kernel<R><<<grid, kTh, smem, st>>>(f, g, w);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool bwd_tc_shape(const ScanArgs& a) {
+  return a.bf16 && a.N == kN && a.P == kP &&
+         (a.R == 1 || a.R == 2 || a.R == 4 || a.R == 8);
+}
+
+cudaError_t bwd_tc_sums_launch(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaStream_t st) {
+  switch (f.R) {
+    case 1: return sums_r<1>(f, g, w, st);
+    case 2: return sums_r<2>(f, g, w, st);
+    case 4: return sums_r<4>(f, g, w, st);
+    case 8: return sums_r<8>(f, g, w, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t bwd_tc_chunk_launch(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaStream_t st) {
+  switch (f.R) {
+    case 1: return chunk_r<1>(f, g, w, st);
+    case 2: return chunk_r<2>(f, g, w, st);
+    case 4: return chunk_r<4>(f, g, w, st);
+    case 8: return chunk_r<8>(f, g, w, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace m3

@@ -279,13 +279,15 @@ def bwd_workspace_size(shape: Shape) -> int:
 
 
 def m3_scan_bwd(x, dt, A, lam, theta, B, C, dy, chunk: int = 64, h0=None, B_prev=None,
-                x_prev=None, d_final=None, *, want_dh0=True, workspace=None, stream=None):
+                x_prev=None, d_final=None, *, want_dh0=True, workspace=None, simt=False,
+                stream=None):
     """Backward of m3_scan_fwd: gradients of sum(y * dy) + sum(final * d_final)
     with respect to every input.  dy has x's dtype, or fp32 (read unrounded).
     Returns a dict of fp32 tensors: x, dt, A, lam, theta, B, C, and h0 (when
     want_dh0), B_prev and x_prev (when B_prev is given), each in its input's
-    layout."""
-    shape = scan_shape(x, B, chunk, False, theta)
+    layout.  bf16 io at N = 128, P = 64 runs on the tensor cores (bf16
+    operands) unless simt is set (CUDA cores, fp32 throughout)."""
+    shape = scan_shape(x, B, chunk, simt, theta)
     shape.flags |= dy_flag(dy, x)
     dev, f32 = x.device, torch.float32
     g = {"x": torch.empty(x.shape, dtype=f32, device=dev),
@@ -316,9 +318,10 @@ def m3_scan_bwd(x, dt, A, lam, theta, B, C, dy, chunk: int = 64, h0=None, B_prev
 
 def m3_scan_bwd_varlen(cu_seqlens, x, dt, A, lam, theta, B, C, dy, chunk: int = 64, h0=None,
                        B_prev=None, x_prev=None, d_final=None, *, max_seqlen=None,
-                       want_dh0=True, workspace=None, stream=None):
+                       want_dh0=True, workspace=None, simt=False, stream=None):
     """Backward of m3_scan_fwd_varlen (packed tensors without a batch
-    dimension, as there).  Returns the gradient dict of m3_scan_bwd."""
+    dimension, as there).  Returns the gradient dict of m3_scan_bwd; simt as
+    there."""
     if cu_seqlens.dtype != torch.int32:
         raise TypeError("cu_seqlens must be int32")
     S = cu_seqlens.numel() - 1
@@ -326,7 +329,7 @@ def m3_scan_bwd_varlen(cu_seqlens, x, dt, A, lam, theta, B, C, dy, chunk: int = 
     G, N = B.shape[1], B.shape[3]
     if max_seqlen is None:
         max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item()) if S > 0 else 0
-    shape = make_shape(S, max_seqlen, H, G, P, N, R, chunk, x.dtype, False)
+    shape = make_shape(S, max_seqlen, H, G, P, N, R, chunk, x.dtype, simt)
     shape.flags |= theta_flag(theta.shape[1], G, H) | dy_flag(dy, x)
     dev, f32 = x.device, torch.float32
     g = {k: torch.empty(v.shape, dtype=f32, device=dev)

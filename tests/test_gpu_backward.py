@@ -2,10 +2,12 @@
 gradient oracle (fp64 autograd through the token recurrence, pinned in
 test_grad_oracle.py).
 
-Bar, for every gradient tensor separately: max |err| / max |ref| <= 1e-4 for
-fp32 io.  bf16 io shares the rounded inputs with the oracle and computes in
-fp32 as well, so it is held to the same 1e-4 (the io bar of 2e-2 applies to
-rounded outputs; these gradients are fp32).
+Bars, for every gradient tensor separately, as max |err| / max |ref|:
+  - CUDA-core path (fp32 io, other shapes, or simt): 1e-4.  bf16 io shares the
+    rounded inputs with the oracle and computes in fp32 as well, so it is held
+    to the same 1e-4.
+  - tensor-core path (bf16 io at N = 128, P = 64, the default there): its MMA
+    operands are rounded to bf16, so BWD_TC_BAR (parity_helpers states why).
 """
 import numpy as np
 import pytest
@@ -14,7 +16,7 @@ import torch
 from oracle import m3_grad
 from selective_state_space_exp_b200 import inputs as I
 from selective_state_space_exp_b200 import m3
-from parity_helpers import need_gpu, rel_err, to_dev
+from parity_helpers import BWD_TC_BAR, need_gpu, rel_err, to_dev
 
 pytestmark = pytest.mark.gpu
 BAR = 1e-4
@@ -38,11 +40,17 @@ def case(batch=2, L=150, H=4, P=16, N=16, R=1, G=1, io="f32", decay="slow", h0=T
     return inp
 
 
-def compare(inp, chunk=64, with_final=True):
+def on_tc(inp, simt=False):
+    """Whether m3_scan_bwd takes the tensor-core path for these inputs."""
+    x, B = inp["x"], inp["B"]
+    return not simt and x.dtype == torch.bfloat16 and B.shape[4] == 128 and x.shape[4] == 64
+
+
+def compare(inp, chunk=64, with_final=True, simt=False):
     g = to_dev(inp)
     got = m3.m3_scan_bwd(g["x"], g["dt"], g["A"], g["lam"], g["theta"], g["B"], g["C"],
                          g["dy"], chunk, g.get("h0"), g.get("B_prev"), g.get("x_prev"),
-                         g["d_final"] if with_final else None)
+                         g["d_final"] if with_final else None, simt=simt)
     assert m3.m3_stream_status() == 0
     _, _, ref = m3_grad.scan_grads(*[inp.get(k) for k in m3_grad.NAMES], dy=inp["dy"],
                                    d_final=inp["d_final"] if with_final else None)
@@ -58,8 +66,9 @@ def compare(inp, chunk=64, with_final=True):
                                       h0=np.zeros(tuple(got["h0"].shape)), dy=inp["dy"],
                                       d_final=inp["d_final"] if with_final else None)
         errs["h0"] = rel_err(got["h0"].cpu().numpy(), r0["h0"])
-    bad = {k: v for k, v in errs.items() if not v <= BAR}
-    assert not bad, f"errors above {BAR}: {bad} (all: {errs})"
+    bar = BWD_TC_BAR if on_tc(inp, simt) else BAR
+    bad = {k: v for k, v in errs.items() if not v <= bar}
+    assert not bad, f"errors above {bar}: {bad} (all: {errs})"
     return errs
 
 
@@ -89,24 +98,25 @@ def test_bwd_edge_lengths(L):
     compare(case(batch=1, L=L, H=2, R=2, seed=500 + L))
 
 
-def test_bwd_bf16_layer_shape():
-    """bf16 io at the layer's N = 128, P = 64 (a few chains)."""
-    compare(case(batch=1, L=200, H=2, N=128, P=64, R=4, io="bf16", seed=600))
+@pytest.mark.parametrize("simt", [True, False], ids=["cuda_core", "tcgen05"])
+def test_bwd_bf16_layer_shape(simt):
+    """bf16 io at the layer's N = 128, P = 64 (a few chains), both paths."""
+    compare(case(batch=1, L=200, H=2, N=128, P=64, R=4, io="bf16", seed=600), simt=simt)
 
 
 def test_bwd_bf16_inputs_fp32_dy():
-    """bf16 inputs with an fp32 output gradient (M3_FLAG_DY_F32): dy is read
-    unrounded, so the gradients meet the 1e-4 bar against the oracle run with
-    the same fp32 dy; the same dy rounded to bf16 first misses that bar, so
-    the flag is what keeps the extra precision."""
+    """bf16 inputs with an fp32 output gradient (M3_FLAG_DY_F32), CUDA-core
+    path: dy is read unrounded, so the gradients meet the 1e-4 bar against the
+    oracle run with the same fp32 dy; the same dy rounded to bf16 first misses
+    that bar, so the flag is what keeps the extra precision."""
     inp = case(batch=1, L=200, H=2, N=128, P=64, R=4, io="bf16", seed=610)
     gen = torch.Generator().manual_seed(611)
     inp["dy"] = torch.randn(inp["x"].shape, generator=gen)  # fp32, not rounded
-    compare(inp)
+    compare(inp, simt=True)
     g = to_dev(inp)
     rounded = m3.m3_scan_bwd(g["x"], g["dt"], g["A"], g["lam"], g["theta"], g["B"], g["C"],
                              g["dy"].to(torch.bfloat16), 64, g["h0"], g["B_prev"], g["x_prev"],
-                             g["d_final"])
+                             g["d_final"], simt=True)
     _, _, ref = m3_grad.scan_grads(*[inp.get(k) for k in m3_grad.NAMES], dy=inp["dy"],
                                    d_final=inp["d_final"])
     assert rel_err(rounded["x"].cpu().numpy(), ref["x"]) > BAR
@@ -133,8 +143,9 @@ def test_bwd_chunk_invariant():
             rel_err(outs[0][k].cpu().numpy(), outs[1][k].cpu().numpy()) < 1e-6, k
 
 
+@pytest.mark.parametrize("simt", [False, True], ids=["tcgen05", "cuda_core"])
 @pytest.mark.parametrize("R", [1, 4])
-def test_bwd_full_size_sampled_chains(R):
+def test_bwd_full_size_sampled_chains(R, simt):
     """The bench's backward workload (b=8, L=2048, H=64, N=128, P=64, bf16 io,
     the workload's input recipe), gradients of a seeded sample of (batch, head)
     chains: everything a chain owns (dx, d dt, dA, d lam, dh0) against the
@@ -148,9 +159,10 @@ def test_bwd_full_size_sampled_chains(R):
     dfin = torch.randn(inp["h0"].shape, generator=gen)
     g = to_dev(inp)
     got = m3.m3_scan_bwd(g["x"], g["dt"], g["A"], g["lam"], g["theta"], g["B"], g["C"],
-                         dy.cuda(), 64, g["h0"], None, None, dfin.cuda())
+                         dy.cuda(), 64, g["h0"], None, None, dfin.cuda(), simt=simt)
     assert m3.m3_stream_status() == 0
     got = {k: v.cpu().numpy() for k, v in got.items()}
+    bar = BAR if simt else BWD_TC_BAR
     for c in I.sample_chains(8, 64, 3, seed=11 + R):
         b, h = divmod(c, 64)
         one = {"x": inp["x"][b:b + 1, :, h:h + 1], "dt": inp["dt"][b:b + 1, :, h:h + 1],
@@ -165,7 +177,7 @@ def test_bwd_full_size_sampled_chains(R):
                 "A": rel_err(got["A"][b, :, h], ref["A"][0, :, 0]),
                 "lam": rel_err(got["lam"][b, :, h], ref["lam"][0, :, 0]),
                 "h0": rel_err(got["h0"][b, h], ref["h0"][0, 0])}
-        bad = {k: v for k, v in errs.items() if not v <= BAR}
+        bad = {k: v for k, v in errs.items() if not v <= bar}
         assert not bad, (c, errs)
 
 
@@ -211,3 +223,54 @@ def test_bwd_sequence_split_emulated_on_one_gpu(world, io):
     bar = BAR if io == "f32" else 2e-2
     bad = {k: v for k, v in errs.items() if not v <= bar}
     assert not bad, errs
+
+
+# ---- the tensor-core path (bf16 io, N = 128, P = 64) ----------------------------
+# Chunks of 64 rows: Q = 64 / R tokens.  Every case also runs the CUDA-core
+# path on the same inputs, and the two must agree within the tensor-core bar.
+
+def both_paths(inp, with_final=True):
+    e_tc = compare(inp, with_final=with_final)
+    e_sm = compare(inp, with_final=with_final, simt=True)
+    g = to_dev(inp)
+    outs = [m3.m3_scan_bwd(g["x"], g["dt"], g["A"], g["lam"], g["theta"], g["B"], g["C"],
+                           g["dy"], 64, g.get("h0"), g.get("B_prev"), g.get("x_prev"),
+                           g["d_final"] if with_final else None, simt=s) for s in (False, True)]
+    for k in outs[1]:
+        d = rel_err(outs[0][k].cpu().numpy(), outs[1][k].cpu().numpy())
+        assert d <= BWD_TC_BAR, (k, d)
+    return e_tc, e_sm
+
+
+@pytest.mark.parametrize("R", [1, 2, 4, 8])
+def test_tc_bwd_ranks(R):
+    """Ragged length (150 is not a multiple of 64 / R), h0, previous token,
+    d_final, slow decay so that the adjoint crosses many chunks."""
+    both_paths(case(batch=2, L=150, H=4, N=128, P=64, R=R, io="bf16", seed=1300 + R))
+
+
+@pytest.mark.parametrize("G,tph", [(2, False), (4, False), (1, True), (2, True)])
+def test_tc_bwd_groups_and_angle_rates(G, tph):
+    both_paths(case(batch=1, L=100, H=4, N=128, P=64, R=2, G=G, io="bf16", tph=tph,
+                    seed=1400 + G + 10 * tph))
+
+
+def test_tc_bwd_fast_decay_no_prev_no_final():
+    both_paths(case(batch=2, L=130, H=2, N=128, P=64, R=4, io="bf16", decay="fast", h0=False,
+                    prev=False, seed=1500), with_final=False)
+
+
+@pytest.mark.parametrize("R,L", [(1, 1), (1, 2), (1, 63), (1, 64), (1, 65), (4, 15), (4, 16),
+                                 (4, 17), (8, 9)])
+def test_tc_bwd_edge_lengths(R, L):
+    """Lengths around the chunk (64 / R tokens): one token, a chunk less one,
+    a chunk, a chunk and one."""
+    both_paths(case(batch=1, L=L, H=2, N=128, P=64, R=R, io="bf16", seed=1600 + 100 * R + L))
+
+
+def test_tc_bwd_fp32_dy():
+    """An fp32 dy (M3_FLAG_DY_F32) on the tensor-core path."""
+    inp = case(batch=1, L=120, H=2, N=128, P=64, R=4, io="bf16", seed=1700)
+    gen = torch.Generator().manual_seed(1701)
+    inp["dy"] = torch.randn(inp["x"].shape, generator=gen)
+    compare(inp)

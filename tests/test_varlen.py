@@ -16,7 +16,7 @@ import torch
 import oracle
 from selective_state_space_exp_b200 import inputs as I
 from selective_state_space_exp_b200 import m3
-from parity_helpers import TOL, need_gpu, rel_err, to_dev
+from parity_helpers import BWD_TC_BAR, TOL, need_gpu, rel_err, to_dev
 
 
 def workload(H=2, P=16, N=16, R=1, G=1, chunk=64, io="f32", bc="normal", decay="slow",
@@ -211,12 +211,15 @@ def test_varlen_bench_workload(R):
 # ---- backward of packed batches ------------------------------------------------
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("io,N,P,R", [("f32", 16, 16, 2), ("bf16", 128, 64, 1),
-                                      ("bf16", 128, 64, 4)])
-def test_varlen_backward(io, N, P, R):
+@pytest.mark.parametrize("io,N,P,R,simt", [("f32", 16, 16, 2, False), ("bf16", 128, 64, 1, True),
+                                           ("bf16", 128, 64, 4, True), ("bf16", 128, 64, 1, False),
+                                           ("bf16", 128, 64, 4, False)])
+def test_varlen_backward(io, N, P, R, simt):
     """m3_scan_bwd_varlen on a length mix (0, 1, Q-1, Q, Q+1, the maximum and
     random lengths) against the gradient oracle run sequence by sequence:
-    every gradient within 1e-4 of max |ref|."""
+    every gradient within 1e-4 of max |ref| on the CUDA cores (fp32
+    throughout), within the bf16-operand bar on the tensor cores (bf16 io at
+    N = 128, P = 64 without simt)."""
     need_gpu()
     from oracle import m3_grad
     w = workload(H=2, P=P, N=N, R=R, chunk=64, io=io, bc="rmsnorm" if io == "bf16" else "normal")
@@ -228,11 +231,12 @@ def test_varlen_backward(io, N, P, R):
     g = to_dev(inp)
     got = m3.m3_scan_bwd_varlen(g["cu_seqlens"], g["x"], g["dt"], g["A"], g["lam"], g["theta"],
                                 g["B"], g["C"], dy.cuda(), 64, g["h0"], g["B_prev"],
-                                g["x_prev"], dfin.cuda(), max_seqlen=max(lengths))
+                                g["x_prev"], dfin.cuda(), max_seqlen=max(lengths), simt=simt)
     assert m3.m3_stream_status() == 0
     ref = m3_grad.scan_grads_varlen(inp["cu_seqlens"], inp["x"], inp["dt"], inp["A"],
                                     inp["lam"], inp["theta"], inp["B"], inp["C"], inp["h0"],
                                     inp["B_prev"], inp["x_prev"], dy=dy, d_final=dfin)
     errs = {k: rel_err(got[k].cpu().numpy(), ref[k]) for k in ref}
-    bad = {k: v for k, v in errs.items() if not v <= 1e-4}
+    bar = BWD_TC_BAR if (io == "bf16" and not simt) else 1e-4
+    bad = {k: v for k, v in errs.items() if not v <= bar}
     assert not bad, errs
