@@ -171,10 +171,16 @@ __global__ void __launch_bounds__(512) bwd_sums_kernel(const ScanArgs a, const B
       }
     }
   }
-  // an empty chunk (past a short packed sequence) passes both states unchanged
-  float* su = w.sums + cidx * (1 + K);
-  if (tid == 0) su[0] = q.nt > 0 ? lcum[q.nt - 1] : 0.f;
-  for (int k = tid; k < K; k += nth) su[1 + k] = q.nt > 0 ? phi[(q.nt - 1) * K + k] : 0.f;
+  // the chunk's transition factors: exp(Lam_end), cos and sin of Phi_end; an
+  // empty chunk (past a short packed sequence) passes both states unchanged
+  float* su = w.sums + cidx * (1 + N);
+  if (tid == 0) su[0] = q.nt > 0 ? expf(lcum[q.nt - 1]) : 1.f;
+  for (int k = tid; k < K; k += nth) {
+    float sn = 0.f, cs = 1.f;
+    if (q.nt > 0) sincosf(phi[(q.nt - 1) * K + k], &sn, &cs);
+    su[1 + 2 * k] = cs;
+    su[2 + 2 * k] = sn;
+  }
 }
 
 // ---- step 2: both state passes ---------------------------------------------------
@@ -222,11 +228,12 @@ __global__ void __launch_bounds__(kThreads) bwd_pass_kernel(const ScanArgs a, co
       const int64_t c = c0 + j;
       if (c >= a.nchunks) break;
       const float* S = w.G + (chain0 + c) * (int64_t)N * P;
-      const float* su = w.sums + (chain0 + c) * (1 + K);
+      const float* su = w.sums + (chain0 + c) * (1 + N);
       s0[j] = S[i0];
       s1[j] = S[i1];
-      dec[j] = expf(su[0]);
-      sincosf(su[1 + k], &sn[j], &cs[j]);
+      dec[j] = su[0];
+      cs[j] = su[1 + 2 * k];
+      sn[j] = su[2 + 2 * k];
     }
 #pragma unroll
     for (int j = 0; j < kPipe; ++j) {
@@ -253,11 +260,12 @@ __global__ void __launch_bounds__(kThreads) bwd_pass_kernel(const ScanArgs a, co
       const int64_t c = c0 - j;
       if (c < 0) break;
       const float* Dc = w.D + (chain0 + c) * (int64_t)N * P;
-      const float* su = w.sums + (chain0 + c) * (1 + K);
+      const float* su = w.sums + (chain0 + c) * (1 + N);
       e0[j] = Dc[i0];
       e1[j] = Dc[i1];
-      dec[j] = expf(su[0]);
-      sincosf(su[1 + k], &sn[j], &cs[j]);
+      dec[j] = su[0];
+      cs[j] = su[1 + 2 * k];
+      sn[j] = su[2 + 2 * k];
     }
 #pragma unroll
     for (int j = 0; j < kPipe; ++j) {
@@ -939,20 +947,36 @@ cudaError_t launch_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaSt
 
 }  // namespace
 
+// Workspace of chunking f: chunk states G [b][H][nc][N][P], chunk factors
+// [b][H][nc][1 + N] (exp(Lam_end), then cos, sin of Phi_end per pair), the
+// adjoints D [b][H][nc][N][P] and the final states [b][H][N][P], each 256-byte
+// aligned.
+namespace {
+struct WsSizes {
+  size_t g, sums, d, fin;
+};
+WsSizes ws_sizes(const ScanArgs& f) {
+  const size_t chains = (size_t)f.batch * f.nheads;
+  return {align_up(sizeof(float) * chains * f.nchunks * f.N * f.P, 256),
+          align_up(sizeof(float) * chains * f.nchunks * (1 + f.N), 256),
+          align_up(sizeof(float) * chains * f.nchunks * f.N * f.P, 256),
+          align_up(sizeof(float) * chains * f.N * f.P, 256)};
+}
+}  // namespace
+
 BwdWs bwd_carve(const ScanArgs& f) {
+  const WsSizes z = ws_sizes(f);
   BwdWs w;
-  simt_state_views(f, &w.G, &w.sums);
-  const size_t fwd = simt_scan_workspace(f);
-  const size_t dbytes = align_up(sizeof(float) * f.batch * f.nheads * f.nchunks * f.N * f.P, 256);
-  w.D = reinterpret_cast<float*>(f.ws + fwd);
-  w.fin = reinterpret_cast<float*>(f.ws + fwd + dbytes);
+  w.G = reinterpret_cast<float*>(f.ws);
+  w.sums = reinterpret_cast<float*>(f.ws + z.g);
+  w.D = reinterpret_cast<float*>(f.ws + z.g + z.sums);
+  w.fin = reinterpret_cast<float*>(f.ws + z.g + z.sums + z.d);
   return w;
 }
 
 size_t bwd_ws_bytes(const ScanArgs& f) {
-  return simt_scan_workspace(f) +
-         align_up(sizeof(float) * f.batch * f.nheads * f.nchunks * f.N * f.P, 256) +
-         align_up(sizeof(float) * f.batch * f.nheads * f.N * f.P, 256);
+  const WsSizes z = ws_sizes(f);
+  return z.g + z.sums + z.d + z.fin;
 }
 
 cudaError_t bwd_pass_launch(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaStream_t st) {

@@ -9,7 +9,7 @@ namespace m3 {
 
 struct BwdWs {
   float* G;     // [b][H][nc][N][P] chunk-start states (forward)
-  float* sums;  // [b][H][nc][1 + K] chunk totals (forward)
+  float* sums;  // [b][H][nc][1 + N] chunk factors: exp(Lam_end), (cos, sin) of Phi_end per pair
   float* D;     // [b][H][nc][N][P] D_c, then the adjoint of chunk c's outgoing state
   float* fin;   // [b][H][N][P] final state (forward)
 };

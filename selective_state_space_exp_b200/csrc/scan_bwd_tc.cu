@@ -43,12 +43,13 @@ namespace {
 
 using namespace tc;
 using simt::chunk_geo;
-using simt::chunk_prep;
 using simt::Geo;
 
 constexpr int kN = 128;                 // dstate
 constexpr int kP = 64;                  // headdim
 constexpr int kK = kN / 2;              // rotation pairs
+constexpr int kKP = kK + 1;             // row stride of the per-token angle arrays (odd:
+                                        // 16 rows of one pair fall on 16 banks)
 constexpr int kM = (int)kBwdTcRows;     // rows per chunk
 constexpr int kTh = 256;
 constexpr int kOPB = kM * 128;          // one [64 rows][128 B] operand block
@@ -78,17 +79,6 @@ __device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t bytes) {
   return d + (uint64_t)(bytes >> 4);
 }
 
-// 8 consecutive bf16 values (16 bytes) as floats.
-__device__ __forceinline__ void ld8_bf16(const void* base, int64_t idx, float (&v)[8]) {
-  const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + idx));
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float2 f = unpack_bf16(w[j]);
-    v[2 * j] = f.x;
-    v[2 * j + 1] = f.y;
-  }
-}
 __device__ __forceinline__ void ld8_f32(const float* p, float (&v)[8]) {
   const float4 a = __ldg(reinterpret_cast<const float4*>(p));
   const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
@@ -115,6 +105,83 @@ __device__ __forceinline__ void ld16_sw(const uint8_t* blk, int row, int c0, flo
   }
 }
 
+// Chunk-local prefix sums into shared memory: lcum[Q] (Lam), phi[Q][kKP]
+// (Phi, padded rows), and the per-token gamma, delta, dt.  Each prefix sum
+// (the decay and the K angle pairs) is one warp's inclusive scan over the
+// chunk's tokens, Q / 32 tokens per lane.
+template <int Q>
+__device__ void prep_tc(const ScanArgs& a, const Geo& q, float* lcum, float* gam, float* del,
+                        float* dts, float* phi) {
+  const int64_t H = a.nheads;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < q.nt; i += kTh) {
+    const int64_t bt = q.base + q.t0 + i;
+    const float dt = __ldg(a.dt + bt * H + q.h), lam = __ldg(a.lam + bt * H + q.h);
+    float nxt = 0.f;
+    if (q.t0 + i + 1 < q.len)
+      nxt = (1.f - __ldg(a.lam + (bt + 1) * H + q.h)) * __ldg(a.dt + (bt + 1) * H + q.h);
+    dts[i] = dt;
+    gam[i] = lam * dt;
+    del[i] = lam * dt + nxt;
+    lcum[i] = dt * __ldg(a.A + bt * H + q.h);
+  }
+  {  // the chunk's angle rates: every load issued before the first store
+    constexpr int PER = (Q * kK + kTh - 1) / kTh;
+    float th[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int e = tid + j * kTh, i = e / kK, k = e % kK;
+      th[j] = (e < q.nt * kK) ? __ldg(a.theta + ((q.base + q.t0 + i) * a.tgroups + q.tg) * kK + k)
+                              : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int e = tid + j * kTh;
+      if (e < q.nt * kK) phi[(e / kK) * kKP + e % kK] = th[j];
+    }
+  }
+  __syncthreads();
+  // column c of warp w: c = w + 8 j; the warp's columns are scanned together
+  constexpr int TPL = Q > 32 ? Q / 32 : 1;  // tokens per lane
+  constexpr int NW = kTh / 32, CPW = (kK + NW) / NW;  // columns 0..kK (kK: the decay)
+  float v[CPW][TPL], run[CPW], incl[CPW];
+#pragma unroll
+  for (int j = 0; j < CPW; ++j) {
+    const int col = warp + NW * j;
+    run[j] = 0.f;
+#pragma unroll
+    for (int u = 0; u < TPL; ++u) {
+      const int t = lane * TPL + u;
+      float x = 0.f;
+      if (col <= kK && t < q.nt) x = col < kK ? dts[t] * phi[t * kKP + col] : lcum[t];
+      run[j] += x;
+      v[j][u] = run[j];
+    }
+    incl[j] = run[j];
+  }
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1)
+#pragma unroll
+    for (int j = 0; j < CPW; ++j) {
+      const float y = __shfl_up_sync(0xffffffffu, incl[j], off);
+      if (lane >= off) incl[j] += y;
+    }
+#pragma unroll
+  for (int j = 0; j < CPW; ++j) {
+    const int col = warp + NW * j;
+    const float excl = incl[j] - run[j];
+#pragma unroll
+    for (int u = 0; u < TPL; ++u) {
+      const int t = lane * TPL + u;
+      if (col <= kK && t < q.nt) {
+        if (col < kK) phi[t * kKP + col] = v[j][u] + excl;
+        else lcum[t] = v[j][u] + excl;
+      }
+    }
+  }
+  __syncthreads();
+}
+
 // Sine and cosine of an angle of any size (reduced to about [-pi, pi] first).
 __device__ __forceinline__ void sincos_r(float x, float* s, float* c) {
   __sincosf(reduce_2pi(x), s, c);
@@ -127,31 +194,38 @@ template <int R>
 __device__ __forceinline__ void stage_bc(const ScanArgs& a, const Geo& q, const float* phi,
                                          const float* sb, const float* sc, uint8_t* bt,
                                          uint8_t* ct) {
-  for (int e = threadIdx.x; e < kM * 16; e += blockDim.x) {
-    const int i = e >> 4, c16 = e & 15, t = i / R, r = i % R;
-    float bv[8], cv[8];
+  constexpr int PER = kM * 16 / kTh;
+  uint4 rb[PER], rc[PER];  // every load issued before the first use
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int e = (int)threadIdx.x + j * kTh, i = e >> 4, c16 = e & 15, t = i / R, r = i % R;
+    rb[j] = rc[j] = make_uint4(0u, 0u, 0u, 0u);
     if (t < q.nt) {
       const int64_t base = ((q.base + q.t0 + t) * a.ngroups + q.g) * R * kN + (int64_t)r * kN + 8 * c16;
-      ld8_bf16(a.B, base, bv);
-      ld8_bf16(a.C, base, cv);
+      rb[j] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.B) + base));
+      rc[j] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.C) + base));
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int e = (int)threadIdx.x + j * kTh, i = e >> 4, c16 = e & 15, t = i / R;
+    uint32_t ob[4] = {0u, 0u, 0u, 0u}, oc[4] = {0u, 0u, 0u, 0u};
+    if (t < q.nt) {
+      const uint32_t wb[4] = {rb[j].x, rb[j].y, rb[j].z, rb[j].w};
+      const uint32_t wc[4] = {rc[j].x, rc[j].y, rc[j].z, rc[j].w};
       const float fb = sb ? sb[t] : 1.f, fc = sc ? sc[t] : 1.f;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int u = 0; u < 4; ++u) {
         float sn, cs;
-        sincos_r(phi[t * kK + 4 * c16 + j], &sn, &cs);
-        const float b0 = bv[2 * j], b1 = bv[2 * j + 1], c0 = cv[2 * j], c1 = cv[2 * j + 1];
-        bv[2 * j] = fb * (cs * b0 + sn * b1);
-        bv[2 * j + 1] = fb * (-sn * b0 + cs * b1);
-        cv[2 * j] = fc * (cs * c0 + sn * c1);
-        cv[2 * j + 1] = fc * (-sn * c0 + cs * c1);
+        sincos_r(phi[t * kKP + 4 * c16 + u], &sn, &cs);
+        const float2 b = unpack_bf16(wb[u]), c = unpack_bf16(wc[u]);
+        ob[u] = pack_bf16(fb * (cs * b.x + sn * b.y), fb * (-sn * b.x + cs * b.y));
+        oc[u] = pack_bf16(fc * (cs * c.x + sn * c.y), fc * (-sn * c.x + cs * c.y));
       }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) bv[j] = cv[j] = 0.f;
     }
     const uint32_t off = (c16 >> 3) * kOPB + sw128_off(i, c16 & 7);
-    *reinterpret_cast<uint4*>(bt + off) = pack8(bv);
-    *reinterpret_cast<uint4*>(ct + off) = pack8(cv);
+    *reinterpret_cast<uint4*>(bt + off) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+    *reinterpret_cast<uint4*>(ct + off) = make_uint4(oc[0], oc[1], oc[2], oc[3]);
   }
 }
 
@@ -159,20 +233,35 @@ __device__ __forceinline__ void stage_bc(const ScanArgs& a, const Geo& q, const 
 template <int R>
 __device__ __forceinline__ void stage_xdy(const ScanArgs& a, const BwdArgs& g, const Geo& q,
                                           uint8_t* xs, uint8_t* dys) {
-  for (int e = threadIdx.x; e < kM * 8; e += blockDim.x) {
-    const int i = e >> 3, c8 = e & 7, t = i / R, r = i % R;
-    float xv[8], yv[8];
+  constexpr int PER = kM * 8 / kTh;
+  uint4 rx[PER], ry[PER], ry2[PER];  // ry2: the second half of an fp32 dy row piece
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int e = (int)threadIdx.x + j * kTh, i = e >> 3, c8 = e & 7, t = i / R, r = i % R;
+    rx[j] = ry[j] = ry2[j] = make_uint4(0u, 0u, 0u, 0u);
     if (t < q.nt) {
       const int64_t o = ((q.base + q.t0 + t) * a.nheads + q.h) * R * kP + (int64_t)r * kP + 8 * c8;
-      ld8_bf16(a.x, o, xv);
-      if (g.dy_f32) ld8_f32(static_cast<const float*>(g.dy) + o, yv);
-      else ld8_bf16(g.dy, o, yv);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) xv[j] = yv[j] = 0.f;
+      rx[j] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.x) + o));
+      if (g.dy_f32) {
+        const uint4* py = reinterpret_cast<const uint4*>(static_cast<const float*>(g.dy) + o);
+        ry[j] = __ldg(py);
+        ry2[j] = __ldg(py + 1);
+      } else {
+        ry[j] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(g.dy) + o));
+      }
     }
-    *reinterpret_cast<uint4*>(xs + sw128_off(i, c8)) = pack8(xv);
-    *reinterpret_cast<uint4*>(dys + sw128_off(i, c8)) = pack8(yv);
+  }
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int e = (int)threadIdx.x + j * kTh, i = e >> 3, c8 = e & 7;
+    uint4 yv = ry[j];
+    if (g.dy_f32)  // eight fp32 values -> bf16
+      yv = make_uint4(pack_bf16(__uint_as_float(ry[j].x), __uint_as_float(ry[j].y)),
+                      pack_bf16(__uint_as_float(ry[j].z), __uint_as_float(ry[j].w)),
+                      pack_bf16(__uint_as_float(ry2[j].x), __uint_as_float(ry2[j].y)),
+                      pack_bf16(__uint_as_float(ry2[j].z), __uint_as_float(ry2[j].w)));
+    *reinterpret_cast<uint4*>(xs + sw128_off(i, c8)) = rx[j];
+    *reinterpret_cast<uint4*>(dys + sw128_off(i, c8)) = yv;
   }
 }
 
@@ -183,7 +272,7 @@ __device__ __forceinline__ void stage_xdy(const ScanArgs& a, const BwdArgs& g, c
 struct SumsSmem {
   static constexpr int WB = 0, EC = 2 * kOPB, XS = 4 * kOPB, DYS = 5 * kOPB;
   static constexpr int SMALL = 6 * kOPB;
-  static constexpr int bytes(int Q) { return SMALL + (Q * kK + 6 * Q) * 4 + 32; }
+  static constexpr int bytes(int Q) { return SMALL + (Q * kKP + 6 * Q) * 4 + 32; }
 };
 
 template <int R>
@@ -198,13 +287,13 @@ __global__ void __launch_bounds__(kTh) bwd_tc_sums_kernel(const ScanArgs a, cons
   const int64_t cidx = (q.b * a.nheads + q.h) * a.nchunks + q.c;
   float* S = w.G + cidx * (int64_t)kN * kP;  // turned into G_c by the state pass
   float* D = w.D + cidx * (int64_t)kN * kP;
-  float* su = w.sums + cidx * (1 + kK);
+  float* su = w.sums + cidx * (1 + kN);
   if (q.nt <= 0) {  // past a short packed sequence: both states pass unchanged
     for (int e = tid; e < kN * kP / 4; e += kTh) {
       reinterpret_cast<float4*>(S)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
       reinterpret_cast<float4*>(D)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    for (int k = tid; k < 1 + kK; k += kTh) su[k] = 0.f;
+    for (int k = tid; k < 1 + kN; k += kTh) su[k] = (k == 0 || (k & 1)) ? 1.f : 0.f;
     return;
   }
   if ((sbase & 1023u) != 0) {
@@ -212,16 +301,17 @@ __global__ void __launch_bounds__(kTh) bwd_tc_sums_kernel(const ScanArgs a, cons
     return;
   }
   float* phi = reinterpret_cast<float*>(sm + L::SMALL);
-  float* lcum = phi + Q * kK;
+  float* lcum = phi + Q * kKP;
   float* gam = lcum + Q;
   float* del = gam + Q;
   float* dts = del + Q;
   float* s_w = dts + Q;  // w_s, the row scale of Bt
   float* s_e = s_w + Q;  // exp(Lam_t), the row scale of Ct
+  // 8-byte aligned: 71 Q floats (Q even) before it
   uint64_t* bar = reinterpret_cast<uint64_t*>(s_e + Q);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar + 1);
 
-  chunk_prep(a, q, lcum, gam, del, dts, phi);
+  prep_tc<Q>(a, q, lcum, gam, del, dts, phi);
   const float lend = lcum[q.nt - 1];
   for (int i = tid; i < Q; i += kTh) {
     s_w[i] = i < q.nt ? expf(lend - lcum[i]) * del[i] : 0.f;
@@ -277,8 +367,13 @@ __global__ void __launch_bounds__(kTh) bwd_tc_sums_kernel(const ScanArgs a, cons
             make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
                         __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
     }
-    if (tid == 0) su[0] = lend;
-    for (int k = tid; k < kK; k += kTh) su[1 + k] = phi[(q.nt - 1) * kK + k];
+    if (tid == 0) su[0] = expf(lend);
+    for (int k = tid; k < kK; k += kTh) {
+      float sn, cs;
+      sincosf(phi[(q.nt - 1) * kKP + k], &sn, &cs);
+      su[1 + 2 * k] = cs;
+      su[2 + 2 * k] = sn;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -290,16 +385,20 @@ __global__ void __launch_bounds__(kTh) bwd_tc_sums_kernel(const ScanArgs a, cons
 //   CT, BT   Ct, Bt: 2 K-major blocks each
 //   XS, DYS  x, dy: 1 block each
 //   GM       G_c in bf16, [128 rows n][64 p]; after phase A: M o S, M o DX
-//   DG       dGhat in bf16, [128 rows n][64 p]; after phase A: dPhi, fp32 [Q][K]
-//   SMALL    Phi [Q][K], per-token arrays, end-angle cos / sin, barriers
+//   DG       dGhat in bf16, [128 rows n][64 p]; after phase A: dPhi, fp32 [Q][kKP]
+//   SMALL    Phi [Q][kKP], per-token arrays, end-angle cos / sin, barriers
+template <int Q>
 struct ChunkTc {
   static constexpr int CT = 0, BT = 2 * kOPB, XS = 4 * kOPB, DYS = 5 * kOPB;
   static constexpr int GM = 6 * kOPB, MS = GM, MD = GM + kOPB;
   static constexpr int DG = GM + kN * 128;
-  static constexpr int SMALL = DG + kN * 128;
+  static constexpr int DG_BYTES =
+      ((Q * kKP * 4 > kN * 128 ? Q * kKP * 4 : kN * 128) + 1023) / 1024 * 1024;
+  static constexpr int SMALL = DG + DG_BYTES;
   static constexpr int NTOK = 12;  // per-token float arrays
-  static constexpr int bytes(int Q) {
-    return SMALL + (Q * kK + NTOK * Q + kK + 2 * kK + 32) * 4 + 32;
+  // the barriers follow 77 Q + 224 floats (Q even): 8-byte aligned
+  static constexpr int bytes() {
+    return SMALL + (Q * kKP + NTOK * Q + kK + 2 * kK + 32) * 4 + 32;
   }
   // TMEM columns
   static constexpr int S_COL = 0, DX_COL = 64, AX_COL = 128, AC_COL = 192, AB_COL = 320;
@@ -310,7 +409,7 @@ template <int R>
 __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, const BwdArgs g,
                                                               const BwdWs w) {
   constexpr int Q = kM / R;
-  using L = ChunkTc;
+  using L = ChunkTc<Q>;
   extern __shared__ __align__(1024) uint8_t sm[];
   const uint32_t sbase = smem_u32(sm);
   const Geo q = chunk_geo(a, blockIdx.x);
@@ -323,7 +422,7 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
   }
   const int64_t H = a.nheads;
   float* phi = reinterpret_cast<float*>(sm + L::SMALL);
-  float* lcum = phi + Q * kK;
+  float* lcum = phi + Q * kKP;
   float* gam = lcum + Q;
   float* del = gam + Q;
   float* dts = del + Q;
@@ -343,7 +442,7 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
   float* dPhi = reinterpret_cast<float*>(sm + L::DG);  // after phase A
 
   // ---- prologue: prefix sums, operands (before TMEM is taken) ----------------
-  chunk_prep(a, q, lcum, gam, del, dts, phi);
+  prep_tc<Q>(a, q, lcum, gam, del, dts, phi);
   const int t1 = nt - 1;
   const float lam_end = lcum[t1];
   for (int i = tid; i < Q; i += kTh) {
@@ -353,7 +452,7 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
   }
   for (int k = tid; k < kK; k += kTh) {
     float sn, cs;
-    sincos_r(phi[t1 * kK + k], &sn, &cs);
+    sincos_r(phi[t1 * kKP + k], &sn, &cs);
     ecs[2 * k] = cs;
     ecs[2 * k + 1] = sn;
   }
@@ -368,7 +467,9 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
   // G_c and dGhat = Rot(-Phi_end) dG_c+1 by row pairs (2k, 2k+1) and 8 columns;
   // <dGhat, G_c> and the outgoing rotation's angle gradient in fp32
   float dgg = 0.f;
-  for (int e = tid; e < kK * 8; e += kTh) {
+#pragma unroll
+  for (int e0 = 0; e0 < kK * 8; e0 += kTh) {
+    const int e = e0 + tid;
     const int k = e >> 3, c8 = e & 7;
     float g0[8], g1[8], o0[8], o1[8], n0[8], n1[8];
     ld8_f32(Gc + (2 * k) * kP + 8 * c8, g0);
@@ -576,7 +677,7 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
       if (hl == 0 && trow) atomicAdd(dLam + tr, el * cdot);
     }
     // dPhi goes over dGhat, which phase A has read
-    for (int i = tid; i < Q * kK; i += kTh) dPhi[i] = 0.f;
+    for (int i = tid; i < Q * kKP; i += kTh) dPhi[i] = 0.f;
     tmem_st_wait();
   }
   fence_async_smem();
@@ -610,36 +711,49 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
     const int64_t tok = q.base + q.t0 + tr;
     const int64_t bcb = (tok * a.ngroups + q.g) * R * kN + (int64_t)rr * kN;
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {  // 0: AC -> dC with Ct, 1: AB -> dB with Bt
-      const int acol = which ? L::AB_COL : L::AC_COL;
-      const uint8_t* opnd = sm + (which ? L::BT : L::CT);
-      float* gout = which ? g.dB : g.dC;
+    for (int pc = 0; pc < 2; ++pc) {
+      const int col = 64 * hh + 32 * pc;  // the warp's 32 columns; this thread's 16 from n0
+      const int n0 = col + 16 * hl;
+      uint32_t vc[16], vb[16];
+      tmem_ld16x2<16>(lb + L::AC_COL + col, vc);
+      tmem_ld16x2<16>(lb + L::AB_COL + col, vb);
+      tmem_ld_wait();
+      float dph[8];
 #pragma unroll
-      for (int pc = 0; pc < 2; ++pc) {
-        const int col = 64 * hh + 32 * pc;
-        const int n0 = col + 16 * hl;
-        uint32_t v[16];
-        tmem_ld16x2<16>(lb + acol + col, v);
-        tmem_ld_wait();
-        if (trow) {
-          float ov[16];
-          ld16_sw(opnd + (n0 >> 6) * kOPB, rho, n0 & 63, ov);
-          float res[16];
+      for (int j = 0; j < 8; ++j) dph[j] = 0.f;
+      if (trow) {
+        float oc[16], ob[16], rc[16], rb[16];
+        ld16_sw(sm + L::CT + (n0 >> 6) * kOPB, rho, n0 & 63, oc);
+        ld16_sw(sm + L::BT + (n0 >> 6) * kOPB, rho, n0 & 63, ob);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int k = n0 / 2 + j;
-            const float d0 = __uint_as_float(v[2 * j]), d1 = __uint_as_float(v[2 * j + 1]);
-            atomicAdd(dPhi + tr * kK + k, d0 * ov[2 * j + 1] - d1 * ov[2 * j]);
-            float sn, cs;
-            sincos_r(phi[tr * kK + k], &sn, &cs);
-            res[2 * j] = cs * d0 - sn * d1;  // Rot(Phi_t) of the rotated-frame gradient
-            res[2 * j + 1] = sn * d0 + cs * d1;
-          }
-#pragma unroll
-          for (int j = 0; j < 16; j += 4)
-            atomicAdd(reinterpret_cast<float4*>(gout + bcb + n0 + j),
-                      make_float4(res[j], res[j + 1], res[j + 2], res[j + 3]));
+        for (int j = 0; j < 8; ++j) {
+          const float c0 = __uint_as_float(vc[2 * j]), c1 = __uint_as_float(vc[2 * j + 1]);
+          const float b0 = __uint_as_float(vb[2 * j]), b1 = __uint_as_float(vb[2 * j + 1]);
+          // angle gradient of the rotations of C and B (pair n0 / 2 + j)
+          dph[j] = c0 * oc[2 * j + 1] - c1 * oc[2 * j] + b0 * ob[2 * j + 1] - b1 * ob[2 * j];
+          float sn, cs;
+          sincos_r(phi[tr * kKP + n0 / 2 + j], &sn, &cs);
+          rc[2 * j] = cs * c0 - sn * c1;  // Rot(Phi_t) of the rotated-frame gradients
+          rc[2 * j + 1] = sn * c0 + cs * c1;
+          rb[2 * j] = cs * b0 - sn * b1;
+          rb[2 * j + 1] = sn * b0 + cs * b1;
         }
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+          atomicAdd(reinterpret_cast<float4*>(g.dC + bcb + n0 + j),
+                    make_float4(rc[j], rc[j + 1], rc[j + 2], rc[j + 3]));
+          atomicAdd(reinterpret_cast<float4*>(g.dB + bcb + n0 + j),
+                    make_float4(rb[j], rb[j + 1], rb[j + 2], rb[j + 3]));
+        }
+      }
+      // the R rows of a token are R consecutive lanes: one shared-memory add
+      // per token and pair
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float v = dph[j];
+#pragma unroll
+        for (int off = 1; off < R; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (trow && (lane % R) == 0) atomicAdd(dPhi + tr * kKP + n0 / 2 + j, v);
       }
     }
     {  // dX
@@ -662,7 +776,7 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
   if (aborted) return;
 
   // ---- the scalar gradients (as on the CUDA cores) ----------------------------
-  for (int k = tid; k < kK; k += kTh) dPhi[t1 * kK + k] += s_pe[k];
+  for (int k = tid; k < kK; k += kTh) dPhi[t1 * kKP + k] += s_pe[k];
   for (int u = tid; u < nt; u += kTh) {
     float dl = -wv[u] * beta[u] - del[u] * colF[u];
     if (u == t1) {
@@ -675,31 +789,74 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
     ddel[u] += expf(lam_end - lcum[u]) * beta[u] + colF[u];
   }
   __syncthreads();
-  // suffix sums of dPhi over the chunk's tokens are d(dt theta)
-  for (int k = tid; k < kK; k += kTh) {
-    float run = 0.f;
-    for (int u = nt - 1; u >= 0; --u) {
-      run += dPhi[u * kK + k];
-      dPhi[u * kK + k] = run;
+  // Suffix sums over the chunk's tokens, one warp's scan per column: of dPhi
+  // (they are d(dt theta)) and of dLam (column kK; the gradient of a token's
+  // dt A term collects every later Lam of the chunk).
+  {
+    constexpr int TPL = Q > 32 ? Q / 32 : 1;
+    constexpr int NW = kTh / 32, CPW = (kK + NW) / NW;  // column c = warp + 8 j
+    float x[CPW][TPL], run[CPW], incl[CPW];
+#pragma unroll
+    for (int j = 0; j < CPW; ++j) {
+      const int col = warp + NW * j;
+      run[j] = 0.f;
+#pragma unroll
+      for (int u = 0; u < TPL; ++u) {
+        const int t = lane * TPL + u;
+        x[j][u] = 0.f;
+        if (col <= kK && t < nt) x[j][u] = col < kK ? dPhi[t * kKP + col] : dLam[t];
+        run[j] += x[j][u];
+      }
+      incl[j] = run[j];
+    }
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1)
+#pragma unroll
+      for (int j = 0; j < CPW; ++j) {
+        const float y = __shfl_up_sync(0xffffffffu, incl[j], off);
+        if (lane >= off) incl[j] += y;
+      }
+#pragma unroll
+    for (int j = 0; j < CPW; ++j) {
+      const int col = warp + NW * j;
+      const float total = __shfl_sync(0xffffffffu, incl[j], 31);
+      float pre = incl[j] - run[j];  // sum over the tokens before this lane's
+#pragma unroll
+      for (int u = 0; u < TPL; ++u) {
+        const int t = lane * TPL + u;
+        if (col <= kK && t < nt) {
+          if (col < kK) dPhi[t * kKP + col] = total - pre;
+          else dLam[t] = total - pre;
+        }
+        pre += x[j][u];
+      }
     }
   }
   __syncthreads();
   {
     constexpr int K4 = kK / 4;  // 16 float4 groups per token
-    for (int e0 = 0; e0 < nt * K4; e0 += kTh) {
-      const int e = e0 + tid;
+    constexpr int PER = (Q * K4 + kTh - 1) / kTh;
+    float4 th[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {  // every theta load issued first
+      const int e = tid + j * kTh, u = e / K4, k4 = e % K4;
+      th[j] = e < nt * K4
+                  ? __ldg(reinterpret_cast<const float4*>(
+                        a.theta + ((q.base + q.t0 + u) * a.tgroups + q.tg) * kK + 4 * k4))
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int e = tid + j * kTh, u = e / K4, k4 = e % K4;
       float part = 0.f;
-      int u = 0;
       if (e < nt * K4) {
-        u = e / K4;
-        const int k4 = e % K4;
         const int64_t to = ((q.base + q.t0 + u) * a.tgroups + q.tg) * kK + 4 * k4;
-        const float4 dp = *reinterpret_cast<const float4*>(dPhi + u * kK + 4 * k4);
+        const float* dpr = dPhi + u * kKP + 4 * k4;
+        const float4 dp = make_float4(dpr[0], dpr[1], dpr[2], dpr[3]);
         const float d = dts[u];
         atomicAdd(reinterpret_cast<float4*>(g.dtheta + to),
                   make_float4(d * dp.x, d * dp.y, d * dp.z, d * dp.w));
-        const float4 th = __ldg(reinterpret_cast<const float4*>(a.theta + to));
-        part = th.x * dp.x + th.y * dp.y + th.z * dp.z + th.w * dp.w;
+        part = th[j].x * dp.x + th[j].y * dp.y + th[j].z * dp.z + th[j].w * dp.w;
       }
 #pragma unroll
       for (int off = 1; off < K4; off <<= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
@@ -709,8 +866,7 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
   __syncthreads();
   // per token: dt, A, lam (gamma = lam dt, eps = (1 - lam) dt, delta_s = gamma_s + eps_s+1)
   for (int u = tid; u < nt; u += kTh) {
-    float run = 0.f;
-    for (int t = u; t < nt; ++t) run += dLam[t];
+    const float run = dLam[u];  // sum over t >= u of dLam_t
     const int64_t o = (q.base + q.t0 + u) * H + q.h;
     const float dt = dts[u], lam = __ldg(a.lam + o), Av = __ldg(a.A + o);
     const float dgv = dgam[u] + ddel[u];
@@ -744,7 +900,7 @@ cudaError_t sums_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaStre
 
 template <int R>
 cudaError_t chunk_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaStream_t st) {
-  const size_t smem = ChunkTc::bytes(kM / R);
+  const size_t smem = ChunkTc<kM / R>::bytes();
   cudaError_t e = set_smem(bwd_tc_chunk_kernel<R>, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)f.nchunks, (unsigned)f.nheads, (unsigned)f.batch);
