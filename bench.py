@@ -148,13 +148,18 @@ def varlen_line(s, rank, world, steps, warmup, flush, peaks, psrc):
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def bwd_rows(s: I.Shape):
-    """Rows per chunk the backward picks (the library's rule: 32 rows, two
-    CTAs per SM)."""
-    return 32
+def bwd_tc(s: I.Shape) -> bool:
+    """Whether m3_scan_bwd runs on the tensor cores (bf16 io at N = 128, P = 64)."""
+    return s.io == "bf16" and s.dstate == 128 and s.headdim == 64
 
 
-def bwd_work(s: I.Shape):
+def bwd_rows(s: I.Shape, simt=False):
+    """Rows per chunk the backward picks (the library's rule: 64 on the
+    tensor cores, else 32 rows, two CTAs per SM)."""
+    return 64 if bwd_tc(s) and not simt else 32
+
+
+def bwd_work(s: I.Shape, simt=False):
     """Algorithmic FLOPs and bytes of one m3_scan_bwd.
 
     Per chunk-head of the backward's chunking (M = Qb * R rows, causal token
@@ -164,7 +169,7 @@ def bwd_work(s: I.Shape):
     dGhat x, dGhat^T Bt): 10 * M * N * P.  Bytes: every input and dy read
     once, every gradient (fp32) and the final-state adjoint written once."""
     R, N, P = s.rank, s.dstate, s.headdim
-    M = bwd_rows(s)
+    M = bwd_rows(s, simt)
     Qb = M // R
     causal = Qb * (Qb + 1) // 2 * R * R
     nc = math.ceil(s.seqlen / Qb)
@@ -194,16 +199,17 @@ def alu_roofline(flops, byt, seconds, peaks):
             "frac": round(ach / peaks["hbm_gbs"], 4), "roofline_time_us": round(t_hbm * 1e6, 2)}
 
 
-def time_bwd(inp, s, steps, warmup, flush):
+def time_bwd(inp, s, steps, warmup, flush, simt=False):
     gen = torch.Generator(device="cuda").manual_seed(77)
     dy = torch.randn(inp["x"].shape, generator=gen, device="cuda").to(inp["x"].dtype)
     dfin = torch.randn((s.batch, s.nheads, s.dstate, s.headdim), generator=gen, device="cuda")
-    ws = torch.empty(max(m3.bwd_workspace_size(m3.scan_shape(inp["x"], inp["B"], s.chunk)), 1),
+    ws = torch.empty(max(m3.bwd_workspace_size(m3.scan_shape(inp["x"], inp["B"], s.chunk, simt)),
+                         1),
                      dtype=torch.uint8, device="cuda")
 
     def step():
         m3.m3_scan_bwd(inp["x"], inp["dt"], inp["A"], inp["lam"], inp["theta"], inp["B"],
-                       inp["C"], dy, s.chunk, d_final=dfin, workspace=ws)
+                       inp["C"], dy, s.chunk, d_final=dfin, workspace=ws, simt=simt)
 
     for _ in range(warmup):
         step()
@@ -222,15 +228,22 @@ def time_bwd(inp, s, steps, warmup, flush):
     return [a.elapsed_time(b) * 1e-3 for a, b in ev]
 
 
-def bwd_line(inp, s, world, steps, warmup, flush, peaks):
+def bwd_line(inp, s, world, steps, warmup, flush, peaks, psrc, simt=False):
     barrier(world)
-    t = max_over_ranks(sum(time_bwd(inp, s, steps, warmup, flush)), world) / steps
-    f, b = bwd_work(s)
-    return {"metric": "backward tokens/s", "value": round(world * s.batch * s.seqlen / t, 1),
-            "unit": "tokens/s", "ms_per_step": round(t * 1e3, 4),
-            "path": "m3_scan_bwd: 3 launches (per-chunk sums, both state passes, "
-                    "per-chunk gradients), CUDA cores fp32",
-            "roofline": alu_roofline(f, b, t, peaks)}
+    t = max_over_ranks(sum(time_bwd(inp, s, steps, warmup, flush, simt)), world) / steps
+    f, b = bwd_work(s, simt)
+    line = {"metric": "backward tokens/s", "value": round(world * s.batch * s.seqlen / t, 1),
+            "unit": "tokens/s", "ms_per_step": round(t * 1e3, 4)}
+    if bwd_tc(s) and not simt:
+        line["path"] = ("m3_scan_bwd: 3 launches (per-chunk sums and per-chunk gradients on the "
+                        "tensor cores, tcgen05 bf16 operands, fp32 accumulators; both state "
+                        f"passes on the CUDA cores), chunks of {bwd_rows(s)} rows")
+        line["roofline"] = roofline(f, b, t, peaks, psrc)
+    else:
+        line["path"] = ("m3_scan_bwd: 3 launches (per-chunk sums, both state passes, "
+                        "per-chunk gradients), CUDA cores fp32")
+        line["roofline"] = alu_roofline(f, b, t, peaks)
+    return line
 
 
 def prep_line(s, world, steps, warmup, flush, peaks, psrc):
@@ -807,6 +820,8 @@ def main():
                     help="run one part only (for profiling); prints its own line")
     ap.add_argument("--batch", type=int, default=None,
                     help="with --only: override the workload's batch (small profiling cases)")
+    ap.add_argument("--simt", action="store_true",
+                    help="with --only bwd: the CUDA-core backward (profiling)")
     ap.add_argument("--chunk", type=int, default=None,
                     help="with --only: override the workload's chunk length")
     args = ap.parse_args()
@@ -855,7 +870,7 @@ def main():
         inp = I.make_scan_inputs(I.Workload(s), seed=1001, device="cuda")
         flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
         print(json.dumps({"only": "bwd", **bwd_line(inp, s, 1, args.steps, args.warmup, flush,
-                                                    peaks)}))
+                                                    peaks, psrc, args.simt)}))
         return
     if args.only == "varlen":
         flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
@@ -943,14 +958,14 @@ def main():
     if siso_inp is None:
         siso_inp = I.make_scan_inputs(I.SISO_PREFILL, seed=SEEDS["siso_prefill"] + 7919 * rank,
                                       device="cuda")
-    line["backward"] = bwd_line(siso_inp, ss, world, 3, args.warmup, flush, peaks)
+    line["backward"] = bwd_line(siso_inp, ss, world, 3, args.warmup, flush, peaks, psrc)
     del siso_inp
     # the block projections around the layer (tensor-core GEMMs, MIMO up / down, gate)
     line["block"] = block_line(world, 10, args.warmup, flush, peaks, psrc)
     ms = I.MIMO_PREFILL.shape
     mimo_inp = I.make_scan_inputs(I.MIMO_PREFILL, seed=SEEDS["mimo_prefill"] + 7919 * rank,
                                   device="cuda")
-    line["backward_mimo"] = bwd_line(mimo_inp, ms, world, 3, args.warmup, flush, peaks)
+    line["backward_mimo"] = bwd_line(mimo_inp, ms, world, 3, args.warmup, flush, peaks, psrc)
     del mimo_inp
     if rank == 0:
         print(json.dumps(line), flush=True)

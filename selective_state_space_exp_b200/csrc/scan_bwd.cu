@@ -191,22 +191,48 @@ __global__ void __launch_bounds__(512) bwd_sums_kernel(const ScanArgs a, const B
 // dG_c+1 (its outgoing state's adjoint) over D_c; dG_0 gives dh0 and the
 // previous token's gradients.  Chunks go in batches of kPipe whose loads are
 // all issued before the batch's dependent updates.
+// TC (the tensor-core form): G_c is written in bf16 in the MMA operand layout
+// instead (and the final state after the last chunk's), and the reverse pass
+// writes dGhat_c = Rot(-Phi_c) dG_c+1 the same way instead of dG_c+1.
+// Four consecutive columns p0..p0+3 of row `row` in bf16 (8 bytes) at their
+// place in a [rows][64] block of the MMA operand layout.
+__device__ __forceinline__ void st4_bf16_sw(uint8_t* blk, int row, int p0, float4 v) {
+  const uint32_t off = row * 128u + ((((uint32_t)p0 >> 3) ^ ((uint32_t)row & 7u)) << 4) +
+                       ((uint32_t)p0 & 7u) * 2u;
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+  *reinterpret_cast<uint2*>(blk + off) =
+      make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+}
+
+__device__ __forceinline__ float4 f4fma(float a, float4 x, float4 y) {
+  return make_float4(fmaf(a, x.x, y.x), fmaf(a, x.y, y.y), fmaf(a, x.z, y.z), fmaf(a, x.w, y.w));
+}
+__device__ __forceinline__ float4 f4lin(float a, float4 x, float b, float4 y) {  // a x + b y
+  return make_float4(a * x.x + b * y.x, a * x.y + b * y.y, a * x.z + b * y.z, a * x.w + b * y.w);
+}
+__device__ __forceinline__ float f4c(const float4& v, int k) {
+  return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
+}
+
+// Thread (k, p0) of chain (b, h) holds the pair (2k, 2k+1) of columns p0..p0+3.
+template <bool TC>
 __global__ void __launch_bounds__(kThreads) bwd_pass_kernel(const ScanArgs a, const BwdArgs g,
                                                             const BwdWs w) {
-  const int N = (int)a.N, P = (int)a.P, K = N / 2, R = (int)a.R;
+  const int N = (int)a.N, P = (int)a.P, K = N / 2, R = (int)a.R, PG = P / 4;
   const int64_t b = blockIdx.z, h = blockIdx.y, H = a.nheads;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= K * P) return;  // K * P is a multiple of 32: whole warps leave
-  const int k = idx / P, p = idx % P;
+  if (idx >= K * PG) return;  // K * P / 4 is a multiple of 32: whole warps leave
+  const int k = idx / PG, p0 = 4 * (idx % PG);
   const int64_t so = (b * H + h) * (int64_t)N * P;
   const int64_t grp = h / (H / a.ngroups);
   const Chain chn = chain_of(a, b);
-  const int64_t i0 = (2 * k) * P + p, i1 = (2 * k + 1) * P + p;
-  constexpr int kPipe = 8;
+  const int64_t i0 = (2 * k) * P + p0, i1 = (2 * k + 1) * P + p0;
+  constexpr int kPipe = 4;
   const int64_t chain0 = (b * H + h) * a.nchunks;
+  const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
 
   // forward
-  float g0 = a.h0 ? a.h0[so + i0] : 0.f, g1 = a.h0 ? a.h0[so + i1] : 0.f;
+  float4 g0 = a.h0 ? ld4(a.h0 + so + i0) : z4, g1 = a.h0 ? ld4(a.h0 + so + i1) : z4;
   float eps0 = 0.f, lam0 = 0.f, dt0 = 0.f;
   int64_t t0 = 0;
   if (a.B_prev && chn.len > 0) {  // the left endpoint term waits for a token
@@ -216,21 +242,24 @@ __global__ void __launch_bounds__(kThreads) bwd_pass_kernel(const ScanArgs a, co
     eps0 = (1.f - lam0) * dt0;
     for (int r = 0; r < R; ++r) {
       const int64_t bb = ((b * a.ngroups + grp) * R + r) * N;
-      const float xv = io_load(a.x_prev, ((b * H + h) * R + r) * P + p, a.bf16);
-      g0 = fmaf(eps0 * io_load(a.B_prev, bb + 2 * k, a.bf16), xv, g0);
-      g1 = fmaf(eps0 * io_load(a.B_prev, bb + 2 * k + 1, a.bf16), xv, g1);
+      const int64_t xo = ((b * H + h) * R + r) * P + p0;
+      const float4 xv = make_float4(io_load(a.x_prev, xo, a.bf16), io_load(a.x_prev, xo + 1, a.bf16),
+                                    io_load(a.x_prev, xo + 2, a.bf16), io_load(a.x_prev, xo + 3, a.bf16));
+      g0 = f4fma(eps0 * io_load(a.B_prev, bb + 2 * k, a.bf16), xv, g0);
+      g1 = f4fma(eps0 * io_load(a.B_prev, bb + 2 * k + 1, a.bf16), xv, g1);
     }
   }
   for (int64_t c0 = 0; c0 < a.nchunks; c0 += kPipe) {
-    float s0[kPipe], s1[kPipe], dec[kPipe], sn[kPipe], cs[kPipe];
+    float4 s0[kPipe], s1[kPipe];
+    float dec[kPipe], sn[kPipe], cs[kPipe];
 #pragma unroll
     for (int j = 0; j < kPipe; ++j) {
       const int64_t c = c0 + j;
       if (c >= a.nchunks) break;
       const float* S = w.G + (chain0 + c) * (int64_t)N * P;
       const float* su = w.sums + (chain0 + c) * (1 + N);
-      s0[j] = S[i0];
-      s1[j] = S[i1];
+      s0[j] = ld4(S + i0);
+      s1[j] = ld4(S + i1);
       dec[j] = su[0];
       cs[j] = su[1 + 2 * k];
       sn[j] = su[2 + 2 * k];
@@ -239,30 +268,42 @@ __global__ void __launch_bounds__(kThreads) bwd_pass_kernel(const ScanArgs a, co
     for (int j = 0; j < kPipe; ++j) {
       const int64_t c = c0 + j;
       if (c >= a.nchunks) break;
-      float* S = w.G + (chain0 + c) * (int64_t)N * P;
-      S[i0] = g0;  // chunk-start state, true frame
-      S[i1] = g1;
-      const float v0 = fmaf(dec[j], g0, s0[j]), v1 = fmaf(dec[j], g1, s1[j]);
-      g0 = cs[j] * v0 - sn[j] * v1;
-      g1 = sn[j] * v0 + cs[j] * v1;
+      if (TC) {  // chunk-start state, true frame
+        uint8_t* blk = w.Gb + ((b * H + h) * (a.nchunks + 1) + c) * (int64_t)N * P * 2;
+        st4_bf16_sw(blk, 2 * k, p0, g0);
+        st4_bf16_sw(blk, 2 * k + 1, p0, g1);
+      } else {
+        float* S = w.G + (chain0 + c) * (int64_t)N * P;
+        *reinterpret_cast<float4*>(S + i0) = g0;
+        *reinterpret_cast<float4*>(S + i1) = g1;
+      }
+      const float4 v0 = f4fma(dec[j], g0, s0[j]), v1 = f4fma(dec[j], g1, s1[j]);
+      g0 = f4lin(cs[j], v0, -sn[j], v1);
+      g1 = f4lin(sn[j], v0, cs[j], v1);
     }
   }
-  w.fin[so + i0] = g0;
-  w.fin[so + i1] = g1;
+  *reinterpret_cast<float4*>(w.fin + so + i0) = g0;
+  *reinterpret_cast<float4*>(w.fin + so + i1) = g1;
+  if (TC) {  // the final state as block nc of the chain
+    uint8_t* blk = w.Gb + ((b * H + h) * (a.nchunks + 1) + a.nchunks) * (int64_t)N * P * 2;
+    st4_bf16_sw(blk, 2 * k, p0, g0);
+    st4_bf16_sw(blk, 2 * k + 1, p0, g1);
+  }
 
   // reverse
-  float d0 = g.d_final ? g.d_final[so + i0] : 0.f;
-  float d1 = g.d_final ? g.d_final[so + i1] : 0.f;
+  float4 d0 = g.d_final ? ld4(g.d_final + so + i0) : z4;
+  float4 d1 = g.d_final ? ld4(g.d_final + so + i1) : z4;
   for (int64_t c0 = a.nchunks - 1; c0 >= 0; c0 -= kPipe) {
-    float e0[kPipe], e1[kPipe], dec[kPipe], sn[kPipe], cs[kPipe];
+    float4 e0[kPipe], e1[kPipe];
+    float dec[kPipe], sn[kPipe], cs[kPipe];
 #pragma unroll
     for (int j = 0; j < kPipe; ++j) {
       const int64_t c = c0 - j;
       if (c < 0) break;
       const float* Dc = w.D + (chain0 + c) * (int64_t)N * P;
       const float* su = w.sums + (chain0 + c) * (1 + N);
-      e0[j] = Dc[i0];
-      e1[j] = Dc[i1];
+      e0[j] = ld4(Dc + i0);
+      e1[j] = ld4(Dc + i1);
       dec[j] = su[0];
       cs[j] = su[1 + 2 * k];
       sn[j] = su[2 + 2 * k];
@@ -271,18 +312,23 @@ __global__ void __launch_bounds__(kThreads) bwd_pass_kernel(const ScanArgs a, co
     for (int j = 0; j < kPipe; ++j) {
       const int64_t c = c0 - j;
       if (c < 0) break;
-      float* Dc = w.D + (chain0 + c) * (int64_t)N * P;
-      Dc[i0] = d0;  // adjoint of chunk c's outgoing state
-      Dc[i1] = d1;
-      const float n0 = fmaf(dec[j], cs[j] * d0 + sn[j] * d1, e0[j]);  // D_c + exp(Lam) Rot(-Phi) dG
-      const float n1 = fmaf(dec[j], -sn[j] * d0 + cs[j] * d1, e1[j]);
-      d0 = n0;
-      d1 = n1;
+      const float4 h0 = f4lin(cs[j], d0, sn[j], d1), h1 = f4lin(-sn[j], d0, cs[j], d1);  // Rot(-Phi) dG
+      if (TC) {
+        uint8_t* blk = w.Hb + (chain0 + c) * (int64_t)N * P * 2;
+        st4_bf16_sw(blk, 2 * k, p0, h0);
+        st4_bf16_sw(blk, 2 * k + 1, p0, h1);
+      } else {
+        float* Dc = w.D + (chain0 + c) * (int64_t)N * P;
+        *reinterpret_cast<float4*>(Dc + i0) = d0;  // adjoint of chunk c's outgoing state
+        *reinterpret_cast<float4*>(Dc + i1) = d1;
+      }
+      d0 = f4fma(dec[j], h0, e0[j]);  // D_c + exp(Lam) Rot(-Phi) dG
+      d1 = f4fma(dec[j], h1, e1[j]);
     }
   }
   if (g.dh0) {
-    g.dh0[so + i0] = d0;
-    g.dh0[so + i1] = d1;
+    *reinterpret_cast<float4*>(g.dh0 + so + i0) = d0;
+    *reinterpret_cast<float4*>(g.dh0 + so + i1) = d1;
   }
   if (a.B_prev && chn.len > 0) {  // G_0 = h0 + eps_0 B_prev x_prev^T
     float part = 0.f;
@@ -290,14 +336,20 @@ __global__ void __launch_bounds__(kThreads) bwd_pass_kernel(const ScanArgs a, co
       const int64_t bb = ((b * a.ngroups + grp) * R + r) * N;
       const float bp0 = io_load(a.B_prev, bb + 2 * k, a.bf16);
       const float bp1 = io_load(a.B_prev, bb + 2 * k + 1, a.bf16);
-      const int64_t xo = ((b * H + h) * R + r) * P + p;
-      const float xv = io_load(a.x_prev, xo, a.bf16);
-      const float gb = d0 * bp0 + d1 * bp1;
-      part = fmaf(gb, xv, part);
+      const int64_t xo = ((b * H + h) * R + r) * P + p0;
+      float db0 = 0.f, db1 = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float xv = io_load(a.x_prev, xo + u, a.bf16);
+        const float gb = f4c(d0, u) * bp0 + f4c(d1, u) * bp1;
+        part = fmaf(gb, xv, part);
+        db0 = fmaf(f4c(d0, u), xv, db0);
+        db1 = fmaf(f4c(d1, u), xv, db1);
+        if (g.dB_prev) atomicAdd(g.dx_prev + xo + u, eps0 * gb);
+      }
       if (g.dB_prev) {
-        atomicAdd(g.dB_prev + bb + 2 * k, eps0 * d0 * xv);
-        atomicAdd(g.dB_prev + bb + 2 * k + 1, eps0 * d1 * xv);
-        atomicAdd(g.dx_prev + xo, eps0 * gb);
+        atomicAdd(g.dB_prev + bb + 2 * k, eps0 * db0);
+        atomicAdd(g.dB_prev + bb + 2 * k + 1, eps0 * db1);
       }
     }
 #pragma unroll
@@ -359,9 +411,6 @@ __device__ __forceinline__ float sum16(float v) {
   return v;
 }
 
-__device__ __forceinline__ float f4c(const float4& v, int k) {
-  return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
-}
 
 // acc[i][c][:] += sum_kk a4[i].kk * B[kk][4 gi .. 4 gi + 3], gi = tx + 16 c:
 // four k-steps of an N-wide product whose A operand was loaded 4 k wide.
@@ -951,38 +1000,46 @@ cudaError_t launch_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaSt
 // [b][H][nc][1 + N] (exp(Lam_end), then cos, sin of Phi_end per pair), the
 // adjoints D [b][H][nc][N][P] and the final states [b][H][N][P], each 256-byte
 // aligned.
+// The tensor-core form adds the bf16 operand blocks: G_c and the final state
+// ([b][H][nc + 1][N][P]) and dGhat_c ([b][H][nc][N][P]).
 namespace {
 struct WsSizes {
-  size_t g, sums, d, fin;
+  size_t g, sums, d, fin, gb, hb;
 };
-WsSizes ws_sizes(const ScanArgs& f) {
+WsSizes ws_sizes(const ScanArgs& f, bool tc) {
   const size_t chains = (size_t)f.batch * f.nheads;
   return {align_up(sizeof(float) * chains * f.nchunks * f.N * f.P, 256),
           align_up(sizeof(float) * chains * f.nchunks * (1 + f.N), 256),
           align_up(sizeof(float) * chains * f.nchunks * f.N * f.P, 256),
-          align_up(sizeof(float) * chains * f.N * f.P, 256)};
+          align_up(sizeof(float) * chains * f.N * f.P, 256),
+          tc ? align_up(2 * chains * (f.nchunks + 1) * f.N * f.P, 256) : 0,
+          tc ? align_up(2 * chains * f.nchunks * f.N * f.P, 256) : 0};
 }
 }  // namespace
 
-BwdWs bwd_carve(const ScanArgs& f) {
-  const WsSizes z = ws_sizes(f);
+BwdWs bwd_carve(const ScanArgs& f, bool tc) {
+  const WsSizes z = ws_sizes(f, tc);
   BwdWs w;
-  w.G = reinterpret_cast<float*>(f.ws);
-  w.sums = reinterpret_cast<float*>(f.ws + z.g);
-  w.D = reinterpret_cast<float*>(f.ws + z.g + z.sums);
-  w.fin = reinterpret_cast<float*>(f.ws + z.g + z.sums + z.d);
+  char* p = f.ws;
+  w.G = reinterpret_cast<float*>(p); p += z.g;
+  w.sums = reinterpret_cast<float*>(p); p += z.sums;
+  w.D = reinterpret_cast<float*>(p); p += z.d;
+  w.fin = reinterpret_cast<float*>(p); p += z.fin;
+  w.Gb = tc ? reinterpret_cast<uint8_t*>(p) : nullptr; p += z.gb;
+  w.Hb = tc ? reinterpret_cast<uint8_t*>(p) : nullptr;
   return w;
 }
 
-size_t bwd_ws_bytes(const ScanArgs& f) {
-  const WsSizes z = ws_sizes(f);
-  return z.g + z.sums + z.d + z.fin;
+size_t bwd_ws_bytes(const ScanArgs& f, bool tc) {
+  const WsSizes z = ws_sizes(f, tc);
+  return z.g + z.sums + z.d + z.fin + z.gb + z.hb;
 }
 
 cudaError_t bwd_pass_launch(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaStream_t st) {
-  dim3 pgrid((unsigned)(((f.N / 2) * f.P + kThreads - 1) / kThreads), (unsigned)f.nheads,
+  dim3 pgrid((unsigned)(((f.N / 2) * (f.P / 4) + kThreads - 1) / kThreads), (unsigned)f.nheads,
              (unsigned)f.batch);
-  bwd_pass_kernel<<<pgrid, kThreads, 0, st>>>(f, g, w);
+  if (w.Gb) bwd_pass_kernel<true><<<pgrid, kThreads, 0, st>>>(f, g, w);
+  else bwd_pass_kernel<false><<<pgrid, kThreads, 0, st>>>(f, g, w);
   return cudaGetLastError();
 }
 
@@ -998,7 +1055,7 @@ bool bwd_use_tc(const ScanArgs& a, bool allow) { return allow && bwd_tc_shape(a)
 size_t bwd_workspace(const ScanArgs& a, bool tc) {
   const int64_t M = chunk_rows(a, tc);
   if (M == 0 || a.seqlen == 0) return 0;
-  return bwd_ws_bytes(bwd_fwd_args(a, M / a.R));
+  return bwd_ws_bytes(bwd_fwd_args(a, M / a.R), tc && bwd_tc_shape(a));
 }
 
 cudaError_t bwd_zero_outputs(const ScanArgs& a, const BwdArgs& g, cudaStream_t st) {
@@ -1021,11 +1078,12 @@ cudaError_t bwd_launch(const ScanArgs& a, const BwdArgs& g, bool tc, cudaStream_
   const int64_t M = chunk_rows(a, tc);
   if (M == 0) return cudaErrorInvalidValue;
   ScanArgs f = bwd_fwd_args(a, M / a.R);
-  BwdWs w = bwd_carve(f);
+  const bool use_tc = tc && bwd_tc_shape(a);
+  BwdWs w = bwd_carve(f, use_tc);
   f.final_state = w.fin;
   cudaError_t e = bwd_zero_outputs(a, g, st);
   if (e != cudaSuccess) return e;
-  if (tc && bwd_tc_shape(a)) {
+  if (use_tc) {
     e = bwd_tc_sums_launch(f, g, w, st);
     if (e != cudaSuccess) return e;
     e = bwd_pass_launch(f, g, w, st);

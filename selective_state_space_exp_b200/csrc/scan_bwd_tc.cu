@@ -79,16 +79,6 @@ __device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t bytes) {
   return d + (uint64_t)(bytes >> 4);
 }
 
-__device__ __forceinline__ void ld8_f32(const float* p, float (&v)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-__device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
-  return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
-                    pack_bf16(v[6], v[7]));
-}
 // 16 consecutive bf16 values of row `row` from column c0 (a multiple of 16)
 // of a [rows][64] swizzled block, as floats.
 __device__ __forceinline__ void ld16_sw(const uint8_t* blk, int row, int c0, float (&v)[16]) {
@@ -396,9 +386,9 @@ struct ChunkTc {
       ((Q * kKP * 4 > kN * 128 ? Q * kKP * 4 : kN * 128) + 1023) / 1024 * 1024;
   static constexpr int SMALL = DG + DG_BYTES;
   static constexpr int NTOK = 12;  // per-token float arrays
-  // the barriers follow 77 Q + 224 floats (Q even): 8-byte aligned
+  // the barriers follow 77 Q + 96 floats (Q even): 8-byte aligned
   static constexpr int bytes() {
-    return SMALL + (Q * kKP + NTOK * Q + kK + 2 * kK + 32) * 4 + 32;
+    return SMALL + (Q * kKP + NTOK * Q + kK + 32) * 4 + 32;
   }
   // TMEM columns
   static constexpr int S_COL = 0, DX_COL = 64, AX_COL = 128, AC_COL = 192, AB_COL = 320;
@@ -435,13 +425,39 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
   float* colF = ddel + Q;  // sum over t > s of F_ts
   float* thT = colF + Q;   // sum_k theta_k d(dt theta)_k
   float* s_pe = thT + Q;   // the outgoing rotation's angle gradient, [K]
-  float* ecs = s_pe + kK;  // cos, sin of Phi_end, [K][2]
-  float* red = ecs + 2 * kK;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 32);
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2);
+  float* red = s_pe + kK;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 32);  // phase A, phase B, G / dGhat copy
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 3);
   float* dPhi = reinterpret_cast<float*>(sm + L::DG);  // after phase A
+  const int64_t cidx = (q.b * H + q.h) * a.nchunks + q.c;
+  const int64_t gbi = (q.b * H + q.h) * (a.nchunks + 1) + q.c;  // G_c's block
 
-  // ---- prologue: prefix sums, operands (before TMEM is taken) ----------------
+  // ---- prologue: operand blocks of the state pass in flight, prefix sums,
+  // rotated operands (all before TMEM is taken) --------------------------------
+  if (tid == 0) {
+    mbar_init(bars, 1);
+    mbar_init(bars + 1, 1);
+    mbar_init(bars + 2, 1);
+    fence_mbar_init();
+    mbar_expect_tx(bars + 2, 2 * kN * kP * 2);
+    bulk_load(sm + L::GM, w.Gb + gbi * kN * kP * 2, kN * kP * 2, bars + 2);
+    bulk_load(sm + L::DG, w.Hb + cidx * (int64_t)kN * kP * 2, kN * kP * 2, bars + 2);
+  }
+  // G_c+1 (the next block of the chain: the next chunk's start state, or the
+  // final state), for the outgoing rotation's angle gradient.  Item e = (pair
+  // k, logical 16-byte chunk u of P): rows 2k and 2k + 1 at u's swizzled place.
+  constexpr int kItems = kK * 8 / kTh;
+  uint4 gn[kItems][2];
+#pragma unroll
+  for (int j = 0; j < kItems; ++j) {
+    const int e = tid + j * kTh, k = e >> 3, u = e & 7;
+    const uint8_t* nb = w.Gb + (gbi + 1) * kN * kP * 2;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int row = 2 * k + r;
+      gn[j][r] = __ldg(reinterpret_cast<const uint4*>(nb + sw128_off(row, u)));
+    }
+  }
   prep_tc<Q>(a, q, lcum, gam, del, dts, phi);
   const int t1 = nt - 1;
   const float lam_end = lcum[t1];
@@ -450,69 +466,61 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
     lg[i] = (i < nt) ? lcum[i] * kL2E : 0.f;
     beta[i] = dLam[i] = dgam[i] = ddel[i] = colF[i] = thT[i] = 0.f;
   }
-  for (int k = tid; k < kK; k += kTh) {
-    float sn, cs;
-    sincos_r(phi[t1 * kKP + k], &sn, &cs);
-    ecs[2 * k] = cs;
-    ecs[2 * k + 1] = sn;
-  }
   __syncthreads();
   stage_bc<R>(a, q, phi, nullptr, nullptr, sm + L::BT, sm + L::CT);
   stage_xdy<R>(a, g, q, sm + L::XS, sm + L::DYS);
-  const int64_t cidx = (q.b * H + q.h) * a.nchunks + q.c;
-  const float* Gc = w.G + cidx * (int64_t)kN * kP;  // state entering the chunk
-  const float* Do = w.D + cidx * (int64_t)kN * kP;  // adjoint of the state leaving it
-  const float* Gn = (q.c + 1 < a.nchunks) ? Gc + (int64_t)kN * kP  // next chunk's start state
-                                          : w.fin + (q.b * H + q.h) * (int64_t)kN * kP;
-  // G_c and dGhat = Rot(-Phi_end) dG_c+1 by row pairs (2k, 2k+1) and 8 columns;
-  // <dGhat, G_c> and the outgoing rotation's angle gradient in fp32
-  float dgg = 0.f;
-#pragma unroll
-  for (int e0 = 0; e0 < kK * 8; e0 += kTh) {
-    const int e = e0 + tid;
-    const int k = e >> 3, c8 = e & 7;
-    float g0[8], g1[8], o0[8], o1[8], n0[8], n1[8];
-    ld8_f32(Gc + (2 * k) * kP + 8 * c8, g0);
-    ld8_f32(Gc + (2 * k + 1) * kP + 8 * c8, g1);
-    ld8_f32(Do + (2 * k) * kP + 8 * c8, o0);
-    ld8_f32(Do + (2 * k + 1) * kP + 8 * c8, o1);
-    ld8_f32(Gn + (2 * k) * kP + 8 * c8, n0);
-    ld8_f32(Gn + (2 * k + 1) * kP + 8 * c8, n1);
-    const float ce = ecs[2 * k], se = ecs[2 * k + 1];
-    float h0[8], h1[8], cr = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      h0[j] = ce * o0[j] + se * o1[j];
-      h1[j] = -se * o0[j] + ce * o1[j];
-      dgg = fmaf(h0[j], g0[j], fmaf(h1[j], g1[j], dgg));
-      cr = fmaf(o1[j], n0[j], fmaf(-o0[j], n1[j], cr));
-    }
-    *reinterpret_cast<uint4*>(sm + L::GM + sw128_off(2 * k, c8)) = pack8(g0);
-    *reinterpret_cast<uint4*>(sm + L::GM + sw128_off(2 * k + 1, c8)) = pack8(g1);
-    *reinterpret_cast<uint4*>(sm + L::DG + sw128_off(2 * k, c8)) = pack8(h0);
-    *reinterpret_cast<uint4*>(sm + L::DG + sw128_off(2 * k + 1, c8)) = pack8(h1);
-    // the 8 column groups of pair k are 8 consecutive lanes
-    cr += __shfl_xor_sync(0xffffffffu, cr, 1);
-    cr += __shfl_xor_sync(0xffffffffu, cr, 2);
-    cr += __shfl_xor_sync(0xffffffffu, cr, 4);
-    if (c8 == 0) s_pe[k] = cr;
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) dgg += __shfl_xor_sync(0xffffffffu, dgg, off);
-  if (lane == 0) red[warp] = dgg;
   fence_async_smem();
+  const bool okc = (tid == 0) ? wait_mma(bars + 2, 0, a.status) : true;
   if (warp == 0) {
     tmem_alloc(s_tmem, L::TMEM_COLS);
     tmem_relinquish();
   }
-  if (tid == 0) {
-    mbar_init(bars, 1);
-    mbar_init(bars + 1, 1);
-    fence_mbar_init();
-  }
   tc_fence_before();
-  __syncthreads();
+  bool aborted = __syncthreads_or(!okc);
   tc_fence_after();
+  {
+    // <dGhat, G_c> and, per pair k, sum_p (dG1 G'0 - dG0 G'1) with dG =
+    // Rot(Phi_end) dGhat and G' = G_c+1 (the angle gradient of the chunk's
+    // outgoing rotation), from the bf16 blocks
+    float dgg = 0.f;
+#pragma unroll
+    for (int j = 0; j < kItems; ++j) {
+      const int e = tid + j * kTh, k = e >> 3, u = e & 7;
+      float sn, cs;
+      sincos_r(phi[t1 * kKP + k], &sn, &cs);
+      float gv[2][8], hv[2][8], nv[2][8];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const uint32_t off = sw128_off(2 * k + r, u);
+        const uint4 gu = *reinterpret_cast<const uint4*>(sm + L::GM + off);
+        const uint4 hu = *reinterpret_cast<const uint4*>(sm + L::DG + off);
+        const uint32_t gw[4] = {gu.x, gu.y, gu.z, gu.w}, hw[4] = {hu.x, hu.y, hu.z, hu.w};
+        const uint32_t nw[4] = {gn[j][r].x, gn[j][r].y, gn[j][r].z, gn[j][r].w};
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const float2 gf = unpack_bf16(gw[v]), hf = unpack_bf16(hw[v]), nf = unpack_bf16(nw[v]);
+          gv[r][2 * v] = gf.x; gv[r][2 * v + 1] = gf.y;
+          hv[r][2 * v] = hf.x; hv[r][2 * v + 1] = hf.y;
+          nv[r][2 * v] = nf.x; nv[r][2 * v + 1] = nf.y;
+        }
+      }
+      float cr = 0.f;
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        dgg = fmaf(hv[0][v], gv[0][v], fmaf(hv[1][v], gv[1][v], dgg));
+        const float o0 = cs * hv[0][v] - sn * hv[1][v], o1 = sn * hv[0][v] + cs * hv[1][v];
+        cr = fmaf(o1, nv[0][v], fmaf(-o0, nv[1][v], cr));
+      }
+      // the 8 chunks of pair k are 8 consecutive lanes
+      cr += __shfl_xor_sync(0xffffffffu, cr, 1);
+      cr += __shfl_xor_sync(0xffffffffu, cr, 2);
+      cr += __shfl_xor_sync(0xffffffffu, cr, 4);
+      if (u == 0) s_pe[k] = cr;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dgg += __shfl_xor_sync(0xffffffffu, dgg, off);
+    if (lane == 0) red[warp] = dgg;
+  }
   const uint32_t tm = *s_tmem;
 
   const uint64_t kCT = sw128_desc(sbase + L::CT, 16, 1024), mCT = sw128_desc(sbase + L::CT, kOPB, 1024);
@@ -525,7 +533,7 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
   const uint64_t mMS = sw128_desc(sbase + L::MS, kOPB, 1024);
 
   // ---- phase A ----------------------------------------------------------------
-  if (tid == 0) {
+  if (!aborted && tid == 0) {
     const uint32_t id64 = idesc_bf16(kM, 64, 0, 0), id128 = idesc_bf16(kM, 128, 0, 0);
     const uint32_t idAX = idesc_bf16(kM, kP, 0, 1);
 #pragma unroll
@@ -551,8 +559,8 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
     }
     mma_commit(bars);
   }
-  bool ok = (tid == 0) ? wait_mma(bars, 0, a.status) : true;
-  bool aborted = __syncthreads_or(!ok);
+  bool ok = (!aborted && tid == 0) ? wait_mma(bars, 0, a.status) : true;
+  aborted = __syncthreads_or(aborted || !ok);
   tc_fence_after();
 
   // Thread layout over 64-row accumulators: warp w reads TMEM lanes
