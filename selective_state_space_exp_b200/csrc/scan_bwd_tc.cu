@@ -265,27 +265,33 @@ struct SumsSmem {
   static constexpr int bytes(int Q) { return SMALL + (Q * kKP + 6 * Q) * 4 + 32; }
 };
 
+// Chunk c of chain (b, h): its tokens and groups.
+__device__ __forceinline__ Geo geo_at(const ScanArgs& a, int64_t b, int64_t h, int64_t c) {
+  Geo q;
+  q.b = b;
+  q.h = h;
+  q.g = h / (a.nheads / a.ngroups);
+  q.tg = h / (a.nheads / a.tgroups);
+  q.c = c;
+  q.t0 = c * a.Q;
+  const Chain ch = chain_of(a, b);
+  q.base = ch.base;
+  q.len = ch.len;
+  const int64_t rem = ch.len - q.t0;
+  q.nt = (int)(rem < 0 ? 0 : rem < a.Q ? rem : a.Q);
+  return q;
+}
+
+// Persistent: CTA i takes chunks i, i + gridDim.x, ... of all chains (index
+// (b H + h) nc + c), keeping its TMEM columns for the whole run.
 template <int R>
-__global__ void __launch_bounds__(kTh) bwd_tc_sums_kernel(const ScanArgs a, const BwdArgs g,
-                                                          const BwdWs w) {
+__global__ void __launch_bounds__(kTh, 3) bwd_tc_sums_kernel(const ScanArgs a, const BwdArgs g,
+                                                             const BwdWs w) {
   constexpr int Q = kM / R;
   using L = SumsSmem;
   extern __shared__ __align__(1024) uint8_t sm[];
   const uint32_t sbase = smem_u32(sm);
-  const Geo q = chunk_geo(a, blockIdx.x);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t cidx = (q.b * a.nheads + q.h) * a.nchunks + q.c;
-  float* S = w.G + cidx * (int64_t)kN * kP;  // turned into G_c by the state pass
-  float* D = w.D + cidx * (int64_t)kN * kP;
-  float* su = w.sums + cidx * (1 + kN);
-  if (q.nt <= 0) {  // past a short packed sequence: both states pass unchanged
-    for (int e = tid; e < kN * kP / 4; e += kTh) {
-      reinterpret_cast<float4*>(S)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-      reinterpret_cast<float4*>(D)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    for (int k = tid; k < 1 + kN; k += kTh) su[k] = (k == 0 || (k & 1)) ? 1.f : 0.f;
-    return;
-  }
   if ((sbase & 1023u) != 0) {
     if (tid == 0 && a.status) atomicCAS(a.status, 0, (int)M3_ERR_CUDA);
     return;
@@ -300,17 +306,6 @@ __global__ void __launch_bounds__(kTh) bwd_tc_sums_kernel(const ScanArgs a, cons
   // 8-byte aligned: 71 Q floats (Q even) before it
   uint64_t* bar = reinterpret_cast<uint64_t*>(s_e + Q);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar + 1);
-
-  prep_tc<Q>(a, q, lcum, gam, del, dts, phi);
-  const float lend = lcum[q.nt - 1];
-  for (int i = tid; i < Q; i += kTh) {
-    s_w[i] = i < q.nt ? expf(lend - lcum[i]) * del[i] : 0.f;
-    s_e[i] = i < q.nt ? expf(lcum[i]) : 0.f;
-  }
-  __syncthreads();
-  stage_bc<R>(a, q, phi, s_w, s_e, sm + L::WB, sm + L::EC);
-  stage_xdy<R>(a, g, q, sm + L::XS, sm + L::DYS);
-  fence_async_smem();
   if (warp == 0) {
     tmem_alloc(s_tmem, 128);
     tmem_relinquish();
@@ -323,50 +318,84 @@ __global__ void __launch_bounds__(kTh) bwd_tc_sums_kernel(const ScanArgs a, cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *s_tmem;
-  if (tid == 0) {
-    // M = 128 state rows (MN-major A: rows i of the chunk are K), N = 64
-    const uint32_t id = idesc_bf16(kN, kP, 1, 1);
-    const uint64_t dWB = sw128_desc(sbase + L::WB, kOPB, 1024);
-    const uint64_t dEC = sw128_desc(sbase + L::EC, kOPB, 1024);
-    const uint64_t dXS = sw128_desc(sbase + L::XS, kOPB, 1024);
-    const uint64_t dDY = sw128_desc(sbase + L::DYS, kOPB, 1024);
+  const uint64_t dWB = sw128_desc(sbase + L::WB, kOPB, 1024);
+  const uint64_t dEC = sw128_desc(sbase + L::EC, kOPB, 1024);
+  const uint64_t dXS = sw128_desc(sbase + L::XS, kOPB, 1024);
+  const uint64_t dDY = sw128_desc(sbase + L::DYS, kOPB, 1024);
+  const int64_t total = a.batch * a.nheads * a.nchunks;
+  uint32_t phase = 0;
+  bool aborted = false;
+  for (int64_t it = blockIdx.x; it < total && !aborted; it += gridDim.x) {
+    const int64_t bh = it / a.nchunks;
+    const Geo q = geo_at(a, bh / a.nheads, bh % a.nheads, it % a.nchunks);
+    float* S = w.G + it * (int64_t)kN * kP;  // turned into G_c by the state pass
+    float* D = w.D + it * (int64_t)kN * kP;
+    float* su = w.sums + it * (1 + kN);
+    if (q.nt <= 0) {  // past a short packed sequence: both states pass unchanged
+      for (int e = tid; e < kN * kP / 4; e += kTh) {
+        reinterpret_cast<float4*>(S)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<float4*>(D)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      for (int k = tid; k < 1 + kN; k += kTh) su[k] = (k == 0 || (k & 1)) ? 1.f : 0.f;
+      continue;  // uniform over the block
+    }
+    prep_tc<Q>(a, q, lcum, gam, del, dts, phi);
+    const float lend = lcum[q.nt - 1];
+    for (int i = tid; i < Q; i += kTh) {
+      s_w[i] = i < q.nt ? expf(lend - lcum[i]) * del[i] : 0.f;
+      s_e[i] = i < q.nt ? expf(lcum[i]) : 0.f;
+    }
+    __syncthreads();
+    stage_bc<R>(a, q, phi, s_w, s_e, sm + L::WB, sm + L::EC);
+    stage_xdy<R>(a, g, q, sm + L::XS, sm + L::DYS);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      // M = 128 state rows (MN-major A: rows i of the chunk are K), N = 64
+      const uint32_t id = idesc_bf16(kN, kP, 1, 1);
 #pragma unroll
-    for (int ks = 0; ks < kM / 16; ++ks)
-      mma_bf16_ss(tm, dadd(dWB, ks * 2048), dadd(dXS, ks * 2048), id, ks != 0);
+      for (int ks = 0; ks < kM / 16; ++ks)
+        mma_bf16_ss(tm, dadd(dWB, ks * 2048), dadd(dXS, ks * 2048), id, ks != 0);
 #pragma unroll
-    for (int ks = 0; ks < kM / 16; ++ks)
-      mma_bf16_ss(tm + kP, dadd(dEC, ks * 2048), dadd(dDY, ks * 2048), id, ks != 0);
-    mma_commit(bar);
+      for (int ks = 0; ks < kM / 16; ++ks)
+        mma_bf16_ss(tm + kP, dadd(dEC, ks * 2048), dadd(dDY, ks * 2048), id, ks != 0);
+      mma_commit(bar);
+    }
+    const bool ok = (tid == 0) ? wait_mma(bar, phase, a.status) : true;
+    phase ^= 1;
+    aborted = __syncthreads_or(!ok);
+    tc_fence_after();
+    if (!aborted) {
+      // warps 0-3: S_c, warps 4-7: D_c; thread row n = 32 (warp % 4) + lane
+      const int qd = warp & 3, which = warp >> 2;
+      const int n = 32 * qd + lane;
+      float* dst = (which ? D : S) + (int64_t)n * kP;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t v[32];
+        tmem_ld32(tm + ((uint32_t)(32 * qd) << 16) + which * kP + 32 * half, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(dst + 32 * half + j) =
+              make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                          __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+      }
+      if (tid == 0) su[0] = expf(lend);
+      for (int k = tid; k < kK; k += kTh) {
+        float sn, cs;
+        sincosf(phi[(q.nt - 1) * kKP + k], &sn, &cs);
+        su[1 + 2 * k] = cs;
+        su[2 + 2 * k] = sn;
+      }
+    }
+    // TMEM read and shared memory free before the next chunk
+    tc_fence_before();
+    __syncthreads();
   }
-  const bool ok = (tid == 0) ? wait_mma(bar, 0, a.status) : true;
-  const bool aborted = __syncthreads_or(!ok);
   tc_fence_after();
-  if (!aborted) {
-    // warps 0-3: S_c, warps 4-7: D_c; thread row n = 32 (warp % 4) + lane
-    const int qd = warp & 3, which = warp >> 2;
-    const int n = 32 * qd + lane;
-    float* dst = (which ? D : S) + (int64_t)n * kP;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint32_t v[32];
-      tmem_ld32(tm + ((uint32_t)(32 * qd) << 16) + which * kP + 32 * half, v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4*>(dst + 32 * half + j) =
-            make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                        __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-    }
-    if (tid == 0) su[0] = expf(lend);
-    for (int k = tid; k < kK; k += kTh) {
-      float sn, cs;
-      sincosf(phi[(q.nt - 1) * kKP + k], &sn, &cs);
-      su[1 + 2 * k] = cs;
-      su[2 + 2 * k] = sn;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
   if (warp == 0) tmem_dealloc(tm, 128);
 }
 
@@ -901,8 +930,15 @@ cudaError_t sums_r(const ScanArgs& f, const BwdArgs& g, const BwdWs& w, cudaStre
   const size_t smem = SumsSmem::bytes(kM / R);
   cudaError_t e = set_smem(bwd_tc_sums_kernel<R>, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)f.nchunks, (unsigned)f.nheads, (unsigned)f.batch);
-  bwd_tc_sums_kernel<R><<<grid, kTh, smem, st>>>(f, g, w);
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  // three CTAs per SM: shared memory (under 75 KB each), registers (at most
+  // 85 per thread, the launch bounds) and TMEM (3 x 128 of 512 columns)
+  static_assert(3 * (SumsSmem::bytes(kM) + 1024) <= 232448, "three CTAs per SM");
+  const int64_t total = f.batch * f.nheads * f.nchunks;
+  const int64_t slots = 3 * (int64_t)sms;
+  bwd_tc_sums_kernel<R><<<(unsigned)(total < slots ? total : slots), kTh, smem, st>>>(f, g, w);
   return cudaGetLastError();
 }
 
