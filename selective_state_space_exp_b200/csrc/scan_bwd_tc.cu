@@ -255,6 +255,82 @@ __device__ __forceinline__ void stage_xdy(const ScanArgs& a, const BwdArgs& g, c
   }
 }
 
+// A chunk's raw B, C, x and dy pieces in registers, loaded ahead of their use
+// (the loads of a chunk are in flight while its prefix sums run), then
+// rotated and staged as stage_bc and stage_xdy do.
+template <int R>
+struct RawChunk {
+  static constexpr int PB = kM * 16 / kTh, PX = kM * 8 / kTh;
+  uint4 b[PB], c[PB], x[PX], y[PX], y2[PX];
+
+  __device__ __forceinline__ void load(const ScanArgs& a, const BwdArgs& g, const Geo& q) {
+#pragma unroll
+    for (int j = 0; j < PB; ++j) {
+      const int e = (int)threadIdx.x + j * kTh, i = e >> 4, c16 = e & 15, t = i / R, r = i % R;
+      b[j] = c[j] = make_uint4(0u, 0u, 0u, 0u);
+      if (t < q.nt) {
+        const int64_t base =
+            ((q.base + q.t0 + t) * a.ngroups + q.g) * R * kN + (int64_t)r * kN + 8 * c16;
+        b[j] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.B) + base));
+        c[j] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.C) + base));
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < PX; ++j) {
+      const int e = (int)threadIdx.x + j * kTh, i = e >> 3, c8 = e & 7, t = i / R, r = i % R;
+      x[j] = y[j] = y2[j] = make_uint4(0u, 0u, 0u, 0u);
+      if (t < q.nt) {
+        const int64_t o = ((q.base + q.t0 + t) * a.nheads + q.h) * R * kP + (int64_t)r * kP + 8 * c8;
+        x[j] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.x) + o));
+        if (g.dy_f32) {
+          const uint4* py = reinterpret_cast<const uint4*>(static_cast<const float*>(g.dy) + o);
+          y[j] = __ldg(py);
+          y2[j] = __ldg(py + 1);
+        } else {
+          y[j] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(g.dy) + o));
+        }
+      }
+    }
+  }
+
+  // Rot(-Phi_t) B and C (unscaled) into 2 K-major blocks each; x, dy into one.
+  __device__ __forceinline__ void stage(const BwdArgs& g, const Geo& q, const float* phi,
+                                        uint8_t* bt, uint8_t* ct, uint8_t* xs, uint8_t* dys) const {
+#pragma unroll
+    for (int j = 0; j < PB; ++j) {
+      const int e = (int)threadIdx.x + j * kTh, i = e >> 4, c16 = e & 15, t = i / R;
+      uint32_t ob[4] = {0u, 0u, 0u, 0u}, oc[4] = {0u, 0u, 0u, 0u};
+      if (t < q.nt) {
+        const uint32_t wb[4] = {b[j].x, b[j].y, b[j].z, b[j].w};
+        const uint32_t wc[4] = {c[j].x, c[j].y, c[j].z, c[j].w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float sn, cs;
+          sincos_r(phi[t * kKP + 4 * c16 + u], &sn, &cs);
+          const float2 bf = unpack_bf16(wb[u]), cf = unpack_bf16(wc[u]);
+          ob[u] = pack_bf16(cs * bf.x + sn * bf.y, -sn * bf.x + cs * bf.y);
+          oc[u] = pack_bf16(cs * cf.x + sn * cf.y, -sn * cf.x + cs * cf.y);
+        }
+      }
+      const uint32_t off = (c16 >> 3) * kOPB + sw128_off(i, c16 & 7);
+      *reinterpret_cast<uint4*>(bt + off) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+      *reinterpret_cast<uint4*>(ct + off) = make_uint4(oc[0], oc[1], oc[2], oc[3]);
+    }
+#pragma unroll
+    for (int j = 0; j < PX; ++j) {
+      const int e = (int)threadIdx.x + j * kTh, i = e >> 3, c8 = e & 7;
+      uint4 yv = y[j];
+      if (g.dy_f32)  // eight fp32 values -> bf16
+        yv = make_uint4(pack_bf16(__uint_as_float(y[j].x), __uint_as_float(y[j].y)),
+                        pack_bf16(__uint_as_float(y[j].z), __uint_as_float(y[j].w)),
+                        pack_bf16(__uint_as_float(y2[j].x), __uint_as_float(y2[j].y)),
+                        pack_bf16(__uint_as_float(y2[j].z), __uint_as_float(y2[j].w)));
+      *reinterpret_cast<uint4*>(xs + sw128_off(i, c8)) = x[j];
+      *reinterpret_cast<uint4*>(dys + sw128_off(i, c8)) = yv;
+    }
+  }
+};
+
 // ---- step 1: S_c and D_c ----------------------------------------------------
 // Shared memory: w Bt (2 blocks), exp(Lam) Ct (2 blocks), x, dy (1 block
 // each), then the prefix sums.  TMEM: S_c in columns 0-63, D_c in 64-127,
@@ -487,6 +563,8 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
       gn[j][r] = __ldg(reinterpret_cast<const uint4*>(nb + sw128_off(row, u)));
     }
   }
+  RawChunk<R> raw;
+  raw.load(a, g, q);  // in flight during the prefix sums
   prep_tc<Q>(a, q, lcum, gam, del, dts, phi);
   const int t1 = nt - 1;
   const float lam_end = lcum[t1];
@@ -496,8 +574,7 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
     beta[i] = dLam[i] = dgam[i] = ddel[i] = colF[i] = thT[i] = 0.f;
   }
   __syncthreads();
-  stage_bc<R>(a, q, phi, nullptr, nullptr, sm + L::BT, sm + L::CT);
-  stage_xdy<R>(a, g, q, sm + L::XS, sm + L::DYS);
+  raw.stage(g, q, phi, sm + L::BT, sm + L::CT, sm + L::XS, sm + L::DYS);
   fence_async_smem();
   const bool okc = (tid == 0) ? wait_mma(bars + 2, 0, a.status) : true;
   if (warp == 0) {
