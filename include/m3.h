@@ -86,7 +86,10 @@ typedef enum {
   M3_ERR_ALIGNMENT = -3,        /* a pointer violates its alignment rule       */
   M3_ERR_WORKSPACE = -4,        /* workspace null, misaligned or too small     */
   M3_ERR_CUDA = -5,             /* a CUDA launch or runtime call failed        */
-  M3_ERR_TIMEOUT = -6           /* a bounded device-side wait gave up          */
+  M3_ERR_TIMEOUT = -6,          /* a bounded device-side wait gave up          */
+  M3_ERR_BOUNDS = -7            /* bounds-checked builds only: a kernel formed
+                                   an index outside its tensor and skipped the
+                                   access (a library defect, never the caller's) */
 } m3_status;
 
 /* Flags (m3_shape.flags). */

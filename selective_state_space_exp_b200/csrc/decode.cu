@@ -151,6 +151,9 @@ __global__ void __launch_bounds__(kThreads, DecodeOcc<R>::value) decode_kernel(c
   const int hpg = (int)(H / G);  // heads per group
   // thread 0: bring head hd's state and operands into buffer bi
   auto issue = [&](int64_t hd, int64_t bg, int bi, bool with_bc) {
+    // (a skipped copy leaves its barrier incomplete: the wait then times out
+    // after the bounds error is recorded)
+    if (!M3_IN(hd, total, a.status) || !M3_IN(bg, a.batch * G, a.status)) return;
     uint8_t* st = sm + bi * sp.st_stride;
     uint8_t* ops = sm + sp.ops0 + bi * sp.ops_stride;
     fence_async_smem();
@@ -296,8 +299,10 @@ __global__ void __launch_bounds__(kThreads, DecodeOcc<R>::value) decode_kernel(c
         o0[2 * jj] = w0.x; o0[2 * jj + 1] = w0.y;
         o1[2 * jj] = w1.x; o1[2 * jj + 1] = w1.y;
       }
-      __stcs(dst + (2 * k) * rowq + pv, make_float4(o0[0], o0[1], o0[2], o0[3]));
-      __stcs(dst + (2 * k + 1) * rowq + pv, make_float4(o1[0], o1[1], o1[2], o1[3]));
+      if (M3_IN(hd * (int64_t)N * P / 4 + (2 * k + 1) * rowq + pv, total * N * P / 4, a.status)) {
+        __stcs(dst + (2 * k) * rowq + pv, make_float4(o0[0], o0[1], o0[2], o0[3]));
+        __stcs(dst + (2 * k + 1) * rowq + pv, make_float4(o1[0], o1[1], o1[2], o1[3]));
+      }
     }
 
     // y: kslots of one warp share columns every PV lanes; then across warps
@@ -322,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, DecodeOcc<R>::value) decode_kernel(c
     for (int i = tid; i < R * P; i += kThreads) {
       float acc = 0.f;
       for (int q = 0; q < kWarps; ++q) acc += s_red[q * R * P + i];
-      io_store(a.y, hd * R * P + i, acc, a.bf16);
+      if (M3_IN(hd * R * P + i, total * R * P, a.status)) io_store(a.y, hd * R * P + i, acc, a.bf16);
     }
     __syncthreads();  // buffer bi, staging and partial sums free
     if (nbuf == 1 && tid == 0 && ihd < h_end) issue_next();  // one buffer: the next head now
@@ -402,6 +407,9 @@ __global__ void __launch_bounds__(kStreamThreads, 7) stream_decode_kernel(const 
   const float4* src = reinterpret_cast<const float4*>(a.state_in + bh * (int64_t)N * P);
   float4* dst = reinterpret_cast<float4*>(a.state_out + bh * (int64_t)N * P);
   const int rowq = P / 4;
+  // the head's float4 pieces end inside the state tensor
+  if (!M3_IN((bh + 1) * (int64_t)N * P / 4 - 1, a.batch * a.nheads * (int64_t)N * P / 4, a.status))
+    return;  // uniform over the block
 
   // the first row pairs' loads go out before the per-head operands are staged
   float4 r0[kStreamPairs], r1[kStreamPairs];
@@ -486,7 +494,7 @@ __global__ void __launch_bounds__(kStreamThreads, 7) stream_decode_kernel(const 
   for (int i = tid; i < P; i += kStreamThreads) {
     float acc = 0.f;
     for (int q = 0; q < nslots; ++q) acc += s_red[q * P + i];
-    io_store(a.y, bh * P + i, acc, a.bf16);
+    if (M3_IN(bh * P + i, a.batch * a.nheads * P, a.status)) io_store(a.y, bh * P + i, acc, a.bf16);
   }
 }
 

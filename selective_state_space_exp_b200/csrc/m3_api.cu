@@ -140,6 +140,7 @@ M3_API const char* m3_status_string(int st) {
     case M3_ERR_WORKSPACE: return "M3_ERR_WORKSPACE";
     case M3_ERR_CUDA: return "M3_ERR_CUDA";
     case M3_ERR_TIMEOUT: return "M3_ERR_TIMEOUT";
+    case M3_ERR_BOUNDS: return "M3_ERR_BOUNDS";
     default: return "M3_ERR_UNKNOWN";
   }
 }

@@ -10,6 +10,22 @@
 
 namespace m3 {
 
+// Bounds-checked builds (compiled with -DM3_DEBUG_BOUNDS; `_build.build(debug=True)`
+// writes lib/libm3_debug.so): the kernels' global writes, and their reads of
+// tensors and the workspace at computed indices, first test the index against
+// the extent of the tensor it addresses (elements, from the call's shape);
+// an index outside records M3_ERR_BOUNDS in the device status word and the
+// access is skipped.  In normal builds the test is the constant true.
+#ifdef M3_DEBUG_BOUNDS
+static __device__ __noinline__ void bounds_fail(int* status) {
+  if (status) atomicCAS(status, 0, (int)M3_ERR_BOUNDS);
+}
+#define M3_IN(i, n, st) \
+  (((int64_t)(i) >= 0 && (int64_t)(i) < (int64_t)(n)) ? true : (::m3::bounds_fail(st), false))
+#else
+#define M3_IN(i, n, st) true
+#endif
+
 // Element access for the io dtype (fp32 or bf16).
 __device__ __forceinline__ float io_load(const void* p, int64_t i, bool bf16) {
   return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i])

@@ -67,6 +67,7 @@ template <int R, int TPT>
 __global__ void __launch_bounds__(512) bwd_sums_kernel(const ScanArgs a, const BwdArgs g,
                                                        const BwdWs w) {
   const Geo q = chunk_geo(a, blockIdx.x);
+  if (!simt::geo_ok(a, q)) return;  // uniform over the block
   const int N = (int)a.N, P = (int)a.P, K = N / 2, Q = (int)a.Q;
   const int tid = threadIdx.x, nth = blockDim.x;
   extern __shared__ __align__(16) float sm[];
@@ -224,6 +225,7 @@ __global__ void __launch_bounds__(kThreads) bwd_pass_kernel(const ScanArgs a, co
   if (idx >= K * PG) return;  // K * P / 4 is a multiple of 32: whole warps leave
   const int k = idx / PG, p0 = 4 * (idx % PG);
   const int64_t so = (b * H + h) * (int64_t)N * P;
+  if (!M3_IN(b, a.batch, a.status) || !M3_IN(h, H, a.status)) return;
   const int64_t grp = h / (H / a.ngroups);
   const Chain chn = chain_of(a, b);
   const int64_t i0 = (2 * k) * P + p0, i1 = (2 * k + 1) * P + p0;
@@ -478,6 +480,7 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(const ScanArgs a, c
   constexpr int NGT = NGT_ ? NGT_ : 8 / TI;  // N-wide products: 4-column groups per thread
   constexpr int PCT = PCT_ ? PCT_ : 128 / 16;  // dX columns per thread
   const Geo q = chunk_geo(a, blockIdx.x);
+  if (!simt::geo_ok(a, q)) return;  // uniform over the block
   const int N = (int)a.N, P = (int)a.P, K = N / 2;
   const int64_t H = a.nheads;
   const ChunkSmem L(M, N, P, Q);

@@ -404,6 +404,7 @@ __global__ void __launch_bounds__(kTh, 3) bwd_tc_sums_kernel(const ScanArgs a, c
   for (int64_t it = blockIdx.x; it < total && !aborted; it += gridDim.x) {
     const int64_t bh = it / a.nchunks;
     const Geo q = geo_at(a, bh / a.nheads, bh % a.nheads, it % a.nchunks);
+    if (!simt::geo_ok(a, q)) continue;  // uniform over the block
     float* S = w.G + it * (int64_t)kN * kP;  // turned into G_c by the state pass
     float* D = w.D + it * (int64_t)kN * kP;
     float* su = w.sums + it * (1 + kN);
@@ -509,7 +510,7 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
   const uint32_t sbase = smem_u32(sm);
   const Geo q = chunk_geo(a, blockIdx.x);
   const int nt = q.nt;
-  if (nt <= 0) return;  // uniform over the block
+  if (nt <= 0 || !simt::geo_ok(a, q)) return;  // uniform over the block
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if ((sbase & 1023u) != 0) {
     if (tid == 0 && a.status) atomicCAS(a.status, 0, (int)M3_ERR_CUDA);

@@ -90,6 +90,7 @@ __host__ __device__ __forceinline__ WsView ws_view(const ScanArgs& a) {
 template <int R, int TPT>
 __global__ void __launch_bounds__(kThreads) chunk_state_kernel(const ScanArgs a) {
   const Geo q = chunk_geo(a, blockIdx.x);
+  if (!simt::geo_ok(a, q)) return;  // uniform over the block
   const int N = (int)a.N, P = (int)a.P, K = N / 2, Q = (int)a.Q;
   extern __shared__ __align__(16) float sm[];
   float* lcum = sm;
@@ -170,6 +171,7 @@ __global__ void __launch_bounds__(kThreads) state_pass_kernel(const ScanArgs a) 
   const Chain ch = chain_of(a, b);
   float g0 = 0.f, g1 = 0.f;
   const int64_t so = ((b * H + h) * N) * P;
+  if (!M3_IN(b, a.batch, a.status) || !M3_IN(h, a.nheads, a.status)) return;
   if (a.h0) {
     g0 = a.h0[so + (2 * k) * P + p];
     g1 = a.h0[so + (2 * k + 1) * P + p];
@@ -213,7 +215,7 @@ __global__ void __launch_bounds__(kThreads) state_pass_kernel(const ScanArgs a) 
       g1 = sn[j] * v0 + cs[j] * v1;
     }
   }
-  if (a.final_state) {
+  if (a.final_state && M3_IN(so + (2 * k + 1) * P + p, a.batch * H * N * P, a.status)) {
     a.final_state[so + (2 * k) * P + p] = g0;
     a.final_state[so + (2 * k + 1) * P + p] = g1;
   }
@@ -227,6 +229,7 @@ __global__ void __launch_bounds__(kThreads) chunk_output_kernel(const ScanArgs a
   const int64_t c = blockIdx.x / tiles_per_chunk;
   const int tile = blockIdx.x % tiles_per_chunk;
   const Geo q = chunk_geo(a, c);
+  if (!simt::geo_ok(a, q)) return;  // uniform over the block
   const int TT = kOutRows / R;          // tokens per output tile
   const int tt0 = tile * TT;            // first token (chunk-local) of the tile
   if (tt0 >= q.nt) return;
@@ -324,9 +327,9 @@ __global__ void __launch_bounds__(kThreads) chunk_output_kernel(const ScanArgs a
   for (int i = 0; i < YPT; ++i) {
     const int ro = ro0 + i * RS;
     const int t = tt0 + ro / R, r = ro % R;
-    if (t < tt1)
-      io_store(a.y, ((q.base + q.t0 + t) * a.nheads + q.h) * R * P + (int64_t)r * P + p,
-               acc[i], a.bf16);
+    const int64_t yo = ((q.base + q.t0 + t) * a.nheads + q.h) * R * P + (int64_t)r * P + p;
+    if (t < tt1 && M3_IN(yo, a.total_tokens * a.nheads * R * P, a.status))
+      io_store(a.y, yo, acc[i], a.bf16);
   }
 }
 

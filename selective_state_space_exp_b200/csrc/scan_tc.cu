@@ -223,6 +223,10 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   const int64_t L = chn.len, tokb = chn.base;
   const int64_t g = h / (H / G);
   const int64_t tg = h / (H / a.tgroups);  // theta group
+  // bounds-checked builds: the CTA's chain and segment, and its tokens
+  if (!M3_IN(b, a.batch, a.status) || !M3_IN(h, H, a.status) || !M3_IN(seg, pl.nseg, a.status) ||
+      (L > 0 && !M3_IN(tokb + L - 1, a.total_tokens, a.status)))
+    return;  // uniform over the block
 
   if (warp == 0) {
     tmem_alloc(s_tmem, C::TMEM_COLS);
@@ -934,6 +938,7 @@ __global__ void __launch_bounds__(256) tc_seg_pass_kernel(const ScanArgs a, cons
   const int64_t g = h / (H / G);
   const Chain chn = chain_of(a, b);
   const int64_t so = (b * H + h) * kN * kP;
+  if (!M3_IN(b, a.batch, a.status) || !M3_IN(h, H, a.status)) return;
   float g0 = a.h0 ? a.h0[so + (2 * k) * kP + p] : 0.f;
   float g1 = a.h0 ? a.h0[so + (2 * k + 1) * kP + p] : 0.f;
   if (a.B_prev && chn.len > 0) {  // the left endpoint term waits for a token

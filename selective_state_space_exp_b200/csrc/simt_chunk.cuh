@@ -29,6 +29,14 @@ __device__ __forceinline__ Geo chunk_geo(const ScanArgs& a, int64_t c) {
   return q;
 }
 
+// Bounds-checked builds: the chunk's batch, head and chunk indices and its
+// token range lie inside the call's tensors (always true otherwise).
+__device__ __forceinline__ bool geo_ok(const ScanArgs& a, const Geo& q) {
+  return M3_IN(q.b, a.batch, a.status) && M3_IN(q.h, a.nheads, a.status) &&
+         M3_IN(q.c, a.nchunks, a.status) &&
+         (q.nt <= 0 || M3_IN(q.base + q.t0 + q.nt - 1, a.total_tokens, a.status));
+}
+
 // Chunk-local prefix sums and trapezoid weights into shared memory:
 // lcum[Q], gam[Q], del[Q], dts[Q], phi[Q][K].
 __device__ __forceinline__ void chunk_prep(const ScanArgs& a, const Geo& q, float* lcum, float* gam,

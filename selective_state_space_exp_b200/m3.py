@@ -14,7 +14,10 @@ import threading
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "lib", "libm3.so")
+# M3_LIBRARY=debug selects the bounds-checked build (lib/libm3_debug.so, see
+# _build.build(debug=True)), whose kernels report M3_ERR_BOUNDS.
+LIB_PATH = os.path.join(_PKG, "lib", "libm3_debug.so" if os.environ.get("M3_LIBRARY") == "debug"
+                        else "libm3.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "m3.h")
 
 M3_F32, M3_BF16 = 0, 1
@@ -37,7 +40,7 @@ def theta_flag(theta_groups: int, ngroups: int, nheads: int) -> int:
 
 STATUS = {0: "M3_OK", -1: "M3_ERR_INVALID_ARGUMENT", -2: "M3_ERR_UNSUPPORTED",
           -3: "M3_ERR_ALIGNMENT", -4: "M3_ERR_WORKSPACE", -5: "M3_ERR_CUDA",
-          -6: "M3_ERR_TIMEOUT"}
+          -6: "M3_ERR_TIMEOUT", -7: "M3_ERR_BOUNDS"}
 
 
 class M3Error(RuntimeError):
@@ -66,7 +69,7 @@ def load() -> ctypes.CDLL:
         if _lib is None:
             if not os.path.exists(LIB_PATH):
                 raise RuntimeError(
-                    f"libm3.so not built ({LIB_PATH}); run selective_state_space_exp_b200/_build.py")
+                    f"library not built ({LIB_PATH}); run selective_state_space_exp_b200/_build.py")
             L = ctypes.CDLL(LIB_PATH)
             vp, sp = ctypes.c_void_p, ctypes.POINTER(Shape)
             L.m3_version.restype = ctypes.c_char_p
