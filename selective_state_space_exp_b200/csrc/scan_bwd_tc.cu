@@ -27,10 +27,12 @@
 //             AB += (M o DX)^T Ct    -> dBt = (M o DX)^T Ct + w X dGhat^T
 //             AX += (M o S)^T dY     -> dX  = (M o S)^T dY + w Bt dGhat
 // then the rotations back to B and C, the angle gradients and the backward
-// of the chunk-local prefix sums, as on the CUDA cores.  TMEM holds 448 of
-// its 512 columns; the global loads of a chunk are staged before its TMEM is
+// of the chunk-local prefix sums, as on the CUDA cores.  G_c, dGhat and
+// G_c+1 arrive as bf16 blocks in the MMA operand layout written by step 2
+// (the first two by bulk copy into shared memory).  TMEM holds 448 of its
+// 512 columns; the global loads of a chunk are staged before its TMEM is
 // allocated, so a second CTA on the SM prepares its chunk while the first
-// one computes.
+// one computes.  Step 1 is persistent: three CTAs per SM walk the chunks.
 #include <cuda_bf16.h>
 
 #include "m3_internal.cuh"
