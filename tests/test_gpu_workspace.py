@@ -85,19 +85,23 @@ def test_poisoned_workspace_varlen(simt):
 ATOMIC = ("dt", "A", "lam", "theta", "B", "C", "B_prev", "x_prev")
 
 
-def test_poisoned_workspace_bwd():
+@pytest.mark.parametrize("simt", [False, True], ids=["tcgen05", "cuda_core"])
+def test_poisoned_workspace_bwd(simt):
+    """Both backward forms (the tensor-core one also reads the state pass's
+    bf16 operand blocks from the workspace)."""
     w = I.Workload(I.Shape(2, 300, 4, 64, 128, 2, 1, 64, "bf16"), decay="slow", with_h0=True,
                    with_prev=True)
     g = to_dev(I.make_scan_inputs(w, seed=9520))
     gen = torch.Generator(device="cuda").manual_seed(9521)
     dy = torch.randn(g["x"].shape, generator=gen, device="cuda").to(torch.bfloat16)
     dfin = torch.randn(g["h0"].shape, generator=gen, device="cuda")
-    n = m3.bwd_workspace_size(m3.scan_shape(g["x"], g["B"], 64, False, g["theta"]))
+    n = m3.bwd_workspace_size(m3.scan_shape(g["x"], g["B"], 64, simt, g["theta"]))
     assert n > 0
     args = (g["x"], g["dt"], g["A"], g["lam"], g["theta"], g["B"], g["C"], dy, 64, g["h0"],
             g["B_prev"], g["x_prev"], dfin)
-    r1 = m3.m3_scan_bwd(*args, workspace=nan_bytes(n))
-    r0 = m3.m3_scan_bwd(*args, workspace=torch.zeros(n, dtype=torch.uint8, device="cuda"))
+    r1 = m3.m3_scan_bwd(*args, workspace=nan_bytes(n), simt=simt)
+    r0 = m3.m3_scan_bwd(*args, workspace=torch.zeros(n, dtype=torch.uint8, device="cuda"),
+                        simt=simt)
     assert m3.m3_stream_status() == 0
     for k in r0:
         assert torch.isfinite(r1[k]).all(), k
