@@ -447,20 +447,33 @@ __global__ void __launch_bounds__(kTh, 3) bwd_tc_sums_kernel(const ScanArgs a, c
     aborted = __syncthreads_or(!ok);
     tc_fence_after();
     if (!aborted) {
-      // warps 0-3: S_c, warps 4-7: D_c; thread row n = 32 (warp % 4) + lane
-      const int qd = warp & 3, which = warp >> 2;
+      // S_c, then D_c, through a 32 KB staging block over the consumed operands:
+      // thread row n = 32 (warp % 4) + lane, column half warp / 4; float4 j of
+      // row n sits in slot (j + n) mod 16 of the row (no bank conflicts either
+      // way), then all threads write the matrix out in contiguous 16-byte pieces.
+      const int qd = warp & 3, hf = warp >> 2;
       const int n = 32 * qd + lane;
-      float* dst = (which ? D : S) + (int64_t)n * kP;
+      float* stg = reinterpret_cast<float*>(sm + L::WB);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      for (int which = 0; which < 2; ++which) {
         uint32_t v[32];
-        tmem_ld32(tm + ((uint32_t)(32 * qd) << 16) + which * kP + 32 * half, v);
+        tmem_ld32(tm + ((uint32_t)(32 * qd) << 16) + which * kP + 32 * hf, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(dst + 32 * half + j) =
-              make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                          __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const int j = 8 * hf + j4;
+          *reinterpret_cast<float4*>(stg + n * kP + ((j + n) & 15) * 4) =
+              make_float4(__uint_as_float(v[4 * j4]), __uint_as_float(v[4 * j4 + 1]),
+                          __uint_as_float(v[4 * j4 + 2]), __uint_as_float(v[4 * j4 + 3]));
+        }
+        __syncthreads();
+        float4* dst = reinterpret_cast<float4*>(which ? D : S);
+#pragma unroll
+        for (int it = 0; it < kN * kP / 4 / kTh; ++it) {
+          const int e = tid + it * kTh, r = e >> 4, j = e & 15;
+          dst[e] = *reinterpret_cast<const float4*>(stg + r * kP + ((j + r) & 15) * 4);
+        }
+        __syncthreads();
       }
       if (tid == 0) su[0] = expf(lend);
       for (int k = tid; k < kK; k += kTh) {
@@ -873,17 +886,18 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
         if (trow && (lane % R) == 0) atomicAdd(dPhi + tr * kKP + n0 / 2 + j, v);
       }
     }
-    {  // dX
+    {  // dX, staged over the masked scores (phase B has read them): float4 j of
+       // row i in slot (j + i) mod 16, written out once TMEM is released
       uint32_t v[16];
       tmem_ld16x2<16>(lb + L::AX_COL + 32 * hh, v);
       tmem_ld_wait();
-      if (trow) {
-        float* dxo = g.dx + ((q.base + q.t0 + tr) * H + q.h) * R * kP + (int64_t)rr * kP + c64;
+      float* stg = reinterpret_cast<float*>(sm + L::GM);
 #pragma unroll
-        for (int j = 0; j < 16; j += 4)
-          *reinterpret_cast<float4*>(dxo + j) =
-              make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                          __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+      for (int j4 = 0; j4 < 4; ++j4) {
+        const int j = c64 / 4 + j4;
+        *reinterpret_cast<float4*>(stg + rho * kP + ((j + rho) & 15) * 4) =
+            make_float4(__uint_as_float(v[4 * j4]), __uint_as_float(v[4 * j4 + 1]),
+                        __uint_as_float(v[4 * j4 + 2]), __uint_as_float(v[4 * j4 + 3]));
       }
     }
   }
@@ -891,6 +905,18 @@ __global__ void __launch_bounds__(kTh, 2) bwd_tc_chunk_kernel(const ScanArgs a, 
   __syncthreads();
   if (warp == 0) tmem_dealloc(tm, L::TMEM_COLS);
   if (aborted) return;
+  {  // dx of the chunk's tokens: a token's R rows are contiguous, 16-byte pieces
+    const float* stg = reinterpret_cast<const float*>(sm + L::GM);
+#pragma unroll
+    for (int e0 = 0; e0 < kM * 16; e0 += kTh) {
+      const int e = e0 + tid, i = e >> 4, j = e & 15, t = i / R, r = i % R;
+      if (t < nt) {
+        float* dxo = g.dx + ((q.base + q.t0 + t) * H + q.h) * R * kP + (int64_t)r * kP + 4 * j;
+        *reinterpret_cast<float4*>(dxo) =
+            *reinterpret_cast<const float4*>(stg + i * kP + ((j + i) & 15) * 4);
+      }
+    }
+  }
 
   // ---- the scalar gradients (as on the CUDA cores) ----------------------------
   for (int k = tid; k < kK; k += kTh) dPhi[t1 * kKP + k] += s_pe[k];
