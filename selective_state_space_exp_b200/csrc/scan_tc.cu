@@ -126,6 +126,17 @@ struct Cfg {
   }
   __host__ __device__ static constexpr int acc_col(int mt) { return NT == 2 ? y_col(mt) : MT; }
   static_assert(SC_COL + kP <= TMEM_COLS, "TMEM columns");
+  // Two-tile chunks (M = 256) run three MMA chains side by side instead of
+  // one dependent chain: the chunk state in two halves over the rows (K),
+  // rows 0-127 into SC_COL and rows 128-255 into SC2_COL, interleaved with
+  // tile 0's scores; once the state update has read both halves, the output
+  // accumulators of tile 0 and tile 1 take their columns (Y2T_COL / SC_COL)
+  // and both tiles' Ct G products are issued together before the masks.  The
+  // masked scores stay in TMEM as packed bf16 (each warp's 16-column step
+  // over columns it has already read) and are P x's A operand.
+  static constexpr int SC2_COL = 448;
+  __host__ __device__ static constexpr int acc2_col(int mt) { return mt == 0 ? SC2_COL : SC_COL; }
+  static_assert(NT != 2 || SC2_COL + kP <= TMEM_COLS, "TMEM columns");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -575,7 +586,12 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       for (int ks = 0; ks < M / 16; ++ks) {
         const uint64_t ad = dadd(dBmn, ks * 2048);
         const uint64_t bd = dadd(dX, ks * 2048);
-        mma_bf16_ss(tm + C::SC_COL, ad, bd, id3, ks != 0);
+        if constexpr (NT == 2) {  // two row halves as interleaved chains
+          const int hf = ks & 1, kst = (ks >> 1) + 8 * hf;
+          mma_bf16_ss(tm + (hf ? C::SC2_COL : C::SC_COL), dadd(dBmn, kst * 2048), dadd(dX, kst * 2048),
+                      id3, ks > 1);
+        } else
+          mma_bf16_ss(tm + C::SC_COL, ad, bd, id3, ks != 0);
       }
     };
     auto issue_mma1 = [&]() {  // S' = Ct Bh^T per tile, each on its own barrier (one thread)
@@ -597,6 +613,28 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       if (MODE == MODE_STATE) {
         issue_mma3();
         mma_commit(s_bar);
+      } else if (NT == 2 && !plain) {  // tile 0's scores and both chunk-state halves interleaved
+        const uint32_t id3 = idesc_bf16(kN, kP, 1, 1);
+        const uint32_t id0 = idesc_bf16(MT, MT, 0, 0);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          mma_bf16_ss(tm + C::s_col(0), dadd(dC, (k >> 2) * C::OPB + (k & 3) * 32),
+                      dadd(dB, (k >> 2) * C::OPB + (k & 3) * 32), id0, k != 0);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {  // rows 16 (k + 8 hf) .. of half hf
+            const uint32_t kst = (uint32_t)(k + 8 * hf);
+            mma_bf16_ss(tm + (hf ? C::SC2_COL : C::SC_COL), dadd(dBmn, kst * 2048), dadd(dX, kst * 2048),
+                        id3, k != 0);
+          }
+        }
+        mma_commit(s_bar);
+        mma_commit(s_bar1);
+        const uint32_t id1 = idesc_bf16(MT, 2 * MT, 0, 0);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_bf16_ss(tm + C::s_col(1), dadd(dC, (k >> 2) * C::OPB + MT * 128 + (k & 3) * 32),
+                      dadd(dB, (k >> 2) * C::OPB + (k & 3) * 32), id1, k != 0);
+        mma_commit(s_bar1b);
       } else if (!plain) {  // MMA3 (and MMA4 for one-tile chunks) first, then the scores
         issue_mma3();
         if (C::EARLY4) issue_mma4(0, C::acc_col(0), false);
@@ -630,6 +668,21 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
           ov[e] = pack_bf16(g.x, g.y);
         }
         *reinterpret_cast<uint4*>(pq) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+        if constexpr (NT == 2 && MODE == MODE_FULL) {
+          // two-tile chunks: Ct_t <- exp(Lam_t) Ct_t, so that Ct G lands in the
+          // one output accumulator already scaled (MMA1 has read Ct)
+          const float fc = ex2(s_lg[t]);
+          uint8_t* pc = sm + C::C_OFF + ((q >> 3) & 1) * C::OPB + sw128_off(row, q & 7);
+          const uint4 w = *reinterpret_cast<const uint4*>(pc);
+          const uint32_t iw[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 g = fmul2(make_float2(fc, fc), make_float2(__uint_as_float(iw[e] << 16),
+                                                                  __uint_as_float(iw[e] & 0xffff0000u)));
+            ov[e] = pack_bf16(g.x, g.y);
+          }
+          *reinterpret_cast<uint4*>(pc) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+        }
       }
       fence_async_smem();
       tc_fence_before();
@@ -659,6 +712,13 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       for (int pc = 0; pc < CW / 16; ++pc) {
         uint32_t sv[16];
         tmem_ld16(tm + lane_base + C::SC_COL + CW * cq + 16 * pc, sv);
+        if constexpr (NT == 2) {  // the second half of the rows
+          uint32_t sw[16];
+          tmem_ld16(tm + lane_base + C::SC2_COL + CW * cq + 16 * pc, sw);
+          tmem_ld_wait();
+#pragma unroll
+          for (int p = 0; p < 16; ++p) sv[p] = __float_as_uint(__uint_as_float(sv[p]) + __uint_as_float(sw[p]));
+        }
         tmem_ld_wait();
 #pragma unroll
         for (int p = 0; p < 16; p += 2) {
@@ -682,9 +742,21 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     if (MODE == MODE_FULL) {
       const bool ok1 = (tid == 0) ? wait_bar(s_bar1, phase1, a.status) : true;
       phase1 ^= 1;
+      tc_fence_before();  // the chunk-state columns are read
       if (__syncthreads_or(!ok1)) { aborted = true; break; }
       tc_fence_after();
       if (C::EARLY4) prefetch_c(c + 1);  // MMA1 and MMA4 have read Ct
+      if constexpr (NT == 2) {  // Ct G of both tiles, interleaved, into the freed state columns
+        if (tid == 0) {
+          const uint32_t id4 = idesc_bf16(MT, kP, 0, 1);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+              mma_bf16_ss(tm + C::acc2_col(mt), dadd(dC, (k >> 2) * C::OPB + mt * MT * 128 + (k & 3) * 32),
+                          dadd(dG, k * 2048), id4, k != 0);
+        }
+      }
 
       // ---- per score tile: mask into P (bf16, K-major), then its MMA2 (P x) -----
       //   factored: P'[(t,r),(s,r')] = S' * (s < t ? 1 : s == t ? gamma_t / delta_t : 0)
@@ -755,6 +827,26 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
           const int ch0 = cth / 8;
           *reinterpret_cast<uint4*>(blk + sw128_off(rho, ch0)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           *reinterpret_cast<uint4*>(blk + sw128_off(rho, ch0 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else if constexpr (NT == 2) {
+          // P' in TMEM: step st reads the warp's score columns [16 st, +16)
+          // and stores their packed bf16 over columns [8 st, +8), which this
+          // or an earlier step has read (K step j of the tile: part
+          // 16 j / cpt, 8-column step j mod (cpt / 16))
+          const uint32_t pbase = tm + lane_base + C::s_col(mt) + cq * cpt;
+          for (int st = 0; st < cpt / 16; ++st) {
+            const int s0 = (cq * cpt + 16 * st) / R;  // first key token of the step
+            uint32_t pk[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) pk[j] = 0u;
+            if (s0 <= t_hi) {  // warp-uniform: steps wholly above the diagonal stay zero
+              uint32_t v[16];
+              tmem_ld16(pbase + 16 * st, v);
+              tmem_ld_wait();
+              if (trow) mask16(v, s0, pk);
+            }
+            tmem_st8(pbase + 8 * st, pk);
+          }
+          tmem_st_wait();
         } else {
           for (int cc = cq * cpt / 16; cc < (cq + 1) * cpt / 16; cc += 2) {
             const int s0 = cc * 16 / R;  // first token of these 32 columns
@@ -783,7 +875,15 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        if (tid == 0) {  // MMA2 for this tile (and MMA4 for two-tile chunks)
+        if (NT == 2 && tid == 0) {  // P' x onto Ct G, P' from TMEM
+          const uint32_t id2 = idesc_bf16(MT, kP, 0, 1);
+          const int cps = cpt / 16;  // K steps per part
+#pragma unroll 4
+          for (int j = 0; j < (mt + 1) * MT / 16; ++j)
+            mma_bf16_ts(tm + C::acc2_col(mt), tm + C::s_col(mt) + cpt * (j / cps) + 8 * (j % cps),
+                        dadd(dX, j * 2048), id2, 1);
+          if (mt == NT - 1) mma_commit(s_bar);
+        } else if (tid == 0) {  // MMA2 for this tile (and MMA4 for two-tile chunks)
           const uint32_t id2 = idesc_bf16(MT, kP, 0, 1);
           const int kblocks = (mt + 1) * MT / 64;
           // factored: one accumulator, Ct G' (MMA4) first; plain: P x alone
@@ -823,9 +923,12 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         const int rho = (MT == 64) ? 16 * qd + (lane & 15) : 32 * qd + lane;
         const int i = mt * MT + rho;  // row (t, r) of the chunk
         const int t = i / R;
-        // plain: (1, exp(Lam_t)) on (Y, Y2); factored: exp(Lam_t - ref) on Y'
-        const float el = (t < nt) ? ex2(plain ? s_lg[t] : s_lg[t] - l2ref) : 0.f;
-        const int ycol = plain ? C::y_col(mt) : C::acc_col(mt);
+        // plain: (1, exp(Lam_t)) on (Y, Y2); factored: exp(Lam_t - ref) on Y'.
+        // Two-tile chunks keep one accumulator in both forms (the plain form's
+        // Ct G is scaled through Ct), at acc2_col.
+        const bool two = plain && NT != 2;
+        const float el = (t < nt) ? ((NT == 2 && plain) ? 1.f : ex2(plain ? s_lg[t] : s_lg[t] - l2ref)) : 0.f;
+        const int ycol = NT == 2 ? C::acc2_col(mt) : plain ? C::y_col(mt) : C::acc_col(mt);
         constexpr int NPC = (MT == 64) ? CW / 32 : CW / 16;  // 16-column pieces per thread
         static_assert(MT != 64 || CW % 32 == 0, "64-row tiles: 32 columns per thread group");
 #pragma unroll
@@ -835,11 +938,11 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
           if (MT == 64) {
             col = CW * cq + 32 * pc + 16 * (lane >> 4);
             tmem_ld16x2<16>(tm + lane_base + ycol + CW * cq + 32 * pc, yv);
-            if (plain) tmem_ld16x2<16>(tm + lane_base + C::y2_col(mt) + CW * cq + 32 * pc, zv);
+            if (two) tmem_ld16x2<16>(tm + lane_base + C::y2_col(mt) + CW * cq + 32 * pc, zv);
           } else {
             col = CW * cq + 16 * pc;
             tmem_ld16(tm + lane_base + ycol + col, yv);
-            if (plain) tmem_ld16(tm + lane_base + C::y2_col(mt) + col, zv);
+            if (two) tmem_ld16(tm + lane_base + C::y2_col(mt) + col, zv);
           }
           tmem_ld_wait();
           {
@@ -851,7 +954,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
                 const int j = q * 8 + 2 * e;
                 const float2 yy = make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1]));
                 const float2 f =
-                    plain ? ffma2(make_float2(el, el),
+                    two ? ffma2(make_float2(el, el),
                                   make_float2(__uint_as_float(zv[j]), __uint_as_float(zv[j + 1])), yy)
                           : fmul2(make_float2(el, el), yy);
                 w4[e] = pack_bf16(f.x, f.y);
