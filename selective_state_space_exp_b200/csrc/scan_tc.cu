@@ -635,11 +635,20 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
           mma_bf16_ss(tm + C::s_col(1), dadd(dC, (k >> 2) * C::OPB + MT * 128 + (k & 3) * 32),
                       dadd(dB, (k >> 2) * C::OPB + (k & 3) * 32), id1, k != 0);
         mma_commit(s_bar1b);
-      } else if (!plain) {  // MMA3 (and MMA4 for one-tile chunks) first, then the scores
-        issue_mma3();
-        if (C::EARLY4) issue_mma4(0, C::acc_col(0), false);
+      } else if (!plain) {  // one tile: scores, Ct G and the chunk state as three interleaved chains
+        static_assert(NT == 2 || M / 16 <= 8, "one-tile chunk state in at most 8 K steps");
+        const uint32_t id1 = idesc_bf16(MT, MT, 0, 0);
+        const uint32_t id3 = idesc_bf16(kN, kP, 1, 1);
+        const uint32_t id4 = idesc_bf16(MT, kP, 0, 1);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t ko = (k >> 2) * C::OPB + (k & 3) * 32;  // K step k of N = 128
+          mma_bf16_ss(tm + C::s_col(0), dadd(dC, ko), dadd(dB, ko), id1, k != 0);
+          mma_bf16_ss(tm + C::acc_col(0), dadd(dC, ko), dadd(dG, k * 2048), id4, k != 0);
+          if (k < M / 16) mma_bf16_ss(tm + C::SC_COL, dadd(dBmn, k * 2048), dadd(dX, k * 2048), id3, k != 0);
+        }
         mma_commit(s_bar);
-        issue_mma1();
+        mma_commit(s_bar1);
       } else {  // plain form: the scores read Bh before it is rescaled for MMA3
         if (C::EARLY4) issue_mma4(0, C::y2_col(0), false);
         issue_mma1();
