@@ -719,7 +719,7 @@ def prefill_line(name, rank, world, steps, warmup, flush, peaks, psrc, cpu=True)
         "config": {"workload": name, **shape_cfg(s),
                    "l2": "flushed between timed steps (256 MiB write)",
                    "path": f"{kern}, {plan['launches']} launch(es) per call, "
-                           f"{plan['segments']} segment(s) per sequence"},
+                           f"at most {plan['segments']} segment(s) per sequence"},
         "roofline": {**roofline(flops, byt, per_step, peaks, psrc),
                      "scope": ("the one kernel launch of each m3_scan_fwd call, CUDA events on "
                                "the launching stream" if plan["launches"] == 1 else

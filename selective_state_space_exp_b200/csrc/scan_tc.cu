@@ -154,6 +154,15 @@ struct TcPlan {
   int64_t slots;  // segment summaries per chain: nseg - 1, or nseg for the state only
   float* wsT;    // [b][H][nseg-1][N][P]: local end states, then incoming states
   float* wsSum;  // [b][H][nseg-1][1 + N/2]: segment log-decay and angles
+  // Tail split (nseg == 1 plans whose last wave of chains is partial): the
+  // last `ntail` chains (b * H + h order) run as two halves of cps2 chunks,
+  // so that the last wave holds 2 * ntail half chains; their summaries are
+  // [ntail][N][P] and [ntail][1 + N/2], indexed by the chain's tail index.
+  // Grids are then one-dimensional: the full pass takes the whole chains
+  // first, then the halves (tail chain i: blocks 2i and 2i + 1 after them);
+  // the state-only pass and the combine take the tail chains' first halves.
+  int64_t ntail;
+  int64_t cps2;
 };
 
 __device__ __forceinline__ unsigned long long global_ns() {
@@ -227,7 +236,30 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, cq = warp >> 2;
   const int kg = lane & 15, tq = (warp << 1) | (lane >> 4);
-  const int64_t seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // this CTA's chain, segment and segment length (see TcPlan for the tail split)
+  int64_t seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z, nseg_c = pl.nseg, cps_c = pl.cps;
+  int64_t ti = -1;  // tail index of a split chain
+  if (pl.ntail > 0) {
+    const int64_t nfull = a.batch * a.nheads - pl.ntail;
+    int64_t chain;
+    if (MODE == MODE_STATE) {
+      ti = blockIdx.x;
+      chain = nfull + ti;
+      seg = 0;
+    } else if ((int64_t)blockIdx.x < nfull) {
+      chain = blockIdx.x;
+      seg = 0;
+    } else {
+      const int64_t k = (int64_t)blockIdx.x - nfull;
+      ti = k >> 1;
+      chain = nfull + ti;
+      seg = k & 1;
+    }
+    nseg_c = ti >= 0 ? 2 : 1;
+    cps_c = ti >= 0 ? pl.cps2 : a.nchunks;
+    b = chain / a.nheads;
+    h = chain % a.nheads;
+  }
   const int64_t H = a.nheads, G = a.ngroups;
   // this chain's sequence: tokens [tokb, tokb + L) of the token dimension
   const Chain chn = chain_of(a, b);
@@ -235,7 +267,7 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   const int64_t g = h / (H / G);
   const int64_t tg = h / (H / a.tgroups);  // theta group
   // bounds-checked builds: the CTA's chain and segment, and its tokens
-  if (!M3_IN(b, a.batch, a.status) || !M3_IN(h, H, a.status) || !M3_IN(seg, pl.nseg, a.status) ||
+  if (!M3_IN(b, a.batch, a.status) || !M3_IN(h, H, a.status) || !M3_IN(seg, nseg_c, a.status) ||
       (L > 0 && !M3_IN(tokb + L - 1, a.total_tokens, a.status)))
     return;  // uniform over the block
 
@@ -291,7 +323,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       }
     }
   } else {
-    const float* src = pl.wsT + (((b * H + h) * pl.slots + (seg - 1)) * kN + n) * kP + p0;
+    const int64_t slot_in = ti >= 0 ? ti : (b * H + h) * pl.slots + (seg - 1);
+    const float* src = pl.wsT + (slot_in * kN + n) * kP + p0;
 #pragma unroll
     for (int p = 0; p < CW; p += 4) {
       const float4 v = *reinterpret_cast<const float4*>(src + p);
@@ -315,8 +348,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
   // angle in fp64 (thousands of radians over a long segment), stored mod 2 pi
   float l2seg = 0.f;
   double phi_seg = 0.0;
-  const int64_t c_begin = seg * pl.cps;
-  const int64_t c_end = min(c_begin + pl.cps, (L + Q - 1) / Q);
+  const int64_t c_begin = seg * cps_c;
+  const int64_t c_end = min(c_begin + cps_c, (L + Q - 1) / Q);
 
   // Prefetch of a chunk's inputs in three steps, each as soon as its buffer is
   // free: theta (TMA, on s_tbT) and the gates (cp.async) once the previous
@@ -1008,14 +1041,14 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
 
   if (!aborted) {
     if (MODE == MODE_FULL) {
-      if (seg == pl.nseg - 1 && a.final_state) {
+      if (seg == nseg_c - 1 && a.final_state) {
         float* dst = a.final_state + ((b * H + h) * kN + n) * kP + p0;
 #pragma unroll
         for (int p = 0; p < CW; p += 4)
           *reinterpret_cast<float4*>(dst + p) = make_float4(gst[p], gst[p + 1], gst[p + 2], gst[p + 3]);
       }
     } else {
-      const int64_t slot = (b * H + h) * pl.slots + seg;
+      const int64_t slot = ti >= 0 ? ti : (b * H + h) * pl.slots + seg;
       float* dst = pl.wsT + (slot * kN + n) * kP + p0;
 #pragma unroll
       for (int p = 0; p < CW; p += 4)
@@ -1042,7 +1075,15 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
 // calls) instead of the incoming state of each later segment.
 template <bool TO_FINAL>
 __global__ void __launch_bounds__(256) tc_seg_pass_kernel(const ScanArgs a, const TcPlan pl) {
-  const int64_t b = blockIdx.z, h = blockIdx.y;
+  int64_t b = blockIdx.z, h = blockIdx.y;
+  int64_t nsum = TO_FINAL ? pl.nseg : pl.nseg - 1, slot0 = (b * a.nheads + h) * pl.slots;
+  if (!TO_FINAL && pl.ntail > 0) {  // tail split: blockIdx.y is the tail index
+    const int64_t chain = a.batch * a.nheads - pl.ntail + blockIdx.y;
+    b = chain / a.nheads;
+    h = chain % a.nheads;
+    nsum = 1;
+    slot0 = blockIdx.y;
+  }
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= kPairs * kP) return;
   const int k = idx / kP, p = idx % kP;
@@ -1062,8 +1103,8 @@ __global__ void __launch_bounds__(256) tc_seg_pass_kernel(const ScanArgs a, cons
       g1 = fmaf(eps * io_load(a.B_prev, bb + 2 * k + 1, true), xv, g1);
     }
   }
-  for (int64_t s = 0; s < (TO_FINAL ? pl.nseg : pl.nseg - 1); ++s) {
-    const int64_t slot = (b * H + h) * pl.slots + s;
+  for (int64_t s = 0; s < nsum; ++s) {
+    const int64_t slot = slot0 + s;
     float* T = pl.wsT + slot * kN * kP;
     const float* su = pl.wsSum + slot * (1 + kPairs);
     const float e = expf(su[0]);
@@ -1112,6 +1153,24 @@ TcPlan make_plan(const ScanArgs& a) {
   if (best.nseg < 1) {
     best.nseg = 1;
     best.cps = a.nchunks;
+  }
+  // Tail split: whole chains in the full waves, the chains of a last, partial
+  // wave cut in two so that their halves fill one wave (cost: a state-only
+  // pass over their first halves, one partial wave).  Fixed-length full
+  // scans only.
+  best.ntail = 0;
+  best.cps2 = 0;
+  if (best.nseg == 1 && !a.state_only && !a.cu_seqlens && a.nchunks >= 2) {
+    const int64_t rounds = (chains + slots - 1) / slots;
+    const int64_t rem = chains - (rounds - 1) * slots;  // chains in the last wave
+    const int64_t cps2 = (a.nchunks + 1) / 2;
+    if (rounds >= 2 && 2 * rem <= slots) {
+      const double split = (double)(rounds - 1) * a.nchunks + (1.0 + kStateCost) * cps2;
+      if (split < 0.97 * (double)rounds * a.nchunks) {
+        best.ntail = rem;
+        best.cps2 = cps2;
+      }
+    }
   }
   return best;
 }
@@ -1190,15 +1249,21 @@ bool make_maps(const ScanArgs& a, TcMaps* m) {
 }
 
 template <int R, int Q, int MODE>
-cudaError_t launch_kernel(const ScanArgs& a, const TcPlan& pl, const TcMaps& maps,
-                          int64_t nblocks, cudaStream_t st) {
+cudaError_t launch_grid(const ScanArgs& a, const TcPlan& pl, const TcMaps& maps, dim3 grid,
+                        cudaStream_t st) {
   using C = Cfg<R, Q>;
   auto kern = tc_scan_kernel<R, Q, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)nblocks, (unsigned)a.nheads, (unsigned)a.batch);
   kern<<<grid, C::NTH, C::SMEM, st>>>(a, pl, maps);
   return cudaGetLastError();
+}
+
+template <int R, int Q, int MODE>
+cudaError_t launch_kernel(const ScanArgs& a, const TcPlan& pl, const TcMaps& maps,
+                          int64_t nblocks, cudaStream_t st) {
+  return launch_grid<R, Q, MODE>(a, pl, maps,
+                                 dim3((unsigned)nblocks, (unsigned)a.nheads, (unsigned)a.batch), st);
 }
 
 template <int R, int Q>
@@ -1212,6 +1277,15 @@ cudaError_t launch_rq(const ScanArgs& a, TcPlan pl, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     tc_seg_pass_kernel<true><<<pg, 256, 0, st>>>(a, pl);
     return cudaGetLastError();
+  }
+  if (pl.ntail > 0) {  // tail split: first halves' local states, their fold, then all chains
+    const int64_t nfull = a.batch * a.nheads - pl.ntail;
+    cudaError_t e = launch_grid<R, Q, MODE_STATE>(a, pl, maps, dim3((unsigned)pl.ntail), st);
+    if (e != cudaSuccess) return e;
+    tc_seg_pass_kernel<false><<<dim3(pg.x, (unsigned)pl.ntail, 1), 256, 0, st>>>(a, pl);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_grid<R, Q, MODE_FULL>(a, pl, maps, dim3((unsigned)(nfull + 2 * pl.ntail)), st);
   }
   if (pl.nseg > 1) {
     cudaError_t e = launch_kernel<R, Q, MODE_STATE>(a, pl, maps, pl.nseg - 1, st);
@@ -1233,13 +1307,16 @@ bool tc_scan_supported(const ScanArgs& a) {
   return (a.R == 1 || a.R == 2 || a.R == 4) && (m == 64 || m == 128 || m == 256) && a.Q >= 16;
 }
 
-int64_t tc_scan_segments(const ScanArgs& a) { return make_plan(a).nseg; }
+int64_t tc_scan_segments(const ScanArgs& a) {
+  const TcPlan pl = make_plan(a);
+  return pl.ntail > 0 ? 2 : pl.nseg;
+}
 
 size_t tc_scan_workspace(const ScanArgs& a) {
   const TcPlan pl = make_plan(a);
   const int64_t per = a.state_only ? pl.nseg : pl.nseg - 1;
-  if (per <= 0) return 0;
-  const size_t slots = (size_t)a.batch * a.nheads * per;
+  if (per <= 0 && pl.ntail == 0) return 0;
+  const size_t slots = pl.ntail > 0 ? (size_t)pl.ntail : (size_t)a.batch * a.nheads * per;
   return align_up(sizeof(float) * slots * kN * kP, 256) +
          align_up(sizeof(float) * slots * (1 + kPairs), 256);
 }
@@ -1247,8 +1324,8 @@ size_t tc_scan_workspace(const ScanArgs& a) {
 cudaError_t tc_scan_launch(const ScanArgs& a, cudaStream_t st) {
   TcPlan pl = make_plan(a);
   pl.slots = a.state_only ? pl.nseg : pl.nseg - 1;
-  if (pl.slots > 0) {
-    const size_t slots = (size_t)a.batch * a.nheads * pl.slots;
+  if (pl.slots > 0 || pl.ntail > 0) {
+    const size_t slots = pl.ntail > 0 ? (size_t)pl.ntail : (size_t)a.batch * a.nheads * pl.slots;
     pl.wsT = reinterpret_cast<float*>(a.ws);
     pl.wsSum = reinterpret_cast<float*>(a.ws + align_up(sizeof(float) * slots * kN * kP, 256));
   }
