@@ -685,10 +685,12 @@ PROFILE = {"siso_prefill": "tc_scan_kernel_siso_prefill.md",
 
 
 def prefill_traffic(name, plan):
-    """DRAM bytes per launch of the scan kernel from its committed ncu summary
-    (one-launch calls only), and where it came from."""
+    """DRAM bytes per launch of the scan kernel's full pass from its committed
+    ncu summary, and where it came from: one-launch calls, and calls that cut
+    only a last wave's chains in two (their full pass covers every token once;
+    its state-only and combine launches are not counted)."""
     summary = PROFILE.get(name)
-    if not summary or not plan["tensor_core"] or plan["segments"] != 1:
+    if not summary or not plan["tensor_core"] or plan["segments"] > 2:
         return None, None
     t = profile_traffic(summary)
     return t, (f"profiles/{summary}" if t is not None else None)

@@ -144,8 +144,10 @@ M3_API size_t m3_scan_workspace_bytes(const m3_shape* shape);
 
 /* How m3_scan_fwd will run `shape` (host-only): *tensor_core = 1 for the
  * tcgen05 path (bf16 io, N = 128, P = 64, chunk * rank in {64, 128, 256},
- * M3_FLAG_SIMT clear), 0 for the CUDA-core fp32 path; *segments = pieces
- * each (batch, head) sequence is cut into (tensor-core path; 1 otherwise);
+ * M3_FLAG_SIMT clear), 0 for the CUDA-core fp32 path; *segments = the most
+ * pieces any (batch, head) sequence is cut into (tensor-core path; 1
+ * otherwise; a plan may cut only the sequences that would run in a last,
+ * partly empty wave of CTAs);
  * *launches = kernel launches per call (0 when seqlen == 0).  Any output
  * pointer may be NULL.  Returns M3_OK or the m3_check_shape error. */
 M3_API int m3_scan_plan(const m3_shape* shape, int* tensor_core, int64_t* segments,
