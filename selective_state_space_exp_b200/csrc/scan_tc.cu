@@ -683,12 +683,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         }
         mma_commit(s_bar);
         mma_commit(s_bar1);
-        const uint32_t id1 = idesc_bf16(MT, 2 * MT, 0, 0);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          mma_bf16_ss(tm + C::s_col(1), dadd(dC, (k >> 2) * C::OPB + MT * 128 + (k & 3) * 32),
-                      dadd(dB, (k >> 2) * C::OPB + (k & 3) * 32), id1, k != 0);
-        mma_commit(s_bar1b);
+        // tile 1's scores follow once the chunk state is done (below), so that
+        // they run under the state update instead of ahead of it
       } else if (!plain) {  // one tile: scores, Ct G and the chunk state as three interleaved chains
         static_assert(NT == 2 || M / 16 <= 8, "one-tile chunk state in at most 8 K steps");
         const uint32_t id1 = idesc_bf16(MT, MT, 0, 0);
@@ -760,6 +756,14 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
     phase ^= 1;
     if (__syncthreads_or(!ok3)) { aborted = true; break; }
     tc_fence_after();
+    if (MODE == MODE_FULL && NT == 2 && !plain && tid == 0) {  // tile 1's scores (N = 256)
+      const uint32_t id1 = idesc_bf16(MT, 2 * MT, 0, 0);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        mma_bf16_ss(tm + C::s_col(1), dadd(dC, (k >> 2) * C::OPB + MT * 128 + (k & 3) * 32),
+                    dadd(dB, (k >> 2) * C::OPB + (k & 3) * 32), id1, k != 0);
+      mma_commit(s_bar1b);
+    }
     if (MODE == MODE_STATE) prefetch_bx(c + 1);  // B and x are free once MMA3 is done
 
     // ---- state update G <- Rot(Phi_end) (exp(Lam_end) G + Sc), under MMA1 -------
