@@ -37,6 +37,11 @@
 // Operands live in shared memory in the 128-byte-swizzled canonical layout
 // and are read by tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) issued by one
 // thread; accumulators live in TMEM and are read back with tcgen05.ld.
+// Independent accumulators are issued as interleaved chains (an MMA waits on
+// the previous one into the same tile), and 256-row chunks keep their masked
+// scores in TMEM as the A operand of P x.  When one segment per chain leaves
+// the last wave of CTAs partly empty, only that wave's chains are cut in two
+// (TcPlan's tail split).
 // Supported: N = 128, P = 64, M = Q*R in {64, 128, 256}.
 #include <cuda.h>  // CUtensorMap (the encoder is reached through the runtime)
 
@@ -151,8 +156,9 @@ struct Cfg {
   // one dependent chain: the chunk state in two halves over the rows (K),
   // rows 0-127 into SC_COL and rows 128-255 into SC2_COL, interleaved with
   // tile 0's scores; once the state update has read both halves, the output
-  // accumulators of tile 0 and tile 1 take their columns (Y2T_COL / SC_COL)
-  // and both tiles' Ct G products are issued together before the masks.  The
+  // accumulators of tile 0 and tile 1 take their columns (acc2_col: SC2_COL /
+  // SC_COL) and both tiles' Ct G products are issued together before the
+  // masks; tile 1's scores are issued after the chunk-state wait.  The
   // masked scores stay in TMEM as packed bf16 (each warp's 16-column step
   // over columns it has already read) and are P x's A operand.
   static constexpr int SC2_COL = 448;
