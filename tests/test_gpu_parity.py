@@ -148,6 +148,30 @@ def test_tc_tiles_segments_ragged(R, chunk, L, batch, H):
     check(compare_scan(inp, chunk, "bf16"), "bf16")
 
 
+@pytest.mark.parametrize("R,batch,H", [(4, 6, 75), (1, 8, 75)], ids=["r4_450_chains", "r1_600_chains"])
+def test_tc_tail_split(R, batch, H):
+    """Chains that fill a few waves and spill a handful into one more (450
+    rank-4 chains on 148 one-CTA SMs, 600 rank-1 chains on 148 two-CTA SMs):
+    the plan cuts only the last wave's chains in two (a state-only pass over
+    their first halves, their fold, one full pass).  Five chunks, the last
+    ragged, so the halves are unequal; initial state and previous token, slow
+    decay so the folded state matters; every chain against the oracle, and
+    the last eight (the cut ones among them) on their own."""
+    w = I.Workload(I.Shape(batch, 300, H, 64, 128, R, 1, 64, "bf16"), decay="slow",
+                   with_h0=True, with_prev=True)
+    inp = I.make_scan_inputs(w, seed=7700 + R)
+    plan = m3.scan_plan(m3.scan_shape(inp["x"], inp["B"], 64))
+    assert plan["tensor_core"] and plan["segments"] == 2 and plan["launches"] == 3, plan
+    yg, hg = gpu_scan(inp, 64)
+    yo, ho = oracle_scan(inp)
+    assert np.isfinite(yg).all() and np.isfinite(hg).all()
+    check((rel_err(yg, yo), rel_err(hg, ho)), "bf16")
+    last = list(range(batch * H - 8, batch * H))
+    gy, gh = chain_rows(yg, hg, last, H)
+    oy, oh = chain_rows(yo, ho, last, H)
+    check((rel_err(gy, oy), rel_err(gh, oh)), "bf16")
+
+
 @pytest.mark.parametrize("R,chunk", [(1, 64), (2, 32), (2, 64), (4, 64), (4, 32)])
 def test_tc_large_decay_chunks(R, chunk):
     """Every other chunk decays by hundreds of nats (dt ten times larger and
