@@ -187,7 +187,9 @@ struct TcPlan {
   // [ntail][N][P] and [ntail][1 + N/2], indexed by the chain's tail index.
   // Grids are then one-dimensional: the full pass takes the whole chains
   // first, then the halves (tail chain i: blocks 2i and 2i + 1 after them);
-  // the state-only pass and the combine take the tail chains' first halves.
+  // the state-only pass takes the tail chains' first halves, and the full
+  // pass runs as its programmatic dependent: the second halves wait for it
+  // and fold its summaries into their incoming state themselves.
   int64_t ntail;
   int64_t cps2;
 };
@@ -298,6 +300,9 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
       (L > 0 && !M3_IN(tokb + L - 1, a.total_tokens, a.status)))
     return;  // uniform over the block
 
+  // a state-only pass lets a programmatically dependent full pass start now:
+  // the full pass's CTAs that need this pass's summaries wait for it
+  if (MODE == MODE_STATE) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (warp == 0) {
     tmem_alloc(s_tmem, C::TMEM_COLS);
     tmem_relinquish();
@@ -349,8 +354,39 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
         for (int p = 0; p < CW; ++p) gst[p] = fmaf(bp, io_load(a.x_prev, xo + p, true), gst[p]);
       }
     }
+  } else if (ti >= 0) {
+    // Second half of a tail chain: the state-only pass over the first half
+    // may still be running (this grid is its programmatic dependent), so wait
+    // for it, then fold its summary here: G_1 = Rot(Phi_0) exp(Lam_0) G_0 + T_0
+    // with G_0 the chain's initial state (rows n and n ^ 1 of a pair are
+    // adjacent lanes).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int64_t so = ((b * H + h) * kN + n) * kP + p0;
+#pragma unroll
+    for (int p = 0; p < CW; ++p) gst[p] = a.h0 ? __ldg(a.h0 + so + p) : 0.f;
+    if (a.B_prev && L > 0) {
+      const float eps0 = (1.f - __ldg(a.lam + tokb * H + h)) * __ldg(a.dt + tokb * H + h);
+      for (int r = 0; r < R; ++r) {
+        const float bp = eps0 * io_load(a.B_prev, ((b * G + g) * R + r) * kN + n, true);
+        const int64_t xo = ((b * H + h) * R + r) * kP + p0;
+#pragma unroll
+        for (int p = 0; p < CW; ++p) gst[p] = fmaf(bp, io_load(a.x_prev, xo + p, true), gst[p]);
+      }
+    }
+    const float* T = pl.wsT + (ti * kN + n) * kP + p0;
+    const float* su = pl.wsSum + ti * (1 + kPairs);
+    const float e = expf(su[0]);
+    float sn, cs;
+    sincosf(su[1 + (n >> 1)], &sn, &cs);
+    const float ss = (n & 1) ? sn : -sn;  // even row: c u - s u'; odd row: c u + s u'
+#pragma unroll
+    for (int p = 0; p < CW; ++p) {
+      const float u = e * gst[p];
+      const float o = __shfl_xor_sync(0xffffffffu, u, 1);
+      gst[p] = fmaf(cs, u, fmaf(ss, o, T[p]));
+    }
   } else {
-    const int64_t slot_in = ti >= 0 ? ti : (b * H + h) * pl.slots + (seg - 1);
+    const int64_t slot_in = (b * H + h) * pl.slots + (seg - 1);
     const float* src = pl.wsT + (slot_in * kN + n) * kP + p0;
 #pragma unroll
     for (int p = 0; p < CW; p += 4) {
@@ -1106,15 +1142,8 @@ tc_scan_kernel(const ScanArgs a, const TcPlan pl, const __grid_constant__ TcMaps
 // calls) instead of the incoming state of each later segment.
 template <bool TO_FINAL>
 __global__ void __launch_bounds__(256) tc_seg_pass_kernel(const ScanArgs a, const TcPlan pl) {
-  int64_t b = blockIdx.z, h = blockIdx.y;
-  int64_t nsum = TO_FINAL ? pl.nseg : pl.nseg - 1, slot0 = (b * a.nheads + h) * pl.slots;
-  if (!TO_FINAL && pl.ntail > 0) {  // tail split: blockIdx.y is the tail index
-    const int64_t chain = a.batch * a.nheads - pl.ntail + blockIdx.y;
-    b = chain / a.nheads;
-    h = chain % a.nheads;
-    nsum = 1;
-    slot0 = blockIdx.y;
-  }
+  const int64_t b = blockIdx.z, h = blockIdx.y;
+  const int64_t nsum = TO_FINAL ? pl.nseg : pl.nseg - 1, slot0 = (b * a.nheads + h) * pl.slots;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= kPairs * kP) return;
   const int k = idx / kP, p = idx % kP;
@@ -1279,15 +1308,30 @@ bool make_maps(const ScanArgs& a, TcMaps* m) {
                     CU_TENSOR_MAP_SWIZZLE_128B));
 }
 
+// dependent: launched as a programmatic dependent of the kernel before it on
+// the stream (it may start once that kernel's CTAs have all signalled).
 template <int R, int Q, int MODE>
 cudaError_t launch_grid(const ScanArgs& a, const TcPlan& pl, const TcMaps& maps, dim3 grid,
-                        cudaStream_t st) {
+                        cudaStream_t st, bool dependent = false) {
   using C = Cfg<R, Q>;
   auto kern = tc_scan_kernel<R, Q, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, C::NTH, C::SMEM, st>>>(a, pl, maps);
-  return cudaGetLastError();
+  if (!dependent) {
+    kern<<<grid, C::NTH, C::SMEM, st>>>(a, pl, maps);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(C::NTH);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, pl, maps);
 }
 
 template <int R, int Q, int MODE>
@@ -1309,14 +1353,15 @@ cudaError_t launch_rq(const ScanArgs& a, TcPlan pl, cudaStream_t st) {
     tc_seg_pass_kernel<true><<<pg, 256, 0, st>>>(a, pl);
     return cudaGetLastError();
   }
-  if (pl.ntail > 0) {  // tail split: first halves' local states, their fold, then all chains
+  if (pl.ntail > 0) {
+    // tail split: the first halves' local end states, and the full pass over
+    // every chain launched as its programmatic dependent (the whole chains
+    // start while the state-only pass runs; the second halves wait for it and
+    // fold its summaries themselves)
     const int64_t nfull = a.batch * a.nheads - pl.ntail;
     cudaError_t e = launch_grid<R, Q, MODE_STATE>(a, pl, maps, dim3((unsigned)pl.ntail), st);
     if (e != cudaSuccess) return e;
-    tc_seg_pass_kernel<false><<<dim3(pg.x, (unsigned)pl.ntail, 1), 256, 0, st>>>(a, pl);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    return launch_grid<R, Q, MODE_FULL>(a, pl, maps, dim3((unsigned)(nfull + 2 * pl.ntail)), st);
+    return launch_grid<R, Q, MODE_FULL>(a, pl, maps, dim3((unsigned)(nfull + 2 * pl.ntail)), st, true);
   }
   if (pl.nseg > 1) {
     cudaError_t e = launch_kernel<R, Q, MODE_STATE>(a, pl, maps, pl.nseg - 1, st);
