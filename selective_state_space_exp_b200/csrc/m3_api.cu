@@ -178,6 +178,13 @@ M3_API int m3_scan_state_workspace_size(const m3_shape* s, size_t* bytes) {
   return workspace_query(s, bytes, true);
 }
 
+extern "C++" {
+namespace m3 {
+// Kernel launches of one tensor-core scan call (scan_tc.cu).
+int tc_scan_launches(const ScanArgs& a);
+}  // namespace m3
+}
+
 M3_API int m3_scan_plan(const m3_shape* s, int* tensor_core, int64_t* segments, int* launches) {
   int st = check_common(s);
   if (st != M3_OK) return st;
@@ -186,7 +193,7 @@ M3_API int m3_scan_plan(const m3_shape* s, int* tensor_core, int64_t* segments, 
   const int64_t nseg = (tc && s->seqlen > 0) ? tc_scan_segments(a) : 1;
   if (tensor_core) *tensor_core = tc ? 1 : 0;
   if (segments) *segments = nseg;
-  if (launches) *launches = s->seqlen == 0 ? 0 : (tc ? (nseg > 1 ? 3 : 1) : 3);
+  if (launches) *launches = s->seqlen == 0 ? 0 : (tc ? tc_scan_launches(a) : 3);
   return M3_OK;
 }
 

@@ -1388,6 +1388,13 @@ int64_t tc_scan_segments(const ScanArgs& a) {
   return pl.ntail > 0 ? 2 : pl.nseg;
 }
 
+// Kernel launches of one full scan call: one; three with segments (state-only
+// pass, fold, full pass); two with the tail split (the fold is in the full pass).
+int tc_scan_launches(const ScanArgs& a) {
+  const TcPlan pl = make_plan(a);
+  return pl.ntail > 0 ? 2 : pl.nseg > 1 ? 3 : 1;
+}
+
 size_t tc_scan_workspace(const ScanArgs& a) {
   const TcPlan pl = make_plan(a);
   const int64_t per = a.state_only ? pl.nseg : pl.nseg - 1;
