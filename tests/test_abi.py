@@ -76,6 +76,11 @@ def test_workspace_size(lib):
     # many chains: one segment per chain, no workspace at all
     s = shape(batch=8, nheads=64, seqlen=2048)
     assert lib.m3_scan_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0 and n.value == 0
+    # rank 4 (one CTA per SM on 148 SMs): 512 chains leave a fourth wave of 68,
+    # which are cut in two -> one N x P state and 1 + N/2 totals per cut chain
+    s = shape(batch=8, nheads=64, seqlen=2048, rank=4)
+    assert lib.m3_scan_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0
+    assert n.value == 68 * 128 * 64 * 4 + (68 * 65 * 4 + 255) // 256 * 256  # parts 256-byte aligned
     assert lib.m3_scan_workspace_size(ctypes.byref(s), None) == -1
     assert lib.m3_scan_workspace_size(None, ctypes.byref(n)) == -1
 
@@ -152,6 +157,7 @@ def test_decode_rejects_bad_arguments(lib):
 
 @pytest.mark.parametrize("kw,tc,seg,launches", [
     (dict(batch=8, nheads=64, seqlen=2048), 1, 1, 1),            # many chains: one segment
+    (dict(batch=8, nheads=64, seqlen=2048, rank=4), 1, 2, 2),    # last wave's chains cut in two
     (dict(batch=1, nheads=64, seqlen=32768, rank=4), 1, None, 3),  # few chains: segments
     (dict(batch=8, nheads=64, seqlen=2048, flags=1), 0, 1, 3),     # forced CUDA-core path
     (dict(io_dtype=0, dstate=16, headdim=16), 0, 1, 3),            # fp32 io
